@@ -1,0 +1,290 @@
+/*
+ * moe_awq.h -- C ABI of the B200 (sm_100a) frozen AWQ routed-experts FFN.
+ *
+ * The operation (forward):
+ *   route   : top-k over FP32 router logits (+ optional selection-only bias),
+ *             FP32 weights from the softmax of the unbiased logits;
+ *   dispatch: COPY of every selected (token, expert) row into an
+ *             expert-sorted buffer;
+ *   experts : per expert, gate/up projections from AWQ int4 words, SwiGLU,
+ *             down projection;
+ *   combine : per token, FP32-weighted sum of its expert rows in ascending
+ *             expert-ID order.
+ * and its first-order input VJP (the transpose of the same rounded
+ * coefficients).  Sources of each statement are cited per function:
+ *   [PE] ruda-tensor 0.21.34, src/packed_experts.rs
+ *   [FA] ruda-tensor 0.21.33, src/frozen_awq.rs
+ *   [MX] ruda-tensor 0.21.38, src/moe_exchange.rs
+ *
+ * Conventions for every function:
+ *  - Every tensor argument is CALLER-OWNED DEVICE memory, row-major and
+ *    contiguous, unless the comment says "host".  The library never
+ *    allocates device memory; scratch comes from a caller workspace sized by
+ *    the matching *_workspace_size query.
+ *  - Every call is asynchronous on `stream` (a cudaStream_t; NULL means the
+ *    legacy default stream) and never synchronises.  Host-side argument
+ *    errors are reported before anything is launched.
+ *  - Return value: MOE_OK, or an error code; moe_last_error_string() (per
+ *    host thread) then describes it.
+ *  - Data errors that only the device can see (an expert ID outside the
+ *    resident range, inconsistent offsets, a row index outside [0, A)) are
+ *    OR-ed into *device_status (an int32 in device memory that the caller
+ *    zeroes); the offending rows are skipped, nothing traps.
+ *  - Packed weights are frozen: no function produces weight, zero-point,
+ *    scale or bias gradients ([PE] PackedExpertAutodiffError::TrainableMetadata,
+ *    [FA] FrozenAwqError::TrainableBase), and there is no dense or
+ *    requantized fallback ([FA] FrozenAwqError::Native, FrozenAwqOps doc).
+ *  - 16-bit floating tensors are IEEE binary16 (MOE_F16) or bfloat16
+ *    (MOE_BF16); FP32 is MOE_F32.
+ *
+ * AWQ projection payload of E experts, input width K, output width N
+ * ([PE] AwqExpertPayload, AwqExpertOptions; [FA] FrozenAwqOps doc):
+ *   qweight  int32 [E, K, N/8]     eight 4-bit codes per word; nibble slot s
+ *                                  (bits 4s..4s+3, word read as unsigned)
+ *                                  holds logical column 8w + P[s],
+ *                                  P = {0,2,4,6,1,3,5,7}
+ *   qzeros   int32 [E, K/group, N/8] zero codes, same packing
+ *   scales   [E, K/group, N]       F16 or BF16 (scale_dtype)
+ *   bias     [E, N] or NULL        F32, F16 or BF16 (bias_dtype), added to
+ *                                  the FP32 accumulator before rounding
+ *   coefficient W[e,kk,n] = RNE_scale_dtype((q - z[kk/group, n]) * s[kk/group, n]):
+ *   the exact product rounded once to the scale dtype.
+ *   Requirements: N % 8 == 0, K % group == 0, group % 16 == 0.
+ *   The tensor-core products run in the scale dtype; activations are
+ *   converted to it when they differ (BF16 -> F16 is exact for values in
+ *   F16's normal range).  FP32 scales are rejected with
+ *   MOE_ERR_UNSUPPORTED_DTYPE.
+ */
+#ifndef MOE_AWQ_H_
+#define MOE_AWQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Symbols of this ABI are the only ones the shared library exports. */
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARGUMENT = 1,  /* null/misaligned pointer, bad shape or size */
+  MOE_ERR_UNSUPPORTED_DTYPE = 2, /* dtype combination this library does not run */
+  MOE_ERR_WORKSPACE = 3,         /* workspace NULL or smaller than required */
+  MOE_ERR_CUDA = 4               /* a CUDA runtime call or launch failed */
+} moe_status;
+
+typedef enum { MOE_F32 = 0, MOE_F16 = 1, MOE_BF16 = 2 } moe_dtype;
+
+/* Bits OR-ed into *device_status by kernels. */
+#define MOE_DEVICE_ERR_EXPERT_RANGE 1 /* an expert ID outside [expert_start, expert_start+E) */
+#define MOE_DEVICE_ERR_OFFSETS 2      /* offsets not monotone, offsets[0] != 0 or offsets[E] != A */
+#define MOE_DEVICE_ERR_ROW_RANGE 4    /* a row_of entry outside [0, A) */
+#define MOE_DEVICE_ERR_TIMEOUT 8      /* a bounded device wait gave up */
+
+/* Limits of this implementation. */
+#define MOE_MAX_EXPERTS 4096
+#define MOE_MAX_TOP_K 32
+
+/* Description of the last error returned on this host thread. */
+MOE_API const char *moe_last_error_string(void);
+
+/* Library version string. */
+MOE_API const char *moe_version(void);
+
+/* ------------------------------------------------------------------------
+ * moe_route_dispatch -- [MX] MoeDispatchOps::moe_dispatch ("selection and
+ * continuous weights followed by device COPY dispatch") and MoeDispatched.
+ *
+ *  x                [T, H]  activations (F32, F16 or BF16: x_dtype); copied
+ *                           bit for bit, never rounded
+ *  logits           [T, E]  FP32 router logits
+ *  sel_bias         [E]     FP32 selection-only bias, or NULL; it changes
+ *                           which experts are chosen, never the weights
+ *  expert_start             first global expert ID of the resident bank
+ *                           ([PE] AwqExpertOptions::expert_start)
+ *  top_k                    1 <= top_k <= min(E, MOE_MAX_TOP_K)
+ *  renormalize              1: weights = softmax of the selected unbiased
+ *                           logits (softmax -> top-k -> renormalise);
+ *                           0: weights = full-softmax probabilities of the
+ *                           selected experts
+ * Outputs (A = T * top_k):
+ *  values           [A, H]  expert-sorted row copies ([MX] MoeDispatched::values)
+ *  weights          [T, k]  FP32 ([MX] MoeDispatched::weights)
+ *  selected_experts [T, k]  uint32 global IDs, descending score, ties to the
+ *                           lower ID ([MX] MoeDispatched::selected_experts)
+ *  row_experts      [A]     uint32 global IDs of each row, ascending
+ *                           ([MX] MoeDispatched::row_experts)
+ *  offsets          [E+1]   int32 exclusive prefix of per-expert row counts;
+ *                           an empty expert has offsets[e] == offsets[e+1]
+ *  src_token        [A]     int32 source token of each row; ascending inside
+ *                           each expert (stable order)
+ *  row_of           [T, k]  int32 row holding (token t, selection j)
+ *  workspace                device scratch of at least
+ *                           moe_route_dispatch_workspace_size(T, E, top_k)
+ *                           bytes, 16-byte aligned; contents need no
+ *                           initialisation and are dead after the call
+ * Errors: MOE_ERR_INVALID_ARGUMENT for T < 0, H < 1, E < 1 or
+ * E > MOE_MAX_EXPERTS, top_k out of range, a NULL pointer with T > 0;
+ * MOE_ERR_WORKSPACE if workspace is too small.  NaN logits are invalid input:
+ * the result is then unspecified but every index stays in range.
+ * ---------------------------------------------------------------------- */
+MOE_API size_t moe_route_dispatch_workspace_size(int64_t T, int64_t E, int32_t top_k);
+
+MOE_API moe_status moe_route_dispatch(const void *x, moe_dtype x_dtype, int64_t T, int64_t H,
+                              const float *logits, const float *sel_bias, int64_t E,
+                              int32_t expert_start, int32_t top_k, int32_t renormalize,
+                              void *values, float *weights, uint32_t *selected_experts,
+                              uint32_t *row_experts, int32_t *offsets, int32_t *src_token,
+                              int32_t *row_of, void *workspace, size_t workspace_bytes,
+                              int32_t *device_status, void *stream);
+
+/* ------------------------------------------------------------------------
+ * awq_grouped_gate_up_swiglu -- [PE] FrozenPackedExpertOps::packed_swiglu_forward
+ * (gate and up projections of the selected experts and the storage-rounded
+ * SwiGLU; "AD preserves required actual input caches": G and U are written
+ * when gate_out/up_out are non-NULL).
+ *
+ *  values   [A, H]   expert-sorted rows (act_dtype F16 or BF16); rows
+ *                    offsets[e]..offsets[e+1] belong to local expert e
+ *  offsets  [E+1]    int32, as written by moe_route_dispatch
+ *  gate/up payloads  AWQ payloads with K = H, N = I (see the file header);
+ *                    both share scale_dtype, bias_dtype and group
+ *  h        [A, I]   act_dtype: RNE(silu(G) * U), silu(v) = v / (1 + e^-v)
+ *  gate_out [A, I]   act_dtype G = RNE(sum_kk values*Wg + bias_g), or NULL
+ *  up_out   [A, I]   act_dtype U = RNE(sum_kk values*Wu + bias_u), or NULL
+ * The GPU path (small per-expert batches on warp-level tensor-core tiles,
+ * large ones on tcgen05/TMEM tiles) is chosen inside from A and E.
+ * Device errors: MOE_DEVICE_ERR_OFFSETS.
+ * ---------------------------------------------------------------------- */
+MOE_API moe_status awq_grouped_gate_up_swiglu(
+    const void *values, moe_dtype act_dtype, int64_t A, int64_t H, int64_t I,
+    const int32_t *offsets, int64_t E,
+    const int32_t *qweight_gate, const int32_t *qzeros_gate, const void *scales_gate,
+    const void *bias_gate,
+    const int32_t *qweight_up, const int32_t *qzeros_up, const void *scales_up,
+    const void *bias_up,
+    moe_dtype scale_dtype, moe_dtype bias_dtype, int64_t group_size,
+    void *h, void *gate_out, void *up_out, int32_t *device_status, void *stream);
+
+/* ------------------------------------------------------------------------
+ * awq_grouped_down -- the down projection of [PE] packed_swiglu_forward; also
+ * the grouped single projection [PE] FrozenPackedExpertOps::packed_expert_forward
+ * on expert-sorted rows, and with E = 1, offsets = {0, A} the single frozen
+ * linear [FA] FrozenAwqOps::frozen_awq_forward.
+ *
+ *  input [A, K] act_dtype (F16 or BF16); output [A, N] act_dtype:
+ *  output[r, n] = RNE(sum_kk input[r,kk] * W[e,kk,n] + bias[e,n]).
+ * Device errors: MOE_DEVICE_ERR_OFFSETS.
+ * ---------------------------------------------------------------------- */
+MOE_API moe_status awq_grouped_down(const void *input, moe_dtype act_dtype, int64_t A, int64_t K,
+                            int64_t N, const int32_t *offsets, int64_t E,
+                            const int32_t *qweight, const int32_t *qzeros, const void *scales,
+                            const void *bias, moe_dtype scale_dtype, moe_dtype bias_dtype,
+                            int64_t group_size, void *output, int32_t *device_status,
+                            void *stream);
+
+/* ------------------------------------------------------------------------
+ * moe_combine -- [MX] MoeDispatchOps::moe_combine ("ascending expert-ID
+ * combine after actual expert rows have returned to their source").
+ *
+ *  y [A, H] expert rows (act_dtype), weights [T, k] FP32,
+ *  selected_experts [T, k], row_of [T, k] as written by moe_route_dispatch.
+ *  out[t, :] = RNE(sum over j in ascending selected_experts[t, j] of
+ *              weights[t, j] * y[row_of[t, j], :]), FP32 accumulation from +0.
+ * Device errors: MOE_DEVICE_ERR_ROW_RANGE (that term is skipped).
+ * ---------------------------------------------------------------------- */
+MOE_API moe_status moe_combine(const void *y, moe_dtype act_dtype, int64_t A, const float *weights,
+                       const uint32_t *selected_experts, const int32_t *row_of, int64_t T,
+                       int64_t H, int32_t top_k, void *out, int32_t *device_status,
+                       void *stream);
+
+/* ------------------------------------------------------------------------
+ * moe_combine_backward -- [MX] MoeDispatchOps::moe_combine_backward with
+ * MoeCombineSelection: each requested output is non-NULL.
+ *
+ *  dy[row_of[t,j], :] = RNE(weights[t,j] * d_out[t, :])     ([A, H], act_dtype)
+ *  dweights[t, j]     = sum_c d_out[t,c] * y[row_of[t,j], c] ([T, k], FP32)
+ * Device errors: MOE_DEVICE_ERR_ROW_RANGE.
+ * ---------------------------------------------------------------------- */
+MOE_API moe_status moe_combine_backward(const void *d_out, const void *y, moe_dtype act_dtype, int64_t A,
+                                const float *weights, const int32_t *row_of, int64_t T,
+                                int64_t H, int32_t top_k, void *dy, float *dweights,
+                                int32_t *device_status, void *stream);
+
+/* ------------------------------------------------------------------------
+ * awq_input_backward -- [FA] FrozenAwqOps::frozen_awq_input_backward and
+ * [PE] packed_expert_input_backward / packed_swiglu_input_backward: the
+ * transpose of the same rounded coefficients, per expert.
+ *
+ *  grad   [A, N] grad_dtype (F16 or BF16), payload with K_in = K, width N
+ *  grad2  [A, N] or NULL, with a second payload (qweight2, qzeros2, scales2)
+ *  dinput[r, kk] = RNE(sum_n grad[r,n] W[e,kk,n] + sum_n grad2[r,n] W2[e,kk,n])
+ *  ([A, K], grad_dtype; the two sums share one accumulator and one rounding)
+ * Device errors: MOE_DEVICE_ERR_OFFSETS.
+ * ---------------------------------------------------------------------- */
+MOE_API moe_status awq_input_backward(const void *grad, moe_dtype grad_dtype, int64_t A, int64_t N,
+                              int64_t K, const int32_t *offsets, int64_t E,
+                              const int32_t *qweight, const int32_t *qzeros, const void *scales,
+                              moe_dtype scale_dtype, int64_t group_size, const void *grad2,
+                              const int32_t *qweight2, const int32_t *qzeros2,
+                              const void *scales2, void *dinput, int32_t *device_status,
+                              void *stream);
+
+/* ------------------------------------------------------------------------
+ * moe_swiglu_backward -- the SwiGLU step of [PE] packed_swiglu_input_backward,
+ * from the stored G and U (act_dtype, [A, I] each):
+ *   s = 1 / (1 + e^-G),  dG = RNE(dh * U * s * (1 + G (1 - s))),  dU = RNE(dh * G * s)
+ * ---------------------------------------------------------------------- */
+MOE_API moe_status moe_swiglu_backward(const void *dh, const void *G, const void *U, moe_dtype act_dtype,
+                               int64_t A, int64_t I, void *dG, void *dU, void *stream);
+
+/* ------------------------------------------------------------------------
+ * moe_dispatch_backward -- [MX] MoeDispatchOps::moe_dispatch_backward ("COPY
+ * VJP sums selected expert-row seeds without multiplying routing weights
+ * again"):
+ *   dx[t, :] = RNE(sum over j in ascending selected_experts[t, j] of
+ *              dvalues[row_of[t, j], :]), FP32 accumulation.
+ * Device errors: MOE_DEVICE_ERR_ROW_RANGE.
+ * ---------------------------------------------------------------------- */
+MOE_API moe_status moe_dispatch_backward(const void *dvalues, moe_dtype act_dtype, int64_t A,
+                                 const int32_t *row_of, const uint32_t *selected_experts,
+                                 int64_t T, int64_t H, int32_t top_k, void *dx,
+                                 int32_t *device_status, void *stream);
+
+/* ------------------------------------------------------------------------
+ * awq_dequant_coefficients -- the coefficients W[kk, n] of ONE expert's
+ * payload ([K, N/8] words, [K/group, N/8] zero words, [K/group, N] scales),
+ * formed by the same device code the projection kernels run, written out in
+ * the scale dtype ([K, N] uint16 bit patterns).  For verification: the
+ * rounded coefficient is what [FA] FrozenAwqOps preserves.
+ *  pairing 0: the register pairing of the forward warp-level tiles (one
+ *             column at two consecutive input rows);
+ *  pairing 1: the pairing of the input-VJP and tcgen05 tiles (two columns of
+ *             one word).
+ * ---------------------------------------------------------------------- */
+MOE_API moe_status awq_dequant_coefficients(const int32_t *qweight, const int32_t *qzeros,
+                                    const void *scales, moe_dtype scale_dtype, int64_t K,
+                                    int64_t N, int64_t group_size, int32_t pairing,
+                                    uint16_t *coefficients, void *stream);
+
+/* ------------------------------------------------------------------------
+ * Projection tile path: 0 = chosen from A and E (default), 1 = warp-level
+ * tiles (small per-expert batches), 2 = tcgen05/TMEM tiles (large batches).
+ * Both paths compute the same operation; the knob exists so tests and
+ * benchmarks can run either on the same inputs.  Process-wide; returns the
+ * previous value, or -1 for an unknown path.
+ * ---------------------------------------------------------------------- */
+MOE_API int32_t moe_set_projection_path(int32_t path);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_AWQ_H_ */

@@ -1,0 +1,261 @@
+// Combine, its VJP, the COPY-dispatch VJP and the SwiGLU VJP.
+//
+// ruda-tensor 0.21.38, src/moe_exchange.rs:
+//   moe_combine           -- per token, ascending expert-ID combine of the
+//                            expert rows with the FP32 weights;
+//   moe_combine_backward  -- requested expert-row and FP32 weight VJPs
+//                            (MoeCombineSelection / MoeCombineBackward);
+//   moe_dispatch_backward -- the COPY VJP sums the selected row seeds without
+//                            applying the routing weights again.
+// ruda-tensor 0.21.34, src/packed_experts.rs, packed_swiglu_input_backward --
+//   the SwiGLU step of the input VJP.
+//
+// One CTA per token: warp 0 orders the token's k selections by expert ID
+// (k <= 32, one lane each), then every thread accumulates 8 columns in FP32
+// from +0 in that order and rounds once.  Memory-bound: each kernel reads
+// and writes each row once with 16-byte accesses.
+#include "common.cuh"
+
+namespace moe {
+
+constexpr int kCombThreads = 256;
+
+struct CombineParams {
+  const void *y;  // [A, H] rows (or dvalues)
+  int dt;
+  int64_t A;
+  const float *weights;  // NULL: plain sum (COPY VJP)
+  const uint32_t *selected;
+  const int32_t *row_of;
+  int64_t T, H;
+  int k;
+  void *out;
+  int32_t *status;
+};
+
+// Fills ord_row/ord_w (shared) with the token's rows in ascending expert ID;
+// invalid rows get -1.
+__device__ __forceinline__ void order_token(const uint32_t *sel, const int32_t *row_of, const float *w,
+                                            int k, int64_t A, int64_t t, int32_t *ord_row, float *ord_w,
+                                            int32_t *status) {
+  if (threadIdx.x < 32) {
+    const int lane = threadIdx.x;
+    uint32_t id = lane < k ? sel[t * k + lane] : 0xFFFFFFFFu;
+    int32_t r = lane < k ? row_of[t * k + lane] : -1;
+    float wv = (lane < k && w) ? w[t * k + lane] : 1.f;
+    int pos = 0;
+    for (int j = 0; j < k; ++j) {
+      uint32_t oj = __shfl_sync(0xffffffffu, id, j);
+      pos += (oj < id || (oj == id && j < lane)) ? 1 : 0;
+    }
+    if (lane < k) {
+      if (r < 0 || (int64_t)r >= A) {
+        report(status, MOE_DEVICE_ERR_ROW_RANGE);
+        r = -1;
+      }
+      ord_row[pos] = r;
+      ord_w[pos] = wv;
+    }
+  }
+  __syncthreads();
+}
+
+template <bool VEC>
+__global__ void __launch_bounds__(kCombThreads) combine_kernel(CombineParams p) {
+  __shared__ int32_t ord_row[MOE_MAX_TOP_K];
+  __shared__ float ord_w[MOE_MAX_TOP_K];
+  const int64_t t = blockIdx.x;
+  order_token(p.selected, p.row_of, p.weights, p.k, p.A, t, ord_row, ord_w, p.status);
+  const uint16_t *y = static_cast<const uint16_t *>(p.y);
+  uint16_t *out = static_cast<uint16_t *>(p.out);
+  if (VEC) {
+    for (int64_t c0 = (int64_t)threadIdx.x * 8; c0 < p.H; c0 += (int64_t)blockDim.x * 8) {
+      float acc[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+      for (int j = 0; j < p.k; ++j) {
+        const int32_t r = ord_row[j];
+        if (r < 0) continue;
+        const float wv = ord_w[j];
+        uint4 v = *reinterpret_cast<const uint4 *>(y + (int64_t)r * p.H + c0);
+        const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          float lo = bits_to_f32(uint16_t(u[i] & 0xFFFF), p.dt), hi = bits_to_f32(uint16_t(u[i] >> 16), p.dt);
+          if (p.weights) {
+            acc[2 * i] = __fadd_rn(acc[2 * i], __fmul_rn(wv, lo));
+            acc[2 * i + 1] = __fadd_rn(acc[2 * i + 1], __fmul_rn(wv, hi));
+          } else {
+            acc[2 * i] = __fadd_rn(acc[2 * i], lo);
+            acc[2 * i + 1] = __fadd_rn(acc[2 * i + 1], hi);
+          }
+        }
+      }
+      uint32_t o[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        o[i] = uint32_t(f32_to_bits(acc[2 * i], p.dt)) | (uint32_t(f32_to_bits(acc[2 * i + 1], p.dt)) << 16);
+      *reinterpret_cast<uint4 *>(out + t * p.H + c0) = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+  } else {
+    for (int64_t c = threadIdx.x; c < p.H; c += blockDim.x) {
+      float acc = 0.f;
+      for (int j = 0; j < p.k; ++j) {
+        const int32_t r = ord_row[j];
+        if (r < 0) continue;
+        float v = bits_to_f32(y[(int64_t)r * p.H + c], p.dt);
+        acc = p.weights ? __fadd_rn(acc, __fmul_rn(ord_w[j], v)) : __fadd_rn(acc, v);
+      }
+      out[t * p.H + c] = f32_to_bits(acc, p.dt);
+    }
+  }
+}
+
+struct CombineBwdParams {
+  const void *d_out;
+  const void *y;
+  int dt;
+  int64_t A;
+  const float *weights;
+  const int32_t *row_of;
+  int64_t T, H;
+  int k;
+  void *dy;
+  float *dweights;
+  int32_t *status;
+};
+
+// One CTA per token.  dy rows are written with one rounding of the exact
+// FP32 product; the dots are reduced in a fixed tree (per thread, warp, CTA).
+__global__ void __launch_bounds__(kCombThreads) combine_bwd_kernel(CombineBwdParams p) {
+  __shared__ float red[kCombThreads / 32][MOE_MAX_TOP_K];
+  const int64_t t = blockIdx.x;
+  const uint16_t *g = static_cast<const uint16_t *>(p.d_out);
+  const uint16_t *y = static_cast<const uint16_t *>(p.y);
+  uint16_t *dy = static_cast<uint16_t *>(p.dy);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int j = 0; j < p.k; ++j) {
+    int32_t r = p.row_of[t * p.k + j];
+    const bool ok = r >= 0 && (int64_t)r < p.A;
+    if (!ok && threadIdx.x == 0) report(p.status, MOE_DEVICE_ERR_ROW_RANGE);
+    const float w = p.weights[t * p.k + j];
+    float dot = 0.f;
+    if (ok) {
+      for (int64_t c = threadIdx.x; c < p.H; c += blockDim.x) {
+        float gv = bits_to_f32(g[t * p.H + c], p.dt);
+        if (dy) dy[(int64_t)r * p.H + c] = f32_to_bits(__fmul_rn(w, gv), p.dt);
+        if (p.dweights) dot = fmaf(gv, bits_to_f32(y[(int64_t)r * p.H + c], p.dt), dot);
+      }
+    }
+    if (p.dweights) {
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+      if (lane == 0) red[warp][j] = dot;
+    }
+  }
+  if (!p.dweights) return;
+  __syncthreads();
+  if (threadIdx.x < p.k) {
+    float s = 0.f;
+    for (int w = 0; w < kCombThreads / 32; ++w) s += red[w][threadIdx.x];
+    p.dweights[t * p.k + threadIdx.x] = s;
+  }
+}
+
+struct SwigluBwdParams {
+  const uint16_t *dh, *G, *U;
+  uint16_t *dG, *dU;
+  int dt;
+  int64_t n;
+};
+
+__global__ void __launch_bounds__(256) swiglu_bwd_kernel(SwigluBwdParams p) {
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < p.n; i += (int64_t)gridDim.x * blockDim.x) {
+    float d = bits_to_f32(p.dh[i], p.dt), g = bits_to_f32(p.G[i], p.dt), u = bits_to_f32(p.U[i], p.dt);
+    float s = 1.f / (1.f + expf(-g));
+    p.dG[i] = f32_to_bits(d * u * s * (1.f + g * (1.f - s)), p.dt);
+    p.dU[i] = f32_to_bits(d * g * s, p.dt);
+  }
+}
+
+static moe_status launch_combine(const CombineParams &p, cudaStream_t st, const char *what) {
+  if (p.T == 0) return MOE_OK;
+  const bool vec = aligned16(p.y) && aligned16(p.out) && p.H % 8 == 0;
+  if (vec)
+    combine_kernel<true><<<(unsigned)p.T, kCombThreads, 0, st>>>(p);
+  else
+    combine_kernel<false><<<(unsigned)p.T, kCombThreads, 0, st>>>(p);
+  return check_launch(what);
+}
+
+static moe_status check_tk(const char *fn, int64_t T, int64_t H, int32_t k, int64_t A) {
+  if (T < 0 || H < 1 || k < 1 || k > MOE_MAX_TOP_K || A < 0)
+    return set_error(MOE_ERR_INVALID_ARGUMENT, "%s: bad sizes T=%lld H=%lld top_k=%d A=%lld", fn, (long long)T,
+                     (long long)H, k, (long long)A);
+  if (T > INT32_MAX) return set_error(MOE_ERR_INVALID_ARGUMENT, "%s: T too large", fn);
+  return MOE_OK;
+}
+
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" moe_status moe_combine(const void *y, moe_dtype act_dtype, int64_t A, const float *weights,
+                                  const uint32_t *selected_experts, const int32_t *row_of, int64_t T, int64_t H,
+                                  int32_t top_k, void *out, int32_t *device_status, void *stream) {
+  moe_status s = check_tk("moe_combine", T, H, top_k, A);
+  if (s != MOE_OK) return s;
+  if (act_dtype != MOE_F16 && act_dtype != MOE_BF16)
+    return set_error(MOE_ERR_UNSUPPORTED_DTYPE, "moe_combine: act_dtype must be F16 or BF16");
+  if (T > 0 && (!y || !weights || !selected_experts || !row_of || !out))
+    return set_error(MOE_ERR_INVALID_ARGUMENT, "moe_combine: NULL tensor pointer");
+  CombineParams p{y, (int)act_dtype, A, weights, selected_experts, row_of, T, H, top_k, out, device_status};
+  return launch_combine(p, as_stream(stream), "moe_combine");
+}
+
+extern "C" moe_status moe_dispatch_backward(const void *dvalues, moe_dtype act_dtype, int64_t A,
+                                            const int32_t *row_of, const uint32_t *selected_experts, int64_t T,
+                                            int64_t H, int32_t top_k, void *dx, int32_t *device_status,
+                                            void *stream) {
+  moe_status s = check_tk("moe_dispatch_backward", T, H, top_k, A);
+  if (s != MOE_OK) return s;
+  if (act_dtype != MOE_F16 && act_dtype != MOE_BF16)
+    return set_error(MOE_ERR_UNSUPPORTED_DTYPE, "moe_dispatch_backward: act_dtype must be F16 or BF16");
+  if (T > 0 && (!dvalues || !selected_experts || !row_of || !dx))
+    return set_error(MOE_ERR_INVALID_ARGUMENT, "moe_dispatch_backward: NULL tensor pointer");
+  CombineParams p{dvalues, (int)act_dtype, A, nullptr, selected_experts, row_of, T, H, top_k, dx, device_status};
+  return launch_combine(p, as_stream(stream), "moe_dispatch_backward");
+}
+
+extern "C" moe_status moe_combine_backward(const void *d_out, const void *y, moe_dtype act_dtype, int64_t A,
+                                           const float *weights, const int32_t *row_of, int64_t T, int64_t H,
+                                           int32_t top_k, void *dy, float *dweights, int32_t *device_status,
+                                           void *stream) {
+  moe_status s = check_tk("moe_combine_backward", T, H, top_k, A);
+  if (s != MOE_OK) return s;
+  if (act_dtype != MOE_F16 && act_dtype != MOE_BF16)
+    return set_error(MOE_ERR_UNSUPPORTED_DTYPE, "moe_combine_backward: act_dtype must be F16 or BF16");
+  if (T == 0 || (!dy && !dweights)) return MOE_OK;
+  if (!d_out || !weights || !row_of || (dweights && !y))
+    return set_error(MOE_ERR_INVALID_ARGUMENT, "moe_combine_backward: NULL tensor pointer");
+  CombineBwdParams p{d_out, y, (int)act_dtype, A, weights, row_of, T, H, top_k, dy, dweights, device_status};
+  combine_bwd_kernel<<<(unsigned)T, kCombThreads, 0, as_stream(stream)>>>(p);
+  return check_launch("moe_combine_backward");
+}
+
+extern "C" moe_status moe_swiglu_backward(const void *dh, const void *G, const void *U, moe_dtype act_dtype,
+                                          int64_t A, int64_t I, void *dG, void *dU, void *stream) {
+  if (A < 0 || I < 1) return set_error(MOE_ERR_INVALID_ARGUMENT, "moe_swiglu_backward: bad sizes");
+  if (act_dtype != MOE_F16 && act_dtype != MOE_BF16)
+    return set_error(MOE_ERR_UNSUPPORTED_DTYPE, "moe_swiglu_backward: act_dtype must be F16 or BF16");
+  if (A == 0) return MOE_OK;
+  if (!dh || !G || !U || !dG || !dU) return set_error(MOE_ERR_INVALID_ARGUMENT, "moe_swiglu_backward: NULL pointer");
+  SwigluBwdParams p{static_cast<const uint16_t *>(dh), static_cast<const uint16_t *>(G),
+                    static_cast<const uint16_t *>(U), static_cast<uint16_t *>(dG), static_cast<uint16_t *>(dU),
+                    (int)act_dtype, A * I};
+  int64_t blocks = (p.n + 255) / 256;
+  int64_t cap = (int64_t)num_sms() * 8;
+  if (blocks > cap) blocks = cap;
+  swiglu_bwd_kernel<<<(unsigned)blocks, 256, 0, as_stream(stream)>>>(p);
+  return check_launch("moe_swiglu_backward");
+}

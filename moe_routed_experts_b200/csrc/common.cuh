@@ -1,0 +1,164 @@
+// Shared helpers of the CUDA library: host error reporting, storage-dtype
+// loads and stores, device status flags, and the AWQ coefficient primitive
+// used by every projection kernel.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <type_traits>
+
+#include "moe_awq.h"
+
+namespace moe {
+
+// ---------------------------------------------------------------- host side
+
+moe_status set_error(moe_status s, const char *fmt, ...);
+moe_status check_launch(const char *what);
+inline cudaStream_t as_stream(void *s) { return reinterpret_cast<cudaStream_t>(s); }
+inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline int dtype_bytes(moe_dtype d) { return d == MOE_F32 ? 4 : 2; }
+inline bool valid_dtype(int d) { return d == MOE_F32 || d == MOE_F16 || d == MOE_BF16; }
+int num_sms();
+
+// ---------------------------------------------------------------- device side
+
+__device__ __forceinline__ void report(int32_t *status, int bits) {
+  if (status) atomicOr(status, bits);
+}
+
+__device__ __forceinline__ float ld_as_float(const void *base, int dt, int64_t i) {
+  if (dt == MOE_F32) return reinterpret_cast<const float *>(base)[i];
+  uint16_t b = reinterpret_cast<const uint16_t *>(base)[i];
+  if (dt == MOE_BF16) return __uint_as_float(uint32_t(b) << 16);
+  return __half2float(__ushort_as_half(b));
+}
+
+// Round-to-nearest-even FP32 -> storage dtype bits.
+__device__ __forceinline__ uint16_t f32_to_bits(float v, int dt) {
+  if (dt == MOE_BF16) return __bfloat16_as_ushort(__float2bfloat16_rn(v));
+  return __half_as_ushort(__float2half_rn(v));
+}
+
+__device__ __forceinline__ float bits_to_f32(uint16_t b, int dt) {
+  if (dt == MOE_BF16) return __uint_as_float(uint32_t(b) << 16);
+  return __half2float(__ushort_as_half(b));
+}
+
+// ---------------------------------------------------------------- AWQ coefficients
+//
+// A pair register holds two 16-bit lanes.  `q` carries two 4-bit codes in
+// bits 0..3 and 16..19.  OR-ing them under the bit pattern of a power of two
+// whose binade has unit spacing (1024 for F16, 128 for BF16) gives the
+// floats 1024+q (or 128+q) exactly; subtracting 1024+z (128+z) gives q-z
+// exactly; multiplying by the scale rounds (q-z)*s once, in the scale dtype.
+// This is the int->float "magic number" conversion (Kim et al., "Who Says
+// Elephants Can't Run", 2022), used here only to form q-z exactly.
+
+template <typename MT>
+struct Dq;
+
+template <>
+struct Dq<__half> {
+  static constexpr uint32_t kMagic2 = 0x64006400u;  // 1024.0 in both lanes
+  __device__ __forceinline__ static uint32_t coef(uint32_t q_or_magic, uint32_t zc, uint32_t sc) {
+    uint32_t d, c;
+    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(q_or_magic), "r"(zc));
+    asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(c) : "r"(d), "r"(sc));
+    return c;
+  }
+};
+
+template <>
+struct Dq<__nv_bfloat16> {
+  static constexpr uint32_t kMagic2 = 0x43004300u;  // 128.0 in both lanes
+  __device__ __forceinline__ static uint32_t coef(uint32_t q_or_magic, uint32_t zc, uint32_t sc) {
+    uint32_t d, c;
+    asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(q_or_magic), "r"(zc));
+    asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(c) : "r"(d), "r"(sc));
+    return c;
+  }
+};
+
+// (x & 0x000F000F) | magic in one LOP3.
+template <uint32_t kMagic2>
+__device__ __forceinline__ uint32_t nib_pair(uint32_t x) {
+  uint32_t r;
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(r) : "r"(x), "n"(0x000F000Fu), "n"(kMagic2));
+  return r;
+}
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t r;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
+  return r;
+}
+
+// Two BF16 (bits) -> two F16 (bits), through FP32; exact in F16's normal range.
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t v) {
+  float lo = __uint_as_float(v << 16), hi = __uint_as_float(v & 0xFFFF0000u);
+  __half2 h = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<uint32_t *>(&h);
+}
+// Two F16 -> two BF16 (rounds to BF16's 8 significant bits).
+__device__ __forceinline__ uint32_t f16x2_to_bf16x2(uint32_t v) {
+  __half2 h = *reinterpret_cast<__half2 *>(&v);
+  float2 f = __half22float2(h);
+  __nv_bfloat162 b = __floats2bfloat162_rn(f.x, f.y);
+  return *reinterpret_cast<uint32_t *>(&b);
+}
+
+template <typename MT>
+__device__ __forceinline__ uint32_t act_pair_to_mt(uint32_t v, int act_dt) {
+  if constexpr (sizeof(MT) == 2 && std::is_same<MT, __half>::value) {
+    return act_dt == MOE_BF16 ? bf16x2_to_f16x2(v) : v;
+  } else {
+    return act_dt == MOE_F16 ? f16x2_to_bf16x2(v) : v;
+  }
+}
+
+// mma.sync m16n8k16, FP32 accumulate.
+template <typename MT>
+__device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  if constexpr (std::is_same<MT, __half>::value) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+  } else {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+  }
+}
+
+__device__ __forceinline__ uint32_t ldg_nc_u32(const int32_t *p) {
+  uint32_t v;
+  asm volatile("ld.global.nc.L1::no_allocate.b32 %0, [%1];" : "=r"(v) : "l"(p));
+  return v;
+}
+
+// Offsets check shared by the projection kernels: returns the row range of
+// local expert e, or an empty range (and a status bit) if the mapping is
+// inconsistent.
+__device__ __forceinline__ bool expert_rows(const int32_t *offsets, int E, int64_t A, int e,
+                                            int32_t *status, int64_t &r0, int64_t &r1) {
+  int32_t a = offsets[e], b = offsets[e + 1];
+  bool bad = (a < 0) || (b < a) || (int64_t)b > A || (e == 0 && a != 0) || (e == E - 1 && (int64_t)b != A);
+  if (bad) {
+    if (threadIdx.x == 0) report(status, MOE_DEVICE_ERR_OFFSETS);
+    r0 = r1 = 0;
+    return false;
+  }
+  r0 = a;
+  r1 = b;
+  return true;
+}
+
+}  // namespace moe

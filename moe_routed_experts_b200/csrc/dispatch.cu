@@ -1,0 +1,406 @@
+// Top-k routing and stable expert-sorted COPY dispatch.
+//
+// ruda-tensor 0.21.38, src/moe_exchange.rs -- MoeDispatchOps::moe_dispatch:
+// selection and FP32 continuous weights, then a device COPY of each selected
+// row into an expert-sorted buffer whose U32 row_experts ascend.
+//
+// Three launches (two when the tokens fit one chunk):
+//   1. route_rank: one warp per token selects its top-k experts and their
+//      weights; per chunk of tokens, one warp assigns each (token, j) its
+//      rank among the chunk's rows of the same expert in token order
+//      (__match_any_sync groups equal experts; lanes are ordered by token),
+//      and the chunk histogram is written.  A single chunk also scans its
+//      histogram into the expert offsets.
+//   2. scan: per expert, an exclusive scan of the chunk histograms in chunk
+//      order (the chunk bases) and of the totals in expert order (offsets).
+//   3. scatter: row = offsets[e] + chunk_base[chunk][e] + rank; writes the
+//      row maps and copies the activation rows, spread over warps in
+//      512-byte segments.
+// Row order is (expert, token) by construction, with no atomics whose order
+// could vary between runs.
+#include <math.h>
+
+#include "common.cuh"
+
+namespace moe {
+
+constexpr int kRouteThreads = 512;
+constexpr int kScanThreads = 1024;
+constexpr int kMaxChunks = 64;
+
+// Tokens per chunk: a multiple of 64 keeping the chunk count <= kMaxChunks.
+static int64_t route_chunk(int64_t T) {
+  int64_t c = 64;
+  while ((T + c - 1) / c > kMaxChunks) c *= 2;
+  return c;
+}
+
+static int64_t round_up(int64_t v, int64_t m) { return (v + m - 1) / m * m; }
+
+struct RouteWs {
+  int64_t chunk, nchunks;
+  size_t hist_off, rank_off, bytes;
+};
+
+static RouteWs route_ws_layout(int64_t T, int64_t E, int32_t k) {
+  RouteWs w;
+  w.chunk = route_chunk(T > 0 ? T : 1);
+  w.nchunks = (T + w.chunk - 1) / w.chunk;
+  if (w.nchunks < 1) w.nchunks = 1;
+  w.hist_off = 0;
+  w.rank_off = (size_t)round_up(w.nchunks * E * 4, 256);
+  w.bytes = w.rank_off + (size_t)round_up(T * (int64_t)k * 4, 256);
+  if (w.bytes < 256) w.bytes = 256;
+  return w;
+}
+
+// Order key of a score: an unsigned integer that orders like the float
+// (higher score -> larger key).  NaN scores map to the key of -inf so that
+// every round still picks a valid, untaken expert.  0 is below every key.
+__device__ __forceinline__ uint32_t score_key(const float *l, const float *bias, int e) {
+  float s = bias ? __fadd_rn(l[e], bias[e]) : l[e];
+  if (isnan(s)) s = -INFINITY;
+  const uint32_t b = __float_as_uint(s);
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+
+// Block-wide exclusive scan of cnt[0..n) (in shared memory) into out[0..n],
+// out[n] = total.  All threads of the block must call it.
+__device__ void block_exclusive_scan(const int32_t *cnt, int n, int32_t *out, int32_t *tmp) {
+  const int tid = threadIdx.x, nt = blockDim.x;
+  const int per = (n + nt - 1) / nt;
+  const int b = tid * per, e = min(n, b + per);
+  int32_t local = 0;
+  for (int i = b; i < e; ++i) local += cnt[i];
+  // warp inclusive scan
+  const int lane = tid & 31, warp = tid >> 5;
+  int32_t v = local;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    int32_t u = __shfl_up_sync(0xffffffffu, v, o);
+    if (lane >= o) v += u;
+  }
+  if (lane == 31) tmp[warp] = v;
+  __syncthreads();
+  if (warp == 0) {
+    int nw = nt >> 5;
+    int32_t w = lane < nw ? tmp[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      int32_t u = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += u;
+    }
+    if (lane < nw) tmp[lane] = w;
+  }
+  __syncthreads();
+  int32_t run = v - local + (warp > 0 ? tmp[warp - 1] : 0);
+  for (int i = b; i < e; ++i) {
+    out[i] = run;
+    run += cnt[i];
+  }
+  if (tid == nt - 1) out[n] = run;  // the last thread's range ends at n (or is empty)
+  __syncthreads();
+}
+
+struct RouteParams {
+  const float *logits;
+  const float *sel_bias;
+  int64_t T;
+  int E, k, renorm;
+  uint32_t expert_start;
+  int64_t chunk;
+  float *weights;
+  uint32_t *selected;
+  int32_t *rank;      // [T*k] rank of (t, j) inside its chunk's rows of the same expert
+  int32_t *hist;      // [nchunks][E]; single chunk: zeroed (the chunk base)
+  int32_t *offsets;   // written when single != 0
+  int single;
+};
+
+__global__ void __launch_bounds__(1024) route_rank_kernel(RouteParams p) {
+  extern __shared__ int32_t sm[];
+  int32_t *cnt = sm;                      // [E]
+  int32_t *tmp = cnt + p.E;               // [32]
+  int16_t *sel_s = reinterpret_cast<int16_t *>(tmp + 32);  // [chunk * k]
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+  const int64_t t0 = (int64_t)blockIdx.x * p.chunk;
+  const int64_t t1 = min(p.T, t0 + p.chunk);
+  const int E = p.E, k = p.k;
+  for (int i = threadIdx.x; i < E; i += blockDim.x) cnt[i] = 0;
+
+  for (int64_t t = t0 + warp; t < t1; t += nwarps) {
+    const float *l = p.logits + t * E;
+    // k rounds of (score desc, id asc) argmax over the candidates that come
+    // after the previous winner in that order; two warp reductions a round
+    uint32_t prev_key = 0xFFFFFFFFu;
+    int prev_e = -1;
+    int my_e = 0;  // lane j keeps the j-th selection
+    for (int j = 0; j < k; ++j) {
+      uint32_t bk = 0u;
+      int be = 0x7FFFFFFF;
+      for (int e = lane; e < E; e += 32) {
+        const uint32_t key = score_key(l, p.sel_bias, e);
+        const bool after = key < prev_key || (key == prev_key && e > prev_e);
+        if (after && (key > bk || (key == bk && e < be))) {
+          bk = key;
+          be = e;
+        }
+      }
+      const uint32_t wk = __reduce_max_sync(0xffffffffu, bk);
+      const int we = (int)__reduce_min_sync(0xffffffffu, (bk == wk) ? (uint32_t)be : 0x7FFFFFFFu);
+      prev_key = wk;
+      prev_e = we;
+      if (lane == j) my_e = we;
+    }
+    // weights from the unbiased logits
+    float lj = (lane < k) ? l[my_e] : -INFINITY;
+    float m, den;
+    if (p.renorm) {
+      m = lj;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+      float ex = (lane < k) ? expf(lj - m) : 0.f;
+      den = ex;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+    } else {
+      m = -INFINITY;
+      for (int e = lane; e < E; e += 32) m = fmaxf(m, l[e]);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+      den = 0.f;
+      for (int e = lane; e < E; e += 32) den += expf(l[e] - m);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+    }
+    if (lane < k) {
+      p.weights[t * k + lane] = expf(lj - m) / den;
+      p.selected[t * k + lane] = p.expert_start + (uint32_t)my_e;
+      sel_s[(t - t0) * k + lane] = (int16_t)my_e;
+    }
+  }
+  __syncthreads();
+
+  if (warp == 0) {
+    const int tpi = 32 / k;  // tokens per warp iteration
+    const int n = (int)(t1 - t0);
+    for (int tt = 0; tt < n; tt += tpi) {
+      const int lt = tt + lane / k, j = lane % k;
+      const bool active = lane < tpi * k && lt < n;
+      const int e = active ? sel_s[lt * k + j] : -1 - lane;
+      const unsigned grp = __match_any_sync(0xffffffffu, e);
+      const int before = __popc(grp & ((1u << lane) - 1u));
+      const int base = active ? cnt[e] : 0;
+      __syncwarp();
+      if (active) {
+        p.rank[(t0 + lt) * k + j] = base + before;
+        if ((grp >> lane) == 1u) cnt[e] = base + __popc(grp);  // highest lane of the group
+      }
+      __syncwarp();
+    }
+  }
+  __syncthreads();
+
+  if (!p.single) {
+    for (int i = threadIdx.x; i < E; i += blockDim.x) p.hist[(int64_t)blockIdx.x * E + i] = cnt[i];
+    return;
+  }
+  block_exclusive_scan(cnt, E, p.offsets, tmp);
+  for (int i = threadIdx.x; i < E; i += blockDim.x) p.hist[i] = 0;
+}
+
+// Chunk bases (in place over hist) and offsets, one block.
+__global__ void __launch_bounds__(kScanThreads) route_scan_kernel(int32_t *hist, int nch, int E,
+                                                                   int32_t *offsets) {
+  extern __shared__ int32_t sm[];
+  int32_t *totals = sm;                // [E]
+  int32_t *tmp = totals + E;           // [32]
+  int32_t *part = tmp + 32;            // [tpe * E] partial sums
+  int tpe = 1;
+  while (tpe * 2 * E <= (int)blockDim.x && tpe * 2 <= nch) tpe *= 2;
+  const int cpp = (nch + tpe - 1) / tpe;  // chunks per part
+  for (int u = threadIdx.x; u < tpe * E; u += blockDim.x) {
+    int e = u % E, q = u / E;
+    int c0 = q * cpp, c1 = min(nch, c0 + cpp);
+    int32_t s = 0;
+    for (int c = c0; c < c1; ++c) s += hist[(int64_t)c * E + e];
+    part[q * E + e] = s;
+  }
+  __syncthreads();
+  for (int u = threadIdx.x; u < tpe * E; u += blockDim.x) {
+    int e = u % E, q = u / E;
+    int32_t run = 0;
+    for (int qq = 0; qq < q; ++qq) run += part[qq * E + e];
+    if (q == tpe - 1) {
+      int32_t tot = run + part[q * E + e];
+      totals[e] = tot;
+    }
+    int c0 = q * cpp, c1 = min(nch, c0 + cpp);
+    for (int c = c0; c < c1; ++c) {
+      int32_t h = hist[(int64_t)c * E + e];
+      hist[(int64_t)c * E + e] = run;
+      run += h;
+    }
+  }
+  __syncthreads();
+  block_exclusive_scan(totals, E, offsets, tmp);
+}
+
+struct ScatterParams {
+  const uint8_t *x;
+  uint8_t *values;
+  int64_t row_bytes;
+  int64_t A;
+  int k, E;
+  uint32_t expert_start;
+  int64_t chunk;
+  const uint32_t *selected;
+  const int32_t *offsets;
+  const int32_t *chunk_base;
+  const int32_t *rank;
+  int32_t *row_of;
+  uint32_t *row_experts;
+  int32_t *src_token;
+  int vec16;
+  int64_t nseg;  // copy segments per row
+};
+
+// One warp per (assignment, 512-byte segment), grid-stride.
+__global__ void __launch_bounds__(256) route_scatter_kernel(ScatterParams p) {
+  const int lane = threadIdx.x & 31;
+  const int64_t wid = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nw = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  const int64_t units = p.A * p.nseg;
+  for (int64_t u = wid; u < units; u += nw) {
+    const int64_t a = u / p.nseg, s = u % p.nseg;
+    const int64_t t = a / p.k;
+    int64_t pos = 0;
+    if (lane == 0) {
+      const int e = (int)(p.selected[a] - p.expert_start);
+      const int64_t c = t / p.chunk;
+      pos = (int64_t)p.offsets[e] + p.chunk_base[c * p.E + e] + p.rank[a];
+      if (s == 0) {
+        p.row_of[a] = (int32_t)pos;
+        p.row_experts[pos] = p.expert_start + (uint32_t)e;
+        p.src_token[pos] = (int32_t)t;
+      }
+    }
+    pos = __shfl_sync(0xffffffffu, pos, 0);
+    const uint8_t *src = p.x + t * p.row_bytes;
+    uint8_t *dst = p.values + pos * p.row_bytes;
+    if (p.vec16) {
+      const int64_t off = s * 512 + lane * 16;
+      if (off < p.row_bytes)
+        *reinterpret_cast<uint4 *>(dst + off) = __ldg(reinterpret_cast<const uint4 *>(src + off));
+    } else {
+      const int64_t off = s * 64 + lane * 2;
+      if (off < p.row_bytes)
+        *reinterpret_cast<uint16_t *>(dst + off) = *reinterpret_cast<const uint16_t *>(src + off);
+    }
+  }
+}
+
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" size_t moe_route_dispatch_workspace_size(int64_t T, int64_t E, int32_t top_k) {
+  if (T < 0 || E < 1 || top_k < 1) return 0;
+  return route_ws_layout(T, E, top_k).bytes;
+}
+
+extern "C" moe_status moe_route_dispatch(const void *x, moe_dtype x_dtype, int64_t T, int64_t H,
+                                         const float *logits, const float *sel_bias, int64_t E,
+                                         int32_t expert_start, int32_t top_k, int32_t renormalize,
+                                         void *values, float *weights, uint32_t *selected_experts,
+                                         uint32_t *row_experts, int32_t *offsets, int32_t *src_token,
+                                         int32_t *row_of, void *workspace, size_t workspace_bytes,
+                                         int32_t *device_status, void *stream) {
+  (void)device_status;  // every index is produced here; nothing to report
+  if (!valid_dtype(x_dtype)) return set_error(MOE_ERR_UNSUPPORTED_DTYPE, "moe_route_dispatch: bad x_dtype %d", (int)x_dtype);
+  if (T < 0 || H < 1 || E < 1 || E > MOE_MAX_EXPERTS)
+    return set_error(MOE_ERR_INVALID_ARGUMENT, "moe_route_dispatch: bad sizes T=%lld H=%lld E=%lld",
+                     (long long)T, (long long)H, (long long)E);
+  if (top_k < 1 || top_k > MOE_MAX_TOP_K || top_k > E)
+    return set_error(MOE_ERR_INVALID_ARGUMENT, "moe_route_dispatch: top_k=%d outside [1, min(E, %d)]", top_k,
+                     MOE_MAX_TOP_K);
+  if (expert_start < 0 || (int64_t)expert_start + E > (int64_t)UINT32_MAX)
+    return set_error(MOE_ERR_INVALID_ARGUMENT, "moe_route_dispatch: bad expert_start %d", expert_start);
+  if (!offsets) return set_error(MOE_ERR_INVALID_ARGUMENT, "moe_route_dispatch: offsets is NULL");
+  cudaStream_t st = as_stream(stream);
+  if (T == 0) {
+    if (cudaMemsetAsync(offsets, 0, sizeof(int32_t) * (size_t)(E + 1), st) != cudaSuccess)
+      return check_launch("moe_route_dispatch: memset offsets");
+    return MOE_OK;
+  }
+  if (!x || !logits || !values || !weights || !selected_experts || !row_experts || !src_token || !row_of)
+    return set_error(MOE_ERR_INVALID_ARGUMENT, "moe_route_dispatch: NULL tensor pointer");
+  if (T * (int64_t)top_k > INT32_MAX)
+    return set_error(MOE_ERR_INVALID_ARGUMENT, "moe_route_dispatch: T*top_k exceeds int32 row indices");
+  RouteWs lay = route_ws_layout(T, E, top_k);
+  if (!workspace || workspace_bytes < lay.bytes)
+    return set_error(MOE_ERR_WORKSPACE, "moe_route_dispatch: workspace of %zu bytes, need %zu", workspace_bytes,
+                     lay.bytes);
+  if ((reinterpret_cast<uintptr_t>(workspace) & 15u) != 0)
+    return set_error(MOE_ERR_INVALID_ARGUMENT, "moe_route_dispatch: workspace not 16-byte aligned");
+  int32_t *hist = reinterpret_cast<int32_t *>(static_cast<char *>(workspace) + lay.hist_off);
+  int32_t *rank = reinterpret_cast<int32_t *>(static_cast<char *>(workspace) + lay.rank_off);
+
+  RouteParams rp;
+  rp.logits = logits;
+  rp.sel_bias = sel_bias;
+  rp.T = T;
+  rp.E = (int)E;
+  rp.k = top_k;
+  rp.renorm = renormalize ? 1 : 0;
+  rp.expert_start = (uint32_t)expert_start;
+  rp.chunk = lay.chunk;
+  rp.weights = weights;
+  rp.selected = selected_experts;
+  rp.rank = rank;
+  rp.hist = hist;
+  rp.offsets = offsets;
+  rp.single = lay.nchunks == 1;
+  size_t smem = sizeof(int32_t) * (size_t)(E + 32) + sizeof(int16_t) * (size_t)(lay.chunk * top_k);
+  smem = (smem + 15) & ~size_t(15);
+  if (smem > 48 * 1024) cudaFuncSetAttribute(route_rank_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  // a warp per token: small batches get a wider block
+  const int threads = (T <= 32 && lay.nchunks == 1) ? 1024 : kRouteThreads;
+  route_rank_kernel<<<(unsigned)lay.nchunks, threads, smem, st>>>(rp);
+  moe_status s = check_launch("moe_route_dispatch: route_rank_kernel");
+  if (s != MOE_OK) return s;
+  if (!rp.single) {
+    int tpe = 1;
+    while (tpe * 2 * E <= kScanThreads && tpe * 2 <= lay.nchunks) tpe *= 2;
+    size_t ssm = sizeof(int32_t) * (size_t)(E + 32 + tpe * E);
+    if (ssm > 48 * 1024) cudaFuncSetAttribute(route_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ssm);
+    route_scan_kernel<<<1, kScanThreads, ssm, st>>>(hist, (int)lay.nchunks, (int)E, offsets);
+    s = check_launch("moe_route_dispatch: route_scan_kernel");
+    if (s != MOE_OK) return s;
+  }
+  ScatterParams sp;
+  sp.x = static_cast<const uint8_t *>(x);
+  sp.values = static_cast<uint8_t *>(values);
+  sp.row_bytes = H * dtype_bytes(x_dtype);
+  sp.A = T * top_k;
+  sp.k = top_k;
+  sp.E = (int)E;
+  sp.expert_start = (uint32_t)expert_start;
+  sp.chunk = lay.chunk;
+  sp.selected = selected_experts;
+  sp.offsets = offsets;
+  sp.chunk_base = hist;
+  sp.rank = rank;
+  sp.row_of = row_of;
+  sp.row_experts = row_experts;
+  sp.src_token = src_token;
+  sp.vec16 = aligned16(x) && aligned16(values) && (sp.row_bytes % 16 == 0);
+  const int64_t seg = sp.vec16 ? 512 : 64;
+  sp.nseg = (sp.row_bytes + seg - 1) / seg;
+  int64_t units = sp.A * sp.nseg;
+  int64_t blocks = (units + 7) / 8;
+  int64_t cap = (int64_t)num_sms() * 16;
+  if (blocks > cap) blocks = cap;
+  route_scatter_kernel<<<(unsigned)blocks, 256, 0, st>>>(sp);
+  return check_launch("moe_route_dispatch: route_scatter_kernel");
+}

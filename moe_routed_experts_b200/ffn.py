@@ -1,0 +1,120 @@
+"""The routed-experts FFN as a sequence of C-ABI calls.
+
+``forward`` = moe_route_dispatch -> awq_grouped_gate_up_swiglu ->
+awq_grouped_down -> moe_combine; ``backward`` = moe_combine_backward ->
+awq_input_backward(down) -> moe_swiglu_backward -> awq_input_backward(gate
++ up, one accumulation) -> moe_dispatch_backward.  Only argument
+marshalling happens here; every step runs in the library's kernels.
+"""
+from dataclasses import dataclass
+from typing import Optional
+
+import numpy as np
+import torch
+
+from . import binding as B
+
+_SDT = {"f16": torch.float16, "bf16": torch.bfloat16, "f32": torch.float32}
+
+
+def _t16(a: np.ndarray, dt: torch.dtype, device) -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(dt).to(device)
+
+
+def projection_to_device(proj: dict, scale_dtype: str, device="cuda") -> dict:
+    out = {"qweight": torch.from_numpy(np.ascontiguousarray(proj["qweight"])).to(device),
+           "qzeros": torch.from_numpy(np.ascontiguousarray(proj["qzeros"])).to(device)}
+    if scale_dtype == "f32":
+        out["scales"] = torch.from_numpy(np.ascontiguousarray(proj["scales"], np.float32)).to(device)
+    else:
+        out["scales"] = _t16(proj["scales"], _SDT[scale_dtype], device)
+    out["bias"] = None if proj.get("bias") is None else torch.from_numpy(proj["bias"]).to(device)
+    return out
+
+
+def to_device(inp: dict, device="cuda") -> dict:
+    """Generated NumPy inputs (moe_routed_experts_b200.inputs) -> device tensors."""
+    w = inp["workload"]
+    d = {"workload": w,
+         "x": _t16(inp["x"], torch.bfloat16, device),
+         "logits": torch.from_numpy(inp["logits"]).to(device),
+         "sel_bias": None if inp["sel_bias"] is None else torch.from_numpy(inp["sel_bias"]).to(device)}
+    for name in ("gate", "up", "down"):
+        d[name] = projection_to_device(inp[name], w.scale_dtype, device)
+    d["d_out"] = None if inp.get("d_out") is None else _t16(inp["d_out"], torch.bfloat16, device)
+    return d
+
+
+@dataclass
+class Buffers:
+    """Preallocated device outputs and scratch for one workload."""
+    route: dict
+    workspace: torch.Tensor
+    h: torch.Tensor
+    G: Optional[torch.Tensor]
+    U: Optional[torch.Tensor]
+    y: torch.Tensor
+    out: torch.Tensor
+    status: torch.Tensor
+
+
+def alloc(w, device="cuda", keep_gu: bool = False) -> Buffers:
+    T, H, I, E, k = w.T, w.H, w.I, w.E, w.top_k
+    A = T * k
+    route = {
+        "values": torch.empty((A, H), dtype=torch.bfloat16, device=device),
+        "weights": torch.empty((T, k), dtype=torch.float32, device=device),
+        "selected_experts": torch.empty((T, k), dtype=torch.int32, device=device),
+        "row_experts": torch.empty((A,), dtype=torch.int32, device=device),
+        "offsets": torch.empty((E + 1,), dtype=torch.int32, device=device),
+        "src_token": torch.empty((A,), dtype=torch.int32, device=device),
+        "row_of": torch.empty((T, k), dtype=torch.int32, device=device),
+    }
+    ws = torch.empty(max(B.route_dispatch_workspace_size(T, E, k), 256), dtype=torch.uint8, device=device)
+    h = torch.empty((A, I), dtype=torch.bfloat16, device=device)
+    G = torch.empty_like(h) if keep_gu else None
+    U = torch.empty_like(h) if keep_gu else None
+    y = torch.empty((A, H), dtype=torch.bfloat16, device=device)
+    out = torch.empty((T, H), dtype=torch.bfloat16, device=device)
+    return Buffers(route, ws, h, G, U, y, out, torch.zeros(1, dtype=torch.int32, device=device))
+
+
+def forward(dev: dict, buf: Buffers) -> torch.Tensor:
+    """One forward pass of the whole hot path into ``buf``; returns buf.out."""
+    w = dev["workload"]
+    r = B.moe_route_dispatch(dev["x"], dev["logits"], w.top_k, E=w.E, sel_bias=dev["sel_bias"],
+                             expert_start=w.expert_start, renormalize=w.renormalize, workspace=buf.workspace,
+                             device_status=buf.status, out=buf.route)
+    lib, st = B.lib(), B._stream()
+    gate, up, down = dev["gate"], dev["up"], dev["down"]
+    A = w.A
+    s = lib.awq_grouped_gate_up_swiglu(
+        B._ptr(r["values"]), B.MOE_BF16, A, w.H, w.I, B._ptr(r["offsets"]), w.E,
+        B._ptr(gate["qweight"]), B._ptr(gate["qzeros"]), B._ptr(gate["scales"]), B._ptr(gate["bias"]),
+        B._ptr(up["qweight"]), B._ptr(up["qzeros"]), B._ptr(up["scales"]), B._ptr(up["bias"]),
+        B._dt(gate["scales"].dtype), B.MOE_F32, w.group, B._ptr(buf.h), B._ptr(buf.G), B._ptr(buf.U),
+        B._ptr(buf.status), st)
+    B._check("awq_grouped_gate_up_swiglu", s)
+    s = lib.awq_grouped_down(
+        B._ptr(buf.h), B.MOE_BF16, A, w.I, w.H, B._ptr(r["offsets"]), w.E, B._ptr(down["qweight"]),
+        B._ptr(down["qzeros"]), B._ptr(down["scales"]), B._ptr(down["bias"]), B._dt(down["scales"].dtype),
+        B.MOE_F32, w.group, B._ptr(buf.y), B._ptr(buf.status), st)
+    B._check("awq_grouped_down", s)
+    s = lib.moe_combine(B._ptr(buf.y), B.MOE_BF16, A, B._ptr(r["weights"]), B._ptr(r["selected_experts"]),
+                        B._ptr(r["row_of"]), w.T, w.H, w.top_k, B._ptr(buf.out), B._ptr(buf.status), st)
+    B._check("moe_combine", s)
+    return buf.out
+
+
+def backward(dev: dict, buf: Buffers, d_out: torch.Tensor) -> dict:
+    """Input VJP of the forward held in ``buf`` (needs G and U kept)."""
+    w = dev["workload"]
+    r = buf.route
+    assert buf.G is not None and buf.U is not None, "allocate with keep_gu=True"
+    dy, dw = B.moe_combine_backward(d_out, buf.y, r["weights"], r["row_of"], device_status=buf.status)
+    dh = B.awq_input_backward(dy, r["offsets"], dev["down"], w.group, device_status=buf.status)
+    dG, dU = B.moe_swiglu_backward(dh, buf.G, buf.U)
+    dvalues = B.awq_input_backward(dG, r["offsets"], dev["gate"], w.group, grad2=dU, proj2=dev["up"],
+                                   device_status=buf.status)
+    dx = B.moe_dispatch_backward(dvalues, r["row_of"], r["selected_experts"], device_status=buf.status)
+    return {"dy": dy, "dweights": dw, "dh": dh, "dG": dG, "dU": dU, "dvalues": dvalues, "dx": dx}

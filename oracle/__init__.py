@@ -12,7 +12,7 @@ import os
 
 import numpy as np
 
-from .build import build
+from .build import build as _build_library
 
 DT = {"f32": 0, "f16": 1, "bf16": 2, "f64": 3}
 
@@ -22,7 +22,7 @@ _lib = None
 def lib():
     global _lib
     if _lib is None:
-        _lib = C.CDLL(build())
+        _lib = C.CDLL(_build_library())
         _declare(_lib)
     return _lib
 
@@ -130,6 +130,8 @@ def coefficient(q: int, z: int, scale_bits: int, sdt: str):
 
 def dequant(qw, qz, sc, sdt: str, K: int, N: int, g: int):
     """One expert's coefficients: (W float64 [K,N], bits uint32 [K,N])."""
+    if g < 1 or K % g or N % 8:
+        raise ValueError("dequant: incomplete group or N % 8 != 0")
     qw, qz, sc = _c(qw, np.int32), _c(qz, np.int32), _sdt_array(sc, sdt)
     W = np.zeros((K, N), np.float64)
     Wb = np.zeros((K, N), np.uint32)
@@ -200,7 +202,7 @@ def project(x, xdt: str, row_expert, proj: dict, sdt: str, g: int, exact: bool =
     rc = lib().oracle_project(_p(x), DT[xdt], R, K, N, _p(re), E, _p(qw), _p(qz), _p(sc), DT[sdt],
                               _p(bias), DT[bias_dt], g, 1 if exact else 0, _p(out), DT[odt])
     if rc != 0:
-        raise ValueError("oracle_project: expert index out of range")
+        raise ValueError("oracle_project: " + ("incomplete group or N % 8 != 0" if rc == -2 else "expert index out of range"))
     return out
 
 
@@ -253,7 +255,7 @@ def input_backward(grad, gdt: str, row_expert, proj: dict, sdt: str, g: int, gra
     rc = lib().oracle_input_backward(_p(grad), DT[gdt], R, N, K, _p(re), E, _p(qw), _p(qz), _p(sc), DT[sdt], g,
                                      _p(g2), _p(qw2), _p(qz2), _p(sc2), 1 if exact else 0, _p(out), DT[odt])
     if rc != 0:
-        raise ValueError("oracle_input_backward: expert index out of range")
+        raise ValueError("oracle_input_backward: " + ("incomplete group or N % 8 != 0" if rc == -2 else "expert index out of range"))
     return out
 
 

@@ -320,11 +320,14 @@ void oracle_copy_rows(const void *x, int64_t H, int64_t elem_bytes, const int32_
  * mode 0: out is stored in odt, rounded once (RNE) from the double sum.
  * mode 1: out is double [R,N], no output rounding (exact-math mode; the
  *         coefficients stay rounded because they are the operator).
- * Returns 0, or -1 on a bad expert index. */
+ * Returns 0, -1 on a bad expert index, -2 when K is not a whole number of
+ * groups or N is not a multiple of 8 (AwqExpertOptions: complete
+ * input-channel groups, output width divisible by eight). */
 int oracle_project(const void *x, int xdt, int64_t R, int64_t K, int64_t N,
                    const int32_t *row_expert, int64_t E,
                    const int32_t *qw, const int32_t *qz, const void *sc, int sdt,
                    const void *bias, int bdt, int64_t g, int mode, void *out, int odt) {
+    if (g < 1 || K % g != 0 || N % 8 != 0) return -2; /* complete groups, 8 columns per word */
     for (int64_t r = 0; r < R; ++r)
         if (row_expert[r] < 0 || row_expert[r] >= E) return -1;
     int64_t NW = N / 8, G = K / g;
@@ -424,6 +427,7 @@ int oracle_input_backward(const void *grad, int gdt, int64_t R, int64_t N, int64
                           const int32_t *qw, const int32_t *qz, const void *sc, int sdt, int64_t g,
                           const void *grad2, const int32_t *qw2, const int32_t *qz2, const void *sc2,
                           int mode, void *out, int odt) {
+    if (g < 1 || K % g != 0 || N % 8 != 0) return -2; /* complete groups, 8 columns per word */
     for (int64_t r = 0; r < R; ++r)
         if (row_expert[r] < 0 || row_expert[r] >= E) return -1;
     int64_t NW = N / 8, G = K / g;

@@ -1,0 +1,103 @@
+"""GPU parity of the backward chain: combine VJP (expert rows and FP32
+weights), the down and gate+up input VJPs (transpose of the same rounded
+coefficients), the SwiGLU VJP and the COPY-dispatch VJP.  Each step is fed
+the device's own inputs and compared with the oracle on the same values."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from helpers import as_f64, bits, check_close, generated, gpu_forward, sample_rows
+from moe_routed_experts_b200 import binding as B
+from moe_routed_experts_b200 import ffn
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(params=[1, 2], ids=["warp_tiles", "tcgen05_tiles"])
+def path(request):
+    try:
+        prev = B.set_projection_path(request.param)
+    except ValueError:
+        pytest.skip("projection path %d not available" % request.param)
+    yield request.param
+    B.set_projection_path(prev)
+
+
+def _chain(name, kw, rows=None, tokens=None):
+    inp = generated(name, **kw)
+    w = inp["workload"]
+    dev, buf = gpu_forward(inp, keep_gu=True)
+    d_out = dev["d_out"]
+    g = ffn.backward(dev, buf, d_out)
+    torch.cuda.synchronize()
+    r = buf.route
+    row_of = r["row_of"].cpu().numpy()
+    sel = r["selected_experts"].cpu().numpy().view(np.uint32)
+    wts = r["weights"].cpu().numpy()
+    offsets = r["offsets"].cpu().numpy()
+    rexp_all = (r["row_experts"].cpu().numpy().view(np.uint32).astype(np.int64) - w.expert_start).astype(np.int32)
+    y, G, U = bits(buf.y), bits(buf.G), bits(buf.U)
+    dy, dh, dG, dU, dv, dx = (bits(g[k]) for k in ("dy", "dh", "dG", "dU", "dvalues", "dx"))
+    dw = g["dweights"].cpu().numpy()
+    dout = inp["d_out"]
+    if rows is None:
+        rows = np.arange(w.A)
+    if tokens is None:
+        tokens = np.arange(w.T)
+    # combine VJP on the sampled tokens
+    o_dy, o_dw = oracle.combine_backward(dout[tokens], y, "bf16", wts[tokens], row_of[tokens])
+    check_close(dy[row_of[tokens].reshape(-1)], o_dy[row_of[tokens].reshape(-1)], name + "/dy")
+    assert np.max(np.abs(dw[tokens] - o_dw)) <= 2e-2 * np.sqrt(np.mean(o_dw.astype(np.float64) ** 2)), "dweights"
+    # down input VJP, SwiGLU VJP, gate+up input VJP on the sampled rows
+    re = rexp_all[rows]
+    o_dh = oracle.input_backward(dy[rows], "bf16", re, inp["down"], w.scale_dtype, w.group)
+    check_close(dh[rows], o_dh, name + "/dh")
+    o_dG, o_dU = oracle.swiglu_backward(dh[rows], G[rows], U[rows])
+    check_close(dG[rows], o_dG, name + "/dG")
+    check_close(dU[rows], o_dU, name + "/dU")
+    o_dv = oracle.input_backward(dG[rows], "bf16", re, inp["gate"], w.scale_dtype, w.group, grad2=dU[rows],
+                                 proj2=inp["up"])
+    check_close(dv[rows], o_dv, name + "/dvalues")
+    o_dx = oracle.dispatch_backward(dv, "bf16", sel[tokens], row_of[tokens])
+    check_close(dx[tokens], o_dx, name + "/dx")
+    assert int(buf.status.item()) == 0
+    return w, offsets
+
+
+SMALL = {"skewed": dict(T=1024, H=512, I=256, E=16), "prefill": dict(T=512, H=256, I=128, E=16, backward=True),
+         "decode": dict(backward=True), "tiny": dict(backward=True)}
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_backward_chain_every_row(name, path):
+    _chain(name, SMALL[name])
+
+
+def test_backward_full_size_skewed_sampled(path):
+    inp = generated("skewed")
+    w = inp["workload"]
+    sel, _ = oracle.route(inp["logits"], None, w.top_k)
+    off, _, _, _ = oracle.dispatch(sel, w.E)
+    rows = sample_rows(off, n_experts=3, rows_per=4)
+    tokens = np.array([0, 5, w.T // 2, w.T - 1])
+    _chain("skewed", {}, rows=rows, tokens=tokens)
+
+
+def test_whole_chain_against_oracle_chain():
+    """Oracle forward + backward from scratch vs the device chain (no shared intermediates)."""
+    inp = generated("skewed", T=256, H=256, I=128, E=8)
+    w = inp["workload"]
+    dev, buf = gpu_forward(inp, keep_gu=True)
+    g = ffn.backward(dev, buf, dev["d_out"])
+    torch.cuda.synchronize()
+    f = oracle.forward(inp)
+    rexp = (f["row_experts"].astype(np.int64) - w.expert_start).astype(np.int32)
+    o_dy, o_dw = oracle.combine_backward(inp["d_out"], f["y"], "bf16", f["weights"], f["row_of"])
+    o_dh = oracle.input_backward(o_dy, "bf16", rexp, inp["down"], w.scale_dtype, w.group)
+    o_dG, o_dU = oracle.swiglu_backward(o_dh, f["G"], f["U"])
+    o_dv = oracle.input_backward(o_dG, "bf16", rexp, inp["gate"], w.scale_dtype, w.group, grad2=o_dU,
+                                 proj2=inp["up"])
+    o_dx = oracle.dispatch_backward(o_dv, "bf16", f["selected"], f["row_of"])
+    check_close(bits(g["dx"]), o_dx, "chain/dx")
+    check_close(bits(g["dvalues"]), o_dv, "chain/dvalues")

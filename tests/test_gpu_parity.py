@@ -1,0 +1,172 @@
+"""GPU parity of every C-ABI entry point against the CPU oracle, on the same
+seeded inputs.  Indices, dispatch order, offsets and the rounded
+coefficients bit for bit; FP32 weights within 2e-6; BF16/F16 outputs and
+gradients within 2e-2 * rms(oracle)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from helpers import (TOL, as_f64, bits, check_close, check_routing, generated, gpu_forward, gpu_forward_numpy,
+                     sample_rows, u32)
+from moe_routed_experts_b200 import binding as B
+from moe_routed_experts_b200 import ffn, inputs
+from moe_routed_experts_b200.configs import WORKLOADS, Workload, scaled
+
+pytestmark = pytest.mark.gpu
+
+PATHS = [1, 2]
+
+
+@pytest.fixture(params=PATHS, ids=["warp_tiles", "tcgen05_tiles"])
+def path(request):
+    p = request.param
+    try:
+        prev = B.set_projection_path(p)
+    except ValueError:
+        pytest.skip("projection path %d not available" % p)
+    yield p
+    B.set_projection_path(prev)
+
+
+# ------------------------------------------------------------------ coefficients
+
+@pytest.mark.parametrize("sdt", ["f16", "bf16"])
+@pytest.mark.parametrize("pairing", [0, 1])
+def test_coefficients_bit_exact(sdt, pairing):
+    rng = np.random.default_rng(21)
+    K, N, g = 512, 512, 16
+    proj = inputs.draw_projection(rng, 1, K, N, g, sdt, False, 0.0)
+    # widen the scale range well beyond the workloads', including F16 subnormals
+    raw = rng.integers(0, 0x7B00 if sdt == "f16" else 0x7F00, size=proj["scales"].shape).astype(np.uint16)
+    raw[0, 0, :64] = np.arange(64, dtype=np.uint16)  # smallest magnitudes / subnormals
+    proj["scales"] = raw
+    dev = ffn.projection_to_device(proj, sdt)
+    got = bits(B.awq_dequant_coefficients(dev["qweight"][0], dev["qzeros"][0], dev["scales"][0], g, pairing))
+    _, want = oracle.dequant(proj["qweight"][0], proj["qzeros"][0], proj["scales"][0], sdt, K, N, g)
+    mism = np.nonzero(got != want.astype(np.uint16))
+    assert mism[0].size == 0, "first mismatches at %s" % (list(zip(*[m[:5] for m in mism])),)
+
+
+# ------------------------------------------------------------------ routing and dispatch
+
+@pytest.mark.parametrize("name", list(WORKLOADS))
+def test_route_dispatch_full_size(name):
+    inp = generated(name)
+    w = inp["workload"]
+    dev = ffn.to_device(inp)
+    st = B.new_status()
+    r = B.moe_route_dispatch(dev["x"], dev["logits"], w.top_k, E=w.E, sel_bias=dev["sel_bias"], device_status=st)
+    torch.cuda.synchronize()
+    sel, wts = oracle.route(inp["logits"], inp["sel_bias"], w.top_k)
+    off, rexp, src, row_of = oracle.dispatch(sel, w.E)
+    got = {"selected": u32(r["selected_experts"]), "weights": r["weights"].cpu().numpy(),
+           "offsets": r["offsets"].cpu().numpy(), "row_experts": u32(r["row_experts"]),
+           "src_token": r["src_token"].cpu().numpy(), "row_of": r["row_of"].cpu().numpy()}
+    check_routing(got, {"selected": sel, "weights": wts, "offsets": off, "row_experts": rexp, "src_token": src,
+                        "row_of": row_of}, name)
+    src_t = torch.from_numpy(src.astype(np.int64)).cuda()
+    assert torch.equal(r["values"], dev["x"][src_t]), "values are not bit copies of x[src_token]"
+    assert int(st.item()) == 0
+
+
+@pytest.mark.parametrize("renorm,expert_start", [(0, 0), (1, 7), (0, 100)])
+def test_route_dispatch_options(renorm, expert_start):
+    w = Workload("opt", T=300, H=64, I=32, E=40, top_k=5, group=16, scale_dtype="f16", sel_bias_std=0.3,
+                 expert_start=expert_start, renormalize=renorm)
+    inp = inputs.generate(w)
+    dev = ffn.to_device(inp)
+    r = B.moe_route_dispatch(dev["x"], dev["logits"], w.top_k, E=w.E, sel_bias=dev["sel_bias"],
+                             expert_start=expert_start, renormalize=renorm)
+    sel, wts = oracle.route(inp["logits"], inp["sel_bias"], w.top_k, renorm, expert_start)
+    off, rexp, src, row_of = oracle.dispatch(sel, w.E, expert_start)
+    got = {"selected": u32(r["selected_experts"]), "weights": r["weights"].cpu().numpy(),
+           "offsets": r["offsets"].cpu().numpy(), "row_experts": u32(r["row_experts"]),
+           "src_token": r["src_token"].cpu().numpy(), "row_of": r["row_of"].cpu().numpy()}
+    check_routing(got, {"selected": sel, "weights": wts, "offsets": off, "row_experts": rexp, "src_token": src,
+                        "row_of": row_of}, "options")
+
+
+def test_route_ties_and_empty_experts():
+    # many exact ties (logits on a coarse grid) and experts nobody picks
+    T, E, k = 700, 96, 4
+    rng = np.random.default_rng(3)
+    logits = (rng.integers(0, 3, (T, E)).astype(np.float32))
+    logits[:, 50:] = -5.0
+    x = inputs.random_bf16(rng, (T, 24))
+    xd = torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).cuda()
+    r = B.moe_route_dispatch(xd, torch.from_numpy(logits).cuda(), k, E=E)
+    sel, wts = oracle.route(logits, None, k)
+    off, rexp, src, row_of = oracle.dispatch(sel, E)
+    assert np.array_equal(u32(r["selected_experts"]), sel)
+    assert np.array_equal(r["offsets"].cpu().numpy(), off)
+    assert np.array_equal(r["src_token"].cpu().numpy(), src)
+    assert np.array_equal(r["row_of"].cpu().numpy(), row_of)
+    assert np.all(np.diff(off)[50:] == 0)
+
+
+def test_route_large_expert_count_and_top_k_32():
+    T, E, k = 130, 4096, 32
+    rng = np.random.default_rng(4)
+    logits = rng.standard_normal((T, E)).astype(np.float32)
+    x = inputs.random_bf16(rng, (T, 8))
+    xd = torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).cuda()
+    r = B.moe_route_dispatch(xd, torch.from_numpy(logits).cuda(), k, E=E)
+    sel, wts = oracle.route(logits, None, k)
+    off, rexp, src, row_of = oracle.dispatch(sel, E)
+    assert np.array_equal(u32(r["selected_experts"]), sel)
+    assert np.max(np.abs(r["weights"].cpu().numpy() - wts)) <= 2e-6
+    assert np.array_equal(r["offsets"].cpu().numpy(), off)
+    assert np.array_equal(r["row_of"].cpu().numpy(), row_of)
+
+
+# ------------------------------------------------------------------ forward, every row
+
+SMALL = {
+    "tiny": {},
+    "decode": {},
+    "prefill": dict(T=512, H=256, I=128, E=16),
+    "wide": dict(T=256, H=256, I=128, E=64),
+    "skewed": dict(T=1024, H=512, I=256, E=16),
+}
+
+
+def _oracle_forward_all(inp):
+    return oracle.forward(inp)
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_forward_every_row(name, path):
+    inp = generated(name, **SMALL[name])
+    res, dev, buf = gpu_forward_numpy(inp)
+    want = _oracle_forward_all(inp)
+    check_routing(res, want, name)
+    assert np.array_equal(res["values"], want["values"])
+    for key in ("G", "U", "h", "y", "out"):
+        check_close(res[key], want[key], "%s/%s" % (name, key))
+    assert res["status"] == 0
+
+
+def test_forward_is_deterministic(path):
+    inp = generated("prefill", **SMALL["prefill"])
+    a, _, _ = gpu_forward_numpy(inp)
+    b, _, _ = gpu_forward_numpy(inp)
+    for key in ("values", "G", "U", "h", "y", "out"):
+        assert np.array_equal(a[key], b[key]), key
+
+
+# ------------------------------------------------------------------ forward, full size, sampled rows
+
+@pytest.mark.parametrize("name", ["decode", "prefill", "wide", "skewed"])
+def test_forward_full_size_sampled(name, path):
+    inp = generated(name)
+    w = inp["workload"]
+    res, dev, buf = gpu_forward_numpy(inp)
+    rows = sample_rows(res["offsets"], n_experts=4, rows_per=6)
+    tokens = np.array([0, w.T // 3, w.T - 1], np.int64)
+    want = oracle.forward(inp, rows=rows, tokens=tokens)
+    used = want["rows_used"]
+    for key in ("G", "U", "h", "y"):
+        check_close(res[key][used], want[key], "%s/%s" % (name, key))
+    check_close(res["out"][tokens], want["out"], name + "/out")
+    assert res["status"] == 0

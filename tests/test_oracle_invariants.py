@@ -113,6 +113,13 @@ def test_dweights_closed_form_and_dy():
     assert only_dw[0] is None and np.array_equal(only_dw[1], dw)
 
 
+def test_incomplete_group_is_rejected():
+    rng = np.random.default_rng(1)
+    proj = inputs.draw_projection(rng, 1, 48, 16, 16, "f16", False, 0.0)
+    with pytest.raises(ValueError):
+        oracle.project(np.zeros((1, 48), np.uint16), "bf16", np.zeros(1, np.int32), proj, "f16", 32)
+
+
 @pytest.mark.parametrize("sdt", ["f16", "bf16"])
 def test_projection_adjoint_identity(sdt):
     rng = np.random.default_rng(8)
@@ -147,7 +154,7 @@ def _exact_chain(inp, xs, route_res):
 
 @pytest.mark.parametrize("sdt", ["f16", "bf16"])
 def test_whole_ffn_vjp_matches_finite_difference(sdt):
-    w = scaled(WORKLOADS["tiny"], T=6, H=32, I=24, E=4, top_k=2, group=16, scale_dtype=sdt)
+    w = scaled(WORKLOADS["tiny"], T=6, H=32, I=48, E=4, top_k=2, group=16, scale_dtype=sdt)
     inp = inputs.generate(w)
     rng = np.random.default_rng(9)
     sel, wts = oracle.route(inp["logits"], None, w.top_k)

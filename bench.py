@@ -173,9 +173,6 @@ def main():
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
     stream = torch.cuda.current_stream()
 
-    # dominant-kernel events: the gate/up projection launch
-    k_ev = []
-
     def step(record=None):
         if record is not None:
             ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -184,13 +181,16 @@ def main():
                                  device_status=buf.status, out=buf.route)
         if record is not None:
             ev0.record()
-        B.awq_grouped_gate_up_swiglu(r["values"], r["offsets"], dev["gate"], dev["up"], w.group,
-                                     device_status=buf.status, out=buf.h) if buf.G is None else \
+        if buf.G is None:
+            B.awq_grouped_gate_up_swiglu(r["values"], r["offsets"], dev["gate"], dev["up"], w.group,
+                                         device_status=buf.status, out=buf.h, workspace=buf.proj_ws)
+        else:
             _gate_up_keep(B, r, dev, w, buf)
         if record is not None:
             ev1.record()
             record.append((ev0, ev1))
-        B.awq_grouped_down(buf.h, r["offsets"], dev["down"], w.group, device_status=buf.status, out=buf.y)
+        B.awq_grouped_down(buf.h, r["offsets"], dev["down"], w.group, device_status=buf.status, out=buf.y,
+                           workspace=buf.proj_ws)
         B.moe_combine(buf.y, r["weights"], r["selected_experts"], r["row_of"], device_status=buf.status,
                       out=buf.out)
         if w.backward:
@@ -356,7 +356,7 @@ def _gate_up_keep(B, r, dev, w, buf):
         B._ptr(gate["qweight"]), B._ptr(gate["qzeros"]), B._ptr(gate["scales"]), B._ptr(gate["bias"]),
         B._ptr(up["qweight"]), B._ptr(up["qzeros"]), B._ptr(up["scales"]), B._ptr(up["bias"]),
         B._dt(gate["scales"].dtype), B.MOE_F32, w.group, B._ptr(buf.h), B._ptr(buf.G), B._ptr(buf.U),
-        B._ptr(buf.status), st)
+        B._ptr(buf.proj_ws), 0 if buf.proj_ws is None else buf.proj_ws.numel(), B._ptr(buf.status), st)
     B._check("awq_grouped_gate_up_swiglu", s)
 
 

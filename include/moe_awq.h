@@ -161,6 +161,10 @@ MOE_API moe_status moe_route_dispatch(const void *x, moe_dtype x_dtype, int64_t 
  *  up_out   [A, I]   act_dtype U = RNE(sum_kk values*Wu + bias_u), or NULL
  * The GPU path (small per-expert batches on warp-level tensor-core tiles,
  * large ones on tcgen05/TMEM tiles) is chosen inside from A and E.
+ *  workspace  device scratch of awq_projection_workspace_size(A, H, I, E, group_size, 2)
+ *             bytes (16-byte aligned; may be NULL when that size is 0):
+ *             split-K partial sums of the small-batch tiles.  Its contents
+ *             need no initialisation and are dead after the call.
  * Device errors: MOE_DEVICE_ERR_OFFSETS.
  * ---------------------------------------------------------------------- */
 MOE_API moe_status awq_grouped_gate_up_swiglu(
@@ -171,7 +175,14 @@ MOE_API moe_status awq_grouped_gate_up_swiglu(
     const int32_t *qweight_up, const int32_t *qzeros_up, const void *scales_up,
     const void *bias_up,
     moe_dtype scale_dtype, moe_dtype bias_dtype, int64_t group_size,
-    void *h, void *gate_out, void *up_out, int32_t *device_status, void *stream);
+    void *h, void *gate_out, void *up_out, void *workspace, size_t workspace_bytes,
+    int32_t *device_status, void *stream);
+
+/* Workspace bytes the projection of A rows (input width K, output width N,
+ * E experts, AWQ group size; nproj = 2 for the gate/up pair, 1 for a single
+ * projection) needs under the current projection path; 0 if none. */
+MOE_API size_t awq_projection_workspace_size(int64_t A, int64_t K, int64_t N, int64_t E,
+                                             int64_t group_size, int32_t nproj);
 
 /* ------------------------------------------------------------------------
  * awq_grouped_down -- the down projection of [PE] packed_swiglu_forward; also
@@ -181,14 +192,16 @@ MOE_API moe_status awq_grouped_gate_up_swiglu(
  *
  *  input [A, K] act_dtype (F16 or BF16); output [A, N] act_dtype:
  *  output[r, n] = RNE(sum_kk input[r,kk] * W[e,kk,n] + bias[e,n]).
+ *  workspace: awq_projection_workspace_size(A, K, N, E, group_size, 1) bytes (see
+ *  awq_grouped_gate_up_swiglu).
  * Device errors: MOE_DEVICE_ERR_OFFSETS.
  * ---------------------------------------------------------------------- */
 MOE_API moe_status awq_grouped_down(const void *input, moe_dtype act_dtype, int64_t A, int64_t K,
                             int64_t N, const int32_t *offsets, int64_t E,
                             const int32_t *qweight, const int32_t *qzeros, const void *scales,
                             const void *bias, moe_dtype scale_dtype, moe_dtype bias_dtype,
-                            int64_t group_size, void *output, int32_t *device_status,
-                            void *stream);
+                            int64_t group_size, void *output, void *workspace,
+                            size_t workspace_bytes, int32_t *device_status, void *stream);
 
 /* ------------------------------------------------------------------------
  * moe_combine -- [MX] MoeDispatchOps::moe_combine ("ascending expert-ID

@@ -43,8 +43,10 @@ _SIGS = {
     "moe_route_dispatch_workspace_size": (SZ, [I64, I64, I32]),
     "moe_route_dispatch": (C.c_int, [P, C.c_int, I64, I64, P, P, I64, I32, I32, I32, P, P, P, P, P, P, P, P, SZ, P, P]),
     "awq_grouped_gate_up_swiglu": (C.c_int, [P, C.c_int, I64, I64, I64, P, I64, P, P, P, P, P, P, P, P, C.c_int,
-                                             C.c_int, I64, P, P, P, P, P]),
-    "awq_grouped_down": (C.c_int, [P, C.c_int, I64, I64, I64, P, I64, P, P, P, P, C.c_int, C.c_int, I64, P, P, P]),
+                                             C.c_int, I64, P, P, P, P, SZ, P, P]),
+    "awq_projection_workspace_size": (SZ, [I64, I64, I64, I64, I64, I32]),
+    "awq_grouped_down": (C.c_int, [P, C.c_int, I64, I64, I64, P, I64, P, P, P, P, C.c_int, C.c_int, I64, P, P, SZ, P,
+                                   P]),
     "moe_combine": (C.c_int, [P, C.c_int, I64, P, P, P, I64, I64, I32, P, P, P]),
     "moe_combine_backward": (C.c_int, [P, P, C.c_int, I64, P, P, I64, I64, I32, P, P, P, P]),
     "awq_input_backward": (C.c_int, [P, C.c_int, I64, I64, I64, P, I64, P, P, P, C.c_int, I64, P, P, P, P, P, P, P]),
@@ -152,7 +154,20 @@ def _bias_dt(*biases):
     return MOE_F32
 
 
-def awq_grouped_gate_up_swiglu(values, offsets, gate, up, group, want_gu=False, device_status=None, out=None):
+def projection_workspace_size(A, K, N, E, group, nproj):
+    return int(lib().awq_projection_workspace_size(A, K, N, E, group, nproj))
+
+
+def _workspace(nbytes, device, workspace=None):
+    if nbytes == 0:
+        return None
+    if workspace is not None and workspace.numel() >= nbytes:
+        return workspace
+    return torch.empty(nbytes, dtype=torch.uint8, device=device)
+
+
+def awq_grouped_gate_up_swiglu(values, offsets, gate, up, group, want_gu=False, device_status=None, out=None,
+                               workspace=None):
     A, H = values.shape
     E = offsets.numel() - 1
     I = gate["qweight"].shape[2] * 8
@@ -160,25 +175,27 @@ def awq_grouped_gate_up_swiglu(values, offsets, gate, up, group, want_gu=False, 
     h = out if out is not None else torch.empty((A, I), dtype=values.dtype, device=values.device)
     G = torch.empty_like(h) if want_gu else None
     U = torch.empty_like(h) if want_gu else None
+    ws = _workspace(projection_workspace_size(A, H, I, E, group, 2), values.device, workspace)
     st = lib().awq_grouped_gate_up_swiglu(
         _ptr(values), _dt(values.dtype), A, H, I, _ptr(offsets), E,
         _ptr(gate["qweight"]), _ptr(gate["qzeros"]), _ptr(gate["scales"]), _ptr(gate.get("bias")),
         _ptr(up["qweight"]), _ptr(up["qzeros"]), _ptr(up["scales"]), _ptr(up.get("bias")),
-        sdt, _bias_dt(gate.get("bias"), up.get("bias")), group, _ptr(h), _ptr(G), _ptr(U), _ptr(device_status),
-        _stream())
+        sdt, _bias_dt(gate.get("bias"), up.get("bias")), group, _ptr(h), _ptr(G), _ptr(U), _ptr(ws),
+        0 if ws is None else ws.numel(), _ptr(device_status), _stream())
     _check("awq_grouped_gate_up_swiglu", st)
     return (h, G, U) if want_gu else h
 
 
-def awq_grouped_down(inp, offsets, proj, group, device_status=None, out=None):
+def awq_grouped_down(inp, offsets, proj, group, device_status=None, out=None, workspace=None):
     A, K = inp.shape
     E = offsets.numel() - 1
     N = proj["qweight"].shape[2] * 8
     y = out if out is not None else torch.empty((A, N), dtype=inp.dtype, device=inp.device)
+    ws = _workspace(projection_workspace_size(A, K, N, E, group, 1), inp.device, workspace)
     st = lib().awq_grouped_down(
         _ptr(inp), _dt(inp.dtype), A, K, N, _ptr(offsets), E, _ptr(proj["qweight"]), _ptr(proj["qzeros"]),
         _ptr(proj["scales"]), _ptr(proj.get("bias")), _dt(proj["scales"].dtype), _bias_dt(proj.get("bias")), group,
-        _ptr(y), _ptr(device_status), _stream())
+        _ptr(y), _ptr(ws), 0 if ws is None else ws.numel(), _ptr(device_status), _stream())
     _check("awq_grouped_down", st)
     return y
 

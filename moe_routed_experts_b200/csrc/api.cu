@@ -47,6 +47,9 @@ static int choose_path(int64_t A, int64_t E) {
   return (A >= 32 * E) ? 2 : 1;
 }
 
+// Token columns per warp-level tile: 16 when experts average >= 12 rows.
+static int small_tile_tokens(int64_t A, int64_t E) { return A >= 12 * E ? 2 : 1; }
+
 static moe_status check_payload_geom(const char *fn, int64_t A, int64_t K, int64_t N, int64_t E, int64_t group,
                                      moe_dtype act_dt, moe_dtype scale_dt) {
   if (act_dt != MOE_F16 && act_dt != MOE_BF16)
@@ -88,12 +91,20 @@ extern "C" int32_t moe_set_projection_path(int32_t path) {
   return g_path.exchange(path);
 }
 
+extern "C" size_t awq_projection_workspace_size(int64_t A, int64_t K, int64_t N, int64_t E, int64_t group_size,
+                                                int32_t nproj) {
+  if (A <= 0 || E < 1 || K < 16 || N < 8 || group_size < 16 || (nproj != 1 && nproj != 2)) return 0;
+  if (choose_path(A, E) != 1) return 0;
+  const StreamPlan pl = stream_plan(A, K, N, E, group_size, nproj, small_tile_tokens(A, E));
+  return pl.fits ? pl.bytes : 0;
+}
+
 extern "C" moe_status awq_grouped_gate_up_swiglu(
     const void *values, moe_dtype act_dtype, int64_t A, int64_t H, int64_t I, const int32_t *offsets, int64_t E,
     const int32_t *qweight_gate, const int32_t *qzeros_gate, const void *scales_gate, const void *bias_gate,
     const int32_t *qweight_up, const int32_t *qzeros_up, const void *scales_up, const void *bias_up,
     moe_dtype scale_dtype, moe_dtype bias_dtype, int64_t group_size, void *h, void *gate_out, void *up_out,
-    int32_t *device_status, void *stream) {
+    void *workspace, size_t workspace_bytes, int32_t *device_status, void *stream) {
   const char *fn = "awq_grouped_gate_up_swiglu";
   moe_status s = check_payload_geom(fn, A, H, I, E, group_size, act_dtype, scale_dtype);
   if (s != MOE_OK) return s;
@@ -128,7 +139,9 @@ extern "C" moe_status awq_grouped_gate_up_swiglu(
   cudaStream_t st = as_stream(stream);
   const bool bf = scale_dtype == MOE_BF16;
   if (choose_path(A, E) == 2) return launch_fwd_tc(p, 2, bf, st);
-  launch_fwd_mma(p, 2, bf, A >= 12 * E ? 2 : 1, st);
+  const int nt = small_tile_tokens(A, E);
+  if (stream_plan(A, H, I, E, group_size, 2, nt).fits) return launch_fwd_stream(p, 2, bf, nt, workspace, workspace_bytes, st);
+  launch_fwd_mma(p, 2, bf, nt, st);
   return check_launch(fn);
 }
 
@@ -136,7 +149,8 @@ extern "C" moe_status awq_grouped_down(const void *input, moe_dtype act_dtype, i
                                        const int32_t *offsets, int64_t E, const int32_t *qweight,
                                        const int32_t *qzeros, const void *scales, const void *bias,
                                        moe_dtype scale_dtype, moe_dtype bias_dtype, int64_t group_size,
-                                       void *output, int32_t *device_status, void *stream) {
+                                       void *output, void *workspace, size_t workspace_bytes,
+                                       int32_t *device_status, void *stream) {
   const char *fn = "awq_grouped_down";
   moe_status s = check_payload_geom(fn, A, K, N, E, group_size, act_dtype, scale_dtype);
   if (s != MOE_OK) return s;
@@ -163,7 +177,9 @@ extern "C" moe_status awq_grouped_down(const void *input, moe_dtype act_dtype, i
   cudaStream_t st = as_stream(stream);
   const bool bf = scale_dtype == MOE_BF16;
   if (choose_path(A, E) == 2) return launch_fwd_tc(p, 1, bf, st);
-  launch_fwd_mma(p, 1, bf, A >= 12 * E ? 2 : 1, st);
+  const int nt = small_tile_tokens(A, E);
+  if (stream_plan(A, K, N, E, group_size, 1, nt).fits) return launch_fwd_stream(p, 1, bf, nt, workspace, workspace_bytes, st);
+  launch_fwd_mma(p, 1, bf, nt, st);
   return check_launch(fn);
 }
 

@@ -24,52 +24,10 @@
 //   MMA's K = output features): one word gives (slot p, slot p+4) = logical
 //   columns (2p, 2p+1) at the same row, which is an A pair as it stands.
 //   CTA = (64 input rows, one expert), 4 warps splitting the feature range.
+#include "dequant.cuh"
 #include "proj.cuh"
 
 namespace moe {
-
-// ------------------------------------------------------------------ coefficient helpers
-//
-// Forward constants of one word column for one group: zero pairs
-// (magic+z, magic+z) of logical columns 2p (zlo) and 2p+1 (zhi), and scale
-// pairs (s, s) of the same columns.
-template <typename MT>
-struct FwdConsts {
-  uint32_t zlo[4], zhi[4], slo[4], shi[4];
-  __device__ __forceinline__ void load(uint32_t zw, uint4 sv) {
-    constexpr uint32_t M = Dq<MT>::kMagic2;
-    const uint32_t sw[4] = {sv.x, sv.y, sv.z, sv.w};
-#pragma unroll
-    for (int p = 0; p < 4; ++p) {
-      zlo[p] = (((zw >> (4 * p)) & 0xFu) * 0x10001u) | M;       // slot p   -> column 2p
-      zhi[p] = (((zw >> (4 * p + 16)) & 0xFu) * 0x10001u) | M;  // slot p+4 -> column 2p+1
-      slo[p] = (sw[p] & 0xFFFFu) * 0x10001u;                      // s[2p]
-      shi[p] = (sw[p] >> 16) * 0x10001u;                          // s[2p+1]
-    }
-  }
-};
-
-// Coefficient pairs of column 2p (lo) and 2p+1 (hi) at two consecutive input
-// rows, from the words wa (row kk) and wb (row kk+1) of the same column.
-template <typename MT>
-__device__ __forceinline__ void fwd_pairs(uint32_t wa, uint32_t wb, int p, const FwdConsts<MT> &c, uint32_t &lo,
-                                          uint32_t &hi) {
-  constexpr uint32_t M = Dq<MT>::kMagic2;
-  const uint32_t u = prmt(wa, wb, 0x5410u);  // slots 0..3 of wa | slots 0..3 of wb
-  const uint32_t v = prmt(wa, wb, 0x7632u);  // slots 4..7 of wa | slots 4..7 of wb
-  lo = Dq<MT>::coef(nib_pair<M>(u >> (4 * p)), c.zlo[p], c.slo[p]);
-  hi = Dq<MT>::coef(nib_pair<M>(v >> (4 * p)), c.zhi[p], c.shi[p]);
-}
-
-// Input-VJP extraction: coefficient pair of logical columns (2p, 2p+1) of one
-// word, with zero word zw and the scale pair sp = (s[2p], s[2p+1]).
-template <typename MT>
-__device__ __forceinline__ uint32_t word_pair(uint32_t w, uint32_t zw, uint32_t sp, int p) {
-  constexpr uint32_t M = Dq<MT>::kMagic2;
-  return Dq<MT>::coef(nib_pair<M>(w >> (4 * p)), nib_pair<M>(zw >> (4 * p)), sp);
-}
-
-__device__ __forceinline__ uint4 ldg16(const uint16_t *p) { return __ldg(reinterpret_cast<const uint4 *>(p)); }
 
 // ------------------------------------------------------------------ forward
 
@@ -141,7 +99,7 @@ __global__ void __launch_bounds__(128) awq_fwd_mma_kernel(ProjParams p) {
       for (int d = 0; d < D; ++d) {
         const int64_t s = base + d;
         if (s < s_end) {
-          const int64_t grp = (s * 16) / p.group;
+          const int64_t grp = (int64_t)((uint32_t)(s * 16) / (uint32_t)p.group);
           if (grp != cur_grp) {
             cur_grp = grp;
 #pragma unroll
@@ -281,9 +239,14 @@ __global__ void __launch_bounds__(128) awq_bwd_mma_kernel(BwdParams p) {
       gok[nt] = tr < m;
       grow[nt] = (r0 + (gok[nt] ? tr : 0)) * p.N;
     }
-    for (int64_t s = s_begin; s < s_end; ++s) {
-      const int j = (int)(s / spp);
-      const int64_t wc = (s % spp) * 4 + t;
+    int j = (int)(s_begin / spp);
+    int64_t sj = s_begin - (int64_t)j * spp;  // step within projection j
+    for (int64_t s = s_begin; s < s_end; ++s, ++sj) {
+      if (sj == spp) {
+        sj = 0;
+        ++j;
+      }
+      const int64_t wc = sj * 4 + t;
       const bool wc_ok = wc < NW;
       const int64_t wcs = wc_ok ? wc : 0;
       const int32_t *qw = p.qw[j] + (int64_t)e * p.K * NW + wcs;

@@ -1,0 +1,561 @@
+// Grouped AWQ forward for small per-expert batches (decode): packed words
+// stream through shared memory by TMA and warp-level tensor-core tiles
+// (mma.sync m16n8k16, FP32 accumulate) consume them.  Here the packed-weight
+// bytes bound the time, so the design is about reading each weight byte
+// exactly once, in whole 128-byte lines, with enough bytes in flight.
+//
+// ruda-tensor 0.21.34, src/packed_experts.rs -- packed_expert_forward /
+//   packed_swiglu_forward (gate/up/down of the selected experts, SwiGLU);
+// ruda-tensor 0.21.33, src/frozen_awq.rs -- AWQ nibble order and scale-dtype
+//   coefficient rounding.
+//
+// Work unit = (expert e, token tile tt of 8*NT rows, slab sl, K split kq).
+// A slab is 512 output columns: for the gate/up pair, 32 packed word
+// columns (one 128-byte row segment) of each projection; for a single
+// projection, 64 word columns (two 128-byte segments).  A unit covers K/KQ
+// input rows.  Persistent CTAs (1 producer warp + 8 consumer warps) take
+// contiguous ranges of the expert-major unit list.
+//   producer: per unit, 1-D bulk copies of the tile's activation rows
+//     (double-buffered), then per 32 input rows one stage = two TMA boxes of
+//     [32 rows][32 words] with 128-byte swizzle (8 KB), kStages in flight.
+//   consumer warp w: box w/4, word columns (w%4)*8 .. +7 of it, all rows of
+//     the unit.  Lane (g, t) reads rows t, t+4, t+8, t+12 of column g (the
+//     MMA's K index {2t, 2t+1, 2t+8, 2t+9} stands for them); the swizzle
+//     keeps those reads at most 2-way bank-conflicted.  The activation tile
+//     is converted to the scale dtype and permuted to that row order once
+//     per unit, so each B fragment is one 8-byte shared load.
+//   epilogue: with the whole K in the unit (KQ = 1), accumulators go
+//     through shared memory to bias, rounding and SwiGLU; with KQ > 1 each
+//     unit stores its FP32 partial sums to the workspace and a second kernel
+//     sums the KQ splits in kq order (deterministic) and finishes the rows.
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "dequant.cuh"
+#include "proj.cuh"
+#include "tma.cuh"
+
+namespace moe {
+
+// ------------------------------------------------------------------ host: tensor maps
+
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+bool make_map_2d(CUtensorMap *map, const void *base, CUtensorMapDataType dt, int elem_bytes, uint64_t inner,
+                 uint64_t outer, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swizzle) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {inner * (uint64_t)elem_bytes};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, dt, 2, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// ------------------------------------------------------------------ device
+
+namespace stream {
+constexpr int kCW = 8;                    // consumer warps
+constexpr int kThreads = (kCW + 1) * 32;  // + one producer warp
+constexpr int kStages = 6;
+constexpr int kRows = 32;                 // input rows per stage (two 16-row MMA steps)
+constexpr int kBoxW = 32;                 // words per box row (128 bytes)
+constexpr int kBox = kRows * kBoxW * 4;   // [32 rows][32 words] = 4 KB
+constexpr int kStageBytes = 2 * kBox;     // two boxes per stage
+constexpr int kF = 512;                   // output columns of a unit
+constexpr int kBarBytes = 1024;           // barrier block; stages start 1024-byte aligned
+}  // namespace stream
+
+// Largest e with pre[e] <= u (pre is the exclusive prefix of units per expert).
+__device__ __forceinline__ int unit_expert(const int32_t *pre, int E, int64_t u) {
+  int lo = 0, hi = E - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (pre[mid] <= u) lo = mid;
+    else hi = mid - 1;
+  }
+  return lo;
+}
+
+// Byte offset of word (row, col) in a [32][32]-word box written by TMA with
+// 128-byte swizzle (16-byte chunk index XOR row mod 8).
+__device__ __forceinline__ int box_offset(int row, int col) {
+  return row * 128 + ((((col >> 2) ^ row) & 7) << 4) + ((col & 3) << 2);
+}
+
+struct UnitInfo {
+  int e, tt, sl, kq;
+  int64_t r0;
+  int m;
+};
+
+__device__ __forceinline__ UnitInfo unit_info(const int32_t *pre, const int32_t *offsets, int E, int S, int KQ,
+                                              int64_t u) {
+  UnitInfo ui;
+  ui.e = unit_expert(pre, E, u);
+  const int64_t local = u - pre[ui.e];
+  ui.kq = (int)(local % KQ);
+  ui.sl = (int)((local / KQ) % S);
+  ui.tt = (int)(local / ((int64_t)KQ * S));
+  ui.r0 = offsets[ui.e];
+  ui.m = offsets[ui.e + 1] - (int32_t)ui.r0;
+  return ui;
+}
+
+// Final values of 8 consecutive output columns n0.. of row `row` of local
+// expert e from FP32 sums (gate sums g, up sums u for the pair): bias, one
+// rounding to the activation dtype, SwiGLU from the rounded G and U.
+template <int NPROJ>
+__device__ __forceinline__ void finish8(const ProjParams &p, int e, int64_t row, int64_t n0, const float *g,
+                                        const float *u) {
+  uint32_t o[4];
+  if (NPROJ == 2) {
+    uint32_t og[4], ou[4];
+#pragma unroll
+    for (int i = 0; i < 8; i += 2) {
+      float gv[2], uv[2];
+#pragma unroll
+      for (int d = 0; d < 2; ++d) {
+        gv[d] = g[i + d];
+        uv[d] = u[i + d];
+        if (p.bias[0]) gv[d] += ld_as_float(p.bias[0], p.bias_dt, (int64_t)e * p.N + n0 + i + d);
+        if (p.bias[1]) uv[d] += ld_as_float(p.bias[1], p.bias_dt, (int64_t)e * p.N + n0 + i + d);
+      }
+      const uint16_t gb0 = f32_to_bits(gv[0], p.act_dt), gb1 = f32_to_bits(gv[1], p.act_dt);
+      const uint16_t ub0 = f32_to_bits(uv[0], p.act_dt), ub1 = f32_to_bits(uv[1], p.act_dt);
+      const float g0 = bits_to_f32(gb0, p.act_dt), g1 = bits_to_f32(gb1, p.act_dt);
+      const float x0 = bits_to_f32(ub0, p.act_dt), x1 = bits_to_f32(ub1, p.act_dt);
+      const float h0 = g0 / (1.f + expf(-g0)) * x0, h1 = g1 / (1.f + expf(-g1)) * x1;
+      og[i / 2] = uint32_t(gb0) | (uint32_t(gb1) << 16);
+      ou[i / 2] = uint32_t(ub0) | (uint32_t(ub1) << 16);
+      o[i / 2] = uint32_t(f32_to_bits(h0, p.act_dt)) | (uint32_t(f32_to_bits(h1, p.act_dt)) << 16);
+    }
+    if (p.gout) *reinterpret_cast<uint4 *>(p.gout + row * p.N + n0) = make_uint4(og[0], og[1], og[2], og[3]);
+    if (p.uout) *reinterpret_cast<uint4 *>(p.uout + row * p.N + n0) = make_uint4(ou[0], ou[1], ou[2], ou[3]);
+  } else {
+#pragma unroll
+    for (int i = 0; i < 8; i += 2) {
+      float yv[2];
+#pragma unroll
+      for (int d = 0; d < 2; ++d) {
+        yv[d] = g[i + d];
+        if (p.bias[0]) yv[d] += ld_as_float(p.bias[0], p.bias_dt, (int64_t)e * p.N + n0 + i + d);
+      }
+      o[i / 2] = uint32_t(f32_to_bits(yv[0], p.act_dt)) | (uint32_t(f32_to_bits(yv[1], p.act_dt)) << 16);
+    }
+  }
+  *reinterpret_cast<uint4 *>(p.out + row * p.N + n0) = make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+template <typename MT, int NPROJ, int NT>
+__global__ void __launch_bounds__(stream::kThreads, 2)
+    awq_fwd_stream_kernel(const __grid_constant__ CUtensorMap map0, const __grid_constant__ CUtensorMap map1,
+                          ProjParams p) {
+  using namespace stream;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  // 128-byte-swizzled TMA boxes need 1024-byte aligned destinations
+  uint8_t *smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
+  const int E = p.E, KQ = p.kq;
+  const int64_t K = p.K, Kq = K / KQ;
+  const int64_t NW = p.N / 8;
+  constexpr int kSlabW = NPROJ == 2 ? kBoxW : 2 * kBoxW;  // word columns of a slab
+  const int S = (int)((NW + kSlabW - 1) / kSlabW);       // slabs per expert
+  const int nst = (int)(Kq / kRows);                     // stages per unit
+  const int xs_pitch = (int)(Kq * 2 + 16);  // bytes per converted token row (pad: conflict-free B loads)
+  const int xraw_bytes = (int)(8 * NT * Kq * 2);
+  const int64_t ncols = (int64_t)NPROJ * p.N;  // columns of the split-K partial rows
+
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem);
+  uint64_t *empty = full + kStages;
+  uint64_t *xfull = empty + kStages;
+  uint64_t *xempty = xfull + 2;
+  uint8_t *stages = smem + kBarBytes;
+  uint8_t *xraw = stages + kStages * kStageBytes;  // 2 buffers
+  uint8_t *xs = xraw + 2 * xraw_bytes;
+  float *red = reinterpret_cast<float *>(xs + 8 * NT * xs_pitch);  // [8*NT][kF]
+  int32_t *pre = reinterpret_cast<int32_t *>(red + 8 * NT * kF);    // [E + 1]
+  int32_t *cnt = pre + (E + 1);                                    // [E]
+  int32_t *tmp = cnt + E;                                          // [32]
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kCW);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&xfull[b], 1);
+      mbar_init(&xempty[b], kCW);
+    }
+    fence_mbar_init();
+  }
+  // units per expert; an inconsistent row range is flagged and skipped
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    const int32_t a = p.offsets[e], b = p.offsets[e + 1];
+    const bool bad = a < 0 || b < a || (int64_t)b > p.A || (e == 0 && a != 0) || (e == E - 1 && (int64_t)b != p.A);
+    if (bad && blockIdx.x == 0) report(p.status, MOE_DEVICE_ERR_OFFSETS);
+    cnt[e] = bad ? 0 : S * KQ * ((b - a + 8 * NT - 1) / (8 * NT));
+  }
+  __syncthreads();
+  block_exclusive_scan(cnt, E, pre, tmp);
+  const int64_t U = pre[E];
+  const int64_t u0 = U * blockIdx.x / gridDim.x, u1 = U * (blockIdx.x + 1) / gridDim.x;
+
+  if (warp == kCW) {
+    // ---------------- producer (one lane).  The activation tile of unit
+    // u+1 is requested when unit u starts, one unit ahead of its use.
+    if (lane != 0) return;
+    auto load_x = [&](int64_t u, uint32_t xi) {
+      const UnitInfo ui = unit_info(pre, p.offsets, E, S, KQ, u);
+      const int tok0 = ui.tt * 8 * NT, mrows = min(8 * NT, ui.m - tok0);
+      const uint32_t xb = xi & 1, xuse = xi >> 1;
+      if (xuse > 0 && !mbar_wait(&xempty[xb], (xuse - 1) & 1, p.status)) return;
+      mbar_arrive_expect_tx(&xfull[xb], (uint32_t)(mrows * Kq * 2));
+      for (int r = 0; r < mrows; ++r)
+        bulk_load(xraw + xb * xraw_bytes + r * Kq * 2, p.x + (ui.r0 + tok0 + r) * K + ui.kq * Kq,
+                  (uint32_t)(Kq * 2), &xfull[xb]);
+    };
+    if (u0 < u1) load_x(u0, 0);
+    uint32_t it = 0, xi = 0;
+    for (int64_t u = u0; u < u1; ++u, ++xi) {
+      if (u + 1 < u1) load_x(u + 1, xi + 1);
+      const UnitInfo ui = unit_info(pre, p.offsets, E, S, KQ, u);
+      const int32_t row0 = (int32_t)(ui.e * K + ui.kq * Kq);
+      for (int c = 0; c < nst; ++c, ++it) {
+        const uint32_t s = it % kStages, use = it / kStages;
+        if (use > 0 && !mbar_wait(&empty[s], (use - 1) & 1, p.status)) continue;
+        mbar_arrive_expect_tx(&full[s], kStageBytes);
+        uint8_t *dst = stages + s * kStageBytes;
+        if (NPROJ == 2) {
+          tma_load_2d(dst, &map0, &full[s], ui.sl * kBoxW, row0 + kRows * c);
+          tma_load_2d(dst + kBox, &map1, &full[s], ui.sl * kBoxW, row0 + kRows * c);
+        } else {
+          tma_load_2d(dst, &map0, &full[s], ui.sl * 2 * kBoxW, row0 + kRows * c);
+          tma_load_2d(dst + kBox, &map0, &full[s], ui.sl * 2 * kBoxW + kBoxW, row0 + kRows * c);
+        }
+      }
+    }
+    return;
+  }
+
+  // ---------------- consumers
+  const int g = lane >> 2, t = lane & 3;
+  const int bw = warp >> 2, cgw = warp & 3;  // box and column group of this warp
+  const int jw = NPROJ == 2 ? bw : 0;        // projection of this warp
+  const int64_t ngroups = K / p.group;
+  const int32_t *qz = p.qz[jw];
+  const uint16_t *sc = p.sc[jw];
+  // byte offsets of rows t and t+4 of column cgw*8+g in a swizzled box; rows
+  // t + 4i + 16h differ from these by multiples of 8 rows (same swizzle)
+  const int woff0 = box_offset(t, cgw * 8 + g), woff1 = box_offset(t + 4, cgw * 8 + g);
+  uint32_t it = 0, xi = 0;
+  for (int64_t u = u0; u < u1; ++u, ++xi) {
+    const UnitInfo ui = unit_info(pre, p.offsets, E, S, KQ, u);
+    const int tok0 = ui.tt * 8 * NT, mrows = min(8 * NT, ui.m - tok0);
+    const int e = ui.e;
+    const int64_t wc = NPROJ == 2 ? (int64_t)ui.sl * kBoxW + cgw * 8 + g
+                                  : (int64_t)ui.sl * 2 * kBoxW + bw * kBoxW + cgw * 8 + g;
+    const bool wc_ok = wc < NW;
+    const int64_t wcs = wc_ok ? wc : 0;
+    const int64_t kbase = (int64_t)ui.kq * Kq;
+    const int32_t *qzp = qz + (e * ngroups) * NW + wcs;
+    const uint16_t *scp = sc + (e * ngroups) * p.N + 8 * wcs;
+    int64_t grp = kbase / p.group;
+    // the first group's zeros/scales are requested before the activation
+    // tile is converted, so their latency overlaps that work
+    uint32_t pf_zw = wc_ok ? (uint32_t)__ldg(qzp + grp * NW) : 0u;
+    uint4 pf_sv = wc_ok ? __ldg(reinterpret_cast<const uint4 *>(scp + grp * p.N)) : make_uint4(0, 0, 0, 0);
+
+    // activation tile: raw rows -> scale dtype, row order t, t+4, t+8, t+12 per 16
+    const uint32_t xb = xi & 1;
+    mbar_wait(&xfull[xb], (xi >> 1) & 1, p.status);
+    {
+      const uint8_t *src = xraw + xb * xraw_bytes;
+      const int64_t halves = (int64_t)mrows * (Kq / 8);
+      for (int64_t q = threadIdx.x; q < halves; q += kCW * 32) {
+        const int tok = (int)(q / (Kq / 8));
+        const int64_t hb = q % (Kq / 8), blk = hb >> 1, h = hb & 1;
+        const uint4 v = *reinterpret_cast<const uint4 *>(src + (tok * Kq + blk * 16 + h * 8) * 2);
+        const uint32_t pr[4] = {prmt(v.x, v.z, 0x5410u), prmt(v.x, v.z, 0x7632u), prmt(v.y, v.w, 0x5410u),
+                                prmt(v.y, v.w, 0x7632u)};  // (row i, row i+4) of the half
+        uint8_t *dst = xs + tok * xs_pitch + (blk * 16 + 2 * h) * 2;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) *reinterpret_cast<uint32_t *>(dst + 8 * i) = act_pair_to_mt<MT>(pr[i], p.act_dt);
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&xempty[xb]);
+    named_barrier(1, kCW * 32);
+
+    // acc: every slot in its true scale; acc16: odd slots taken 16 times
+    // larger (F16 groups whose scales allow it, see fwd_pairs16)
+    float acc[NT][4][4], acc16[NT][2][4];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc[nt][q][i] = 0.f;
+#pragma unroll
+      for (int q = 0; q < 2; ++q)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc16[nt][q][i] = 0.f;
+    }
+    FwdConsts<MT> cst;
+    bool x16 = false;
+    const int spg = p.group / kRows;  // stages per group (group % 32 == 0 on this path)
+    int gstage = (int)((kbase % p.group) / kRows);
+    for (int c = 0; c < nst; ++c, ++it) {
+      const uint32_t s = it % kStages, ph = (it / kStages) & 1;
+      if (c == 0 || gstage == 0) {  // a stage lies inside one group
+        if (std::is_same<MT, __half>::value) {  // |s| <= 256 for all 8 scales of this column group
+          const uint32_t w4[4] = {pf_sv.x, pf_sv.y, pf_sv.z, pf_sv.w};
+          uint32_t big = 0;
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            big |= ((w4[i] & 0x7FFFu) > 0x5C00u) | (((w4[i] >> 16) & 0x7FFFu) > 0x5C00u);
+          x16 = big == 0;
+        }
+        cst.load(pf_zw, pf_sv, x16);
+        if (wc_ok && (grp + 1) * p.group < kbase + Kq) {  // prefetch the next group
+          pf_zw = (uint32_t)__ldg(qzp + (grp + 1) * NW);
+          pf_sv = __ldg(reinterpret_cast<const uint4 *>(scp + (grp + 1) * p.N));
+        }
+      }
+      if (++gstage == spg) {
+        gstage = 0;
+        ++grp;
+      }
+      if (mbar_wait(&full[s], ph, p.status)) {
+        const uint8_t *box = stages + s * kStageBytes + bw * kBox;
+        uint32_t w[2][4];
+        uint32_t b0[2][NT], b1[2][NT];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {  // two 16-row steps: rows 16h + {t, t+4, t+8, t+12}
+          w[h][0] = *reinterpret_cast<const uint32_t *>(box + woff0 + (16 * h) * 128);
+          w[h][1] = *reinterpret_cast<const uint32_t *>(box + woff1 + (16 * h) * 128);
+          w[h][2] = *reinterpret_cast<const uint32_t *>(box + woff0 + (16 * h + 8) * 128);
+          w[h][3] = *reinterpret_cast<const uint32_t *>(box + woff1 + (16 * h + 8) * 128);
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) {
+            const uint2 bv =
+                *reinterpret_cast<const uint2 *>(xs + (nt * 8 + g) * xs_pitch + (kRows * c + 16 * h + 4 * t) * 2);
+            b0[h][nt] = bv.x;
+            b1[h][nt] = bv.y;
+          }
+        }
+        bool done = false;
+        if constexpr (std::is_same<MT, __half>::value) {
+          if (x16) {
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              uint32_t af[4][4];
+              fwd_step<MT, true>(w[h][0], w[h][1], w[h][2], w[h][3], cst, af);
+#pragma unroll
+              for (int q = 0; q < 4; ++q)
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                  if (q & 1) mma16816<MT>(acc16[nt][q >> 1], af[q], b0[h][nt], b1[h][nt]);
+                  else mma16816<MT>(acc[nt][q], af[q], b0[h][nt], b1[h][nt]);
+                }
+            }
+            done = true;
+          }
+        }
+        if (!done) {
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            uint32_t af[4][4];
+            fwd_step<MT, false>(w[h][0], w[h][1], w[h][2], w[h][3], cst, af);
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+#pragma unroll
+              for (int nt = 0; nt < NT; ++nt) mma16816<MT>(acc[nt][q], af[q], b0[h][nt], b1[h][nt]);
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[s]);
+    }
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {  // fold the 16x-scaled odd slots back (exact power-of-two scaling)
+        acc[nt][1][i] += acc16[nt][0][i] * 0.0625f;
+        acc[nt][3][i] += acc16[nt][1][i] * 0.0625f;
+      }
+
+    if (KQ > 1) {
+      // split K: this unit's partial sums go to partials[kq][row][column];
+      // a second kernel sums the splits in kq order and finishes the outputs
+      float *prow = p.partials + ((int64_t)ui.kq * p.A + ui.r0 + tok0) * ncols;
+      if (wc_ok) {
+        const int64_t col0 = (int64_t)jw * p.N + wc * 8;
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+          for (int d = 0; d < 2; ++d) {
+            const int tk = nt * 8 + 2 * t + d;
+            if (tk < mrows) {
+#pragma unroll
+              for (int q = 0; q < 4; ++q)
+                __stcg(reinterpret_cast<float2 *>(prow + tk * ncols + col0 + 2 * q),
+                       make_float2(acc[nt][q][d], acc[nt][q][2 + d]));
+            }
+          }
+      }
+      continue;
+    }
+
+    // whole K in this unit: accumulators -> red[token][column], epilogue
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int f = bw * 256 + cgw * 64 + 8 * g + 2 * q, tk = nt * 8 + 2 * t;
+        red[tk * kF + f] = acc[nt][q][0];
+        red[(tk + 1) * kF + f] = acc[nt][q][1];
+        red[tk * kF + f + 1] = acc[nt][q][2];
+        red[(tk + 1) * kF + f + 1] = acc[nt][q][3];
+      }
+    named_barrier(1, kCW * 32);
+    constexpr int kOut = NPROJ == 2 ? kF / 2 : kF;  // output columns of the unit
+    for (int v8 = threadIdx.x; v8 < mrows * (kOut / 8); v8 += kCW * 32) {
+      const int tk = v8 / (kOut / 8), fq = (v8 % (kOut / 8)) * 8;
+      const int64_t n0 = (int64_t)ui.sl * kOut + fq;
+      if (n0 >= p.N) continue;
+      const float *g8 = red + tk * kF + fq;
+      finish8<NPROJ>(p, e, ui.r0 + tok0 + tk, n0, g8, g8 + 256);
+    }
+    named_barrier(1, kCW * 32);  // red is free again
+  }
+}
+
+// Split-K reduction: out[r, n..n+8) from sum over kq of partials[kq][r][.]
+// (in kq order), then bias, rounding and SwiGLU as in the fused epilogue.
+template <int NPROJ>
+__global__ void __launch_bounds__(256) awq_stream_reduce_kernel(ProjParams p) {
+  const int64_t ncols = (int64_t)NPROJ * p.N;
+  const int64_t per_row = p.N / 8;
+  const int64_t total = p.A * per_row;
+  for (int64_t v = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; v < total; v += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t r = v / per_row, n0 = (v % per_row) * 8;
+    float a[NPROJ][8];
+#pragma unroll
+    for (int j = 0; j < NPROJ; ++j)
+#pragma unroll
+      for (int i = 0; i < 8; ++i) a[j][i] = 0.f;
+    for (int kq = 0; kq < p.kq; ++kq) {
+      const float *src = p.partials + ((int64_t)kq * p.A + r) * ncols + n0;
+#pragma unroll
+      for (int j = 0; j < NPROJ; ++j) {
+        const float4 x0 = __ldcg(reinterpret_cast<const float4 *>(src + j * p.N));
+        const float4 x1 = __ldcg(reinterpret_cast<const float4 *>(src + j * p.N + 4));
+        a[j][0] += x0.x; a[j][1] += x0.y; a[j][2] += x0.z; a[j][3] += x0.w;
+        a[j][4] += x1.x; a[j][5] += x1.y; a[j][6] += x1.z; a[j][7] += x1.w;
+      }
+    }
+    // expert of row r: largest e with offsets[e] <= r (non-empty range)
+    int lo = 0, hi = p.E - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (p.offsets[mid] <= r) lo = mid;
+      else hi = mid - 1;
+    }
+    finish8<NPROJ>(p, lo, r, n0, a[0], a[NPROJ - 1]);
+  }
+}
+
+// ------------------------------------------------------------------ launch
+
+static size_t stream_smem(int nt, int64_t Kq, int64_t E) {
+  using namespace stream;
+  return 1024 /* alignment slack */ + kBarBytes + (size_t)kStages * kStageBytes + 2 * (size_t)8 * nt * Kq * 2 +
+         (size_t)8 * nt * (Kq * 2 + 16) + (size_t)8 * nt * kF * 4 + (size_t)(2 * E + 1 + 32) * 4;
+}
+
+// K splits: keep each unit at >= 384 input rows when K allows, whole
+// stages, and the split-K partials (KQ * A * columns FP32) bounded.
+StreamPlan stream_plan(int64_t A, int64_t K, int64_t N, int64_t E, int64_t group, int nproj, int nt) {
+  StreamPlan pl{};
+  pl.fits = false;
+  // TMA needs 16-byte word-row pitches; a stage of 32 rows lies in one group
+  if (N % 32 != 0 || K % stream::kRows != 0 || group % stream::kRows != 0) return pl;
+  int kq = 1;
+  for (int d = 8; d >= 2; d >>= 1)
+    if ((K / stream::kRows) % d == 0 && K / d >= 384) {
+      kq = d;
+      break;
+    }
+  while (kq > 1 && (size_t)kq * A * nproj * N * 4 > ((size_t)256 << 20)) kq >>= 1;
+  if (stream_smem(nt, K / kq, E) > 200 * 1024) return pl;
+  pl.fits = true;
+  pl.kq = kq;
+  if (kq > 1) {
+    pl.partial_off = 0;
+    pl.bytes = (size_t)kq * A * nproj * N * 4;
+    pl.counter_off = pl.bytes;
+  }
+  return pl;
+}
+
+template <typename MT, int NPROJ, int NT>
+static moe_status launch_stream_t(const ProjParams &p, cudaStream_t st) {
+  using namespace stream;
+  CUtensorMap m0, m1;
+  const uint64_t NW = p.N / 8, rows = (uint64_t)p.E * p.K;
+  if (!make_map_2d(&m0, p.qw[0], CU_TENSOR_MAP_DATA_TYPE_INT32, 4, NW, rows, kBoxW, kRows,
+                   CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map_2d(&m1, p.qw[NPROJ - 1], CU_TENSOR_MAP_DATA_TYPE_INT32, 4, NW, rows, kBoxW, kRows,
+                   CU_TENSOR_MAP_SWIZZLE_128B))
+    return set_error(MOE_ERR_CUDA, "tensor map encoding failed for the packed words");
+  const size_t smem = stream_smem(NT, p.K / p.kq, p.E);
+  auto kern = awq_fwd_stream_kernel<MT, NPROJ, NT>;
+  cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  const int per_sm = smem <= 110 * 1024 ? 2 : 1;
+  kern<<<num_sms() * per_sm, kThreads, smem, st>>>(m0, m1, p);
+  moe_status s = check_launch("awq_fwd_stream_kernel");
+  if (s != MOE_OK || p.kq == 1) return s;
+  const int64_t work = p.A * (p.N / 8);
+  int64_t blocks = (work + 255) / 256;
+  const int64_t cap = (int64_t)num_sms() * 8;
+  if (blocks > cap) blocks = cap;
+  awq_stream_reduce_kernel<NPROJ><<<(unsigned)blocks, 256, 0, st>>>(p);
+  return check_launch("awq_stream_reduce_kernel");
+}
+
+moe_status launch_fwd_stream(ProjParams p, int nproj, bool bf16_mma, int nt, void *ws, size_t ws_bytes,
+                             cudaStream_t st) {
+  const StreamPlan pl = stream_plan(p.A, p.K, p.N, p.E, p.group, nproj, nt);
+  p.kq = pl.kq;
+  p.partials = nullptr;
+  p.counters = nullptr;
+  if (pl.kq > 1) {
+    if (!ws || ws_bytes < pl.bytes || !aligned16(ws))
+      return set_error(MOE_ERR_WORKSPACE, "projection workspace of %zu bytes, need %zu (16-byte aligned)", ws_bytes,
+                       pl.bytes);
+    p.partials = reinterpret_cast<float *>(static_cast<char *>(ws) + pl.partial_off);
+  }
+  if (bf16_mma) {
+    if (nproj == 2) return nt == 2 ? launch_stream_t<__nv_bfloat16, 2, 2>(p, st) : launch_stream_t<__nv_bfloat16, 2, 1>(p, st);
+    return nt == 2 ? launch_stream_t<__nv_bfloat16, 1, 2>(p, st) : launch_stream_t<__nv_bfloat16, 1, 1>(p, st);
+  }
+  if (nproj == 2) return nt == 2 ? launch_stream_t<__half, 2, 2>(p, st) : launch_stream_t<__half, 2, 1>(p, st);
+  return nt == 2 ? launch_stream_t<__half, 1, 2>(p, st) : launch_stream_t<__half, 1, 1>(p, st);
+}
+
+}  // namespace moe

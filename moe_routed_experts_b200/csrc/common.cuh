@@ -124,14 +124,12 @@ __device__ __forceinline__ uint32_t act_pair_to_mt(uint32_t v, int act_dt) {
 template <typename MT>
 __device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
   if constexpr (std::is_same<MT, __half>::value) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
         "{%0,%1,%2,%3};"
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
   } else {
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
         "{%0,%1,%2,%3};"
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
@@ -142,6 +140,44 @@ __device__ __forceinline__ uint32_t ldg_nc_u32(const int32_t *p) {
   uint32_t v;
   asm volatile("ld.global.nc.L1::no_allocate.b32 %0, [%1];" : "=r"(v) : "l"(p));
   return v;
+}
+
+// Block-wide exclusive scan of cnt[0..n) (in shared memory) into out[0..n],
+// out[n] = total.  All threads of the block must call it.
+__device__ __forceinline__ void block_exclusive_scan(const int32_t *cnt, int n, int32_t *out, int32_t *tmp) {
+  const int tid = threadIdx.x, nt = blockDim.x;
+  const int per = (n + nt - 1) / nt;
+  const int b = tid * per, e = min(n, b + per);
+  int32_t local = 0;
+  for (int i = b; i < e; ++i) local += cnt[i];
+  // warp inclusive scan
+  const int lane = tid & 31, warp = tid >> 5;
+  int32_t v = local;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    int32_t u = __shfl_up_sync(0xffffffffu, v, o);
+    if (lane >= o) v += u;
+  }
+  if (lane == 31) tmp[warp] = v;
+  __syncthreads();
+  if (warp == 0) {
+    int nw = nt >> 5;
+    int32_t w = lane < nw ? tmp[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      int32_t u = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += u;
+    }
+    if (lane < nw) tmp[lane] = w;
+  }
+  __syncthreads();
+  int32_t run = v - local + (warp > 0 ? tmp[warp - 1] : 0);
+  for (int i = b; i < e; ++i) {
+    out[i] = run;
+    run += cnt[i];
+  }
+  if (tid == nt - 1) out[n] = run;  // the last thread's range ends at n (or is empty)
+  __syncthreads();
 }
 
 // Offsets check shared by the projection kernels: returns the row range of

@@ -64,44 +64,6 @@ __device__ __forceinline__ uint32_t score_key(const float *l, const float *bias,
   return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
 }
 
-// Block-wide exclusive scan of cnt[0..n) (in shared memory) into out[0..n],
-// out[n] = total.  All threads of the block must call it.
-__device__ void block_exclusive_scan(const int32_t *cnt, int n, int32_t *out, int32_t *tmp) {
-  const int tid = threadIdx.x, nt = blockDim.x;
-  const int per = (n + nt - 1) / nt;
-  const int b = tid * per, e = min(n, b + per);
-  int32_t local = 0;
-  for (int i = b; i < e; ++i) local += cnt[i];
-  // warp inclusive scan
-  const int lane = tid & 31, warp = tid >> 5;
-  int32_t v = local;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    int32_t u = __shfl_up_sync(0xffffffffu, v, o);
-    if (lane >= o) v += u;
-  }
-  if (lane == 31) tmp[warp] = v;
-  __syncthreads();
-  if (warp == 0) {
-    int nw = nt >> 5;
-    int32_t w = lane < nw ? tmp[lane] : 0;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      int32_t u = __shfl_up_sync(0xffffffffu, w, o);
-      if (lane >= o) w += u;
-    }
-    if (lane < nw) tmp[lane] = w;
-  }
-  __syncthreads();
-  int32_t run = v - local + (warp > 0 ? tmp[warp - 1] : 0);
-  for (int i = b; i < e; ++i) {
-    out[i] = run;
-    run += cnt[i];
-  }
-  if (tid == nt - 1) out[n] = run;  // the last thread's range ends at n (or is empty)
-  __syncthreads();
-}
-
 struct RouteParams {
   const float *logits;
   const float *sel_bias;

@@ -21,6 +21,10 @@ struct ProjParams {
   uint16_t *gout;  // G (two projections), or NULL
   uint16_t *uout;  // U (two projections), or NULL
   int32_t *status;
+  // split-K scratch of the streaming tile (workspace)
+  float *partials;
+  int32_t *counters;
+  int kq;  // K splits
 };
 
 struct BwdParams {
@@ -41,6 +45,15 @@ void launch_fwd_mma(const ProjParams &p, int nproj, bool bf16_mma, int nt, cudaS
 void launch_bwd_mma(const BwdParams &p, int nproj, bool bf16_mma, int nt, cudaStream_t st);
 void launch_dump(const int32_t *qw, const int32_t *qz, const uint16_t *sc, int64_t K, int64_t N, int group,
                  uint16_t *out, int mode, bool bf16_mma, cudaStream_t st);
+struct StreamPlan {
+  bool fits;      // the streaming tile can run this shape
+  int kq;         // K splits across CTAs
+  size_t bytes;   // workspace bytes (partials + counters)
+  size_t partial_off, counter_off;
+};
+StreamPlan stream_plan(int64_t A, int64_t K, int64_t N, int64_t E, int64_t group, int nproj, int nt);
+moe_status launch_fwd_stream(ProjParams p, int nproj, bool bf16_mma, int nt, void *ws, size_t ws_bytes,
+                             cudaStream_t st);
 bool tc_available();
 moe_status launch_fwd_tc(const ProjParams &p, int nproj, bool bf16_mma, cudaStream_t st);
 moe_status launch_bwd_tc(const BwdParams &p, int nproj, bool bf16_mma, cudaStream_t st);

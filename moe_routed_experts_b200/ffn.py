@@ -56,6 +56,7 @@ class Buffers:
     y: torch.Tensor
     out: torch.Tensor
     status: torch.Tensor
+    proj_ws: Optional[torch.Tensor] = None
 
 
 def alloc(w, device="cuda", keep_gu: bool = False) -> Buffers:
@@ -76,7 +77,9 @@ def alloc(w, device="cuda", keep_gu: bool = False) -> Buffers:
     U = torch.empty_like(h) if keep_gu else None
     y = torch.empty((A, H), dtype=torch.bfloat16, device=device)
     out = torch.empty((T, H), dtype=torch.bfloat16, device=device)
-    return Buffers(route, ws, h, G, U, y, out, torch.zeros(1, dtype=torch.int32, device=device))
+    pws = max(B.projection_workspace_size(A, H, I, E, w.group, 2), B.projection_workspace_size(A, I, H, E, w.group, 1))
+    proj_ws = torch.empty(pws, dtype=torch.uint8, device=device) if pws else None
+    return Buffers(route, ws, h, G, U, y, out, torch.zeros(1, dtype=torch.int32, device=device), proj_ws)
 
 
 def forward(dev: dict, buf: Buffers) -> torch.Tensor:
@@ -93,12 +96,13 @@ def forward(dev: dict, buf: Buffers) -> torch.Tensor:
         B._ptr(gate["qweight"]), B._ptr(gate["qzeros"]), B._ptr(gate["scales"]), B._ptr(gate["bias"]),
         B._ptr(up["qweight"]), B._ptr(up["qzeros"]), B._ptr(up["scales"]), B._ptr(up["bias"]),
         B._dt(gate["scales"].dtype), B.MOE_F32, w.group, B._ptr(buf.h), B._ptr(buf.G), B._ptr(buf.U),
-        B._ptr(buf.status), st)
+        B._ptr(buf.proj_ws), 0 if buf.proj_ws is None else buf.proj_ws.numel(), B._ptr(buf.status), st)
     B._check("awq_grouped_gate_up_swiglu", s)
     s = lib.awq_grouped_down(
         B._ptr(buf.h), B.MOE_BF16, A, w.I, w.H, B._ptr(r["offsets"]), w.E, B._ptr(down["qweight"]),
         B._ptr(down["qzeros"]), B._ptr(down["scales"]), B._ptr(down["bias"]), B._dt(down["scales"].dtype),
-        B.MOE_F32, w.group, B._ptr(buf.y), B._ptr(buf.status), st)
+        B.MOE_F32, w.group, B._ptr(buf.y), B._ptr(buf.proj_ws), 0 if buf.proj_ws is None else buf.proj_ws.numel(),
+        B._ptr(buf.status), st)
     B._check("awq_grouped_down", s)
     s = lib.moe_combine(B._ptr(buf.y), B.MOE_BF16, A, B._ptr(r["weights"]), B._ptr(r["selected_experts"]),
                         B._ptr(r["row_of"]), w.T, w.H, w.top_k, B._ptr(buf.out), B._ptr(buf.status), st)

@@ -51,7 +51,7 @@ def ulp(v: np.ndarray, dt: str) -> np.ndarray:
     return np.ldexp(1.0, (e - mant).astype(np.int64))
 
 
-def check_close(got, want, name, dt="bf16", tol=TOL, max_widened=2e-3):
+def check_close(got, want, name, dt="bf16", tol=TOL, max_widened=2e-3, ulps=1):
     g, w = as_f64(got, dt), as_f64(want, dt)
     assert g.shape == w.shape, (name, g.shape, w.shape)
     assert np.all(np.isfinite(g)), name + ": non-finite values"
@@ -60,7 +60,7 @@ def check_close(got, want, name, dt="bf16", tol=TOL, max_widened=2e-3):
     rms = float(np.sqrt(np.mean(w * w)))
     err = np.abs(g - w)
     strict = tol * rms
-    bound = strict + ulp(w, dt)
+    bound = strict + ulps * ulp(w, dt)
     worst = int(np.argmax(err - bound))
     assert np.all(err <= bound), "%s: err %.4g at value %.4g > %.3g * rms %.4g + 1 ulp" % (
         name, err.reshape(-1)[worst], w.reshape(-1)[worst], tol, rms)
@@ -98,6 +98,31 @@ def gpu_forward_numpy(inp):
            "values": bits(r["values"]), "G": bits(buf.G), "U": bits(buf.U), "h": bits(buf.h), "y": bits(buf.y),
            "out": bits(buf.out), "status": int(buf.status.item())}
     return res, dev, buf
+
+
+def check_forward_steps(inp, res, want, name, rows=None, tokens=None):
+    """Each forward step against the oracle on the device's inputs of that
+    step (one storage rounding apart), then the end-to-end output against the
+    oracle's own chain (two roundings may compound: two-ulp slack)."""
+    w = inp["workload"]
+    if rows is None:
+        rows = np.arange(w.A)
+    rexp = (res["row_experts"][rows].astype(np.int64) - w.expert_start).astype(np.int32)
+    G, U, h = res["G"][rows], res["U"][rows], res["h"][rows]
+    check_close(G, want["G"], name + "/G")
+    check_close(U, want["U"], name + "/U")
+    check_close(h, oracle.swiglu(G, U, "bf16"), name + "/h")
+    y = oracle.project(h, "bf16", rexp, inp["down"], w.scale_dtype, w.group)
+    check_close(res["y"][rows], y, name + "/y")
+    if tokens is None:
+        out = oracle.combine(res["y"], "bf16", res["weights"], res["selected"], res["row_of"])
+        check_close(res["out"], out, name + "/out")
+        check_close(res["out"], want["out"], name + "/out(end-to-end)", ulps=2)
+    else:
+        sel_t, w_t = res["selected"][tokens], res["weights"][tokens]
+        out = oracle.combine(res["y"], "bf16", w_t, sel_t, res["row_of"][tokens])
+        check_close(res["out"][tokens], out, name + "/out")
+        check_close(res["out"][tokens], want["out"], name + "/out(end-to-end)", ulps=2)
 
 
 def check_routing(res, want, name):

@@ -9,7 +9,7 @@ import pytest
 import torch
 
 import oracle
-from helpers import bits, check_close, check_routing, gpu_forward_numpy
+from helpers import bits, check_close, check_forward_steps, check_routing, gpu_forward_numpy
 from moe_routed_experts_b200 import binding as B
 from moe_routed_experts_b200 import ffn, inputs
 from moe_routed_experts_b200.configs import Workload
@@ -34,8 +34,7 @@ def _run(w, logits_fn=None):
     res, dev, buf = gpu_forward_numpy(inp)
     want = oracle.forward(inp)
     check_routing(res, want, w.name)
-    for key in ("G", "U", "h", "y", "out"):
-        check_close(res[key], want[key], "%s/%s" % (w.name, key))
+    check_forward_steps(inp, res, want, w.name)
     assert res["status"] == 0
     return res, want
 
@@ -108,7 +107,8 @@ def test_activation_and_scale_dtypes(act, sdt, path):
     oh = oracle.swiglu(oG, oU, act)
     check_close(bits(G), oG, "G", dt=act)
     check_close(bits(U), oU, "U", dt=act)
-    check_close(bits(h), oh, "h", dt=act)
+    check_close(bits(h), oracle.swiglu(bits(G), bits(U), act), "h", dt=act)
+    check_close(bits(h), oh, "h(end-to-end)", dt=act, ulps=2)
     down = ffn.projection_to_device(inp["down"], sdt)
     y = B.awq_grouped_down(h, offd, down, w.group)
     oy = oracle.project(bits(h), act, re, inp["down"], sdt, w.group)

@@ -7,8 +7,8 @@ import pytest
 import torch
 
 import oracle
-from helpers import (TOL, as_f64, bits, check_close, check_routing, generated, gpu_forward, gpu_forward_numpy,
-                     sample_rows, u32)
+from helpers import (TOL, as_f64, bits, check_close, check_forward_steps, check_routing, generated, gpu_forward,
+                     gpu_forward_numpy, sample_rows, u32)
 from moe_routed_experts_b200 import binding as B
 from moe_routed_experts_b200 import ffn, inputs
 from moe_routed_experts_b200.configs import WORKLOADS, Workload, scaled
@@ -142,8 +142,7 @@ def test_forward_every_row(name, path):
     want = _oracle_forward_all(inp)
     check_routing(res, want, name)
     assert np.array_equal(res["values"], want["values"])
-    for key in ("G", "U", "h", "y", "out"):
-        check_close(res[key], want[key], "%s/%s" % (name, key))
+    check_forward_steps(inp, res, want, name)
     assert res["status"] == 0
 
 
@@ -165,8 +164,5 @@ def test_forward_full_size_sampled(name, path):
     rows = sample_rows(res["offsets"], n_experts=4, rows_per=6)
     tokens = np.array([0, w.T // 3, w.T - 1], np.int64)
     want = oracle.forward(inp, rows=rows, tokens=tokens)
-    used = want["rows_used"]
-    for key in ("G", "U", "h", "y"):
-        check_close(res[key][used], want[key], "%s/%s" % (name, key))
-    check_close(res["out"][tokens], want["out"], name + "/out")
+    check_forward_steps(inp, res, want, name, rows=want["rows_used"], tokens=tokens)
     assert res["status"] == 0

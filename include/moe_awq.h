@@ -146,6 +146,36 @@ MOE_API moe_status moe_route_dispatch(const void *x, moe_dtype x_dtype, int64_t 
                               int32_t *device_status, void *stream);
 
 /* ------------------------------------------------------------------------
+ * moe_route_dispatch_noalloc -- moe_route_dispatch for callers that cannot
+ * allocate device memory for a workspace: serving loops that must not call
+ * cudaMalloc/cudaFree (those calls can synchronise the device and stall
+ * every stream), or host frameworks that own all device memory through their
+ * own pool and forbid allocations outside it.  The method's pages have no
+ * counterpart of this entry point; it is a property of this library.
+ *
+ * Same arguments, results and errors as moe_route_dispatch, minus the
+ * workspace: the scratch is a fixed 1 MiB array compiled into the library
+ * (every GPU that loads the library holds it until the process exits).
+ *  - Sizes whose scratch (moe_route_dispatch_workspace_size(T, E, top_k))
+ *    exceeds 1 MiB are rejected with MOE_ERR_WORKSPACE before any launch.
+ *  - The first call on a device looks the array's device address up
+ *    (cudaGetSymbolAddress) with the caller's current device, which must be
+ *    the device of `stream`; make that first call before any stream capture.
+ *  - Every call shares the one array, which keeps the last call's contents
+ *    (nothing in it needs to start at zero).  Calls whose kernels overlap on
+ *    the GPU (other streams, other host threads) race on it: serialise them.
+ *  - Nothing is allocated: no cudaMalloc, cudaFree or allocating library
+ *    routine is called.
+ * ---------------------------------------------------------------------- */
+MOE_API moe_status moe_route_dispatch_noalloc(const void *x, moe_dtype x_dtype, int64_t T, int64_t H,
+                                              const float *logits, const float *sel_bias, int64_t E,
+                                              int32_t expert_start, int32_t top_k,
+                                              int32_t renormalize, void *values, float *weights,
+                                              uint32_t *selected_experts, uint32_t *row_experts,
+                                              int32_t *offsets, int32_t *src_token, int32_t *row_of,
+                                              int32_t *device_status, void *stream);
+
+/* ------------------------------------------------------------------------
  * awq_grouped_gate_up_swiglu -- [PE] FrozenPackedExpertOps::packed_swiglu_forward
  * (gate and up projections of the selected experts and the storage-rounded
  * SwiGLU; "AD preserves required actual input caches": G and U are written

@@ -42,6 +42,8 @@ _SIGS = {
     "moe_version": (C.c_char_p, []),
     "moe_route_dispatch_workspace_size": (SZ, [I64, I64, I32]),
     "moe_route_dispatch": (C.c_int, [P, C.c_int, I64, I64, P, P, I64, I32, I32, I32, P, P, P, P, P, P, P, P, SZ, P, P]),
+    "moe_route_dispatch_noalloc": (C.c_int, [P, C.c_int, I64, I64, P, P, I64, I32, I32, I32, P, P, P, P, P, P, P, P,
+                                             P]),
     "awq_grouped_gate_up_swiglu": (C.c_int, [P, C.c_int, I64, I64, I64, P, I64, P, P, P, P, P, P, P, P, C.c_int,
                                              C.c_int, I64, P, P, P, P, SZ, P, P]),
     "awq_projection_workspace_size": (SZ, [I64, I64, I64, I64, I64, I32]),
@@ -144,6 +146,20 @@ def moe_route_dispatch(x, logits, top_k, E=None, sel_bias=None, expert_start=0, 
         _ptr(out["offsets"]), _ptr(out["src_token"]), _ptr(out["row_of"]), _ptr(workspace), workspace.numel(),
         _ptr(device_status), _stream())
     _check("moe_route_dispatch", st)
+    return out
+
+
+def moe_route_dispatch_noalloc(x, logits, top_k, out, E=None, sel_bias=None, expert_start=0, renormalize=1,
+                               device_status=None):
+    """moe_route_dispatch with the library's built-in scratch; `out` holds
+    preallocated outputs (same keys as moe_route_dispatch returns)."""
+    T, H = x.shape
+    E = E if E is not None else logits.shape[1]
+    st = lib().moe_route_dispatch_noalloc(
+        _ptr(x), _dt(x.dtype), T, H, _ptr(logits), _ptr(sel_bias), E, expert_start, top_k, renormalize,
+        _ptr(out["values"]), _ptr(out["weights"]), _ptr(out["selected_experts"]), _ptr(out["row_experts"]),
+        _ptr(out["offsets"]), _ptr(out["src_token"]), _ptr(out["row_of"]), _ptr(device_status), _stream())
+    _check("moe_route_dispatch_noalloc", st)
     return out
 
 

@@ -366,3 +366,66 @@ extern "C" moe_status moe_route_dispatch(const void *x, moe_dtype x_dtype, int64
   route_scatter_kernel<<<(unsigned)blocks, 256, 0, st>>>(sp);
   return check_launch("moe_route_dispatch: route_scatter_kernel");
 }
+
+// ------------------------------------------------------------------ allocation-free variant
+//
+// Some callers cannot allocate device memory for a workspace: a serving
+// loop that must not call cudaMalloc/cudaFree (they can synchronise the
+// device and stall every stream), or a host framework that owns all device
+// memory through its own pool and forbids allocations outside it.  For them
+// the routing scratch lives in a fixed array compiled into this library.
+
+#include <mutex>
+
+namespace moe {
+
+constexpr size_t kStaticRouteScratchBytes = size_t(1) << 20;  // 1 MiB per device
+static __device__ __align__(256) uint8_t g_route_scratch[kStaticRouteScratchBytes];
+
+constexpr int kMaxScratchDevices = 64;
+static std::mutex g_route_scratch_mu;
+static void *g_route_scratch_ptr[kMaxScratchDevices] = {};
+
+// Device address of g_route_scratch on the current device (looked up once per
+// device; the host-side name is only a stand-in for the symbol).
+static moe_status route_scratch_address(void **out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxScratchDevices)
+    return set_error(MOE_ERR_CUDA, "moe_route_dispatch_noalloc: no usable current device");
+  std::lock_guard<std::mutex> lock(g_route_scratch_mu);
+  if (!g_route_scratch_ptr[dev]) {
+    void *p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_route_scratch);
+    if (e != cudaSuccess || !p)
+      return set_error(MOE_ERR_CUDA, "moe_route_dispatch_noalloc: cudaGetSymbolAddress failed: %s",
+                       cudaGetErrorString(e));
+    g_route_scratch_ptr[dev] = p;
+  }
+  *out = g_route_scratch_ptr[dev];
+  return MOE_OK;
+}
+
+}  // namespace moe
+
+extern "C" moe_status moe_route_dispatch_noalloc(const void *x, moe_dtype x_dtype, int64_t T, int64_t H,
+                                                 const float *logits, const float *sel_bias, int64_t E,
+                                                 int32_t expert_start, int32_t top_k, int32_t renormalize,
+                                                 void *values, float *weights, uint32_t *selected_experts,
+                                                 uint32_t *row_experts, int32_t *offsets, int32_t *src_token,
+                                                 int32_t *row_of, int32_t *device_status, void *stream) {
+  if (T < 0 || E < 1 || top_k < 1)
+    return set_error(MOE_ERR_INVALID_ARGUMENT, "moe_route_dispatch_noalloc: bad sizes T=%lld E=%lld top_k=%d",
+                     (long long)T, (long long)E, top_k);
+  const size_t need = route_ws_layout(T, E, top_k).bytes;
+  if (need > kStaticRouteScratchBytes)
+    return set_error(MOE_ERR_WORKSPACE,
+                     "moe_route_dispatch_noalloc: T=%lld, E=%lld, top_k=%d need %zu bytes of scratch; the built-in "
+                     "scratch holds %zu (use moe_route_dispatch with a workspace)",
+                     (long long)T, (long long)E, top_k, need, kStaticRouteScratchBytes);
+  void *scratch = nullptr;
+  const moe_status s = route_scratch_address(&scratch);
+  if (s != MOE_OK) return s;
+  return moe_route_dispatch(x, x_dtype, T, H, logits, sel_bias, E, expert_start, top_k, renormalize, values,
+                            weights, selected_experts, row_experts, offsets, src_token, row_of, scratch,
+                            kStaticRouteScratchBytes, device_status, stream);
+}

@@ -39,7 +39,8 @@ int num_sms() {
 static std::atomic<int> g_path{0};
 
 // Both tile paths hold the same operation; the warp-level one is chosen when
-// the average batch per expert is too small to fill a 128-row tcgen05 tile.
+// the average batch per expert is too small to fill a 128-row tcgen05 tile,
+// or when the shape is one the tcgen05 tile does not take (see tc_fits).
 static int choose_path(int64_t A, int64_t E) {
   int forced = g_path.load();
   if (forced == 1 || forced == 2) return forced;
@@ -94,7 +95,13 @@ extern "C" int32_t moe_set_projection_path(int32_t path) {
 extern "C" size_t awq_projection_workspace_size(int64_t A, int64_t K, int64_t N, int64_t E, int64_t group_size,
                                                 int32_t nproj) {
   if (A <= 0 || E < 1 || K < 16 || N < 8 || group_size < 16 || (nproj != 1 && nproj != 2)) return 0;
-  if (choose_path(A, E) != 1) return 0;
+  ProjParams probe{};
+  probe.A = A;
+  probe.K = K;
+  probe.N = N;
+  probe.E = (int)E;
+  probe.group = (int)group_size;
+  if (choose_path(A, E) == 2 && tc_fits(probe)) return 0;
   const StreamPlan pl = stream_plan(A, K, N, E, group_size, nproj, small_tile_tokens(A, E));
   return pl.fits ? pl.bytes : 0;
 }
@@ -138,7 +145,7 @@ extern "C" moe_status awq_grouped_gate_up_swiglu(
   p.status = device_status;
   cudaStream_t st = as_stream(stream);
   const bool bf = scale_dtype == MOE_BF16;
-  if (choose_path(A, E) == 2) return launch_fwd_tc(p, 2, bf, st);
+  if (choose_path(A, E) == 2 && tc_fits(p)) return launch_fwd_tc(p, 2, bf, st);
   const int nt = small_tile_tokens(A, E);
   if (stream_plan(A, H, I, E, group_size, 2, nt).fits) return launch_fwd_stream(p, 2, bf, nt, workspace, workspace_bytes, st);
   launch_fwd_mma(p, 2, bf, nt, st);
@@ -176,7 +183,7 @@ extern "C" moe_status awq_grouped_down(const void *input, moe_dtype act_dtype, i
   p.status = device_status;
   cudaStream_t st = as_stream(stream);
   const bool bf = scale_dtype == MOE_BF16;
-  if (choose_path(A, E) == 2) return launch_fwd_tc(p, 1, bf, st);
+  if (choose_path(A, E) == 2 && tc_fits(p)) return launch_fwd_tc(p, 1, bf, st);
   const int nt = small_tile_tokens(A, E);
   if (stream_plan(A, K, N, E, group_size, 1, nt).fits) return launch_fwd_stream(p, 1, bf, nt, workspace, workspace_bytes, st);
   launch_fwd_mma(p, 1, bf, nt, st);
@@ -220,7 +227,7 @@ extern "C" moe_status awq_input_backward(const void *grad, moe_dtype grad_dtype,
   cudaStream_t st = as_stream(stream);
   const bool bf = scale_dtype == MOE_BF16;
   const int nproj = grad2 ? 2 : 1;
-  if (choose_path(A, E) == 2) return launch_bwd_tc(p, nproj, bf, st);
+  if (choose_path(A, E) == 2 && tc_bwd_fits(p)) return launch_bwd_tc(p, nproj, bf, st);
   launch_bwd_mma(p, nproj, bf, A >= 12 * E ? 2 : 1, st);
   return check_launch(fn);
 }

@@ -1,16 +1,396 @@
-// Grouped AWQ projections on tcgen05/TMEM tiles (large per-expert batches).
+// Grouped AWQ projections on tcgen05 tensor cores with TMEM accumulators,
+// for per-expert batches large enough to fill 128-row tiles (prefill).
+//
+// ruda-tensor 0.21.34, src/packed_experts.rs -- packed_expert_forward /
+//   packed_swiglu_forward (gate/up/down of the selected experts, SwiGLU);
+// ruda-tensor 0.21.33, src/frozen_awq.rs -- AWQ nibble order and scale-dtype
+//   coefficient rounding; the tensor-core products run in the scale dtype.
+//
+// Tile: 128 expert rows x 256 output columns (for the gate/up pair: 128
+// features of each projection, so SwiGLU sees G and U of a feature in the
+// same thread), K in steps of 64.  Persistent CTAs walk the tile list
+// (expert-major, row tile, column tile) round-robin.  Warp roles:
+//   warp 0  producer: TMA of the activation tile (128 x 64, 128-byte
+//           swizzle, K-major) and of the packed words of the step
+//           (64 rows x 32 words) into a 3-stage ring;
+//   warp 1  allocates 256 TMEM columns; lane 0 issues tcgen05.mma
+//           (M=128, N=256, K=16, FP32 accumulate in TMEM) and commits each
+//           stage back to the producer and the finished tile to the epilogue;
+//   warps 2-9 dequantize: each thread forms the coefficients of 8 packed
+//           words (8 features at one input row each, in logical order) and
+//           stores them as 16-byte chunks of the B operand, laid out MN-major
+//           with 128-byte swizzle (8-row x 64-column atoms); when the
+//           activations are not in the scale dtype they also convert the
+//           activation tile in place.  After a tile's last step they read the
+//           accumulator from TMEM (tcgen05.ld 32x32b), add the bias, round,
+//           apply SwiGLU and store.
+// Coefficients are exact per the operation: RNE_scale((q - z) s) formed with
+// the magic-number conversion (see common.cuh), never written to HBM.
+#include <cudaTypedefs.h>
+
+#include "dequant.cuh"
 #include "proj.cuh"
+#include "tma.cuh"
 
 namespace moe {
 
-bool tc_available() { return false; }
+namespace tc {
+constexpr int kBM = 128, kBN = 256, kBK = 64;
+constexpr int kStages = 3;
+constexpr int kDqWarps = 8;
+constexpr int kThreads = (2 + kDqWarps) * 32;  // 320
+constexpr int kABytes = kBM * kBK * 2;          // 16 KB activation tile
+constexpr int kBBytes = kBN * kBK * 2;          // 32 KB coefficient tile
+constexpr int kPBytes = kBK * (kBN / 8) * 4;    // 8 KB packed words
+constexpr int kStageBytes = kABytes + kBBytes + kPBytes;
+constexpr int kTmemCols = 256;
+}  // namespace tc
 
-moe_status launch_fwd_tc(const ProjParams &, int, bool, cudaStream_t) {
-  return set_error(MOE_ERR_UNSUPPORTED_DTYPE, "tcgen05 projection tiles are not built");
+// ------------------------------------------------------------------ tcgen05 wrappers
+
+__device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+  // start >> 4 | LBO >> 4 << 16 | SBO >> 4 << 32 | version 1 << 46 | 128-byte swizzle (2) << 61
+  return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+         ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
 }
 
+__device__ __forceinline__ void umma_f16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                         uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}" ::"r"(tmem_d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void umma_commit(uint64_t *bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// 32 consecutive FP32 accumulator columns of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,"
+      "%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+        "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]),
+        "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// Bounded wait that gives up at once after any timeout in the CTA (abort).
+__device__ __forceinline__ bool tc_wait(uint64_t *bar, uint32_t parity, int32_t *status, volatile int32_t *abort) {
+  if (*abort) return false;
+  if (mbar_wait(bar, parity, status)) return true;
+  *abort = 1;
+  return false;
+}
+
+// ------------------------------------------------------------------ kernel
+
+struct TileInfo {
+  int e, mt, nt;
+  int64_t r0;  // first row of the expert
+  int m;       // rows of the expert
+};
+
+template <typename MT, int NPROJ>
+__global__ void __launch_bounds__(tc::kThreads, 1)
+    awq_fwd_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_w0,
+                      const __grid_constant__ CUtensorMap map_w1, ProjParams p) {
+  using namespace tc;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t *smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
+  uint8_t *stages = smem;  // kStages x [A | B | packed]
+  uint64_t *full = reinterpret_cast<uint64_t *>(stages + kStages * kStageBytes);
+  uint64_t *bready = full + kStages;
+  uint64_t *empty = bready + kStages;
+  uint64_t *accfull = empty + kStages;
+  uint64_t *accempty = accfull + 1;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(accempty + 1);
+  volatile int32_t *abort = reinterpret_cast<volatile int32_t *>(tmem_slot + 1);
+  int32_t *pre = reinterpret_cast<int32_t *>(tmem_slot + 4);  // [E + 1]
+  int32_t *cnt = pre + (p.E + 1);                             // [E]
+  int32_t *tmp = cnt + p.E;                                   // [32]
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int E = p.E;
+  const int64_t K = p.K, NW = p.N / 8;
+  const int feat_tile = NPROJ == 2 ? kBN / 2 : kBN;          // output features per tile
+  const int NT = (int)((p.N + feat_tile - 1) / feat_tile);  // column tiles per row tile
+  const int nk = (int)(K / kBK);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&bready[s], kDqWarps);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(accfull, 1);
+    mbar_init(accempty, kDqWarps);
+    *abort = 0;
+    fence_mbar_init();
+  }
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    const int32_t a = p.offsets[e], b = p.offsets[e + 1];
+    const bool bad = a < 0 || b < a || (int64_t)b > p.A || (e == 0 && a != 0) || (e == E - 1 && (int64_t)b != p.A);
+    if (bad && blockIdx.x == 0) report(p.status, MOE_DEVICE_ERR_OFFSETS);
+    cnt[e] = bad ? 0 : NT * ((b - a + kBM - 1) / kBM);
+  }
+  __syncthreads();
+  block_exclusive_scan(cnt, E, pre, tmp);
+  const int64_t total = pre[E];
+  if ((int64_t)blockIdx.x >= total) return;  // no tile for this CTA (uniform)
+
+  auto tile_info = [&](int64_t tile) {
+    TileInfo ti;
+    int lo = 0, hi = E - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (pre[mid] <= tile) lo = mid;
+      else hi = mid - 1;
+    }
+    ti.e = lo;
+    const int64_t local = tile - pre[lo];
+    ti.mt = (int)(local / NT);
+    ti.nt = (int)(local % NT);
+    ti.r0 = p.offsets[lo];
+    ti.m = p.offsets[lo + 1] - (int32_t)ti.r0;
+    return ti;
+  };
+
+  if (warp == 1) {  // TMEM allocation (whole warp)
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                 "r"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ---------------- producer
+    if (lane == 0) {
+      uint32_t it = 0;
+      for (int64_t tile = blockIdx.x; tile < total; tile += gridDim.x) {
+        const TileInfo ti = tile_info(tile);
+        const int32_t row0 = (int32_t)(ti.r0 + (int64_t)ti.mt * kBM);
+        for (int kb = 0; kb < nk; ++kb, ++it) {
+          const uint32_t s = it % kStages, use = it / kStages;
+          if (use > 0) tc_wait(&empty[s], (use - 1) & 1, p.status, abort);
+          uint8_t *st = stages + s * kStageBytes;
+          mbar_arrive_expect_tx(&full[s], kABytes + kPBytes);
+          tma_load_2d(st, &map_x, &full[s], kb * kBK, row0);
+          const int32_t wrow = (int32_t)(ti.e * K + (int64_t)kb * kBK);
+          if (NPROJ == 2) {
+            tma_load_2d(st + kABytes + kBBytes, &map_w0, &full[s], ti.nt * 16, wrow);
+            tma_load_2d(st + kABytes + kBBytes + kPBytes / 2, &map_w1, &full[s], ti.nt * 16, wrow);
+          } else {
+            tma_load_2d(st + kABytes + kBBytes, &map_w0, &full[s], ti.nt * 32, wrow);
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t fmt = std::is_same<MT, __half>::value ? 0u : 1u;
+      // D F32, A/B in the scale dtype, A K-major, B MN-major, N = 256, M = 128
+      const uint32_t idesc = (1u << 4) | (fmt << 7) | (fmt << 10) | (1u << 16) | ((uint32_t)(kBN >> 3) << 17) |
+                             ((uint32_t)(kBM >> 4) << 24);
+      uint32_t it = 0, tcount = 0;
+      for (int64_t tile = blockIdx.x; tile < total; tile += gridDim.x, ++tcount) {
+        if (tcount > 0) tc_wait(accempty, (tcount - 1) & 1, p.status, abort);
+        tc_fence_after();
+        for (int kb = 0; kb < nk; ++kb, ++it) {
+          const uint32_t s = it % kStages, ph = (it / kStages) & 1;
+          tc_wait(&full[s], ph, p.status, abort);
+          tc_wait(&bready[s], ph, p.status, abort);
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(stages + s * kStageBytes);
+          const uint32_t b_addr = a_addr + kABytes;
+          const uint64_t adesc = smem_desc(a_addr, 16, 1024);     // K-major, 8-row groups 1 KB apart
+          const uint64_t bdesc = smem_desc(b_addr, 8192, 1024);   // MN-major: 64-col groups 8 KB, 8-row groups 1 KB
+#pragma unroll
+          for (int j = 0; j < kBK / 16; ++j)
+            umma_f16(tmem, adesc + (uint64_t)(2 * j), bdesc + (uint64_t)(128 * j), idesc, (kb | j) != 0);
+          umma_commit(&empty[s]);
+        }
+        umma_commit(accfull);
+      }
+    }
+  } else {
+    // ---------------- dequant + epilogue warps
+    const int td = threadIdx.x - 64;  // 0..255
+    const int col = td & 31;          // word column of the tile (gate 0..15 | up 16..31, or 0..31)
+    const int rg = td >> 5;           // rows rg, rg + 8, ..., of each 64-row step
+    constexpr uint32_t M = Dq<MT>::kMagic2;
+    const int jw = NPROJ == 2 ? (col >> 4) : 0;
+    const int64_t ngroups = K / p.group;
+    const int32_t *qz = p.qz[jw];
+    const uint16_t *sc = p.sc[jw];
+    uint32_t it = 0, tcount = 0;
+    for (int64_t tile = blockIdx.x; tile < total; tile += gridDim.x, ++tcount) {
+      const TileInfo ti = tile_info(tile);
+      const int64_t wc = NPROJ == 2 ? (int64_t)ti.nt * 16 + (col & 15) : (int64_t)ti.nt * 32 + col;
+      const bool wc_ok = wc < NW;
+      const int64_t wcs = wc_ok ? wc : 0;
+      const int32_t *qzp = qz + (int64_t)ti.e * ngroups * NW + wcs;
+      const uint16_t *scp = sc + (int64_t)ti.e * ngroups * p.N + 8 * wcs;
+      // B: features col*8 .. col*8+7 -> 64-column block col/8, 16-byte chunk col%8
+      const int nblk = (col >> 3) * 8192, chunk = col & 7;
+      int64_t cur_grp = -1;
+      uint32_t zp[4] = {0, 0, 0, 0}, sp[4] = {0, 0, 0, 0};
+      for (int kb = 0; kb < nk; ++kb, ++it) {
+        const uint32_t s = it % kStages, ph = (it / kStages) & 1;
+        const int64_t grp = (int64_t)kb * kBK / p.group;  // whole steps lie in one group (group % 64 == 0)
+        if (grp != cur_grp) {
+          cur_grp = grp;
+          const uint32_t zw = wc_ok ? (uint32_t)__ldg(qzp + grp * NW) : 0u;
+          const uint4 sv = wc_ok ? __ldg(reinterpret_cast<const uint4 *>(scp + grp * p.N)) : make_uint4(0, 0, 0, 0);
+          const uint32_t s4[4] = {sv.x, sv.y, sv.z, sv.w};
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            zp[q] = nib_pair<M>(zw >> (4 * q));
+            sp[q] = s4[q];
+          }
+        }
+        tc_wait(&full[s], ph, p.status, abort);
+        uint8_t *st = stages + s * kStageBytes;
+        if (p.act_dt != (std::is_same<MT, __half>::value ? MOE_F16 : MOE_BF16)) {
+          // activation tile to the scale dtype, in place (layout-agnostic)
+          uint4 *a4 = reinterpret_cast<uint4 *>(st);
+#pragma unroll
+          for (int i = 0; i < kABytes / 16 / 256; ++i) {
+            uint4 v = a4[td + 256 * i];
+            v.x = act_pair_to_mt<MT>(v.x, p.act_dt);
+            v.y = act_pair_to_mt<MT>(v.y, p.act_dt);
+            v.z = act_pair_to_mt<MT>(v.z, p.act_dt);
+            v.w = act_pair_to_mt<MT>(v.w, p.act_dt);
+            a4[td + 256 * i] = v;
+          }
+        }
+        const uint32_t *pk = reinterpret_cast<const uint32_t *>(st + kABytes + kBBytes);
+        uint8_t *bt = st + kABytes;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int r = rg + 8 * i;  // row of the step
+          const uint32_t w =
+              NPROJ == 2 ? pk[(col >> 4) * (kBK * 16) + r * 16 + (col & 15)] : pk[r * 32 + col];
+          uint4 c;
+          c.x = Dq<MT>::coef(nib_pair<M>(w), zp[0], sp[0]);        // columns 0, 1
+          c.y = Dq<MT>::coef(nib_pair<M>(w >> 4), zp[1], sp[1]);   // columns 2, 3
+          c.z = Dq<MT>::coef(nib_pair<M>(w >> 8), zp[2], sp[2]);   // columns 4, 5
+          c.w = Dq<MT>::coef(nib_pair<M>(w >> 12), zp[3], sp[3]);  // columns 6, 7
+          // (row r, 8 features) -> 8-row atom r/8, row r%8 of it, chunk XOR (r%8)
+          *reinterpret_cast<uint4 *>(bt + nblk + (r >> 3) * 1024 + (r & 7) * 128 + ((chunk ^ (r & 7)) << 4)) = c;
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bready[s]);
+      }
+
+      // ---- epilogue: TMEM -> registers -> bias, rounding, SwiGLU -> HBM
+      tc_wait(accfull, tcount & 1, p.status, abort);
+      tc_fence_after();
+      const int q = warp & 3;         // TMEM lane quarter of this warp
+      const int hf = (warp - 2) >> 2;  // column half
+      const int trow = ti.mt * kBM + 32 * q + lane;  // row within the expert
+      const bool row_ok = trow < ti.m && !*abort;
+      const int64_t row = ti.r0 + trow;
+      const uint32_t tbase = tmem + ((uint32_t)(32 * q) << 16);
+      if (NPROJ == 2) {
+#pragma unroll 1
+        for (int c2 = 0; c2 < 2; ++c2) {
+          const int f0 = hf * 64 + c2 * 32;  // feature within the tile
+          float gv[32], uv[32];
+          tmem_ld32(tbase + f0, gv);
+          tmem_ld32(tbase + 128 + f0, uv);
+          const int64_t n0 = (int64_t)ti.nt * 128 + f0;
+          if (row_ok && n0 < p.N) {
+#pragma unroll
+            for (int v8 = 0; v8 < 4; ++v8) finish8<2>(p, ti.e, row, n0 + 8 * v8, gv + 8 * v8, uv + 8 * v8);
+          }
+        }
+      } else {
+#pragma unroll 1
+        for (int c4 = 0; c4 < 4; ++c4) {
+          const int f0 = hf * 128 + c4 * 32;
+          float yv[32];
+          tmem_ld32(tbase + f0, yv);
+          const int64_t n0 = (int64_t)ti.nt * 256 + f0;
+          if (row_ok && n0 < p.N) {
+#pragma unroll
+            for (int v8 = 0; v8 < 4; ++v8) finish8<1>(p, ti.e, row, n0 + 8 * v8, yv + 8 * v8, yv + 8 * v8);
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(accempty);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
+  }
+}
+
+// ------------------------------------------------------------------ launch
+
+static size_t tc_smem(int64_t E) {
+  return 1024 + (size_t)tc::kStages * tc::kStageBytes + 256 + (size_t)(2 * E + 1 + 32) * 4;
+}
+
+// The tile needs whole 64-row steps inside one group, 16-byte word-row
+// pitches for TMA, and a 16-bit activation tile.
+bool tc_fits(const ProjParams &p) {
+  return p.K % tc::kBK == 0 && p.group % tc::kBK == 0 && p.N % 32 == 0 && tc_smem(p.E) <= 227 * 1024;
+}
+
+bool tc_available() { return true; }
+
+template <typename MT, int NPROJ>
+static moe_status launch_tc_t(const ProjParams &p, cudaStream_t st) {
+  using namespace tc;
+  CUtensorMap mx, m0, m1;
+  const uint64_t NW = p.N / 8, rows = (uint64_t)p.E * p.K;
+  const uint32_t box_w = NPROJ == 2 ? 16 : 32;
+  if (!make_map_2d(&mx, p.x, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, p.K, p.A, kBK, kBM, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map_2d(&m0, p.qw[0], CU_TENSOR_MAP_DATA_TYPE_INT32, 4, NW, rows, box_w, kBK, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !make_map_2d(&m1, p.qw[NPROJ - 1], CU_TENSOR_MAP_DATA_TYPE_INT32, 4, NW, rows, box_w, kBK,
+                   CU_TENSOR_MAP_SWIZZLE_NONE))
+    return set_error(MOE_ERR_CUDA, "tensor map encoding failed (tcgen05 projection)");
+  const size_t smem = tc_smem(p.E);
+  auto kern = awq_fwd_tc_kernel<MT, NPROJ>;
+  cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  kern<<<num_sms(), kThreads, smem, st>>>(mx, m0, m1, p);
+  return check_launch("awq_fwd_tc_kernel");
+}
+
+moe_status launch_fwd_tc(const ProjParams &p, int nproj, bool bf16_mma, cudaStream_t st) {
+  if (bf16_mma) return nproj == 2 ? launch_tc_t<__nv_bfloat16, 2>(p, st) : launch_tc_t<__nv_bfloat16, 1>(p, st);
+  return nproj == 2 ? launch_tc_t<__half, 2>(p, st) : launch_tc_t<__half, 1>(p, st);
+}
+
+bool tc_bwd_fits(const BwdParams &) { return false; }
+
 moe_status launch_bwd_tc(const BwdParams &, int, bool, cudaStream_t) {
-  return set_error(MOE_ERR_UNSUPPORTED_DTYPE, "tcgen05 projection tiles are not built");
+  return set_error(MOE_ERR_UNSUPPORTED_DTYPE, "tcgen05 input-VJP tiles are not built");
 }
 
 }  // namespace moe

@@ -13,7 +13,7 @@
 //   warp 0  producer: TMA of the activation tile (128 x 64, 128-byte
 //           swizzle, K-major) and of the packed words of the step
 //           (64 rows x 32 words) into a 3-stage ring;
-//   warp 1  allocates 256 TMEM columns; lane 0 issues tcgen05.mma
+//   warp 1  allocates 512 TMEM columns (two accumulators); lane 0 issues tcgen05.mma
 //           (M=128, N=256, K=16, FP32 accumulate in TMEM) and commits each
 //           stage back to the producer and the finished tile to the epilogue;
 //   warps 2-9 dequantize: each thread forms the coefficients of 8 packed
@@ -21,9 +21,10 @@
 //           stores them as 16-byte chunks of the B operand, laid out MN-major
 //           with 128-byte swizzle (8-row x 64-column atoms); when the
 //           activations are not in the scale dtype they also convert the
-//           activation tile in place.  After a tile's last step they read the
-//           accumulator from TMEM (tcgen05.ld 32x32b), add the bias, round,
-//           apply SwiGLU and store.
+//           activation tile in place;
+//   warps 10-13 (one per TMEM lane quarter) read a finished accumulator
+//           (tcgen05.ld 32x32b), add the bias, round, apply SwiGLU and store,
+//           while the tensor core fills the other of the two TMEM buffers.
 // Coefficients are exact per the operation: RNE_scale((q - z) s) formed with
 // the magic-number conversion (see common.cuh), never written to HBM.
 #include <cudaTypedefs.h>
@@ -38,12 +39,13 @@ namespace tc {
 constexpr int kBM = 128, kBN = 256, kBK = 64;
 constexpr int kStages = 3;
 constexpr int kDqWarps = 8;
-constexpr int kThreads = (2 + kDqWarps) * 32;  // 320
+constexpr int kEpWarps = 4;                                // one per TMEM lane quarter
+constexpr int kThreads = (2 + kDqWarps + kEpWarps) * 32;  // 448
 constexpr int kABytes = kBM * kBK * 2;          // 16 KB activation tile
 constexpr int kBBytes = kBN * kBK * 2;          // 32 KB coefficient tile
 constexpr int kPBytes = kBK * (kBN / 8) * 4;    // 8 KB packed words
 constexpr int kStageBytes = kABytes + kBBytes + kPBytes;
-constexpr int kTmemCols = 256;
+constexpr int kTmemCols = 512;  // two 128 x 256 FP32 accumulators
 }  // namespace tc
 
 // ------------------------------------------------------------------ tcgen05 wrappers
@@ -114,9 +116,9 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
   uint64_t *full = reinterpret_cast<uint64_t *>(stages + kStages * kStageBytes);
   uint64_t *bready = full + kStages;
   uint64_t *empty = bready + kStages;
-  uint64_t *accfull = empty + kStages;
-  uint64_t *accempty = accfull + 1;
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(accempty + 1);
+  uint64_t *accfull = empty + kStages;  // [2]
+  uint64_t *accempty = accfull + 2;     // [2]
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(accempty + 2);
   volatile int32_t *abort = reinterpret_cast<volatile int32_t *>(tmem_slot + 1);
   int32_t *pre = reinterpret_cast<int32_t *>(tmem_slot + 4);  // [E + 1]
   int32_t *cnt = pre + (p.E + 1);                             // [E]
@@ -135,8 +137,10 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
       mbar_init(&bready[s], kDqWarps);
       mbar_init(&empty[s], 1);
     }
-    mbar_init(accfull, 1);
-    mbar_init(accempty, kDqWarps);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&accfull[b], 1);
+      mbar_init(&accempty[b], kEpWarps);
+    }
     *abort = 0;
     fence_mbar_init();
   }
@@ -203,7 +207,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
       }
     }
   } else if (warp == 1) {
-    // ---------------- MMA issuer
+    // ---------------- MMA issuer: tile t accumulates in TMEM buffer t & 1
     if (lane == 0) {
       constexpr uint32_t fmt = std::is_same<MT, __half>::value ? 0u : 1u;
       // D F32, A/B in the scale dtype, A K-major, B MN-major, N = 256, M = 128
@@ -211,8 +215,10 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
                              ((uint32_t)(kBM >> 4) << 24);
       uint32_t it = 0, tcount = 0;
       for (int64_t tile = blockIdx.x; tile < total; tile += gridDim.x, ++tcount) {
-        if (tcount > 0) tc_wait(accempty, (tcount - 1) & 1, p.status, abort);
+        const uint32_t buf = tcount & 1, use = tcount >> 1;
+        if (use > 0) tc_wait(&accempty[buf], (use - 1) & 1, p.status, abort);
         tc_fence_after();
+        const uint32_t dacc = tmem + buf * kBN;
         for (int kb = 0; kb < nk; ++kb, ++it) {
           const uint32_t s = it % kStages, ph = (it / kStages) & 1;
           tc_wait(&full[s], ph, p.status, abort);
@@ -220,55 +226,68 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
           tc_fence_after();
           const uint32_t a_addr = smem_u32(stages + s * kStageBytes);
           const uint32_t b_addr = a_addr + kABytes;
-          const uint64_t adesc = smem_desc(a_addr, 16, 1024);     // K-major, 8-row groups 1 KB apart
-          const uint64_t bdesc = smem_desc(b_addr, 8192, 1024);   // MN-major: 64-col groups 8 KB, 8-row groups 1 KB
+          const uint64_t adesc = smem_desc(a_addr, 16, 1024);    // K-major, 8-row groups 1 KB apart
+          const uint64_t bdesc = smem_desc(b_addr, 8192, 1024);  // MN-major: 64-col groups 8 KB, 8-row groups 1 KB
 #pragma unroll
           for (int j = 0; j < kBK / 16; ++j)
-            umma_f16(tmem, adesc + (uint64_t)(2 * j), bdesc + (uint64_t)(128 * j), idesc, (kb | j) != 0);
+            umma_f16(dacc, adesc + (uint64_t)(2 * j), bdesc + (uint64_t)(128 * j), idesc, (kb | j) != 0);
           umma_commit(&empty[s]);
         }
-        umma_commit(accfull);
+        umma_commit(&accfull[buf]);
       }
     }
-  } else {
-    // ---------------- dequant + epilogue warps
+  } else if (warp < 2 + kDqWarps) {
+    // ---------------- dequant warps
     const int td = threadIdx.x - 64;  // 0..255
     const int col = td & 31;          // word column of the tile (gate 0..15 | up 16..31, or 0..31)
-    const int rg = td >> 5;           // rows rg, rg + 8, ..., of each 64-row step
-    constexpr uint32_t M = Dq<MT>::kMagic2;
     const int jw = NPROJ == 2 ? (col >> 4) : 0;
+    // rows rg, rg + 8, ... of each 64-row step; the up lanes take the
+    // neighbouring row so gate and up words sit in different banks
+    const int rg = (td >> 5) ^ jw;
+    constexpr uint32_t M = Dq<MT>::kMagic2;
     const int64_t ngroups = K / p.group;
     const int32_t *qz = p.qz[jw];
     const uint16_t *sc = p.sc[jw];
-    uint32_t it = 0, tcount = 0;
-    for (int64_t tile = blockIdx.x; tile < total; tile += gridDim.x, ++tcount) {
+    const int pk0 = NPROJ == 2 ? jw * (kBK * 16) + rg * 16 + (col & 15) : rg * 32 + col;
+    constexpr int pk_step = NPROJ == 2 ? 8 * 16 : 8 * 32;  // words between rows r and r + 8
+    // B: features col*8 .. col*8+7 -> 64-column block col/8, 16-byte chunk col%8 XOR row%8
+    const int b0 = (col >> 3) * 8192 + rg * 128 + (((col & 7) ^ rg) << 4);  // + 1 KB per 8 rows
+    const int spg = p.group / kBK;  // steps per group
+    const bool convert = p.act_dt != (std::is_same<MT, __half>::value ? MOE_F16 : MOE_BF16);
+    uint32_t it = 0;
+    for (int64_t tile = blockIdx.x; tile < total; tile += gridDim.x) {
       const TileInfo ti = tile_info(tile);
       const int64_t wc = NPROJ == 2 ? (int64_t)ti.nt * 16 + (col & 15) : (int64_t)ti.nt * 32 + col;
       const bool wc_ok = wc < NW;
       const int64_t wcs = wc_ok ? wc : 0;
       const int32_t *qzp = qz + (int64_t)ti.e * ngroups * NW + wcs;
       const uint16_t *scp = sc + (int64_t)ti.e * ngroups * p.N + 8 * wcs;
-      // B: features col*8 .. col*8+7 -> 64-column block col/8, 16-byte chunk col%8
-      const int nblk = (col >> 3) * 8192, chunk = col & 7;
-      int64_t cur_grp = -1;
-      uint32_t zp[4] = {0, 0, 0, 0}, sp[4] = {0, 0, 0, 0};
+      uint32_t zp[4], sp[4];
+      uint32_t pf_zw = wc_ok ? (uint32_t)__ldg(qzp) : 0u;
+      uint4 pf_sv = wc_ok ? __ldg(reinterpret_cast<const uint4 *>(scp)) : make_uint4(0, 0, 0, 0);
+      int64_t grp = 0;
+      int gstage = 0;
       for (int kb = 0; kb < nk; ++kb, ++it) {
         const uint32_t s = it % kStages, ph = (it / kStages) & 1;
-        const int64_t grp = (int64_t)kb * kBK / p.group;  // whole steps lie in one group (group % 64 == 0)
-        if (grp != cur_grp) {
-          cur_grp = grp;
-          const uint32_t zw = wc_ok ? (uint32_t)__ldg(qzp + grp * NW) : 0u;
-          const uint4 sv = wc_ok ? __ldg(reinterpret_cast<const uint4 *>(scp + grp * p.N)) : make_uint4(0, 0, 0, 0);
-          const uint32_t s4[4] = {sv.x, sv.y, sv.z, sv.w};
+        if (gstage == 0) {  // a new group: take the prefetched zeros/scales, prefetch the next
+          const uint32_t s4[4] = {pf_sv.x, pf_sv.y, pf_sv.z, pf_sv.w};
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
-            zp[q] = nib_pair<M>(zw >> (4 * q));
+            zp[q] = nib_pair<M>(pf_zw >> (4 * q));
             sp[q] = s4[q];
           }
+          if (wc_ok && grp + 1 < ngroups) {
+            pf_zw = (uint32_t)__ldg(qzp + (grp + 1) * NW);
+            pf_sv = __ldg(reinterpret_cast<const uint4 *>(scp + (grp + 1) * p.N));
+          }
+        }
+        if (++gstage == spg) {
+          gstage = 0;
+          ++grp;
         }
         tc_wait(&full[s], ph, p.status, abort);
         uint8_t *st = stages + s * kStageBytes;
-        if (p.act_dt != (std::is_same<MT, __half>::value ? MOE_F16 : MOE_BF16)) {
+        if (convert) {
           // activation tile to the scale dtype, in place (layout-agnostic)
           uint4 *a4 = reinterpret_cast<uint4 *>(st);
 #pragma unroll
@@ -281,39 +300,42 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
             a4[td + 256 * i] = v;
           }
         }
-        const uint32_t *pk = reinterpret_cast<const uint32_t *>(st + kABytes + kBBytes);
-        uint8_t *bt = st + kABytes;
+        const uint32_t *pk = reinterpret_cast<const uint32_t *>(st + kABytes + kBBytes) + pk0;
+        uint8_t *bt = st + kABytes + b0;
+        uint32_t w[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) w[i] = pk[i * pk_step];
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-          const int r = rg + 8 * i;  // row of the step
-          const uint32_t w =
-              NPROJ == 2 ? pk[(col >> 4) * (kBK * 16) + r * 16 + (col & 15)] : pk[r * 32 + col];
           uint4 c;
-          c.x = Dq<MT>::coef(nib_pair<M>(w), zp[0], sp[0]);        // columns 0, 1
-          c.y = Dq<MT>::coef(nib_pair<M>(w >> 4), zp[1], sp[1]);   // columns 2, 3
-          c.z = Dq<MT>::coef(nib_pair<M>(w >> 8), zp[2], sp[2]);   // columns 4, 5
-          c.w = Dq<MT>::coef(nib_pair<M>(w >> 12), zp[3], sp[3]);  // columns 6, 7
-          // (row r, 8 features) -> 8-row atom r/8, row r%8 of it, chunk XOR (r%8)
-          *reinterpret_cast<uint4 *>(bt + nblk + (r >> 3) * 1024 + (r & 7) * 128 + ((chunk ^ (r & 7)) << 4)) = c;
+          c.x = Dq<MT>::coef(nib_pair<M>(w[i]), zp[0], sp[0]);        // columns 0, 1
+          c.y = Dq<MT>::coef(nib_pair<M>(w[i] >> 4), zp[1], sp[1]);   // columns 2, 3
+          c.z = Dq<MT>::coef(nib_pair<M>(w[i] >> 8), zp[2], sp[2]);   // columns 4, 5
+          c.w = Dq<MT>::coef(nib_pair<M>(w[i] >> 12), zp[3], sp[3]);  // columns 6, 7
+          *reinterpret_cast<uint4 *>(bt + i * 1024) = c;
         }
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bready[s]);
       }
-
-      // ---- epilogue: TMEM -> registers -> bias, rounding, SwiGLU -> HBM
-      tc_wait(accfull, tcount & 1, p.status, abort);
+    }
+  } else {
+    // ---------------- epilogue warps: TMEM -> registers -> bias, rounding, SwiGLU -> HBM
+    const int q = warp & 3;  // TMEM lane quarter of this warp
+    uint32_t tcount = 0;
+    for (int64_t tile = blockIdx.x; tile < total; tile += gridDim.x, ++tcount) {
+      const TileInfo ti = tile_info(tile);
+      const uint32_t buf = tcount & 1;
+      tc_wait(&accfull[buf], (tcount >> 1) & 1, p.status, abort);
       tc_fence_after();
-      const int q = warp & 3;         // TMEM lane quarter of this warp
-      const int hf = (warp - 2) >> 2;  // column half
       const int trow = ti.mt * kBM + 32 * q + lane;  // row within the expert
       const bool row_ok = trow < ti.m && !*abort;
       const int64_t row = ti.r0 + trow;
-      const uint32_t tbase = tmem + ((uint32_t)(32 * q) << 16);
+      const uint32_t tbase = tmem + ((uint32_t)(32 * q) << 16) + buf * kBN;
       if (NPROJ == 2) {
 #pragma unroll 1
-        for (int c2 = 0; c2 < 2; ++c2) {
-          const int f0 = hf * 64 + c2 * 32;  // feature within the tile
+        for (int c4 = 0; c4 < 4; ++c4) {
+          const int f0 = c4 * 32;  // feature within the tile
           float gv[32], uv[32];
           tmem_ld32(tbase + f0, gv);
           tmem_ld32(tbase + 128 + f0, uv);
@@ -325,8 +347,8 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
         }
       } else {
 #pragma unroll 1
-        for (int c4 = 0; c4 < 4; ++c4) {
-          const int f0 = hf * 128 + c4 * 32;
+        for (int c8 = 0; c8 < 8; ++c8) {
+          const int f0 = c8 * 32;
           float yv[32];
           tmem_ld32(tbase + f0, yv);
           const int64_t n0 = (int64_t)ti.nt * 256 + f0;
@@ -338,7 +360,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(accempty);
+      if (lane == 0) mbar_arrive(&accempty[buf]);
     }
   }
   tc_fence_before();

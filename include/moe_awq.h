@@ -49,7 +49,8 @@
  *                                  the FP32 accumulator before rounding
  *   coefficient W[e,kk,n] = RNE_scale_dtype((q - z[kk/group, n]) * s[kk/group, n]):
  *   the exact product rounded once to the scale dtype.
- *   Requirements: N % 8 == 0, K % group == 0, group % 16 == 0.
+ *   Requirements: N % 8 == 0, K % group == 0, group % 16 == 0; qweight,
+ *   scales, bias and the activation/output tensors 16-byte aligned.
  *   The tensor-core products run in the scale dtype; activations are
  *   converted to it when they differ (BF16 -> F16 is exact for values in
  *   F16's normal range).  FP32 scales are rejected with
@@ -319,10 +320,13 @@ MOE_API moe_status awq_dequant_coefficients(const int32_t *qweight, const int32_
 
 /* ------------------------------------------------------------------------
  * Projection tile path: 0 = chosen from A and E (default), 1 = warp-level
- * tiles (small per-expert batches), 2 = tcgen05/TMEM tiles (large batches).
- * Both paths compute the same operation; the knob exists so tests and
- * benchmarks can run either on the same inputs.  Process-wide; returns the
- * previous value, or -1 for an unknown path.
+ * tiles (small per-expert batches), 2 = tcgen05/TMEM tiles of 128 rows on one
+ * SM (mid-size batches), 3 = tcgen05 tiles of 256 rows on a CTA pair
+ * (cta_group::2, batches of several hundred rows per expert).  All paths
+ * compute the same operation; the knob exists so tests and benchmarks can
+ * run any of them on the same inputs.  A shape a tcgen05 path does not take
+ * runs on the next path down.  Process-wide; returns the previous value, or
+ * -1 for an unknown path.
  * ---------------------------------------------------------------------- */
 MOE_API int32_t moe_set_projection_path(int32_t path);
 

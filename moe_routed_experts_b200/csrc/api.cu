@@ -38,14 +38,31 @@ int num_sms() {
 
 static std::atomic<int> g_path{0};
 
-// Both tile paths hold the same operation; the warp-level one is chosen when
+// All tile paths hold the same operation.  The warp-level one is chosen when
 // the average batch per expert is too small to fill a 128-row tcgen05 tile,
-// or when the shape is one the tcgen05 tile does not take (see tc_fits).
+// the CTA-pair one when experts average 384 rows or more (a 256-row tile is
+// then at most a third empty on average), and a shape a tcgen05 tile does
+// not take (tc_fits / tc2_fits) falls to the next path down.
 static int choose_path(int64_t A, int64_t E) {
   int forced = g_path.load();
-  if (forced == 1 || forced == 2) return forced;
+  if (forced >= 1 && forced <= 3) return forced;
   if (!tc_available()) return 1;
+  if (A >= 384 * E) return 3;
   return (A >= 32 * E) ? 2 : 1;
+}
+
+// Launches the tcgen05 forward tile for the chosen path; returns false if
+// the shape is not one those tiles take.
+static bool try_fwd_tc(int path, const ProjParams &p, int nproj, bool bf, cudaStream_t st, moe_status *out) {
+  if (path == 3 && tc2_fits(p)) {
+    *out = launch_fwd_tc2(p, nproj, bf, st);
+    return true;
+  }
+  if (path >= 2 && tc_fits(p)) {
+    *out = launch_fwd_tc(p, nproj, bf, st);
+    return true;
+  }
+  return false;
 }
 
 // Token columns per warp-level tile: 16 when experts average >= 12 rows.
@@ -87,8 +104,8 @@ extern "C" const char *moe_last_error_string(void) { return g_err; }
 extern "C" const char *moe_version(void) { return "moe_awq 0.1.0 sm_100a"; }
 
 extern "C" int32_t moe_set_projection_path(int32_t path) {
-  if (path < 0 || path > 2) return -1;
-  if (path == 2 && !tc_available()) return -1;
+  if (path < 0 || path > 3) return -1;
+  if (path >= 2 && !tc_available()) return -1;
   return g_path.exchange(path);
 }
 
@@ -101,7 +118,8 @@ extern "C" size_t awq_projection_workspace_size(int64_t A, int64_t K, int64_t N,
   probe.N = N;
   probe.E = (int)E;
   probe.group = (int)group_size;
-  if (choose_path(A, E) == 2 && tc_fits(probe)) return 0;
+  const int path = choose_path(A, E);
+  if ((path == 3 && tc2_fits(probe)) || (path >= 2 && tc_fits(probe))) return 0;
   const StreamPlan pl = stream_plan(A, K, N, E, group_size, nproj, small_tile_tokens(A, E));
   return pl.fits ? pl.bytes : 0;
 }
@@ -119,7 +137,7 @@ extern "C" moe_status awq_grouped_gate_up_swiglu(
     return set_error(MOE_ERR_UNSUPPORTED_DTYPE, "%s: bad bias dtype", fn);
   if (A == 0) return MOE_OK;
   s = check_ptrs(fn, {values, offsets, qweight_gate, qzeros_gate, scales_gate, qweight_up, qzeros_up, scales_up, h},
-                 {values, scales_gate, scales_up, h, gate_out, up_out, qweight_gate, qweight_up});
+                 {values, scales_gate, scales_up, h, gate_out, up_out, qweight_gate, qweight_up, bias_gate, bias_up});
   if (s != MOE_OK) return s;
   ProjParams p{};
   p.x = static_cast<const uint16_t *>(values);
@@ -145,7 +163,8 @@ extern "C" moe_status awq_grouped_gate_up_swiglu(
   p.status = device_status;
   cudaStream_t st = as_stream(stream);
   const bool bf = scale_dtype == MOE_BF16;
-  if (choose_path(A, E) == 2 && tc_fits(p)) return launch_fwd_tc(p, 2, bf, st);
+  moe_status ts;
+  if (try_fwd_tc(choose_path(A, E), p, 2, bf, st, &ts)) return ts;
   const int nt = small_tile_tokens(A, E);
   if (stream_plan(A, H, I, E, group_size, 2, nt).fits) return launch_fwd_stream(p, 2, bf, nt, workspace, workspace_bytes, st);
   launch_fwd_mma(p, 2, bf, nt, st);
@@ -163,7 +182,7 @@ extern "C" moe_status awq_grouped_down(const void *input, moe_dtype act_dtype, i
   if (s != MOE_OK) return s;
   if (bias && !valid_dtype(bias_dtype)) return set_error(MOE_ERR_UNSUPPORTED_DTYPE, "%s: bad bias dtype", fn);
   if (A == 0) return MOE_OK;
-  s = check_ptrs(fn, {input, offsets, qweight, qzeros, scales, output}, {input, scales, output, qweight});
+  s = check_ptrs(fn, {input, offsets, qweight, qzeros, scales, output}, {input, scales, output, qweight, bias});
   if (s != MOE_OK) return s;
   ProjParams p{};
   p.x = static_cast<const uint16_t *>(input);
@@ -183,7 +202,8 @@ extern "C" moe_status awq_grouped_down(const void *input, moe_dtype act_dtype, i
   p.status = device_status;
   cudaStream_t st = as_stream(stream);
   const bool bf = scale_dtype == MOE_BF16;
-  if (choose_path(A, E) == 2 && tc_fits(p)) return launch_fwd_tc(p, 1, bf, st);
+  moe_status ts;
+  if (try_fwd_tc(choose_path(A, E), p, 1, bf, st, &ts)) return ts;
   const int nt = small_tile_tokens(A, E);
   if (stream_plan(A, K, N, E, group_size, 1, nt).fits) return launch_fwd_stream(p, 1, bf, nt, workspace, workspace_bytes, st);
   launch_fwd_mma(p, 1, bf, nt, st);
@@ -227,7 +247,7 @@ extern "C" moe_status awq_input_backward(const void *grad, moe_dtype grad_dtype,
   cudaStream_t st = as_stream(stream);
   const bool bf = scale_dtype == MOE_BF16;
   const int nproj = grad2 ? 2 : 1;
-  if (choose_path(A, E) == 2 && tc_bwd_fits(p)) return launch_bwd_tc(p, nproj, bf, st);
+  if (choose_path(A, E) >= 2 && tc_bwd_fits(p)) return launch_bwd_tc(p, nproj, bf, st);
   launch_bwd_mma(p, nproj, bf, A >= 12 * E ? 2 : 1, st);
   return check_launch(fn);
 }

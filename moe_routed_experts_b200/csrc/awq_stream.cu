@@ -277,13 +277,18 @@ __global__ void __launch_bounds__(stream::kThreads, 2)
     for (int c = 0; c < nst; ++c, ++it) {
       const uint32_t s = it % kStages, ph = (it / kStages) & 1;
       if (c == 0 || gstage == 0) {  // a stage lies inside one group
-        if (std::is_same<MT, __half>::value) {  // |s| <= 256 for all 8 scales of this column group
+        if (std::is_same<MT, __half>::value) {
+          // 16 RNE((q - z) s) = RNE(16 (q - z) s) needs every nonzero product
+          // normal before and after the scaling: 0 or 2^-14 <= |s| <= 256 for
+          // all 8 scales of this column group
           const uint32_t w4[4] = {pf_sv.x, pf_sv.y, pf_sv.z, pf_sv.w};
-          uint32_t big = 0;
+          uint32_t bad = 0;
 #pragma unroll
-          for (int i = 0; i < 4; ++i)
-            big |= ((w4[i] & 0x7FFFu) > 0x5C00u) | (((w4[i] >> 16) & 0x7FFFu) > 0x5C00u);
-          x16 = big == 0;
+          for (int i = 0; i < 4; ++i) {
+            const uint32_t lo = w4[i] & 0x7FFFu, hi = (w4[i] >> 16) & 0x7FFFu;
+            bad |= (lo > 0x5C00u) | (hi > 0x5C00u) | (lo != 0u && lo < 0x0400u) | (hi != 0u && hi < 0x0400u);
+          }
+          x16 = bad == 0;
         }
         cst.load(pf_zw, pf_sv, x16);
         if (wc_ok && (grp + 1) * p.group < kbase + Kq) {  // prefetch the next group

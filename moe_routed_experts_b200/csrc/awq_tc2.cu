@@ -1,0 +1,389 @@
+// Grouped AWQ projections on CTA pairs: one 256-row x 256-column tile per
+// cluster of two SMs (tcgen05.mma.cta_group::2, M = 256), for experts whose
+// batches fill 256-row tiles (long prefill batches, hot experts).
+//
+// ruda-tensor 0.21.34, src/packed_experts.rs -- packed_expert_forward /
+//   packed_swiglu_forward (gate/up/down of the selected experts, SwiGLU);
+// ruda-tensor 0.21.33, src/frozen_awq.rs -- AWQ nibble order and scale-dtype
+//   coefficient rounding; the tensor-core products run in the scale dtype.
+//
+// Why a pair: the coefficient tile is formed in shared memory from packed
+// words, so its cost (dequant instructions and shared-memory stores) is paid
+// once per row tile.  With M = 256 the pair MMA reads each CTA's 128-column
+// half of B for all 256 rows, so each SM dequantizes half as many
+// coefficients per FLOP as a 128-row single-SM tile, and each SM's tensor
+// core reads 8 KB of operands per 128 x 256 x 16 step instead of 12 KB.
+//
+// Split of one tile over the pair (CTA rank r = 0, 1):
+//   A: rows 128 r .. 128 r + 127 of the tile, in CTA r (TMA, 128B swizzle);
+//   B: output columns 128 r .. 128 r + 127 in CTA r -- for the gate/up pair
+//      CTA 0 forms the gate coefficients and CTA 1 the up coefficients of the
+//      same 128 features, so SwiGLU still sees G and U of a feature in one
+//      TMEM lane;
+//   D: rows 128 r .. of the tile, all 256 columns, in CTA r's TMEM.
+// Warp roles in each CTA: warp 0 TMA producer (activations + this CTA's
+// packed words, 6-stage ring); warp 1 TMEM allocation, and in CTA 0 lane 0
+// issues the pair MMAs; warps 2-17 dequantize this CTA's B half (two words
+// per thread and step) into a 4-stage coefficient ring and signal CTA 0;
+// warps 18-21 drain this CTA's accumulator (two TMEM buffers, so draining
+// overlaps the next tile).
+// Every wait is bounded.  CTA 1's dequant and epilogue warps arrive on CTA
+// 0's barriers through the cluster shared-memory window.
+#include <cudaTypedefs.h>
+
+#include "dequant.cuh"
+#include "proj.cuh"
+#include "tcgen05.cuh"
+
+namespace moe {
+
+namespace tc2 {
+constexpr int kBM = 128;   // rows per CTA (256 per pair)
+constexpr int kBN = 256;   // accumulator columns
+constexpr int kHalf = 128; // B columns held by each CTA
+constexpr int kBK = 64;
+constexpr int kLStages = 6, kBStages = 4;
+constexpr int kDqWarps = 16, kEpWarps = 4;
+constexpr int kThreads = (2 + kDqWarps + kEpWarps) * 32;  // 704
+constexpr int kRowGroups = kDqWarps * 2;                   // 16 word columns x kRowGroups threads
+constexpr int kWordsPerThread = kBK / kRowGroups;          // rows rg, rg + kRowGroups, ...
+constexpr int kABytes = kBM * kBK * 2;        // 16 KB
+constexpr int kPBytes = kBK * (kHalf / 8) * 4;  // 4 KB packed words
+constexpr int kLBytes = kABytes + kPBytes;    // one TMA stage
+constexpr int kBBytes = kHalf * kBK * 2;      // 16 KB coefficient half-tile
+constexpr int kTmemCols = 512;
+}  // namespace tc2
+
+struct PairTile {
+  int e, mt, nt;
+  int64_t r0;
+  int m;
+};
+
+template <typename MT, int NPROJ>
+__global__ void __launch_bounds__(tc2::kThreads, 1)
+    awq_fwd_tc2_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_w0,
+                       const __grid_constant__ CUtensorMap map_w1, ProjParams p) {
+  using namespace tc2;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t *smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
+  uint8_t *lring = smem;
+  uint8_t *bring = smem + kLStages * kLBytes;
+  uint64_t *lfull = reinterpret_cast<uint64_t *>(bring + kBStages * kBBytes);
+  uint64_t *lempty = lfull + kLStages;
+  uint64_t *bready = lempty + kLStages;  // used in CTA 0 (both CTAs' dequant warps)
+  uint64_t *bfree = bready + kBStages;
+  uint64_t *accfull = bfree + kBStages;  // [2]
+  uint64_t *accempty = accfull + 2;      // [2], used in CTA 0 (both CTAs' epilogues)
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(accempty + 2);
+  volatile int32_t *abort = reinterpret_cast<volatile int32_t *>(tmem_slot + 1);
+  int32_t *pre = reinterpret_cast<int32_t *>(tmem_slot + 4);  // [E + 1]
+  int32_t *cnt = pre + (p.E + 1);                             // [E]
+  int32_t *tmp = cnt + p.E;                                   // [32]
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank();
+  const int64_t pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+  const int E = p.E;
+  const int64_t K = p.K, NW = p.N / 8;
+  const int feat_tile = NPROJ == 2 ? kHalf : kBN;
+  const int NT = (int)((p.N + feat_tile - 1) / feat_tile);
+  const int nk = (int)(K / kBK);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kLStages; ++s) {
+      mbar_init(&lfull[s], 1);
+      mbar_init(&lempty[s], 1 + kDqWarps);  // pair-MMA commit + this CTA's dequant warps
+    }
+    for (int s = 0; s < kBStages; ++s) {
+      mbar_init(&bready[s], 2 * kDqWarps);
+      mbar_init(&bfree[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&accfull[b], 1);
+      mbar_init(&accempty[b], 2 * kEpWarps);
+    }
+    *abort = 0;
+    fence_mbar_init();
+  }
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    const int32_t a = p.offsets[e], b = p.offsets[e + 1];
+    const bool bad = a < 0 || b < a || (int64_t)b > p.A || (e == 0 && a != 0) || (e == E - 1 && (int64_t)b != p.A);
+    if (bad && blockIdx.x == 0) report(p.status, MOE_DEVICE_ERR_OFFSETS);
+    cnt[e] = bad ? 0 : NT * ((b - a + 2 * kBM - 1) / (2 * kBM));
+  }
+  __syncthreads();
+  block_exclusive_scan(cnt, E, pre, tmp);
+  const int64_t total = pre[E];
+  if (pair >= total) return;  // same answer in both CTAs of the pair
+
+  auto tile_info = [&](int64_t tile) {
+    PairTile ti;
+    int lo = 0, hi = E - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (pre[mid] <= tile) lo = mid;
+      else hi = mid - 1;
+    }
+    ti.e = lo;
+    const int64_t local = tile - pre[lo];
+    ti.mt = (int)(local / NT);
+    ti.nt = (int)(local % NT);
+    ti.r0 = p.offsets[lo];
+    ti.m = p.offsets[lo + 1] - (int32_t)ti.r0;
+    return ti;
+  };
+
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                 "r"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  cluster_sync_all();  // barriers of both CTAs initialised, TMEM allocated
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ---------------- producer: this CTA's activation rows and packed half
+    if (lane == 0) {
+      const CUtensorMap *mw = (NPROJ == 2 && rank == 1) ? &map_w1 : &map_w0;
+      uint32_t it = 0;
+      for (int64_t tile = pair; tile < total; tile += npairs) {
+        const PairTile ti = tile_info(tile);
+        const int32_t row0 = (int32_t)(ti.r0 + (int64_t)ti.mt * 2 * kBM + kBM * rank);
+        const int32_t wcol = NPROJ == 2 ? ti.nt * 16 : ti.nt * 32 + 16 * (int)rank;
+        for (int kb = 0; kb < nk; ++kb, ++it) {
+          const uint32_t s = it % kLStages, use = it / kLStages;
+          if (use > 0) tc_wait(&lempty[s], (use - 1) & 1, p.status, abort);
+          uint8_t *st = lring + s * kLBytes;
+          mbar_arrive_expect_tx(&lfull[s], kLBytes);
+          tma_load_2d(st, &map_x, &lfull[s], kb * kBK, row0);
+          tma_load_2d(st + kABytes, mw, &lfull[s], wcol, (int32_t)(ti.e * K + (int64_t)kb * kBK));
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- pair MMA issuer (CTA 0 only)
+    if (rank == 0 && lane == 0) {
+      constexpr uint32_t fmt = std::is_same<MT, __half>::value ? 0u : 1u;
+      // D F32, A/B in the scale dtype, A K-major, B MN-major, N = 256, M = 256
+      const uint32_t idesc = (1u << 4) | (fmt << 7) | (fmt << 10) | (1u << 16) | ((uint32_t)(kBN >> 3) << 17) |
+                             ((uint32_t)((2 * kBM) >> 4) << 24);
+      uint32_t it = 0, tcount = 0;
+      for (int64_t tile = pair; tile < total; tile += npairs, ++tcount) {
+        const uint32_t buf = tcount & 1, use = tcount >> 1;
+        if (use > 0) tc_wait_cluster(&accempty[buf], (use - 1) & 1, p.status, abort);
+        tc_fence_after();
+        const uint32_t dacc = tmem + buf * kBN;
+        for (int kb = 0; kb < nk; ++kb, ++it) {
+          const uint32_t ls = it % kLStages, bs = it % kBStages;
+          // both CTAs' dequant warps arrive only after their own TMA stage landed
+          tc_wait_cluster(&bready[bs], (it / kBStages) & 1, p.status, abort);
+          tc_fence_after();
+          const uint64_t adesc = smem_desc(smem_u32(lring + ls * kLBytes), 16, 1024);
+          const uint64_t bdesc = smem_desc(smem_u32(bring + bs * kBBytes), 8192, 1024);
+#pragma unroll
+          for (int j = 0; j < kBK / 16; ++j)
+            umma2_f16(dacc, adesc + (uint64_t)(2 * j), bdesc + (uint64_t)(128 * j), idesc, (kb | j) != 0);
+          umma2_commit_both(&lempty[ls]);
+          umma2_commit_both(&bfree[bs]);
+        }
+        umma2_commit_both(&accfull[buf]);
+      }
+    }
+  } else if (warp < 2 + kDqWarps) {
+    // ---------------- dequant warps: this CTA's 128-column half of B
+    const int td = threadIdx.x - 64;  // 0 .. 32 kDqWarps - 1
+    const int col = td & 15;          // word column within the half
+    const int rg = td >> 4;           // rows rg, rg + kRowGroups, ... of each step
+    const int proj = NPROJ == 2 ? (int)rank : 0;
+    constexpr uint32_t M = Dq<MT>::kMagic2;
+    const int64_t ngroups = K / p.group;
+    const int32_t *qz = p.qz[proj];
+    const uint16_t *sc = p.sc[proj];
+    const int pk0 = rg * 16 + col;
+    // features col*8 .. col*8+7 of the half -> 64-column block col/8, 16-byte
+    // chunk col%8 XOR row%8 (MN-major, 128-byte swizzle, 8-row x 64-column atoms)
+    const int b0 = (col >> 3) * 8192 + (rg >> 3) * 1024 + (rg & 7) * 128 + (((col & 7) ^ (rg & 7)) << 4);
+    const int spg = p.group / kBK;
+    const bool convert = p.act_dt != (std::is_same<MT, __half>::value ? MOE_F16 : MOE_BF16);
+    uint64_t *bready0 = bready;  // CTA 0's barriers, addressed through the cluster window
+    uint32_t it = 0;
+    for (int64_t tile = pair; tile < total; tile += npairs) {
+      const PairTile ti = tile_info(tile);
+      const int64_t wc = NPROJ == 2 ? (int64_t)ti.nt * 16 + col : (int64_t)ti.nt * 32 + 16 * rank + col;
+      const bool wc_ok = wc < NW;
+      const int64_t wcs = wc_ok ? wc : 0;
+      const int32_t *qzp = qz + (int64_t)ti.e * ngroups * NW + wcs;
+      const uint16_t *scp = sc + (int64_t)ti.e * ngroups * p.N + 8 * wcs;
+      uint32_t zp[4], sp[4];
+      uint32_t pf_zw = wc_ok ? (uint32_t)__ldg(qzp) : 0u;
+      uint4 pf_sv = wc_ok ? __ldg(reinterpret_cast<const uint4 *>(scp)) : make_uint4(0, 0, 0, 0);
+      int64_t grp = 0;
+      int gstage = 0;
+      for (int kb = 0; kb < nk; ++kb, ++it) {
+        const uint32_t ls = it % kLStages, bs = it % kBStages, buse = it / kBStages;
+        if (gstage == 0) {
+          const uint32_t s4[4] = {pf_sv.x, pf_sv.y, pf_sv.z, pf_sv.w};
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            zp[q] = nib_pair<M>(pf_zw >> (4 * q));
+            sp[q] = s4[q];
+          }
+          if (wc_ok && grp + 1 < ngroups) {
+            pf_zw = (uint32_t)__ldg(qzp + (grp + 1) * NW);
+            pf_sv = __ldg(reinterpret_cast<const uint4 *>(scp + (grp + 1) * p.N));
+          }
+        }
+        if (++gstage == spg) {
+          gstage = 0;
+          ++grp;
+        }
+        tc_wait(&lfull[ls], (it / kLStages) & 1, p.status, abort);
+        uint8_t *st = lring + ls * kLBytes;
+        uint32_t w[kWordsPerThread];
+        {
+          const uint32_t *pk = reinterpret_cast<const uint32_t *>(st + kABytes) + pk0;
+#pragma unroll
+          for (int i = 0; i < kWordsPerThread; ++i) w[i] = pk[i * kRowGroups * 16];
+        }
+        if (convert) {
+          uint4 *a4 = reinterpret_cast<uint4 *>(st);
+#pragma unroll
+          for (int i = 0; i < kABytes / 16 / (32 * kDqWarps); ++i) {
+            uint4 v = a4[td + 32 * kDqWarps * i];
+            v.x = act_pair_to_mt<MT>(v.x, p.act_dt);
+            v.y = act_pair_to_mt<MT>(v.y, p.act_dt);
+            v.z = act_pair_to_mt<MT>(v.z, p.act_dt);
+            v.w = act_pair_to_mt<MT>(v.w, p.act_dt);
+            a4[td + 32 * kDqWarps * i] = v;
+          }
+          fence_proxy_async_smem();
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&lempty[ls]);  // packed words read (the pair commit frees A)
+        if (buse > 0) tc_wait(&bfree[bs], (buse - 1) & 1, p.status, abort);
+        uint8_t *bt = bring + bs * kBBytes + b0;
+#pragma unroll
+        for (int i = 0; i < kWordsPerThread; ++i) {
+          uint4 c;
+          c.x = Dq<MT>::coef(nib_pair<M>(w[i]), zp[0], sp[0]);
+          c.y = Dq<MT>::coef(nib_pair<M>(w[i] >> 4), zp[1], sp[1]);
+          c.z = Dq<MT>::coef(nib_pair<M>(w[i] >> 8), zp[2], sp[2]);
+          c.w = Dq<MT>::coef(nib_pair<M>(w[i] >> 12), zp[3], sp[3]);
+          *reinterpret_cast<uint4 *>(bt + i * kRowGroups * 128) = c;  // rows + kRowGroups
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(cluster_addr(&bready0[bs], 0));
+      }
+    }
+  } else {
+    // ---------------- epilogue warps: this CTA's 128 rows of the tile
+    const int q = warp & 3;
+    uint32_t tcount = 0;
+    for (int64_t tile = pair; tile < total; tile += npairs, ++tcount) {
+      const PairTile ti = tile_info(tile);
+      const uint32_t buf = tcount & 1;
+      tc_wait(&accfull[buf], (tcount >> 1) & 1, p.status, abort);
+      tc_fence_after();
+      const int trow = ti.mt * 2 * kBM + kBM * (int)rank + 32 * q + lane;
+      const bool row_ok = trow < ti.m && !*abort;
+      const int64_t row = ti.r0 + trow;
+      const uint32_t tbase = tmem + ((uint32_t)(32 * q) << 16) + buf * kBN;
+      if (NPROJ == 2) {
+#pragma unroll 1
+        for (int c8 = 0; c8 < 8; ++c8) {
+          const int f0 = c8 * 16;
+          float gv[16], uv[16];
+          tmem_ld16(tbase + f0, gv);
+          tmem_ld16(tbase + kHalf + f0, uv);
+          const int64_t n0 = (int64_t)ti.nt * kHalf + f0;
+          if (row_ok && n0 < p.N) {
+#pragma unroll
+            for (int v8 = 0; v8 < 2; ++v8) finish8<2>(p, ti.e, row, n0 + 8 * v8, gv + 8 * v8, uv + 8 * v8);
+          }
+        }
+      } else {
+#pragma unroll 1
+        for (int c16 = 0; c16 < 16; ++c16) {
+          const int f0 = c16 * 16;
+          float yv[16];
+          tmem_ld16(tbase + f0, yv);
+          const int64_t n0 = (int64_t)ti.nt * kBN + f0;
+          if (row_ok && n0 < p.N) {
+#pragma unroll
+            for (int v8 = 0; v8 < 2; ++v8) finish8<1>(p, ti.e, row, n0 + 8 * v8, yv + 8 * v8, yv + 8 * v8);
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(cluster_addr(&accempty[buf], 0));
+    }
+  }
+  // Neither CTA leaves while its peer may still read its shared memory or
+  // arrive on its barriers; then both release the pair's TMEM.
+  __syncwarp();
+  tc_fence_before();
+  cluster_sync_all();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
+  }
+}
+
+// ------------------------------------------------------------------ launch
+
+static size_t tc2_smem(int64_t E) {
+  return 1024 + (size_t)tc2::kLStages * tc2::kLBytes + (size_t)tc2::kBStages * tc2::kBBytes + 256 +
+         (size_t)(2 * E + 1 + 32) * 4;
+}
+
+bool tc2_fits(const ProjParams &p) {
+  return p.K % tc2::kBK == 0 && p.group % tc2::kBK == 0 && p.N % 32 == 0 && tc2_smem(p.E) <= 227 * 1024;
+}
+
+template <typename MT, int NPROJ>
+static moe_status launch_tc2_t(const ProjParams &p, cudaStream_t st) {
+  using namespace tc2;
+  CUtensorMap mx, m0, m1;
+  const uint64_t NW = p.N / 8, rows = (uint64_t)p.E * p.K;
+  if (!make_map_2d(&mx, p.x, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, p.K, p.A, kBK, kBM, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map_2d(&m0, p.qw[0], CU_TENSOR_MAP_DATA_TYPE_INT32, 4, NW, rows, 16, kBK, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !make_map_2d(&m1, p.qw[NPROJ - 1], CU_TENSOR_MAP_DATA_TYPE_INT32, 4, NW, rows, 16, kBK,
+                   CU_TENSOR_MAP_SWIZZLE_NONE))
+    return set_error(MOE_ERR_CUDA, "tensor map encoding failed (tcgen05 pair projection)");
+  const size_t smem = tc2_smem(p.E);
+  auto kern = awq_fwd_tc2_kernel<MT, NPROJ>;
+  cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cfg.gridDim = dim3(2 * (num_sms() / 2));
+  int clusters = 0;
+  if (cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg) != cudaSuccess || clusters < 1) {
+    cudaGetLastError();
+    return set_error(MOE_ERR_CUDA, "no co-resident SM pair for the tcgen05 pair projection");
+  }
+  cfg.gridDim = dim3(2 * clusters);  // persistent: every pair resident at once
+  cudaLaunchKernelEx(&cfg, kern, mx, m0, m1, p);
+  return check_launch("awq_fwd_tc2_kernel");
+}
+
+moe_status launch_fwd_tc2(const ProjParams &p, int nproj, bool bf16_mma, cudaStream_t st) {
+  if (bf16_mma) return nproj == 2 ? launch_tc2_t<__nv_bfloat16, 2>(p, st) : launch_tc2_t<__nv_bfloat16, 1>(p, st);
+  return nproj == 2 ? launch_tc2_t<__half, 2>(p, st) : launch_tc2_t<__half, 1>(p, st);
+}
+
+}  // namespace moe

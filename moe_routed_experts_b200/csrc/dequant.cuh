@@ -45,8 +45,10 @@ __device__ __forceinline__ void fwd_pairs(uint32_t wa, uint32_t wb, int p, const
 // F16 variant of fwd_pairs with fewer shifts: the code of an odd slot is
 // used where it sits (bits 4..7 of its byte), so the lane holds 1024 + 16q
 // (exact: below 2048) and the coefficient comes out as
-// RNE(16 (q - z) s) = 16 RNE((q - z) s), exact whenever 16 * 15 * |s| does
-// not overflow F16 (the caller checks |s| <= 256).  The MMAs of the odd
+// RNE(16 (q - z) s) = 16 RNE((q - z) s), exact whenever every nonzero
+// product stays a normal F16 number before and after the scaling (the caller
+// checks s = 0 or 2^-14 <= |s| <= 256; a subnormal product would be rounded
+// on a coarser grid than its 16-times-larger normal image).  The MMAs of the odd
 // slots therefore accumulate 16 times the true sum, which the caller
 // rescales by 1/16 (exact) at the end.
 __device__ __forceinline__ void fwd_pairs16(uint32_t wa, uint32_t wb, int p, const FwdConsts<__half> &c,

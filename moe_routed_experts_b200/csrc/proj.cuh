@@ -41,49 +41,81 @@ struct BwdParams {
   int32_t *status;
 };
 
+// 8 bias values n0.. of local expert e (0 without a bias), with 16-byte loads.
+__device__ __forceinline__ void bias8(const void *bias, int dt, int64_t i0, float (&b)[8]) {
+  if (!bias) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) b[i] = 0.f;
+  } else if (dt == MOE_F32) {
+    const float4 *q = reinterpret_cast<const float4 *>(reinterpret_cast<const float *>(bias) + i0);
+    const float4 v0 = __ldg(q), v1 = __ldg(q + 1);
+    b[0] = v0.x, b[1] = v0.y, b[2] = v0.z, b[3] = v0.w, b[4] = v1.x, b[5] = v1.y, b[6] = v1.z, b[7] = v1.w;
+  } else {
+    const uint4 v = __ldg(reinterpret_cast<const uint4 *>(reinterpret_cast<const uint16_t *>(bias) + i0));
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      b[2 * i] = bits_to_f32((uint16_t)(w[i] & 0xFFFFu), dt);
+      b[2 * i + 1] = bits_to_f32((uint16_t)(w[i] >> 16), dt);
+    }
+  }
+}
+
+// Two FP32 values rounded (RNE) to the activation dtype, packed low/high.
+template <bool BF>
+__device__ __forceinline__ uint32_t round_pair(float a, float b) {
+  if (BF) {
+    const __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
+    return *reinterpret_cast<const uint32_t *>(&v);
+  }
+  const __half2 v = __floats2half2_rn(a, b);
+  return *reinterpret_cast<const uint32_t *>(&v);
+}
+
+template <bool BF>
+__device__ __forceinline__ float2 unpack_pair(uint32_t v) {
+  return make_float2(bits_to_f32((uint16_t)(v & 0xFFFFu), BF ? MOE_BF16 : MOE_F16),
+                     bits_to_f32((uint16_t)(v >> 16), BF ? MOE_BF16 : MOE_F16));
+}
+
+// silu(G) U from the rounded G and U.  Fast exponential and division: their
+// few-ulp FP32 error is far below one rounding of the 16-bit result.
+__device__ __forceinline__ float swiglu1(float G, float U) { return __fdividef(G, 1.f + __expf(-G)) * U; }
+
+template <int NPROJ, bool BF>
+__device__ __forceinline__ void finish8_t(const ProjParams &p, int e, int64_t row, int64_t n0, const float *g,
+                                          const float *u) {
+  float bg[8];
+  bias8(p.bias[0], p.bias_dt, (int64_t)e * p.N + n0, bg);
+  uint32_t o[4];
+  if (NPROJ == 2) {
+    float bu[8];
+    bias8(p.bias[1], p.bias_dt, (int64_t)e * p.N + n0, bu);
+    uint32_t og[4], ou[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      og[i] = round_pair<BF>(g[2 * i] + bg[2 * i], g[2 * i + 1] + bg[2 * i + 1]);
+      ou[i] = round_pair<BF>(u[2 * i] + bu[2 * i], u[2 * i + 1] + bu[2 * i + 1]);
+      const float2 G = unpack_pair<BF>(og[i]), U = unpack_pair<BF>(ou[i]);
+      o[i] = round_pair<BF>(swiglu1(G.x, U.x), swiglu1(G.y, U.y));
+    }
+    if (p.gout) *reinterpret_cast<uint4 *>(p.gout + row * p.N + n0) = make_uint4(og[0], og[1], og[2], og[3]);
+    if (p.uout) *reinterpret_cast<uint4 *>(p.uout + row * p.N + n0) = make_uint4(ou[0], ou[1], ou[2], ou[3]);
+  } else {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) o[i] = round_pair<BF>(g[2 * i] + bg[2 * i], g[2 * i + 1] + bg[2 * i + 1]);
+  }
+  *reinterpret_cast<uint4 *>(p.out + row * p.N + n0) = make_uint4(o[0], o[1], o[2], o[3]);
+}
+
 // Final values of 8 consecutive output columns n0.. of row `row` of local
 // expert e from FP32 sums (gate sums g, up sums u for the pair): bias, one
 // rounding to the activation dtype, SwiGLU from the rounded G and U.
 template <int NPROJ>
 __device__ __forceinline__ void finish8(const ProjParams &p, int e, int64_t row, int64_t n0, const float *g,
                                         const float *u) {
-  uint32_t o[4];
-  if (NPROJ == 2) {
-    uint32_t og[4], ou[4];
-#pragma unroll
-    for (int i = 0; i < 8; i += 2) {
-      float gv[2], uv[2];
-#pragma unroll
-      for (int d = 0; d < 2; ++d) {
-        gv[d] = g[i + d];
-        uv[d] = u[i + d];
-        if (p.bias[0]) gv[d] += ld_as_float(p.bias[0], p.bias_dt, (int64_t)e * p.N + n0 + i + d);
-        if (p.bias[1]) uv[d] += ld_as_float(p.bias[1], p.bias_dt, (int64_t)e * p.N + n0 + i + d);
-      }
-      const uint16_t gb0 = f32_to_bits(gv[0], p.act_dt), gb1 = f32_to_bits(gv[1], p.act_dt);
-      const uint16_t ub0 = f32_to_bits(uv[0], p.act_dt), ub1 = f32_to_bits(uv[1], p.act_dt);
-      const float g0 = bits_to_f32(gb0, p.act_dt), g1 = bits_to_f32(gb1, p.act_dt);
-      const float x0 = bits_to_f32(ub0, p.act_dt), x1 = bits_to_f32(ub1, p.act_dt);
-      const float h0 = g0 / (1.f + expf(-g0)) * x0, h1 = g1 / (1.f + expf(-g1)) * x1;
-      og[i / 2] = uint32_t(gb0) | (uint32_t(gb1) << 16);
-      ou[i / 2] = uint32_t(ub0) | (uint32_t(ub1) << 16);
-      o[i / 2] = uint32_t(f32_to_bits(h0, p.act_dt)) | (uint32_t(f32_to_bits(h1, p.act_dt)) << 16);
-    }
-    if (p.gout) *reinterpret_cast<uint4 *>(p.gout + row * p.N + n0) = make_uint4(og[0], og[1], og[2], og[3]);
-    if (p.uout) *reinterpret_cast<uint4 *>(p.uout + row * p.N + n0) = make_uint4(ou[0], ou[1], ou[2], ou[3]);
-  } else {
-#pragma unroll
-    for (int i = 0; i < 8; i += 2) {
-      float yv[2];
-#pragma unroll
-      for (int d = 0; d < 2; ++d) {
-        yv[d] = g[i + d];
-        if (p.bias[0]) yv[d] += ld_as_float(p.bias[0], p.bias_dt, (int64_t)e * p.N + n0 + i + d);
-      }
-      o[i / 2] = uint32_t(f32_to_bits(yv[0], p.act_dt)) | (uint32_t(f32_to_bits(yv[1], p.act_dt)) << 16);
-    }
-  }
-  *reinterpret_cast<uint4 *>(p.out + row * p.N + n0) = make_uint4(o[0], o[1], o[2], o[3]);
+  if (p.act_dt == MOE_BF16) finish8_t<NPROJ, true>(p, e, row, n0, g, u);
+  else finish8_t<NPROJ, false>(p, e, row, n0, g, u);
 }
 
 void launch_fwd_mma(const ProjParams &p, int nproj, bool bf16_mma, int nt, cudaStream_t st);
@@ -104,5 +136,7 @@ bool tc_fits(const ProjParams &p);
 bool tc_bwd_fits(const BwdParams &p);
 moe_status launch_fwd_tc(const ProjParams &p, int nproj, bool bf16_mma, cudaStream_t st);
 moe_status launch_bwd_tc(const BwdParams &p, int nproj, bool bf16_mma, cudaStream_t st);
+bool tc2_fits(const ProjParams &p);
+moe_status launch_fwd_tc2(const ProjParams &p, int nproj, bool bf16_mma, cudaStream_t st);
 
 }  // namespace moe

@@ -103,5 +103,7 @@ def test_combine_family_rejects_bad_arguments(L):
 def test_projection_path_knob(L):
     assert L.moe_set_projection_path(7) == -1
     prev = L.moe_set_projection_path(1)
-    assert prev in (0, 1, 2)
+    assert prev in (0, 1, 2, 3)
+    assert L.moe_set_projection_path(3) == 1
+    assert L.moe_set_projection_path(1) == 3
     assert L.moe_set_projection_path(prev) == 1

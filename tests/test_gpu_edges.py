@@ -17,7 +17,7 @@ from moe_routed_experts_b200.configs import Workload
 pytestmark = pytest.mark.gpu
 
 
-@pytest.fixture(params=[1, 2], ids=["warp_tiles", "tcgen05_tiles"])
+@pytest.fixture(params=[1, 2, 3], ids=["warp_tiles", "tcgen05_tiles", "tcgen05_pair_tiles"])
 def path(request):
     try:
         prev = B.set_projection_path(request.param)

@@ -15,10 +15,10 @@ from moe_routed_experts_b200.configs import WORKLOADS, Workload, scaled
 
 pytestmark = pytest.mark.gpu
 
-PATHS = [1, 2]
+PATHS = [1, 2, 3]
 
 
-@pytest.fixture(params=PATHS, ids=["warp_tiles", "tcgen05_tiles"])
+@pytest.fixture(params=PATHS, ids=["warp_tiles", "tcgen05_tiles", "tcgen05_pair_tiles"])
 def path(request):
     p = request.param
     try:

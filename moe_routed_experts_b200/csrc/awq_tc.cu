@@ -361,10 +361,6 @@ moe_status launch_fwd_tc(const ProjParams &p, int nproj, bool bf16_mma, cudaStre
   return nproj == 2 ? launch_tc_t<__half, 2>(p, st) : launch_tc_t<__half, 1>(p, st);
 }
 
-bool tc_bwd_fits(const BwdParams &) { return false; }
 
-moe_status launch_bwd_tc(const BwdParams &, int, bool, cudaStream_t) {
-  return set_error(MOE_ERR_UNSUPPORTED_DTYPE, "tcgen05 input-VJP tiles are not built");
-}
 
 }  // namespace moe

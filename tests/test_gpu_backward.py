@@ -66,12 +66,14 @@ def _chain(name, kw, rows=None, tokens=None):
 
 
 SMALL = {"skewed": dict(T=1024, H=512, I=256, E=16), "prefill": dict(T=512, H=256, I=128, E=16, backward=True),
-         "decode": dict(backward=True), "tiny": dict(backward=True)}
+         "decode": dict(backward=True), "tiny": dict(backward=True),
+         # output widths that end inside a 256-column tile, four zero/scale groups per tile
+         "ragged": dict(T=512, H=320, I=192, E=8, group=64)}
 
 
 @pytest.mark.parametrize("name", list(SMALL))
 def test_backward_chain_every_row(name, path):
-    _chain(name, SMALL[name])
+    _chain("skewed" if name == "ragged" else name, SMALL[name])
 
 
 def test_backward_full_size_skewed_sampled(path):

@@ -300,23 +300,24 @@ def main():
         offsets = buf.route["offsets"].cpu().numpy()
         counts = np.diff(offsets)
         pk = peaks()
+        kname = gate_up_kernel_name(B, w)
         if w.name in ("decode", "tiny"):
             alg = packed_bytes(inp, counts, ("gate", "up"))
             achieved = alg / (kernel_ms * 1e-3) / 1e9
-            roof = {"bound": "hbm", "kernel": "awq_fwd_mma_kernel<gate+up>", "achieved": achieved,
+            roof = {"bound": "hbm", "kernel": kname, "achieved": achieved,
                     "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": achieved / pk["hbm_gbs"],
                     "traffic": traffic_for("gate_up_" + w.name), "algorithmic_bytes": alg,
                     "kernel_ms": kernel_ms, "peak_source": pk["source"]}
         else:
             flops = 2.0 * w.A * w.H * 2 * w.I
             achieved = flops / (kernel_ms * 1e-3) / 1e12
-            roof = {"bound": "tensor", "kernel": "gate+up projection", "achieved": achieved,
+            roof = {"bound": "tensor", "kernel": kname, "achieved": achieved,
                     "peak": pk["bf16_tflops"], "unit": "TFLOP/s", "frac": achieved / pk["bf16_tflops"],
                     "traffic": traffic_for("gate_up_" + w.name), "algorithmic_flops": flops,
                     "kernel_ms": kernel_ms, "peak_source": pk["source"] + " burst"}
         all_packed = packed_bytes(inp, counts, ("gate", "up", "down"))
         fwd_flops = 2.0 * w.A * 3 * w.H * w.I
-        launches_per_step = (2 if w.T <= 64 else 3) + 3 + (5 if w.backward else 0)
+        launches_per_step = launches_per_step_of(B, w)
         line = {
             "metric": METRIC, "value": world * w.T / (ms * 1e-3), "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
@@ -358,6 +359,39 @@ def _gate_up_keep(B, r, dev, w, buf):
         B._dt(gate["scales"].dtype), B.MOE_F32, w.group, B._ptr(buf.h), B._ptr(buf.G), B._ptr(buf.U),
         B._ptr(buf.proj_ws), 0 if buf.proj_ws is None else buf.proj_ws.numel(), B._ptr(buf.status), st)
     B._check("awq_grouped_gate_up_swiglu", s)
+
+
+def _path_of(w):
+    """Projection tile path the library picks for this workload (mirrors its rule)."""
+    if w.A >= 384 * w.E:
+        return 3
+    return 2 if w.A >= 32 * w.E else 1
+
+
+def gate_up_kernel_name(B, w):
+    path = _path_of(w)
+    if path == 3:
+        return "awq_grouped_gate_up_swiglu: awq_fwd_tc2_kernel (tcgen05 CTA pair)"
+    if path == 2:
+        return "awq_grouped_gate_up_swiglu: awq_fwd_tc_kernel (tcgen05)"
+    if B.projection_workspace_size(w.A, w.H, w.I, w.E, w.group, 2) > 0:
+        return "awq_grouped_gate_up_swiglu: awq_fwd_stream_kernel + awq_stream_reduce_kernel"
+    return "awq_grouped_gate_up_swiglu: awq_fwd_stream_kernel"
+
+
+def launches_per_step_of(B, w):
+    """Kernel launches of one step: route (2, or 3 past one token chunk), each
+    projection (1, or 2 with the split-K reduce), combine, and the backward's five."""
+    n = 2 if w.T <= 64 else 3
+    if _path_of(w) == 1:
+        n += 1 + (B.projection_workspace_size(w.A, w.H, w.I, w.E, w.group, 2) > 0)
+        n += 1 + (B.projection_workspace_size(w.A, w.I, w.H, w.E, w.group, 1) > 0)
+    else:
+        n += 2
+    n += 1
+    if w.backward:
+        n += 5
+    return n
 
 
 def traffic_for(key):

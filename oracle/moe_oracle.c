@@ -30,7 +30,7 @@
  *     - moe_dispatch_weights_backward: the logit VJP of the FP32 weights at a
  *       fixed selection.
  *
- * Readings taken where the pages are silent (each is listed in the design doc):
+ * Readings taken where the pages are silent:
  *   - nibble order: slot s (bits 4s..4s+3 of the word read as unsigned)
  *     holds logical column 8w+P[s], P = {0,2,4,6,1,3,5,7};
  *   - coefficient W = RNE_sdt((q - z) * s): the product is exact, then

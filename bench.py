@@ -141,9 +141,14 @@ def main():
     ap.add_argument("--no-graph", action="store_true", help="launch kernels directly instead of a CUDA graph")
     ap.add_argument("--soak-seconds", type=float, default=1.0)
     ap.add_argument("--reference-tokens", type=int, default=8)
+    ap.add_argument("--tokens", type=int, default=0,
+                    help="override the workload's token count (smaller profiling captures); 0 keeps it")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     w = WORKLOADS[args.config]
+    if args.tokens > 0:
+        from moe_routed_experts_b200.configs import scaled
+        w = scaled(w, T=args.tokens)
     if args.impl == "reference":
         run_reference(args, w)
         return

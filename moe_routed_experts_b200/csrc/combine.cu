@@ -73,21 +73,29 @@ __global__ void __launch_bounds__(kCombThreads) combine_kernel(CombineParams p) 
       float acc[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) acc[i] = 0.f;
-      for (int j = 0; j < p.k; ++j) {
-        const int32_t r = ord_row[j];
-        if (r < 0) continue;
-        const float wv = ord_w[j];
-        uint4 v = *reinterpret_cast<const uint4 *>(y + (int64_t)r * p.H + c0);
-        const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+      for (int j0 = 0; j0 < p.k; j0 += 8) {
+        // issue up to 8 row loads before summing them in ascending-ID order
+        uint4 v[8];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          float lo = bits_to_f32(uint16_t(u[i] & 0xFFFF), p.dt), hi = bits_to_f32(uint16_t(u[i] >> 16), p.dt);
-          if (p.weights) {
-            acc[2 * i] = __fadd_rn(acc[2 * i], __fmul_rn(wv, lo));
-            acc[2 * i + 1] = __fadd_rn(acc[2 * i + 1], __fmul_rn(wv, hi));
-          } else {
-            acc[2 * i] = __fadd_rn(acc[2 * i], lo);
-            acc[2 * i + 1] = __fadd_rn(acc[2 * i + 1], hi);
+        for (int jj = 0; jj < 8; ++jj) {
+          const int32_t r = j0 + jj < p.k ? ord_row[j0 + jj] : -1;
+          v[jj] = r >= 0 ? *reinterpret_cast<const uint4 *>(y + (int64_t)r * p.H + c0) : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int jj = 0; jj < 8; ++jj) {
+          if (j0 + jj >= p.k || ord_row[j0 + jj] < 0) continue;
+          const float wv = ord_w[j0 + jj];
+          const uint32_t u[4] = {v[jj].x, v[jj].y, v[jj].z, v[jj].w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            float lo = bits_to_f32(uint16_t(u[i] & 0xFFFF), p.dt), hi = bits_to_f32(uint16_t(u[i] >> 16), p.dt);
+            if (p.weights) {
+              acc[2 * i] = __fadd_rn(acc[2 * i], __fmul_rn(wv, lo));
+              acc[2 * i + 1] = __fadd_rn(acc[2 * i + 1], __fmul_rn(wv, hi));
+            } else {
+              acc[2 * i] = __fadd_rn(acc[2 * i], lo);
+              acc[2 * i + 1] = __fadd_rn(acc[2 * i + 1], hi);
+            }
           }
         }
       }
@@ -127,6 +135,8 @@ struct CombineBwdParams {
 
 // One CTA per token.  dy rows are written with one rounding of the exact
 // FP32 product; the dots are reduced in a fixed tree (per thread, warp, CTA).
+// VEC: 8 columns per thread and access (16-byte loads and stores).
+template <bool VEC>
 __global__ void __launch_bounds__(kCombThreads) combine_bwd_kernel(CombineBwdParams p) {
   __shared__ float red[kCombThreads / 32][MOE_MAX_TOP_K];
   const int64_t t = blockIdx.x;
@@ -140,7 +150,35 @@ __global__ void __launch_bounds__(kCombThreads) combine_bwd_kernel(CombineBwdPar
     if (!ok && threadIdx.x == 0) report(p.status, MOE_DEVICE_ERR_ROW_RANGE);
     const float w = p.weights[t * p.k + j];
     float dot = 0.f;
-    if (ok) {
+    if (ok && VEC) {
+      for (int64_t c0 = (int64_t)threadIdx.x * 8; c0 < p.H; c0 += (int64_t)blockDim.x * 8) {
+        const uint4 gv = *reinterpret_cast<const uint4 *>(g + t * p.H + c0);
+        const uint32_t gu[4] = {gv.x, gv.y, gv.z, gv.w};
+        float gf[8];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          gf[2 * i] = bits_to_f32(uint16_t(gu[i] & 0xFFFF), p.dt);
+          gf[2 * i + 1] = bits_to_f32(uint16_t(gu[i] >> 16), p.dt);
+        }
+        if (dy) {
+          uint32_t o[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            o[i] = uint32_t(f32_to_bits(__fmul_rn(w, gf[2 * i]), p.dt)) |
+                   (uint32_t(f32_to_bits(__fmul_rn(w, gf[2 * i + 1]), p.dt)) << 16);
+          *reinterpret_cast<uint4 *>(dy + (int64_t)r * p.H + c0) = make_uint4(o[0], o[1], o[2], o[3]);
+        }
+        if (p.dweights) {
+          const uint4 yv = *reinterpret_cast<const uint4 *>(y + (int64_t)r * p.H + c0);
+          const uint32_t yu[4] = {yv.x, yv.y, yv.z, yv.w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            dot = fmaf(gf[2 * i], bits_to_f32(uint16_t(yu[i] & 0xFFFF), p.dt), dot);
+            dot = fmaf(gf[2 * i + 1], bits_to_f32(uint16_t(yu[i] >> 16), p.dt), dot);
+          }
+        }
+      }
+    } else if (ok) {
       for (int64_t c = threadIdx.x; c < p.H; c += blockDim.x) {
         float gv = bits_to_f32(g[t * p.H + c], p.dt);
         if (dy) dy[(int64_t)r * p.H + c] = f32_to_bits(__fmul_rn(w, gv), p.dt);
@@ -167,14 +205,46 @@ struct SwigluBwdParams {
   uint16_t *dG, *dU;
   int dt;
   int64_t n;
+  int vec;  // all five tensors 16-byte aligned: 8 elements per access
 };
 
+// sigma = 1/(1+e^-G); dG = dh U sigma (1 + G (1 - sigma)), dU = dh G sigma, each
+// rounded once.  Fast exponential and division: few-ulp FP32 error, far below
+// one rounding of the 16-bit result.  8 elements per thread and access.
+__device__ __forceinline__ void swiglu_bwd1(float d, float g, float u, float &dg, float &du) {
+  const float s = __fdividef(1.f, 1.f + __expf(-g));
+  dg = d * u * s * (1.f + g * (1.f - s));
+  du = d * g * s;
+}
+
 __global__ void __launch_bounds__(256) swiglu_bwd_kernel(SwigluBwdParams p) {
-  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < p.n; i += (int64_t)gridDim.x * blockDim.x) {
-    float d = bits_to_f32(p.dh[i], p.dt), g = bits_to_f32(p.G[i], p.dt), u = bits_to_f32(p.U[i], p.dt);
-    float s = 1.f / (1.f + expf(-g));
-    p.dG[i] = f32_to_bits(d * u * s * (1.f + g * (1.f - s)), p.dt);
-    p.dU[i] = f32_to_bits(d * g * s, p.dt);
+  const int64_t n8 = p.vec ? p.n / 8 : 0;
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t v = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; v < n8; v += stride) {
+    const uint4 dv = reinterpret_cast<const uint4 *>(p.dh)[v];
+    const uint4 gv = reinterpret_cast<const uint4 *>(p.G)[v];
+    const uint4 uv = reinterpret_cast<const uint4 *>(p.U)[v];
+    const uint32_t da[4] = {dv.x, dv.y, dv.z, dv.w}, ga[4] = {gv.x, gv.y, gv.z, gv.w}, ua[4] = {uv.x, uv.y, uv.z, uv.w};
+    uint32_t og[4], ou[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      float dg0, du0, dg1, du1;
+      swiglu_bwd1(bits_to_f32(uint16_t(da[i] & 0xFFFF), p.dt), bits_to_f32(uint16_t(ga[i] & 0xFFFF), p.dt),
+                  bits_to_f32(uint16_t(ua[i] & 0xFFFF), p.dt), dg0, du0);
+      swiglu_bwd1(bits_to_f32(uint16_t(da[i] >> 16), p.dt), bits_to_f32(uint16_t(ga[i] >> 16), p.dt),
+                  bits_to_f32(uint16_t(ua[i] >> 16), p.dt), dg1, du1);
+      og[i] = uint32_t(f32_to_bits(dg0, p.dt)) | (uint32_t(f32_to_bits(dg1, p.dt)) << 16);
+      ou[i] = uint32_t(f32_to_bits(du0, p.dt)) | (uint32_t(f32_to_bits(du1, p.dt)) << 16);
+    }
+    reinterpret_cast<uint4 *>(p.dG)[v] = make_uint4(og[0], og[1], og[2], og[3]);
+    reinterpret_cast<uint4 *>(p.dU)[v] = make_uint4(ou[0], ou[1], ou[2], ou[3]);
+  }
+  // tail (n not a multiple of 8, or unaligned tensors)
+  for (int64_t i = n8 * 8 + (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < p.n; i += stride) {
+    float dg, du;
+    swiglu_bwd1(bits_to_f32(p.dh[i], p.dt), bits_to_f32(p.G[i], p.dt), bits_to_f32(p.U[i], p.dt), dg, du);
+    p.dG[i] = f32_to_bits(dg, p.dt);
+    p.dU[i] = f32_to_bits(du, p.dt);
   }
 }
 
@@ -239,7 +309,11 @@ extern "C" moe_status moe_combine_backward(const void *d_out, const void *y, moe
   if (!d_out || !weights || !row_of || (dweights && !y))
     return set_error(MOE_ERR_INVALID_ARGUMENT, "moe_combine_backward: NULL tensor pointer");
   CombineBwdParams p{d_out, y, (int)act_dtype, A, weights, row_of, T, H, top_k, dy, dweights, device_status};
-  combine_bwd_kernel<<<(unsigned)T, kCombThreads, 0, as_stream(stream)>>>(p);
+  const bool vec = H % 8 == 0 && aligned16(d_out) && (!dy || aligned16(dy)) && (!dweights || aligned16(y));
+  if (vec)
+    combine_bwd_kernel<true><<<(unsigned)T, kCombThreads, 0, as_stream(stream)>>>(p);
+  else
+    combine_bwd_kernel<false><<<(unsigned)T, kCombThreads, 0, as_stream(stream)>>>(p);
   return check_launch("moe_combine_backward");
 }
 
@@ -252,10 +326,12 @@ extern "C" moe_status moe_swiglu_backward(const void *dh, const void *G, const v
   if (!dh || !G || !U || !dG || !dU) return set_error(MOE_ERR_INVALID_ARGUMENT, "moe_swiglu_backward: NULL pointer");
   SwigluBwdParams p{static_cast<const uint16_t *>(dh), static_cast<const uint16_t *>(G),
                     static_cast<const uint16_t *>(U), static_cast<uint16_t *>(dG), static_cast<uint16_t *>(dU),
-                    (int)act_dtype, A * I};
-  int64_t blocks = (p.n + 255) / 256;
+                    (int)act_dtype, A * I, 0};
+  p.vec = aligned16(dh) && aligned16(G) && aligned16(U) && aligned16(dG) && aligned16(dU);
+  int64_t blocks = (p.n / (p.vec ? 8 : 1) + 255) / 256;
   int64_t cap = (int64_t)num_sms() * 8;
   if (blocks > cap) blocks = cap;
+  if (blocks < 1) blocks = 1;
   swiglu_bwd_kernel<<<(unsigned)blocks, 256, 0, as_stream(stream)>>>(p);
   return check_launch("moe_swiglu_backward");
 }

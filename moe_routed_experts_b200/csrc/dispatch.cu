@@ -79,6 +79,9 @@ struct RouteParams {
   int single;
 };
 
+// R > 0: the E <= 32 R candidate keys of a lane stay in registers across the
+// k selection rounds; R = 0 re-reads them each round (large E).
+template <int R>
 __global__ void __launch_bounds__(1024) route_rank_kernel(RouteParams p) {
   extern __shared__ int32_t sm[];
   int32_t *cnt = sm;                      // [E]
@@ -97,22 +100,51 @@ __global__ void __launch_bounds__(1024) route_rank_kernel(RouteParams p) {
     uint32_t prev_key = 0xFFFFFFFFu;
     int prev_e = -1;
     int my_e = 0;  // lane j keeps the j-th selection
-    for (int j = 0; j < k; ++j) {
-      uint32_t bk = 0u;
-      int be = 0x7FFFFFFF;
-      for (int e = lane; e < E; e += 32) {
-        const uint32_t key = score_key(l, p.sel_bias, e);
-        const bool after = key < prev_key || (key == prev_key && e > prev_e);
-        if (after && (key > bk || (key == bk && e < be))) {
-          bk = key;
-          be = e;
-        }
+    if (R > 0) {
+      // the lane's candidates (experts lane, lane + 32, ...) read once
+      uint32_t keys[R > 0 ? R : 1];
+#pragma unroll
+      for (int i = 0; i < R; ++i) {
+        const int e = lane + 32 * i;
+        keys[i] = e < E ? score_key(l, p.sel_bias, e) : 0u;
       }
-      const uint32_t wk = __reduce_max_sync(0xffffffffu, bk);
-      const int we = (int)__reduce_min_sync(0xffffffffu, (bk == wk) ? (uint32_t)be : 0x7FFFFFFFu);
-      prev_key = wk;
-      prev_e = we;
-      if (lane == j) my_e = we;
+      for (int j = 0; j < k; ++j) {
+        uint32_t bk = 0u;
+        int be = 0x7FFFFFFF;
+#pragma unroll
+        for (int i = 0; i < R; ++i) {
+          const int e = lane + 32 * i;
+          const uint32_t key = keys[i];
+          const bool after = key < prev_key || (key == prev_key && e > prev_e);
+          if (e < E && after && key > bk) {  // ascending e per lane: a tie keeps the lower ID
+            bk = key;
+            be = e;
+          }
+        }
+        const uint32_t wk = __reduce_max_sync(0xffffffffu, bk);
+        const int we = (int)__reduce_min_sync(0xffffffffu, (bk == wk) ? (uint32_t)be : 0x7FFFFFFFu);
+        prev_key = wk;
+        prev_e = we;
+        if (lane == j) my_e = we;
+      }
+    } else {
+      for (int j = 0; j < k; ++j) {
+        uint32_t bk = 0u;
+        int be = 0x7FFFFFFF;
+        for (int e = lane; e < E; e += 32) {
+          const uint32_t key = score_key(l, p.sel_bias, e);
+          const bool after = key < prev_key || (key == prev_key && e > prev_e);
+          if (after && (key > bk || (key == bk && e < be))) {
+            bk = key;
+            be = e;
+          }
+        }
+        const uint32_t wk = __reduce_max_sync(0xffffffffu, bk);
+        const int we = (int)__reduce_min_sync(0xffffffffu, (bk == wk) ? (uint32_t)be : 0x7FFFFFFFu);
+        prev_key = wk;
+        prev_e = we;
+        if (lane == j) my_e = we;
+      }
     }
     // weights from the unbiased logits
     float lj = (lane < k) ? l[my_e] : -INFINITY;
@@ -325,10 +357,13 @@ extern "C" moe_status moe_route_dispatch(const void *x, moe_dtype x_dtype, int64
   rp.single = lay.nchunks == 1;
   size_t smem = sizeof(int32_t) * (size_t)(E + 32) + sizeof(int16_t) * (size_t)(lay.chunk * top_k);
   smem = (smem + 15) & ~size_t(15);
-  if (smem > 48 * 1024) cudaFuncSetAttribute(route_rank_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  const int R = E <= 32 ? 1 : E <= 64 ? 2 : E <= 128 ? 4 : E <= 256 ? 8 : E <= 512 ? 16 : 0;
+  auto kern = R == 1 ? route_rank_kernel<1> : R == 2 ? route_rank_kernel<2> : R == 4 ? route_rank_kernel<4>
+            : R == 8 ? route_rank_kernel<8> : R == 16 ? route_rank_kernel<16> : route_rank_kernel<0>;
+  if (smem > 48 * 1024) cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   // a warp per token: small batches get a wider block
   const int threads = (T <= 32 && lay.nchunks == 1) ? 1024 : kRouteThreads;
-  route_rank_kernel<<<(unsigned)lay.nchunks, threads, smem, st>>>(rp);
+  kern<<<(unsigned)lay.nchunks, threads, smem, st>>>(rp);
   moe_status s = check_launch("moe_route_dispatch: route_rank_kernel");
   if (s != MOE_OK) return s;
   if (!rp.single) {

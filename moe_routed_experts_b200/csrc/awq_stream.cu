@@ -71,13 +71,18 @@ bool make_map_2d(CUtensorMap *map, const void *base, CUtensorMapDataType dt, int
 namespace stream {
 constexpr int kCW = 8;                    // consumer warps
 constexpr int kThreads = (kCW + 1) * 32;  // + one producer warp
-constexpr int kStages = 6;
-constexpr int kRows = 32;                 // input rows per stage (two 16-row MMA steps)
 constexpr int kBoxW = 32;                 // words per box row (128 bytes)
-constexpr int kBox = kRows * kBoxW * 4;   // [32 rows][32 words] = 4 KB
-constexpr int kStageBytes = 2 * kBox;     // two boxes per stage
 constexpr int kF = 512;                   // output columns of a unit
 constexpr int kBarBytes = 1024;           // barrier block; stages start 1024-byte aligned
+// A stage is ROWS input rows (ROWS / 16 MMA steps) of two [ROWS][32-word]
+// boxes; 64-row stages halve the per-stage bookkeeping per weight byte.
+template <int ROWS>
+struct Geo {
+  static constexpr int kRows = ROWS;
+  static constexpr int kBox = ROWS * kBoxW * 4;
+  static constexpr int kStageBytes = 2 * kBox;
+  static constexpr int kStages = ROWS == 64 ? 4 : 6;  // 64 KB / 48 KB in flight per CTA
+};
 }  // namespace stream
 
 // Largest e with pre[e] <= u (pre is the exclusive prefix of units per expert).
@@ -116,11 +121,14 @@ __device__ __forceinline__ UnitInfo unit_info(const int32_t *pre, const int32_t 
   return ui;
 }
 
-template <typename MT, int NPROJ, int NT>
+template <typename MT, int NPROJ, int NT, int ROWS>
 __global__ void __launch_bounds__(stream::kThreads, 2)
     awq_fwd_stream_kernel(const __grid_constant__ CUtensorMap map0, const __grid_constant__ CUtensorMap map1,
                           ProjParams p) {
   using namespace stream;
+  constexpr int kRows = Geo<ROWS>::kRows, kBox = Geo<ROWS>::kBox, kStageBytes = Geo<ROWS>::kStageBytes;
+  constexpr int kStages = Geo<ROWS>::kStages;
+  constexpr int kSteps = ROWS / 16;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // 128-byte-swizzled TMA boxes need 1024-byte aligned destinations
   uint8_t *smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
@@ -272,7 +280,7 @@ __global__ void __launch_bounds__(stream::kThreads, 2)
     }
     FwdConsts<MT> cst;
     bool x16 = false;
-    const int spg = p.group / kRows;  // stages per group (group % 32 == 0 on this path)
+    const int spg = p.group / kRows;  // stages per group (group % kRows == 0 on this path)
     int gstage = (int)((kbase % p.group) / kRows);
     for (int c = 0; c < nst; ++c, ++it) {
       const uint32_t s = it % kStages, ph = (it / kStages) & 1;
@@ -301,11 +309,16 @@ __global__ void __launch_bounds__(stream::kThreads, 2)
         ++grp;
       }
       if (mbar_wait(&full[s], ph, p.status)) {
-        const uint8_t *box = stages + s * kStageBytes + bw * kBox;
+        const uint8_t *box0 = stages + s * kStageBytes + bw * kBox;
+        // two 16-row steps at a time keep the register footprint of a 32-row stage
+#pragma unroll 1
+        for (int hh = 0; hh < kSteps; hh += 2) {
+        const uint8_t *box = box0 + (16 * hh) * 128;
+        const int xrow0 = kRows * c + 16 * hh;
         uint32_t w[2][4];
         uint32_t b0[2][NT], b1[2][NT];
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {  // two 16-row steps: rows 16h + {t, t+4, t+8, t+12}
+        for (int h = 0; h < 2; ++h) {  // 16-row steps: rows 16h + {t, t+4, t+8, t+12}
           w[h][0] = *reinterpret_cast<const uint32_t *>(box + woff0 + (16 * h) * 128);
           w[h][1] = *reinterpret_cast<const uint32_t *>(box + woff1 + (16 * h) * 128);
           w[h][2] = *reinterpret_cast<const uint32_t *>(box + woff0 + (16 * h + 8) * 128);
@@ -313,7 +326,7 @@ __global__ void __launch_bounds__(stream::kThreads, 2)
 #pragma unroll
           for (int nt = 0; nt < NT; ++nt) {
             const uint2 bv =
-                *reinterpret_cast<const uint2 *>(xs + (nt * 8 + g) * xs_pitch + (kRows * c + 16 * h + 4 * t) * 2);
+                *reinterpret_cast<const uint2 *>(xs + (nt * 8 + g) * xs_pitch + (xrow0 + 16 * h + 4 * t) * 2);
             b0[h][nt] = bv.x;
             b1[h][nt] = bv.y;
           }
@@ -346,6 +359,7 @@ __global__ void __launch_bounds__(stream::kThreads, 2)
 #pragma unroll
               for (int nt = 0; nt < NT; ++nt) mma16816<MT>(acc[nt][q], af[q], b0[h][nt], b1[h][nt]);
           }
+        }
         }
       }
       __syncwarp();
@@ -442,9 +456,11 @@ __global__ void __launch_bounds__(256) awq_stream_reduce_kernel(ProjParams p) {
 
 // ------------------------------------------------------------------ launch
 
-static size_t stream_smem(int nt, int64_t Kq, int64_t E) {
+static size_t stream_smem(int nt, int64_t Kq, int64_t E, int rows) {
   using namespace stream;
-  return 1024 /* alignment slack */ + kBarBytes + (size_t)kStages * kStageBytes + 2 * (size_t)8 * nt * Kq * 2 +
+  const size_t ring = rows == 64 ? (size_t)Geo<64>::kStages * Geo<64>::kStageBytes
+                                 : (size_t)Geo<32>::kStages * Geo<32>::kStageBytes;
+  return 1024 /* alignment slack */ + kBarBytes + ring + 2 * (size_t)8 * nt * Kq * 2 +
          (size_t)8 * nt * (Kq * 2 + 16) + (size_t)8 * nt * kF * 4 + (size_t)(2 * E + 1 + 32) * 4;
 }
 
@@ -453,16 +469,18 @@ static size_t stream_smem(int nt, int64_t Kq, int64_t E) {
 StreamPlan stream_plan(int64_t A, int64_t K, int64_t N, int64_t E, int64_t group, int nproj, int nt) {
   StreamPlan pl{};
   pl.fits = false;
-  // TMA needs 16-byte word-row pitches; a stage of 32 rows lies in one group
-  if (N % 32 != 0 || K % stream::kRows != 0 || group % stream::kRows != 0) return pl;
+  // TMA needs 16-byte word-row pitches; a stage lies inside one group
+  if (N % 32 != 0 || K % 32 != 0 || group % 32 != 0) return pl;
+  const int rows = (K % 64 == 0 && group % 64 == 0) ? 64 : 32;
   int kq = 1;
   for (int d = 8; d >= 2; d >>= 1)
-    if ((K / stream::kRows) % d == 0 && K / d >= 384) {
+    if ((K / rows) % d == 0 && K / d >= 384) {
       kq = d;
       break;
     }
   while (kq > 1 && (size_t)kq * A * nproj * N * 4 > ((size_t)256 << 20)) kq >>= 1;
-  if (stream_smem(nt, K / kq, E) > 200 * 1024) return pl;
+  if (stream_smem(nt, K / kq, E, rows) > 200 * 1024) return pl;
+  pl.rows = rows;
   pl.fits = true;
   pl.kq = kq;
   if (kq > 1) {
@@ -473,9 +491,10 @@ StreamPlan stream_plan(int64_t A, int64_t K, int64_t N, int64_t E, int64_t group
   return pl;
 }
 
-template <typename MT, int NPROJ, int NT>
-static moe_status launch_stream_t(const ProjParams &p, cudaStream_t st) {
+template <typename MT, int NPROJ, int NT, int ROWS>
+static moe_status launch_stream_r(const ProjParams &p, cudaStream_t st) {
   using namespace stream;
+  constexpr int kRows = Geo<ROWS>::kRows;
   CUtensorMap m0, m1;
   const uint64_t NW = p.N / 8, rows = (uint64_t)p.E * p.K;
   if (!make_map_2d(&m0, p.qw[0], CU_TENSOR_MAP_DATA_TYPE_INT32, 4, NW, rows, kBoxW, kRows,
@@ -483,8 +502,8 @@ static moe_status launch_stream_t(const ProjParams &p, cudaStream_t st) {
       !make_map_2d(&m1, p.qw[NPROJ - 1], CU_TENSOR_MAP_DATA_TYPE_INT32, 4, NW, rows, kBoxW, kRows,
                    CU_TENSOR_MAP_SWIZZLE_128B))
     return set_error(MOE_ERR_CUDA, "tensor map encoding failed for the packed words");
-  const size_t smem = stream_smem(NT, p.K / p.kq, p.E);
-  auto kern = awq_fwd_stream_kernel<MT, NPROJ, NT>;
+  const size_t smem = stream_smem(NT, p.K / p.kq, p.E, ROWS);
+  auto kern = awq_fwd_stream_kernel<MT, NPROJ, NT, ROWS>;
   cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   const int per_sm = smem <= 110 * 1024 ? 2 : 1;
   kern<<<num_sms() * per_sm, kThreads, smem, st>>>(m0, m1, p);
@@ -496,6 +515,11 @@ static moe_status launch_stream_t(const ProjParams &p, cudaStream_t st) {
   if (blocks > cap) blocks = cap;
   awq_stream_reduce_kernel<NPROJ><<<(unsigned)blocks, 256, 0, st>>>(p);
   return check_launch("awq_stream_reduce_kernel");
+}
+
+template <typename MT, int NPROJ, int NT>
+static moe_status launch_stream_t(const ProjParams &p, int rows, cudaStream_t st) {
+  return rows == 64 ? launch_stream_r<MT, NPROJ, NT, 64>(p, st) : launch_stream_r<MT, NPROJ, NT, 32>(p, st);
 }
 
 moe_status launch_fwd_stream(ProjParams p, int nproj, bool bf16_mma, int nt, void *ws, size_t ws_bytes,
@@ -510,12 +534,14 @@ moe_status launch_fwd_stream(ProjParams p, int nproj, bool bf16_mma, int nt, voi
                        pl.bytes);
     p.partials = reinterpret_cast<float *>(static_cast<char *>(ws) + pl.partial_off);
   }
+  const int r = pl.rows;
   if (bf16_mma) {
-    if (nproj == 2) return nt == 2 ? launch_stream_t<__nv_bfloat16, 2, 2>(p, st) : launch_stream_t<__nv_bfloat16, 2, 1>(p, st);
-    return nt == 2 ? launch_stream_t<__nv_bfloat16, 1, 2>(p, st) : launch_stream_t<__nv_bfloat16, 1, 1>(p, st);
+    if (nproj == 2)
+      return nt == 2 ? launch_stream_t<__nv_bfloat16, 2, 2>(p, r, st) : launch_stream_t<__nv_bfloat16, 2, 1>(p, r, st);
+    return nt == 2 ? launch_stream_t<__nv_bfloat16, 1, 2>(p, r, st) : launch_stream_t<__nv_bfloat16, 1, 1>(p, r, st);
   }
-  if (nproj == 2) return nt == 2 ? launch_stream_t<__half, 2, 2>(p, st) : launch_stream_t<__half, 2, 1>(p, st);
-  return nt == 2 ? launch_stream_t<__half, 1, 2>(p, st) : launch_stream_t<__half, 1, 1>(p, st);
+  if (nproj == 2) return nt == 2 ? launch_stream_t<__half, 2, 2>(p, r, st) : launch_stream_t<__half, 2, 1>(p, r, st);
+  return nt == 2 ? launch_stream_t<__half, 1, 2>(p, r, st) : launch_stream_t<__half, 1, 1>(p, r, st);
 }
 
 }  // namespace moe

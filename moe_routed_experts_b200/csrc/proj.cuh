@@ -124,6 +124,7 @@ void launch_dump(const int32_t *qw, const int32_t *qz, const uint16_t *sc, int64
                  uint16_t *out, int mode, bool bf16_mma, cudaStream_t st);
 struct StreamPlan {
   bool fits;      // the streaming tile can run this shape
+  int rows;       // input rows per pipeline stage (32 or 64)
   int kq;         // K splits across CTAs
   size_t bytes;   // workspace bytes (partials + counters)
   size_t partial_off, counter_off;

@@ -4,7 +4,7 @@
 One step = one pass of the whole hot path over one batch of synthetic input:
 route + COPY dispatch -> gate/up + SwiGLU -> down -> combine (and, for a
 workload with a backward, the combine VJP -> down input VJP -> SwiGLU VJP ->
-gate/up input VJP -> COPY VJP).  Inputs are resident in HBM when the timed
+gate/up input VJP -> COPY VJP -> router-logit VJP).  Inputs are resident in HBM when the timed
 region starts; 256 MiB of L2-flushing writes separate the timed steps
 (outside the per-step CUDA events).  Multi-GPU runs are replicas (weak
 scaling): every rank runs its own copy of the workload, no collective on the
@@ -386,7 +386,7 @@ def gate_up_kernel_name(B, w):
 
 def launches_per_step_of(B, w):
     """Kernel launches of one step: route (2, or 3 past one token chunk), each
-    projection (1, or 2 with the split-K reduce), combine, and the backward's five."""
+    projection (1, or 2 with the split-K reduce), combine, and the backward's six."""
     n = 2 if w.T <= 64 else 3
     if _path_of(w) == 1:
         n += 1 + (B.projection_workspace_size(w.A, w.H, w.I, w.E, w.group, 2) > 0)
@@ -395,7 +395,7 @@ def launches_per_step_of(B, w):
         n += 2
     n += 1
     if w.backward:
-        n += 5
+        n += 6
     return n
 
 

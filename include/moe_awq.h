@@ -303,6 +303,27 @@ MOE_API moe_status moe_dispatch_backward(const void *dvalues, moe_dtype act_dtyp
                                  int32_t *device_status, void *stream);
 
 /* ------------------------------------------------------------------------
+ * moe_router_backward -- [MX] MoeDispatchOps::moe_dispatch_weights_backward
+ * (the logit VJP of the FP32 routing weights at a fixed selection; the
+ * selection bias, used only to choose experts, gets no gradient).
+ *  logits     [T, E] f32   the router logits the forward routed with
+ *  selected   [T, top_k]   u32 global expert IDs (moe_route_dispatch output)
+ *  d_weights  [T, top_k]   f32 upstream gradient of the weights
+ *  d_logits   [T, E] f32   output, every element written:
+ *    renormalize = 1: w = softmax of the selected logits,
+ *      d_logits[t, e_j] = w_j (d_weights[t, j] - sum_i w_i d_weights[t, i]),
+ *      0 for experts not selected;
+ *    renormalize = 0: p = softmax over all E logits, for every e
+ *      d_logits[t, e] = p_e (sum_j [e == e_j] d_weights[t, j] - sum_j p_{e_j} d_weights[t, j]).
+ *  FP32 arithmetic.  Device errors: MOE_DEVICE_ERR_EXPERT_RANGE (an ID
+ *  outside [expert_start, expert_start + E); that selection is skipped).
+ * ---------------------------------------------------------------------- */
+MOE_API moe_status moe_router_backward(const float *logits, const uint32_t *selected_experts,
+                                       const float *d_weights, int64_t T, int64_t E, int32_t top_k,
+                                       int32_t renormalize, int32_t expert_start, float *d_logits,
+                                       int32_t *device_status, void *stream);
+
+/* ------------------------------------------------------------------------
  * awq_dequant_coefficients -- the coefficients W[kk, n] of ONE expert's
  * payload ([K, N/8] words, [K/group, N/8] zero words, [K/group, N] scales),
  * formed by the same device code the projection kernels run, written out in

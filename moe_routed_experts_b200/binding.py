@@ -54,6 +54,7 @@ _SIGS = {
     "awq_input_backward": (C.c_int, [P, C.c_int, I64, I64, I64, P, I64, P, P, P, C.c_int, I64, P, P, P, P, P, P, P]),
     "moe_swiglu_backward": (C.c_int, [P, P, P, C.c_int, I64, I64, P, P, P]),
     "moe_dispatch_backward": (C.c_int, [P, C.c_int, I64, P, P, I64, I64, I32, P, P, P]),
+    "moe_router_backward": (C.c_int, [P, P, P, I64, I64, I32, I32, I32, P, P, P]),
     "awq_dequant_coefficients": (C.c_int, [P, P, P, C.c_int, I64, I64, I64, I32, P, P]),
     "moe_set_projection_path": (I32, [I32]),
 }
@@ -267,6 +268,16 @@ def moe_dispatch_backward(dvalues, row_of, selected_experts, device_status=None)
                                      H, k, _ptr(dx), _ptr(device_status), _stream())
     _check("moe_dispatch_backward", st)
     return dx
+
+
+def moe_router_backward(logits, selected_experts, d_weights, renormalize=1, expert_start=0, device_status=None):
+    T, E = logits.shape
+    k = selected_experts.shape[1]
+    dl = torch.empty((T, E), dtype=torch.float32, device=logits.device)
+    st = lib().moe_router_backward(_ptr(logits), _ptr(selected_experts), _ptr(d_weights), T, E, k, int(renormalize),
+                                   int(expert_start), _ptr(dl), _ptr(device_status), _stream())
+    _check("moe_router_backward", st)
+    return dl
 
 
 def awq_dequant_coefficients(qweight, qzeros, scales, group, pairing=0):

@@ -294,6 +294,77 @@ __global__ void __launch_bounds__(256) route_scatter_kernel(ScatterParams p) {
   }
 }
 
+// Router-logit VJP at a fixed selection (one warp per token).
+struct RouterBwdParams {
+  const float *logits;
+  const uint32_t *selected;
+  const float *dw;
+  int64_t T;
+  int E, k, renorm;
+  uint32_t expert_start;
+  float *dl;
+  int32_t *status;
+};
+
+__global__ void __launch_bounds__(256) router_bwd_kernel(RouterBwdParams p) {
+  const int lane = threadIdx.x & 31;
+  const int64_t t = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  if (t >= p.T) return;
+  const float *l = p.logits + t * p.E;
+  float *dl = p.dl + t * p.E;
+  const int E = p.E, k = p.k;
+  // lane j < k holds selection j
+  int ej = -1;
+  float lj = -INFINITY, dwj = 0.f;
+  if (lane < k) {
+    const uint32_t id = p.selected[t * k + lane];
+    if (id >= p.expert_start && id - p.expert_start < (uint32_t)E) {
+      ej = (int)(id - p.expert_start);
+      lj = l[ej];
+      dwj = p.dw[t * k + lane];
+    } else {
+      report(p.status, MOE_DEVICE_ERR_EXPERT_RANGE);
+    }
+  }
+  float m, den;
+  if (p.renorm) {
+    m = lj;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    den = ej >= 0 ? expf(lj - m) : 0.f;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+  } else {
+    m = -INFINITY;
+    for (int e = lane; e < E; e += 32) m = fmaxf(m, l[e]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    den = 0.f;
+    for (int e = lane; e < E; e += 32) den += expf(l[e] - m);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+  }
+  const float wj = ej >= 0 ? expf(lj - m) / den : 0.f;
+  float dot = wj * dwj;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+  if (p.renorm) {
+    for (int e = lane; e < E; e += 32) dl[e] = 0.f;
+    __syncwarp();
+    if (ej >= 0) dl[ej] = wj * (dwj - dot);
+  } else {
+    for (int e = lane; e < E; e += 32) {
+      float seed = 0.f;  // d_weights of the selection that chose e, if any
+      for (int j = 0; j < k; ++j) {
+        const int ejj = __shfl_sync(0xffffffffu, ej, j);
+        const float dwjj = __shfl_sync(0xffffffffu, dwj, j);
+        if (ejj == e) seed = dwjj;
+      }
+      dl[e] = expf(l[e] - m) / den * (seed - dot);
+    }
+  }
+}
+
 }  // namespace moe
 
 using namespace moe;
@@ -463,4 +534,21 @@ extern "C" moe_status moe_route_dispatch_noalloc(const void *x, moe_dtype x_dtyp
   return moe_route_dispatch(x, x_dtype, T, H, logits, sel_bias, E, expert_start, top_k, renormalize, values,
                             weights, selected_experts, row_experts, offsets, src_token, row_of, scratch,
                             kStaticRouteScratchBytes, device_status, stream);
+}
+
+extern "C" moe_status moe_router_backward(const float *logits, const uint32_t *selected_experts,
+                                          const float *d_weights, int64_t T, int64_t E, int32_t top_k,
+                                          int32_t renormalize, int32_t expert_start, float *d_logits,
+                                          int32_t *device_status, void *stream) {
+  if (T < 0 || E < 1 || E > MOE_MAX_EXPERTS || top_k < 1 || top_k > MOE_MAX_TOP_K || top_k > E || expert_start < 0)
+    return set_error(MOE_ERR_INVALID_ARGUMENT, "moe_router_backward: bad sizes T=%lld E=%lld top_k=%d",
+                     (long long)T, (long long)E, top_k);
+  if (T == 0) return MOE_OK;
+  if (!logits || !selected_experts || !d_weights || !d_logits)
+    return set_error(MOE_ERR_INVALID_ARGUMENT, "moe_router_backward: NULL tensor pointer");
+  RouterBwdParams p{logits, selected_experts, d_weights, T, (int)E, top_k, renormalize ? 1 : 0,
+                    (uint32_t)expert_start, d_logits, device_status};
+  const int64_t blocks = (T * 32 + 255) / 256;
+  router_bwd_kernel<<<(unsigned)blocks, 256, 0, as_stream(stream)>>>(p);
+  return check_launch("moe_router_backward");
 }

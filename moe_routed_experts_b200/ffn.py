@@ -3,8 +3,9 @@
 ``forward`` = moe_route_dispatch -> awq_grouped_gate_up_swiglu ->
 awq_grouped_down -> moe_combine; ``backward`` = moe_combine_backward ->
 awq_input_backward(down) -> moe_swiglu_backward -> awq_input_backward(gate
-+ up, one accumulation) -> moe_dispatch_backward.  Only argument
-marshalling happens here; every step runs in the library's kernels.
++ up, one accumulation) -> moe_dispatch_backward, and moe_router_backward
+for the router logits.  Only argument marshalling happens here; every step
+runs in the library's kernels.
 """
 from dataclasses import dataclass
 from typing import Optional
@@ -121,4 +122,7 @@ def backward(dev: dict, buf: Buffers, d_out: torch.Tensor) -> dict:
     dvalues = B.awq_input_backward(dG, r["offsets"], dev["gate"], w.group, grad2=dU, proj2=dev["up"],
                                    device_status=buf.status)
     dx = B.moe_dispatch_backward(dvalues, r["row_of"], r["selected_experts"], device_status=buf.status)
-    return {"dy": dy, "dweights": dw, "dh": dh, "dG": dG, "dU": dU, "dvalues": dvalues, "dx": dx}
+    dlogits = B.moe_router_backward(dev["logits"], r["selected_experts"], dw, renormalize=w.renormalize,
+                                    expert_start=w.expert_start, device_status=buf.status)
+    return {"dy": dy, "dweights": dw, "dh": dh, "dG": dG, "dU": dU, "dvalues": dvalues, "dx": dx,
+            "dlogits": dlogits}

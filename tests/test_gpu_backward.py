@@ -61,8 +61,38 @@ def _chain(name, kw, rows=None, tokens=None):
     check_close(dv[rows], o_dv, name + "/dvalues")
     o_dx = oracle.dispatch_backward(dv, "bf16", sel[tokens], row_of[tokens])
     check_close(dx[tokens], o_dx, name + "/dx")
+    # router-logit VJP from the device dweights (FP32 softmax algebra)
+    dl = g["dlogits"].cpu().numpy()
+    o_dl = oracle.router_backward(inp["logits"][tokens], sel[tokens], dw[tokens], renormalize=w.renormalize,
+                                  expert_start=w.expert_start)
+    assert np.max(np.abs(dl[tokens] - o_dl)) <= ROUTER_TOL * max(1.0, float(np.max(np.abs(dw[tokens])))), "dlogits"
     assert int(buf.status.item()) == 0
     return w, offsets
+
+
+# d_logits = w (dw - <w, dw>) in FP32: a few ulps of max|dw| (weights <= 1)
+ROUTER_TOL = 1e-5
+
+
+@pytest.mark.parametrize("renorm", [1, 0])
+@pytest.mark.parametrize("E,k", [(8, 2), (64, 6), (512, 10), (4096, 32)])
+def test_router_backward_against_oracle(renorm, E, k):
+    rng = np.random.default_rng(E + k)
+    T = 37
+    logits = (rng.standard_normal((T, E)) * 1.5).astype(np.float32)
+    sel, _ = oracle.route(logits, None, k, renormalize=renorm, expert_start=3)
+    dw = rng.standard_normal((T, k)).astype(np.float32)
+    o_dl = oracle.router_backward(logits, sel, dw, renormalize=renorm, expert_start=3)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    dl = B.moe_router_backward(torch.from_numpy(logits).cuda(), torch.from_numpy(sel.view(np.int32)).cuda(),
+                               torch.from_numpy(dw).cuda(), renormalize=renorm, expert_start=3, device_status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    assert np.max(np.abs(dl.cpu().numpy() - o_dl)) <= ROUTER_TOL * max(1.0, float(np.max(np.abs(dw))))
+    if renorm:  # unselected experts get exactly zero
+        mask = np.ones((T, E), bool)
+        np.put_along_axis(mask, (sel.astype(np.int64) - 3), False, axis=1)
+        assert np.all(dl.cpu().numpy()[mask] == 0)
 
 
 SMALL = {"skewed": dict(T=1024, H=512, I=256, E=16), "prefill": dict(T=512, H=256, I=128, E=16, backward=True),

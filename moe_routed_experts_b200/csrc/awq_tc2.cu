@@ -41,16 +41,18 @@ namespace tc2 {
 constexpr int kBM = 128;   // rows per CTA (256 per pair)
 constexpr int kBN = 256;   // accumulator columns
 constexpr int kHalf = 128; // B columns held by each CTA
-constexpr int kBK = 64;
-constexpr int kLStages = 6, kBStages = 4;
+constexpr int kBK = 128;   // K per pipeline stage: two 64-element swizzle atoms
+constexpr int kLStages = 3, kBStages = 3;
 constexpr int kDqWarps = 16, kEpWarps = 4;
 constexpr int kThreads = (2 + kDqWarps + kEpWarps) * 32;  // 704
 constexpr int kRowGroups = kDqWarps * 2;                   // 16 word columns x kRowGroups threads
 constexpr int kWordsPerThread = kBK / kRowGroups;          // rows rg, rg + kRowGroups, ...
-constexpr int kABytes = kBM * kBK * 2;        // 16 KB
-constexpr int kPBytes = kBK * (kHalf / 8) * 4;  // 4 KB packed words
+constexpr int kAtom = kBM * 64 * 2;          // 16 KB: 128 rows x 64 K (128B swizzle)
+constexpr int kABytes = kBM * kBK * 2;        // 32 KB
+constexpr int kPBytes = kBK * (kHalf / 8) * 4;  // 8 KB packed words
 constexpr int kLBytes = kABytes + kPBytes;    // one TMA stage
-constexpr int kBBytes = kHalf * kBK * 2;      // 16 KB coefficient half-tile
+constexpr int kBBytes = kHalf * kBK * 2;      // 32 KB coefficient half-tile
+constexpr int kNBlock = kBK * 128;            // bytes between 64-column blocks of B (MN-major)
 constexpr int kTmemCols = 512;
 }  // namespace tc2
 
@@ -160,6 +162,7 @@ __global__ void __launch_bounds__(tc2::kThreads, 1)
           uint8_t *st = lring + s * kLBytes;
           mbar_arrive_expect_tx(&lfull[s], kLBytes);
           tma_load_2d(st, &map_x, &lfull[s], kb * kBK, row0);
+          tma_load_2d(st + kAtom, &map_x, &lfull[s], kb * kBK + 64, row0);
           tma_load_2d(st + kABytes, mw, &lfull[s], wcol, (int32_t)(ti.e * K + (int64_t)kb * kBK));
         }
       }
@@ -182,11 +185,12 @@ __global__ void __launch_bounds__(tc2::kThreads, 1)
           // both CTAs' dequant warps arrive only after their own TMA stage landed
           tc_wait_cluster(&bready[bs], (it / kBStages) & 1, p.status, abort);
           tc_fence_after();
-          const uint64_t adesc = smem_desc(smem_u32(lring + ls * kLBytes), 16, 1024);
-          const uint64_t bdesc = smem_desc(smem_u32(bring + bs * kBBytes), 8192, 1024);
+          const uint32_t a_addr = smem_u32(lring + ls * kLBytes);
+          const uint64_t bdesc = smem_desc(smem_u32(bring + bs * kBBytes), kNBlock, 1024);
 #pragma unroll
-          for (int j = 0; j < kBK / 16; ++j)
-            umma2_f16(dacc, adesc + (uint64_t)(2 * j), bdesc + (uint64_t)(128 * j), idesc, (kb | j) != 0);
+          for (int j = 0; j < kBK / 16; ++j)  // K steps of 16: atom j / 4, 32 bytes each inside it
+            umma2_f16(dacc, smem_desc(a_addr + (j >> 2) * kAtom, 16, 1024) + (uint64_t)(2 * (j & 3)),
+                      bdesc + (uint64_t)(128 * j), idesc, (kb | j) != 0);
           umma2_commit_both(&lempty[ls]);
           umma2_commit_both(&bfree[bs]);
         }
@@ -206,7 +210,7 @@ __global__ void __launch_bounds__(tc2::kThreads, 1)
     const int pk0 = rg * 16 + col;
     // features col*8 .. col*8+7 of the half -> 64-column block col/8, 16-byte
     // chunk col%8 XOR row%8 (MN-major, 128-byte swizzle, 8-row x 64-column atoms)
-    const int b0 = (col >> 3) * 8192 + (rg >> 3) * 1024 + (rg & 7) * 128 + (((col & 7) ^ (rg & 7)) << 4);
+    const int b0 = (col >> 3) * kNBlock + (rg >> 3) * 1024 + (rg & 7) * 128 + (((col & 7) ^ (rg & 7)) << 4);
     const int spg = p.group / kBK;
     const bool convert = p.act_dt != (std::is_same<MT, __half>::value ? MOE_F16 : MOE_BF16);
     uint64_t *bready0 = bready;  // CTA 0's barriers, addressed through the cluster window
@@ -351,7 +355,7 @@ static moe_status launch_tc2_t(const ProjParams &p, cudaStream_t st) {
   using namespace tc2;
   CUtensorMap mx, m0, m1;
   const uint64_t NW = p.N / 8, rows = (uint64_t)p.E * p.K;
-  if (!make_map_2d(&mx, p.x, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, p.K, p.A, kBK, kBM, CU_TENSOR_MAP_SWIZZLE_128B) ||
+  if (!make_map_2d(&mx, p.x, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, p.K, p.A, 64, kBM, CU_TENSOR_MAP_SWIZZLE_128B) ||
       !make_map_2d(&m0, p.qw[0], CU_TENSOR_MAP_DATA_TYPE_INT32, 4, NW, rows, 16, kBK, CU_TENSOR_MAP_SWIZZLE_NONE) ||
       !make_map_2d(&m1, p.qw[NPROJ - 1], CU_TENSOR_MAP_DATA_TYPE_INT32, 4, NW, rows, 16, kBK,
                    CU_TENSOR_MAP_SWIZZLE_NONE))

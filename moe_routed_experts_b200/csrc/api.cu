@@ -251,7 +251,9 @@ extern "C" moe_status awq_input_backward(const void *grad, moe_dtype grad_dtype,
   cudaStream_t st = as_stream(stream);
   const bool bf = scale_dtype == MOE_BF16;
   const int nproj = grad2 ? 2 : 1;
-  if (choose_path(A, E) >= 2 && tc_bwd_fits(p)) return launch_bwd_tc(p, nproj, bf, st);
+  const int path = choose_path(A, E);
+  if (path == 3 && tc2_bwd_fits(p)) return launch_bwd_tc2(p, nproj, bf, st);
+  if (path >= 2 && tc_bwd_fits(p)) return launch_bwd_tc(p, nproj, bf, st);
   launch_bwd_mma(p, nproj, bf, A >= 12 * E ? 2 : 1, st);
   return check_launch(fn);
 }

@@ -138,6 +138,8 @@ bool tc_bwd_fits(const BwdParams &p);
 moe_status launch_fwd_tc(const ProjParams &p, int nproj, bool bf16_mma, cudaStream_t st);
 moe_status launch_bwd_tc(const BwdParams &p, int nproj, bool bf16_mma, cudaStream_t st);
 bool tc2_fits(const ProjParams &p);
+bool tc2_bwd_fits(const BwdParams &p);
+moe_status launch_bwd_tc2(const BwdParams &p, int nproj, bool bf16_mma, cudaStream_t st);
 moe_status launch_fwd_tc2(const ProjParams &p, int nproj, bool bf16_mma, cudaStream_t st);
 
 }  // namespace moe

@@ -98,12 +98,14 @@ def test_router_backward_against_oracle(renorm, E, k):
 SMALL = {"skewed": dict(T=1024, H=512, I=256, E=16), "prefill": dict(T=512, H=256, I=128, E=16, backward=True),
          "decode": dict(backward=True), "tiny": dict(backward=True),
          # output widths that end inside a 256-column tile, four zero/scale groups per tile
-         "ragged": dict(T=512, H=320, I=192, E=8, group=64)}
+         "ragged": dict(T=512, H=320, I=192, E=8, group=64),
+         # pair-tile input VJP with an output width ending mid-tile and two group rows per CTA
+         "ragged_pair": dict(T=512, H=384, I=256, E=8, group=64)}
 
 
 @pytest.mark.parametrize("name", list(SMALL))
 def test_backward_chain_every_row(name, path):
-    _chain("skewed" if name == "ragged" else name, SMALL[name])
+    _chain("skewed" if name.startswith("ragged") else name, SMALL[name])
 
 
 def test_backward_full_size_skewed_sampled(path):

@@ -22,9 +22,10 @@
 //           with 128-byte swizzle (8-row x 64-column atoms); when the
 //           activations are not in the scale dtype they also convert the
 //           activation tile in place;
-//   warps 10-13 (one per TMEM lane quarter) read a finished accumulator
-//           (tcgen05.ld 32x32b), add the bias, round, apply SwiGLU and store,
-//           while the tensor core fills the other of the two TMEM buffers.
+//   warps 10-17 (two per TMEM lane quarter, one per column half) read a
+//           finished accumulator (tcgen05.ld 32x32b), add the bias, round,
+//           apply SwiGLU and store, while the tensor core fills the other of
+//           the two TMEM buffers.
 // Coefficients are exact per the operation: RNE_scale((q - z) s) formed with
 // the magic-number conversion (see common.cuh), never written to HBM.
 #include <cudaTypedefs.h>
@@ -40,8 +41,8 @@ namespace tc {
 constexpr int kBM = 128, kBN = 256, kBK = 64;
 constexpr int kStages = 3;
 constexpr int kDqWarps = 8;
-constexpr int kEpWarps = 4;                                // one per TMEM lane quarter
-constexpr int kThreads = (2 + kDqWarps + kEpWarps) * 32;  // 448
+constexpr int kEpWarps = 8;                                // two per TMEM lane quarter (column halves)
+constexpr int kThreads = (2 + kDqWarps + kEpWarps) * 32;  // 576
 constexpr int kABytes = kBM * kBK * 2;          // 16 KB activation tile
 constexpr int kBBytes = kBN * kBK * 2;          // 32 KB coefficient tile
 constexpr int kPBytes = kBK * (kBN / 8) * 4;    // 8 KB packed words
@@ -273,7 +274,8 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
     }
   } else {
     // ---------------- epilogue warps: TMEM -> registers -> bias, rounding, SwiGLU -> HBM
-    const int q = warp & 3;  // TMEM lane quarter of this warp
+    const int q = warp & 3;                          // TMEM lane quarter of this warp
+    const int hf = (warp - 2 - kDqWarps) >> 2;       // column half drained by this warp
     uint32_t tcount = 0;
     for (int64_t tile = blockIdx.x; tile < total; tile += gridDim.x, ++tcount) {
       const TileInfo ti = tile_info(tile);
@@ -286,20 +288,20 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
       const uint32_t tbase = tmem + ((uint32_t)(32 * q) << 16) + buf * kBN;
       if (NPROJ == 2) {
 #pragma unroll 1
-        for (int c4 = 0; c4 < 4; ++c4) {
-          const int f0 = c4 * 32;  // feature within the tile
-          float gv[32], uv[32];
-          tmem_ld32(tbase + f0, gv);
-          tmem_ld32(tbase + 128 + f0, uv);
+        for (int c8 = 4 * hf; c8 < 4 * hf + 4; ++c8) {
+          const int f0 = c8 * 16;  // feature within the tile
+          float gv[16], uv[16];
+          tmem_ld16(tbase + f0, gv);
+          tmem_ld16(tbase + 128 + f0, uv);
           const int64_t n0 = (int64_t)ti.nt * 128 + f0;
           if (row_ok && n0 < p.N) {
 #pragma unroll
-            for (int v8 = 0; v8 < 4; ++v8) finish8<2>(p, ti.e, row, n0 + 8 * v8, gv + 8 * v8, uv + 8 * v8);
+            for (int v8 = 0; v8 < 2; ++v8) finish8<2>(p, ti.e, row, n0 + 8 * v8, gv + 8 * v8, uv + 8 * v8);
           }
         }
       } else {
 #pragma unroll 1
-        for (int c8 = 0; c8 < 8; ++c8) {
+        for (int c8 = 4 * hf; c8 < 4 * hf + 4; ++c8) {
           const int f0 = c8 * 32;
           float yv[32];
           tmem_ld32(tbase + f0, yv);

@@ -23,10 +23,10 @@
 //   D: rows 128 r .. of the tile, all 256 columns, in CTA r's TMEM.
 // Warp roles in each CTA: warp 0 TMA producer (activations + this CTA's
 // packed words, 6-stage ring); warp 1 TMEM allocation, and in CTA 0 lane 0
-// issues the pair MMAs; warps 2-17 dequantize this CTA's B half (two words
-// per thread and step) into a 4-stage coefficient ring and signal CTA 0;
-// warps 18-21 drain this CTA's accumulator (two TMEM buffers, so draining
-// overlaps the next tile).
+// issues the pair MMAs; warps 2-9 dequantize this CTA's B half (eight words
+// per thread and step) into a 3-stage coefficient ring and signal CTA 0;
+// warps 10-17 (two per TMEM lane quarter, one per column half) drain this
+// CTA's accumulator (two TMEM buffers, so draining overlaps the next tile).
 // Every wait is bounded.  CTA 1's dequant and epilogue warps arrive on CTA
 // 0's barriers through the cluster shared-memory window.
 #include <cudaTypedefs.h>
@@ -43,8 +43,8 @@ constexpr int kBN = 256;   // accumulator columns
 constexpr int kHalf = 128; // B columns held by each CTA
 constexpr int kBK = 128;   // K per pipeline stage: two 64-element swizzle atoms
 constexpr int kLStages = 3, kBStages = 3;
-constexpr int kDqWarps = 16, kEpWarps = 4;
-constexpr int kThreads = (2 + kDqWarps + kEpWarps) * 32;  // 704
+constexpr int kDqWarps = 8, kEpWarps = 8;
+constexpr int kThreads = (2 + kDqWarps + kEpWarps) * 32;  // 576
 constexpr int kRowGroups = kDqWarps * 2;                   // 16 word columns x kRowGroups threads
 constexpr int kWordsPerThread = kBK / kRowGroups;          // rows rg, rg + kRowGroups, ...
 constexpr int kAtom = kBM * 64 * 2;          // 16 KB: 128 rows x 64 K (128B swizzle)
@@ -286,7 +286,8 @@ __global__ void __launch_bounds__(tc2::kThreads, 1)
     }
   } else {
     // ---------------- epilogue warps: this CTA's 128 rows of the tile
-    const int q = warp & 3;
+    const int q = warp & 3;                     // TMEM lane quarter
+    const int hf = (warp - 2 - kDqWarps) >> 2;  // column half drained by this warp
     uint32_t tcount = 0;
     for (int64_t tile = pair; tile < total; tile += npairs, ++tcount) {
       const PairTile ti = tile_info(tile);
@@ -299,7 +300,7 @@ __global__ void __launch_bounds__(tc2::kThreads, 1)
       const uint32_t tbase = tmem + ((uint32_t)(32 * q) << 16) + buf * kBN;
       if (NPROJ == 2) {
 #pragma unroll 1
-        for (int c8 = 0; c8 < 8; ++c8) {
+        for (int c8 = 4 * hf; c8 < 4 * hf + 4; ++c8) {
           const int f0 = c8 * 16;
           float gv[16], uv[16];
           tmem_ld16(tbase + f0, gv);
@@ -312,7 +313,7 @@ __global__ void __launch_bounds__(tc2::kThreads, 1)
         }
       } else {
 #pragma unroll 1
-        for (int c16 = 0; c16 < 16; ++c16) {
+        for (int c16 = 8 * hf; c16 < 8 * hf + 8; ++c16) {
           const int f0 = c16 * 16;
           float yv[16];
           tmem_ld16(tbase + f0, yv);

@@ -18,7 +18,8 @@
 // output columns, in lane i of CTA r's TMEM.  Warp roles and barriers follow
 // the forward pair tile: warp 0 TMA producer (gradient, packed words, and
 // the zero/scale rows of the step), warp 1 TMEM + (CTA 0) MMA issue, warps
-// 2-17 dequantize, warps 18-21 drain the double-buffered accumulator.
+// 2-17 dequantize, warps 18-25 (two per TMEM lane quarter) drain the
+// double-buffered accumulator.
 #include <cudaTypedefs.h>
 
 #include "dequant.cuh"
@@ -33,8 +34,8 @@ constexpr int kBN = 256;   // output columns per pair tile
 constexpr int kHalf = 128; // output columns formed by each CTA
 constexpr int kBK = 128;   // reduction per stage (16 words)
 constexpr int kLStages = 3, kBStages = 3;
-constexpr int kDqWarps = 16, kEpWarps = 4;
-constexpr int kThreads = (2 + kDqWarps + kEpWarps) * 32;  // 704
+constexpr int kDqWarps = 16, kEpWarps = 8;
+constexpr int kThreads = (2 + kDqWarps + kEpWarps) * 32;  // 832
 constexpr int kAtom = kBM * 64 * 2;                       // 16 KB: 128 rows x 64 (128B swizzle)
 constexpr int kABytes = kBM * kBK * 2;                    // 32 KB gradient tile
 constexpr int kPBytes = kHalf * (kBK / 8) * 4;            // 8 KB packed words (128 rows x 16 words)
@@ -261,7 +262,8 @@ __global__ void __launch_bounds__(tc2b::kThreads, 1)
     }
   } else {
     // ---------------- epilogue warps: this CTA's 128 rows, 256 output columns
-    const int q = warp & 3;
+    const int q = warp & 3;                     // TMEM lane quarter
+    const int hf = (warp - 2 - kDqWarps) >> 2;  // column half drained by this warp
     const bool bf = p.gdt == MOE_BF16;
     uint32_t tcount = 0;
     for (int64_t tile = pair; tile < total; tile += npairs, ++tcount) {
@@ -274,7 +276,7 @@ __global__ void __launch_bounds__(tc2b::kThreads, 1)
       const int64_t row = ti.r0 + trow;
       const uint32_t tbase = tmem + ((uint32_t)(32 * q) << 16) + buf * kBN;
 #pragma unroll 1
-      for (int c16 = 0; c16 < kBN / 16; ++c16) {
+      for (int c16 = 8 * hf; c16 < 8 * hf + 8; ++c16) {
         float v[16];
         tmem_ld16(tbase + c16 * 16, v);
         const int64_t kk = (int64_t)ti.ct * kBN + c16 * 16;

@@ -17,8 +17,9 @@
 // second (grad, payload).  Warp roles as in the forward tile: warp 0 TMA
 // producer (gradient tile, packed words, and the zero/scale rows of the
 // step, 3-stage ring); warp 1 TMEM allocation + single-thread MMA issue;
-// warps 2-9 dequantize; warps 10-13 drain a double-buffered TMEM
-// accumulator, round once to the gradient dtype and store.
+// warps 2-9 dequantize; warps 10-17 (two per TMEM lane quarter) drain a
+// double-buffered TMEM accumulator, round once to the gradient dtype and
+// store.
 #include <cudaTypedefs.h>
 
 #include "dequant.cuh"
@@ -30,8 +31,8 @@ namespace moe {
 namespace tcb {
 constexpr int kBM = 128, kBN = 256, kBK = 64;
 constexpr int kStages = 3;
-constexpr int kDqWarps = 8, kEpWarps = 4;
-constexpr int kThreads = (2 + kDqWarps + kEpWarps) * 32;  // 448
+constexpr int kDqWarps = 8, kEpWarps = 8;
+constexpr int kThreads = (2 + kDqWarps + kEpWarps) * 32;  // 576
 constexpr int kABytes = kBM * kBK * 2;     // 16 KB gradient tile
 constexpr int kBBytes = kBN * kBK * 2;     // 32 KB coefficient tile (256 rows x 128 B)
 constexpr int kPBytes = kBN * (kBK / 8) * 4;  // 8 KB packed words (256 rows x 8 words)
@@ -251,7 +252,8 @@ __global__ void __launch_bounds__(tcb::kThreads, 1)
     }
   } else {
     // ---------------- epilogue warps
-    const int q = warp & 3;
+    const int q = warp & 3;                     // TMEM lane quarter
+    const int hf = (warp - 2 - kDqWarps) >> 2;  // column half drained by this warp
     const bool bf = p.gdt == MOE_BF16;
     uint32_t tcount = 0;
     for (int64_t tile = blockIdx.x; tile < total; tile += gridDim.x, ++tcount) {
@@ -264,7 +266,7 @@ __global__ void __launch_bounds__(tcb::kThreads, 1)
       const int64_t row = ti.r0 + trow;
       const uint32_t tbase = tmem + ((uint32_t)(32 * q) << 16) + buf * kBN;
 #pragma unroll 1
-      for (int c16 = 0; c16 < kBN / 16; ++c16) {
+      for (int c16 = 8 * hf; c16 < 8 * hf + 8; ++c16) {
         float v[16];
         tmem_ld16(tbase + c16 * 16, v);
         const int64_t kk = (int64_t)ti.ct * kBN + c16 * 16;

@@ -75,13 +75,14 @@ constexpr int kBoxW = 32;                 // words per box row (128 bytes)
 constexpr int kF = 512;                   // output columns of a unit
 constexpr int kBarBytes = 1024;           // barrier block; stages start 1024-byte aligned
 // A stage is ROWS input rows (ROWS / 16 MMA steps) of two [ROWS][32-word]
-// boxes; 64-row stages halve the per-stage bookkeeping per weight byte.
+// boxes; deeper stages spread the per-stage bookkeeping over more weight
+// bytes (a 128-row stage is 32 KB, so two of them keep 64 KB in flight).
 template <int ROWS>
 struct Geo {
   static constexpr int kRows = ROWS;
   static constexpr int kBox = ROWS * kBoxW * 4;
   static constexpr int kStageBytes = 2 * kBox;
-  static constexpr int kStages = ROWS == 64 ? 4 : 6;  // 64 KB / 48 KB in flight per CTA
+  static constexpr int kStages = ROWS == 128 ? 2 : ROWS == 64 ? 4 : 6;  // 64 / 64 / 48 KB in flight per CTA
 };
 }  // namespace stream
 
@@ -458,8 +459,9 @@ __global__ void __launch_bounds__(256) awq_stream_reduce_kernel(ProjParams p) {
 
 static size_t stream_smem(int nt, int64_t Kq, int64_t E, int rows) {
   using namespace stream;
-  const size_t ring = rows == 64 ? (size_t)Geo<64>::kStages * Geo<64>::kStageBytes
-                                 : (size_t)Geo<32>::kStages * Geo<32>::kStageBytes;
+  const size_t ring = rows == 128  ? (size_t)Geo<128>::kStages * Geo<128>::kStageBytes
+                     : rows == 64 ? (size_t)Geo<64>::kStages * Geo<64>::kStageBytes
+                                  : (size_t)Geo<32>::kStages * Geo<32>::kStageBytes;
   return 1024 /* alignment slack */ + kBarBytes + ring + 2 * (size_t)8 * nt * Kq * 2 +
          (size_t)8 * nt * (Kq * 2 + 16) + (size_t)8 * nt * kF * 4 + (size_t)(2 * E + 1 + 32) * 4;
 }
@@ -471,7 +473,7 @@ StreamPlan stream_plan(int64_t A, int64_t K, int64_t N, int64_t E, int64_t group
   pl.fits = false;
   // TMA needs 16-byte word-row pitches; a stage lies inside one group
   if (N % 32 != 0 || K % 32 != 0 || group % 32 != 0) return pl;
-  const int rows = (K % 64 == 0 && group % 64 == 0) ? 64 : 32;
+  const int rows = (K % 128 == 0 && group % 128 == 0) ? 128 : (K % 64 == 0 && group % 64 == 0) ? 64 : 32;
   int kq = 1;
   for (int d = 8; d >= 2; d >>= 1)
     if ((K / rows) % d == 0 && K / d >= 384) {
@@ -519,6 +521,7 @@ static moe_status launch_stream_r(const ProjParams &p, cudaStream_t st) {
 
 template <typename MT, int NPROJ, int NT>
 static moe_status launch_stream_t(const ProjParams &p, int rows, cudaStream_t st) {
+  if (rows == 128) return launch_stream_r<MT, NPROJ, NT, 128>(p, st);
   return rows == 64 ? launch_stream_r<MT, NPROJ, NT, 64>(p, st) : launch_stream_r<MT, NPROJ, NT, 32>(p, st);
 }
 

@@ -203,11 +203,7 @@ extern "C" moe_status awq_grouped_down(const void *input, moe_dtype act_dtype, i
   cudaStream_t st = as_stream(stream);
   const bool bf = scale_dtype == MOE_BF16;
   moe_status ts;
-  // a single projection gains from the CTA pair only on very long batches
-  // (its reduction is the short side, so ragged 256-row tiles cost more)
-  int path = choose_path(A, E);
-  if (path == 3 && g_path.load() != 3 && A < 1024 * E) path = 2;
-  if (try_fwd_tc(path, p, 1, bf, st, &ts)) return ts;
+  if (try_fwd_tc(choose_path(A, E), p, 1, bf, st, &ts)) return ts;
   const int nt = small_tile_tokens(A, E);
   if (stream_plan(A, K, N, E, group_size, 1, nt).fits) return launch_fwd_stream(p, 1, bf, nt, workspace, workspace_bytes, st);
   launch_fwd_mma(p, 1, bf, nt, st);

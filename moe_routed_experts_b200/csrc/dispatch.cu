@@ -432,8 +432,8 @@ extern "C" moe_status moe_route_dispatch(const void *x, moe_dtype x_dtype, int64
   auto kern = R == 1 ? route_rank_kernel<1> : R == 2 ? route_rank_kernel<2> : R == 4 ? route_rank_kernel<4>
             : R == 8 ? route_rank_kernel<8> : R == 16 ? route_rank_kernel<16> : route_rank_kernel<0>;
   if (smem > 48 * 1024) cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  // a warp per token: small batches get a wider block
-  const int threads = (T <= 32 && lay.nchunks == 1) ? 1024 : kRouteThreads;
+  // a warp per token (or per few tokens): the widest block the kernel takes
+  const int threads = 1024;
   kern<<<(unsigned)lay.nchunks, threads, smem, st>>>(rp);
   moe_status s = check_launch("moe_route_dispatch: route_rank_kernel");
   if (s != MOE_OK) return s;

@@ -259,38 +259,58 @@ struct ScatterParams {
   int64_t nseg;  // copy segments per row
 };
 
-// One warp per (assignment, 512-byte segment), grid-stride.
+// Row position of assignment a = t*k + j and, on its first visit, the row maps.
+__device__ __forceinline__ int64_t scatter_pos(const ScatterParams &p, int64_t a, bool write_maps) {
+  const int64_t t = a / p.k;
+  const int e = (int)(p.selected[a] - p.expert_start);
+  const int64_t c = t / p.chunk;
+  const int64_t pos = (int64_t)p.offsets[e] + p.chunk_base[c * p.E + e] + p.rank[a];
+  if (write_maps) {
+    p.row_of[a] = (int32_t)pos;
+    p.row_experts[pos] = p.expert_start + (uint32_t)e;
+    p.src_token[pos] = (int32_t)t;
+  }
+  return pos;
+}
+
+// 16-byte rows: one warp per assignment (grid-stride), four 512-byte
+// segments loaded before they are stored.  Otherwise one warp per
+// (assignment, 64-byte segment) with 2-byte accesses.
 __global__ void __launch_bounds__(256) route_scatter_kernel(ScatterParams p) {
   const int lane = threadIdx.x & 31;
   const int64_t wid = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int64_t nw = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  if (p.vec16) {
+    const int64_t n16 = p.row_bytes / 16;
+    for (int64_t a = wid; a < p.A; a += nw) {
+      int64_t pos = 0;
+      if (lane == 0) pos = scatter_pos(p, a, true);
+      pos = __shfl_sync(0xffffffffu, pos, 0);
+      const uint4 *src = reinterpret_cast<const uint4 *>(p.x + (a / p.k) * p.row_bytes);
+      uint4 *dst = reinterpret_cast<uint4 *>(p.values + pos * p.row_bytes);
+      for (int64_t i0 = lane; i0 < n16; i0 += 32 * 4) {
+        uint4 v[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          if (i0 + 32 * j < n16) v[j] = __ldg(src + i0 + 32 * j);
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          if (i0 + 32 * j < n16) dst[i0 + 32 * j] = v[j];
+      }
+    }
+    return;
+  }
   const int64_t units = p.A * p.nseg;
   for (int64_t u = wid; u < units; u += nw) {
     const int64_t a = u / p.nseg, s = u % p.nseg;
-    const int64_t t = a / p.k;
     int64_t pos = 0;
-    if (lane == 0) {
-      const int e = (int)(p.selected[a] - p.expert_start);
-      const int64_t c = t / p.chunk;
-      pos = (int64_t)p.offsets[e] + p.chunk_base[c * p.E + e] + p.rank[a];
-      if (s == 0) {
-        p.row_of[a] = (int32_t)pos;
-        p.row_experts[pos] = p.expert_start + (uint32_t)e;
-        p.src_token[pos] = (int32_t)t;
-      }
-    }
+    if (lane == 0) pos = scatter_pos(p, a, s == 0);
     pos = __shfl_sync(0xffffffffu, pos, 0);
-    const uint8_t *src = p.x + t * p.row_bytes;
+    const uint8_t *src = p.x + (a / p.k) * p.row_bytes;
     uint8_t *dst = p.values + pos * p.row_bytes;
-    if (p.vec16) {
-      const int64_t off = s * 512 + lane * 16;
-      if (off < p.row_bytes)
-        *reinterpret_cast<uint4 *>(dst + off) = __ldg(reinterpret_cast<const uint4 *>(src + off));
-    } else {
-      const int64_t off = s * 64 + lane * 2;
-      if (off < p.row_bytes)
-        *reinterpret_cast<uint16_t *>(dst + off) = *reinterpret_cast<const uint16_t *>(src + off);
-    }
+    const int64_t off = s * 64 + lane * 2;
+    if (off < p.row_bytes)
+      *reinterpret_cast<uint16_t *>(dst + off) = *reinterpret_cast<const uint16_t *>(src + off);
   }
 }
 
@@ -463,9 +483,8 @@ extern "C" moe_status moe_route_dispatch(const void *x, moe_dtype x_dtype, int64
   sp.row_experts = row_experts;
   sp.src_token = src_token;
   sp.vec16 = aligned16(x) && aligned16(values) && (sp.row_bytes % 16 == 0);
-  const int64_t seg = sp.vec16 ? 512 : 64;
-  sp.nseg = (sp.row_bytes + seg - 1) / seg;
-  int64_t units = sp.A * sp.nseg;
+  sp.nseg = (sp.row_bytes + 63) / 64;  // 2-byte path only
+  int64_t units = sp.vec16 ? sp.A : sp.A * sp.nseg;
   int64_t blocks = (units + 7) / 8;
   int64_t cap = (int64_t)num_sms() * 16;
   if (blocks > cap) blocks = cap;

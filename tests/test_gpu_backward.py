@@ -135,3 +135,9 @@ def test_whole_chain_against_oracle_chain():
     o_dx = oracle.dispatch_backward(o_dv, "bf16", f["selected"], f["row_of"])
     check_close(bits(g["dx"]), o_dx, "chain/dx")
     check_close(bits(g["dvalues"]), o_dv, "chain/dvalues")
+
+
+@pytest.mark.parametrize("group", [256, 512])
+def test_backward_chain_large_groups(group, path):
+    # zero/scale groups spanning two or four 128-deep steps of the tcgen05 tiles
+    _chain("skewed", dict(T=300, H=1024, I=512, E=8, group=group))

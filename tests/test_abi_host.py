@@ -107,3 +107,22 @@ def test_projection_path_knob(L):
     assert L.moe_set_projection_path(3) == 1
     assert L.moe_set_projection_path(1) == 3
     assert L.moe_set_projection_path(prev) == 1
+
+
+def test_router_backward_rejects_bad_arguments(L):
+    # (logits, selected, d_weights, T, E, top_k, renormalize, expert_start, d_logits, status, stream)
+    assert L.moe_router_backward(FAKE, FAKE, FAKE, 4, 8, 0, 1, 0, FAKE, None, None) == 1      # top_k < 1
+    assert L.moe_router_backward(FAKE, FAKE, FAKE, 4, 8, 9, 1, 0, FAKE, None, None) == 1      # top_k > E
+    assert L.moe_router_backward(FAKE, FAKE, FAKE, 4, 64, 33, 1, 0, FAKE, None, None) == 1    # above 32 lanes
+    assert L.moe_router_backward(FAKE, FAKE, FAKE, 4, 0, 1, 1, 0, FAKE, None, None) == 1      # E < 1
+    assert L.moe_router_backward(FAKE, FAKE, FAKE, 4, 8, 2, 1, -1, FAKE, None, None) == 1     # expert_start
+    assert L.moe_router_backward(FAKE, None, FAKE, 4, 8, 2, 1, 0, FAKE, None, None) == 1      # NULL tensor
+    assert L.moe_router_backward(FAKE, FAKE, FAKE, 0, 8, 2, 1, 0, FAKE, None, None) == 0      # nothing to do
+
+
+def test_projection_path_knob_accepts_every_path(L):
+    prev = L.moe_set_projection_path(0)
+    for path in (1, 2, 3, 0):
+        L.moe_set_projection_path(path)
+    assert L.moe_set_projection_path(4) == -1
+    L.moe_set_projection_path(prev)

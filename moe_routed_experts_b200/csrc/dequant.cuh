@@ -21,11 +21,13 @@ struct FwdConsts {
     const uint32_t sw[4] = {sv.x, sv.y, sv.z, sv.w};
 #pragma unroll
     for (int p = 0; p < 4; ++p) {
-      const uint32_t f = (x16 && (p & 1)) ? 16u : 1u;
-      zlo[p] = ((((zw >> (4 * p)) & 0xFu) * f) * 0x10001u) | M;       // slot p   -> column 2p
-      zhi[p] = ((((zw >> (4 * p + 16)) & 0xFu) * f) * 0x10001u) | M;  // slot p+4 -> column 2p+1
-      slo[p] = (sw[p] & 0xFFFFu) * 0x10001u;                            // s[2p]
-      shi[p] = (sw[p] >> 16) * 0x10001u;                                // s[2p+1]
+      // slots p (column 2p) and p+4 (column 2p+1) in the low/high halves
+      uint32_t t = (zw >> (4 * p)) & 0x000F000Fu;
+      if (x16 && (p & 1)) t <<= 4;
+      zlo[p] = prmt(t, 0u, 0x1010u) | M;  // (z[2p], z[2p]) under the magic
+      zhi[p] = prmt(t, 0u, 0x3232u) | M;  // (z[2p+1], z[2p+1])
+      slo[p] = prmt(sw[p], 0u, 0x1010u);  // (s[2p], s[2p])
+      shi[p] = prmt(sw[p], 0u, 0x3232u);  // (s[2p+1], s[2p+1])
     }
   }
 };

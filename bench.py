@@ -98,6 +98,17 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
+def max_over_ranks(values, device):
+    """Element-wise max of per-rank timings (every rank gets the result); the
+    job is as slow as its slowest replica."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
 def run_reference(args, w):
     """CPU oracle on the host cores: each step is a bounded sample of the workload."""
     if int(os.environ.get("RANK", "0")) != 0:
@@ -296,10 +307,7 @@ def main():
     clocks = sampler.stop()
     status = int(buf.status.item())
 
-    t = torch.tensor([ms, e2e_ms, kernel_ms], dtype=torch.float64, device="cuda")
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms, e2e_ms, kernel_ms = t.tolist()
+    ms, e2e_ms, kernel_ms = max_over_ranks([ms, e2e_ms, kernel_ms], "cuda")
 
     if rank == 0:
         offsets = buf.route["offsets"].cpu().numpy()

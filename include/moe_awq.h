@@ -190,8 +190,10 @@ MOE_API moe_status moe_route_dispatch_noalloc(const void *x, moe_dtype x_dtype, 
  *  h        [A, I]   act_dtype: RNE(silu(G) * U), silu(v) = v / (1 + e^-v)
  *  gate_out [A, I]   act_dtype G = RNE(sum_kk values*Wg + bias_g), or NULL
  *  up_out   [A, I]   act_dtype U = RNE(sum_kk values*Wu + bias_u), or NULL
- * The GPU path (small per-expert batches on warp-level tensor-core tiles,
- * large ones on tcgen05/TMEM tiles) is chosen inside from A and E.
+ * The tile path is chosen inside from A and E (see moe_set_projection_path):
+ * small per-expert batches on warp-level tensor-core tiles that stream the
+ * packed words, mid-size ones on 128-row tcgen05/TMEM tiles, long ones on
+ * 256-row tcgen05 tiles over a CTA pair.
  *  workspace  device scratch of awq_projection_workspace_size(A, H, I, E, group_size, 2)
  *             bytes (16-byte aligned; may be NULL when that size is 0):
  *             split-K partial sums of the small-batch tiles.  Its contents
@@ -271,6 +273,9 @@ MOE_API moe_status moe_combine_backward(const void *d_out, const void *y, moe_dt
  *  grad2  [A, N] or NULL, with a second payload (qweight2, qzeros2, scales2)
  *  dinput[r, kk] = RNE(sum_n grad[r,n] W[e,kk,n] + sum_n grad2[r,n] W2[e,kk,n])
  *  ([A, K], grad_dtype; the two sums share one accumulator and one rounding)
+ * Tile paths as for the forward projections (warp-level, 128-row tcgen05,
+ * 256-row CTA-pair tcgen05); the tensor-core products run in the scale
+ * dtype, gradients converted to it when they differ.
  * Device errors: MOE_DEVICE_ERR_OFFSETS.
  * ---------------------------------------------------------------------- */
 MOE_API moe_status awq_input_backward(const void *grad, moe_dtype grad_dtype, int64_t A, int64_t N,

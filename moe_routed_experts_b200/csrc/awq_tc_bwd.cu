@@ -37,7 +37,6 @@ constexpr int kABytes = kBM * kBK * 2;     // 16 KB gradient tile
 constexpr int kBBytes = kBN * kBK * 2;     // 32 KB coefficient tile (256 rows x 128 B)
 constexpr int kPBytes = kBN * (kBK / 8) * 4;  // 8 KB packed words (256 rows x 8 words)
 constexpr int kZBytes = 4 * 8 * 4;         // zero words: up to 4 group rows x 8 words
-constexpr int kSBytes = 4 * kBK * 2;       // scales: up to 4 group rows x 64
 constexpr int kCBytes = 1024;              // zero + scale region (padded)
 constexpr int kStageBytes = kABytes + kBBytes + kPBytes + kCBytes;
 constexpr int kTmemCols = 512;

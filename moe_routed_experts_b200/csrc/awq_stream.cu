@@ -474,9 +474,12 @@ StreamPlan stream_plan(int64_t A, int64_t K, int64_t N, int64_t E, int64_t group
   // TMA needs 16-byte word-row pitches; a stage lies inside one group
   if (N % 32 != 0 || K % 32 != 0 || group % 32 != 0) return pl;
   const int rows = (K % 128 == 0 && group % 128 == 0) ? 128 : (K % 64 == 0 && group % 64 == 0) ? 64 : 32;
+  // K splits: 4 when each split keeps >= 256 input rows (whole stages),
+  // else 3 or 2 (a split count that leaves about five units per CTA evens
+  // out the tail of the persistent grid better than fewer, longer units)
   int kq = 1;
-  for (int d = 8; d >= 2; d >>= 1)
-    if ((K / rows) % d == 0 && K / d >= 384) {
+  for (int d : {4, 3, 2})
+    if ((K / rows) % d == 0 && K / d >= 256) {
       kq = d;
       break;
     }

@@ -22,7 +22,9 @@ _lib = None
 def lib():
     global _lib
     if _lib is None:
-        _lib = C.CDLL(_build_library())
+        # ORACLE_LIB: a planted-mistake build for the mutant test (tests only)
+        path = os.environ.get("ORACLE_LIB") or _build_library()
+        _lib = C.CDLL(path)
         _declare(_lib)
     return _lib
 

@@ -22,5 +22,13 @@ def build(force: bool = False) -> str:
     return LIB
 
 
+def build_mutant(mutant: int, out_dir: str) -> str:
+    """A copy of the oracle with one known mistake planted (ORACLE_MUTANT);
+    for the test that shows the pins catch it.  Never used elsewhere."""
+    lib = os.path.join(out_dir, "libmoe_oracle_mutant%d.so" % mutant)
+    subprocess.check_call(["gcc", *CFLAGS, "-DORACLE_MUTANT=%d" % mutant, "-o", lib, SRC, "-lm"])
+    return lib
+
+
 if __name__ == "__main__":
     print(build(force=True))

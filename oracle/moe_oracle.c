@@ -48,6 +48,10 @@
  * 2 = BF16, 3 = FP64 (exact-math chaining of the tests; never rounded).
  * 16-bit tensors are passed as their bit patterns (uint16).
  *
+ * ORACLE_MUTANT (a compile-time switch used only by tests/test_oracle_mutants.py;
+ * 0 in every other build) plants one known mistake in one step, so that the
+ * test can show that the pins below catch it.
+ *
  * Parity pins: tests/test_oracle_pins.py (hand-worked words and
  * coefficients), tests/test_oracle_bruteforce.py (independent NumPy
  * dequantize-then-matmul), tests/test_oracle_invariants.py (routing and
@@ -55,6 +59,10 @@
  */
 #include <math.h>
 #include <stdint.h>
+
+#ifndef ORACLE_MUTANT
+#define ORACLE_MUTANT 0
+#endif
 #include <stdlib.h>
 #include <string.h>
 
@@ -178,7 +186,8 @@ static const int PACK_ORDER[8] = {0, 2, 4, 6, 1, 3, 5, 7};
 
 /* codes[j] = code of logical column 8w+j.  The word is read as unsigned. */
 void oracle_unpack_word(uint32_t word, int32_t codes[8]) {
-    for (int s = 0; s < 8; ++s) codes[PACK_ORDER[s]] = (int32_t)((word >> (4 * s)) & 0xFu);
+    for (int s = 0; s < 8; ++s)
+        codes[ORACLE_MUTANT == 1 ? s : PACK_ORDER[s]] = (int32_t)((word >> (4 * s)) & 0xFu);
 }
 
 uint32_t oracle_pack_word(const int32_t codes[8]) {
@@ -192,6 +201,7 @@ double oracle_coefficient(int32_t q, int32_t z, uint32_t scale_bits, int sdt, ui
     double s = oracle_decode(scale_bits, sdt);
     double exact = (double)(q - z) * s;      /* |q-z| <= 15: exact in double */
     double w = oracle_round(exact, sdt);
+    if (ORACLE_MUTANT == 2) w = oracle_round(oracle_round(q * s, sdt) - oracle_round(z * s, sdt), sdt);
     if (bits) *bits = oracle_encode(w, sdt);
     return w;
 }
@@ -204,10 +214,11 @@ void oracle_dequant(const int32_t *qw, const int32_t *qz, const void *sc, int sd
 #pragma omp parallel for schedule(static)
     for (int64_t kk = 0; kk < K; ++kk) {
         int64_t grp = kk / g;
+        int64_t zgrp = (ORACLE_MUTANT == 3 && grp + 1 < K / g) ? grp + 1 : grp;
         for (int64_t w = 0; w < NW; ++w) {
             int32_t qc[8], zc[8];
             oracle_unpack_word((uint32_t)qw[kk * NW + w], qc);
-            oracle_unpack_word((uint32_t)qz[grp * NW + w], zc);
+            oracle_unpack_word((uint32_t)qz[zgrp * NW + w], zc);
             for (int j = 0; j < 8; ++j) {
                 int64_t n = 8 * w + j;
                 uint32_t sb = (sdt == DT_F32) ? 0u : ((const uint16_t *)sc)[grp * N + n];
@@ -244,18 +255,20 @@ int oracle_route(const float *logits, const float *sel_bias, int64_t T, int64_t 
                 if (taken[e]) continue;
                 float s = sel_bias ? (float)(l[e] + sel_bias[e]) : l[e];
                 /* strictly greater keeps the lower ID on ties */
-                if (best < 0 || s > bs) { best = e; bs = s; }
+                if (best < 0 || s > bs || (ORACLE_MUTANT == 4 && s == bs)) { best = e; bs = s; }
             }
             taken[best] = 1;
             sel[j] = best;
             selected[t * k + j] = expert_start + (uint32_t)best;
         }
         if (renormalize) {
-            double m = -INFINITY, den = 0.0;
-            for (int32_t j = 0; j < k; ++j) m = fmax(m, (double)l[sel[j]]);
-            for (int32_t j = 0; j < k; ++j) den += exp((double)l[sel[j]] - m);
+            double m = -INFINITY, den = 0.0, lb[64];
             for (int32_t j = 0; j < k; ++j)
-                weights[t * k + j] = (float)(exp((double)l[sel[j]] - m) / den);
+                lb[j] = (double)l[sel[j]] + ((ORACLE_MUTANT == 5 && sel_bias) ? (double)sel_bias[sel[j]] : 0.0);
+            for (int32_t j = 0; j < k; ++j) m = fmax(m, lb[j]);
+            for (int32_t j = 0; j < k; ++j) den += exp(lb[j] - m);
+            for (int32_t j = 0; j < k; ++j)
+                weights[t * k + j] = (float)(exp(lb[j] - m) / den);
         } else {
             double m = -INFINITY, den = 0.0;
             for (int64_t e = 0; e < E; ++e) m = fmax(m, (double)l[e]);
@@ -288,7 +301,8 @@ int oracle_dispatch(const uint32_t *selected, int64_t T, int32_t k, int64_t E,
     int64_t *next = (int64_t *)malloc(sizeof(int64_t) * (size_t)E);
     for (int64_t e = 0; e < E; ++e) next[e] = offsets[e];
     /* tokens in ascending order: each expert's rows ascend by token */
-    for (int64_t t = 0; t < T; ++t) {
+    for (int64_t tt = 0; tt < T; ++tt) {
+        int64_t t = ORACLE_MUTANT == 6 ? T - 1 - tt : tt;
         for (int32_t j = 0; j < k; ++j) {
             int64_t e = (int64_t)selected[t * k + j] - (int64_t)expert_start;
             int64_t r = next[e]++;
@@ -350,7 +364,7 @@ int oracle_project(const void *x, int xdt, int64_t R, int64_t K, int64_t N,
                 for (int64_t n = 0; n < N; ++n) acc[n] += xv * Wr[n];
             }
             for (int64_t n = 0; n < N; ++n) {
-                double v = acc[n] + (be ? load_val(be, bdt, n) : 0.0);
+                double v = acc[n] + ((be && ORACLE_MUTANT != 7) ? load_val(be, bdt, n) : 0.0);
                 if (mode == 1) ((double *)out)[r * N + n] = v;
                 else store_val(out, odt, r * N + n, v);
             }
@@ -366,7 +380,9 @@ void oracle_swiglu(const void *G, const void *U, int dt, int64_t n, void *h) {
 #pragma omp parallel for schedule(static)
     for (int64_t i = 0; i < n; ++i) {
         double gv = load_val(G, dt, i), uv = load_val(U, dt, i);
-        store_val(h, dt, i, gv / (1.0 + exp(-gv)) * uv);
+        double silu = gv / (1.0 + exp(-gv));
+        if (ORACLE_MUTANT == 8) silu = 1.0 / (1.0 + exp(-gv));
+        store_val(h, dt, i, silu * uv);
     }
 }
 
@@ -391,7 +407,8 @@ void oracle_combine(const void *y, int dt, const float *weights, const uint32_t 
             double acc = 0.0;
             for (int32_t i = 0; i < k; ++i) {
                 int32_t j = order[i];
-                acc += (double)weights[t * k + j] * load_val(y, dt, (int64_t)row_of[t * k + j] * H + c);
+                acc += (ORACLE_MUTANT == 10 ? 1.0 : (double)weights[t * k + j]) *
+                       load_val(y, dt, (int64_t)row_of[t * k + j] * H + c);
             }
             store_val(out, dt, t * H + c, acc);
         }
@@ -412,7 +429,7 @@ void oracle_combine_backward(const void *d_out, const void *y, int dt, const flo
             for (int64_t c = 0; c < H; ++c) {
                 double g = load_val(d_out, dt, t * H + c);
                 if (dy) store_val(dy, dt, r * H + c, w * g);
-                dot += g * load_val(y, dt, r * H + c);
+                dot += g * (ORACLE_MUTANT == 13 ? g : load_val(y, dt, r * H + c));
             }
             if (dweights) dweights[t * k + j] = (float)dot;
         }
@@ -449,7 +466,7 @@ int oracle_input_backward(const void *grad, int gdt, int64_t R, int64_t N, int64
             for (int64_t kk = 0; kk < K; ++kk) {
                 double acc = 0.0;
                 for (int64_t n = 0; n < N; ++n) acc += load_val(grad, gdt, r * N + n) * W[kk * N + n];
-                if (W2)
+                if (W2 && ORACLE_MUTANT != 9)
                     for (int64_t n = 0; n < N; ++n) acc += load_val(grad2, gdt, r * N + n) * W2[kk * N + n];
                 if (mode == 1) ((double *)out)[r * K + kk] = acc;
                 else store_val(out, odt, r * K + kk, acc);
@@ -469,7 +486,7 @@ void oracle_swiglu_backward(const void *dh, const void *G, const void *U, int dt
     for (int64_t i = 0; i < n; ++i) {
         double d = load_val(dh, dt, i), gv = load_val(G, dt, i), uv = load_val(U, dt, i);
         double s = 1.0 / (1.0 + exp(-gv));
-        store_val(dG, dt, i, d * uv * s * (1.0 + gv * (1.0 - s)));
+        store_val(dG, dt, i, d * uv * s * (ORACLE_MUTANT == 11 ? 1.0 : (1.0 + gv * (1.0 - s))));
         store_val(dU, dt, i, d * gv * s);
     }
 }
@@ -516,7 +533,7 @@ void oracle_router_backward(const float *logits, const uint32_t *selected, const
             for (int32_t j = 0; j < k; ++j) {
                 int64_t e = selected[t * k + j] - expert_start;
                 double w = exp((double)l[e] - m) / den;
-                dl[e] = w * ((double)d_weights[t * k + j] - dot);
+                dl[e] = w * ((double)d_weights[t * k + j] - (ORACLE_MUTANT == 12 ? 0.0 : dot));
             }
         } else {
             for (int64_t e = 0; e < E; ++e) m = fmax(m, (double)l[e]);

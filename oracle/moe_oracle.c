@@ -262,13 +262,15 @@ int oracle_route(const float *logits, const float *sel_bias, int64_t T, int64_t 
             selected[t * k + j] = expert_start + (uint32_t)best;
         }
         if (renormalize) {
-            double m = -INFINITY, den = 0.0, lb[64];
+            double m = -INFINITY, den = 0.0;
+            double *lb = (double *)malloc(sizeof(double) * (size_t)k);
             for (int32_t j = 0; j < k; ++j)
                 lb[j] = (double)l[sel[j]] + ((ORACLE_MUTANT == 5 && sel_bias) ? (double)sel_bias[sel[j]] : 0.0);
             for (int32_t j = 0; j < k; ++j) m = fmax(m, lb[j]);
             for (int32_t j = 0; j < k; ++j) den += exp(lb[j] - m);
             for (int32_t j = 0; j < k; ++j)
                 weights[t * k + j] = (float)(exp(lb[j] - m) / den);
+            free(lb);
         } else {
             double m = -INFINITY, den = 0.0;
             for (int64_t e = 0; e < E; ++e) m = fmax(m, (double)l[e]);

@@ -16,8 +16,9 @@
 // input rows.  Persistent CTAs (1 producer warp + 8 consumer warps) take
 // contiguous ranges of the expert-major unit list.
 //   producer: per unit, 1-D bulk copies of the tile's activation rows
-//     (double-buffered), then per 32 input rows one stage = two TMA boxes of
-//     [32 rows][32 words] with 128-byte swizzle (8 KB), kStages in flight.
+//     (double-buffered), then per ROWS input rows (32, 64 or 128, the
+//     largest the group size allows) one stage = two TMA boxes of
+//     [ROWS rows][32 words] with 128-byte swizzle, 48-64 KB in flight.
 //   consumer warp w: box w/4, word columns (w%4)*8 .. +7 of it, all rows of
 //     the unit.  Lane (g, t) reads rows t, t+4, t+8, t+12 of column g (the
 //     MMA's K index {2t, 2t+1, 2t+8, 2t+9} stands for them); the swizzle

@@ -56,14 +56,14 @@ def _declare(L):
     L.oracle_project.restype = C.c_int
     L.oracle_project.argtypes = [P, C.c_int, I64, I64, I64, P, I64, P, P, P, C.c_int, P, C.c_int,
                                  I64, C.c_int, P, C.c_int]
-    L.oracle_swiglu.argtypes = [P, P, C.c_int, I64, P]
-    L.oracle_combine.argtypes = [P, C.c_int, P, P, P, I64, I64, I32, P]
-    L.oracle_combine_backward.argtypes = [P, P, C.c_int, P, P, I64, I64, I32, P, P]
+    L.oracle_swiglu.argtypes = [P, P, C.c_int, I64, P, C.c_int]
+    L.oracle_combine.argtypes = [P, C.c_int, P, P, P, I64, I64, I32, P, C.c_int]
+    L.oracle_combine_backward.argtypes = [P, P, C.c_int, P, P, I64, I64, I32, P, P, C.c_int]
     L.oracle_input_backward.restype = C.c_int
     L.oracle_input_backward.argtypes = [P, C.c_int, I64, I64, I64, P, I64, P, P, P, C.c_int, I64,
                                         P, P, P, P, C.c_int, P, C.c_int]
-    L.oracle_swiglu_backward.argtypes = [P, P, P, C.c_int, I64, P, P]
-    L.oracle_dispatch_backward.argtypes = [P, C.c_int, P, P, I64, I64, I32, P]
+    L.oracle_swiglu_backward.argtypes = [P, P, P, C.c_int, I64, P, P, C.c_int]
+    L.oracle_dispatch_backward.argtypes = [P, C.c_int, P, P, I64, I64, I32, P, C.c_int]
     L.oracle_router_backward.argtypes = [P, P, P, I64, I64, I32, I32, U32, P]
     L.oracle_num_threads.restype = C.c_int
 
@@ -83,6 +83,11 @@ def _c(a, dtype=None):
 
 def _sdt_array(a, dt):
     return _c(a, np.float32 if dt == "f32" else np.uint16)
+
+
+def _out_dtype(dt):
+    """NumPy storage of a tensor of oracle dtype dt (16-bit formats as bits)."""
+    return {"f32": np.float32, "f64": np.float64}.get(dt, np.uint16)
 
 
 def num_threads() -> int:
@@ -182,8 +187,10 @@ def copy_rows(x, src_token):
 # ---------------------------------------------------------------- projections
 
 def project(x, xdt: str, row_expert, proj: dict, sdt: str, g: int, exact: bool = False,
-            odt: str = None, bias_dt: str = "f32"):
-    """Rows of x through their experts' projection (see oracle_project)."""
+            odt: str = None, bias_dt: str = "f32", magnitude: bool = False):
+    """Rows of x through their experts' projection (see oracle_project).
+    exact: the unrounded double sums; magnitude: the double sums of the
+    products' magnitudes (|x W|, plus |bias|)."""
     x = _c(x)
     R, K = x.shape
     qw = _c(proj["qweight"], np.int32)
@@ -197,47 +204,50 @@ def project(x, xdt: str, row_expert, proj: dict, sdt: str, g: int, exact: bool =
         bias = _c(bias, np.float32 if bias_dt == "f32" else np.uint16)
     re = _c(row_expert, np.int32)
     odt = odt or xdt
-    if exact:
-        out = np.zeros((R, N), np.float64)
-    else:
-        out = np.zeros((R, N), {"f32": np.float32, "f64": np.float64}.get(odt, np.uint16))
+    mode = 2 if magnitude else 1 if exact else 0
+    out = np.zeros((R, N), np.float64 if mode else _out_dtype(odt))
     rc = lib().oracle_project(_p(x), DT[xdt], R, K, N, _p(re), E, _p(qw), _p(qz), _p(sc), DT[sdt],
-                              _p(bias), DT[bias_dt], g, 1 if exact else 0, _p(out), DT[odt])
+                              _p(bias), DT[bias_dt], g, mode, _p(out), DT[odt])
     if rc != 0:
         raise ValueError("oracle_project: " + ("incomplete group or N % 8 != 0" if rc == -2 else "expert index out of range"))
     return out
 
 
-def swiglu(G, U, dt: str = "bf16"):
+def swiglu(G, U, dt: str = "bf16", odt: str = None):
+    """h from stored G and U (dtype dt); odt "f64" gives the unrounded h."""
     G, U = _c(G), _c(U)
-    h = np.zeros_like(G)
-    lib().oracle_swiglu(_p(G), _p(U), DT[dt], G.size, _p(h))
+    odt = odt or dt
+    h = np.zeros(G.shape, _out_dtype(odt))
+    lib().oracle_swiglu(_p(G), _p(U), DT[dt], G.size, _p(h), DT[odt])
     return h
 
 
-def combine(y, dt: str, weights, selected, row_of):
+def combine(y, dt: str, weights, selected, row_of, odt: str = None):
+    """Per-token ascending-ID combine; odt "f64" gives the unrounded sums."""
     y = _c(y)
     w, sel, ro = _c(weights, np.float32), _c(selected, np.uint32), _c(row_of, np.int32)
     T, k = w.shape
     H = y.shape[1]
-    out = np.zeros((T, H), y.dtype)
-    lib().oracle_combine(_p(y), DT[dt], _p(w), _p(sel), _p(ro), T, H, k, _p(out))
+    odt = odt or dt
+    out = np.zeros((T, H), _out_dtype(odt))
+    lib().oracle_combine(_p(y), DT[dt], _p(w), _p(sel), _p(ro), T, H, k, _p(out), DT[odt])
     return out
 
 
-def combine_backward(d_out, y, dt: str, weights, row_of, want_dy=True, want_dw=True):
+def combine_backward(d_out, y, dt: str, weights, row_of, want_dy=True, want_dw=True, dy_dt: str = None):
     d_out, y = _c(d_out), _c(y)
     w, ro = _c(weights, np.float32), _c(row_of, np.int32)
     T, k = w.shape
     H = y.shape[1]
-    dy = np.zeros_like(y) if want_dy else None
+    dy_dt = dy_dt or dt
+    dy = np.zeros(y.shape, _out_dtype(dy_dt)) if want_dy else None
     dw = np.zeros((T, k), np.float32) if want_dw else None
-    lib().oracle_combine_backward(_p(d_out), _p(y), DT[dt], _p(w), _p(ro), T, H, k, _p(dy), _p(dw))
+    lib().oracle_combine_backward(_p(d_out), _p(y), DT[dt], _p(w), _p(ro), T, H, k, _p(dy), _p(dw), DT[dy_dt])
     return dy, dw
 
 
 def input_backward(grad, gdt: str, row_expert, proj: dict, sdt: str, g: int, grad2=None, proj2=None,
-                   exact: bool = False, odt: str = None):
+                   exact: bool = False, odt: str = None, magnitude: bool = False):
     grad = _c(grad)
     R, N = grad.shape
     qw = _c(proj["qweight"], np.int32)
@@ -253,28 +263,31 @@ def input_backward(grad, gdt: str, row_expert, proj: dict, sdt: str, g: int, gra
         sc2 = _sdt_array(proj2["scales"], sdt)
     re = _c(row_expert, np.int32)
     odt = odt or gdt
-    out = np.zeros((R, K), np.float64 if exact else {"f32": np.float32, "f64": np.float64}.get(odt, np.uint16))
+    mode = 2 if magnitude else 1 if exact else 0
+    out = np.zeros((R, K), np.float64 if mode else _out_dtype(odt))
     rc = lib().oracle_input_backward(_p(grad), DT[gdt], R, N, K, _p(re), E, _p(qw), _p(qz), _p(sc), DT[sdt], g,
-                                     _p(g2), _p(qw2), _p(qz2), _p(sc2), 1 if exact else 0, _p(out), DT[odt])
+                                     _p(g2), _p(qw2), _p(qz2), _p(sc2), mode, _p(out), DT[odt])
     if rc != 0:
         raise ValueError("oracle_input_backward: " + ("incomplete group or N % 8 != 0" if rc == -2 else "expert index out of range"))
     return out
 
 
-def swiglu_backward(dh, G, U, dt: str = "bf16"):
+def swiglu_backward(dh, G, U, dt: str = "bf16", odt: str = None):
     dh, G, U = _c(dh), _c(G), _c(U)
-    dG, dU = np.zeros_like(G), np.zeros_like(U)
-    lib().oracle_swiglu_backward(_p(dh), _p(G), _p(U), DT[dt], G.size, _p(dG), _p(dU))
+    odt = odt or dt
+    dG, dU = np.zeros(G.shape, _out_dtype(odt)), np.zeros(U.shape, _out_dtype(odt))
+    lib().oracle_swiglu_backward(_p(dh), _p(G), _p(U), DT[dt], G.size, _p(dG), _p(dU), DT[odt])
     return dG, dU
 
 
-def dispatch_backward(dvalues, dt: str, selected, row_of):
+def dispatch_backward(dvalues, dt: str, selected, row_of, odt: str = None):
     dv = _c(dvalues)
     sel, ro = _c(selected, np.uint32), _c(row_of, np.int32)
     T, k = sel.shape
     H = dv.shape[1]
-    dx = np.zeros((T, H), dv.dtype)
-    lib().oracle_dispatch_backward(_p(dv), DT[dt], _p(sel), _p(ro), T, H, k, _p(dx))
+    odt = odt or dt
+    dx = np.zeros((T, H), _out_dtype(odt))
+    lib().oracle_dispatch_backward(_p(dv), DT[dt], _p(sel), _p(ro), T, H, k, _p(dx), DT[odt])
     return dx
 
 

@@ -254,6 +254,9 @@ int oracle_route(const float *logits, const float *sel_bias, int64_t T, int64_t 
             for (int64_t e = 0; e < E; ++e) {
                 if (taken[e]) continue;
                 float s = sel_bias ? (float)(l[e] + sel_bias[e]) : l[e];
+                /* NaN (invalid input) ranks as -inf, so a round still takes a
+                 * defined expert; -0 and +0 are equal scores (a tie) */
+                if (isnan(s)) s = -INFINITY;
                 /* strictly greater keeps the lower ID on ties */
                 if (best < 0 || s > bs || (ORACLE_MUTANT == 4 && s == bs)) { best = e; bs = s; }
             }
@@ -336,6 +339,9 @@ void oracle_copy_rows(const void *x, int64_t H, int64_t elem_bytes, const int32_
  * mode 0: out is stored in odt, rounded once (RNE) from the double sum.
  * mode 1: out is double [R,N], no output rounding (exact-math mode; the
  *         coefficients stay rounded because they are the operator).
+ * mode 2: out is double [R,N] = sum_kk |x[r,kk] * W[e,kk,n]| (+ |bias|):
+ *         the magnitude that bounds the rounding error of the same sum
+ *         accumulated in a shorter format (used by the parity tolerance).
  * Returns 0, -1 on a bad expert index, -2 when K is not a whole number of
  * groups or N is not a multiple of 8 (AwqExpertOptions: complete
  * input-channel groups, output width divisible by eight). */
@@ -363,11 +369,15 @@ int oracle_project(const void *x, int xdt, int64_t R, int64_t K, int64_t N,
             for (int64_t kk = 0; kk < K; ++kk) {
                 double xv = load_val(x, xdt, r * K + kk);
                 const double *Wr = W + kk * N;
-                for (int64_t n = 0; n < N; ++n) acc[n] += xv * Wr[n];
+                if (mode == 2)
+                    for (int64_t n = 0; n < N; ++n) acc[n] += fabs(xv * Wr[n]);
+                else
+                    for (int64_t n = 0; n < N; ++n) acc[n] += xv * Wr[n];
             }
             for (int64_t n = 0; n < N; ++n) {
-                double v = acc[n] + ((be && ORACLE_MUTANT != 7) ? load_val(be, bdt, n) : 0.0);
-                if (mode == 1) ((double *)out)[r * N + n] = v;
+                double b = (be && ORACLE_MUTANT != 7) ? load_val(be, bdt, n) : 0.0;
+                double v = acc[n] + (mode == 2 ? fabs(b) : b);
+                if (mode >= 1) ((double *)out)[r * N + n] = v;
                 else store_val(out, odt, r * N + n, v);
             }
             free(acc);
@@ -377,14 +387,15 @@ int oracle_project(const void *x, int xdt, int64_t R, int64_t K, int64_t N,
     return 0;
 }
 
-/* h = RNE(silu(G) * U), silu(v) = v / (1 + exp(-v)), from stored G and U. */
-void oracle_swiglu(const void *G, const void *U, int dt, int64_t n, void *h) {
+/* h = RNE(silu(G) * U), silu(v) = v / (1 + exp(-v)), from stored G and U
+ * (dtype dt); h is stored in odt (DT_F64: the unrounded value). */
+void oracle_swiglu(const void *G, const void *U, int dt, int64_t n, void *h, int odt) {
 #pragma omp parallel for schedule(static)
     for (int64_t i = 0; i < n; ++i) {
         double gv = load_val(G, dt, i), uv = load_val(U, dt, i);
         double silu = gv / (1.0 + exp(-gv));
         if (ORACLE_MUTANT == 8) silu = 1.0 / (1.0 + exp(-gv));
-        store_val(h, dt, i, silu * uv);
+        store_val(h, odt, i, silu * uv);
     }
 }
 
@@ -398,9 +409,10 @@ static void ascending_slots(const uint32_t *sel, int32_t k, int32_t *order) {
     }
 }
 
-/* out[t,:] = RNE(sum over selections in ascending expert ID of w * y[row]). */
+/* out[t,:] = RNE(sum over selections in ascending expert ID of w * y[row]),
+ * stored in odt (DT_F64: the unrounded sum). */
 void oracle_combine(const void *y, int dt, const float *weights, const uint32_t *selected,
-                    const int32_t *row_of, int64_t T, int64_t H, int32_t k, void *out) {
+                    const int32_t *row_of, int64_t T, int64_t H, int32_t k, void *out, int odt) {
 #pragma omp parallel for schedule(static)
     for (int64_t t = 0; t < T; ++t) {
         int32_t order[64];
@@ -412,17 +424,17 @@ void oracle_combine(const void *y, int dt, const float *weights, const uint32_t 
                 acc += (ORACLE_MUTANT == 10 ? 1.0 : (double)weights[t * k + j]) *
                        load_val(y, dt, (int64_t)row_of[t * k + j] * H + c);
             }
-            store_val(out, dt, t * H + c, acc);
+            store_val(out, odt, t * H + c, acc);
         }
     }
 }
 
-/* Combine VJP.  dy[row_of[t,j],:] = RNE(w[t,j] * dOut[t,:]);
- * dweights[t,j] = FP32(sum_c dOut[t,c] * y[row_of[t,j],c]).  Either output may
- * be NULL (not requested). */
+/* Combine VJP.  dy[row_of[t,j],:] = RNE(w[t,j] * dOut[t,:]) (stored in
+ * dy_dt; DT_F64: unrounded); dweights[t,j] = FP32(sum_c dOut[t,c] *
+ * y[row_of[t,j],c]).  Either output may be NULL (not requested). */
 void oracle_combine_backward(const void *d_out, const void *y, int dt, const float *weights,
                              const int32_t *row_of, int64_t T, int64_t H, int32_t k,
-                             void *dy, float *dweights) {
+                             void *dy, float *dweights, int dy_dt) {
 #pragma omp parallel for schedule(static)
     for (int64_t t = 0; t < T; ++t) {
         for (int32_t j = 0; j < k; ++j) {
@@ -430,7 +442,7 @@ void oracle_combine_backward(const void *d_out, const void *y, int dt, const flo
             double w = (double)weights[t * k + j], dot = 0.0;
             for (int64_t c = 0; c < H; ++c) {
                 double g = load_val(d_out, dt, t * H + c);
-                if (dy) store_val(dy, dt, r * H + c, w * g);
+                if (dy) store_val(dy, dy_dt, r * H + c, w * g);
                 dot += g * (ORACLE_MUTANT == 13 ? g : load_val(y, dt, r * H + c));
             }
             if (dweights) dweights[t * k + j] = (float)dot;
@@ -440,7 +452,8 @@ void oracle_combine_backward(const void *d_out, const void *y, int dt, const flo
 
 /* Input VJP of one (or two summed) grouped projections:
  *   dinput[r,kk] = sum_n grad[r,n] W[e,kk,n]  (+ sum_n grad2[r,n] W2[e,kk,n])
- * rounded once to odt (mode 0) or left in double (mode 1). */
+ * rounded once to odt (mode 0) or left in double (mode 1); mode 2 gives the
+ * double sum of the products' magnitudes (see oracle_project). */
 int oracle_input_backward(const void *grad, int gdt, int64_t R, int64_t N, int64_t K,
                           const int32_t *row_expert, int64_t E,
                           const int32_t *qw, const int32_t *qz, const void *sc, int sdt, int64_t g,
@@ -467,10 +480,16 @@ int oracle_input_backward(const void *grad, int gdt, int64_t R, int64_t N, int64
             if (row_expert[r] != e) continue;
             for (int64_t kk = 0; kk < K; ++kk) {
                 double acc = 0.0;
-                for (int64_t n = 0; n < N; ++n) acc += load_val(grad, gdt, r * N + n) * W[kk * N + n];
+                for (int64_t n = 0; n < N; ++n) {
+                    double pr = load_val(grad, gdt, r * N + n) * W[kk * N + n];
+                    acc += mode == 2 ? fabs(pr) : pr;
+                }
                 if (W2 && ORACLE_MUTANT != 9)
-                    for (int64_t n = 0; n < N; ++n) acc += load_val(grad2, gdt, r * N + n) * W2[kk * N + n];
-                if (mode == 1) ((double *)out)[r * K + kk] = acc;
+                    for (int64_t n = 0; n < N; ++n) {
+                        double pr = load_val(grad2, gdt, r * N + n) * W2[kk * N + n];
+                        acc += mode == 2 ? fabs(pr) : pr;
+                    }
+                if (mode >= 1) ((double *)out)[r * K + kk] = acc;
                 else store_val(out, odt, r * K + kk, acc);
             }
         }
@@ -481,31 +500,34 @@ int oracle_input_backward(const void *grad, int gdt, int64_t R, int64_t N, int64
 }
 
 /* SwiGLU VJP from the stored G, U:  s = 1/(1+exp(-G)),
- *   dG = RNE(dh * U * s * (1 + G * (1 - s))),  dU = RNE(dh * G * s). */
+ *   dG = RNE(dh * U * s * (1 + G * (1 - s))),  dU = RNE(dh * G * s),
+ * stored in odt (DT_F64: unrounded). */
 void oracle_swiglu_backward(const void *dh, const void *G, const void *U, int dt, int64_t n,
-                            void *dG, void *dU) {
+                            void *dG, void *dU, int odt) {
 #pragma omp parallel for schedule(static)
     for (int64_t i = 0; i < n; ++i) {
         double d = load_val(dh, dt, i), gv = load_val(G, dt, i), uv = load_val(U, dt, i);
         double s = 1.0 / (1.0 + exp(-gv));
-        store_val(dG, dt, i, d * uv * s * (ORACLE_MUTANT == 11 ? 1.0 : (1.0 + gv * (1.0 - s))));
-        store_val(dU, dt, i, d * gv * s);
+        store_val(dG, odt, i, d * uv * s * (ORACLE_MUTANT == 11 ? 1.0 : (1.0 + gv * (1.0 - s))));
+        store_val(dU, odt, i, d * gv * s);
     }
 }
 
 /* COPY VJP: dx[t,:] = RNE(sum over selections in ascending expert ID of
- * dvalues[row_of[t,j],:]); routing weights are not applied. */
+ * dvalues[row_of[t,j],:]); routing weights are not applied.  Stored in odt
+ * (DT_F64: the unrounded sum). */
 void oracle_dispatch_backward(const void *dvalues, int dt, const uint32_t *selected,
-                              const int32_t *row_of, int64_t T, int64_t H, int32_t k, void *dx) {
+                              const int32_t *row_of, int64_t T, int64_t H, int32_t k, void *dx,
+                              int odt) {
 #pragma omp parallel for schedule(static)
     for (int64_t t = 0; t < T; ++t) {
         int32_t order[64];
         ascending_slots(selected + t * k, k, order);
         for (int64_t c = 0; c < H; ++c) {
             double acc = 0.0;
-            for (int32_t i = 0; i < k; ++i)
+            for (int32_t i = 0; i < (ORACLE_MUTANT == 14 ? 1 : k); ++i)
                 acc += load_val(dvalues, dt, (int64_t)row_of[t * k + order[i]] * H + c);
-            store_val(dx, dt, t * H + c, acc);
+            store_val(dx, odt, t * H + c, acc);
         }
     }
 }

@@ -93,6 +93,27 @@ def test_combine_special_cases():
     assert np.array_equal(dx, y[:T][::-1])
 
 
+def test_dispatch_backward_hand_worked_top3():
+    """COPY VJP with top_k = 3 ([MX] moe_dispatch_backward sums the selected
+    expert-row seeds of each token, no routing weights).  Two tokens, six
+    distinct rows; every sum is exact in BF16, so dx is known by hand:
+      token 0 selects experts (5, 2, 9) in rows (3, 0, 5):
+        dx[0] = dv[3] + dv[0] + dv[5] = (0.5 + 1 + 64, -1 + 2 - 128) = (65.5, -127)
+      token 1 selects experts (1, 7, 3) in rows (2, 4, 1):
+        dx[1] = dv[2] + dv[4] + dv[1] = (16 - 3 + 4, 32 + 0.25 + 8) = (17, 40.25)"""
+    dv = np.array([[1, 2], [4, 8], [16, 32], [0.5, -1], [-3, 0.25], [64, -128]], np.float32)
+    sel = np.array([[5, 2, 9], [1, 7, 3]], np.uint32)
+    row_of = np.array([[3, 0, 5], [2, 4, 1]], np.int32)
+    dx = oracle.dispatch_backward(inputs.f32_to_bf16_bits(dv), "bf16", sel, row_of)
+    assert np.array_equal(_f(dx), np.array([[65.5, -127.0], [17.0, 40.25]]))
+    # the same in exact mode, and with the selections of a token permuted
+    dx64 = oracle.dispatch_backward(dv.astype(np.float64), "f64", sel, row_of)
+    assert np.array_equal(dx64, np.array([[65.5, -127.0], [17.0, 40.25]]))
+    perm = np.array([2, 0, 1])
+    dxp = oracle.dispatch_backward(inputs.f32_to_bf16_bits(dv), "bf16", sel[:, perm].copy(), row_of[:, perm].copy())
+    assert np.array_equal(dxp, dx)
+
+
 def test_dweights_closed_form_and_dy():
     rng = np.random.default_rng(4)
     T, H, k = 6, 32, 2
@@ -163,21 +184,13 @@ def test_whole_ffn_vjp_matches_finite_difference(sdt):
     x0 = _f(inp["x"])
     d_out = rng.standard_normal(x0.shape)
     out, (G, U, h, y) = _exact_chain(inp, x0, rr)
-    # VJP chain in exact mode
-    dy = np.zeros_like(y)
-    for t in range(w.T):
-        for j in range(w.top_k):
-            dy[row_of[t, j]] = float(wts[t, j]) * d_out[t]
+    # the oracle's own VJP chain, every step in exact (unrounded double) mode
+    dy, _ = oracle.combine_backward(d_out, y, "f64", wts, row_of, want_dw=False)
     re = rexp.astype(np.int32)
     dh = oracle.input_backward(dy, "f64", re, inp["down"], sdt, w.group, exact=True)
-    s = 1.0 / (1.0 + np.exp(-G))
-    dG = dh * U * s * (1.0 + G * (1.0 - s))
-    dU = dh * G * s
+    dG, dU = oracle.swiglu_backward(dh, G, U, "f64")
     dvals = oracle.input_backward(dG, "f64", re, inp["gate"], sdt, w.group, grad2=dU, proj2=inp["up"], exact=True)
-    dx = np.zeros_like(x0)
-    for t in range(w.T):
-        for j in range(w.top_k):
-            dx[t] += dvals[row_of[t, j]]
+    dx = oracle.dispatch_backward(dvals, "f64", sel, row_of)
     v = rng.standard_normal(x0.shape)
     eps = 1e-6
     fp = np.sum(_exact_chain(inp, x0 + eps * v, rr)[0] * d_out)

@@ -3,7 +3,8 @@ mistake in one step of the oracle (a swapped nibble order, a double
 rounding, a wrong zero-point group, a flipped tie-break, biased weights, a
 reversed dispatch order, a dropped bias, a SwiGLU without its gate factor, a
 dropped gate/up gradient term, unweighted combine, a missing SwiGLU-VJP
-factor, a missing softmax-VJP term, a wrong dweights dot), and the oracle's
+factor, a missing softmax-VJP term, a wrong dweights dot, a COPY VJP that
+sums one selection only), and the oracle's
 own CPU tests must fail on every one of them.  CPU only."""
 import os
 import subprocess
@@ -33,6 +34,7 @@ MUTANTS = {
     11: "SwiGLU VJP drops the (1 + G (1 - s)) factor",
     12: "router-logit VJP drops the - <w, dw> term",
     13: "combine VJP dweights dot uses dOut instead of y",
+    14: "COPY VJP sums only the first selection of each token",
 }
 
 

@@ -143,6 +143,25 @@ def test_route_hand_cases():
     assert sel.tolist() == [[41, 42]]
 
 
+def test_route_signed_zero_and_nan_scores():
+    # -0 and +0 are the same score: the tie goes to the lower ID, whichever
+    # sign it carries (IEEE comparison, not the bit pattern)
+    sel, w = oracle.route(np.array([[-0.0, 0.0, -1.0]], np.float32), None, 1)
+    assert sel.tolist() == [[0]]
+    sel, _ = oracle.route(np.array([[0.0, -0.0, -1.0]], np.float32), None, 2)
+    assert sel.tolist() == [[0, 1]]
+    # scores that are zero only after the selection bias: -0 + -0 = -0 for
+    # expert 0, 1 + (-1) = +0 for expert 1; still a tie, lower ID first
+    logits = np.array([[-0.0, 1.0, -2.0]], np.float32)
+    bias = np.array([-0.0, -1.0, 0.0], np.float32)
+    sel, w = oracle.route(logits, bias, 1)
+    assert sel.tolist() == [[0]]
+    # a NaN score (invalid input) ranks as -inf: chosen only when nothing
+    # else is left, and then before a real -inf with a higher ID
+    sel, _ = oracle.route(np.array([[np.nan, 0.5, -np.inf, 2.0]], np.float32), None, 3)
+    assert sel.tolist() == [[3, 1, 0]]
+
+
 def test_route_top_k_equals_e_is_full_softmax():
     rng = np.random.default_rng(5)
     logits = rng.standard_normal((6, 9)).astype(np.float32)

@@ -53,8 +53,9 @@
  *   scales, bias and the activation/output tensors 16-byte aligned.
  *   The tensor-core products run in the scale dtype; activations are
  *   converted to it when they differ (BF16 -> F16 is exact for values in
- *   F16's normal range).  FP32 scales are rejected with
- *   MOE_ERR_UNSUPPORTED_DTYPE.
+ *   F16's normal range; a value outside it sets MOE_DEVICE_ERR_ACT_RANGE;
+ *   F16 -> BF16 rounds to 8 significant bits).  FP32 scales are rejected
+ *   with MOE_ERR_UNSUPPORTED_DTYPE.
  */
 #ifndef MOE_AWQ_H_
 #define MOE_AWQ_H_
@@ -88,6 +89,10 @@ typedef enum { MOE_F32 = 0, MOE_F16 = 1, MOE_BF16 = 2 } moe_dtype;
 #define MOE_DEVICE_ERR_OFFSETS 2      /* offsets not monotone, offsets[0] != 0 or offsets[E] != A */
 #define MOE_DEVICE_ERR_ROW_RANGE 4    /* a row_of entry outside [0, A) */
 #define MOE_DEVICE_ERR_TIMEOUT 8      /* a bounded device wait gave up */
+#define MOE_DEVICE_ERR_ACT_RANGE 16   /* a BF16 activation or gradient fed to F16-scale tensor cores lies
+                                         outside F16's normal range (|v| > 65504, inf/NaN, or
+                                         0 < |v| < 2^-14): its conversion to F16 was not exact; the
+                                         result is computed from the converted value */
 
 /* Limits of this implementation. */
 #define MOE_MAX_EXPERTS 4096
@@ -133,8 +138,10 @@ MOE_API const char *moe_version(void);
  *                           initialisation and are dead after the call
  * Errors: MOE_ERR_INVALID_ARGUMENT for T < 0, H < 1, E < 1 or
  * E > MOE_MAX_EXPERTS, top_k out of range, a NULL pointer with T > 0;
- * MOE_ERR_WORKSPACE if workspace is too small.  NaN logits are invalid input:
- * the result is then unspecified but every index stays in range.
+ * MOE_ERR_WORKSPACE if workspace is too small.  Scores compare as IEEE
+ * floats: -0 and +0 are equal (a tie, lower ID first).  NaN logits are
+ * invalid input; a NaN score ranks as -inf (so every index stays defined and
+ * in range), and the weights of a token that selects it are NaN.
  * ---------------------------------------------------------------------- */
 MOE_API size_t moe_route_dispatch_workspace_size(int64_t T, int64_t E, int32_t top_k);
 
@@ -145,6 +152,23 @@ MOE_API moe_status moe_route_dispatch(const void *x, moe_dtype x_dtype, int64_t 
                               uint32_t *row_experts, int32_t *offsets, int32_t *src_token,
                               int32_t *row_of, void *workspace, size_t workspace_bytes,
                               int32_t *device_status, void *stream);
+
+/* ------------------------------------------------------------------------
+ * moe_route -- the routing and row maps of moe_route_dispatch without the
+ * COPY of the rows (the gather mode of the dispatch: the gate/up projection
+ * then reads each row from x through src_token, see
+ * awq_grouped_gate_up_swiglu_gather).  [MX] MoeDispatchOps::moe_dispatch
+ * states the device COPY as its contract; this entry point departs from it
+ * on purpose, and moe_route_dispatch keeps it.
+ *
+ * Arguments, outputs and errors as moe_route_dispatch, minus x, x_dtype, H
+ * and values; the workspace is sized by moe_route_dispatch_workspace_size.
+ * ---------------------------------------------------------------------- */
+MOE_API moe_status moe_route(const float *logits, const float *sel_bias, int64_t T, int64_t E,
+                             int32_t expert_start, int32_t top_k, int32_t renormalize, float *weights,
+                             uint32_t *selected_experts, uint32_t *row_experts, int32_t *offsets,
+                             int32_t *src_token, int32_t *row_of, void *workspace, size_t workspace_bytes,
+                             int32_t *device_status, void *stream);
 
 /* ------------------------------------------------------------------------
  * moe_route_dispatch_noalloc -- moe_route_dispatch for callers that cannot
@@ -162,6 +186,10 @@ MOE_API moe_status moe_route_dispatch(const void *x, moe_dtype x_dtype, int64_t 
  *  - The first call on a device looks the array's device address up
  *    (cudaGetSymbolAddress) with the caller's current device, which must be
  *    the device of `stream`; make that first call before any stream capture.
+ *    The address is kept per device and looked up again when the device's
+ *    context has changed (after cudaDeviceReset).
+ *  - Argument errors are those of moe_route_dispatch and are checked first;
+ *    MOE_ERR_WORKSPACE then means only "too large for the built-in scratch".
  *  - Every call shares the one array, which keeps the last call's contents
  *    (nothing in it needs to start at zero).  Calls whose kernels overlap on
  *    the GPU (other streams, other host threads) race on it: serialise them.
@@ -198,7 +226,8 @@ MOE_API moe_status moe_route_dispatch_noalloc(const void *x, moe_dtype x_dtype, 
  *             bytes (16-byte aligned; may be NULL when that size is 0):
  *             split-K partial sums of the small-batch tiles.  Its contents
  *             need no initialisation and are dead after the call.
- * Device errors: MOE_DEVICE_ERR_OFFSETS.
+ * Device errors: MOE_DEVICE_ERR_OFFSETS, MOE_DEVICE_ERR_ACT_RANGE (F16 scales
+ * with BF16 inputs), MOE_DEVICE_ERR_TIMEOUT.
  * ---------------------------------------------------------------------- */
 MOE_API moe_status awq_grouped_gate_up_swiglu(
     const void *values, moe_dtype act_dtype, int64_t A, int64_t H, int64_t I,
@@ -207,6 +236,27 @@ MOE_API moe_status awq_grouped_gate_up_swiglu(
     const void *bias_gate,
     const int32_t *qweight_up, const int32_t *qzeros_up, const void *scales_up,
     const void *bias_up,
+    moe_dtype scale_dtype, moe_dtype bias_dtype, int64_t group_size,
+    void *h, void *gate_out, void *up_out, void *workspace, size_t workspace_bytes,
+    int32_t *device_status, void *stream);
+
+/* ------------------------------------------------------------------------
+ * awq_grouped_gate_up_swiglu_gather -- awq_grouped_gate_up_swiglu on rows
+ * gathered from the tokens instead of a COPY: expert-sorted row r is
+ * x[src_token[r], :] (x [T, H] in act_dtype, src_token [A] int32 as written
+ * by moe_route or moe_route_dispatch).  Same outputs, bit for bit, as
+ * awq_grouped_gate_up_swiglu on values = the COPY of those rows; same
+ * payload arguments, workspace and errors.  A src_token entry outside
+ * [0, T) sets MOE_DEVICE_ERR_ROW_RANGE and that row reads token 0.
+ * The tcgen05 tiles load the rows with TMA tile::gather4 (four rows per
+ * copy, from this GPU's memory, no multicast); the small-batch tiles with
+ * one bulk copy or load per row.
+ * ---------------------------------------------------------------------- */
+MOE_API moe_status awq_grouped_gate_up_swiglu_gather(
+    const void *x, moe_dtype act_dtype, int64_t T, const int32_t *src_token, int64_t A, int64_t H, int64_t I,
+    const int32_t *offsets, int64_t E,
+    const int32_t *qweight_gate, const int32_t *qzeros_gate, const void *scales_gate, const void *bias_gate,
+    const int32_t *qweight_up, const int32_t *qzeros_up, const void *scales_up, const void *bias_up,
     moe_dtype scale_dtype, moe_dtype bias_dtype, int64_t group_size,
     void *h, void *gate_out, void *up_out, void *workspace, size_t workspace_bytes,
     int32_t *device_status, void *stream);
@@ -227,7 +277,8 @@ MOE_API size_t awq_projection_workspace_size(int64_t A, int64_t K, int64_t N, in
  *  output[r, n] = RNE(sum_kk input[r,kk] * W[e,kk,n] + bias[e,n]).
  *  workspace: awq_projection_workspace_size(A, K, N, E, group_size, 1) bytes (see
  *  awq_grouped_gate_up_swiglu).
- * Device errors: MOE_DEVICE_ERR_OFFSETS.
+ * Device errors: MOE_DEVICE_ERR_OFFSETS, MOE_DEVICE_ERR_ACT_RANGE (F16 scales
+ * with BF16 inputs), MOE_DEVICE_ERR_TIMEOUT.
  * ---------------------------------------------------------------------- */
 MOE_API moe_status awq_grouped_down(const void *input, moe_dtype act_dtype, int64_t A, int64_t K,
                             int64_t N, const int32_t *offsets, int64_t E,
@@ -276,7 +327,8 @@ MOE_API moe_status moe_combine_backward(const void *d_out, const void *y, moe_dt
  * Tile paths as for the forward projections (warp-level, 128-row tcgen05,
  * 256-row CTA-pair tcgen05); the tensor-core products run in the scale
  * dtype, gradients converted to it when they differ.
- * Device errors: MOE_DEVICE_ERR_OFFSETS.
+ * Device errors: MOE_DEVICE_ERR_OFFSETS, MOE_DEVICE_ERR_ACT_RANGE (F16 scales
+ * with BF16 inputs), MOE_DEVICE_ERR_TIMEOUT.
  * ---------------------------------------------------------------------- */
 MOE_API moe_status awq_input_backward(const void *grad, moe_dtype grad_dtype, int64_t A, int64_t N,
                               int64_t K, const int32_t *offsets, int64_t E,

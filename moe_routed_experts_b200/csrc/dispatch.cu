@@ -55,10 +55,13 @@ static RouteWs route_ws_layout(int64_t T, int64_t E, int32_t k) {
 }
 
 // Order key of a score: an unsigned integer that orders like the float
-// (higher score -> larger key).  NaN scores map to the key of -inf so that
-// every round still picks a valid, untaken expert.  0 is below every key.
+// (higher score -> larger key).  -0 and +0 are the same score (an IEEE tie,
+// broken by the lower ID), so -0 is read as +0 before the bits are taken.
+// NaN scores map to the key of -inf so that every round still picks a valid,
+// untaken expert.  0 is below every key.
 __device__ __forceinline__ uint32_t score_key(const float *l, const float *bias, int e) {
   float s = bias ? __fadd_rn(l[e], bias[e]) : l[e];
+  if (s == 0.f) s = 0.f;
   if (isnan(s)) s = -INFINITY;
   const uint32_t b = __float_as_uint(s);
   return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
@@ -280,6 +283,11 @@ __global__ void __launch_bounds__(256) route_scatter_kernel(ScatterParams p) {
   const int lane = threadIdx.x & 31;
   const int64_t wid = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int64_t nw = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  if (!p.values) {  // row maps only (no COPY): one thread per assignment
+    for (int64_t a = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; a < p.A; a += (int64_t)gridDim.x * blockDim.x)
+      scatter_pos(p, a, true);
+    return;
+  }
   if (p.vec16) {
     const int64_t n16 = p.row_bytes / 16;
     for (int64_t a = wid; a < p.A; a += nw) {
@@ -389,10 +397,43 @@ __global__ void __launch_bounds__(256) router_bwd_kernel(RouterBwdParams p) {
 
 using namespace moe;
 
+// Host argument checks of moe_route_dispatch (and of its allocation-free
+// variant, before its scratch-size check): MOE_OK or the error to return.
+static moe_status route_check_args(const char *fn, const void *x, moe_dtype x_dtype, int64_t T, int64_t H,
+                                   const float *logits, int64_t E, int32_t expert_start, int32_t top_k,
+                                   const void *values, const float *weights, const uint32_t *selected_experts,
+                                   const uint32_t *row_experts, const int32_t *offsets, const int32_t *src_token,
+                                   const int32_t *row_of) {
+  if (!valid_dtype(x_dtype)) return set_error(MOE_ERR_UNSUPPORTED_DTYPE, "%s: bad x_dtype %d", fn, (int)x_dtype);
+  if (T < 0 || H < 1 || E < 1 || E > MOE_MAX_EXPERTS)
+    return set_error(MOE_ERR_INVALID_ARGUMENT, "%s: bad sizes T=%lld H=%lld E=%lld", fn, (long long)T,
+                     (long long)H, (long long)E);
+  if (top_k < 1 || top_k > MOE_MAX_TOP_K || top_k > E)
+    return set_error(MOE_ERR_INVALID_ARGUMENT, "%s: top_k=%d outside [1, min(E, %d)]", fn, top_k, MOE_MAX_TOP_K);
+  if (expert_start < 0 || (int64_t)expert_start + E > (int64_t)UINT32_MAX)
+    return set_error(MOE_ERR_INVALID_ARGUMENT, "%s: bad expert_start %d", fn, expert_start);
+  if (!offsets) return set_error(MOE_ERR_INVALID_ARGUMENT, "%s: offsets is NULL", fn);
+  if (T == 0) return MOE_OK;
+  if (!x || !logits || !values || !weights || !selected_experts || !row_experts || !src_token || !row_of)
+    return set_error(MOE_ERR_INVALID_ARGUMENT, "%s: NULL tensor pointer", fn);
+  if (T * (int64_t)top_k > INT32_MAX)
+    return set_error(MOE_ERR_INVALID_ARGUMENT, "%s: T*top_k exceeds int32 row indices", fn);
+  return MOE_OK;
+}
+
 extern "C" size_t moe_route_dispatch_workspace_size(int64_t T, int64_t E, int32_t top_k) {
   if (T < 0 || E < 1 || top_k < 1) return 0;
   return route_ws_layout(T, E, top_k).bytes;
 }
+
+// Routing, row maps and (values != NULL) the COPY of the rows; the two entry
+// points below check their own arguments first.
+static moe_status route_impl(const char *fn, const void *x, moe_dtype x_dtype, int64_t T, int64_t H,
+                             const float *logits, const float *sel_bias, int64_t E, int32_t expert_start,
+                             int32_t top_k, int32_t renormalize, void *values, float *weights,
+                             uint32_t *selected_experts, uint32_t *row_experts, int32_t *offsets,
+                             int32_t *src_token, int32_t *row_of, void *workspace, size_t workspace_bytes,
+                             void *stream);
 
 extern "C" moe_status moe_route_dispatch(const void *x, moe_dtype x_dtype, int64_t T, int64_t H,
                                          const float *logits, const float *sel_bias, int64_t E,
@@ -402,32 +443,47 @@ extern "C" moe_status moe_route_dispatch(const void *x, moe_dtype x_dtype, int64
                                          int32_t *row_of, void *workspace, size_t workspace_bytes,
                                          int32_t *device_status, void *stream) {
   (void)device_status;  // every index is produced here; nothing to report
-  if (!valid_dtype(x_dtype)) return set_error(MOE_ERR_UNSUPPORTED_DTYPE, "moe_route_dispatch: bad x_dtype %d", (int)x_dtype);
-  if (T < 0 || H < 1 || E < 1 || E > MOE_MAX_EXPERTS)
-    return set_error(MOE_ERR_INVALID_ARGUMENT, "moe_route_dispatch: bad sizes T=%lld H=%lld E=%lld",
-                     (long long)T, (long long)H, (long long)E);
-  if (top_k < 1 || top_k > MOE_MAX_TOP_K || top_k > E)
-    return set_error(MOE_ERR_INVALID_ARGUMENT, "moe_route_dispatch: top_k=%d outside [1, min(E, %d)]", top_k,
-                     MOE_MAX_TOP_K);
-  if (expert_start < 0 || (int64_t)expert_start + E > (int64_t)UINT32_MAX)
-    return set_error(MOE_ERR_INVALID_ARGUMENT, "moe_route_dispatch: bad expert_start %d", expert_start);
-  if (!offsets) return set_error(MOE_ERR_INVALID_ARGUMENT, "moe_route_dispatch: offsets is NULL");
+  moe_status a = route_check_args("moe_route_dispatch", x, x_dtype, T, H, logits, E, expert_start, top_k, values,
+                                  weights, selected_experts, row_experts, offsets, src_token, row_of);
+  if (a != MOE_OK) return a;
+  return route_impl("moe_route_dispatch", x, x_dtype, T, H, logits, sel_bias, E, expert_start, top_k, renormalize,
+                    values, weights, selected_experts, row_experts, offsets, src_token, row_of, workspace,
+                    workspace_bytes, stream);
+}
+
+extern "C" moe_status moe_route(const float *logits, const float *sel_bias, int64_t T, int64_t E,
+                                int32_t expert_start, int32_t top_k, int32_t renormalize, float *weights,
+                                uint32_t *selected_experts, uint32_t *row_experts, int32_t *offsets,
+                                int32_t *src_token, int32_t *row_of, void *workspace, size_t workspace_bytes,
+                                int32_t *device_status, void *stream) {
+  (void)device_status;
+  // the argument rules of moe_route_dispatch without x and values
+  static const uint16_t kNoRows[8] = {};
+  moe_status a = route_check_args("moe_route", kNoRows, MOE_BF16, T, 1, logits, E, expert_start, top_k, kNoRows,
+                                  weights, selected_experts, row_experts, offsets, src_token, row_of);
+  if (a != MOE_OK) return a;
+  return route_impl("moe_route", nullptr, MOE_BF16, T, 1, logits, sel_bias, E, expert_start, top_k, renormalize,
+                    nullptr, weights, selected_experts, row_experts, offsets, src_token, row_of, workspace,
+                    workspace_bytes, stream);
+}
+
+static moe_status route_impl(const char *fn, const void *x, moe_dtype x_dtype, int64_t T, int64_t H,
+                             const float *logits, const float *sel_bias, int64_t E, int32_t expert_start,
+                             int32_t top_k, int32_t renormalize, void *values, float *weights,
+                             uint32_t *selected_experts, uint32_t *row_experts, int32_t *offsets,
+                             int32_t *src_token, int32_t *row_of, void *workspace, size_t workspace_bytes,
+                             void *stream) {
   cudaStream_t st = as_stream(stream);
   if (T == 0) {
     if (cudaMemsetAsync(offsets, 0, sizeof(int32_t) * (size_t)(E + 1), st) != cudaSuccess)
-      return check_launch("moe_route_dispatch: memset offsets");
+      return check_launch("memset of the offsets");
     return MOE_OK;
   }
-  if (!x || !logits || !values || !weights || !selected_experts || !row_experts || !src_token || !row_of)
-    return set_error(MOE_ERR_INVALID_ARGUMENT, "moe_route_dispatch: NULL tensor pointer");
-  if (T * (int64_t)top_k > INT32_MAX)
-    return set_error(MOE_ERR_INVALID_ARGUMENT, "moe_route_dispatch: T*top_k exceeds int32 row indices");
   RouteWs lay = route_ws_layout(T, E, top_k);
   if (!workspace || workspace_bytes < lay.bytes)
-    return set_error(MOE_ERR_WORKSPACE, "moe_route_dispatch: workspace of %zu bytes, need %zu", workspace_bytes,
-                     lay.bytes);
+    return set_error(MOE_ERR_WORKSPACE, "%s: workspace of %zu bytes, need %zu", fn, workspace_bytes, lay.bytes);
   if ((reinterpret_cast<uintptr_t>(workspace) & 15u) != 0)
-    return set_error(MOE_ERR_INVALID_ARGUMENT, "moe_route_dispatch: workspace not 16-byte aligned");
+    return set_error(MOE_ERR_INVALID_ARGUMENT, "%s: workspace not 16-byte aligned", fn);
   int32_t *hist = reinterpret_cast<int32_t *>(static_cast<char *>(workspace) + lay.hist_off);
   int32_t *rank = reinterpret_cast<int32_t *>(static_cast<char *>(workspace) + lay.rank_off);
 
@@ -455,7 +511,7 @@ extern "C" moe_status moe_route_dispatch(const void *x, moe_dtype x_dtype, int64
   // a warp per token (or per few tokens): the widest block the kernel takes
   const int threads = 1024;
   kern<<<(unsigned)lay.nchunks, threads, smem, st>>>(rp);
-  moe_status s = check_launch("moe_route_dispatch: route_rank_kernel");
+  moe_status s = check_launch("route_rank_kernel");
   if (s != MOE_OK) return s;
   if (!rp.single) {
     int tpe = 1;
@@ -463,7 +519,7 @@ extern "C" moe_status moe_route_dispatch(const void *x, moe_dtype x_dtype, int64
     size_t ssm = sizeof(int32_t) * (size_t)(E + 32 + tpe * E);
     if (ssm > 48 * 1024) cudaFuncSetAttribute(route_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ssm);
     route_scan_kernel<<<1, kScanThreads, ssm, st>>>(hist, (int)lay.nchunks, (int)E, offsets);
-    s = check_launch("moe_route_dispatch: route_scan_kernel");
+    s = check_launch("route_scan_kernel");
     if (s != MOE_OK) return s;
   }
   ScatterParams sp;
@@ -484,12 +540,12 @@ extern "C" moe_status moe_route_dispatch(const void *x, moe_dtype x_dtype, int64
   sp.src_token = src_token;
   sp.vec16 = aligned16(x) && aligned16(values) && (sp.row_bytes % 16 == 0);
   sp.nseg = (sp.row_bytes + 63) / 64;  // 2-byte path only
-  int64_t units = sp.vec16 ? sp.A : sp.A * sp.nseg;
+  int64_t units = !values ? (sp.A + 31) / 32 : sp.vec16 ? sp.A : sp.A * sp.nseg;
   int64_t blocks = (units + 7) / 8;
   int64_t cap = (int64_t)num_sms() * 16;
   if (blocks > cap) blocks = cap;
   route_scatter_kernel<<<(unsigned)blocks, 256, 0, st>>>(sp);
-  return check_launch("moe_route_dispatch: route_scatter_kernel");
+  return check_launch("route_scatter_kernel");
 }
 
 // ------------------------------------------------------------------ allocation-free variant
@@ -499,6 +555,8 @@ extern "C" moe_status moe_route_dispatch(const void *x, moe_dtype x_dtype, int64
 // device and stall every stream), or a host framework that owns all device
 // memory through its own pool and forbids allocations outside it.  For them
 // the routing scratch lives in a fixed array compiled into this library.
+
+#include <cudaTypedefs.h>
 
 #include <mutex>
 
@@ -510,21 +568,53 @@ static __device__ __align__(256) uint8_t g_route_scratch[kStaticRouteScratchByte
 constexpr int kMaxScratchDevices = 64;
 static std::mutex g_route_scratch_mu;
 static void *g_route_scratch_ptr[kMaxScratchDevices] = {};
+static unsigned long long g_route_scratch_ctx[kMaxScratchDevices] = {};
 
-// Device address of g_route_scratch on the current device (looked up once per
-// device; the host-side name is only a stand-in for the symbol).
+// Unique ID of the current CUDA context (0 if the driver cannot say).  A
+// context made after cudaDeviceReset gets a new ID, and the library's device
+// array a new address in it.
+static unsigned long long current_context_id() {
+  static PFN_cuCtxGetCurrent_v4000 get_current = nullptr;
+  static PFN_cuCtxGetId_v12000 get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(p);
+  });
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || !ctx || get_id(ctx, &id) != CUDA_SUCCESS)
+    return 0;
+  return id;
+}
+
+// Device address of g_route_scratch on the current device.  Looked up once
+// per device and context (the host-side name of the array is only a stand-in
+// for the symbol); a new context on the device (after cudaDeviceReset) makes
+// the next call look it up again.
 static moe_status route_scratch_address(void **out) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxScratchDevices)
     return set_error(MOE_ERR_CUDA, "moe_route_dispatch_noalloc: no usable current device");
+  // 0 before the runtime has made the device's context current: the lookup
+  // below does that, and the ID is read again after it
+  const unsigned long long ctx = current_context_id();
   std::lock_guard<std::mutex> lock(g_route_scratch_mu);
-  if (!g_route_scratch_ptr[dev]) {
+  if (!g_route_scratch_ptr[dev] || ctx == 0 || ctx != g_route_scratch_ctx[dev]) {
     void *p = nullptr;
     const cudaError_t e = cudaGetSymbolAddress(&p, g_route_scratch);
     if (e != cudaSuccess || !p)
       return set_error(MOE_ERR_CUDA, "moe_route_dispatch_noalloc: cudaGetSymbolAddress failed: %s",
                        cudaGetErrorString(e));
     g_route_scratch_ptr[dev] = p;
+    g_route_scratch_ctx[dev] = current_context_id();
   }
   *out = g_route_scratch_ptr[dev];
   return MOE_OK;
@@ -538,9 +628,10 @@ extern "C" moe_status moe_route_dispatch_noalloc(const void *x, moe_dtype x_dtyp
                                                  void *values, float *weights, uint32_t *selected_experts,
                                                  uint32_t *row_experts, int32_t *offsets, int32_t *src_token,
                                                  int32_t *row_of, int32_t *device_status, void *stream) {
-  if (T < 0 || E < 1 || top_k < 1)
-    return set_error(MOE_ERR_INVALID_ARGUMENT, "moe_route_dispatch_noalloc: bad sizes T=%lld E=%lld top_k=%d",
-                     (long long)T, (long long)E, top_k);
+  // the same argument errors as moe_route_dispatch, before the scratch check
+  moe_status a = route_check_args("moe_route_dispatch_noalloc", x, x_dtype, T, H, logits, E, expert_start, top_k,
+                                  values, weights, selected_experts, row_experts, offsets, src_token, row_of);
+  if (a != MOE_OK) return a;
   const size_t need = route_ws_layout(T, E, top_k).bytes;
   if (need > kStaticRouteScratchBytes)
     return set_error(MOE_ERR_WORKSPACE,

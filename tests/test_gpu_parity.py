@@ -105,6 +105,32 @@ def test_route_ties_and_empty_experts():
     assert np.all(np.diff(off)[50:] == 0)
 
 
+@pytest.mark.parametrize("with_bias", [False, True])
+def test_route_signed_zero_ties(with_bias):
+    # scores of -0 and +0 are equal (a tie, lower ID first) on both sides;
+    # with the selection bias, zero sums arise as x + (-x) = +0 and
+    # (-0) + (-0) = -0.  A few NaN logits (invalid input) rank as -inf.
+    T, E, k = 257, 40, 6
+    rng = np.random.default_rng(5)
+    logits = rng.choice(np.array([-0.0, 0.0, -1.0, 1.0, -np.inf], np.float32), size=(T, E))
+    logits[rng.integers(0, T, 20), rng.integers(0, E, 20)] = np.nan
+    bias = None
+    if with_bias:
+        bias = rng.choice(np.array([-0.0, 0.0, -1.0, 1.0], np.float32), size=E)
+    x = inputs.random_bf16(rng, (T, 16))
+    xd = torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).cuda()
+    r = B.moe_route_dispatch(xd, torch.from_numpy(logits).cuda(), k, E=E,
+                             sel_bias=None if bias is None else torch.from_numpy(bias).cuda())
+    sel, wts = oracle.route(logits, bias, k)
+    off, rexp, src, row_of = oracle.dispatch(sel, E)
+    assert np.array_equal(u32(r["selected_experts"]), sel)
+    assert np.array_equal(r["offsets"].cpu().numpy(), off)
+    assert np.array_equal(r["src_token"].cpu().numpy(), src)
+    assert np.array_equal(r["row_of"].cpu().numpy(), row_of)
+    ok = np.all(np.isfinite(wts), axis=1)  # tokens whose selection holds no NaN
+    assert np.max(np.abs(r["weights"].cpu().numpy()[ok] - wts[ok])) <= 2e-6
+
+
 def test_route_large_expert_count_and_top_k_32():
     T, E, k = 130, 4096, 32
     rng = np.random.default_rng(4)

@@ -9,7 +9,8 @@ import pytest
 import torch
 
 import oracle
-from helpers import bits, check_close, check_forward_steps, check_routing, gpu_forward_numpy
+from helpers import (bits, check_close, check_forward_steps, check_routing, gpu_forward_numpy, j_chain,
+                     j_input_backward, j_project, j_swiglu)
 from moe_routed_experts_b200 import binding as B
 from moe_routed_experts_b200 import ffn, inputs
 from moe_routed_experts_b200.configs import Workload
@@ -59,8 +60,9 @@ def test_single_projection_narrow_outputs(N, path):
     off = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
     xd = torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).cuda()
     y = B.awq_grouped_down(xd, torch.from_numpy(off).cuda(), ffn.projection_to_device(proj, "f16"), g)
-    want = oracle.project(x, "bf16", np.repeat(np.arange(E), counts).astype(np.int32), proj, "f16", g)
-    check_close(bits(y), want, "narrow")
+    re = np.repeat(np.arange(E), counts).astype(np.int32)
+    want = oracle.project(x, "bf16", re, proj, "f16", g)
+    check_close(bits(y), want, "narrow", justify=j_project(x, "bf16", re, proj, "f16", g))
 
 
 def test_every_row_on_one_expert(path):
@@ -105,17 +107,19 @@ def test_activation_and_scale_dtypes(act, sdt, path):
     oG = oracle.project(values, act, re, inp["gate"], sdt, w.group)
     oU = oracle.project(values, act, re, inp["up"], sdt, w.group)
     oh = oracle.swiglu(oG, oU, act)
-    check_close(bits(G), oG, "G", dt=act)
-    check_close(bits(U), oU, "U", dt=act)
-    check_close(bits(h), oracle.swiglu(bits(G), bits(U), act), "h", dt=act)
-    check_close(bits(h), oh, "h(end-to-end)", dt=act, ulps=2)
+    check_close(bits(G), oG, "G", dt=act, justify=j_project(values, act, re, inp["gate"], sdt, w.group))
+    check_close(bits(U), oU, "U", dt=act, justify=j_project(values, act, re, inp["up"], sdt, w.group))
+    check_close(bits(h), oracle.swiglu(bits(G), bits(U), act), "h", dt=act,
+                justify=j_swiglu(bits(G), bits(U), act))
+    check_close(bits(h), oh, "h(end-to-end)", dt=act,
+                justify=j_chain(j_swiglu(oG, oU, act), j_swiglu(bits(G), bits(U), act)))
     down = ffn.projection_to_device(inp["down"], sdt)
     y = B.awq_grouped_down(h, offd, down, w.group)
     oy = oracle.project(bits(h), act, re, inp["down"], sdt, w.group)
-    check_close(bits(y), oy, "y", dt=act)
+    check_close(bits(y), oy, "y", dt=act, justify=j_project(bits(h), act, re, inp["down"], sdt, w.group))
     dx = B.awq_input_backward(y, offd, down, w.group)
     odx = oracle.input_backward(bits(y), act, re, inp["down"], sdt, w.group)
-    check_close(bits(dx), odx, "dinput", dt=act)
+    check_close(bits(dx), odx, "dinput", dt=act, justify=j_input_backward(bits(y), act, re, inp["down"], sdt, w.group))
 
 
 def test_single_frozen_linear_is_one_expert(path):
@@ -128,7 +132,7 @@ def test_single_frozen_linear_is_one_expert(path):
     off = torch.tensor([0, A], dtype=torch.int32, device="cuda")
     y = B.awq_grouped_down(xd, off, ffn.projection_to_device(proj, "f16"), g)
     want = oracle.project(x, "bf16", np.zeros(A, np.int32), proj, "f16", g)
-    check_close(bits(y), want, "linear")
+    check_close(bits(y), want, "linear", justify=j_project(x, "bf16", np.zeros(A, np.int32), proj, "f16", g))
 
 
 def test_inconsistent_offsets_are_flagged_not_faulted(path):
@@ -144,6 +148,35 @@ def test_inconsistent_offsets_are_flagged_not_faulted(path):
         B.awq_grouped_gate_up_swiglu(values, off, dev["gate"], dev["up"], w.group, device_status=st, out=h)
         torch.cuda.synchronize()
         assert int(st.item()) & 2, bad
+
+
+@pytest.mark.parametrize("value", [70000.0, 1e-6, float("inf")], ids=["above_f16_max", "below_f16_normal", "inf"])
+def test_activation_outside_f16_range_is_flagged(value, path):
+    # F16 scales with BF16 inputs: the tensor-core operand is F16, so a BF16
+    # activation or gradient outside F16's normal range cannot be converted
+    # exactly; the projection and the input VJP report it (and only it)
+    rng = np.random.default_rng(11)
+    E, K, N, g, A = 2, 256, 128, 64, 256
+    proj = inputs.draw_projection(rng, E, K, N, g, "f16", False, 0.0)
+    dproj = ffn.projection_to_device(proj, "f16")
+    off = torch.tensor([0, A // 2, A], dtype=torch.int32, device="cuda")
+    x = torch.from_numpy(inputs.random_bf16(rng, (A, K)).view(np.int16)).view(torch.bfloat16).cuda()
+    st = B.new_status()
+    B.awq_grouped_down(x, off, dproj, g, device_status=st)
+    gr = torch.from_numpy(inputs.random_bf16(rng, (A, N)).view(np.int16)).view(torch.bfloat16).cuda()
+    B.awq_input_backward(gr, off, dproj, g, device_status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0  # in-range inputs: nothing reported
+    x[A - 3, K - 5] = value
+    st = B.new_status()
+    B.awq_grouped_down(x, off, dproj, g, device_status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 16, int(st.item())  # MOE_DEVICE_ERR_ACT_RANGE
+    gr[7, 3] = -value
+    st = B.new_status()
+    B.awq_input_backward(gr, off, dproj, g, device_status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 16, int(st.item())
 
 
 def test_row_index_out_of_range_is_flagged():

@@ -21,7 +21,7 @@ HEADER = os.path.join(os.path.dirname(HERE), "include", "moe_awq.h")
 MOE_F32, MOE_F16, MOE_BF16 = 0, 1, 2
 STATUS = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARGUMENT", 2: "MOE_ERR_UNSUPPORTED_DTYPE", 3: "MOE_ERR_WORKSPACE",
           4: "MOE_ERR_CUDA"}
-DEVICE_ERR = {1: "EXPERT_RANGE", 2: "OFFSETS", 4: "ROW_RANGE", 8: "TIMEOUT"}
+DEVICE_ERR = {1: "EXPERT_RANGE", 2: "OFFSETS", 4: "ROW_RANGE", 8: "TIMEOUT", 16: "ACT_RANGE"}
 
 _TORCH_DT = {torch.float32: MOE_F32, torch.float16: MOE_F16, torch.bfloat16: MOE_BF16}
 _NAME_DT = {"f32": MOE_F32, "f16": MOE_F16, "bf16": MOE_BF16}
@@ -44,8 +44,11 @@ _SIGS = {
     "moe_route_dispatch": (C.c_int, [P, C.c_int, I64, I64, P, P, I64, I32, I32, I32, P, P, P, P, P, P, P, P, SZ, P, P]),
     "moe_route_dispatch_noalloc": (C.c_int, [P, C.c_int, I64, I64, P, P, I64, I32, I32, I32, P, P, P, P, P, P, P, P,
                                              P]),
+    "moe_route": (C.c_int, [P, P, I64, I64, I32, I32, I32, P, P, P, P, P, P, P, SZ, P, P]),
     "awq_grouped_gate_up_swiglu": (C.c_int, [P, C.c_int, I64, I64, I64, P, I64, P, P, P, P, P, P, P, P, C.c_int,
                                              C.c_int, I64, P, P, P, P, SZ, P, P]),
+    "awq_grouped_gate_up_swiglu_gather": (C.c_int, [P, C.c_int, I64, P, I64, I64, I64, P, I64, P, P, P, P, P, P, P,
+                                                    P, C.c_int, C.c_int, I64, P, P, P, P, SZ, P, P]),
     "awq_projection_workspace_size": (SZ, [I64, I64, I64, I64, I64, I32]),
     "awq_grouped_down": (C.c_int, [P, C.c_int, I64, I64, I64, P, I64, P, P, P, P, C.c_int, C.c_int, I64, P, P, SZ, P,
                                    P]),
@@ -150,6 +153,32 @@ def moe_route_dispatch(x, logits, top_k, E=None, sel_bias=None, expert_start=0, 
     return out
 
 
+def moe_route(logits, top_k, E=None, sel_bias=None, expert_start=0, renormalize=1, workspace=None,
+              device_status=None, out=None):
+    """Routing and row maps without the COPY (the gather mode of the dispatch)."""
+    T = logits.shape[0]
+    E = E if E is not None else logits.shape[1]
+    A = T * top_k
+    dev = logits.device
+    if out is None:
+        out = {
+            "weights": torch.empty((T, top_k), dtype=torch.float32, device=dev),
+            "selected_experts": torch.empty((T, top_k), dtype=torch.int32, device=dev),
+            "row_experts": torch.empty((A,), dtype=torch.int32, device=dev),
+            "offsets": torch.empty((E + 1,), dtype=torch.int32, device=dev),
+            "src_token": torch.empty((A,), dtype=torch.int32, device=dev),
+            "row_of": torch.empty((T, top_k), dtype=torch.int32, device=dev),
+        }
+    if workspace is None:
+        workspace = torch.empty(max(route_dispatch_workspace_size(T, E, top_k), 256), dtype=torch.uint8, device=dev)
+    st = lib().moe_route(
+        _ptr(logits), _ptr(sel_bias), T, E, expert_start, top_k, renormalize, _ptr(out["weights"]),
+        _ptr(out["selected_experts"]), _ptr(out["row_experts"]), _ptr(out["offsets"]), _ptr(out["src_token"]),
+        _ptr(out["row_of"]), _ptr(workspace), workspace.numel(), _ptr(device_status), _stream())
+    _check("moe_route", st)
+    return out
+
+
 def moe_route_dispatch_noalloc(x, logits, top_k, out, E=None, sel_bias=None, expert_start=0, renormalize=1,
                                device_status=None):
     """moe_route_dispatch with the library's built-in scratch; `out` holds
@@ -200,6 +229,28 @@ def awq_grouped_gate_up_swiglu(values, offsets, gate, up, group, want_gu=False, 
         sdt, _bias_dt(gate.get("bias"), up.get("bias")), group, _ptr(h), _ptr(G), _ptr(U), _ptr(ws),
         0 if ws is None else ws.numel(), _ptr(device_status), _stream())
     _check("awq_grouped_gate_up_swiglu", st)
+    return (h, G, U) if want_gu else h
+
+
+def awq_grouped_gate_up_swiglu_gather(x, src_token, offsets, gate, up, group, want_gu=False, device_status=None,
+                                      out=None, workspace=None):
+    """Gate/up on expert-sorted rows read as x[src_token[r]] (no COPY)."""
+    T, H = x.shape
+    A = src_token.numel()
+    E = offsets.numel() - 1
+    I = gate["qweight"].shape[2] * 8
+    sdt = _dt(gate["scales"].dtype)
+    h = out if out is not None else torch.empty((A, I), dtype=x.dtype, device=x.device)
+    G = torch.empty_like(h) if want_gu else None
+    U = torch.empty_like(h) if want_gu else None
+    ws = _workspace(projection_workspace_size(A, H, I, E, group, 2), x.device, workspace)
+    st = lib().awq_grouped_gate_up_swiglu_gather(
+        _ptr(x), _dt(x.dtype), T, _ptr(src_token), A, H, I, _ptr(offsets), E,
+        _ptr(gate["qweight"]), _ptr(gate["qzeros"]), _ptr(gate["scales"]), _ptr(gate.get("bias")),
+        _ptr(up["qweight"]), _ptr(up["qzeros"]), _ptr(up["scales"]), _ptr(up.get("bias")),
+        sdt, _bias_dt(gate.get("bias"), up.get("bias")), group, _ptr(h), _ptr(G), _ptr(U), _ptr(ws),
+        0 if ws is None else ws.numel(), _ptr(device_status), _stream())
+    _check("awq_grouped_gate_up_swiglu_gather", st)
     return (h, G, U) if want_gu else h
 
 

@@ -35,12 +35,19 @@ def _deps():
         [os.path.join(INCLUDE, f) for f in os.listdir(INCLUDE)]
 
 
-def _compile(src: str, verbose_ptxas: bool) -> str:
-    obj = os.path.join(BUILD, os.path.basename(src) + ".o")
+# A separate build for one test only: MOE_TEST_HOOKS compiles in a switch
+# that makes one bounded device wait run out (moe_test_arm_stall).  The
+# shipped library never contains it.
+TEST_HOOKS_BUILD = os.path.join(BUILD, "test_hooks")
+TEST_HOOKS_LIB = os.path.join(HERE, "libmoe_awq_test_hooks.so")
+
+
+def _compile(src: str, verbose_ptxas: bool, build_dir: str = BUILD, defines=()) -> str:
+    obj = os.path.join(build_dir, os.path.basename(src) + ".o")
     newest_dep = max(os.path.getmtime(d) for d in _deps() + [src])
     if os.path.exists(obj) and os.path.getmtime(obj) >= newest_dep and not verbose_ptxas:
         return obj
-    cmd = [nvcc(), *ARCH, *NVCC_FLAGS, "-c", src, "-o", obj]
+    cmd = [nvcc(), *ARCH, *NVCC_FLAGS, *defines, "-c", src, "-o", obj]
     if verbose_ptxas:
         cmd[1:1] = ["-Xptxas", "-v"]
     r = subprocess.run(cmd, capture_output=True, text=True)
@@ -51,26 +58,28 @@ def _compile(src: str, verbose_ptxas: bool) -> str:
     return obj
 
 
-def build(force: bool = False, verbose_ptxas: bool = False) -> str:
-    os.makedirs(BUILD, exist_ok=True)
+def build(force: bool = False, verbose_ptxas: bool = False, test_hooks: bool = False) -> str:
+    build_dir, lib = (TEST_HOOKS_BUILD, TEST_HOOKS_LIB) if test_hooks else (BUILD, LIB)
+    defines = ("-DMOE_TEST_HOOKS",) if test_hooks else ()
+    os.makedirs(build_dir, exist_ok=True)
     if force:
-        for f in os.listdir(BUILD):
+        for f in os.listdir(build_dir):
             if f.endswith(".o"):
-                os.remove(os.path.join(BUILD, f))
+                os.remove(os.path.join(build_dir, f))
     srcs = sources()
     with cf.ThreadPoolExecutor(max_workers=min(8, len(srcs))) as ex:
-        objs = list(ex.map(lambda s: _compile(s, verbose_ptxas), srcs))
-    if os.path.exists(LIB) and os.path.getmtime(LIB) >= max(os.path.getmtime(o) for o in objs) and not force:
-        return LIB
-    tmp = LIB + ".tmp.%d" % os.getpid()
+        objs = list(ex.map(lambda s: _compile(s, verbose_ptxas, build_dir, defines), srcs))
+    if os.path.exists(lib) and os.path.getmtime(lib) >= max(os.path.getmtime(o) for o in objs) and not force:
+        return lib
+    tmp = lib + ".tmp.%d" % os.getpid()
     # the driver API (tensor-map encoding) is resolved at run time through the
     # runtime's entry-point query, so the library loads without libcuda
     cmd = [nvcc(), *ARCH, "-shared", "-cudart", "static", "-Xcompiler", "-fvisibility=hidden", "-o", tmp, *objs]
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError("link failed:\n%s\n%s" % (r.stdout, r.stderr))
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":

@@ -124,23 +124,28 @@ extern "C" size_t awq_projection_workspace_size(int64_t A, int64_t K, int64_t N,
   return pl.fits ? pl.bytes : 0;
 }
 
-extern "C" moe_status awq_grouped_gate_up_swiglu(
-    const void *values, moe_dtype act_dtype, int64_t A, int64_t H, int64_t I, const int32_t *offsets, int64_t E,
-    const int32_t *qweight_gate, const int32_t *qzeros_gate, const void *scales_gate, const void *bias_gate,
-    const int32_t *qweight_up, const int32_t *qzeros_up, const void *scales_up, const void *bias_up,
-    moe_dtype scale_dtype, moe_dtype bias_dtype, int64_t group_size, void *h, void *gate_out, void *up_out,
-    void *workspace, size_t workspace_bytes, int32_t *device_status, void *stream) {
-  const char *fn = "awq_grouped_gate_up_swiglu";
+// Gate/up projections of expert-sorted rows that are read from `values`
+// (gather == NULL) or as x[gather[r]] (x has T rows).
+static moe_status gate_up_impl(const char *fn, const void *x, const int32_t *gather, int64_t T, moe_dtype act_dtype,
+                               int64_t A, int64_t H, int64_t I, const int32_t *offsets, int64_t E,
+                               const int32_t *qweight_gate, const int32_t *qzeros_gate, const void *scales_gate,
+                               const void *bias_gate, const int32_t *qweight_up, const int32_t *qzeros_up,
+                               const void *scales_up, const void *bias_up, moe_dtype scale_dtype,
+                               moe_dtype bias_dtype, int64_t group_size, void *h, void *gate_out, void *up_out,
+                               void *workspace, size_t workspace_bytes, int32_t *device_status, void *stream) {
   moe_status s = check_payload_geom(fn, A, H, I, E, group_size, act_dtype, scale_dtype);
   if (s != MOE_OK) return s;
   if ((bias_gate || bias_up) && !valid_dtype(bias_dtype))
     return set_error(MOE_ERR_UNSUPPORTED_DTYPE, "%s: bad bias dtype", fn);
+  if (gather && T < 1) return set_error(MOE_ERR_INVALID_ARGUMENT, "%s: T=%lld rows of x", fn, (long long)T);
   if (A == 0) return MOE_OK;
-  s = check_ptrs(fn, {values, offsets, qweight_gate, qzeros_gate, scales_gate, qweight_up, qzeros_up, scales_up, h},
-                 {values, scales_gate, scales_up, h, gate_out, up_out, qweight_gate, qweight_up, bias_gate, bias_up});
+  s = check_ptrs(fn, {x, offsets, qweight_gate, qzeros_gate, scales_gate, qweight_up, qzeros_up, scales_up, h},
+                 {x, scales_gate, scales_up, h, gate_out, up_out, qweight_gate, qweight_up, bias_gate, bias_up});
   if (s != MOE_OK) return s;
   ProjParams p{};
-  p.x = static_cast<const uint16_t *>(values);
+  p.x = static_cast<const uint16_t *>(x);
+  p.gather = gather;
+  p.T = gather ? T : A;
   p.act_dt = act_dtype;
   p.A = A;
   p.K = H;
@@ -169,6 +174,31 @@ extern "C" moe_status awq_grouped_gate_up_swiglu(
   if (stream_plan(A, H, I, E, group_size, 2, nt).fits) return launch_fwd_stream(p, 2, bf, nt, workspace, workspace_bytes, st);
   launch_fwd_mma(p, 2, bf, nt, st);
   return check_launch(fn);
+}
+
+extern "C" moe_status awq_grouped_gate_up_swiglu(
+    const void *values, moe_dtype act_dtype, int64_t A, int64_t H, int64_t I, const int32_t *offsets, int64_t E,
+    const int32_t *qweight_gate, const int32_t *qzeros_gate, const void *scales_gate, const void *bias_gate,
+    const int32_t *qweight_up, const int32_t *qzeros_up, const void *scales_up, const void *bias_up,
+    moe_dtype scale_dtype, moe_dtype bias_dtype, int64_t group_size, void *h, void *gate_out, void *up_out,
+    void *workspace, size_t workspace_bytes, int32_t *device_status, void *stream) {
+  return gate_up_impl("awq_grouped_gate_up_swiglu", values, nullptr, A, act_dtype, A, H, I, offsets, E, qweight_gate,
+                      qzeros_gate, scales_gate, bias_gate, qweight_up, qzeros_up, scales_up, bias_up, scale_dtype,
+                      bias_dtype, group_size, h, gate_out, up_out, workspace, workspace_bytes, device_status, stream);
+}
+
+extern "C" moe_status awq_grouped_gate_up_swiglu_gather(
+    const void *x, moe_dtype act_dtype, int64_t T, const int32_t *src_token, int64_t A, int64_t H, int64_t I,
+    const int32_t *offsets, int64_t E, const int32_t *qweight_gate, const int32_t *qzeros_gate,
+    const void *scales_gate, const void *bias_gate, const int32_t *qweight_up, const int32_t *qzeros_up,
+    const void *scales_up, const void *bias_up, moe_dtype scale_dtype, moe_dtype bias_dtype, int64_t group_size,
+    void *h, void *gate_out, void *up_out, void *workspace, size_t workspace_bytes, int32_t *device_status,
+    void *stream) {
+  const char *fn = "awq_grouped_gate_up_swiglu_gather";
+  if (A > 0 && !src_token) return set_error(MOE_ERR_INVALID_ARGUMENT, "%s: src_token is NULL", fn);
+  return gate_up_impl(fn, x, src_token, T, act_dtype, A, H, I, offsets, E, qweight_gate, qzeros_gate, scales_gate,
+                      bias_gate, qweight_up, qzeros_up, scales_up, bias_up, scale_dtype, bias_dtype, group_size, h,
+                      gate_out, up_out, workspace, workspace_bytes, device_status, stream);
 }
 
 extern "C" moe_status awq_grouped_down(const void *input, moe_dtype act_dtype, int64_t A, int64_t K, int64_t N,

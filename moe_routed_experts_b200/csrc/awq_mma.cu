@@ -33,6 +33,7 @@ namespace moe {
 
 template <typename MT, int NPROJ, int NT>
 __global__ void __launch_bounds__(128) awq_fwd_mma_kernel(ProjParams p) {
+  uint32_t act_bad = 0;  // a converted input outside F16's normal range
   constexpr int D = 2;  // K steps of loads in flight per warp
   __shared__ float red[4][NPROJ][8 * NT][64];
   const int e = blockIdx.y;
@@ -75,7 +76,7 @@ __global__ void __launch_bounds__(128) awq_fwd_mma_kernel(ProjParams p) {
     for (int nt = 0; nt < NT; ++nt) {
       const int tr = tok0 + nt * 8 + g;
       xok[nt] = tr < m;
-      xrow[nt] = p.x + (r0 + (xok[nt] ? tr : 0)) * p.K + 4 * t;
+      xrow[nt] = p.x + act_row(p, r0 + (xok[nt] ? tr : 0)) * p.K + 4 * t;
     }
     FwdConsts<MT> cst[NPROJ];
     int64_t cur_grp = -1;
@@ -112,8 +113,8 @@ __global__ void __launch_bounds__(128) awq_fwd_mma_kernel(ProjParams p) {
           uint32_t b0[NT], b1[NT];
 #pragma unroll
           for (int nt = 0; nt < NT; ++nt) {
-            b0[nt] = act_pair_to_mt<MT>(xbuf[d][nt].x, p.act_dt);
-            b1[nt] = act_pair_to_mt<MT>(xbuf[d][nt].y, p.act_dt);
+            b0[nt] = act_pair_to_mt<MT>(xbuf[d][nt].x, p.act_dt, act_bad);
+            b1[nt] = act_pair_to_mt<MT>(xbuf[d][nt].y, p.act_dt, act_bad);
           }
 #pragma unroll
           for (int j = 0; j < NPROJ; ++j) {
@@ -195,12 +196,14 @@ __global__ void __launch_bounds__(128) awq_fwd_mma_kernel(ProjParams p) {
     }
     __syncthreads();
   }
+  if (act_bad) report(p.status, MOE_DEVICE_ERR_ACT_RANGE);
 }
 
 // ------------------------------------------------------------------ input VJP
 
 template <typename MT, int NPROJ, int NT>
 __global__ void __launch_bounds__(128) awq_bwd_mma_kernel(BwdParams p) {
+  uint32_t act_bad = 0;  // a converted input outside F16's normal range
   __shared__ float red[4][8 * NT][64];
   const int e = blockIdx.y;
   int64_t r0, r1;
@@ -272,8 +275,8 @@ __global__ void __launch_bounds__(128) awq_bwd_mma_kernel(BwdParams p) {
         uint32_t b0[NT], b1[NT];
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
-          b0[nt] = act_pair_to_mt<MT>(q == 0 ? gv[nt].x : gv[nt].z, p.gdt);
-          b1[nt] = act_pair_to_mt<MT>(q == 0 ? gv[nt].y : gv[nt].w, p.gdt);
+          b0[nt] = act_pair_to_mt<MT>(q == 0 ? gv[nt].x : gv[nt].z, p.gdt, act_bad);
+          b1[nt] = act_pair_to_mt<MT>(q == 0 ? gv[nt].y : gv[nt].w, p.gdt, act_bad);
         }
 #pragma unroll
         for (int mt = 0; mt < 4; ++mt) {
@@ -320,6 +323,7 @@ __global__ void __launch_bounds__(128) awq_bwd_mma_kernel(BwdParams p) {
     }
     __syncthreads();
   }
+  if (act_bad) report(p.status, MOE_DEVICE_ERR_ACT_RANGE);
 }
 
 // ------------------------------------------------------------------ coefficient dump

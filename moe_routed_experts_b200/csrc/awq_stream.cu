@@ -155,6 +155,10 @@ __global__ void __launch_bounds__(stream::kThreads, 2)
   int32_t *pre = reinterpret_cast<int32_t *>(red + 8 * NT * kF);    // [E + 1]
   int32_t *cnt = pre + (E + 1);                                    // [E]
   int32_t *tmp = cnt + E;                                          // [32]
+  volatile int32_t *abort = reinterpret_cast<volatile int32_t *>(xempty + 2);
+#ifdef MOE_TEST_HOOKS
+  uint64_t *stall = xempty + 3;  // test build only: a barrier nothing arrives on
+#endif
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -166,6 +170,10 @@ __global__ void __launch_bounds__(stream::kThreads, 2)
       mbar_init(&xfull[b], 1);
       mbar_init(&xempty[b], kCW);
     }
+    *abort = 0;
+#ifdef MOE_TEST_HOOKS
+    mbar_init(stall, 1);
+#endif
     fence_mbar_init();
   }
   // units per expert; an inconsistent row range is flagged and skipped
@@ -182,27 +190,36 @@ __global__ void __launch_bounds__(stream::kThreads, 2)
 
   if (warp == kCW) {
     // ---------------- producer (one lane).  The activation tile of unit
-    // u+1 is requested when unit u starts, one unit ahead of its use.
+    // u+1 is requested when unit u starts, one unit ahead of its use.  A
+    // failed wait (timeout, or an abort elsewhere in the CTA) stops all
+    // further copies; the copies already issued are waited for before the
+    // lane exits (abort protocol, tma.cuh).
     if (lane != 0) return;
-    auto load_x = [&](int64_t u, uint32_t xi) {
+    uint32_t xissued = 0;
+    auto load_x = [&](int64_t u, uint32_t xi) -> bool {
       const UnitInfo ui = unit_info(pre, p.offsets, E, S, KQ, u);
       const int tok0 = ui.tt * 8 * NT, mrows = min(8 * NT, ui.m - tok0);
       const uint32_t xb = xi & 1, xuse = xi >> 1;
-      if (xuse > 0 && !mbar_wait(&xempty[xb], (xuse - 1) & 1, p.status)) return;
+      if (xuse > 0 && !tc_wait(&xempty[xb], (xuse - 1) & 1, p.status, abort)) return false;
       mbar_arrive_expect_tx(&xfull[xb], (uint32_t)(mrows * Kq * 2));
       for (int r = 0; r < mrows; ++r)
-        bulk_load(xraw + xb * xraw_bytes + r * Kq * 2, p.x + (ui.r0 + tok0 + r) * K + ui.kq * Kq,
+        bulk_load(xraw + xb * xraw_bytes + r * Kq * 2, p.x + act_row(p, ui.r0 + tok0 + r) * K + ui.kq * Kq,
                   (uint32_t)(Kq * 2), &xfull[xb]);
+      ++xissued;
+      return true;
     };
-    if (u0 < u1) load_x(u0, 0);
     uint32_t it = 0, xi = 0;
-    for (int64_t u = u0; u < u1; ++u, ++xi) {
-      if (u + 1 < u1) load_x(u + 1, xi + 1);
+    bool live = u0 >= u1 || load_x(u0, 0);
+    for (int64_t u = u0; u < u1 && live; ++u, ++xi) {
+      if (u + 1 < u1 && !load_x(u + 1, xi + 1)) break;
       const UnitInfo ui = unit_info(pre, p.offsets, E, S, KQ, u);
       const int32_t row0 = (int32_t)(ui.e * K + ui.kq * Kq);
       for (int c = 0; c < nst; ++c, ++it) {
         const uint32_t s = it % kStages, use = it / kStages;
-        if (use > 0 && !mbar_wait(&empty[s], (use - 1) & 1, p.status)) continue;
+        if (use > 0 && !tc_wait(&empty[s], (use - 1) & 1, p.status, abort)) {
+          live = false;
+          break;
+        }
         mbar_arrive_expect_tx(&full[s], kStageBytes);
         uint8_t *dst = stages + s * kStageBytes;
         if (NPROJ == 2) {
@@ -214,10 +231,13 @@ __global__ void __launch_bounds__(stream::kThreads, 2)
         }
       }
     }
+    tma_drain(full, it, kStages, p.status);
+    tma_drain(xfull, xissued, 2, p.status);
     return;
   }
 
   // ---------------- consumers
+  uint32_t act_bad = 0;  // a converted input outside F16's normal range
   const int g = lane >> 2, t = lane & 3;
   const int bw = warp >> 2, cgw = warp & 3;  // box and column group of this warp
   const int jw = NPROJ == 2 ? bw : 0;        // projection of this warp
@@ -244,11 +264,28 @@ __global__ void __launch_bounds__(stream::kThreads, 2)
     // tile is converted, so their latency overlaps that work
     uint32_t pf_zw = wc_ok ? (uint32_t)__ldg(qzp + grp * NW) : 0u;
     uint4 pf_sv = wc_ok ? __ldg(reinterpret_cast<const uint4 *>(scp + grp * p.N)) : make_uint4(0, 0, 0, 0);
+    // F16: the odd-slot shortcut (fwd_pairs16) is exact when every scale of
+    // the column group in this unit's K range is 0 or 2^-14 <= |s| <= 256;
+    // then the odd slots accumulate 16 times their value throughout the unit
+    // and are scaled back (exactly) at its end.  The four lanes of a quad
+    // share the column: each checks one scale pair of each group, the quad ORs.
+    bool x16 = false;
+    if (std::is_same<MT, __half>::value) {
+      uint32_t bad = 0;
+      if (wc_ok)
+        for (int64_t gr = grp; gr * p.group < kbase + Kq; ++gr)
+          bad |= f16_pair_blocks_x16(__ldg(reinterpret_cast<const uint32_t *>(scp + gr * p.N) + t));
+      bad |= __shfl_xor_sync(0xffffffffu, bad, 1);
+      bad |= __shfl_xor_sync(0xffffffffu, bad, 2);
+      x16 = bad == 0;
+    }
 
-    // activation tile: raw rows -> scale dtype, row order t, t+4, t+8, t+12 per 16
+    // activation tile: raw rows -> scale dtype, row order t, t+4, t+8, t+12 per 16.
+    // After an abort every consumer warp still runs the loop (the named
+    // barriers stay matched) but waits for, computes and arrives on nothing.
     const uint32_t xb = xi & 1;
-    mbar_wait(&xfull[xb], (xi >> 1) & 1, p.status);
-    {
+    const bool xok = tc_wait(&xfull[xb], (xi >> 1) & 1, p.status, abort);
+    if (xok) {
       const uint8_t *src = xraw + xb * xraw_bytes;
       const int64_t halves = (int64_t)mrows * (Kq / 8);
       for (int64_t q = threadIdx.x; q < halves; q += kCW * 32) {
@@ -259,48 +296,29 @@ __global__ void __launch_bounds__(stream::kThreads, 2)
                                 prmt(v.y, v.w, 0x7632u)};  // (row i, row i+4) of the half
         uint8_t *dst = xs + tok * xs_pitch + (blk * 16 + 2 * h) * 2;
 #pragma unroll
-        for (int i = 0; i < 4; ++i) *reinterpret_cast<uint32_t *>(dst + 8 * i) = act_pair_to_mt<MT>(pr[i], p.act_dt);
+        for (int i = 0; i < 4; ++i) *reinterpret_cast<uint32_t *>(dst + 8 * i) = act_pair_to_mt<MT>(pr[i], p.act_dt, act_bad);
       }
     }
     __syncwarp();
-    if (lane == 0) mbar_arrive(&xempty[xb]);
+    if (lane == 0 && xok) mbar_arrive(&xempty[xb]);
     named_barrier(1, kCW * 32);
 
     // acc: every slot in its true scale; acc16: odd slots taken 16 times
     // larger (F16 groups whose scales allow it, see fwd_pairs16)
-    float acc[NT][4][4], acc16[NT][2][4];
+    float acc[NT][4][4];
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
+    for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
       for (int q = 0; q < 4; ++q)
 #pragma unroll
         for (int i = 0; i < 4; ++i) acc[nt][q][i] = 0.f;
-#pragma unroll
-      for (int q = 0; q < 2; ++q)
-#pragma unroll
-        for (int i = 0; i < 4; ++i) acc16[nt][q][i] = 0.f;
-    }
     FwdConsts<MT> cst;
-    bool x16 = false;
     const int spg = p.group / kRows;  // stages per group (group % kRows == 0 on this path)
     int gstage = (int)((kbase % p.group) / kRows);
     for (int c = 0; c < nst; ++c, ++it) {
       const uint32_t s = it % kStages, ph = (it / kStages) & 1;
       if (c == 0 || gstage == 0) {  // a stage lies inside one group
-        if (std::is_same<MT, __half>::value) {
-          // 16 RNE((q - z) s) = RNE(16 (q - z) s) needs every nonzero product
-          // normal before and after the scaling: 0 or 2^-14 <= |s| <= 256 for
-          // all 8 scales of this column group
-          const uint32_t w4[4] = {pf_sv.x, pf_sv.y, pf_sv.z, pf_sv.w};
-          uint32_t bad = 0;
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const uint32_t lo = w4[i] & 0x7FFFu, hi = (w4[i] >> 16) & 0x7FFFu;
-            bad |= (lo > 0x5C00u) | (hi > 0x5C00u) | (lo != 0u && lo < 0x0400u) | (hi != 0u && hi < 0x0400u);
-          }
-          x16 = bad == 0;
-        }
-        cst.load(pf_zw, pf_sv, x16);
+        load_consts_fast<MT>(cst, pf_zw, pf_sv, x16);
         if (wc_ok && (grp + 1) * p.group < kbase + Kq) {  // prefetch the next group
           pf_zw = (uint32_t)__ldg(qzp + (grp + 1) * NW);
           pf_sv = __ldg(reinterpret_cast<const uint4 *>(scp + (grp + 1) * p.N));
@@ -310,76 +328,53 @@ __global__ void __launch_bounds__(stream::kThreads, 2)
         gstage = 0;
         ++grp;
       }
-      if (mbar_wait(&full[s], ph, p.status)) {
+      const bool sok = tc_wait(&full[s], ph, p.status, abort);
+      if (sok) {
         const uint8_t *box0 = stages + s * kStageBytes + bw * kBox;
-        // two 16-row steps at a time keep the register footprint of a 32-row stage
-#pragma unroll 1
-        for (int hh = 0; hh < kSteps; hh += 2) {
-        const uint8_t *box = box0 + (16 * hh) * 128;
-        const int xrow0 = kRows * c + 16 * hh;
-        uint32_t w[2][4];
-        uint32_t b0[2][NT], b1[2][NT];
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {  // 16-row steps: rows 16h + {t, t+4, t+8, t+12}
-          w[h][0] = *reinterpret_cast<const uint32_t *>(box + woff0 + (16 * h) * 128);
-          w[h][1] = *reinterpret_cast<const uint32_t *>(box + woff1 + (16 * h) * 128);
-          w[h][2] = *reinterpret_cast<const uint32_t *>(box + woff0 + (16 * h + 8) * 128);
-          w[h][3] = *reinterpret_cast<const uint32_t *>(box + woff1 + (16 * h + 8) * 128);
+#pragma unroll 2
+        for (int h = 0; h < kSteps; ++h) {  // 16-row steps: rows 16h + {t, t+4, t+8, t+12}
+          const uint8_t *box = box0 + (16 * h) * 128;
+          const int xrow0 = kRows * c + 16 * h;
+          uint32_t w[4];
+          uint32_t b0[NT], b1[NT];
+          w[0] = *reinterpret_cast<const uint32_t *>(box + woff0);
+          w[1] = *reinterpret_cast<const uint32_t *>(box + woff1);
+          w[2] = *reinterpret_cast<const uint32_t *>(box + woff0 + 8 * 128);
+          w[3] = *reinterpret_cast<const uint32_t *>(box + woff1 + 8 * 128);
 #pragma unroll
           for (int nt = 0; nt < NT; ++nt) {
-            const uint2 bv =
-                *reinterpret_cast<const uint2 *>(xs + (nt * 8 + g) * xs_pitch + (xrow0 + 16 * h + 4 * t) * 2);
-            b0[h][nt] = bv.x;
-            b1[h][nt] = bv.y;
+            const uint2 bv = *reinterpret_cast<const uint2 *>(xs + (nt * 8 + g) * xs_pitch + (xrow0 + 4 * t) * 2);
+            b0[nt] = bv.x;
+            b1[nt] = bv.y;
           }
-        }
-        bool done = false;
-        if constexpr (std::is_same<MT, __half>::value) {
-          if (x16) {
+          uint32_t af[4][4];
+          if (std::is_same<MT, __half>::value && x16) fwd_step<MT, true>(w[0], w[1], w[2], w[3], cst, af);
+          else fwd_step<MT, false>(w[0], w[1], w[2], w[3], cst, af);
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              uint32_t af[4][4];
-              fwd_step<MT, true>(w[h][0], w[h][1], w[h][2], w[h][3], cst, af);
+          for (int q = 0; q < 4; ++q)
 #pragma unroll
-              for (int q = 0; q < 4; ++q)
-#pragma unroll
-                for (int nt = 0; nt < NT; ++nt) {
-                  if (q & 1) mma16816<MT>(acc16[nt][q >> 1], af[q], b0[h][nt], b1[h][nt]);
-                  else mma16816<MT>(acc[nt][q], af[q], b0[h][nt], b1[h][nt]);
-                }
-            }
-            done = true;
-          }
-        }
-        if (!done) {
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            uint32_t af[4][4];
-            fwd_step<MT, false>(w[h][0], w[h][1], w[h][2], w[h][3], cst, af);
-#pragma unroll
-            for (int q = 0; q < 4; ++q)
-#pragma unroll
-              for (int nt = 0; nt < NT; ++nt) mma16816<MT>(acc[nt][q], af[q], b0[h][nt], b1[h][nt]);
-          }
-        }
+            for (int nt = 0; nt < NT; ++nt) mma16816<MT>(acc[nt][q], af[q], b0[nt], b1[nt]);
         }
       }
       __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[s]);
+      if (lane == 0 && sok) mbar_arrive(&empty[s]);
     }
+    const bool unit_ok = !*abort;  // no stores from a unit an abort cut short
+    if (x16) {
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
+      for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {  // fold the 16x-scaled odd slots back (exact power-of-two scaling)
-        acc[nt][1][i] += acc16[nt][0][i] * 0.0625f;
-        acc[nt][3][i] += acc16[nt][1][i] * 0.0625f;
-      }
+        for (int i = 0; i < 4; ++i) {  // the 16x-scaled odd slots back (exact power-of-two scaling)
+          acc[nt][1][i] *= 0.0625f;
+          acc[nt][3][i] *= 0.0625f;
+        }
+    }
 
     if (KQ > 1) {
       // split K: this unit's partial sums go to partials[kq][row][column];
       // a second kernel sums the splits in kq order and finishes the outputs
       float *prow = p.partials + ((int64_t)ui.kq * p.A + ui.r0 + tok0) * ncols;
-      if (wc_ok) {
+      if (wc_ok && unit_ok) {
         const int64_t col0 = (int64_t)jw * p.N + wc * 8;
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt)
@@ -413,12 +408,25 @@ __global__ void __launch_bounds__(stream::kThreads, 2)
     for (int v8 = threadIdx.x; v8 < mrows * (kOut / 8); v8 += kCW * 32) {
       const int tk = v8 / (kOut / 8), fq = (v8 % (kOut / 8)) * 8;
       const int64_t n0 = (int64_t)ui.sl * kOut + fq;
-      if (n0 >= p.N) continue;
+      if (n0 >= p.N || !unit_ok) continue;
       const float *g8 = red + tk * kF + fq;
       finish8<NPROJ>(p, e, ui.r0 + tok0 + tk, n0, g8, g8 + 256);
     }
     named_barrier(1, kCW * 32);  // red is free again
   }
+  if (act_bad) report(p.status, MOE_DEVICE_ERR_ACT_RANGE);
+#ifdef MOE_TEST_HOOKS
+  // Test build only: one consumer thread waits, after every stage and
+  // activation tile of its CTA has landed (each was waited for above), on a
+  // phase that nothing completes, with a 1 ms limit, so a test can watch a
+  // bounded wait give up and report MOE_DEVICE_ERR_TIMEOUT.
+  if (p.test_stall && warp == 0 && lane == 0) {
+    const uint64_t t0 = global_ns();
+    bool done = false;
+    while (!done && global_ns() - t0 < 1000000ull) done = mbar_try_wait(stall, 0);
+    if (!done) report(p.status, MOE_DEVICE_ERR_TIMEOUT);
+  }
+#endif
 }
 
 // Split-K reduction: out[r, n..n+8) from sum over kq of partials[kq][r][.]
@@ -497,8 +505,22 @@ StreamPlan stream_plan(int64_t A, int64_t K, int64_t N, int64_t E, int64_t group
   return pl;
 }
 
+#ifdef MOE_TEST_HOOKS
+// Test build only: arms the stall of the next streaming-tile launches.
+static int g_test_stall = 0;
+extern "C" __attribute__((visibility("default"))) int32_t moe_test_arm_stall(int32_t on) {
+  const int prev = g_test_stall;
+  g_test_stall = on ? 1 : 0;
+  return prev;
+}
+#endif
+
 template <typename MT, int NPROJ, int NT, int ROWS>
-static moe_status launch_stream_r(const ProjParams &p, cudaStream_t st) {
+static moe_status launch_stream_r(const ProjParams &p0, cudaStream_t st) {
+  ProjParams p = p0;
+#ifdef MOE_TEST_HOOKS
+  p.test_stall = g_test_stall;
+#endif
   using namespace stream;
   constexpr int kRows = Geo<ROWS>::kRows;
   CUtensorMap m0, m1;

@@ -71,7 +71,8 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
   uint64_t *empty = bready + kStages;
   uint64_t *accfull = empty + kStages;  // [2]
   uint64_t *accempty = accfull + 2;     // [2]
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(accempty + 2);
+  uint64_t *drain = accempty + 2;       // the issuer's last commit: no MMA in flight at teardown
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
   volatile int32_t *abort = reinterpret_cast<volatile int32_t *>(tmem_slot + 1);
   int32_t *pre = reinterpret_cast<int32_t *>(tmem_slot + 4);  // [E + 1]
   int32_t *cnt = pre + (p.E + 1);                             // [E]
@@ -94,6 +95,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
       mbar_init(&accfull[b], 1);
       mbar_init(&accempty[b], kEpWarps);
     }
+    mbar_init(drain, 1);
     *abort = 0;
     fence_mbar_init();
   }
@@ -137,27 +139,47 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 0) {
-    // ---------------- producer
-    if (lane == 0) {
-      uint32_t it = 0;
-      for (int64_t tile = blockIdx.x; tile < total; tile += gridDim.x) {
+    // ---------------- producer (lane 0; with a gather, every lane loads
+    // four rows of the activation tile through tile::gather4)
+    const bool gather = p.gather != nullptr;
+    if (gather || lane == 0) {
+      uint32_t it = 0;  // stages issued
+      bool live = true;
+      for (int64_t tile = blockIdx.x; tile < total && live; tile += gridDim.x) {
         const TileInfo ti = tile_info(tile);
         const int32_t row0 = (int32_t)(ti.r0 + (int64_t)ti.mt * kBM);
+        int32_t src[4] = {0, 0, 0, 0};  // x rows of tile rows 4 lane .. 4 lane + 3 (rows past the batch: any row)
+        if (gather) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i) src[i] = (int32_t)act_row(p, min((int64_t)row0 + 4 * lane + i, p.A - 1));
+        }
         for (int kb = 0; kb < nk; ++kb, ++it) {
           const uint32_t s = it % kStages, use = it / kStages;
-          if (use > 0) tc_wait(&empty[s], (use - 1) & 1, p.status, abort);
+          bool ok = true;
           uint8_t *st = stages + s * kStageBytes;
-          mbar_arrive_expect_tx(&full[s], kABytes + kPBytes);
-          tma_load_2d(st, &map_x, &full[s], kb * kBK, row0);
-          const int32_t wrow = (int32_t)(ti.e * K + (int64_t)kb * kBK);
-          if (NPROJ == 2) {
-            tma_load_2d(st + kABytes + kBBytes, &map_w0, &full[s], ti.nt * 16, wrow);
-            tma_load_2d(st + kABytes + kBBytes + kPBytes / 2, &map_w1, &full[s], ti.nt * 16, wrow);
-          } else {
-            tma_load_2d(st + kABytes + kBBytes, &map_w0, &full[s], ti.nt * 32, wrow);
+          if (lane == 0) {
+            ok = use == 0 || tc_wait(&empty[s], (use - 1) & 1, p.status, abort);
+            if (ok) mbar_arrive_expect_tx(&full[s], kABytes + kPBytes);
+          }
+          if (gather) ok = __shfl_sync(0xffffffffu, ok, 0);
+          if (!ok) {
+            live = false;
+            break;
+          }
+          if (gather) tma_gather4(st + 4 * lane * 128, &map_x, &full[s], kb * kBK, src[0], src[1], src[2], src[3]);
+          if (lane == 0) {
+            if (!gather) tma_load_2d(st, &map_x, &full[s], kb * kBK, row0);
+            const int32_t wrow = (int32_t)(ti.e * K + (int64_t)kb * kBK);
+            if (NPROJ == 2) {
+              tma_load_2d(st + kABytes + kBBytes, &map_w0, &full[s], ti.nt * 16, wrow);
+              tma_load_2d(st + kABytes + kBBytes + kPBytes / 2, &map_w1, &full[s], ti.nt * 16, wrow);
+            } else {
+              tma_load_2d(st + kABytes + kBBytes, &map_w0, &full[s], ti.nt * 32, wrow);
+            }
           }
         }
       }
+      if (lane == 0) tma_drain(full, it, kStages, p.status);
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer: tile t accumulates in TMEM buffer t & 1
@@ -167,15 +189,18 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
       const uint32_t idesc = (1u << 4) | (fmt << 7) | (fmt << 10) | (1u << 16) | ((uint32_t)(kBN >> 3) << 17) |
                              ((uint32_t)(kBM >> 4) << 24);
       uint32_t it = 0, tcount = 0;
+      bool live = true;
       for (int64_t tile = blockIdx.x; tile < total; tile += gridDim.x, ++tcount) {
         const uint32_t buf = tcount & 1, use = tcount >> 1;
-        if (use > 0) tc_wait(&accempty[buf], (use - 1) & 1, p.status, abort);
+        if (use > 0 && !tc_wait(&accempty[buf], (use - 1) & 1, p.status, abort)) break;
         tc_fence_after();
         const uint32_t dacc = tmem + buf * kBN;
         for (int kb = 0; kb < nk; ++kb, ++it) {
           const uint32_t s = it % kStages, ph = (it / kStages) & 1;
-          tc_wait(&full[s], ph, p.status, abort);
-          tc_wait(&bready[s], ph, p.status, abort);
+          if (!tc_wait(&full[s], ph, p.status, abort) || !tc_wait(&bready[s], ph, p.status, abort)) {
+            live = false;
+            break;
+          }
           tc_fence_after();
           const uint32_t a_addr = smem_u32(stages + s * kStageBytes);
           const uint32_t b_addr = a_addr + kABytes;
@@ -186,8 +211,11 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
             umma_f16(dacc, adesc + (uint64_t)(2 * j), bdesc + (uint64_t)(128 * j), idesc, (kb | j) != 0);
           umma_commit(&empty[s]);
         }
+        if (!live) break;
         umma_commit(&accfull[buf]);
       }
+      umma_commit(drain);  // arrives once every MMA issued above has completed
+      mbar_wait(drain, 0, p.status);
     }
   } else if (warp < 2 + kDqWarps) {
     // ---------------- dequant warps
@@ -206,9 +234,11 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
     // B: features col*8 .. col*8+7 -> 64-column block col/8, 16-byte chunk col%8 XOR row%8
     const int b0 = (col >> 3) * 8192 + rg * 128 + (((col & 7) ^ rg) << 4);  // + 1 KB per 8 rows
     const int spg = p.group / kBK;  // steps per group
+    uint32_t act_bad = 0;  // a converted input outside F16's normal range
     const bool convert = p.act_dt != (std::is_same<MT, __half>::value ? MOE_F16 : MOE_BF16);
     uint32_t it = 0;
-    for (int64_t tile = blockIdx.x; tile < total; tile += gridDim.x) {
+    bool live = true;
+    for (int64_t tile = blockIdx.x; tile < total && live; tile += gridDim.x) {
       const TileInfo ti = tile_info(tile);
       const int64_t wc = NPROJ == 2 ? (int64_t)ti.nt * 16 + (col & 15) : (int64_t)ti.nt * 32 + col;
       const bool wc_ok = wc < NW;
@@ -238,7 +268,10 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
           gstage = 0;
           ++grp;
         }
-        tc_wait(&full[s], ph, p.status, abort);
+        if (!tc_wait(&full[s], ph, p.status, abort)) {
+          live = false;
+          break;
+        }
         uint8_t *st = stages + s * kStageBytes;
         if (convert) {
           // activation tile to the scale dtype, in place (layout-agnostic)
@@ -246,10 +279,10 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
 #pragma unroll
           for (int i = 0; i < kABytes / 16 / 256; ++i) {
             uint4 v = a4[td + 256 * i];
-            v.x = act_pair_to_mt<MT>(v.x, p.act_dt);
-            v.y = act_pair_to_mt<MT>(v.y, p.act_dt);
-            v.z = act_pair_to_mt<MT>(v.z, p.act_dt);
-            v.w = act_pair_to_mt<MT>(v.w, p.act_dt);
+            v.x = act_pair_to_mt<MT>(v.x, p.act_dt, act_bad);
+            v.y = act_pair_to_mt<MT>(v.y, p.act_dt, act_bad);
+            v.z = act_pair_to_mt<MT>(v.z, p.act_dt, act_bad);
+            v.w = act_pair_to_mt<MT>(v.w, p.act_dt, act_bad);
             a4[td + 256 * i] = v;
           }
         }
@@ -272,6 +305,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
         if (lane == 0) mbar_arrive(&bready[s]);
       }
     }
+    if (act_bad) report(p.status, MOE_DEVICE_ERR_ACT_RANGE);
   } else {
     // ---------------- epilogue warps: TMEM -> registers -> bias, rounding, SwiGLU -> HBM
     const int q = warp & 3;                          // TMEM lane quarter of this warp
@@ -280,7 +314,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
     for (int64_t tile = blockIdx.x; tile < total; tile += gridDim.x, ++tcount) {
       const TileInfo ti = tile_info(tile);
       const uint32_t buf = tcount & 1;
-      tc_wait(&accfull[buf], (tcount >> 1) & 1, p.status, abort);
+      if (!tc_wait(&accfull[buf], (tcount >> 1) & 1, p.status, abort)) break;
       tc_fence_after();
       const int trow = ti.mt * kBM + 32 * q + lane;  // row within the expert
       const bool row_ok = trow < ti.m && !*abort;
@@ -346,7 +380,12 @@ static moe_status launch_tc_t(const ProjParams &p, cudaStream_t st) {
   CUtensorMap mx, m0, m1;
   const uint64_t NW = p.N / 8, rows = (uint64_t)p.E * p.K;
   const uint32_t box_w = NPROJ == 2 ? 16 : 32;
-  if (!make_map_2d(&mx, p.x, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, p.K, p.A, kBK, kBM, CU_TENSOR_MAP_SWIZZLE_128B) ||
+  // the activation map: 128-row boxes of the batch, or one-row boxes of x for tile::gather4
+  const bool mx_ok = p.gather ? make_map_2d(&mx, p.x, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, p.K, p.T, kBK, 1,
+                                            CU_TENSOR_MAP_SWIZZLE_128B)
+                              : make_map_2d(&mx, p.x, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, p.K, p.A, kBK, kBM,
+                                            CU_TENSOR_MAP_SWIZZLE_128B);
+  if (!mx_ok ||
       !make_map_2d(&m0, p.qw[0], CU_TENSOR_MAP_DATA_TYPE_INT32, 4, NW, rows, box_w, kBK, CU_TENSOR_MAP_SWIZZLE_NONE) ||
       !make_map_2d(&m1, p.qw[NPROJ - 1], CU_TENSOR_MAP_DATA_TYPE_INT32, 4, NW, rows, box_w, kBK,
                    CU_TENSOR_MAP_SWIZZLE_NONE))

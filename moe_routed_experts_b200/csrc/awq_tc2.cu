@@ -77,7 +77,8 @@ __global__ void __launch_bounds__(tc2::kThreads, 1)
   uint64_t *bfree = bready + kBStages;
   uint64_t *accfull = bfree + kBStages;  // [2]
   uint64_t *accempty = accfull + 2;      // [2], used in CTA 0 (both CTAs' epilogues)
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(accempty + 2);
+  uint64_t *drain = accempty + 2;        // the issuer's last commit: no MMA in flight at teardown
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
   volatile int32_t *abort = reinterpret_cast<volatile int32_t *>(tmem_slot + 1);
   int32_t *pre = reinterpret_cast<int32_t *>(tmem_slot + 4);  // [E + 1]
   int32_t *cnt = pre + (p.E + 1);                             // [E]
@@ -105,6 +106,7 @@ __global__ void __launch_bounds__(tc2::kThreads, 1)
       mbar_init(&accfull[b], 1);
       mbar_init(&accempty[b], 2 * kEpWarps);
     }
+    mbar_init(drain, 1);
     *abort = 0;
     fence_mbar_init();
   }
@@ -149,23 +151,50 @@ __global__ void __launch_bounds__(tc2::kThreads, 1)
 
   if (warp == 0) {
     // ---------------- producer: this CTA's activation rows and packed half
-    if (lane == 0) {
+    // (lane 0; with a gather, every lane loads four rows of each activation
+    // atom through tile::gather4)
+    const bool gather = p.gather != nullptr;
+    if (gather || lane == 0) {
       const CUtensorMap *mw = (NPROJ == 2 && rank == 1) ? &map_w1 : &map_w0;
-      uint32_t it = 0;
-      for (int64_t tile = pair; tile < total; tile += npairs) {
+      uint32_t it = 0;  // stages issued
+      bool live = true;
+      for (int64_t tile = pair; tile < total && live; tile += npairs) {
         const PairTile ti = tile_info(tile);
         const int32_t row0 = (int32_t)(ti.r0 + (int64_t)ti.mt * 2 * kBM + kBM * rank);
         const int32_t wcol = NPROJ == 2 ? ti.nt * 16 : ti.nt * 32 + 16 * (int)rank;
+        int32_t src[4] = {0, 0, 0, 0};  // x rows of tile rows 4 lane .. 4 lane + 3 (rows past the batch: any row)
+        if (gather) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i) src[i] = (int32_t)act_row(p, min((int64_t)row0 + 4 * lane + i, p.A - 1));
+        }
         for (int kb = 0; kb < nk; ++kb, ++it) {
           const uint32_t s = it % kLStages, use = it / kLStages;
-          if (use > 0) tc_wait(&lempty[s], (use - 1) & 1, p.status, abort);
+          bool ok = true;
           uint8_t *st = lring + s * kLBytes;
-          mbar_arrive_expect_tx(&lfull[s], kLBytes);
-          tma_load_2d(st, &map_x, &lfull[s], kb * kBK, row0);
-          tma_load_2d(st + kAtom, &map_x, &lfull[s], kb * kBK + 64, row0);
-          tma_load_2d(st + kABytes, mw, &lfull[s], wcol, (int32_t)(ti.e * K + (int64_t)kb * kBK));
+          if (lane == 0) {
+            ok = use == 0 || tc_wait(&lempty[s], (use - 1) & 1, p.status, abort);
+            if (ok) mbar_arrive_expect_tx(&lfull[s], kLBytes);
+          }
+          if (gather) ok = __shfl_sync(0xffffffffu, ok, 0);
+          if (!ok) {
+            live = false;
+            break;
+          }
+          if (gather) {
+            tma_gather4(st + 4 * lane * 128, &map_x, &lfull[s], kb * kBK, src[0], src[1], src[2], src[3]);
+            tma_gather4(st + kAtom + 4 * lane * 128, &map_x, &lfull[s], kb * kBK + 64, src[0], src[1], src[2],
+                        src[3]);
+          }
+          if (lane == 0) {
+            if (!gather) {
+              tma_load_2d(st, &map_x, &lfull[s], kb * kBK, row0);
+              tma_load_2d(st + kAtom, &map_x, &lfull[s], kb * kBK + 64, row0);
+            }
+            tma_load_2d(st + kABytes, mw, &lfull[s], wcol, (int32_t)(ti.e * K + (int64_t)kb * kBK));
+          }
         }
       }
+      if (lane == 0) tma_drain(lfull, it, kLStages, p.status);
     }
   } else if (warp == 1) {
     // ---------------- pair MMA issuer (CTA 0 only)
@@ -175,15 +204,19 @@ __global__ void __launch_bounds__(tc2::kThreads, 1)
       const uint32_t idesc = (1u << 4) | (fmt << 7) | (fmt << 10) | (1u << 16) | ((uint32_t)(kBN >> 3) << 17) |
                              ((uint32_t)((2 * kBM) >> 4) << 24);
       uint32_t it = 0, tcount = 0;
+      bool live = true;
       for (int64_t tile = pair; tile < total; tile += npairs, ++tcount) {
         const uint32_t buf = tcount & 1, use = tcount >> 1;
-        if (use > 0) tc_wait_cluster(&accempty[buf], (use - 1) & 1, p.status, abort);
+        if (use > 0 && !tc_wait_cluster(&accempty[buf], (use - 1) & 1, p.status, abort)) break;
         tc_fence_after();
         const uint32_t dacc = tmem + buf * kBN;
         for (int kb = 0; kb < nk; ++kb, ++it) {
           const uint32_t ls = it % kLStages, bs = it % kBStages;
           // both CTAs' dequant warps arrive only after their own TMA stage landed
-          tc_wait_cluster(&bready[bs], (it / kBStages) & 1, p.status, abort);
+          if (!tc_wait_cluster(&bready[bs], (it / kBStages) & 1, p.status, abort)) {
+            live = false;
+            break;
+          }
           tc_fence_after();
           const uint32_t a_addr = smem_u32(lring + ls * kLBytes);
           const uint64_t bdesc = smem_desc(smem_u32(bring + bs * kBBytes), kNBlock, 1024);
@@ -194,9 +227,12 @@ __global__ void __launch_bounds__(tc2::kThreads, 1)
           umma2_commit_both(&lempty[ls]);
           umma2_commit_both(&bfree[bs]);
         }
+        if (!live) break;
         umma2_commit_both(&accfull[buf]);
       }
+      umma2_commit_both(drain);  // arrives in both CTAs once every MMA issued above has completed
     }
+    if (lane == 0) mbar_wait(drain, 0, p.status);
   } else if (warp < 2 + kDqWarps) {
     // ---------------- dequant warps: this CTA's 128-column half of B
     const int td = threadIdx.x - 64;  // 0 .. 32 kDqWarps - 1
@@ -212,10 +248,12 @@ __global__ void __launch_bounds__(tc2::kThreads, 1)
     // chunk col%8 XOR row%8 (MN-major, 128-byte swizzle, 8-row x 64-column atoms)
     const int b0 = (col >> 3) * kNBlock + (rg >> 3) * 1024 + (rg & 7) * 128 + (((col & 7) ^ (rg & 7)) << 4);
     const int spg = p.group / kBK;
+    uint32_t act_bad = 0;  // a converted input outside F16's normal range
     const bool convert = p.act_dt != (std::is_same<MT, __half>::value ? MOE_F16 : MOE_BF16);
     uint64_t *bready0 = bready;  // CTA 0's barriers, addressed through the cluster window
     uint32_t it = 0;
-    for (int64_t tile = pair; tile < total; tile += npairs) {
+    bool live = true;
+    for (int64_t tile = pair; tile < total && live; tile += npairs) {
       const PairTile ti = tile_info(tile);
       const int64_t wc = NPROJ == 2 ? (int64_t)ti.nt * 16 + col : (int64_t)ti.nt * 32 + 16 * rank + col;
       const bool wc_ok = wc < NW;
@@ -245,7 +283,10 @@ __global__ void __launch_bounds__(tc2::kThreads, 1)
           gstage = 0;
           ++grp;
         }
-        tc_wait(&lfull[ls], (it / kLStages) & 1, p.status, abort);
+        if (!tc_wait(&lfull[ls], (it / kLStages) & 1, p.status, abort)) {
+          live = false;
+          break;
+        }
         uint8_t *st = lring + ls * kLBytes;
         uint32_t w[kWordsPerThread];
         {
@@ -258,17 +299,20 @@ __global__ void __launch_bounds__(tc2::kThreads, 1)
 #pragma unroll
           for (int i = 0; i < kABytes / 16 / (32 * kDqWarps); ++i) {
             uint4 v = a4[td + 32 * kDqWarps * i];
-            v.x = act_pair_to_mt<MT>(v.x, p.act_dt);
-            v.y = act_pair_to_mt<MT>(v.y, p.act_dt);
-            v.z = act_pair_to_mt<MT>(v.z, p.act_dt);
-            v.w = act_pair_to_mt<MT>(v.w, p.act_dt);
+            v.x = act_pair_to_mt<MT>(v.x, p.act_dt, act_bad);
+            v.y = act_pair_to_mt<MT>(v.y, p.act_dt, act_bad);
+            v.z = act_pair_to_mt<MT>(v.z, p.act_dt, act_bad);
+            v.w = act_pair_to_mt<MT>(v.w, p.act_dt, act_bad);
             a4[td + 32 * kDqWarps * i] = v;
           }
           fence_proxy_async_smem();
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&lempty[ls]);  // packed words read (the pair commit frees A)
-        if (buse > 0) tc_wait(&bfree[bs], (buse - 1) & 1, p.status, abort);
+        if (buse > 0 && !tc_wait(&bfree[bs], (buse - 1) & 1, p.status, abort)) {
+          live = false;
+          break;
+        }
         uint8_t *bt = bring + bs * kBBytes + b0;
 #pragma unroll
         for (int i = 0; i < kWordsPerThread; ++i) {
@@ -284,6 +328,7 @@ __global__ void __launch_bounds__(tc2::kThreads, 1)
         if (lane == 0) mbar_arrive_cluster(cluster_addr(&bready0[bs], 0));
       }
     }
+    if (act_bad) report(p.status, MOE_DEVICE_ERR_ACT_RANGE);
   } else {
     // ---------------- epilogue warps: this CTA's 128 rows of the tile
     const int q = warp & 3;                     // TMEM lane quarter
@@ -292,7 +337,7 @@ __global__ void __launch_bounds__(tc2::kThreads, 1)
     for (int64_t tile = pair; tile < total; tile += npairs, ++tcount) {
       const PairTile ti = tile_info(tile);
       const uint32_t buf = tcount & 1;
-      tc_wait(&accfull[buf], (tcount >> 1) & 1, p.status, abort);
+      if (!tc_wait(&accfull[buf], (tcount >> 1) & 1, p.status, abort)) break;
       tc_fence_after();
       const int trow = ti.mt * 2 * kBM + kBM * (int)rank + 32 * q + lane;
       const bool row_ok = trow < ti.m && !*abort;
@@ -356,7 +401,12 @@ static moe_status launch_tc2_t(const ProjParams &p, cudaStream_t st) {
   using namespace tc2;
   CUtensorMap mx, m0, m1;
   const uint64_t NW = p.N / 8, rows = (uint64_t)p.E * p.K;
-  if (!make_map_2d(&mx, p.x, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, p.K, p.A, 64, kBM, CU_TENSOR_MAP_SWIZZLE_128B) ||
+  // the activation map: 128-row boxes of the batch, or one-row boxes of x for tile::gather4
+  const bool mx_ok = p.gather ? make_map_2d(&mx, p.x, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, p.K, p.T, 64, 1,
+                                            CU_TENSOR_MAP_SWIZZLE_128B)
+                              : make_map_2d(&mx, p.x, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, p.K, p.A, 64, kBM,
+                                            CU_TENSOR_MAP_SWIZZLE_128B);
+  if (!mx_ok ||
       !make_map_2d(&m0, p.qw[0], CU_TENSOR_MAP_DATA_TYPE_INT32, 4, NW, rows, 16, kBK, CU_TENSOR_MAP_SWIZZLE_NONE) ||
       !make_map_2d(&m1, p.qw[NPROJ - 1], CU_TENSOR_MAP_DATA_TYPE_INT32, 4, NW, rows, 16, kBK,
                    CU_TENSOR_MAP_SWIZZLE_NONE))

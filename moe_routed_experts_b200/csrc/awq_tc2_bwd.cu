@@ -71,7 +71,8 @@ __global__ void __launch_bounds__(tc2b::kThreads, 1)
   uint64_t *bfree = bready + kBStages;
   uint64_t *accfull = bfree + kBStages;  // [2]
   uint64_t *accempty = accfull + 2;      // [2], used in CTA 0
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(accempty + 2);
+  uint64_t *drain = accempty + 2;        // the issuer's last commit: no MMA in flight at teardown
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
   volatile int32_t *abort = reinterpret_cast<volatile int32_t *>(tmem_slot + 1);
   int32_t *pre = reinterpret_cast<int32_t *>(tmem_slot + 4);  // [E + 1]
   int32_t *cnt = pre + (p.E + 1);                             // [E]
@@ -101,6 +102,7 @@ __global__ void __launch_bounds__(tc2b::kThreads, 1)
       mbar_init(&accfull[b], 1);
       mbar_init(&accempty[b], 2 * kEpWarps);
     }
+    mbar_init(drain, 1);
     *abort = 0;
     fence_mbar_init();
   }
@@ -146,8 +148,9 @@ __global__ void __launch_bounds__(tc2b::kThreads, 1)
   if (warp == 0) {
     // ---------------- producer: gradient rows, packed half, zero/scale rows
     if (lane == 0) {
-      uint32_t it = 0;
-      for (int64_t tile = pair; tile < total; tile += npairs) {
+      uint32_t it = 0;  // stages issued
+      bool live = true;
+      for (int64_t tile = pair; tile < total && live; tile += npairs) {
         const PairBwdTile ti = tile_info(tile);
         const int32_t row0 = (int32_t)(ti.r0 + (int64_t)ti.mt * 2 * kBM + kBM * rank);
         const int64_t kk0 = (int64_t)ti.ct * kBN + kHalf * rank;  // this CTA's first output column
@@ -155,7 +158,10 @@ __global__ void __launch_bounds__(tc2b::kThreads, 1)
         const int32_t grow = (int32_t)((ti.e * K + kk0) / p.group);
         for (int kb = 0; kb < nk; ++kb, ++it) {
           const uint32_t s = it % kLStages, use = it / kLStages;
-          if (use > 0) tc_wait(&lempty[s], (use - 1) & 1, p.status, abort);
+          if (use > 0 && !tc_wait(&lempty[s], (use - 1) & 1, p.status, abort)) {
+            live = false;
+            break;
+          }
           const int j = NPROJ == 2 ? kb / nkp : 0;
           const int32_t n0 = (kb - j * nkp) * kBK;
           uint8_t *st = lring + s * kLBytes;
@@ -168,6 +174,7 @@ __global__ void __launch_bounds__(tc2b::kThreads, 1)
           tma_load_2d(cs + kZBytes, &maps.sc[j], &lfull[s], n0, grow);
         }
       }
+      tma_drain(lfull, it, kLStages, p.status);
     }
   } else if (warp == 1) {
     // ---------------- pair MMA issuer (CTA 0 only)
@@ -177,14 +184,18 @@ __global__ void __launch_bounds__(tc2b::kThreads, 1)
       const uint32_t idesc =
           (1u << 4) | (fmt << 7) | (fmt << 10) | ((uint32_t)(kBN >> 3) << 17) | ((uint32_t)((2 * kBM) >> 4) << 24);
       uint32_t it = 0, tcount = 0;
+      bool live = true;
       for (int64_t tile = pair; tile < total; tile += npairs, ++tcount) {
         const uint32_t buf = tcount & 1, use = tcount >> 1;
-        if (use > 0) tc_wait_cluster(&accempty[buf], (use - 1) & 1, p.status, abort);
+        if (use > 0 && !tc_wait_cluster(&accempty[buf], (use - 1) & 1, p.status, abort)) break;
         tc_fence_after();
         const uint32_t dacc = tmem + buf * kBN;
         for (int kb = 0; kb < nk; ++kb, ++it) {
           const uint32_t ls = it % kLStages, bs = it % kBStages;
-          tc_wait_cluster(&bready[bs], (it / kBStages) & 1, p.status, abort);
+          if (!tc_wait_cluster(&bready[bs], (it / kBStages) & 1, p.status, abort)) {
+            live = false;
+            break;
+          }
           tc_fence_after();
           const uint32_t a_addr = smem_u32(lring + ls * kLBytes);
           const uint32_t b_addr = smem_u32(bring + bs * kBBytes);
@@ -196,9 +207,12 @@ __global__ void __launch_bounds__(tc2b::kThreads, 1)
           umma2_commit_both(&lempty[ls]);
           umma2_commit_both(&bfree[bs]);
         }
+        if (!live) break;
         umma2_commit_both(&accfull[buf]);
       }
+      umma2_commit_both(drain);  // arrives in both CTAs once every MMA issued above has completed
     }
+    if (lane == 0) mbar_wait(drain, 0, p.status);
   } else if (warp < 2 + kDqWarps) {
     // ---------------- dequant warps: 128 output columns x 16 words per step
     const int td = threadIdx.x - 64;  // 0..511
@@ -208,13 +222,18 @@ __global__ void __launch_bounds__(tc2b::kThreads, 1)
     // K-major B: row r at atom (wcol / 8), chunk (wcol % 8) XOR (r % 8)
     const int b0 = (wcol >> 3) * kBAtom + (rband >> 3) * 1024 + (rband & 7) * 128 + (((wcol & 7) ^ (rband & 7)) << 4);
     const int gshift = p.group >= kHalf ? 8 : 6;  // group row of band i: (32 i) >> gshift (groups 64 or >= 128)
+    uint32_t act_bad = 0;  // a converted input outside F16's normal range
     const bool convert = p.gdt != (std::is_same<MT, __half>::value ? MOE_F16 : MOE_BF16);
     uint64_t *bready0 = bready;
     uint32_t it = 0;
-    for (int64_t tile = pair; tile < total; tile += npairs) {
+    bool live = true;
+    for (int64_t tile = pair; tile < total && live; tile += npairs) {
       for (int kb = 0; kb < nk; ++kb, ++it) {
         const uint32_t ls = it % kLStages, bs = it % kBStages, buse = it / kBStages;
-        tc_wait(&lfull[ls], (it / kLStages) & 1, p.status, abort);
+        if (!tc_wait(&lfull[ls], (it / kLStages) & 1, p.status, abort)) {
+          live = false;
+          break;
+        }
         uint8_t *st = lring + ls * kLBytes;
         const uint32_t *pk = reinterpret_cast<const uint32_t *>(st + kABytes) + rband * 16 + wcol;
         const uint8_t *cs = st + kABytes + kPBytes;
@@ -231,17 +250,20 @@ __global__ void __launch_bounds__(tc2b::kThreads, 1)
 #pragma unroll
           for (int i = 0; i < kABytes / 16 / (32 * kDqWarps); ++i) {
             uint4 v = a4[td + 32 * kDqWarps * i];
-            v.x = act_pair_to_mt<MT>(v.x, p.gdt);
-            v.y = act_pair_to_mt<MT>(v.y, p.gdt);
-            v.z = act_pair_to_mt<MT>(v.z, p.gdt);
-            v.w = act_pair_to_mt<MT>(v.w, p.gdt);
+            v.x = act_pair_to_mt<MT>(v.x, p.gdt, act_bad);
+            v.y = act_pair_to_mt<MT>(v.y, p.gdt, act_bad);
+            v.z = act_pair_to_mt<MT>(v.z, p.gdt, act_bad);
+            v.w = act_pair_to_mt<MT>(v.w, p.gdt, act_bad);
             a4[td + 32 * kDqWarps * i] = v;
           }
           fence_proxy_async_smem();
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&lempty[ls]);  // packed words and constants read
-        if (buse > 0) tc_wait(&bfree[bs], (buse - 1) & 1, p.status, abort);
+        if (buse > 0 && !tc_wait(&bfree[bs], (buse - 1) & 1, p.status, abort)) {
+          live = false;
+          break;
+        }
         uint8_t *bt = bring + bs * kBBytes + b0;
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
@@ -260,6 +282,7 @@ __global__ void __launch_bounds__(tc2b::kThreads, 1)
         if (lane == 0) mbar_arrive_cluster(cluster_addr(&bready0[bs], 0));
       }
     }
+    if (act_bad) report(p.status, MOE_DEVICE_ERR_ACT_RANGE);
   } else {
     // ---------------- epilogue warps: this CTA's 128 rows, 256 output columns
     const int q = warp & 3;                     // TMEM lane quarter
@@ -269,7 +292,7 @@ __global__ void __launch_bounds__(tc2b::kThreads, 1)
     for (int64_t tile = pair; tile < total; tile += npairs, ++tcount) {
       const PairBwdTile ti = tile_info(tile);
       const uint32_t buf = tcount & 1;
-      tc_wait(&accfull[buf], (tcount >> 1) & 1, p.status, abort);
+      if (!tc_wait(&accfull[buf], (tcount >> 1) & 1, p.status, abort)) break;
       tc_fence_after();
       const int trow = ti.mt * 2 * kBM + kBM * (int)rank + 32 * q + lane;
       const bool row_ok = trow < ti.m && !*abort;

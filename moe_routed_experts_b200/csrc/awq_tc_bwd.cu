@@ -64,7 +64,8 @@ __global__ void __launch_bounds__(tcb::kThreads, 1)
   uint64_t *empty = bready + kStages;
   uint64_t *accfull = empty + kStages;  // [2]
   uint64_t *accempty = accfull + 2;     // [2]
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(accempty + 2);
+  uint64_t *drain = accempty + 2;       // the issuer's last commit: no MMA in flight at teardown
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
   volatile int32_t *abort = reinterpret_cast<volatile int32_t *>(tmem_slot + 1);
   int32_t *pre = reinterpret_cast<int32_t *>(tmem_slot + 4);  // [E + 1]
   int32_t *cnt = pre + (p.E + 1);                             // [E]
@@ -89,6 +90,7 @@ __global__ void __launch_bounds__(tcb::kThreads, 1)
       mbar_init(&accfull[b], 1);
       mbar_init(&accempty[b], kEpWarps);
     }
+    mbar_init(drain, 1);
     *abort = 0;
     fence_mbar_init();
   }
@@ -134,8 +136,9 @@ __global__ void __launch_bounds__(tcb::kThreads, 1)
   if (warp == 0) {
     // ---------------- producer
     if (lane == 0) {
-      uint32_t it = 0;
-      for (int64_t tile = blockIdx.x; tile < total; tile += gridDim.x) {
+      uint32_t it = 0;  // stages issued
+      bool live = true;
+      for (int64_t tile = blockIdx.x; tile < total && live; tile += gridDim.x) {
         const BwdTile ti = tile_info(tile);
         const int32_t row0 = (int32_t)(ti.r0 + (int64_t)ti.mt * kBM);
         const int64_t kk0 = (int64_t)ti.ct * kBN;
@@ -143,7 +146,10 @@ __global__ void __launch_bounds__(tcb::kThreads, 1)
         const int32_t grow = (int32_t)((ti.e * K + kk0) / p.group);
         for (int kb = 0; kb < nk; ++kb, ++it) {
           const uint32_t s = it % kStages, use = it / kStages;
-          if (use > 0) tc_wait(&empty[s], (use - 1) & 1, p.status, abort);
+          if (use > 0 && !tc_wait(&empty[s], (use - 1) & 1, p.status, abort)) {
+            live = false;
+            break;
+          }
           const int j = NPROJ == 2 ? kb / nkp : 0;
           const int32_t n0 = (kb - j * nkp) * kBK;
           uint8_t *st = stages + s * kStageBytes;
@@ -155,6 +161,7 @@ __global__ void __launch_bounds__(tcb::kThreads, 1)
           tma_load_2d(cs + kZBytes, &maps.sc[j], &full[s], n0, grow);
         }
       }
+      tma_drain(full, it, kStages, p.status);
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer
@@ -164,15 +171,18 @@ __global__ void __launch_bounds__(tcb::kThreads, 1)
       const uint32_t idesc =
           (1u << 4) | (fmt << 7) | (fmt << 10) | ((uint32_t)(kBN >> 3) << 17) | ((uint32_t)(kBM >> 4) << 24);
       uint32_t it = 0, tcount = 0;
+      bool live = true;
       for (int64_t tile = blockIdx.x; tile < total; tile += gridDim.x, ++tcount) {
         const uint32_t buf = tcount & 1, use = tcount >> 1;
-        if (use > 0) tc_wait(&accempty[buf], (use - 1) & 1, p.status, abort);
+        if (use > 0 && !tc_wait(&accempty[buf], (use - 1) & 1, p.status, abort)) break;
         tc_fence_after();
         const uint32_t dacc = tmem + buf * kBN;
         for (int kb = 0; kb < nk; ++kb, ++it) {
           const uint32_t s = it % kStages, ph = (it / kStages) & 1;
-          tc_wait(&full[s], ph, p.status, abort);
-          tc_wait(&bready[s], ph, p.status, abort);
+          if (!tc_wait(&full[s], ph, p.status, abort) || !tc_wait(&bready[s], ph, p.status, abort)) {
+            live = false;
+            break;
+          }
           tc_fence_after();
           const uint32_t a_addr = smem_u32(stages + s * kStageBytes);
           const uint64_t adesc = smem_desc(a_addr, 16, 1024);
@@ -182,8 +192,11 @@ __global__ void __launch_bounds__(tcb::kThreads, 1)
             umma_f16(dacc, adesc + (uint64_t)(2 * jj), bdesc + (uint64_t)(2 * jj), idesc, (kb | jj) != 0);
           umma_commit(&empty[s]);
         }
+        if (!live) break;
         umma_commit(&accfull[buf]);
       }
+      umma_commit(drain);  // arrives once every MMA issued above has completed
+      mbar_wait(drain, 0, p.status);
     }
   } else if (warp < 2 + kDqWarps) {
     // ---------------- dequant warps: 256 coefficient rows x 8 words per step
@@ -192,24 +205,29 @@ __global__ void __launch_bounds__(tcb::kThreads, 1)
     const int rband = td >> 3;        // rows rband + 32 i, i = 0..7
     constexpr uint32_t M = Dq<MT>::kMagic2;
     const int b0 = (rband >> 3) * 1024 + (rband & 7) * 128 + ((wcol ^ (rband & 7)) << 4);
+    uint32_t act_bad = 0;  // a converted input outside F16's normal range
     const bool convert = p.gdt != (std::is_same<MT, __half>::value ? MOE_F16 : MOE_BF16);
     // group row of band i = (32 i) / group; groups here are 64, 128 or >= 256 (one per tile)
     const int gshift = p.group >= kBN ? 8 : (p.group == 128 ? 7 : 6);
     uint32_t it = 0;
-    for (int64_t tile = blockIdx.x; tile < total; tile += gridDim.x) {
+    bool live = true;
+    for (int64_t tile = blockIdx.x; tile < total && live; tile += gridDim.x) {
       for (int kb = 0; kb < nk; ++kb, ++it) {
         const uint32_t s = it % kStages, ph = (it / kStages) & 1;
-        tc_wait(&full[s], ph, p.status, abort);
+        if (!tc_wait(&full[s], ph, p.status, abort)) {
+          live = false;
+          break;
+        }
         uint8_t *st = stages + s * kStageBytes;
         if (convert) {
           uint4 *a4 = reinterpret_cast<uint4 *>(st);
 #pragma unroll
           for (int i = 0; i < kABytes / 16 / 256; ++i) {
             uint4 v = a4[td + 256 * i];
-            v.x = act_pair_to_mt<MT>(v.x, p.gdt);
-            v.y = act_pair_to_mt<MT>(v.y, p.gdt);
-            v.z = act_pair_to_mt<MT>(v.z, p.gdt);
-            v.w = act_pair_to_mt<MT>(v.w, p.gdt);
+            v.x = act_pair_to_mt<MT>(v.x, p.gdt, act_bad);
+            v.y = act_pair_to_mt<MT>(v.y, p.gdt, act_bad);
+            v.z = act_pair_to_mt<MT>(v.z, p.gdt, act_bad);
+            v.w = act_pair_to_mt<MT>(v.w, p.gdt, act_bad);
             a4[td + 256 * i] = v;
           }
         }
@@ -249,6 +267,7 @@ __global__ void __launch_bounds__(tcb::kThreads, 1)
         if (lane == 0) mbar_arrive(&bready[s]);
       }
     }
+    if (act_bad) report(p.status, MOE_DEVICE_ERR_ACT_RANGE);
   } else {
     // ---------------- epilogue warps
     const int q = warp & 3;                     // TMEM lane quarter
@@ -258,7 +277,7 @@ __global__ void __launch_bounds__(tcb::kThreads, 1)
     for (int64_t tile = blockIdx.x; tile < total; tile += gridDim.x, ++tcount) {
       const BwdTile ti = tile_info(tile);
       const uint32_t buf = tcount & 1;
-      tc_wait(&accfull[buf], (tcount >> 1) & 1, p.status, abort);
+      if (!tc_wait(&accfull[buf], (tcount >> 1) & 1, p.status, abort)) break;
       tc_fence_after();
       const int trow = ti.mt * kBM + 32 * q + lane;
       const bool row_ok = trow < ti.m && !*abort;

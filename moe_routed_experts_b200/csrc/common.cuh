@@ -111,10 +111,26 @@ __device__ __forceinline__ uint32_t f16x2_to_bf16x2(uint32_t v) {
   return *reinterpret_cast<uint32_t *>(&b);
 }
 
+// Nonzero when a BF16 value of the pair lies outside F16's normal range
+// (|v| >= 65536, inf or NaN, or 0 < |v| < 2^-14): there BF16 -> F16 is not
+// exact (overflow to inf, or a subnormal with fewer significant bits).  BF16
+// has no values in (65504, 65536).
+__device__ __forceinline__ uint32_t bf16x2_outside_f16_normal(uint32_t v) {
+  const uint32_t lo = v & 0x7FFFu, hi = (v >> 16) & 0x7FFFu;
+  return (uint32_t)(lo >= 0x4780u) | (uint32_t)(lo - 1u < 0x387Fu) | (uint32_t)(hi >= 0x4780u) |
+         (uint32_t)(hi - 1u < 0x387Fu);
+}
+
+// Activation (or gradient) pair in the tensor-core operand dtype MT.  A
+// BF16 -> F16 conversion outside F16's normal range ORs 1 into `bad` (the
+// caller reports MOE_DEVICE_ERR_ACT_RANGE); F16 -> BF16 always fits the range
+// and rounds to BF16's 8 significant bits.
 template <typename MT>
-__device__ __forceinline__ uint32_t act_pair_to_mt(uint32_t v, int act_dt) {
+__device__ __forceinline__ uint32_t act_pair_to_mt(uint32_t v, int act_dt, uint32_t &bad) {
   if constexpr (sizeof(MT) == 2 && std::is_same<MT, __half>::value) {
-    return act_dt == MOE_BF16 ? bf16x2_to_f16x2(v) : v;
+    if (act_dt != MOE_BF16) return v;
+    bad |= bf16x2_outside_f16_normal(v);
+    return bf16x2_to_f16x2(v);
   } else {
     return act_dt == MOE_F16 ? f16x2_to_bf16x2(v) : v;
   }

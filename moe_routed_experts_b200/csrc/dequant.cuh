@@ -32,6 +32,38 @@ struct FwdConsts {
   }
 };
 
+// The same constants with fewer instructions, for the streaming tile: the
+// four zero-slot pairs come from one shift and four masks (odd slots read in
+// place when x16, 16 times larger, as the odd-slot codes are), and each
+// register is one byte permute of them under the magic number's high byte.
+template <typename MT>
+__device__ __forceinline__ void load_consts_fast(FwdConsts<MT> &c, uint32_t zw, uint4 sv, bool x16) {
+  constexpr uint32_t M = Dq<MT>::kMagic2;
+  const uint32_t z8 = zw >> 8;
+  uint32_t t4[4];
+  t4[0] = zw & 0x000F000Fu;
+  t4[1] = x16 ? (zw & 0x00F000F0u) : ((zw >> 4) & 0x000F000Fu);
+  t4[2] = z8 & 0x000F000Fu;
+  t4[3] = x16 ? (z8 & 0x00F000F0u) : ((zw >> 12) & 0x000F000Fu);
+  const uint32_t sw[4] = {sv.x, sv.y, sv.z, sv.w};
+#pragma unroll
+  for (int p = 0; p < 4; ++p) {
+    // byte 0 (slot p) or byte 2 (slot p + 4) of t4[p], under the magic's high byte (byte 5 of {t4, M})
+    c.zlo[p] = prmt(t4[p], M, 0x5050u);
+    c.zhi[p] = prmt(t4[p], M, 0x5252u);
+    c.slo[p] = prmt(sw[p], 0u, 0x1010u);
+    c.shi[p] = prmt(sw[p], 0u, 0x3232u);
+  }
+}
+
+// Nonzero if a scale of the F16 pair is outside {0} U [2^-14, 256] (where the
+// odd-slot shortcut of fwd_pairs16 would not be exact).
+__device__ __forceinline__ uint32_t f16_pair_blocks_x16(uint32_t w) {
+  const uint32_t lo = w & 0x7FFFu, hi = (w >> 16) & 0x7FFFu;
+  return (uint32_t)(lo > 0x5C00u) | (uint32_t)(hi > 0x5C00u) | (uint32_t)(lo - 1u < 0x03FFu) |
+         (uint32_t)(hi - 1u < 0x03FFu);
+}
+
 // Coefficient pairs of column 2p (lo) and 2p+1 (hi) at two consecutive input
 // rows, from the words wa (row kk) and wb (row kk+1) of the same column.
 template <typename MT>

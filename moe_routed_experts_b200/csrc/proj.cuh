@@ -6,7 +6,9 @@
 namespace moe {
 
 struct ProjParams {
-  const uint16_t *x;  // [A, K] activations
+  const uint16_t *x;  // [A, K] activations, or [T, K] read through `gather`
+  const int32_t *gather;  // NULL, or [A]: batch row r is x row gather[r] (in [0, T))
+  int64_t T;              // rows of x when gathering
   int act_dt;
   int64_t A, K, N;
   const int32_t *offsets;
@@ -25,6 +27,9 @@ struct ProjParams {
   float *partials;
   int32_t *counters;
   int kq;  // K splits
+#ifdef MOE_TEST_HOOKS
+  int test_stall;  // test build only: see moe_test_arm_stall
+#endif
 };
 
 struct BwdParams {
@@ -40,6 +45,18 @@ struct BwdParams {
   uint16_t *out;  // [A, K]
   int32_t *status;
 };
+
+// Row of x that batch row r reads: r itself, or gather[r] (an index outside
+// [0, T) is reported and row 0 is read instead).
+__device__ __forceinline__ int64_t act_row(const ProjParams &p, int64_t r) {
+  if (!p.gather) return r;
+  const int32_t v = __ldg(p.gather + r);
+  if (v < 0 || (int64_t)v >= p.T) {
+    report(p.status, MOE_DEVICE_ERR_ROW_RANGE);
+    return 0;
+  }
+  return v;
+}
 
 // 8 bias values n0.. of local expert e (0 without a bias), with 16-byte loads.
 __device__ __forceinline__ void bias8(const void *bias, int dt, int64_t i0, float (&b)[8]) {

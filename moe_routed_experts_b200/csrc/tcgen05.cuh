@@ -60,14 +60,6 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
   for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
 
-// Bounded wait that gives up at once after any timeout in the CTA (abort).
-__device__ __forceinline__ bool tc_wait(uint64_t *bar, uint32_t parity, int32_t *status, volatile int32_t *abort) {
-  if (*abort) return false;
-  if (mbar_wait(bar, parity, status)) return true;
-  *abort = 1;
-  return false;
-}
-
 // ---- CTA pair (cluster of two, cta_group::2)
 
 __device__ __forceinline__ uint32_t cluster_rank() {
@@ -118,6 +110,7 @@ __device__ __forceinline__ bool tc_wait_cluster(uint64_t *bar, uint32_t parity, 
   for (;;) {
     for (int i = 0; i < 32; ++i)
       if (mbar_try_wait_cluster(bar, parity)) return true;
+    if (*abort) return false;
     if (global_ns() - t0 > kWaitNs) break;
   }
   report(status, MOE_DEVICE_ERR_TIMEOUT);

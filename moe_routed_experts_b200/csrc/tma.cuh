@@ -73,6 +73,41 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, int32_
   return false;
 }
 
+// Abort protocol of the warp-specialised kernels (TMA producer, consumers,
+// and for tcgen05 an MMA issuer).  Every wait is
+// bounded; a wait that runs out reports MOE_DEVICE_ERR_TIMEOUT and sets the
+// CTA's abort flag, and a wait in progress elsewhere in the CTA gives up as
+// soon as it sees the flag.  A role whose wait fails leaves its loop at once,
+// so after an abort nothing issues another TMA copy, MMA, commit or barrier
+// arrival.  Before the CTA exits, the TMA producer waits (bounded) until
+// every stage it issued has landed, and the MMA issuer commits a drain
+// barrier that the TMEM owner waits on, so no asynchronous copy or MMA is in
+// flight when shared memory and TMEM are released.
+
+// Bounded wait that gives up after a timeout anywhere in the CTA (abort).
+__device__ __forceinline__ bool tc_wait(uint64_t *bar, uint32_t parity, int32_t *status, volatile int32_t *abort) {
+  if (*abort) return false;
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_ns();
+  for (;;) {
+    for (int i = 0; i < 32; ++i)
+      if (mbar_try_wait(bar, parity)) return true;
+    if (*abort) return false;
+    if (global_ns() - t0 > kWaitNs) break;
+  }
+  report(status, MOE_DEVICE_ERR_TIMEOUT);
+  *abort = 1;
+  return false;
+}
+
+// Waits (bounded, whatever the abort flag says) until the last `issued` TMA
+// stages of a ring of `stages` full-barriers have landed.  Stage j of the
+// issue order used barrier j % stages in phase j / stages.
+__device__ __forceinline__ void tma_drain(uint64_t *full, uint32_t issued, uint32_t stages, int32_t *status) {
+  const uint32_t first = issued > stages ? issued - stages : 0;
+  for (uint32_t j = first; j < issued; ++j) mbar_wait(&full[j % stages], (j / stages) & 1, status);
+}
+
 // 2-D tiled TMA load (no multicast) completing on `bar`.  c0 is the inner
 // coordinate; c0 * element size must be a multiple of 16 bytes.
 __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, uint64_t *bar, int32_t c0, int32_t c1) {
@@ -80,6 +115,18 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, u
       "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];" ::"r"(
           smem_u32(dst)),
       "l"(map), "r"(smem_u32(bar)), "r"(c0), "r"(c1)
+      : "memory");
+}
+
+// Four rows r0..r3 of a 2-D tensor map whose box is one row high, columns
+// c0 .. c0 + box width, into four consecutive box rows at dst (no
+// multicast); c0 * element size must be a multiple of 16 bytes.
+__device__ __forceinline__ void tma_gather4(void *dst, const CUtensorMap *map, uint64_t *bar, int32_t c0, int32_t r0,
+                                            int32_t r1, int32_t r2, int32_t r3) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, "
+      "%5, %6, %7}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(map), "r"(smem_u32(bar)), "r"(c0), "r"(r0), "r"(r1), "r"(r2), "r"(r3)
       : "memory");
 }
 

@@ -83,22 +83,33 @@ def alloc(w, device="cuda", keep_gu: bool = False) -> Buffers:
     return Buffers(route, ws, h, G, U, y, out, torch.zeros(1, dtype=torch.int32, device=device), proj_ws)
 
 
-def forward(dev: dict, buf: Buffers) -> torch.Tensor:
-    """One forward pass of the whole hot path into ``buf``; returns buf.out."""
+def forward(dev: dict, buf: Buffers, gather: bool = False) -> torch.Tensor:
+    """One forward pass of the whole hot path into ``buf``; returns buf.out.
+    gather: route without the COPY and let the gate/up projection read each
+    row from x through src_token (buf.route["values"] is then not written)."""
     w = dev["workload"]
-    r = B.moe_route_dispatch(dev["x"], dev["logits"], w.top_k, E=w.E, sel_bias=dev["sel_bias"],
-                             expert_start=w.expert_start, renormalize=w.renormalize, workspace=buf.workspace,
-                             device_status=buf.status, out=buf.route)
+    if gather:
+        r = B.moe_route(dev["logits"], w.top_k, E=w.E, sel_bias=dev["sel_bias"], expert_start=w.expert_start,
+                        renormalize=w.renormalize, workspace=buf.workspace, device_status=buf.status, out=buf.route)
+    else:
+        r = B.moe_route_dispatch(dev["x"], dev["logits"], w.top_k, E=w.E, sel_bias=dev["sel_bias"],
+                                 expert_start=w.expert_start, renormalize=w.renormalize, workspace=buf.workspace,
+                                 device_status=buf.status, out=buf.route)
     lib, st = B.lib(), B._stream()
     gate, up, down = dev["gate"], dev["up"], dev["down"]
     A = w.A
-    s = lib.awq_grouped_gate_up_swiglu(
-        B._ptr(r["values"]), B.MOE_BF16, A, w.H, w.I, B._ptr(r["offsets"]), w.E,
-        B._ptr(gate["qweight"]), B._ptr(gate["qzeros"]), B._ptr(gate["scales"]), B._ptr(gate["bias"]),
-        B._ptr(up["qweight"]), B._ptr(up["qzeros"]), B._ptr(up["scales"]), B._ptr(up["bias"]),
-        B._dt(gate["scales"].dtype), B.MOE_F32, w.group, B._ptr(buf.h), B._ptr(buf.G), B._ptr(buf.U),
-        B._ptr(buf.proj_ws), 0 if buf.proj_ws is None else buf.proj_ws.numel(), B._ptr(buf.status), st)
-    B._check("awq_grouped_gate_up_swiglu", s)
+    pay = (B._ptr(gate["qweight"]), B._ptr(gate["qzeros"]), B._ptr(gate["scales"]), B._ptr(gate["bias"]),
+           B._ptr(up["qweight"]), B._ptr(up["qzeros"]), B._ptr(up["scales"]), B._ptr(up["bias"]),
+           B._dt(gate["scales"].dtype), B.MOE_F32, w.group, B._ptr(buf.h), B._ptr(buf.G), B._ptr(buf.U),
+           B._ptr(buf.proj_ws), 0 if buf.proj_ws is None else buf.proj_ws.numel(), B._ptr(buf.status), st)
+    if gather:
+        s = lib.awq_grouped_gate_up_swiglu_gather(B._ptr(dev["x"]), B.MOE_BF16, w.T, B._ptr(r["src_token"]), A, w.H,
+                                                  w.I, B._ptr(r["offsets"]), w.E, *pay)
+        B._check("awq_grouped_gate_up_swiglu_gather", s)
+    else:
+        s = lib.awq_grouped_gate_up_swiglu(B._ptr(r["values"]), B.MOE_BF16, A, w.H, w.I, B._ptr(r["offsets"]), w.E,
+                                           *pay)
+        B._check("awq_grouped_gate_up_swiglu", s)
     s = lib.awq_grouped_down(
         B._ptr(buf.h), B.MOE_BF16, A, w.I, w.H, B._ptr(r["offsets"]), w.E, B._ptr(down["qweight"]),
         B._ptr(down["qzeros"]), B._ptr(down["scales"]), B._ptr(down["bias"]), B._dt(down["scales"].dtype),

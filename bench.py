@@ -152,6 +152,8 @@ def main():
     ap.add_argument("--no-graph", action="store_true", help="launch kernels directly instead of a CUDA graph")
     ap.add_argument("--soak-seconds", type=float, default=1.0)
     ap.add_argument("--reference-tokens", type=int, default=8)
+    ap.add_argument("--workloads", default="prefill,wide,skewed",
+                    help="other workloads timed in the same run, reported under 'workloads' ('none': skip)")
     ap.add_argument("--tokens", type=int, default=0,
                     help="override the workload's token count (smaller profiling captures); 0 keeps it")
     args = ap.parse_args()
@@ -183,13 +185,38 @@ def main():
         dist.barrier()
     B.lib()
 
+    line = measure(w, args, args.steps, world, rank, local, cpu=not args.no_cpu_baseline and world == 1)
+    extra = [] if args.workloads in ("", "none") else [n for n in args.workloads.split(",") if n != w.name]
+    if extra and rank == 0:
+        line["workloads"] = {}
+    for name in extra:
+        sub = measure(WORKLOADS[name], args, min(args.steps, 20), world, rank, local, cpu=False)
+        if rank == 0:
+            line["workloads"][name] = {k: sub[k] for k in (
+                "value", "unit", "ms_per_step", "fwd_ms", "bwd_ms", "tflops", "packed_weight_gbs",
+                "packed_weight_frac", "roofline", "e2e", "gpu_launches", "clocks", "device_status", "config", "steps")
+                if k in sub}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def measure(w, args, steps, world, rank, local, cpu):
+    """One workload: graph-replayed (forward-only) or direct steps, timed
+    with CUDA events under the L2-flush protocol; returns the JSON fields
+    (rank 0; other ranks return None after taking part in the max)."""
+    import torch
+    from moe_routed_experts_b200 import binding as B
+    from moe_routed_experts_b200 import ffn
+
     inp = inputs.generate(w)
     dev = ffn.to_device(inp)
     buf = ffn.alloc(w, keep_gu=w.backward)
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
-    stream = torch.cuda.current_stream()
 
-    def step(record=None):
+    def step(record=None, parts=None):
         if record is not None:
             ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         r = B.moe_route_dispatch(dev["x"], dev["logits"], w.top_k, E=w.E, sel_bias=dev["sel_bias"],
@@ -210,6 +237,10 @@ def main():
         B.moe_combine(buf.y, r["weights"], r["selected_experts"], r["row_of"], device_status=buf.status,
                       out=buf.out)
         if w.backward:
+            if parts is not None:
+                mid = torch.cuda.Event(enable_timing=True)
+                mid.record()
+                parts.append(mid)
             ffn.backward(dev, buf, dev["d_out"])
 
     for _ in range(args.warmup):
@@ -229,11 +260,11 @@ def main():
         torch.cuda.current_stream().wait_stream(s)
         torch.cuda.synchronize()
 
-    def run_step():
+    def run_step(parts=None):
         if graph is not None:
             graph.replay()
         else:
-            step()
+            step(parts=parts)
 
     bus = None
     try:
@@ -251,25 +282,31 @@ def main():
         torch.cuda.synchronize()
 
     # timed region: K steps, events per step, L2 flush between steps outside the events
+    import torch.distributed as dist
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    for i in range(args.steps):
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    mids = []
+    for i in range(steps):
         flush.fill_(i & 0xFF)
         starts[i].record()
-        run_step()
+        run_step(parts=mids if w.backward else None)
         ends[i].record()
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
     ms = sum(step_ms) / len(step_ms)
+    fwd_ms = bwd_ms = None
+    if w.backward:
+        fwd_ms = sum(s.elapsed_time(m) for s, m in zip(starts, mids)) / steps
+        bwd_ms = sum(m.elapsed_time(e) for m, e in zip(mids, ends)) / steps
 
     # dominant kernel duration (direct launches, same flush protocol)
     k_ms = []
-    for i in range(min(args.steps, 50)):
+    for i in range(min(steps, 50)):
         flush.fill_(i & 0xFF)
         rec = []
         step(record=rec)
@@ -278,7 +315,7 @@ def main():
     kernel_ms = statistics.median(k_ms)
     # a plain-launch time of the whole step (no graph), for context
     nog = []
-    for i in range(min(args.steps, 50)):
+    for i in range(min(steps, 50)):
         flush.fill_(i & 0xFF)
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record()
@@ -293,73 +330,79 @@ def main():
     l_host = torch.from_numpy(inp["logits"]).pin_memory()
     out_host = torch.empty(buf.out.shape, dtype=buf.out.dtype).pin_memory()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    n_e2e = args.steps
     torch.cuda.synchronize()
     e0.record()
-    for i in range(n_e2e):
+    for i in range(steps):
         dev["x"].copy_(x_host, non_blocking=True)
         dev["logits"].copy_(l_host, non_blocking=True)
         run_step()
         out_host.copy_(buf.out, non_blocking=True)
     e1.record()
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1) / n_e2e
+    e2e_ms = e0.elapsed_time(e1) / steps
     clocks = sampler.stop()
     status = int(buf.status.item())
 
-    ms, e2e_ms, kernel_ms = max_over_ranks([ms, e2e_ms, kernel_ms], "cuda")
+    vals = [ms, e2e_ms, kernel_ms] + ([fwd_ms, bwd_ms] if w.backward else [])
+    vals = max_over_ranks(vals, "cuda")
+    ms, e2e_ms, kernel_ms = vals[:3]
+    if w.backward:
+        fwd_ms, bwd_ms = vals[3:]
+    if rank != 0:
+        return None
 
-    if rank == 0:
-        offsets = buf.route["offsets"].cpu().numpy()
-        counts = np.diff(offsets)
-        pk = peaks()
-        kname = gate_up_kernel_name(B, w)
-        if w.name in ("decode", "tiny"):
-            alg = packed_bytes(inp, counts, ("gate", "up"))
-            achieved = alg / (kernel_ms * 1e-3) / 1e9
-            roof = {"bound": "hbm", "kernel": kname, "achieved": achieved,
-                    "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": achieved / pk["hbm_gbs"],
-                    "traffic": traffic_for("gate_up_" + w.name), "algorithmic_bytes": alg,
-                    "kernel_ms": kernel_ms, "peak_source": pk["source"]}
-        else:
-            flops = 2.0 * w.A * w.H * 2 * w.I
-            achieved = flops / (kernel_ms * 1e-3) / 1e12
-            roof = {"bound": "tensor", "kernel": kname, "achieved": achieved,
-                    "peak": pk["bf16_tflops"], "unit": "TFLOP/s", "frac": achieved / pk["bf16_tflops"],
-                    "traffic": traffic_for("gate_up_" + w.name), "algorithmic_flops": flops,
-                    "kernel_ms": kernel_ms, "peak_source": pk["source"] + " burst"}
-        all_packed = packed_bytes(inp, counts, ("gate", "up", "down"))
-        fwd_flops = 2.0 * w.A * 3 * w.H * w.I
-        launches_per_step = launches_per_step_of(B, w)
-        line = {
-            "metric": METRIC, "value": world * w.T / (ms * 1e-3), "unit": "tokens/s", "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None,
-            "dtype": "f16" if w.scale_dtype == "f16" else "bf16", "data": "synthetic",
-            "config": {"workload": w.name, "T": w.T, "H": w.H, "I": w.I, "E": w.E, "top_k": w.top_k,
-                       "group": w.group, "scale_dtype": w.scale_dtype, "activations": "bf16",
-                       "mma": "%s x %s -> f32" % (w.scale_dtype, w.scale_dtype), "backward": w.backward,
-                       "parallelism": "replicas x%d" % world, "graph": graph is not None,
-                       "l2": "256 MiB flush between steps, outside the per-step events",
-                       "experts_touched": int((counts > 0).sum())},
-            "packed_weight_gbs": all_packed / (ms * 1e-3) / 1e9,
-            "packed_weight_frac": all_packed / (ms * 1e-3) / 1e9 / pk["hbm_gbs"],
-            "tflops": fwd_flops / (ms * 1e-3) / 1e12,
-            "no_graph_ms_per_step": nograph_ms,
-            "roofline": roof,
-            "e2e": {"value": world * w.T / (e2e_ms * 1e-3), "unit": "tokens/s",
-                    "h2d_bytes_per_step": int(x_host.numel() * 2 + l_host.numel() * 4),
-                    "d2h_bytes_per_step": int(out_host.numel() * 2)},
-            "gpu_launches": launches_per_step * args.steps,
-            "clocks": clocks,
-            "device_status": status,
-        }
-        if not args.no_cpu_baseline and world == 1:
-            line["cpu_baseline"] = cpu_baseline(inp, w)
-        print(json.dumps(line), flush=True)
-    if world > 1:
-        dist.barrier()
-        dist.destroy_process_group()
+    offsets = buf.route["offsets"].cpu().numpy()
+    counts = np.diff(offsets)
+    pk = peaks()
+    kname = gate_up_kernel_name(B, w)
+    if w.name in ("decode", "tiny"):
+        alg = packed_bytes(inp, counts, ("gate", "up"))
+        achieved = alg / (kernel_ms * 1e-3) / 1e9
+        roof = {"bound": "hbm", "kernel": kname, "achieved": achieved,
+                "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": achieved / pk["hbm_gbs"],
+                "traffic": traffic_for("gate_up_" + w.name), "algorithmic_bytes": alg,
+                "kernel_ms": kernel_ms, "peak_source": pk["source"]}
+    else:
+        flops = 2.0 * w.A * w.H * 2 * w.I
+        achieved = flops / (kernel_ms * 1e-3) / 1e12
+        roof = {"bound": "tensor", "kernel": kname, "achieved": achieved,
+                "peak": pk["bf16_tflops"], "unit": "TFLOP/s", "frac": achieved / pk["bf16_tflops"],
+                "traffic": traffic_for("gate_up_" + w.name), "algorithmic_flops": flops,
+                "kernel_ms": kernel_ms, "peak_source": pk["source"] + " burst"}
+    all_packed = packed_bytes(inp, counts, ("gate", "up", "down"))
+    fwd_flops = 2.0 * w.A * 3 * w.H * w.I
+    launches_per_step = launches_per_step_of(B, w)
+    line = {
+        "metric": METRIC, "value": world * w.T / (ms * 1e-3), "unit": "tokens/s", "n_gpus": world,
+        "steps": steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None,
+        "dtype": "f16" if w.scale_dtype == "f16" else "bf16", "data": "synthetic",
+        "config": {"workload": w.name, "T": w.T, "H": w.H, "I": w.I, "E": w.E, "top_k": w.top_k,
+                   "group": w.group, "scale_dtype": w.scale_dtype, "activations": "bf16",
+                   "mma": "%s x %s -> f32" % (w.scale_dtype, w.scale_dtype), "backward": w.backward,
+                   "parallelism": "replicas x%d" % world, "graph": graph is not None,
+                   "l2": "256 MiB flush between steps, outside the per-step events",
+                   "experts_touched": int((counts > 0).sum())},
+        "packed_weight_gbs": all_packed / (ms * 1e-3) / 1e9,
+        "packed_weight_frac": all_packed / (ms * 1e-3) / 1e9 / pk["hbm_gbs"],
+        "tflops": fwd_flops * (2 if w.backward else 1) / (ms * 1e-3) / 1e12,
+        "no_graph_ms_per_step": nograph_ms,
+        "roofline": roof,
+        "e2e": {"value": world * w.T / (e2e_ms * 1e-3), "unit": "tokens/s",
+                "h2d_bytes_per_step": int(x_host.numel() * 2 + l_host.numel() * 4),
+                "d2h_bytes_per_step": int(out_host.numel() * 2)},
+        "gpu_launches": launches_per_step * steps,
+        "clocks": clocks,
+        "device_status": status,
+    }
+    if w.backward:
+        line["fwd_ms"] = fwd_ms
+        line["bwd_ms"] = bwd_ms
+    if cpu:
+        line["cpu_baseline"] = cpu_baseline(inp, w)
+    del dev, buf, flush, graph
+    torch.cuda.empty_cache()
+    return line
 
 
 def _gate_up_keep(B, r, dev, w, buf):

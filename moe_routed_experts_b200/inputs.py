@@ -104,3 +104,33 @@ def generate(w: Workload, with_grad: Optional[bool] = None) -> Dict[str, object]
 
 def random_bf16(rng: np.random.Generator, shape, std: float = 1.0) -> np.ndarray:
     return f32_to_bf16_bits(rng.standard_normal(shape, dtype=np.float32) * np.float32(std))
+
+
+def nf4_codebook() -> np.ndarray:
+    """The 16 values of the 4-bit NormalFloat data type (Dettmers et al.,
+    "QLoRA", 2023, section 3): quantiles of N(0, 1) at evenly spaced
+    probabilities, 8 on the positive side and 7 on the negative side plus an
+    exact zero, scaled so the extremes are -1 and 1.  The outermost
+    probability is the midpoint of 1 - 1/(2*15) and 1 - 1/(2*16) (the two
+    halves' own outermost quantiles).  A payload input: the operation takes
+    whatever codebook the caller passes (tests pin this construction against
+    the paper's table)."""
+    from scipy.stats import norm
+    top = 1.0 - 0.5 * (1.0 / 30.0 + 1.0 / 32.0)
+    pos = norm.ppf(np.linspace(top, 0.5, 9)[:-1])
+    neg = -norm.ppf(np.linspace(top, 0.5, 8)[:-1])
+    v = np.sort(np.concatenate([pos, [0.0], neg]))
+    return (v / np.max(np.abs(v))).astype(np.float32)
+
+
+def draw_nf4_projection(rng: np.random.Generator, E: int, K_in: int, N: int, block: int, bias: bool = False,
+                        bias_std: float = 0.02) -> Dict[str, np.ndarray]:
+    """NF4 payload of E experts ([K_in, N] each): uniform random code bytes
+    (two uniform 4-bit codes per byte), absmax scales uniform[0.5, 1.5) /
+    sqrt(K_in) per block of `block` flat elements, the NF4 codebook."""
+    codes = rng.integers(0, 256, size=(E, K_in * N // 2), dtype=np.uint8)
+    absmax = (rng.uniform(0.5, 1.5, size=(E, K_in * N // block)) / math.sqrt(K_in)).astype(np.float32)
+    out = {"codes": codes, "absmax": absmax, "codebook": nf4_codebook(), "block": block, "N": N, "bias": None}
+    if bias:
+        out["bias"] = (rng.standard_normal((E, N), dtype=np.float32) * np.float32(bias_std)).astype(np.float32)
+    return out

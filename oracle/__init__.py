@@ -66,6 +66,15 @@ def _declare(L):
     L.oracle_dispatch_backward.argtypes = [P, C.c_int, P, P, I64, I64, I32, P, C.c_int]
     L.oracle_router_backward.argtypes = [P, P, P, I64, I64, I32, I32, U32, P]
     L.oracle_num_threads.restype = C.c_int
+    L.oracle_nf4_code.restype = I32
+    L.oracle_nf4_code.argtypes = [P, I64]
+    L.oracle_nf4_dequant.argtypes = [P, P, P, I64, I64, I64, C.c_int, P, P]
+    L.oracle_nf4_project.restype = C.c_int
+    L.oracle_nf4_project.argtypes = [P, C.c_int, I64, I64, I64, P, I64, P, P, P, I64, C.c_int, P, C.c_int, C.c_int,
+                                     P, C.c_int]
+    L.oracle_nf4_input_backward.restype = C.c_int
+    L.oracle_nf4_input_backward.argtypes = [P, C.c_int, I64, I64, I64, P, I64, P, P, P, I64, C.c_int, C.c_int, P,
+                                            C.c_int]
 
 
 def _p(a):
@@ -346,3 +355,63 @@ def forward(inp: dict, rows=None, tokens=None):
     elif rows.shape[0] == A:
         res["out"] = combine(y, "bf16", wts, sel, row_of)
     return res
+
+
+# ---------------------------------------------------------------- NF4 payloads
+
+def nf4_code(codes, f: int) -> int:
+    codes = _c(codes, np.uint8)
+    return int(lib().oracle_nf4_code(_p(codes), int(f)))
+
+
+def nf4_dequant(codes, absmax, codebook, K: int, N: int, B: int, cdt: str):
+    """One expert's NF4 coefficients: (W float64 [K,N], bits uint32 [K,N])."""
+    codes, absmax, cb = _c(codes, np.uint8), _c(absmax, np.float32), _c(codebook, np.float32)
+    W = np.zeros((K, N), np.float64)
+    Wb = np.zeros((K, N), np.uint32)
+    lib().oracle_nf4_dequant(_p(codes), _p(absmax), _p(cb), K, N, B, DT[cdt], _p(W), _p(Wb))
+    return W, Wb
+
+
+def nf4_project(x, xdt: str, row_expert, payload: dict, cdt: str, exact: bool = False, odt: str = None,
+                bias_dt: str = "f32", magnitude: bool = False):
+    """Rows of x through their experts' NF4 projection (see oracle_nf4_project).
+    payload: codes uint8 [E, K*N/2], absmax f32 [E, K*N/B], codebook f32 [16],
+    block B, N; optional bias [E, N]."""
+    x = _c(x)
+    R, K = x.shape
+    N, B = payload["N"], payload["block"]
+    codes, absmax = _c(payload["codes"], np.uint8), _c(payload["absmax"], np.float32)
+    cb = _c(payload["codebook"], np.float32)
+    E = codes.shape[0]
+    bias = payload.get("bias")
+    if bias is not None:
+        bias = _c(bias, np.float32 if bias_dt == "f32" else np.uint16)
+    re = _c(row_expert, np.int32)
+    odt = odt or xdt
+    mode = 2 if magnitude else 1 if exact else 0
+    out = np.zeros((R, N), np.float64 if mode else _out_dtype(odt))
+    rc = lib().oracle_nf4_project(_p(x), DT[xdt], R, K, N, _p(re), E, _p(codes), _p(absmax), _p(cb), B, DT[cdt],
+                                  _p(bias), DT[bias_dt], mode, _p(out), DT[odt])
+    if rc != 0:
+        raise ValueError("oracle_nf4_project: " + ("bad block layout" if rc == -2 else "expert index out of range"))
+    return out
+
+
+def nf4_input_backward(grad, gdt: str, row_expert, payload: dict, K: int, cdt: str, exact: bool = False,
+                       odt: str = None, magnitude: bool = False):
+    grad = _c(grad)
+    R, N = grad.shape
+    B = payload["block"]
+    codes, absmax = _c(payload["codes"], np.uint8), _c(payload["absmax"], np.float32)
+    cb = _c(payload["codebook"], np.float32)
+    E = codes.shape[0]
+    re = _c(row_expert, np.int32)
+    odt = odt or gdt
+    mode = 2 if magnitude else 1 if exact else 0
+    out = np.zeros((R, K), np.float64 if mode else _out_dtype(odt))
+    rc = lib().oracle_nf4_input_backward(_p(grad), DT[gdt], R, N, K, _p(re), E, _p(codes), _p(absmax), _p(cb), B,
+                                         DT[cdt], mode, _p(out), DT[odt])
+    if rc != 0:
+        raise ValueError("oracle_nf4_input_backward: " + ("bad block layout" if rc == -2 else "expert index out of range"))
+    return out

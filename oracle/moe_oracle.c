@@ -333,6 +333,59 @@ void oracle_copy_rows(const void *x, int64_t H, int64_t elem_bytes, const int32_
 /* Grouped projection of selected rows.                                */
 /* ------------------------------------------------------------------ */
 
+/* Rows r with row_expert[r] == e: out[r,n] = sum_kk x[r,kk] * W[kk,n] (+ bias[n]),
+ * accumulated in double; mode 0 stores RNE in odt, 1 the double sum, 2 the
+ * double sum of magnitudes (see oracle_project). */
+static void expert_rows_times_W(const void *x, int xdt, int64_t R, int64_t K, int64_t N,
+                                const int32_t *row_expert, int64_t e, const double *W,
+                                const void *be, int bdt, int mode, void *out, int odt) {
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t r = 0; r < R; ++r) {
+        if (row_expert[r] != e) continue;
+        double *acc = (double *)calloc((size_t)N, sizeof(double));
+        for (int64_t kk = 0; kk < K; ++kk) {
+            double xv = load_val(x, xdt, r * K + kk);
+            const double *Wr = W + kk * N;
+            if (mode == 2)
+                for (int64_t n = 0; n < N; ++n) acc[n] += fabs(xv * Wr[n]);
+            else
+                for (int64_t n = 0; n < N; ++n) acc[n] += xv * Wr[n];
+        }
+        for (int64_t n = 0; n < N; ++n) {
+            double b = (be && ORACLE_MUTANT != 7) ? load_val(be, bdt, n) : 0.0;
+            double v = acc[n] + (mode == 2 ? fabs(b) : b);
+            if (mode >= 1) ((double *)out)[r * N + n] = v;
+            else store_val(out, odt, r * N + n, v);
+        }
+        free(acc);
+    }
+}
+
+/* Rows r with row_expert[r] == e: out[r,kk] = sum_n grad[r,n] W[kk,n]
+ * (+ sum_n grad2[r,n] W2[kk,n]), one double accumulator; modes as above. */
+static void expert_rows_times_WT(const void *grad, int gdt, int64_t R, int64_t N, int64_t K,
+                                 const int32_t *row_expert, int64_t e, const double *W,
+                                 const void *grad2, const double *W2, int mode, void *out, int odt) {
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t r = 0; r < R; ++r) {
+        if (row_expert[r] != e) continue;
+        for (int64_t kk = 0; kk < K; ++kk) {
+            double acc = 0.0;
+            for (int64_t n = 0; n < N; ++n) {
+                double pr = load_val(grad, gdt, r * N + n) * W[kk * N + n];
+                acc += mode == 2 ? fabs(pr) : pr;
+            }
+            if (W2 && ORACLE_MUTANT != 9)
+                for (int64_t n = 0; n < N; ++n) {
+                    double pr = load_val(grad2, gdt, r * N + n) * W2[kk * N + n];
+                    acc += mode == 2 ? fabs(pr) : pr;
+                }
+            if (mode >= 1) ((double *)out)[r * K + kk] = acc;
+            else store_val(out, odt, r * K + kk, acc);
+        }
+    }
+}
+
 /* Rows r < R of x ([R,K] in dtype xdt) go through the projection of their
  * expert row_expert[r] (local index < E):
  *   acc[r,n] = sum_kk x[r,kk] * W[e,kk,n]  (+ bias[e,n])
@@ -362,26 +415,85 @@ int oracle_project(const void *x, int xdt, int64_t R, int64_t K, int64_t N,
         oracle_dequant(qw + e * K * NW, qz + e * G * NW, (const char *)sc + (size_t)(e * G * N) * sbytes, sdt,
                        K, N, g, W, NULL);
         const void *be = bias ? (const void *)((const char *)bias + (size_t)(e * N) * bbytes) : NULL;
-#pragma omp parallel for schedule(dynamic, 1)
-        for (int64_t r = 0; r < R; ++r) {
-            if (row_expert[r] != e) continue;
-            double *acc = (double *)calloc((size_t)N, sizeof(double));
-            for (int64_t kk = 0; kk < K; ++kk) {
-                double xv = load_val(x, xdt, r * K + kk);
-                const double *Wr = W + kk * N;
-                if (mode == 2)
-                    for (int64_t n = 0; n < N; ++n) acc[n] += fabs(xv * Wr[n]);
-                else
-                    for (int64_t n = 0; n < N; ++n) acc[n] += xv * Wr[n];
-            }
-            for (int64_t n = 0; n < N; ++n) {
-                double b = (be && ORACLE_MUTANT != 7) ? load_val(be, bdt, n) : 0.0;
-                double v = acc[n] + (mode == 2 ? fabs(b) : b);
-                if (mode >= 1) ((double *)out)[r * N + n] = v;
-                else store_val(out, odt, r * N + n, v);
-            }
-            free(acc);
+        expert_rows_times_W(x, xdt, R, K, N, row_expert, e, W, be, bdt, mode, out, odt);
+    }
+    free(W);
+    return 0;
+}
+
+/* ------------------------------------------------------------------ */
+/* NF4 payload: ruda-tensor 0.21.34, src/packed_experts.rs,             */
+/* PackedExpertPayload::Nf4 ("original RUDA high-nibble-first flat-block */
+/* NF4"; packed scales and codebook frozen).  The pages print no layout; */
+/* the reading: the 4-bit NormalFloat data type of Dettmers et al.,      */
+/* "QLoRA: Efficient Finetuning of Quantized LLMs" (2023): 16 code       */
+/* values (the codebook, an input), one absmax scale per block of B      */
+/* consecutive elements of the flattened weight.                         */
+/*   codes  uint8 [K*N/2]: the logical [K,N] matrix, flat index          */
+/*          f = kk*N + n; byte f/2, high nibble (bits 4..7) for even f,  */
+/*          low nibble for odd f;                                        */
+/*   absmax f32 [K*N/B]; codebook f32 [16];                              */
+/*   W[kk,n] = RNE_cdt(codebook[q] * absmax[f / B]): the F32 x F32       */
+/*   product (exact in double) rounded once to the coefficient dtype.    */
+/* ------------------------------------------------------------------ */
+
+int32_t oracle_nf4_code(const uint8_t *codes, int64_t f) {
+    uint8_t b = codes[f / 2];
+    int high_first = ORACLE_MUTANT == 15 ? 0 : 1;
+    return ((f % 2 == 0) == high_first) ? (int32_t)(b >> 4) : (int32_t)(b & 0xF);
+}
+
+void oracle_nf4_dequant(const uint8_t *codes, const float *absmax, const float *codebook, int64_t K,
+                        int64_t N, int64_t B, int cdt, double *W, uint32_t *Wbits) {
+#pragma omp parallel for schedule(static)
+    for (int64_t kk = 0; kk < K; ++kk)
+        for (int64_t n = 0; n < N; ++n) {
+            int64_t f = kk * N + n;
+            double exact = (double)codebook[oracle_nf4_code(codes, f)] * (double)absmax[f / B];
+            double w = oracle_round(exact, cdt);
+            if (W) W[f] = w;
+            if (Wbits) Wbits[f] = oracle_encode(w, cdt);
         }
+}
+
+/* Grouped projection with NF4 payloads (rows, modes and return codes as
+ * oracle_project; -2 when K*N is odd or not a whole number of blocks). */
+int oracle_nf4_project(const void *x, int xdt, int64_t R, int64_t K, int64_t N,
+                       const int32_t *row_expert, int64_t E, const uint8_t *codes, const float *absmax,
+                       const float *codebook, int64_t B, int cdt, const void *bias, int bdt, int mode,
+                       void *out, int odt) {
+    if (B < 2 || (K * N) % B != 0 || (K * N) % 2 != 0) return -2;
+    for (int64_t r = 0; r < R; ++r)
+        if (row_expert[r] < 0 || row_expert[r] >= E) return -1;
+    size_t bbytes = (bdt == DT_F32) ? 4 : 2;
+    double *W = (double *)malloc(sizeof(double) * (size_t)(K * N));
+    for (int64_t e = 0; e < E; ++e) {
+        int any = 0;
+        for (int64_t r = 0; r < R && !any; ++r) any = (row_expert[r] == e);
+        if (!any) continue;
+        oracle_nf4_dequant(codes + e * (K * N / 2), absmax + e * (K * N / B), codebook, K, N, B, cdt, W, NULL);
+        const void *be = bias ? (const void *)((const char *)bias + (size_t)(e * N) * bbytes) : NULL;
+        expert_rows_times_W(x, xdt, R, K, N, row_expert, e, W, be, bdt, mode, out, odt);
+    }
+    free(W);
+    return 0;
+}
+
+/* Input VJP through the same NF4 coefficients (one payload). */
+int oracle_nf4_input_backward(const void *grad, int gdt, int64_t R, int64_t N, int64_t K,
+                              const int32_t *row_expert, int64_t E, const uint8_t *codes,
+                              const float *absmax, const float *codebook, int64_t B, int cdt, int mode,
+                              void *out, int odt) {
+    if (B < 2 || (K * N) % B != 0 || (K * N) % 2 != 0) return -2;
+    for (int64_t r = 0; r < R; ++r)
+        if (row_expert[r] < 0 || row_expert[r] >= E) return -1;
+    double *W = (double *)malloc(sizeof(double) * (size_t)(K * N));
+    for (int64_t e = 0; e < E; ++e) {
+        int any = 0;
+        for (int64_t r = 0; r < R && !any; ++r) any = (row_expert[r] == e);
+        if (!any) continue;
+        oracle_nf4_dequant(codes + e * (K * N / 2), absmax + e * (K * N / B), codebook, K, N, B, cdt, W, NULL);
+        expert_rows_times_WT(grad, gdt, R, N, K, row_expert, e, W, NULL, NULL, mode, out, odt);
     }
     free(W);
     return 0;
@@ -475,24 +587,7 @@ int oracle_input_backward(const void *grad, int gdt, int64_t R, int64_t N, int64
         if (W2)
             oracle_dequant(qw2 + e * K * NW, qz2 + e * G * NW, (const char *)sc2 + (size_t)(e * G * N) * sbytes,
                            sdt, K, N, g, W2, NULL);
-#pragma omp parallel for schedule(dynamic, 1)
-        for (int64_t r = 0; r < R; ++r) {
-            if (row_expert[r] != e) continue;
-            for (int64_t kk = 0; kk < K; ++kk) {
-                double acc = 0.0;
-                for (int64_t n = 0; n < N; ++n) {
-                    double pr = load_val(grad, gdt, r * N + n) * W[kk * N + n];
-                    acc += mode == 2 ? fabs(pr) : pr;
-                }
-                if (W2 && ORACLE_MUTANT != 9)
-                    for (int64_t n = 0; n < N; ++n) {
-                        double pr = load_val(grad2, gdt, r * N + n) * W2[kk * N + n];
-                        acc += mode == 2 ? fabs(pr) : pr;
-                    }
-                if (mode >= 1) ((double *)out)[r * K + kk] = acc;
-                else store_val(out, odt, r * K + kk, acc);
-            }
-        }
+        expert_rows_times_WT(grad, gdt, R, N, K, row_expert, e, W, grad2, W2, mode, out, odt);
     }
     free(W);
     free(W2);

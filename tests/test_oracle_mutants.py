@@ -4,7 +4,7 @@ rounding, a wrong zero-point group, a flipped tie-break, biased weights, a
 reversed dispatch order, a dropped bias, a SwiGLU without its gate factor, a
 dropped gate/up gradient term, unweighted combine, a missing SwiGLU-VJP
 factor, a missing softmax-VJP term, a wrong dweights dot, a COPY VJP that
-sums one selection only), and the oracle's
+sums one selection only, an NF4 byte read low nibble first), and the oracle's
 own CPU tests must fail on every one of them.  CPU only."""
 import os
 import subprocess
@@ -18,7 +18,7 @@ sys.path.insert(0, ROOT)
 from oracle.build import build_mutant  # noqa: E402
 
 PINS = [os.path.join(ROOT, "tests", f) for f in
-        ("test_oracle_pins.py", "test_oracle_bruteforce.py", "test_oracle_invariants.py")]
+        ("test_oracle_pins.py", "test_oracle_bruteforce.py", "test_oracle_invariants.py", "test_oracle_nf4.py")]
 
 MUTANTS = {
     1: "unpack ignores the 0,2,4,6,1,3,5,7 order",
@@ -35,6 +35,7 @@ MUTANTS = {
     12: "router-logit VJP drops the - <w, dw> term",
     13: "combine VJP dweights dot uses dOut instead of y",
     14: "COPY VJP sums only the first selection of each token",
+    15: "NF4 codes read low nibble first",
 }
 
 

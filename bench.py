@@ -152,7 +152,7 @@ def main():
     ap.add_argument("--no-graph", action="store_true", help="launch kernels directly instead of a CUDA graph")
     ap.add_argument("--soak-seconds", type=float, default=1.0)
     ap.add_argument("--reference-tokens", type=int, default=8)
-    ap.add_argument("--workloads", default="prefill,wide,skewed",
+    ap.add_argument("--workloads", default="prefill,wide,skewed,nf4",
                     help="other workloads timed in the same run, reported under 'workloads' ('none': skip)")
     ap.add_argument("--tokens", type=int, default=0,
                     help="override the workload's token count (smaller profiling captures); 0 keeps it")
@@ -189,18 +189,71 @@ def main():
     extra = [] if args.workloads in ("", "none") else [n for n in args.workloads.split(",") if n != w.name]
     if extra and rank == 0:
         line["workloads"] = {}
-    for name in extra:
+    for name in [n for n in extra if n in WORKLOADS]:
         sub = measure(WORKLOADS[name], args, min(args.steps, 20), world, rank, local, cpu=False)
         if rank == 0:
             line["workloads"][name] = {k: sub[k] for k in (
                 "value", "unit", "ms_per_step", "fwd_ms", "bwd_ms", "tflops", "packed_weight_gbs",
                 "packed_weight_frac", "roofline", "e2e", "gpu_launches", "clocks", "device_status", "config", "steps")
                 if k in sub}
+    if "nf4" in extra:
+        sub = measure_nf4(args, min(args.steps, 20), world, rank)
+        if rank == 0:
+            line["workloads"]["nf4"] = sub
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
+
+
+def measure_nf4(args, steps, world, rank):
+    """The NF4 payload path on the decode shape: the down projection of the
+    decode workload (A = 256 rows over E = 128 experts, K = 768, N = 2048)
+    with an NF4 payload (blocks of 64, BF16 coefficients), timed per call
+    under the same flush protocol; HBM roofline on the packed bytes (codes +
+    absmax) of the touched experts."""
+    import torch
+    from moe_routed_experts_b200 import binding as B
+    w = WORKLOADS["decode"]
+    rng = np.random.default_rng(w.seed)
+    K, N, block = w.I, w.H, 64
+    p = inputs.draw_nf4_projection(rng, w.E, K, N, block)
+    dp = B.nf4_payload_to_device(p)
+    inp = inputs.generate(w)
+    dev_logits = torch.from_numpy(inp["logits"]).cuda()
+    r = B.moe_route(dev_logits, w.top_k, E=w.E)
+    x = torch.from_numpy(inputs.random_bf16(rng, (w.A, K)).view(np.int16)).view(torch.bfloat16).cuda()
+    st = B.new_status()
+    out = torch.empty((w.A, N), dtype=torch.bfloat16, device="cuda")
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    for _ in range(args.warmup):
+        B.nf4_grouped_projection(x, r["offsets"], dp, "bf16", device_status=st, out=out)
+    torch.cuda.synchronize()
+    ts = []
+    for i in range(steps):
+        flush.fill_(i & 0xFF)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        B.nf4_grouped_projection(x, r["offsets"], dp, "bf16", device_status=st, out=out)
+        b.record()
+        torch.cuda.synchronize()
+        ts.append(a.elapsed_time(b))
+    ms = max_over_ranks([statistics.median(ts)], "cuda")[0]
+    if rank != 0:
+        return None
+    counts = np.diff(r["offsets"].cpu().numpy())
+    touched = int((counts > 0).sum())
+    alg = touched * (p["codes"][0].nbytes + p["absmax"][0].nbytes)
+    pk = peaks()
+    achieved = alg / (ms * 1e-3) / 1e9
+    return {"ms_per_call": ms, "value": world * w.T / (ms * 1e-3), "unit": "tokens/s",
+            "roofline": {"bound": "hbm", "kernel": "nf4_grouped_projection: nf4_fwd_kernel", "achieved": achieved,
+                         "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": achieved / pk["hbm_gbs"], "traffic": None,
+                         "algorithmic_bytes": alg, "kernel_ms": ms, "peak_source": pk["source"]},
+            "config": {"workload": "nf4 down projection, decode shape", "A": w.A, "K": K, "N": N, "E": w.E,
+                       "block": block, "coef_dtype": "bf16", "experts_touched": touched},
+            "device_status": int(st.item()), "gpu_launches": steps}
 
 
 def measure(w, args, steps, world, rank, local, cpu):

@@ -52,10 +52,11 @@
  *   Requirements: N % 8 == 0, K % group == 0, group % 16 == 0; qweight,
  *   scales, bias and the activation/output tensors 16-byte aligned.
  *   The tensor-core products run in the scale dtype; activations are
- *   converted to it when they differ (BF16 -> F16 is exact for values in
- *   F16's normal range; a value outside it sets MOE_DEVICE_ERR_ACT_RANGE;
- *   F16 -> BF16 rounds to 8 significant bits).  FP32 scales are rejected
- *   with MOE_ERR_UNSUPPORTED_DTYPE.
+ *   converted to it when they differ (BF16 -> F16 is exact in F16's normal
+ *   range; above it a value becomes inf and MOE_DEVICE_ERR_ACT_RANGE is set;
+ *   below 2^-14 it keeps what F16's subnormal grid holds, an absolute change
+ *   under 2^-25; F16 -> BF16 rounds to 8 significant bits).  FP32 scales are
+ *   rejected with MOE_ERR_UNSUPPORTED_DTYPE.
  */
 #ifndef MOE_AWQ_H_
 #define MOE_AWQ_H_
@@ -89,10 +90,9 @@ typedef enum { MOE_F32 = 0, MOE_F16 = 1, MOE_BF16 = 2 } moe_dtype;
 #define MOE_DEVICE_ERR_OFFSETS 2      /* offsets not monotone, offsets[0] != 0 or offsets[E] != A */
 #define MOE_DEVICE_ERR_ROW_RANGE 4    /* a row_of entry outside [0, A) */
 #define MOE_DEVICE_ERR_TIMEOUT 8      /* a bounded device wait gave up */
-#define MOE_DEVICE_ERR_ACT_RANGE 16   /* a BF16 activation or gradient fed to F16-scale tensor cores lies
-                                         outside F16's normal range (|v| > 65504, inf/NaN, or
-                                         0 < |v| < 2^-14): its conversion to F16 was not exact; the
-                                         result is computed from the converted value */
+#define MOE_DEVICE_ERR_ACT_RANGE 16   /* a BF16 activation or gradient fed to F16-scale tensor cores was
+                                         finite above F16's range (|v| > 65504: it became inf) or NaN;
+                                         the result is computed from the converted value */
 
 /* Limits of this implementation. */
 #define MOE_MAX_EXPERTS 4096
@@ -286,6 +286,42 @@ MOE_API moe_status awq_grouped_down(const void *input, moe_dtype act_dtype, int6
                             const void *bias, moe_dtype scale_dtype, moe_dtype bias_dtype,
                             int64_t group_size, void *output, void *workspace,
                             size_t workspace_bytes, int32_t *device_status, void *stream);
+
+/* ------------------------------------------------------------------------
+ * nf4_grouped_projection, nf4_input_backward -- a projection whose frozen
+ * payload is NF4 instead of AWQ: [PE] PackedExpertPayload::Nf4 ("original
+ * RUDA high-nibble-first flat-block NF4"; packed scales and codebook stay
+ * frozen; gate, up and down each pick their format independently).  The
+ * pages print no NF4 layout; this library reads it as the 4-bit NormalFloat
+ * data type of Dettmers et al., "QLoRA" (2023), flat blocks:
+ *   codes    uint8 [E, K*N/2]   the logical [K, N] matrix of each expert
+ *                               flattened row-major; flat element
+ *                               f = kk*N + n sits in byte f/2, in the high
+ *                               nibble (bits 4..7) when f is even
+ *   absmax   f32 [E, K*N/block] one scale per `block` consecutive elements
+ *   codebook f32 [16]           the 16 code values (caller-supplied)
+ *   coefficient W[e,kk,n] = RNE_coef_dtype(codebook[q] * absmax[f / block]):
+ *   the F32 x F32 product, exact, rounded once to coef_dtype (F16 or BF16,
+ *   which is also the tensor-core operand dtype).
+ * nf4_grouped_projection: output[r, n] = RNE(sum_kk input[r,kk] W[e,kk,n]
+ *   + bias[e,n]) for the rows of expert e (offsets as for the AWQ calls);
+ *   input [A, K], output [A, N] (act_dtype), bias [E, N] or NULL.
+ * nf4_input_backward: dinput[r, kk] = RNE(sum_n grad[r,n] W[e,kk,n]);
+ *   grad [A, N], dinput [A, K] (grad_dtype).
+ * Requirements: K and N multiples of 64, block a multiple of 32 dividing
+ * K*N; input/output/codes 16-byte aligned.  Device errors:
+ * MOE_DEVICE_ERR_OFFSETS, MOE_DEVICE_ERR_ACT_RANGE.
+ * ---------------------------------------------------------------------- */
+MOE_API moe_status nf4_grouped_projection(const void *input, moe_dtype act_dtype, int64_t A, int64_t K, int64_t N,
+                                          const int32_t *offsets, int64_t E, const uint8_t *codes,
+                                          const float *absmax, const float *codebook, int64_t block,
+                                          moe_dtype coef_dtype, const void *bias, moe_dtype bias_dtype,
+                                          void *output, int32_t *device_status, void *stream);
+
+MOE_API moe_status nf4_input_backward(const void *grad, moe_dtype grad_dtype, int64_t A, int64_t N, int64_t K,
+                                      const int32_t *offsets, int64_t E, const uint8_t *codes,
+                                      const float *absmax, const float *codebook, int64_t block,
+                                      moe_dtype coef_dtype, void *dinput, int32_t *device_status, void *stream);
 
 /* ------------------------------------------------------------------------
  * moe_combine -- [MX] MoeDispatchOps::moe_combine ("ascending expert-ID

@@ -60,6 +60,9 @@ _SIGS = {
     "moe_router_backward": (C.c_int, [P, P, P, I64, I64, I32, I32, I32, P, P, P]),
     "awq_dequant_coefficients": (C.c_int, [P, P, P, C.c_int, I64, I64, I64, I32, P, P]),
     "moe_set_projection_path": (I32, [I32]),
+    "nf4_grouped_projection": (C.c_int, [P, C.c_int, I64, I64, I64, P, I64, P, P, P, I64, C.c_int, P, C.c_int, P, P,
+                                         P]),
+    "nf4_input_backward": (C.c_int, [P, C.c_int, I64, I64, I64, P, I64, P, P, P, I64, C.c_int, P, P, P]),
 }
 
 
@@ -339,3 +342,37 @@ def awq_dequant_coefficients(qweight, qzeros, scales, group, pairing=0):
                                         pairing, _ptr(out), _stream())
     _check("awq_dequant_coefficients", st)
     return out
+
+
+def nf4_payload_to_device(payload: dict, device="cuda") -> dict:
+    """NF4 payload (codes uint8 [E, K*N/2], absmax f32, codebook f32 [16]) -> device tensors."""
+    d = {"codes": torch.from_numpy(payload["codes"]).to(device), "absmax": torch.from_numpy(payload["absmax"]).to(device),
+         "codebook": torch.from_numpy(payload["codebook"]).to(device), "block": int(payload["block"]),
+         "N": int(payload["N"]), "bias": None}
+    if payload.get("bias") is not None:
+        d["bias"] = torch.from_numpy(payload["bias"]).to(device)
+    return d
+
+
+def nf4_grouped_projection(inp, offsets, payload, coef_dtype="bf16", device_status=None, out=None):
+    A, K = inp.shape
+    E = offsets.numel() - 1
+    N = payload["N"]
+    y = out if out is not None else torch.empty((A, N), dtype=inp.dtype, device=inp.device)
+    st = lib().nf4_grouped_projection(
+        _ptr(inp), _dt(inp.dtype), A, K, N, _ptr(offsets), E, _ptr(payload["codes"]), _ptr(payload["absmax"]),
+        _ptr(payload["codebook"]), payload["block"], _NAME_DT[coef_dtype], _ptr(payload.get("bias")),
+        _bias_dt(payload.get("bias")), _ptr(y), _ptr(device_status), _stream())
+    _check("nf4_grouped_projection", st)
+    return y
+
+
+def nf4_input_backward(grad, offsets, payload, K, coef_dtype="bf16", device_status=None, out=None):
+    A, N = grad.shape
+    E = offsets.numel() - 1
+    d = out if out is not None else torch.empty((A, K), dtype=grad.dtype, device=grad.device)
+    st = lib().nf4_input_backward(
+        _ptr(grad), _dt(grad.dtype), A, N, K, _ptr(offsets), E, _ptr(payload["codes"]), _ptr(payload["absmax"]),
+        _ptr(payload["codebook"]), payload["block"], _NAME_DT[coef_dtype], _ptr(d), _ptr(device_status), _stream())
+    _check("nf4_input_backward", st)
+    return d

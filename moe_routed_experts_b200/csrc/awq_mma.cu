@@ -33,6 +33,7 @@ namespace moe {
 
 template <typename MT, int NPROJ, int NT>
 __global__ void __launch_bounds__(128) awq_fwd_mma_kernel(ProjParams p) {
+  pdl_enter();  // programmatic dependent launch: the previous kernel is done
   uint32_t act_bad = 0;  // a converted input outside F16's normal range
   constexpr int D = 2;  // K steps of loads in flight per warp
   __shared__ float red[4][NPROJ][8 * NT][64];
@@ -374,9 +375,9 @@ template <typename MT, int NPROJ>
 static void launch_fwd_t(const ProjParams &p, int nt, cudaStream_t st) {
   dim3 grid((unsigned)((p.N / 8 + 7) / 8), (unsigned)p.E);
   if (nt == 2)
-    awq_fwd_mma_kernel<MT, NPROJ, 2><<<grid, 128, 0, st>>>(p);
+    launch_pdl(awq_fwd_mma_kernel<MT, NPROJ, 2>, grid, dim3(128), 0, st, p);
   else
-    awq_fwd_mma_kernel<MT, NPROJ, 1><<<grid, 128, 0, st>>>(p);
+    launch_pdl(awq_fwd_mma_kernel<MT, NPROJ, 1>, grid, dim3(128), 0, st, p);
 }
 
 void launch_fwd_mma(const ProjParams &p, int nproj, bool bf16_mma, int nt, cudaStream_t st) {

@@ -127,6 +127,7 @@ template <typename MT, int NPROJ, int NT, int ROWS>
 __global__ void __launch_bounds__(stream::kThreads, 2)
     awq_fwd_stream_kernel(const __grid_constant__ CUtensorMap map0, const __grid_constant__ CUtensorMap map1,
                           ProjParams p) {
+  pdl_enter();  // programmatic dependent launch: the previous kernel is done
   using namespace stream;
   constexpr int kRows = Geo<ROWS>::kRows, kBox = Geo<ROWS>::kBox, kStageBytes = Geo<ROWS>::kStageBytes;
   constexpr int kStages = Geo<ROWS>::kStages;
@@ -264,21 +265,6 @@ __global__ void __launch_bounds__(stream::kThreads, 2)
     // tile is converted, so their latency overlaps that work
     uint32_t pf_zw = wc_ok ? (uint32_t)__ldg(qzp + grp * NW) : 0u;
     uint4 pf_sv = wc_ok ? __ldg(reinterpret_cast<const uint4 *>(scp + grp * p.N)) : make_uint4(0, 0, 0, 0);
-    // F16: the odd-slot shortcut (fwd_pairs16) is exact when every scale of
-    // the column group in this unit's K range is 0 or 2^-14 <= |s| <= 256;
-    // then the odd slots accumulate 16 times their value throughout the unit
-    // and are scaled back (exactly) at its end.  The four lanes of a quad
-    // share the column: each checks one scale pair of each group, the quad ORs.
-    bool x16 = false;
-    if (std::is_same<MT, __half>::value) {
-      uint32_t bad = 0;
-      if (wc_ok)
-        for (int64_t gr = grp; gr * p.group < kbase + Kq; ++gr)
-          bad |= f16_pair_blocks_x16(__ldg(reinterpret_cast<const uint32_t *>(scp + gr * p.N) + t));
-      bad |= __shfl_xor_sync(0xffffffffu, bad, 1);
-      bad |= __shfl_xor_sync(0xffffffffu, bad, 2);
-      x16 = bad == 0;
-    }
 
     // activation tile: raw rows -> scale dtype, row order t, t+4, t+8, t+12 per 16.
     // After an abort every consumer warp still runs the loop (the named
@@ -305,20 +291,39 @@ __global__ void __launch_bounds__(stream::kThreads, 2)
 
     // acc: every slot in its true scale; acc16: odd slots taken 16 times
     // larger (F16 groups whose scales allow it, see fwd_pairs16)
-    float acc[NT][4][4];
+    float acc[NT][4][4], acc16[NT][2][4];
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
+    for (int nt = 0; nt < NT; ++nt) {
 #pragma unroll
       for (int q = 0; q < 4; ++q)
 #pragma unroll
         for (int i = 0; i < 4; ++i) acc[nt][q][i] = 0.f;
+#pragma unroll
+      for (int q = 0; q < 2; ++q)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc16[nt][q][i] = 0.f;
+    }
     FwdConsts<MT> cst;
+    bool x16 = false;
     const int spg = p.group / kRows;  // stages per group (group % kRows == 0 on this path)
     int gstage = (int)((kbase % p.group) / kRows);
     for (int c = 0; c < nst; ++c, ++it) {
       const uint32_t s = it % kStages, ph = (it / kStages) & 1;
       if (c == 0 || gstage == 0) {  // a stage lies inside one group
-        load_consts_fast<MT>(cst, pf_zw, pf_sv, x16);
+        if (std::is_same<MT, __half>::value) {
+          // 16 RNE((q - z) s) = RNE(16 (q - z) s) needs every nonzero product
+          // normal before and after the scaling: 0 or 2^-14 <= |s| <= 256 for
+          // all 8 scales of this column group
+          const uint32_t w4[4] = {pf_sv.x, pf_sv.y, pf_sv.z, pf_sv.w};
+          uint32_t bad = 0;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const uint32_t lo = w4[i] & 0x7FFFu, hi = (w4[i] >> 16) & 0x7FFFu;
+            bad |= (lo > 0x5C00u) | (hi > 0x5C00u) | (lo != 0u && lo < 0x0400u) | (hi != 0u && hi < 0x0400u);
+          }
+          x16 = bad == 0;
+        }
+        cst.load(pf_zw, pf_sv, x16);
         if (wc_ok && (grp + 1) * p.group < kbase + Kq) {  // prefetch the next group
           pf_zw = (uint32_t)__ldg(qzp + (grp + 1) * NW);
           pf_sv = __ldg(reinterpret_cast<const uint4 *>(scp + (grp + 1) * p.N));
@@ -331,44 +336,69 @@ __global__ void __launch_bounds__(stream::kThreads, 2)
       const bool sok = tc_wait(&full[s], ph, p.status, abort);
       if (sok) {
         const uint8_t *box0 = stages + s * kStageBytes + bw * kBox;
-#pragma unroll 2
-        for (int h = 0; h < kSteps; ++h) {  // 16-row steps: rows 16h + {t, t+4, t+8, t+12}
-          const uint8_t *box = box0 + (16 * h) * 128;
-          const int xrow0 = kRows * c + 16 * h;
-          uint32_t w[4];
-          uint32_t b0[NT], b1[NT];
-          w[0] = *reinterpret_cast<const uint32_t *>(box + woff0);
-          w[1] = *reinterpret_cast<const uint32_t *>(box + woff1);
-          w[2] = *reinterpret_cast<const uint32_t *>(box + woff0 + 8 * 128);
-          w[3] = *reinterpret_cast<const uint32_t *>(box + woff1 + 8 * 128);
+        // two 16-row steps at a time keep the register footprint of a 32-row stage
+#pragma unroll 1
+        for (int hh = 0; hh < kSteps; hh += 2) {
+        const uint8_t *box = box0 + (16 * hh) * 128;
+        const int xrow0 = kRows * c + 16 * hh;
+        uint32_t w[2][4];
+        uint32_t b0[2][NT], b1[2][NT];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {  // 16-row steps: rows 16h + {t, t+4, t+8, t+12}
+          w[h][0] = *reinterpret_cast<const uint32_t *>(box + woff0 + (16 * h) * 128);
+          w[h][1] = *reinterpret_cast<const uint32_t *>(box + woff1 + (16 * h) * 128);
+          w[h][2] = *reinterpret_cast<const uint32_t *>(box + woff0 + (16 * h + 8) * 128);
+          w[h][3] = *reinterpret_cast<const uint32_t *>(box + woff1 + (16 * h + 8) * 128);
 #pragma unroll
           for (int nt = 0; nt < NT; ++nt) {
-            const uint2 bv = *reinterpret_cast<const uint2 *>(xs + (nt * 8 + g) * xs_pitch + (xrow0 + 4 * t) * 2);
-            b0[nt] = bv.x;
-            b1[nt] = bv.y;
+            const uint2 bv =
+                *reinterpret_cast<const uint2 *>(xs + (nt * 8 + g) * xs_pitch + (xrow0 + 16 * h + 4 * t) * 2);
+            b0[h][nt] = bv.x;
+            b1[h][nt] = bv.y;
           }
-          uint32_t af[4][4];
-          if (std::is_same<MT, __half>::value && x16) fwd_step<MT, true>(w[0], w[1], w[2], w[3], cst, af);
-          else fwd_step<MT, false>(w[0], w[1], w[2], w[3], cst, af);
+        }
+        bool done = false;
+        if constexpr (std::is_same<MT, __half>::value) {
+          if (x16) {
 #pragma unroll
-          for (int q = 0; q < 4; ++q)
+            for (int h = 0; h < 2; ++h) {
+              uint32_t af[4][4];
+              fwd_step<MT, true>(w[h][0], w[h][1], w[h][2], w[h][3], cst, af);
 #pragma unroll
-            for (int nt = 0; nt < NT; ++nt) mma16816<MT>(acc[nt][q], af[q], b0[nt], b1[nt]);
+              for (int q = 0; q < 4; ++q)
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                  if (q & 1) mma16816<MT>(acc16[nt][q >> 1], af[q], b0[h][nt], b1[h][nt]);
+                  else mma16816<MT>(acc[nt][q], af[q], b0[h][nt], b1[h][nt]);
+                }
+            }
+            done = true;
+          }
+        }
+        if (!done) {
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            uint32_t af[4][4];
+            fwd_step<MT, false>(w[h][0], w[h][1], w[h][2], w[h][3], cst, af);
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+#pragma unroll
+              for (int nt = 0; nt < NT; ++nt) mma16816<MT>(acc[nt][q], af[q], b0[h][nt], b1[h][nt]);
+          }
+        }
         }
       }
       __syncwarp();
       if (lane == 0 && sok) mbar_arrive(&empty[s]);
     }
     const bool unit_ok = !*abort;  // no stores from a unit an abort cut short
-    if (x16) {
 #pragma unroll
-      for (int nt = 0; nt < NT; ++nt)
+    for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {  // the 16x-scaled odd slots back (exact power-of-two scaling)
-          acc[nt][1][i] *= 0.0625f;
-          acc[nt][3][i] *= 0.0625f;
-        }
-    }
+      for (int i = 0; i < 4; ++i) {  // fold the 16x-scaled odd slots back (exact power-of-two scaling)
+        acc[nt][1][i] += acc16[nt][0][i] * 0.0625f;
+        acc[nt][3][i] += acc16[nt][1][i] * 0.0625f;
+      }
 
     if (KQ > 1) {
       // split K: this unit's partial sums go to partials[kq][row][column];
@@ -433,6 +463,7 @@ __global__ void __launch_bounds__(stream::kThreads, 2)
 // (in kq order), then bias, rounding and SwiGLU as in the fused epilogue.
 template <int NPROJ>
 __global__ void __launch_bounds__(256) awq_stream_reduce_kernel(ProjParams p) {
+  pdl_enter();  // programmatic dependent launch: the previous kernel is done
   const int64_t ncols = (int64_t)NPROJ * p.N;
   const int64_t per_row = p.N / 8;
   const int64_t total = p.A * per_row;
@@ -534,14 +565,14 @@ static moe_status launch_stream_r(const ProjParams &p0, cudaStream_t st) {
   auto kern = awq_fwd_stream_kernel<MT, NPROJ, NT, ROWS>;
   cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   const int per_sm = smem <= 110 * 1024 ? 2 : 1;
-  kern<<<num_sms() * per_sm, kThreads, smem, st>>>(m0, m1, p);
+  launch_pdl(kern, dim3(num_sms() * per_sm), dim3(kThreads), smem, st, m0, m1, p);
   moe_status s = check_launch("awq_fwd_stream_kernel");
   if (s != MOE_OK || p.kq == 1) return s;
   const int64_t work = p.A * (p.N / 8);
   int64_t blocks = (work + 255) / 256;
   const int64_t cap = (int64_t)num_sms() * 8;
   if (blocks > cap) blocks = cap;
-  awq_stream_reduce_kernel<NPROJ><<<(unsigned)blocks, 256, 0, st>>>(p);
+  launch_pdl(awq_stream_reduce_kernel<NPROJ>, dim3((unsigned)blocks), dim3(256), 0, st, p);
   return check_launch("awq_stream_reduce_kernel");
 }
 

@@ -39,14 +39,15 @@ namespace moe {
 
 namespace tc {
 constexpr int kBM = 128, kBN = 256, kBK = 64;
-constexpr int kStages = 3;
+constexpr int kLStages = 6;  // TMA ring: activation tile + packed words, six deep to cover the load latency
+constexpr int kBStages = 2;  // coefficient ring
 constexpr int kDqWarps = 8;
 constexpr int kEpWarps = 8;                                // two per TMEM lane quarter (column halves)
 constexpr int kThreads = (2 + kDqWarps + kEpWarps) * 32;  // 576
 constexpr int kABytes = kBM * kBK * 2;          // 16 KB activation tile
 constexpr int kBBytes = kBN * kBK * 2;          // 32 KB coefficient tile
 constexpr int kPBytes = kBK * (kBN / 8) * 4;    // 8 KB packed words
-constexpr int kStageBytes = kABytes + kBBytes + kPBytes;
+constexpr int kLBytes = kABytes + kPBytes;    // one TMA stage (24 KB: 1 KB aligned)
 constexpr int kTmemCols = 512;  // two 128 x 256 FP32 accumulators
 }  // namespace tc
 
@@ -62,19 +63,23 @@ template <typename MT, int NPROJ>
 __global__ void __launch_bounds__(tc::kThreads, 1)
     awq_fwd_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_w0,
                       const __grid_constant__ CUtensorMap map_w1, ProjParams p) {
+  pdl_enter();  // programmatic dependent launch: the previous kernel is done
   using namespace tc;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t *smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
-  uint8_t *stages = smem;  // kStages x [A | B | packed]
-  uint64_t *full = reinterpret_cast<uint64_t *>(stages + kStages * kStageBytes);
-  uint64_t *bready = full + kStages;
-  uint64_t *empty = bready + kStages;
-  uint64_t *accfull = empty + kStages;  // [2]
+  uint8_t *lring = smem;                           // kLStages x [A | packed]
+  uint8_t *bring = smem + kLStages * kLBytes;      // kBStages x B
+  uint64_t *full = reinterpret_cast<uint64_t *>(bring + kBStages * kBBytes);
+  uint64_t *empty = full + kLStages;               // MMA commit (A read) + dequant warps (words read)
+  uint64_t *bready = empty + kLStages;
+  uint64_t *bfree = bready + kBStages;
+  uint64_t *accfull = bfree + kBStages;  // [2]
   uint64_t *accempty = accfull + 2;     // [2]
   uint64_t *drain = accempty + 2;       // the issuer's last commit: no MMA in flight at teardown
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
   volatile int32_t *abort = reinterpret_cast<volatile int32_t *>(tmem_slot + 1);
-  int32_t *pre = reinterpret_cast<int32_t *>(tmem_slot + 4);  // [E + 1]
+  float *bias_s = reinterpret_cast<float *>(tmem_slot + 4);  // [2 tiles][256]: the tile's bias, staged
+  int32_t *pre = reinterpret_cast<int32_t *>(bias_s + 2 * kBN);  // [E + 1]
   int32_t *cnt = pre + (p.E + 1);                             // [E]
   int32_t *tmp = cnt + p.E;                                   // [32]
 
@@ -86,10 +91,13 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
   const int nk = (int)(K / kBK);
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < kLStages; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&bready[s], kDqWarps);
-      mbar_init(&empty[s], 1);
+      mbar_init(&empty[s], 1 + kDqWarps);
+    }
+    for (int b = 0; b < kBStages; ++b) {
+      mbar_init(&bready[b], kDqWarps);
+      mbar_init(&bfree[b], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&accfull[b], 1);
@@ -154,12 +162,12 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
           for (int i = 0; i < 4; ++i) src[i] = (int32_t)act_row(p, min((int64_t)row0 + 4 * lane + i, p.A - 1));
         }
         for (int kb = 0; kb < nk; ++kb, ++it) {
-          const uint32_t s = it % kStages, use = it / kStages;
+          const uint32_t s = it % kLStages, use = it / kLStages;
           bool ok = true;
-          uint8_t *st = stages + s * kStageBytes;
+          uint8_t *st = lring + s * kLBytes;
           if (lane == 0) {
             ok = use == 0 || tc_wait(&empty[s], (use - 1) & 1, p.status, abort);
-            if (ok) mbar_arrive_expect_tx(&full[s], kABytes + kPBytes);
+            if (ok) mbar_arrive_expect_tx(&full[s], kLBytes);
           }
           if (gather) ok = __shfl_sync(0xffffffffu, ok, 0);
           if (!ok) {
@@ -171,15 +179,15 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
             if (!gather) tma_load_2d(st, &map_x, &full[s], kb * kBK, row0);
             const int32_t wrow = (int32_t)(ti.e * K + (int64_t)kb * kBK);
             if (NPROJ == 2) {
-              tma_load_2d(st + kABytes + kBBytes, &map_w0, &full[s], ti.nt * 16, wrow);
-              tma_load_2d(st + kABytes + kBBytes + kPBytes / 2, &map_w1, &full[s], ti.nt * 16, wrow);
+              tma_load_2d(st + kABytes, &map_w0, &full[s], ti.nt * 16, wrow);
+              tma_load_2d(st + kABytes + kPBytes / 2, &map_w1, &full[s], ti.nt * 16, wrow);
             } else {
-              tma_load_2d(st + kABytes + kBBytes, &map_w0, &full[s], ti.nt * 32, wrow);
+              tma_load_2d(st + kABytes, &map_w0, &full[s], ti.nt * 32, wrow);
             }
           }
         }
       }
-      if (lane == 0) tma_drain(full, it, kStages, p.status);
+      if (lane == 0) tma_drain(full, it, kLStages, p.status);
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer: tile t accumulates in TMEM buffer t & 1
@@ -196,20 +204,22 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
         tc_fence_after();
         const uint32_t dacc = tmem + buf * kBN;
         for (int kb = 0; kb < nk; ++kb, ++it) {
-          const uint32_t s = it % kStages, ph = (it / kStages) & 1;
-          if (!tc_wait(&full[s], ph, p.status, abort) || !tc_wait(&bready[s], ph, p.status, abort)) {
+          const uint32_t s = it % kLStages, b = it % kBStages;
+          // the dequant warps arrive on bready only after the stage's TMA landed
+          if (!tc_wait(&bready[b], (it / kBStages) & 1, p.status, abort)) {
             live = false;
             break;
           }
           tc_fence_after();
-          const uint32_t a_addr = smem_u32(stages + s * kStageBytes);
-          const uint32_t b_addr = a_addr + kABytes;
+          const uint32_t a_addr = smem_u32(lring + s * kLBytes);
+          const uint32_t b_addr = smem_u32(bring + b * kBBytes);
           const uint64_t adesc = smem_desc(a_addr, 16, 1024);    // K-major, 8-row groups 1 KB apart
           const uint64_t bdesc = smem_desc(b_addr, 8192, 1024);  // MN-major: 64-col groups 8 KB, 8-row groups 1 KB
 #pragma unroll
           for (int j = 0; j < kBK / 16; ++j)
             umma_f16(dacc, adesc + (uint64_t)(2 * j), bdesc + (uint64_t)(128 * j), idesc, (kb | j) != 0);
           umma_commit(&empty[s]);
+          umma_commit(&bfree[b]);
         }
         if (!live) break;
         umma_commit(&accfull[buf]);
@@ -251,7 +261,8 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
       int64_t grp = 0;
       int gstage = 0;
       for (int kb = 0; kb < nk; ++kb, ++it) {
-        const uint32_t s = it % kStages, ph = (it / kStages) & 1;
+        const uint32_t s = it % kLStages, ph = (it / kLStages) & 1;
+        const uint32_t b = it % kBStages, buse = it / kBStages;
         if (gstage == 0) {  // a new group: take the prefetched zeros/scales, prefetch the next
           const uint32_t s4[4] = {pf_sv.x, pf_sv.y, pf_sv.z, pf_sv.w};
 #pragma unroll
@@ -272,7 +283,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
           live = false;
           break;
         }
-        uint8_t *st = stages + s * kStageBytes;
+        uint8_t *st = lring + s * kLBytes;
         if (convert) {
           // activation tile to the scale dtype, in place (layout-agnostic)
           uint4 *a4 = reinterpret_cast<uint4 *>(st);
@@ -285,12 +296,19 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
             v.w = act_pair_to_mt<MT>(v.w, p.act_dt, act_bad);
             a4[td + 256 * i] = v;
           }
+          fence_proxy_async_smem();  // the converted tile is read by the tensor core
         }
-        const uint32_t *pk = reinterpret_cast<const uint32_t *>(st + kABytes + kBBytes) + pk0;
-        uint8_t *bt = st + kABytes + b0;
+        const uint32_t *pk = reinterpret_cast<const uint32_t *>(st + kABytes) + pk0;
         uint32_t w[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) w[i] = pk[i * pk_step];
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[s]);  // words read (the MMA commit frees the activations)
+        if (buse > 0 && !tc_wait(&bfree[b], (buse - 1) & 1, p.status, abort)) {
+          live = false;
+          break;
+        }
+        uint8_t *bt = bring + b * kBBytes + b0;
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
           uint4 c;
@@ -302,19 +320,34 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
         }
         fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bready[s]);
+        if (lane == 0) mbar_arrive(&bready[b]);
       }
     }
     if (act_bad) report(p.status, MOE_DEVICE_ERR_ACT_RANGE);
   } else {
-    // ---------------- epilogue warps: TMEM -> registers -> bias, rounding, SwiGLU -> HBM
+    // ---------------- epilogue warps: TMEM -> registers -> bias, rounding,
+    // SwiGLU -> HBM.  The tile's bias is staged in shared memory before its
+    // accumulator is waited for (one named barrier per tile, two buffers) and
+    // TMEM loads are issued in pairs before one wait.  After an abort every
+    // epilogue warp still runs the loop (the named barrier stays matched) but
+    // reads, stores and arrives on nothing.
     const int q = warp & 3;                          // TMEM lane quarter of this warp
     const int hf = (warp - 2 - kDqWarps) >> 2;       // column half drained by this warp
+    const int et = threadIdx.x - (2 + kDqWarps) * 32;  // 0 .. 255
+    const bool bf = p.act_dt == MOE_BF16;
     uint32_t tcount = 0;
     for (int64_t tile = blockIdx.x; tile < total; tile += gridDim.x, ++tcount) {
       const TileInfo ti = tile_info(tile);
       const uint32_t buf = tcount & 1;
-      if (!tc_wait(&accfull[buf], (tcount >> 1) & 1, p.status, abort)) break;
+      float *bt = bias_s + buf * kBN;
+      {  // NPROJ == 2: gate bias of the tile's 128 features, then up; else 256 columns
+        const int j = NPROJ == 2 ? et >> 7 : 0;
+        const int64_t n = NPROJ == 2 ? (int64_t)ti.nt * 128 + (et & 127) : (int64_t)ti.nt * kBN + et;
+        bt[et] = (p.bias[j] && n < p.N) ? ld_as_float(p.bias[j], p.bias_dt, (int64_t)ti.e * p.N + n) : 0.f;
+      }
+      const bool ok = tc_wait(&accfull[buf], (tcount >> 1) & 1, p.status, abort);
+      named_barrier(2, kEpWarps * 32);
+      if (!ok) continue;
       tc_fence_after();
       const int trow = ti.mt * kBM + 32 * q + lane;  // row within the expert
       const bool row_ok = trow < ti.m && !*abort;
@@ -324,25 +357,48 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
 #pragma unroll 1
         for (int c8 = 4 * hf; c8 < 4 * hf + 4; ++c8) {
           const int f0 = c8 * 16;  // feature within the tile
+          uint32_t gr[16], ur[16];
+          tmem_ld16_async(tbase + f0, gr);
+          tmem_ld16_async(tbase + 128 + f0, ur);
+          tmem_wait_ld();
           float gv[16], uv[16];
-          tmem_ld16(tbase + f0, gv);
-          tmem_ld16(tbase + 128 + f0, uv);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            gv[i] = __uint_as_float(gr[i]);
+            uv[i] = __uint_as_float(ur[i]);
+          }
           const int64_t n0 = (int64_t)ti.nt * 128 + f0;
           if (row_ok && n0 < p.N) {
 #pragma unroll
-            for (int v8 = 0; v8 < 2; ++v8) finish8<2>(p, ti.e, row, n0 + 8 * v8, gv + 8 * v8, uv + 8 * v8);
+            for (int v8 = 0; v8 < 2; ++v8) {
+              const float *bg = bt + f0 + 8 * v8, *bu = bt + 128 + f0 + 8 * v8;
+              if (bf) finish8_bt<2, true>(p, row, n0 + 8 * v8, gv + 8 * v8, uv + 8 * v8, bg, bu);
+              else finish8_bt<2, false>(p, row, n0 + 8 * v8, gv + 8 * v8, uv + 8 * v8, bg, bu);
+            }
           }
         }
       } else {
 #pragma unroll 1
         for (int c8 = 4 * hf; c8 < 4 * hf + 4; ++c8) {
           const int f0 = c8 * 32;
+          uint32_t ra[16], rb[16];
+          tmem_ld16_async(tbase + f0, ra);
+          tmem_ld16_async(tbase + f0 + 16, rb);
+          tmem_wait_ld();
           float yv[32];
-          tmem_ld32(tbase + f0, yv);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            yv[i] = __uint_as_float(ra[i]);
+            yv[16 + i] = __uint_as_float(rb[i]);
+          }
           const int64_t n0 = (int64_t)ti.nt * 256 + f0;
           if (row_ok && n0 < p.N) {
 #pragma unroll
-            for (int v8 = 0; v8 < 4; ++v8) finish8<1>(p, ti.e, row, n0 + 8 * v8, yv + 8 * v8, yv + 8 * v8);
+            for (int v8 = 0; v8 < 4; ++v8) {
+              const float *b8 = bt + f0 + 8 * v8;
+              if (bf) finish8_bt<1, true>(p, row, n0 + 8 * v8, yv + 8 * v8, yv + 8 * v8, b8, b8);
+              else finish8_bt<1, false>(p, row, n0 + 8 * v8, yv + 8 * v8, yv + 8 * v8, b8, b8);
+            }
           }
         }
       }
@@ -363,7 +419,8 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
 // ------------------------------------------------------------------ launch
 
 static size_t tc_smem(int64_t E) {
-  return 1024 + (size_t)tc::kStages * tc::kStageBytes + 256 + (size_t)(2 * E + 1 + 32) * 4;
+  return 1024 + (size_t)tc::kLStages * tc::kLBytes + (size_t)tc::kBStages * tc::kBBytes + 256 +
+         (size_t)2 * tc::kBN * 4 + (size_t)(2 * E + 1 + 32) * 4;
 }
 
 // The tile needs whole 64-row steps inside one group, 16-byte word-row
@@ -393,7 +450,7 @@ static moe_status launch_tc_t(const ProjParams &p, cudaStream_t st) {
   const size_t smem = tc_smem(p.E);
   auto kern = awq_fwd_tc_kernel<MT, NPROJ>;
   cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  kern<<<num_sms(), kThreads, smem, st>>>(mx, m0, m1, p);
+  launch_pdl(kern, dim3(num_sms()), dim3(kThreads), smem, st, mx, m0, m1, p);
   return check_launch("awq_fwd_tc_kernel");
 }
 

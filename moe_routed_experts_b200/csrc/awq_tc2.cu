@@ -66,6 +66,7 @@ template <typename MT, int NPROJ>
 __global__ void __launch_bounds__(tc2::kThreads, 1)
     awq_fwd_tc2_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_w0,
                        const __grid_constant__ CUtensorMap map_w1, ProjParams p) {
+  pdl_enter();  // programmatic dependent launch: the previous kernel is done
   using namespace tc2;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t *smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
@@ -80,7 +81,8 @@ __global__ void __launch_bounds__(tc2::kThreads, 1)
   uint64_t *drain = accempty + 2;        // the issuer's last commit: no MMA in flight at teardown
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
   volatile int32_t *abort = reinterpret_cast<volatile int32_t *>(tmem_slot + 1);
-  int32_t *pre = reinterpret_cast<int32_t *>(tmem_slot + 4);  // [E + 1]
+  float *bias_s = reinterpret_cast<float *>(tmem_slot + 4);  // [2 tiles][256]: the tile's bias, staged
+  int32_t *pre = reinterpret_cast<int32_t *>(bias_s + 2 * kBN);  // [E + 1]
   int32_t *cnt = pre + (p.E + 1);                             // [E]
   int32_t *tmp = cnt + p.E;                                   // [32]
 
@@ -330,14 +332,29 @@ __global__ void __launch_bounds__(tc2::kThreads, 1)
     }
     if (act_bad) report(p.status, MOE_DEVICE_ERR_ACT_RANGE);
   } else {
-    // ---------------- epilogue warps: this CTA's 128 rows of the tile
+    // ---------------- epilogue warps: this CTA's 128 rows of the tile.  The
+    // tile's bias is staged in shared memory before its accumulator is
+    // waited for (one named barrier per tile, two buffers), and TMEM loads
+    // are issued in pairs before one wait.  After an abort every epilogue
+    // warp still runs the loop (the named barrier stays matched) but reads,
+    // stores and arrives on nothing.
     const int q = warp & 3;                     // TMEM lane quarter
     const int hf = (warp - 2 - kDqWarps) >> 2;  // column half drained by this warp
+    const int et = threadIdx.x - (2 + kDqWarps) * 32;  // 0 .. 255
+    const bool bf = p.act_dt == MOE_BF16;
     uint32_t tcount = 0;
     for (int64_t tile = pair; tile < total; tile += npairs, ++tcount) {
       const PairTile ti = tile_info(tile);
       const uint32_t buf = tcount & 1;
-      if (!tc_wait(&accfull[buf], (tcount >> 1) & 1, p.status, abort)) break;
+      float *bt = bias_s + buf * kBN;
+      {  // NPROJ == 2: gate bias of the tile's 128 features, then up; else 256 columns
+        const int j = NPROJ == 2 ? et >> 7 : 0;
+        const int64_t n = NPROJ == 2 ? (int64_t)ti.nt * kHalf + (et & (kHalf - 1)) : (int64_t)ti.nt * kBN + et;
+        bt[et] = (p.bias[j] && n < p.N) ? ld_as_float(p.bias[j], p.bias_dt, (int64_t)ti.e * p.N + n) : 0.f;
+      }
+      const bool ok = tc_wait(&accfull[buf], (tcount >> 1) & 1, p.status, abort);
+      named_barrier(2, kEpWarps * 32);
+      if (!ok) continue;
       tc_fence_after();
       const int trow = ti.mt * 2 * kBM + kBM * (int)rank + 32 * q + lane;
       const bool row_ok = trow < ti.m && !*abort;
@@ -347,25 +364,49 @@ __global__ void __launch_bounds__(tc2::kThreads, 1)
 #pragma unroll 1
         for (int c8 = 4 * hf; c8 < 4 * hf + 4; ++c8) {
           const int f0 = c8 * 16;
+          uint32_t gr[16], ur[16];
+          tmem_ld16_async(tbase + f0, gr);
+          tmem_ld16_async(tbase + kHalf + f0, ur);
+          tmem_wait_ld();
           float gv[16], uv[16];
-          tmem_ld16(tbase + f0, gv);
-          tmem_ld16(tbase + kHalf + f0, uv);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            gv[i] = __uint_as_float(gr[i]);
+            uv[i] = __uint_as_float(ur[i]);
+          }
           const int64_t n0 = (int64_t)ti.nt * kHalf + f0;
           if (row_ok && n0 < p.N) {
 #pragma unroll
-            for (int v8 = 0; v8 < 2; ++v8) finish8<2>(p, ti.e, row, n0 + 8 * v8, gv + 8 * v8, uv + 8 * v8);
+            for (int v8 = 0; v8 < 2; ++v8) {
+              const float *bg = bt + f0 + 8 * v8, *bu = bt + kHalf + f0 + 8 * v8;
+              if (bf) finish8_bt<2, true>(p, row, n0 + 8 * v8, gv + 8 * v8, uv + 8 * v8, bg, bu);
+              else finish8_bt<2, false>(p, row, n0 + 8 * v8, gv + 8 * v8, uv + 8 * v8, bg, bu);
+            }
           }
         }
       } else {
 #pragma unroll 1
-        for (int c16 = 8 * hf; c16 < 8 * hf + 8; ++c16) {
-          const int f0 = c16 * 16;
-          float yv[16];
-          tmem_ld16(tbase + f0, yv);
+        for (int c32 = 4 * hf; c32 < 4 * hf + 4; ++c32) {
+          const int f0 = c32 * 32;
+          uint32_t ra[16], rb[16];
+          tmem_ld16_async(tbase + f0, ra);
+          tmem_ld16_async(tbase + f0 + 16, rb);
+          tmem_wait_ld();
+          float yv[32];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            yv[i] = __uint_as_float(ra[i]);
+            yv[16 + i] = __uint_as_float(rb[i]);
+          }
           const int64_t n0 = (int64_t)ti.nt * kBN + f0;
           if (row_ok && n0 < p.N) {
 #pragma unroll
-            for (int v8 = 0; v8 < 2; ++v8) finish8<1>(p, ti.e, row, n0 + 8 * v8, yv + 8 * v8, yv + 8 * v8);
+            for (int v8 = 0; v8 < 4; ++v8) {
+              if (n0 + 8 * v8 >= p.N) break;
+              const float *b8 = bt + f0 + 8 * v8;
+              if (bf) finish8_bt<1, true>(p, row, n0 + 8 * v8, yv + 8 * v8, yv + 8 * v8, b8, b8);
+              else finish8_bt<1, false>(p, row, n0 + 8 * v8, yv + 8 * v8, yv + 8 * v8, b8, b8);
+            }
           }
         }
       }
@@ -389,7 +430,7 @@ __global__ void __launch_bounds__(tc2::kThreads, 1)
 
 static size_t tc2_smem(int64_t E) {
   return 1024 + (size_t)tc2::kLStages * tc2::kLBytes + (size_t)tc2::kBStages * tc2::kBBytes + 256 +
-         (size_t)(2 * E + 1 + 32) * 4;
+         (size_t)2 * tc2::kBN * 4 + (size_t)(2 * E + 1 + 32) * 4;
 }
 
 bool tc2_fits(const ProjParams &p) {
@@ -415,11 +456,13 @@ static moe_status launch_tc2_t(const ProjParams &p, cudaStream_t st) {
   auto kern = awq_fwd_tc2_kernel<MT, NPROJ>;
   cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // see launch_pdl
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
@@ -432,6 +475,7 @@ static moe_status launch_tc2_t(const ProjParams &p, cudaStream_t st) {
     return set_error(MOE_ERR_CUDA, "no co-resident SM pair for the tcgen05 pair projection");
   }
   cfg.gridDim = dim3(2 * clusters);  // persistent: every pair resident at once
+  cfg.numAttrs = 2;
   cudaLaunchKernelEx(&cfg, kern, mx, m0, m1, p);
   return check_launch("awq_fwd_tc2_kernel");
 }

@@ -62,6 +62,7 @@ __device__ __forceinline__ void order_token(const uint32_t *sel, const int32_t *
 
 template <bool VEC>
 __global__ void __launch_bounds__(kCombThreads) combine_kernel(CombineParams p) {
+  pdl_enter();  // programmatic dependent launch: the previous kernel is done
   __shared__ int32_t ord_row[MOE_MAX_TOP_K];
   __shared__ float ord_w[MOE_MAX_TOP_K];
   const int64_t t = blockIdx.x;
@@ -252,9 +253,9 @@ static moe_status launch_combine(const CombineParams &p, cudaStream_t st, const 
   if (p.T == 0) return MOE_OK;
   const bool vec = aligned16(p.y) && aligned16(p.out) && p.H % 8 == 0;
   if (vec)
-    combine_kernel<true><<<(unsigned)p.T, kCombThreads, 0, st>>>(p);
+    launch_pdl(combine_kernel<true>, dim3((unsigned)p.T), dim3(kCombThreads), 0, st, p);
   else
-    combine_kernel<false><<<(unsigned)p.T, kCombThreads, 0, st>>>(p);
+    launch_pdl(combine_kernel<false>, dim3((unsigned)p.T), dim3(kCombThreads), 0, st, p);
   return check_launch(what);
 }
 

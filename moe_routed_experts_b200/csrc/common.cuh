@@ -24,7 +24,37 @@ inline int dtype_bytes(moe_dtype d) { return d == MOE_F32 ? 4 : 2; }
 inline bool valid_dtype(int d) { return d == MOE_F32 || d == MOE_F16 || d == MOE_BF16; }
 int num_sms();
 
+// Launch with programmatic dependent launch: the kernel may be scheduled
+// while the previous kernel of the stream is still finishing; its first
+// statement (pdl_wait) then waits for that kernel's completion and memory,
+// and pdl_trigger lets the next kernel be scheduled in turn.  Saves the
+// launch gap and the tail of each kernel in the forward chain.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                              Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 // ---------------------------------------------------------------- device side
+
+// Wait for the previous kernel of the stream (its writes visible), then
+// allow the next one to be scheduled.  No-ops without programmatic launch.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_enter() {
+  pdl_wait();
+  pdl_trigger();
+}
 
 __device__ __forceinline__ void report(int32_t *status, int bits) {
   if (status) atomicOr(status, bits);
@@ -111,26 +141,22 @@ __device__ __forceinline__ uint32_t f16x2_to_bf16x2(uint32_t v) {
   return *reinterpret_cast<uint32_t *>(&b);
 }
 
-// Nonzero when a BF16 value of the pair lies outside F16's normal range
-// (|v| >= 65536, inf or NaN, or 0 < |v| < 2^-14): there BF16 -> F16 is not
-// exact (overflow to inf, or a subnormal with fewer significant bits).  BF16
-// has no values in (65504, 65536).
-__device__ __forceinline__ uint32_t bf16x2_outside_f16_normal(uint32_t v) {
-  const uint32_t lo = v & 0x7FFFu, hi = (v >> 16) & 0x7FFFu;
-  return (uint32_t)(lo >= 0x4780u) | (uint32_t)(lo - 1u < 0x387Fu) | (uint32_t)(hi >= 0x4780u) |
-         (uint32_t)(hi - 1u < 0x387Fu);
-}
-
 // Activation (or gradient) pair in the tensor-core operand dtype MT.  A
-// BF16 -> F16 conversion outside F16's normal range ORs 1 into `bad` (the
-// caller reports MOE_DEVICE_ERR_ACT_RANGE); F16 -> BF16 always fits the range
-// and rounds to BF16's 8 significant bits.
+// BF16 -> F16 conversion that changes a value grossly ORs 1 into `bad` (the
+// caller reports MOE_DEVICE_ERR_ACT_RANGE): a finite value above F16's range
+// (it becomes inf) or a NaN.  Values below F16's normal range keep what
+// F16's subnormal grid holds (an absolute change below 2^-25, not reported);
+// F16 -> BF16 always fits the range and rounds to BF16's 8 significant bits.
 template <typename MT>
 __device__ __forceinline__ uint32_t act_pair_to_mt(uint32_t v, int act_dt, uint32_t &bad) {
   if constexpr (sizeof(MT) == 2 && std::is_same<MT, __half>::value) {
     if (act_dt != MOE_BF16) return v;
-    bad |= bf16x2_outside_f16_normal(v);
-    return bf16x2_to_f16x2(v);
+    const uint32_t r = bf16x2_to_f16x2(v);
+    // result inf/NaN in a lane whose source is not +-inf
+    const uint32_t lo_bad = ((r & 0x7C00u) == 0x7C00u) & ((v & 0x7FFFu) != 0x7F80u);
+    const uint32_t hi_bad = ((r & 0x7C000000u) == 0x7C000000u) & ((v & 0x7FFF0000u) != 0x7F800000u);
+    bad |= lo_bad | hi_bad;
+    return r;
   } else {
     return act_dt == MOE_F16 ? f16x2_to_bf16x2(v) : v;
   }

@@ -86,6 +86,7 @@ struct RouteParams {
 // k selection rounds; R = 0 re-reads them each round (large E).
 template <int R>
 __global__ void __launch_bounds__(1024) route_rank_kernel(RouteParams p) {
+  pdl_enter();  // programmatic dependent launch: the previous kernel is done
   extern __shared__ int32_t sm[];
   int32_t *cnt = sm;                      // [E]
   int32_t *tmp = cnt + p.E;               // [32]
@@ -209,6 +210,7 @@ __global__ void __launch_bounds__(1024) route_rank_kernel(RouteParams p) {
 // Chunk bases (in place over hist) and offsets, one block.
 __global__ void __launch_bounds__(kScanThreads) route_scan_kernel(int32_t *hist, int nch, int E,
                                                                    int32_t *offsets) {
+  pdl_enter();  // programmatic dependent launch: the previous kernel is done
   extern __shared__ int32_t sm[];
   int32_t *totals = sm;                // [E]
   int32_t *tmp = totals + E;           // [32]
@@ -280,6 +282,7 @@ __device__ __forceinline__ int64_t scatter_pos(const ScatterParams &p, int64_t a
 // segments loaded before they are stored.  Otherwise one warp per
 // (assignment, 64-byte segment) with 2-byte accesses.
 __global__ void __launch_bounds__(256) route_scatter_kernel(ScatterParams p) {
+  pdl_enter();  // programmatic dependent launch: the previous kernel is done
   const int lane = threadIdx.x & 31;
   const int64_t wid = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int64_t nw = ((int64_t)gridDim.x * blockDim.x) >> 5;
@@ -510,7 +513,7 @@ static moe_status route_impl(const char *fn, const void *x, moe_dtype x_dtype, i
   if (smem > 48 * 1024) cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   // a warp per token (or per few tokens): the widest block the kernel takes
   const int threads = 1024;
-  kern<<<(unsigned)lay.nchunks, threads, smem, st>>>(rp);
+  launch_pdl(kern, dim3((unsigned)lay.nchunks), dim3(threads), smem, st, rp);
   moe_status s = check_launch("route_rank_kernel");
   if (s != MOE_OK) return s;
   if (!rp.single) {
@@ -518,7 +521,7 @@ static moe_status route_impl(const char *fn, const void *x, moe_dtype x_dtype, i
     while (tpe * 2 * E <= kScanThreads && tpe * 2 <= lay.nchunks) tpe *= 2;
     size_t ssm = sizeof(int32_t) * (size_t)(E + 32 + tpe * E);
     if (ssm > 48 * 1024) cudaFuncSetAttribute(route_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ssm);
-    route_scan_kernel<<<1, kScanThreads, ssm, st>>>(hist, (int)lay.nchunks, (int)E, offsets);
+    launch_pdl(route_scan_kernel, dim3(1), dim3(kScanThreads), ssm, st, hist, (int)lay.nchunks, (int)E, offsets);
     s = check_launch("route_scan_kernel");
     if (s != MOE_OK) return s;
   }
@@ -544,7 +547,7 @@ static moe_status route_impl(const char *fn, const void *x, moe_dtype x_dtype, i
   int64_t blocks = (units + 7) / 8;
   int64_t cap = (int64_t)num_sms() * 16;
   if (blocks > cap) blocks = cap;
-  route_scatter_kernel<<<(unsigned)blocks, 256, 0, st>>>(sp);
+  launch_pdl(route_scatter_kernel, dim3((unsigned)blocks), dim3(256), 0, st, sp);
   return check_launch("route_scatter_kernel");
 }
 

@@ -125,6 +125,29 @@ __device__ __forceinline__ void finish8_t(const ProjParams &p, int e, int64_t ro
   *reinterpret_cast<uint4 *>(p.out + row * p.N + n0) = make_uint4(o[0], o[1], o[2], o[3]);
 }
 
+// finish8_t with the bias of the 8 columns already in registers (bg, bu).
+template <int NPROJ, bool BF>
+__device__ __forceinline__ void finish8_bt(const ProjParams &p, int64_t row, int64_t n0, const float *g, const float *u,
+                                           const float *bg, const float *bu) {
+  uint32_t o[4];
+  if (NPROJ == 2) {
+    uint32_t og[4], ou[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      og[i] = round_pair<BF>(g[2 * i] + bg[2 * i], g[2 * i + 1] + bg[2 * i + 1]);
+      ou[i] = round_pair<BF>(u[2 * i] + bu[2 * i], u[2 * i + 1] + bu[2 * i + 1]);
+      const float2 G = unpack_pair<BF>(og[i]), U = unpack_pair<BF>(ou[i]);
+      o[i] = round_pair<BF>(swiglu1(G.x, U.x), swiglu1(G.y, U.y));
+    }
+    if (p.gout) *reinterpret_cast<uint4 *>(p.gout + row * p.N + n0) = make_uint4(og[0], og[1], og[2], og[3]);
+    if (p.uout) *reinterpret_cast<uint4 *>(p.uout + row * p.N + n0) = make_uint4(ou[0], ou[1], ou[2], ou[3]);
+  } else {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) o[i] = round_pair<BF>(g[2 * i] + bg[2 * i], g[2 * i + 1] + bg[2 * i + 1]);
+  }
+  *reinterpret_cast<uint4 *>(p.out + row * p.N + n0) = make_uint4(o[0], o[1], o[2], o[3]);
+}
+
 // Final values of 8 consecutive output columns n0.. of row `row` of local
 // expert e from FP32 sums (gate sums g, up sums u for the pair): bias, one
 // rounding to the activation dtype, SwiGLU from the rounded G and U.

@@ -150,11 +150,15 @@ def test_inconsistent_offsets_are_flagged_not_faulted(path):
         assert int(st.item()) & 2, bad
 
 
-@pytest.mark.parametrize("value", [70000.0, 1e-6, float("inf")], ids=["above_f16_max", "below_f16_normal", "inf"])
-def test_activation_outside_f16_range_is_flagged(value, path):
-    # F16 scales with BF16 inputs: the tensor-core operand is F16, so a BF16
-    # activation or gradient outside F16's normal range cannot be converted
-    # exactly; the projection and the input VJP report it (and only it)
+@pytest.mark.parametrize("value,flagged", [(70000.0, True), (float("nan"), True), (1e-7, False), (2.0 ** -16, False),
+                                           (65280.0, False), (float("inf"), False)],
+                         ids=["overflow", "nan", "below_f16_subnormal_grid", "on_f16_subnormal_grid",
+                              "bf16_max_below_65504", "inf_converts_exactly"])
+def test_f16_range_overflow_is_flagged(value, flagged, path):
+    # F16 scales with BF16 inputs: the tensor-core operand is F16; a finite
+    # BF16 activation or gradient above F16's range (it would become inf) or
+    # a NaN is reported by the projection and the input VJP, and only those
+    # (tiny values keep what F16's subnormal grid holds: under 2^-25 absolute)
     rng = np.random.default_rng(11)
     E, K, N, g, A = 2, 256, 128, 64, 256
     proj = inputs.draw_projection(rng, E, K, N, g, "f16", False, 0.0)
@@ -167,16 +171,17 @@ def test_activation_outside_f16_range_is_flagged(value, path):
     B.awq_input_backward(gr, off, dproj, g, device_status=st)
     torch.cuda.synchronize()
     assert int(st.item()) == 0  # in-range inputs: nothing reported
+    want = 16 if flagged else 0  # MOE_DEVICE_ERR_ACT_RANGE
     x[A - 3, K - 5] = value
     st = B.new_status()
     B.awq_grouped_down(x, off, dproj, g, device_status=st)
     torch.cuda.synchronize()
-    assert int(st.item()) == 16, int(st.item())  # MOE_DEVICE_ERR_ACT_RANGE
+    assert int(st.item()) == want, int(st.item())
     gr[7, 3] = -value
     st = B.new_status()
     B.awq_input_backward(gr, off, dproj, g, device_status=st)
     torch.cuda.synchronize()
-    assert int(st.item()) == 16, int(st.item())
+    assert int(st.item()) == want, int(st.item())
 
 
 def test_row_index_out_of_range_is_flagged():

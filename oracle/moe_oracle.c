@@ -333,57 +333,113 @@ void oracle_copy_rows(const void *x, int64_t H, int64_t elem_bytes, const int32_
 /* Grouped projection of selected rows.                                */
 /* ------------------------------------------------------------------ */
 
+/* The rows of expert e, in ascending order; returns their count. */
+static int64_t rows_of_expert(const int32_t *row_expert, int64_t R, int64_t e, int64_t *list) {
+    int64_t n = 0;
+    for (int64_t r = 0; r < R; ++r)
+        if (row_expert[r] == e) list[n++] = r;
+    return n;
+}
+
+/* Rows are taken ROW_BLOCK at a time so that each row of W, once loaded,
+ * serves the whole block; every output still takes its terms in order. */
+#define ROW_BLOCK 16
+
 /* Rows r with row_expert[r] == e: out[r,n] = sum_kk x[r,kk] * W[kk,n] (+ bias[n]),
  * accumulated in double; mode 0 stores RNE in odt, 1 the double sum, 2 the
  * double sum of magnitudes (see oracle_project). */
 static void expert_rows_times_W(const void *x, int xdt, int64_t R, int64_t K, int64_t N,
                                 const int32_t *row_expert, int64_t e, const double *W,
                                 const void *be, int bdt, int mode, void *out, int odt) {
+    int64_t *list = (int64_t *)malloc(sizeof(int64_t) * (size_t)(R > 0 ? R : 1));
+    const int64_t nr = rows_of_expert(row_expert, R, e, list);
 #pragma omp parallel for schedule(dynamic, 1)
-    for (int64_t r = 0; r < R; ++r) {
-        if (row_expert[r] != e) continue;
-        double *acc = (double *)calloc((size_t)N, sizeof(double));
+    for (int64_t b0 = 0; b0 < nr; b0 += ROW_BLOCK) {
+        const int64_t nb = nr - b0 < ROW_BLOCK ? nr - b0 : ROW_BLOCK;
+        double *acc = (double *)calloc((size_t)(nb * N), sizeof(double));
         for (int64_t kk = 0; kk < K; ++kk) {
-            double xv = load_val(x, xdt, r * K + kk);
             const double *Wr = W + kk * N;
-            if (mode == 2)
-                for (int64_t n = 0; n < N; ++n) acc[n] += fabs(xv * Wr[n]);
-            else
-                for (int64_t n = 0; n < N; ++n) acc[n] += xv * Wr[n];
+            for (int64_t i = 0; i < nb; ++i) {
+                const double xv = load_val(x, xdt, list[b0 + i] * K + kk);
+                double *a = acc + i * N;
+                /* each a[n] takes its terms in kk order; the n lanes are independent */
+                if (mode == 2) {
+#pragma omp simd
+                    for (int64_t n = 0; n < N; ++n) a[n] += fabs(xv * Wr[n]);
+                } else {
+#pragma omp simd
+                    for (int64_t n = 0; n < N; ++n) a[n] += xv * Wr[n];
+                }
+            }
         }
-        for (int64_t n = 0; n < N; ++n) {
-            double b = (be && ORACLE_MUTANT != 7) ? load_val(be, bdt, n) : 0.0;
-            double v = acc[n] + (mode == 2 ? fabs(b) : b);
-            if (mode >= 1) ((double *)out)[r * N + n] = v;
-            else store_val(out, odt, r * N + n, v);
+        for (int64_t i = 0; i < nb; ++i) {
+            const int64_t r = list[b0 + i];
+            for (int64_t n = 0; n < N; ++n) {
+                double b = (be && ORACLE_MUTANT != 7) ? load_val(be, bdt, n) : 0.0;
+                double v = acc[i * N + n] + (mode == 2 ? fabs(b) : b);
+                if (mode >= 1) ((double *)out)[r * N + n] = v;
+                else store_val(out, odt, r * N + n, v);
+            }
         }
         free(acc);
     }
+    free(list);
 }
 
 /* Rows r with row_expert[r] == e: out[r,kk] = sum_n grad[r,n] W[kk,n]
- * (+ sum_n grad2[r,n] W2[kk,n]), one double accumulator; modes as above. */
+ * (+ sum_n grad2[r,n] W2[kk,n]), one double accumulator per output taking
+ * its terms in n order (grad's, then grad2's); modes as above.  The loops
+ * run over n outside and kk inside (on W transposed) so that the kk lanes,
+ * which are independent, can be vectorised without reordering any sum. */
+static void add_rows_times_WT(const void *grad, int gdt, const int64_t *rows, int64_t nb, int64_t N, int64_t K,
+                              const double *WT, int mode, double *acc) {
+    for (int64_t n = 0; n < N; ++n) {
+        const double *Wc = WT + n * K;
+        for (int64_t i = 0; i < nb; ++i) {
+            const double gv = load_val(grad, gdt, rows[i] * N + n);
+            double *a = acc + i * K;
+            if (mode == 2) {
+#pragma omp simd
+                for (int64_t kk = 0; kk < K; ++kk) a[kk] += fabs(gv * Wc[kk]);
+            } else {
+#pragma omp simd
+                for (int64_t kk = 0; kk < K; ++kk) a[kk] += gv * Wc[kk];
+            }
+        }
+    }
+}
+
+static double *transposed(const double *W, int64_t K, int64_t N) {
+    double *WT = (double *)malloc(sizeof(double) * (size_t)(K * N));
+    for (int64_t kk = 0; kk < K; ++kk)
+        for (int64_t n = 0; n < N; ++n) WT[n * K + kk] = W[kk * N + n];
+    return WT;
+}
+
 static void expert_rows_times_WT(const void *grad, int gdt, int64_t R, int64_t N, int64_t K,
                                  const int32_t *row_expert, int64_t e, const double *W,
                                  const void *grad2, const double *W2, int mode, void *out, int odt) {
+    int64_t *list = (int64_t *)malloc(sizeof(int64_t) * (size_t)(R > 0 ? R : 1));
+    const int64_t nr = rows_of_expert(row_expert, R, e, list);
+    double *WT = transposed(W, K, N);
+    double *W2T = (W2 && ORACLE_MUTANT != 9) ? transposed(W2, K, N) : NULL;
 #pragma omp parallel for schedule(dynamic, 1)
-    for (int64_t r = 0; r < R; ++r) {
-        if (row_expert[r] != e) continue;
-        for (int64_t kk = 0; kk < K; ++kk) {
-            double acc = 0.0;
-            for (int64_t n = 0; n < N; ++n) {
-                double pr = load_val(grad, gdt, r * N + n) * W[kk * N + n];
-                acc += mode == 2 ? fabs(pr) : pr;
+    for (int64_t b0 = 0; b0 < nr; b0 += ROW_BLOCK) {
+        const int64_t nb = nr - b0 < ROW_BLOCK ? nr - b0 : ROW_BLOCK;
+        double *acc = (double *)calloc((size_t)(nb * K), sizeof(double));
+        add_rows_times_WT(grad, gdt, list + b0, nb, N, K, WT, mode, acc);
+        if (W2T) add_rows_times_WT(grad2, gdt, list + b0, nb, N, K, W2T, mode, acc);
+        for (int64_t i = 0; i < nb; ++i)
+            for (int64_t kk = 0; kk < K; ++kk) {
+                const int64_t r = list[b0 + i];
+                if (mode >= 1) ((double *)out)[r * K + kk] = acc[i * K + kk];
+                else store_val(out, odt, r * K + kk, acc[i * K + kk]);
             }
-            if (W2 && ORACLE_MUTANT != 9)
-                for (int64_t n = 0; n < N; ++n) {
-                    double pr = load_val(grad2, gdt, r * N + n) * W2[kk * N + n];
-                    acc += mode == 2 ? fabs(pr) : pr;
-                }
-            if (mode >= 1) ((double *)out)[r * K + kk] = acc;
-            else store_val(out, odt, r * K + kk, acc);
-        }
+        free(acc);
     }
+    free(WT);
+    free(W2T);
+    free(list);
 }
 
 /* Rows r < R of x ([R,K] in dtype xdt) go through the projection of their

@@ -193,7 +193,7 @@ def main():
         sub = measure(WORKLOADS[name], args, min(args.steps, 20), world, rank, local, cpu=False)
         if rank == 0:
             line["workloads"][name] = {k: sub[k] for k in (
-                "value", "unit", "ms_per_step", "fwd_ms", "bwd_ms", "tflops", "packed_weight_gbs",
+                "value", "unit", "ms_per_step", "fwd_ms", "bwd_ms", "gather_mode", "tflops", "packed_weight_gbs",
                 "packed_weight_frac", "roofline", "e2e", "gpu_launches", "clocks", "device_status", "config", "steps")
                 if k in sub}
     if "nf4" in extra:
@@ -378,6 +378,43 @@ def measure(w, args, steps, world, rank, local, cpu):
         nog.append(a.elapsed_time(b))
     nograph_ms = statistics.median(nog)
 
+    # the gather mode of the dispatch (no COPY: the gate/up projection reads
+    # x rows through src_token), same protocol, forward-only workloads
+    gather_ms = None
+    if not w.backward:
+        def step_gather():
+            ffn.forward(dev, buf, gather=True)
+
+        for _ in range(3):
+            step_gather()
+        torch.cuda.synchronize()
+        graph_g = None
+        if not args.no_graph:
+            graph_g = torch.cuda.CUDAGraph()
+            sg = torch.cuda.Stream()
+            sg.wait_stream(torch.cuda.current_stream())
+            with torch.cuda.stream(sg):
+                step_gather()
+                torch.cuda.synchronize()
+                with torch.cuda.graph(graph_g, stream=sg):
+                    step_gather()
+            torch.cuda.current_stream().wait_stream(sg)
+            torch.cuda.synchronize()
+        gt = []
+        for i in range(steps):
+            flush.fill_(i & 0xFF)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            if graph_g is not None:
+                graph_g.replay()
+            else:
+                step_gather()
+            b.record()
+            torch.cuda.synchronize()
+            gt.append(a.elapsed_time(b))
+        gather_ms = sum(gt) / len(gt)
+        del graph_g
+
     # end to end through the public API: pinned host inputs in, output back, every step
     x_host = torch.from_numpy(inp["x"].view(np.int16)).view(torch.bfloat16).pin_memory()
     l_host = torch.from_numpy(inp["logits"]).pin_memory()
@@ -396,11 +433,13 @@ def measure(w, args, steps, world, rank, local, cpu):
     clocks = sampler.stop()
     status = int(buf.status.item())
 
-    vals = [ms, e2e_ms, kernel_ms] + ([fwd_ms, bwd_ms] if w.backward else [])
+    vals = [ms, e2e_ms, kernel_ms] + ([fwd_ms, bwd_ms] if w.backward else [gather_ms])
     vals = max_over_ranks(vals, "cuda")
     ms, e2e_ms, kernel_ms = vals[:3]
     if w.backward:
         fwd_ms, bwd_ms = vals[3:]
+    else:
+        gather_ms = vals[3]
     if rank != 0:
         return None
 
@@ -451,6 +490,10 @@ def measure(w, args, steps, world, rank, local, cpu):
     if w.backward:
         line["fwd_ms"] = fwd_ms
         line["bwd_ms"] = bwd_ms
+    else:
+        line["gather_mode"] = {"ms_per_step": gather_ms, "value": world * w.T / (gather_ms * 1e-3),
+                               "unit": "tokens/s", "tflops": fwd_flops / (gather_ms * 1e-3) / 1e12,
+                               "step": "moe_route -> awq_grouped_gate_up_swiglu_gather -> down -> combine"}
     if cpu:
         line["cpu_baseline"] = cpu_baseline(inp, w)
     del dev, buf, flush, graph
@@ -490,16 +533,19 @@ def gate_up_kernel_name(B, w):
 
 def launches_per_step_of(B, w):
     """Kernel launches of one step: route (2, or 3 past one token chunk), each
-    projection (1, or 2 with the split-K reduce), combine, and the backward's six."""
+    projection (1, or 2 with the split-K reduce; a tcgen05 projection with F16
+    scales adds the one-time F16 copy of its BF16 input), combine, and the
+    backward's six (plus the F16 copies of the three input-VJP gradients)."""
     n = 2 if w.T <= 64 else 3
+    conv = _path_of(w) >= 2 and w.scale_dtype == "f16"
     if _path_of(w) == 1:
         n += 1 + (B.projection_workspace_size(w.A, w.H, w.I, w.E, w.group, 2) > 0)
         n += 1 + (B.projection_workspace_size(w.A, w.I, w.H, w.E, w.group, 1) > 0)
     else:
-        n += 2
+        n += 2 + (2 if conv else 0)
     n += 1
     if w.backward:
-        n += 6
+        n += 6 + (3 if conv else 0)
     return n
 
 

@@ -261,11 +261,22 @@ MOE_API moe_status awq_grouped_gate_up_swiglu_gather(
     void *h, void *gate_out, void *up_out, void *workspace, size_t workspace_bytes,
     int32_t *device_status, void *stream);
 
-/* Workspace bytes the projection of A rows (input width K, output width N,
- * E experts, AWQ group size; nproj = 2 for the gate/up pair, 1 for a single
- * projection) needs under the current projection path; 0 if none. */
+/* Workspace bytes for the projection of A rows (input width K, output width
+ * N, E experts, AWQ group size; nproj = 2 for the gate/up pair, 1 for a
+ * single projection) under the current projection path; 0 if none:
+ *  - the warp-level tiles that stream the packed words: their split-K
+ *    partial sums (required: a smaller workspace is MOE_ERR_WORKSPACE);
+ *  - a tcgen05 tile with F16 scales and BF16 activations: an F16 copy of
+ *    the activations (A x K), made once so that the tile's column blocks do
+ *    not each convert the same rows again (optional: with less workspace
+ *    the tile converts in place, same results, slower).
+ * awq_projection_workspace_size assumes the conversion may be needed;
+ * awq_projection_workspace_size_dt gives the bytes for the actual dtypes. */
 MOE_API size_t awq_projection_workspace_size(int64_t A, int64_t K, int64_t N, int64_t E,
                                              int64_t group_size, int32_t nproj);
+MOE_API size_t awq_projection_workspace_size_dt(int64_t A, int64_t K, int64_t N, int64_t E,
+                                                int64_t group_size, int32_t nproj, moe_dtype act_dtype,
+                                                moe_dtype scale_dtype);
 
 /* ------------------------------------------------------------------------
  * awq_grouped_down -- the down projection of [PE] packed_swiglu_forward; also
@@ -363,6 +374,10 @@ MOE_API moe_status moe_combine_backward(const void *d_out, const void *y, moe_dt
  * Tile paths as for the forward projections (warp-level, 128-row tcgen05,
  * 256-row CTA-pair tcgen05); the tensor-core products run in the scale
  * dtype, gradients converted to it when they differ.
+ *  workspace  device scratch of awq_input_backward_workspace_size(...) bytes
+ *             (16-byte aligned), or NULL: F16 copies of the gradients for a
+ *             tcgen05 tile with F16 scales and BF16 gradients, made once
+ *             (optional: with less the tile converts in place, same results).
  * Device errors: MOE_DEVICE_ERR_OFFSETS, MOE_DEVICE_ERR_ACT_RANGE (F16 scales
  * with BF16 inputs), MOE_DEVICE_ERR_TIMEOUT.
  * ---------------------------------------------------------------------- */
@@ -371,8 +386,14 @@ MOE_API moe_status awq_input_backward(const void *grad, moe_dtype grad_dtype, in
                               const int32_t *qweight, const int32_t *qzeros, const void *scales,
                               moe_dtype scale_dtype, int64_t group_size, const void *grad2,
                               const int32_t *qweight2, const int32_t *qzeros2,
-                              const void *scales2, void *dinput, int32_t *device_status,
-                              void *stream);
+                              const void *scales2, void *dinput, void *workspace,
+                              size_t workspace_bytes, int32_t *device_status, void *stream);
+
+/* Workspace bytes of awq_input_backward for A gradient rows of width N
+ * (nproj = 2 with grad2), output width K, under the current path; 0 if none. */
+MOE_API size_t awq_input_backward_workspace_size(int64_t A, int64_t N, int64_t K, int64_t E,
+                                                 int64_t group_size, int32_t nproj, moe_dtype grad_dtype,
+                                                 moe_dtype scale_dtype);
 
 /* ------------------------------------------------------------------------
  * moe_swiglu_backward -- the SwiGLU step of [PE] packed_swiglu_input_backward,

@@ -50,11 +50,14 @@ _SIGS = {
     "awq_grouped_gate_up_swiglu_gather": (C.c_int, [P, C.c_int, I64, P, I64, I64, I64, P, I64, P, P, P, P, P, P, P,
                                                     P, C.c_int, C.c_int, I64, P, P, P, P, SZ, P, P]),
     "awq_projection_workspace_size": (SZ, [I64, I64, I64, I64, I64, I32]),
+    "awq_projection_workspace_size_dt": (SZ, [I64, I64, I64, I64, I64, I32, C.c_int, C.c_int]),
+    "awq_input_backward_workspace_size": (SZ, [I64, I64, I64, I64, I64, I32, C.c_int, C.c_int]),
     "awq_grouped_down": (C.c_int, [P, C.c_int, I64, I64, I64, P, I64, P, P, P, P, C.c_int, C.c_int, I64, P, P, SZ, P,
                                    P]),
     "moe_combine": (C.c_int, [P, C.c_int, I64, P, P, P, I64, I64, I32, P, P, P]),
     "moe_combine_backward": (C.c_int, [P, P, C.c_int, I64, P, P, I64, I64, I32, P, P, P, P]),
-    "awq_input_backward": (C.c_int, [P, C.c_int, I64, I64, I64, P, I64, P, P, P, C.c_int, I64, P, P, P, P, P, P, P]),
+    "awq_input_backward": (C.c_int, [P, C.c_int, I64, I64, I64, P, I64, P, P, P, C.c_int, I64, P, P, P, P, P, P, SZ,
+                                     P, P]),
     "moe_swiglu_backward": (C.c_int, [P, P, P, C.c_int, I64, I64, P, P, P]),
     "moe_dispatch_backward": (C.c_int, [P, C.c_int, I64, P, P, I64, I64, I32, P, P, P]),
     "moe_router_backward": (C.c_int, [P, P, P, I64, I64, I32, I32, I32, P, P, P]),
@@ -203,8 +206,16 @@ def _bias_dt(*biases):
     return MOE_F32
 
 
-def projection_workspace_size(A, K, N, E, group, nproj):
-    return int(lib().awq_projection_workspace_size(A, K, N, E, group, nproj))
+def projection_workspace_size(A, K, N, E, group, nproj, act_dtype=None, scale_dtype=None):
+    """Workspace bytes of a projection; with the dtypes (torch dtypes), the
+    bytes for exactly those (else enough for any)."""
+    if act_dtype is None or scale_dtype is None:
+        return int(lib().awq_projection_workspace_size(A, K, N, E, group, nproj))
+    return int(lib().awq_projection_workspace_size_dt(A, K, N, E, group, nproj, _dt(act_dtype), _dt(scale_dtype)))
+
+
+def input_backward_workspace_size(A, N, K, E, group, nproj, grad_dtype, scale_dtype):
+    return int(lib().awq_input_backward_workspace_size(A, N, K, E, group, nproj, _dt(grad_dtype), _dt(scale_dtype)))
 
 
 def _workspace(nbytes, device, workspace=None):
@@ -224,7 +235,8 @@ def awq_grouped_gate_up_swiglu(values, offsets, gate, up, group, want_gu=False, 
     h = out if out is not None else torch.empty((A, I), dtype=values.dtype, device=values.device)
     G = torch.empty_like(h) if want_gu else None
     U = torch.empty_like(h) if want_gu else None
-    ws = _workspace(projection_workspace_size(A, H, I, E, group, 2), values.device, workspace)
+    ws = _workspace(projection_workspace_size(A, H, I, E, group, 2, values.dtype, gate["scales"].dtype), values.device,
+                    workspace)
     st = lib().awq_grouped_gate_up_swiglu(
         _ptr(values), _dt(values.dtype), A, H, I, _ptr(offsets), E,
         _ptr(gate["qweight"]), _ptr(gate["qzeros"]), _ptr(gate["scales"]), _ptr(gate.get("bias")),
@@ -246,7 +258,7 @@ def awq_grouped_gate_up_swiglu_gather(x, src_token, offsets, gate, up, group, wa
     h = out if out is not None else torch.empty((A, I), dtype=x.dtype, device=x.device)
     G = torch.empty_like(h) if want_gu else None
     U = torch.empty_like(h) if want_gu else None
-    ws = _workspace(projection_workspace_size(A, H, I, E, group, 2), x.device, workspace)
+    ws = _workspace(projection_workspace_size(A, H, I, E, group, 2, x.dtype, gate["scales"].dtype), x.device, workspace)
     st = lib().awq_grouped_gate_up_swiglu_gather(
         _ptr(x), _dt(x.dtype), T, _ptr(src_token), A, H, I, _ptr(offsets), E,
         _ptr(gate["qweight"]), _ptr(gate["qzeros"]), _ptr(gate["scales"]), _ptr(gate.get("bias")),
@@ -262,7 +274,8 @@ def awq_grouped_down(inp, offsets, proj, group, device_status=None, out=None, wo
     E = offsets.numel() - 1
     N = proj["qweight"].shape[2] * 8
     y = out if out is not None else torch.empty((A, N), dtype=inp.dtype, device=inp.device)
-    ws = _workspace(projection_workspace_size(A, K, N, E, group, 1), inp.device, workspace)
+    ws = _workspace(projection_workspace_size(A, K, N, E, group, 1, inp.dtype, proj["scales"].dtype), inp.device,
+                    workspace)
     st = lib().awq_grouped_down(
         _ptr(inp), _dt(inp.dtype), A, K, N, _ptr(offsets), E, _ptr(proj["qweight"]), _ptr(proj["qzeros"]),
         _ptr(proj["scales"]), _ptr(proj.get("bias")), _dt(proj["scales"].dtype), _bias_dt(proj.get("bias")), group,
@@ -292,16 +305,21 @@ def moe_combine_backward(d_out, y, weights, row_of, want_dy=True, want_dw=True, 
     return dy, dw
 
 
-def awq_input_backward(grad, offsets, proj, group, grad2=None, proj2=None, device_status=None, out=None):
+def awq_input_backward(grad, offsets, proj, group, grad2=None, proj2=None, device_status=None, out=None,
+                       workspace=None):
     A, N = grad.shape
     E = offsets.numel() - 1
     K = proj["qweight"].shape[1]
     d = out if out is not None else torch.empty((A, K), dtype=grad.dtype, device=grad.device)
     p2 = proj2 or {}
+    nbytes = input_backward_workspace_size(A, N, K, E, group, 2 if grad2 is not None else 1, grad.dtype,
+                                           proj["scales"].dtype)
+    ws = _workspace(nbytes, grad.device, workspace)
     st = lib().awq_input_backward(
         _ptr(grad), _dt(grad.dtype), A, N, K, _ptr(offsets), E, _ptr(proj["qweight"]), _ptr(proj["qzeros"]),
         _ptr(proj["scales"]), _dt(proj["scales"].dtype), group, _ptr(grad2), _ptr(p2.get("qweight")),
-        _ptr(p2.get("qzeros")), _ptr(p2.get("scales")), _ptr(d), _ptr(device_status), _stream())
+        _ptr(p2.get("qzeros")), _ptr(p2.get("scales")), _ptr(d), _ptr(ws), 0 if ws is None else ws.numel(),
+        _ptr(device_status), _stream())
     _check("awq_input_backward", st)
     return d
 

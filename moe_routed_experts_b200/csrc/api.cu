@@ -51,18 +51,40 @@ static int choose_path(int64_t A, int64_t E) {
   return (A >= 32 * E) ? 2 : 1;
 }
 
-// Launches the tcgen05 forward tile for the chosen path; returns false if
-// the shape is not one those tiles take.
-static bool try_fwd_tc(int path, const ProjParams &p, int nproj, bool bf, cudaStream_t st, moe_status *out) {
-  if (path == 3 && tc2_fits(p)) {
-    *out = launch_fwd_tc2(p, nproj, bf, st);
-    return true;
+// The tcgen05 forward tile the chosen path runs for this shape: 3 (CTA
+// pair), 2 (single CTA), or 0 when neither takes it.
+static int fwd_tc_kind(int path, const ProjParams &p) {
+  if (path == 3 && tc2_fits(p)) return 3;
+  if (path >= 2 && tc_fits(p)) return 2;
+  return 0;
+}
+
+// Bytes of an F16 copy of `rows` x `cols` BF16 values (16-byte multiple).
+static size_t conv_bytes(int64_t rows, int64_t cols) { return ((size_t)rows * cols * 2 + 255) & ~size_t(255); }
+
+// A tcgen05 tile with F16 coefficients and BF16 inputs: when the workspace
+// holds it, make the F16 copy of the inputs once (src -> ws) and return it,
+// else return NULL (the tile converts in place).
+static const uint16_t *maybe_convert(const void *src, moe_dtype in_dt, moe_dtype scale_dt, int64_t rows, int64_t cols,
+                                     void *ws, size_t ws_bytes, int32_t *status, cudaStream_t st, moe_status *err) {
+  *err = MOE_OK;
+  if (in_dt != MOE_BF16 || scale_dt != MOE_F16 || !ws || ws_bytes < conv_bytes(rows, cols) || !aligned16(ws))
+    return nullptr;
+  *err = launch_act_to_f16(src, ws, rows * cols, status, st);
+  return *err == MOE_OK ? static_cast<const uint16_t *>(ws) : nullptr;
+}
+
+static moe_status run_fwd_tc(int kind, ProjParams p, int nproj, bool bf, moe_dtype scale_dt, void *ws,
+                             size_t ws_bytes, cudaStream_t st) {
+  moe_status err;
+  const uint16_t *conv = maybe_convert(p.x, (moe_dtype)p.act_dt, scale_dt, p.gather ? p.T : p.A, p.K, ws, ws_bytes,
+                                       p.status, st, &err);
+  if (err != MOE_OK) return err;
+  if (conv) {
+    p.x = conv;
+    p.act_dt = MOE_F16;
   }
-  if (path >= 2 && tc_fits(p)) {
-    *out = launch_fwd_tc(p, nproj, bf, st);
-    return true;
-  }
-  return false;
+  return kind == 3 ? launch_fwd_tc2(p, nproj, bf, st) : launch_fwd_tc(p, nproj, bf, st);
 }
 
 // Token columns per warp-level tile: 16 when experts average >= 12 rows.
@@ -109,8 +131,8 @@ extern "C" int32_t moe_set_projection_path(int32_t path) {
   return g_path.exchange(path);
 }
 
-extern "C" size_t awq_projection_workspace_size(int64_t A, int64_t K, int64_t N, int64_t E, int64_t group_size,
-                                                int32_t nproj) {
+extern "C" size_t awq_projection_workspace_size_dt(int64_t A, int64_t K, int64_t N, int64_t E, int64_t group_size,
+                                                   int32_t nproj, moe_dtype act_dtype, moe_dtype scale_dtype) {
   if (A <= 0 || E < 1 || K < 16 || N < 8 || group_size < 16 || (nproj != 1 && nproj != 2)) return 0;
   ProjParams probe{};
   probe.A = A;
@@ -118,10 +140,22 @@ extern "C" size_t awq_projection_workspace_size(int64_t A, int64_t K, int64_t N,
   probe.N = N;
   probe.E = (int)E;
   probe.group = (int)group_size;
-  const int path = choose_path(A, E);
-  if ((path == 3 && tc2_fits(probe)) || (path >= 2 && tc_fits(probe))) return 0;
+  if (fwd_tc_kind(choose_path(A, E), probe))
+    return (act_dtype == MOE_BF16 && scale_dtype == MOE_F16) ? conv_bytes(A, K) : 0;
   const StreamPlan pl = stream_plan(A, K, N, E, group_size, nproj, small_tile_tokens(A, E));
   return pl.fits ? pl.bytes : 0;
+}
+
+extern "C" size_t awq_projection_workspace_size(int64_t A, int64_t K, int64_t N, int64_t E, int64_t group_size,
+                                                int32_t nproj) {
+  return awq_projection_workspace_size_dt(A, K, N, E, group_size, nproj, MOE_BF16, MOE_F16);
+}
+
+extern "C" size_t awq_input_backward_workspace_size(int64_t A, int64_t N, int64_t K, int64_t E, int64_t group_size,
+                                                    int32_t nproj, moe_dtype grad_dtype, moe_dtype scale_dtype) {
+  if (A <= 0 || E < 1 || K < 16 || N < 8 || group_size < 16 || (nproj != 1 && nproj != 2)) return 0;
+  if (grad_dtype != MOE_BF16 || scale_dtype != MOE_F16 || choose_path(A, E) < 2) return 0;
+  return (size_t)nproj * conv_bytes(A, N);
 }
 
 // Gate/up projections of expert-sorted rows that are read from `values`
@@ -168,8 +202,8 @@ static moe_status gate_up_impl(const char *fn, const void *x, const int32_t *gat
   p.status = device_status;
   cudaStream_t st = as_stream(stream);
   const bool bf = scale_dtype == MOE_BF16;
-  moe_status ts;
-  if (try_fwd_tc(choose_path(A, E), p, 2, bf, st, &ts)) return ts;
+  const int kind = fwd_tc_kind(choose_path(A, E), p);
+  if (kind) return run_fwd_tc(kind, p, 2, bf, scale_dtype, workspace, workspace_bytes, st);
   const int nt = small_tile_tokens(A, E);
   if (stream_plan(A, H, I, E, group_size, 2, nt).fits) return launch_fwd_stream(p, 2, bf, nt, workspace, workspace_bytes, st);
   launch_fwd_mma(p, 2, bf, nt, st);
@@ -232,8 +266,8 @@ extern "C" moe_status awq_grouped_down(const void *input, moe_dtype act_dtype, i
   p.status = device_status;
   cudaStream_t st = as_stream(stream);
   const bool bf = scale_dtype == MOE_BF16;
-  moe_status ts;
-  if (try_fwd_tc(choose_path(A, E), p, 1, bf, st, &ts)) return ts;
+  const int kind = fwd_tc_kind(choose_path(A, E), p);
+  if (kind) return run_fwd_tc(kind, p, 1, bf, scale_dtype, workspace, workspace_bytes, st);
   const int nt = small_tile_tokens(A, E);
   if (stream_plan(A, K, N, E, group_size, 1, nt).fits) return launch_fwd_stream(p, 1, bf, nt, workspace, workspace_bytes, st);
   launch_fwd_mma(p, 1, bf, nt, st);
@@ -245,7 +279,8 @@ extern "C" moe_status awq_input_backward(const void *grad, moe_dtype grad_dtype,
                                          const int32_t *qzeros, const void *scales, moe_dtype scale_dtype,
                                          int64_t group_size, const void *grad2, const int32_t *qweight2,
                                          const int32_t *qzeros2, const void *scales2, void *dinput,
-                                         int32_t *device_status, void *stream) {
+                                         void *workspace, size_t workspace_bytes, int32_t *device_status,
+                                         void *stream) {
   const char *fn = "awq_input_backward";
   moe_status s = check_payload_geom(fn, A, K, N, E, group_size, grad_dtype, scale_dtype);
   if (s != MOE_OK) return s;
@@ -278,8 +313,22 @@ extern "C" moe_status awq_input_backward(const void *grad, moe_dtype grad_dtype,
   const bool bf = scale_dtype == MOE_BF16;
   const int nproj = grad2 ? 2 : 1;
   const int path = choose_path(A, E);
-  if (path == 3 && tc2_bwd_fits(p)) return launch_bwd_tc2(p, nproj, bf, st);
-  if (path >= 2 && tc_bwd_fits(p)) return launch_bwd_tc(p, nproj, bf, st);
+  const int kind = (path == 3 && tc2_bwd_fits(p)) ? 3 : (path >= 2 && tc_bwd_fits(p)) ? 2 : 0;
+  if (kind) {
+    // F16 copies of the gradients, once, when the workspace holds both
+    const size_t one = conv_bytes(A, N);
+    if (grad_dtype == MOE_BF16 && scale_dtype == MOE_F16 && workspace && aligned16(workspace) &&
+        workspace_bytes >= (size_t)nproj * one) {
+      char *w = static_cast<char *>(workspace);
+      s = launch_act_to_f16(grad, w, A * N, device_status, st);
+      if (s == MOE_OK && grad2) s = launch_act_to_f16(grad2, w + one, A * N, device_status, st);
+      if (s != MOE_OK) return s;
+      p.grad[0] = reinterpret_cast<const uint16_t *>(w);
+      p.grad[1] = reinterpret_cast<const uint16_t *>(grad2 ? w + one : w);
+      p.gdt = MOE_F16;
+    }
+    return kind == 3 ? launch_bwd_tc2(p, nproj, bf, st) : launch_bwd_tc(p, nproj, bf, st);
+  }
   launch_bwd_mma(p, nproj, bf, A >= 12 * E ? 2 : 1, st);
   return check_launch(fn);
 }

@@ -114,8 +114,10 @@ __global__ void __launch_bounds__(128) awq_fwd_mma_kernel(ProjParams p) {
           uint32_t b0[NT], b1[NT];
 #pragma unroll
           for (int nt = 0; nt < NT; ++nt) {
-            b0[nt] = act_pair_to_mt<MT>(xbuf[d][nt].x, p.act_dt, act_bad);
-            b1[nt] = act_pair_to_mt<MT>(xbuf[d][nt].y, p.act_dt, act_bad);
+            uint32_t bb[2] = {xbuf[d][nt].x, xbuf[d][nt].y};
+            act_pairs_to_mt<MT, 2>(bb, p.act_dt, act_bad);
+            b0[nt] = bb[0];
+            b1[nt] = bb[1];
           }
 #pragma unroll
           for (int j = 0; j < NPROJ; ++j) {
@@ -276,8 +278,10 @@ __global__ void __launch_bounds__(128) awq_bwd_mma_kernel(BwdParams p) {
         uint32_t b0[NT], b1[NT];
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
-          b0[nt] = act_pair_to_mt<MT>(q == 0 ? gv[nt].x : gv[nt].z, p.gdt, act_bad);
-          b1[nt] = act_pair_to_mt<MT>(q == 0 ? gv[nt].y : gv[nt].w, p.gdt, act_bad);
+          uint32_t bb[2] = {q == 0 ? gv[nt].x : gv[nt].z, q == 0 ? gv[nt].y : gv[nt].w};
+          act_pairs_to_mt<MT, 2>(bb, p.gdt, act_bad);
+          b0[nt] = bb[0];
+          b1[nt] = bb[1];
         }
 #pragma unroll
         for (int mt = 0; mt < 4; ++mt) {

@@ -278,11 +278,12 @@ __global__ void __launch_bounds__(stream::kThreads, 2)
         const int tok = (int)(q / (Kq / 8));
         const int64_t hb = q % (Kq / 8), blk = hb >> 1, h = hb & 1;
         const uint4 v = *reinterpret_cast<const uint4 *>(src + (tok * Kq + blk * 16 + h * 8) * 2);
-        const uint32_t pr[4] = {prmt(v.x, v.z, 0x5410u), prmt(v.x, v.z, 0x7632u), prmt(v.y, v.w, 0x5410u),
-                                prmt(v.y, v.w, 0x7632u)};  // (row i, row i+4) of the half
+        uint32_t pr[4] = {prmt(v.x, v.z, 0x5410u), prmt(v.x, v.z, 0x7632u), prmt(v.y, v.w, 0x5410u),
+                          prmt(v.y, v.w, 0x7632u)};  // (row i, row i+4) of the half
+        act_pairs_to_mt<MT, 4>(pr, p.act_dt, act_bad);
         uint8_t *dst = xs + tok * xs_pitch + (blk * 16 + 2 * h) * 2;
 #pragma unroll
-        for (int i = 0; i < 4; ++i) *reinterpret_cast<uint32_t *>(dst + 8 * i) = act_pair_to_mt<MT>(pr[i], p.act_dt, act_bad);
+        for (int i = 0; i < 4; ++i) *reinterpret_cast<uint32_t *>(dst + 8 * i) = pr[i];
       }
     }
     __syncwarp();

@@ -248,16 +248,27 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
     const bool convert = p.act_dt != (std::is_same<MT, __half>::value ? MOE_F16 : MOE_BF16);
     uint32_t it = 0;
     bool live = true;
+    // zeros/scales of a tile's word column; the first group of the next tile
+    // is requested during the last group of the current one
+    struct ZsPtr {
+      const int32_t *qz;
+      const uint16_t *sc;
+      bool ok;
+    };
+    auto zs_ptr = [&](int64_t tile) {
+      const TileInfo tn = tile_info(tile);
+      const int64_t wc = NPROJ == 2 ? (int64_t)tn.nt * 16 + (col & 15) : (int64_t)tn.nt * 32 + col;
+      const bool ok = wc < NW;
+      const int64_t wcs = ok ? wc : 0;
+      return ZsPtr{qz + (int64_t)tn.e * ngroups * NW + wcs, sc + (int64_t)tn.e * ngroups * p.N + 8 * wcs, ok};
+    };
+    ZsPtr cur = zs_ptr((int64_t)blockIdx.x < total ? (int64_t)blockIdx.x : 0);
+    uint32_t pf_zw = ((int64_t)blockIdx.x < total && cur.ok) ? (uint32_t)__ldg(cur.qz) : 0u;
+    uint4 pf_sv = ((int64_t)blockIdx.x < total && cur.ok) ? __ldg(reinterpret_cast<const uint4 *>(cur.sc))
+                                                           : make_uint4(0, 0, 0, 0);
     for (int64_t tile = blockIdx.x; tile < total && live; tile += gridDim.x) {
-      const TileInfo ti = tile_info(tile);
-      const int64_t wc = NPROJ == 2 ? (int64_t)ti.nt * 16 + (col & 15) : (int64_t)ti.nt * 32 + col;
-      const bool wc_ok = wc < NW;
-      const int64_t wcs = wc_ok ? wc : 0;
-      const int32_t *qzp = qz + (int64_t)ti.e * ngroups * NW + wcs;
-      const uint16_t *scp = sc + (int64_t)ti.e * ngroups * p.N + 8 * wcs;
+      const ZsPtr zs = cur;
       uint32_t zp[4], sp[4];
-      uint32_t pf_zw = wc_ok ? (uint32_t)__ldg(qzp) : 0u;
-      uint4 pf_sv = wc_ok ? __ldg(reinterpret_cast<const uint4 *>(scp)) : make_uint4(0, 0, 0, 0);
       int64_t grp = 0;
       int gstage = 0;
       for (int kb = 0; kb < nk; ++kb, ++it) {
@@ -270,9 +281,15 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
             zp[q] = nib_pair<M>(pf_zw >> (4 * q));
             sp[q] = s4[q];
           }
-          if (wc_ok && grp + 1 < ngroups) {
-            pf_zw = (uint32_t)__ldg(qzp + (grp + 1) * NW);
-            pf_sv = __ldg(reinterpret_cast<const uint4 *>(scp + (grp + 1) * p.N));
+          if (grp + 1 < ngroups) {
+            if (zs.ok) {
+              pf_zw = (uint32_t)__ldg(zs.qz + (grp + 1) * NW);
+              pf_sv = __ldg(reinterpret_cast<const uint4 *>(zs.sc + (grp + 1) * p.N));
+            }
+          } else if (tile + gridDim.x < total) {
+            cur = zs_ptr(tile + gridDim.x);
+            pf_zw = cur.ok ? (uint32_t)__ldg(cur.qz) : 0u;
+            pf_sv = cur.ok ? __ldg(reinterpret_cast<const uint4 *>(cur.sc)) : make_uint4(0, 0, 0, 0);
           }
         }
         if (++gstage == spg) {
@@ -290,10 +307,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
 #pragma unroll
           for (int i = 0; i < kABytes / 16 / 256; ++i) {
             uint4 v = a4[td + 256 * i];
-            v.x = act_pair_to_mt<MT>(v.x, p.act_dt, act_bad);
-            v.y = act_pair_to_mt<MT>(v.y, p.act_dt, act_bad);
-            v.z = act_pair_to_mt<MT>(v.z, p.act_dt, act_bad);
-            v.w = act_pair_to_mt<MT>(v.w, p.act_dt, act_bad);
+            act_quad_to_mt<MT>(v, p.act_dt, act_bad);
             a4[td + 256 * i] = v;
           }
           fence_proxy_async_smem();  // the converted tile is read by the tensor core

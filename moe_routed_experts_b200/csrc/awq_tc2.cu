@@ -255,16 +255,30 @@ __global__ void __launch_bounds__(tc2::kThreads, 1)
     uint64_t *bready0 = bready;  // CTA 0's barriers, addressed through the cluster window
     uint32_t it = 0;
     bool live = true;
+    // zeros/scales of a tile's word column; the first group of the next tile
+    // is requested during the last group of the current one
+    struct ZsPtr {
+      const int32_t *qz;
+      const uint16_t *sc;
+      bool ok;
+    };
+    auto zs_ptr = [&](int64_t tile) {
+      const PairTile tn = tile_info(tile);
+      const int64_t wc = NPROJ == 2 ? (int64_t)tn.nt * 16 + col : (int64_t)tn.nt * 32 + 16 * rank + col;
+      const bool ok = wc < NW;
+      const int64_t wcs = ok ? wc : 0;
+      return ZsPtr{qz + (int64_t)tn.e * ngroups * NW + wcs, sc + (int64_t)tn.e * ngroups * p.N + 8 * wcs, ok};
+    };
+    uint32_t pf_zw = 0u;
+    uint4 pf_sv = make_uint4(0, 0, 0, 0);
+    ZsPtr cur = zs_ptr(pair < total ? pair : 0);
+    if (pair < total && cur.ok) {
+      pf_zw = (uint32_t)__ldg(cur.qz);
+      pf_sv = __ldg(reinterpret_cast<const uint4 *>(cur.sc));
+    }
     for (int64_t tile = pair; tile < total && live; tile += npairs) {
-      const PairTile ti = tile_info(tile);
-      const int64_t wc = NPROJ == 2 ? (int64_t)ti.nt * 16 + col : (int64_t)ti.nt * 32 + 16 * rank + col;
-      const bool wc_ok = wc < NW;
-      const int64_t wcs = wc_ok ? wc : 0;
-      const int32_t *qzp = qz + (int64_t)ti.e * ngroups * NW + wcs;
-      const uint16_t *scp = sc + (int64_t)ti.e * ngroups * p.N + 8 * wcs;
+      const ZsPtr zs = cur;
       uint32_t zp[4], sp[4];
-      uint32_t pf_zw = wc_ok ? (uint32_t)__ldg(qzp) : 0u;
-      uint4 pf_sv = wc_ok ? __ldg(reinterpret_cast<const uint4 *>(scp)) : make_uint4(0, 0, 0, 0);
       int64_t grp = 0;
       int gstage = 0;
       for (int kb = 0; kb < nk; ++kb, ++it) {
@@ -276,9 +290,15 @@ __global__ void __launch_bounds__(tc2::kThreads, 1)
             zp[q] = nib_pair<M>(pf_zw >> (4 * q));
             sp[q] = s4[q];
           }
-          if (wc_ok && grp + 1 < ngroups) {
-            pf_zw = (uint32_t)__ldg(qzp + (grp + 1) * NW);
-            pf_sv = __ldg(reinterpret_cast<const uint4 *>(scp + (grp + 1) * p.N));
+          if (grp + 1 < ngroups) {
+            if (zs.ok) {
+              pf_zw = (uint32_t)__ldg(zs.qz + (grp + 1) * NW);
+              pf_sv = __ldg(reinterpret_cast<const uint4 *>(zs.sc + (grp + 1) * p.N));
+            }
+          } else if (tile + npairs < total) {
+            cur = zs_ptr(tile + npairs);
+            pf_zw = cur.ok ? (uint32_t)__ldg(cur.qz) : 0u;
+            pf_sv = cur.ok ? __ldg(reinterpret_cast<const uint4 *>(cur.sc)) : make_uint4(0, 0, 0, 0);
           }
         }
         if (++gstage == spg) {
@@ -301,10 +321,7 @@ __global__ void __launch_bounds__(tc2::kThreads, 1)
 #pragma unroll
           for (int i = 0; i < kABytes / 16 / (32 * kDqWarps); ++i) {
             uint4 v = a4[td + 32 * kDqWarps * i];
-            v.x = act_pair_to_mt<MT>(v.x, p.act_dt, act_bad);
-            v.y = act_pair_to_mt<MT>(v.y, p.act_dt, act_bad);
-            v.z = act_pair_to_mt<MT>(v.z, p.act_dt, act_bad);
-            v.w = act_pair_to_mt<MT>(v.w, p.act_dt, act_bad);
+            act_quad_to_mt<MT>(v, p.act_dt, act_bad);
             a4[td + 32 * kDqWarps * i] = v;
           }
           fence_proxy_async_smem();

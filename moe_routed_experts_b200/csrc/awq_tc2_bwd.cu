@@ -250,10 +250,7 @@ __global__ void __launch_bounds__(tc2b::kThreads, 1)
 #pragma unroll
           for (int i = 0; i < kABytes / 16 / (32 * kDqWarps); ++i) {
             uint4 v = a4[td + 32 * kDqWarps * i];
-            v.x = act_pair_to_mt<MT>(v.x, p.gdt, act_bad);
-            v.y = act_pair_to_mt<MT>(v.y, p.gdt, act_bad);
-            v.z = act_pair_to_mt<MT>(v.z, p.gdt, act_bad);
-            v.w = act_pair_to_mt<MT>(v.w, p.gdt, act_bad);
+            act_quad_to_mt<MT>(v, p.gdt, act_bad);
             a4[td + 32 * kDqWarps * i] = v;
           }
           fence_proxy_async_smem();

@@ -162,6 +162,54 @@ __device__ __forceinline__ uint32_t act_pair_to_mt(uint32_t v, int act_dt, uint3
   }
 }
 
+// Lane-wise maximum of two 16-bit pairs.
+__device__ __forceinline__ uint32_t umax16x2(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("max.u16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+
+// Lane-wise minimum of two 16-bit pairs.
+__device__ __forceinline__ uint32_t umin16x2(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("min.u16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+
+// N activation pairs at once, with the range report of act_pair_to_mt at a
+// fraction of its cost: the pairs are tested one by one only when some
+// source magnitude is at least 65536 (BF16 0x4780, the first value F16
+// cannot hold; +-inf and NaN lie above it).  v << 1 doubles each 16-bit
+// lane's magnitude (the low lane's sign moves into bit 0 of the high lane,
+// which cannot carry it across the even threshold 0x8F00).
+template <typename MT, int N>
+__device__ __forceinline__ void act_pairs_to_mt(uint32_t (&v)[N], int act_dt, uint32_t &bad) {
+  if constexpr (std::is_same<MT, __half>::value) {
+    if (act_dt != MOE_BF16) return;
+    uint32_t m = v[0] << 1;
+#pragma unroll
+    for (int i = 1; i < N; ++i) m = umax16x2(m, v[i] << 1);
+    if ((umax16x2(m, m >> 16) & 0xFFFFu) >= 0x8F00u) {  // the larger lane
+#pragma unroll
+      for (int i = 0; i < N; ++i) v[i] = act_pair_to_mt<MT>(v[i], act_dt, bad);
+      return;
+    }
+#pragma unroll
+    for (int i = 0; i < N; ++i) v[i] = bf16x2_to_f16x2(v[i]);
+  } else {
+    if (act_dt != MOE_F16) return;
+#pragma unroll
+    for (int i = 0; i < N; ++i) v[i] = f16x2_to_bf16x2(v[i]);
+  }
+}
+
+template <typename MT>
+__device__ __forceinline__ void act_quad_to_mt(uint4 &q, int act_dt, uint32_t &bad) {
+  uint32_t v[4] = {q.x, q.y, q.z, q.w};
+  act_pairs_to_mt<MT, 4>(v, act_dt, bad);
+  q = make_uint4(v[0], v[1], v[2], v[3]);
+}
+
 // mma.sync m16n8k16, FP32 accumulate.
 template <typename MT>
 __device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {

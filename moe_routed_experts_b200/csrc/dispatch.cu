@@ -26,9 +26,11 @@ namespace moe {
 
 constexpr int kRouteThreads = 512;
 constexpr int kScanThreads = 1024;
-constexpr int kMaxChunks = 64;
+constexpr int kMaxChunks = 1024;
 
-// Tokens per chunk: a multiple of 64 keeping the chunk count <= kMaxChunks.
+// Tokens per chunk: 64 (the ranks come from one 64-bit token mask per
+// expert), or a larger power of two keeping the chunk count <= kMaxChunks
+// (ranked by one warp in token order).
 static int64_t route_chunk(int64_t T) {
   int64_t c = 64;
   while ((T + c - 1) / c > kMaxChunks) c *= 2;
@@ -87,15 +89,20 @@ struct RouteParams {
 template <int R>
 __global__ void __launch_bounds__(1024) route_rank_kernel(RouteParams p) {
   pdl_enter();  // programmatic dependent launch: the previous kernel is done
-  extern __shared__ int32_t sm[];
-  int32_t *cnt = sm;                      // [E]
+  extern __shared__ __align__(16) int32_t sm[];
+  unsigned long long *mask = reinterpret_cast<unsigned long long *>(sm);  // [E] (64-token chunks)
+  int32_t *cnt = reinterpret_cast<int32_t *>(mask + p.E);  // [E]
   int32_t *tmp = cnt + p.E;               // [32]
   int16_t *sel_s = reinterpret_cast<int16_t *>(tmp + 32);  // [chunk * k]
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
   const int64_t t0 = (int64_t)blockIdx.x * p.chunk;
   const int64_t t1 = min(p.T, t0 + p.chunk);
   const int E = p.E, k = p.k;
-  for (int i = threadIdx.x; i < E; i += blockDim.x) cnt[i] = 0;
+  for (int i = threadIdx.x; i < E; i += blockDim.x) {
+    cnt[i] = 0;
+    mask[i] = 0ull;
+  }
+  __syncthreads();
 
   for (int64_t t = t0 + warp; t < t1; t += nwarps) {
     const float *l = p.logits + t * E;
@@ -175,11 +182,22 @@ __global__ void __launch_bounds__(1024) route_rank_kernel(RouteParams p) {
       p.weights[t * k + lane] = expf(lj - m) / den;
       p.selected[t * k + lane] = p.expert_start + (uint32_t)my_e;
       sel_s[(t - t0) * k + lane] = (int16_t)my_e;
+      // a token picks an expert at most once: bit (t - t0) of the expert's mask
+      if (p.chunk == 64) atomicOr(&mask[my_e], 1ull << (t - t0));
     }
   }
   __syncthreads();
 
-  if (warp == 0) {
+  if (p.chunk == 64) {
+    // rank of (t, j) among the chunk's rows of its expert = selecting tokens
+    // before t (order-independent: the masks are complete)
+    const int n = (int)(t1 - t0);
+    for (int a = threadIdx.x; a < n * k; a += blockDim.x) {
+      const int lt = a / k, e = sel_s[a];
+      p.rank[(t0 + lt) * k + (a % k)] = __popcll(mask[e] & ((1ull << lt) - 1ull));
+    }
+    for (int i = threadIdx.x; i < E; i += blockDim.x) cnt[i] = __popcll(mask[i]);
+  } else if (warp == 0) {
     const int tpi = 32 / k;  // tokens per warp iteration
     const int n = (int)(t1 - t0);
     for (int tt = 0; tt < n; tt += tpi) {
@@ -505,7 +523,8 @@ static moe_status route_impl(const char *fn, const void *x, moe_dtype x_dtype, i
   rp.hist = hist;
   rp.offsets = offsets;
   rp.single = lay.nchunks == 1;
-  size_t smem = sizeof(int32_t) * (size_t)(E + 32) + sizeof(int16_t) * (size_t)(lay.chunk * top_k);
+  size_t smem = sizeof(unsigned long long) * (size_t)E + sizeof(int32_t) * (size_t)(E + 32) +
+                sizeof(int16_t) * (size_t)(lay.chunk * top_k);
   smem = (smem + 15) & ~size_t(15);
   const int R = E <= 32 ? 1 : E <= 64 ? 2 : E <= 128 ? 4 : E <= 256 ? 8 : E <= 512 ? 16 : 0;
   auto kern = R == 1 ? route_rank_kernel<1> : R == 2 ? route_rank_kernel<2> : R == 4 ? route_rank_kernel<4>

@@ -128,9 +128,11 @@ __global__ void __launch_bounds__(128) nf4_fwd_kernel(Nf4Params p) {
       // activations: the MMA's K index 2t, 2t + 1, 2t + 8, 2t + 9 of this step
       uint32_t b0 = 0, b1 = 0;
       if (xok) {
-        b0 = act_pair_to_mt<MT>(__ldg(reinterpret_cast<const uint32_t *>(xrow + 16 * s + 2 * t)), p.act_dt, act_bad);
-        b1 = act_pair_to_mt<MT>(__ldg(reinterpret_cast<const uint32_t *>(xrow + 16 * s + 2 * t + 8)), p.act_dt,
-                                act_bad);
+        uint32_t bb[2] = {__ldg(reinterpret_cast<const uint32_t *>(xrow + 16 * s + 2 * t)),
+                          __ldg(reinterpret_cast<const uint32_t *>(xrow + 16 * s + 2 * t + 8))};
+        act_pairs_to_mt<MT, 2>(bb, p.act_dt, act_bad);
+        b0 = bb[0];
+        b1 = bb[1];
       }
 #pragma unroll
       for (int mt = 0; mt < 4; ++mt) {
@@ -229,8 +231,11 @@ __global__ void __launch_bounds__(128) nf4_bwd_kernel(Nf4Params p) {
         uint32_t b0 = 0, b1 = 0;
         if (gok) {
           const int64_t nn = 32 * s + 16 * h + 2 * t;
-          b0 = act_pair_to_mt<MT>(__ldg(reinterpret_cast<const uint32_t *>(grow + nn)), p.act_dt, act_bad);
-          b1 = act_pair_to_mt<MT>(__ldg(reinterpret_cast<const uint32_t *>(grow + nn + 8)), p.act_dt, act_bad);
+          uint32_t bb[2] = {__ldg(reinterpret_cast<const uint32_t *>(grow + nn)),
+                            __ldg(reinterpret_cast<const uint32_t *>(grow + nn + 8))};
+          act_pairs_to_mt<MT, 2>(bb, p.act_dt, act_bad);
+          b0 = bb[0];
+          b1 = bb[1];
         }
 #pragma unroll
         for (int mt = 0; mt < 4; ++mt) {

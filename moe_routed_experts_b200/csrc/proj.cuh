@@ -181,5 +181,6 @@ bool tc2_fits(const ProjParams &p);
 bool tc2_bwd_fits(const BwdParams &p);
 moe_status launch_bwd_tc2(const BwdParams &p, int nproj, bool bf16_mma, cudaStream_t st);
 moe_status launch_fwd_tc2(const ProjParams &p, int nproj, bool bf16_mma, cudaStream_t st);
+moe_status launch_act_to_f16(const void *src, void *dst, int64_t elems, int32_t *status, cudaStream_t st);
 
 }  // namespace moe

@@ -78,7 +78,9 @@ def alloc(w, device="cuda", keep_gu: bool = False) -> Buffers:
     U = torch.empty_like(h) if keep_gu else None
     y = torch.empty((A, H), dtype=torch.bfloat16, device=device)
     out = torch.empty((T, H), dtype=torch.bfloat16, device=device)
-    pws = max(B.projection_workspace_size(A, H, I, E, w.group, 2), B.projection_workspace_size(A, I, H, E, w.group, 1))
+    sdt = {"f16": torch.float16, "bf16": torch.bfloat16, "f32": torch.float32}[w.scale_dtype]
+    pws = max(B.projection_workspace_size(A, H, I, E, w.group, 2, torch.bfloat16, sdt),
+              B.projection_workspace_size(A, I, H, E, w.group, 1, torch.bfloat16, sdt))
     proj_ws = torch.empty(pws, dtype=torch.uint8, device=device) if pws else None
     return Buffers(route, ws, h, G, U, y, out, torch.zeros(1, dtype=torch.int32, device=device), proj_ws)
 

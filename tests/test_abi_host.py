@@ -88,7 +88,7 @@ def test_projection_rejects_bad_geometry_and_dtypes(L):
     assert L.awq_grouped_down(FAKE, B.MOE_BF16, 4, 64, 12, FAKE, 1, FAKE, FAKE, FAKE, None, B.MOE_F16, B.MOE_F32, 16,
                               FAKE, None, 0, None, None) == 1
     assert L.awq_input_backward(FAKE, B.MOE_BF16, 4, 16, 64, FAKE, 1, FAKE, FAKE, FAKE, B.MOE_BF16, 48, None, None,
-                                None, None, FAKE, None, None) == 1
+                                None, None, FAKE, None, 0, None, None) == 1
 
 
 def test_combine_family_rejects_bad_arguments(L):

@@ -270,6 +270,8 @@ __global__ void __launch_bounds__(stream::kThreads, 2)
     // After an abort every consumer warp still runs the loop (the named
     // barriers stay matched) but waits for, computes and arrives on nothing.
     const uint32_t xb = xi & 1;
+    // every consumer is done reading the previous unit's converted tile
+    named_barrier(1, kCW * 32);
     const bool xok = tc_wait(&xfull[xb], (xi >> 1) & 1, p.status, abort);
     if (xok) {
       const uint8_t *src = xraw + xb * xraw_bytes;
@@ -322,7 +324,9 @@ __global__ void __launch_bounds__(stream::kThreads, 2)
             const uint32_t lo = w4[i] & 0x7FFFu, hi = (w4[i] >> 16) & 0x7FFFu;
             bad |= (lo > 0x5C00u) | (hi > 0x5C00u) | (lo != 0u && lo < 0x0400u) | (hi != 0u && hi < 0x0400u);
           }
-          x16 = bad == 0;
+          // one decision per warp: the MMAs below are warp-wide (mma.sync), so
+          // every lane must take the same branch; a lane without a column votes yes
+          x16 = __all_sync(0xffffffffu, !wc_ok || bad == 0);
         }
         cst.load(pf_zw, pf_sv, x16);
         if (wc_ok && (grp + 1) * p.group < kbase + Kq) {  // prefetch the next group
@@ -334,7 +338,8 @@ __global__ void __launch_bounds__(stream::kThreads, 2)
         gstage = 0;
         ++grp;
       }
-      const bool sok = tc_wait(&full[s], ph, p.status, abort);
+      // warp-uniform: the MMAs below are warp-wide
+      const bool sok = __all_sync(0xffffffffu, tc_wait(&full[s], ph, p.status, abort));
       if (sok) {
         const uint8_t *box0 = stages + s * kStageBytes + bw * kBox;
         // two 16-row steps at a time keep the register footprint of a 32-row stage

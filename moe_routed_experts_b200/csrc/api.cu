@@ -82,7 +82,7 @@ static moe_status run_fwd_tc(int kind, ProjParams p, int nproj, bool bf, moe_dty
   if (err != MOE_OK) return err;
   if (conv) {
     p.x = conv;
-    p.act_dt = MOE_F16;
+    p.preconv = 1;
   }
   return kind == 3 ? launch_fwd_tc2(p, nproj, bf, st) : launch_fwd_tc(p, nproj, bf, st);
 }
@@ -325,7 +325,7 @@ extern "C" moe_status awq_input_backward(const void *grad, moe_dtype grad_dtype,
       if (s != MOE_OK) return s;
       p.grad[0] = reinterpret_cast<const uint16_t *>(w);
       p.grad[1] = reinterpret_cast<const uint16_t *>(grad2 ? w + one : w);
-      p.gdt = MOE_F16;
+      p.preconv = 1;
     }
     return kind == 3 ? launch_bwd_tc2(p, nproj, bf, st) : launch_bwd_tc(p, nproj, bf, st);
   }

@@ -9,26 +9,29 @@
 // ruda-tensor 0.21.33, src/frozen_awq.rs -- AWQ nibble order and scale-dtype
 //   coefficient rounding.
 //
-// Work unit = (expert e, token tile tt of 8*NT rows, slab sl, K split kq).
-// A slab is 512 output columns: for the gate/up pair, 32 packed word
-// columns (one 128-byte row segment) of each projection; for a single
-// projection, 64 word columns (two 128-byte segments).  A unit covers K/KQ
-// input rows.  Persistent CTAs (1 producer warp + 8 consumer warps) take
-// contiguous ranges of the expert-major unit list.
-//   producer: per unit, 1-D bulk copies of the tile's activation rows
-//     (double-buffered), then per ROWS input rows (32, 64 or 128, the
-//     largest the group size allows) one stage = two TMA boxes of
-//     [ROWS rows][32 words] with 128-byte swizzle, 48-64 KB in flight.
-//   consumer warp w: box w/4, word columns (w%4)*8 .. +7 of it, all rows of
-//     the unit.  Lane (g, t) reads rows t, t+4, t+8, t+12 of column g (the
+// Work item = (expert e, token tile tt of 8*NT rows, slab sl).  A slab is
+// 512 output columns: for the gate/up pair, 32 packed word columns (one
+// 128-byte row segment) of each projection; for a single projection, 64 word
+// columns (two 128-byte segments).  An item is K/ROWS pipeline stages of
+// ROWS input rows (32, 64 or 128, the largest the group size allows).  The
+// stages of all items, expert-major, form one list that the persistent CTAs
+// (8 warps; 2 per SM) split into equal contiguous ranges (stream-K), so
+// every CTA streams the same number of weight bytes whatever the routing.
+//   copies (lane 0 of warp 0): per stage two TMA boxes of [ROWS rows][32
+//     words] with 128-byte swizzle into a ring (64 KB in flight for 128-row
+//     stages), each issued once every warp released the ring slot's
+//     previous stage; per 512 input rows of an item, 1-D bulk copies of the
+//     item's activation rows (double-buffered, one chunk ahead).
+//   warp w: box w/4, word columns (w%4)*8 .. +7 of it, all rows of the
+//     stage.  Lane (g, t) reads rows t, t+4, t+8, t+12 of column g (the
 //     MMA's K index {2t, 2t+1, 2t+8, 2t+9} stands for them); the swizzle
-//     keeps those reads at most 2-way bank-conflicted.  The activation tile
-//     is converted to the scale dtype and permuted to that row order once
-//     per unit, so each B fragment is one 8-byte shared load.
-//   epilogue: with the whole K in the unit (KQ = 1), accumulators go
-//     through shared memory to bias, rounding and SwiGLU; with KQ > 1 each
-//     unit stores its FP32 partial sums to the workspace and a second kernel
-//     sums the KQ splits in kq order (deterministic) and finishes the rows.
+//     keeps those reads at most 2-way bank-conflicted.  Each activation
+//     chunk is converted to the scale dtype and permuted to that row order
+//     once, so each B fragment is one 8-byte shared load.
+//   end of a CTA's part of an item: a CTA that holds the whole item sends
+//     the accumulators through shared memory to bias, rounding and SwiGLU;
+//     CTAs sharing an item store FP32 partial sums, and a second kernel adds
+//     the parts in part order (deterministic) and finishes the rows.
 #include <cudaTypedefs.h>
 
 #include <mutex>
@@ -71,7 +74,7 @@ bool make_map_2d(CUtensorMap *map, const void *base, CUtensorMapDataType dt, int
 
 namespace stream {
 constexpr int kCW = 8;                    // consumer warps
-constexpr int kThreads = (kCW + 1) * 32;  // + one producer warp
+constexpr int kThreads = kCW * 32;  // lane 0 of warp 0 also issues the copies
 constexpr int kBoxW = 32;                 // words per box row (128 bytes)
 constexpr int kF = 512;                   // output columns of a unit
 constexpr int kBarBytes = 1024;           // barrier block; stages start 1024-byte aligned
@@ -104,23 +107,45 @@ __device__ __forceinline__ int box_offset(int row, int col) {
   return row * 128 + ((((col >> 2) ^ row) & 7) << 4) + ((col & 3) << 2);
 }
 
-struct UnitInfo {
-  int e, tt, sl, kq;
+// ------------------------------------------------------------------ stream-K schedule
+//
+// Work item = (expert e, token tile tt of 8*NT rows, slab sl), expert-major;
+// an item is nst = K / ROWS pipeline stages.  The stages of all items form
+// one list that the CTAs split evenly (each takes a contiguous range of at
+// least kMinStages stages), so a CTA may start or end inside an item.  A CTA
+// that holds a whole item finishes its rows in the fused epilogue; the CTAs
+// that share an item store their FP32 partial sums in part order (part =
+// the CTA's rank among them) and a second kernel adds the parts in that
+// order (deterministic) and finishes the rows.
+constexpr int kMinStages = 4;
+
+__host__ __device__ __forceinline__ int64_t sk_grid(int64_t G, int64_t grid) {
+  int64_t g = G / kMinStages;
+  if (g > grid) g = grid;
+  return g < 1 ? 1 : g;
+}
+// CTA holding stage s when G stages are split over `grid` CTAs.
+__device__ __forceinline__ int64_t sk_owner(int64_t s, int64_t G, int64_t grid) {
+  return ((s + 1) * grid + G - 1) / G - 1;
+}
+// Parts an item of nst stages can be split into (host bound of the workspace).
+__host__ __device__ __forceinline__ int sk_max_parts(int nst) { return (nst - 1 + kMinStages - 1) / kMinStages + 1; }
+
+struct ItemInfo {
+  int e, tt, sl;
   int64_t r0;
   int m;
 };
 
-__device__ __forceinline__ UnitInfo unit_info(const int32_t *pre, const int32_t *offsets, int E, int S, int KQ,
-                                              int64_t u) {
-  UnitInfo ui;
-  ui.e = unit_expert(pre, E, u);
-  const int64_t local = u - pre[ui.e];
-  ui.kq = (int)(local % KQ);
-  ui.sl = (int)((local / KQ) % S);
-  ui.tt = (int)(local / ((int64_t)KQ * S));
-  ui.r0 = offsets[ui.e];
-  ui.m = offsets[ui.e + 1] - (int32_t)ui.r0;
-  return ui;
+__device__ __forceinline__ ItemInfo item_info(const int32_t *pre, const int32_t *offsets, int E, int S, int64_t i) {
+  ItemInfo ii;
+  ii.e = unit_expert(pre, E, i);
+  const int local = (int)(i - pre[ii.e]);  // item counts fit 32 bits (pre is int32)
+  ii.tt = local / S;
+  ii.sl = local - ii.tt * S;
+  ii.r0 = offsets[ii.e];
+  ii.m = offsets[ii.e + 1] - (int32_t)ii.r0;
+  return ii;
 }
 
 template <typename MT, int NPROJ, int NT, int ROWS>
@@ -132,18 +157,20 @@ __global__ void __launch_bounds__(stream::kThreads, 2)
   constexpr int kRows = Geo<ROWS>::kRows, kBox = Geo<ROWS>::kBox, kStageBytes = Geo<ROWS>::kStageBytes;
   constexpr int kStages = Geo<ROWS>::kStages;
   constexpr int kSteps = ROWS / 16;
+  constexpr int kXst = 512 / ROWS;        // stages per activation chunk
+  constexpr int kXRows = kXst * ROWS;     // input rows per activation chunk (512)
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // 128-byte-swizzled TMA boxes need 1024-byte aligned destinations
   uint8_t *smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
-  const int E = p.E, KQ = p.kq;
-  const int64_t K = p.K, Kq = K / KQ;
+  const int E = p.E;
+  const int64_t K = p.K;
   const int64_t NW = p.N / 8;
   constexpr int kSlabW = NPROJ == 2 ? kBoxW : 2 * kBoxW;  // word columns of a slab
   const int S = (int)((NW + kSlabW - 1) / kSlabW);       // slabs per expert
-  const int nst = (int)(Kq / kRows);                     // stages per unit
-  const int xs_pitch = (int)(Kq * 2 + 16);  // bytes per converted token row (pad: conflict-free B loads)
-  const int xraw_bytes = (int)(8 * NT * Kq * 2);
-  const int64_t ncols = (int64_t)NPROJ * p.N;  // columns of the split-K partial rows
+  const int nst = (int)(K / kRows);                      // stages per item
+  constexpr int xs_pitch = kXRows * 2 + 16;  // bytes per converted token row (pad: conflict-free B loads)
+  constexpr int xraw_bytes = 8 * NT * kXRows * 2;
+  const int64_t ncols = (int64_t)NPROJ * p.N;  // columns of the partial rows
 
   uint64_t *full = reinterpret_cast<uint64_t *>(smem);
   uint64_t *empty = full + kStages;
@@ -177,64 +204,88 @@ __global__ void __launch_bounds__(stream::kThreads, 2)
 #endif
     fence_mbar_init();
   }
-  // units per expert; an inconsistent row range is flagged and skipped
+  // items per expert; an inconsistent row range is flagged and skipped
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
     const int32_t a = p.offsets[e], b = p.offsets[e + 1];
     const bool bad = a < 0 || b < a || (int64_t)b > p.A || (e == 0 && a != 0) || (e == E - 1 && (int64_t)b != p.A);
     if (bad && blockIdx.x == 0) report(p.status, MOE_DEVICE_ERR_OFFSETS);
-    cnt[e] = bad ? 0 : S * KQ * ((b - a + 8 * NT - 1) / (8 * NT));
+    cnt[e] = bad ? 0 : S * ((b - a + 8 * NT - 1) / (8 * NT));
   }
   __syncthreads();
   block_exclusive_scan(cnt, E, pre, tmp);
-  const int64_t U = pre[E];
-  const int64_t u0 = U * blockIdx.x / gridDim.x, u1 = U * (blockIdx.x + 1) / gridDim.x;
+  // the reduction kernel reads the item prefix from the workspace
+  if (blockIdx.x == 0 && p.counters)
+    for (int e = threadIdx.x; e <= E; e += blockDim.x) p.counters[e] = pre[e];
+  const int64_t G = (int64_t)pre[E] * nst;
+  const int64_t grid = sk_grid(G, gridDim.x);
+  if ((int64_t)blockIdx.x >= grid) return;  // nothing issued, nothing waited for
+  const int64_t g0 = G * blockIdx.x / grid, g1 = G * (blockIdx.x + 1) / grid;
 
-  if (warp == kCW) {
-    // ---------------- producer (one lane).  The activation tile of unit
-    // u+1 is requested when unit u starts, one unit ahead of its use.  A
-    // failed wait (timeout, or an abort elsewhere in the CTA) stops all
-    // further copies; the copies already issued are waited for before the
-    // lane exits (abort protocol, tma.cuh).
-    if (lane != 0) return;
-    uint32_t xissued = 0;
-    auto load_x = [&](int64_t u, uint32_t xi) -> bool {
-      const UnitInfo ui = unit_info(pre, p.offsets, E, S, KQ, u);
-      const int tok0 = ui.tt * 8 * NT, mrows = min(8 * NT, ui.m - tok0);
-      const uint32_t xb = xi & 1, xuse = xi >> 1;
-      if (xuse > 0 && !tc_wait(&xempty[xb], (xuse - 1) & 1, p.status, abort)) return false;
-      mbar_arrive_expect_tx(&xfull[xb], (uint32_t)(mrows * Kq * 2));
-      for (int r = 0; r < mrows; ++r)
-        bulk_load(xraw + xb * xraw_bytes + r * Kq * 2, p.x + act_row(p, ui.r0 + tok0 + r) * K + ui.kq * Kq,
-                  (uint32_t)(Kq * 2), &xfull[xb]);
-      ++xissued;
-      return true;
-    };
-    uint32_t it = 0, xi = 0;
-    bool live = u0 >= u1 || load_x(u0, 0);
-    for (int64_t u = u0; u < u1 && live; ++u, ++xi) {
-      if (u + 1 < u1 && !load_x(u + 1, xi + 1)) break;
-      const UnitInfo ui = unit_info(pre, p.offsets, E, S, KQ, u);
-      const int32_t row0 = (int32_t)(ui.e * K + ui.kq * Kq);
-      for (int c = 0; c < nst; ++c, ++it) {
-        const uint32_t s = it % kStages, use = it / kStages;
-        if (use > 0 && !tc_wait(&empty[s], (use - 1) & 1, p.status, abort)) {
-          live = false;
-          break;
-        }
-        mbar_arrive_expect_tx(&full[s], kStageBytes);
-        uint8_t *dst = stages + s * kStageBytes;
-        if (NPROJ == 2) {
-          tma_load_2d(dst, &map0, &full[s], ui.sl * kBoxW, row0 + kRows * c);
-          tma_load_2d(dst + kBox, &map1, &full[s], ui.sl * kBoxW, row0 + kRows * c);
-        } else {
-          tma_load_2d(dst, &map0, &full[s], ui.sl * 2 * kBoxW, row0 + kRows * c);
-          tma_load_2d(dst + kBox, &map0, &full[s], ui.sl * 2 * kBoxW + kBoxW, row0 + kRows * c);
-        }
-      }
+  // ---------------- copies, issued by lane 0 of consumer warp 0: stage
+  // j - g0 of the ring is stage j of the list, issued once all consumers
+  // released the slot's previous stage; activation chunks one ahead.
+  int64_t nxt = g0;        // next stage to issue (thread 0 only)
+  uint32_t xissued = 0;    // activation chunks issued (thread 0 only)
+  bool plive = true;       // thread 0 stops issuing after a failed wait
+  const bool issuer = threadIdx.x == 0;
+  int64_t iss_i = -1;
+  ItemInfo iss_ii{};
+  auto issue_info = [&](int64_t i) -> const ItemInfo & {
+    if (i != iss_i) {
+      iss_i = i;
+      iss_ii = item_info(pre, p.offsets, E, S, i);
     }
-    tma_drain(full, it, kStages, p.status);
-    tma_drain(xfull, xissued, 2, p.status);
-    return;
+    return iss_ii;
+  };
+  // activation chunk of stage j (rows of j's item, the 512 input rows holding j)
+  auto load_x = [&](int64_t j, uint32_t xi) {
+    const int64_t i = j / nst;
+    const int ch = (int)(j - i * nst) / kXst;
+    const ItemInfo &ii = issue_info(i);
+    const int tok0 = ii.tt * 8 * NT, mrows = min(8 * NT, ii.m - tok0);
+    const int64_t k0 = (int64_t)ch * kXRows;
+    const int64_t len = min((int64_t)kXRows, K - k0);
+    const uint32_t xb = xi & 1, xuse = xi >> 1;
+    if (xuse > 0 && !tc_wait(&xempty[xb], (xuse - 1) & 1, p.status, abort)) {
+      plive = false;
+      return;
+    }
+    mbar_arrive_expect_tx(&xfull[xb], (uint32_t)(mrows * len * 2));
+    for (int r = 0; r < mrows; ++r)
+      bulk_load(xraw + xb * xraw_bytes + r * kXRows * 2, p.x + act_row(p, ii.r0 + tok0 + r) * K + k0,
+                (uint32_t)(len * 2), &xfull[xb]);
+    ++xissued;
+  };
+  auto issue_stage = [&](int64_t j) {
+    const uint32_t s = (uint32_t)((j - g0) % kStages);
+    const int64_t i = j / nst;
+    const int c = (int)(j - i * nst);
+    const ItemInfo &ii = issue_info(i);
+    const int32_t row0 = (int32_t)(ii.e * K + (int64_t)c * kRows);
+    mbar_arrive_expect_tx(&full[s], kStageBytes);
+    uint8_t *dst = stages + s * kStageBytes;
+    if (NPROJ == 2) {
+      tma_load_2d(dst, &map0, &full[s], ii.sl * kBoxW, row0);
+      tma_load_2d(dst + kBox, &map1, &full[s], ii.sl * kBoxW, row0);
+    } else {
+      tma_load_2d(dst, &map0, &full[s], ii.sl * 2 * kBoxW, row0);
+      tma_load_2d(dst + kBox, &map0, &full[s], ii.sl * 2 * kBoxW + kBoxW, row0);
+    }
+  };
+  // blocking: issue every stage up to `upto` (waits for the slots' release)
+  auto issue_upto = [&](int64_t upto) {
+    while (plive && nxt <= upto && nxt < g1) {
+      const uint32_t s = (uint32_t)((nxt - g0) % kStages), use = (uint32_t)((nxt - g0) / kStages);
+      if (use > 0 && !tc_wait(&empty[s], (use - 1) & 1, p.status, abort)) {
+        plive = false;
+        break;
+      }
+      issue_stage(nxt++);
+    }
+  };
+  if (issuer && g0 < g1) {
+    load_x(g0, 0);
+    issue_upto(g0 + kStages - 1);
   }
 
   // ---------------- consumers
@@ -248,105 +299,123 @@ __global__ void __launch_bounds__(stream::kThreads, 2)
   // byte offsets of rows t and t+4 of column cgw*8+g in a swizzled box; rows
   // t + 4i + 16h differ from these by multiples of 8 rows (same swizzle)
   const int woff0 = box_offset(t, cgw * 8 + g), woff1 = box_offset(t + 4, cgw * 8 + g);
+  const int spg = p.group / kRows;  // stages per group (group % kRows == 0 on this path)
+
+  float acc[NT][4][4], acc16[NT][2][4];
+  FwdConsts<MT> cst;
+  bool x16 = false;
+  ItemInfo ii{};
+  int tok0 = 0, mrows = 0, seg_c0 = 0, seg_c1 = 0, xbase = 0, gstage = 0;
+  int64_t wc = 0, grp = 0;
+  bool wc_ok = false;
+  const int32_t *qzp = qz;
+  const uint16_t *scp = sc;
+  uint32_t pf_zw = 0u;
+  uint4 pf_sv = make_uint4(0, 0, 0, 0);
   uint32_t it = 0, xi = 0;
-  for (int64_t u = u0; u < u1; ++u, ++xi) {
-    const UnitInfo ui = unit_info(pre, p.offsets, E, S, KQ, u);
-    const int tok0 = ui.tt * 8 * NT, mrows = min(8 * NT, ui.m - tok0);
-    const int e = ui.e;
-    const int64_t wc = NPROJ == 2 ? (int64_t)ui.sl * kBoxW + cgw * 8 + g
-                                  : (int64_t)ui.sl * 2 * kBoxW + bw * kBoxW + cgw * 8 + g;
-    const bool wc_ok = wc < NW;
-    const int64_t wcs = wc_ok ? wc : 0;
-    const int64_t kbase = (int64_t)ui.kq * Kq;
-    const int32_t *qzp = qz + (e * ngroups) * NW + wcs;
-    const uint16_t *scp = sc + (e * ngroups) * p.N + 8 * wcs;
-    int64_t grp = kbase / p.group;
-    // the first group's zeros/scales are requested before the activation
-    // tile is converted, so their latency overlaps that work
-    uint32_t pf_zw = wc_ok ? (uint32_t)__ldg(qzp + grp * NW) : 0u;
-    uint4 pf_sv = wc_ok ? __ldg(reinterpret_cast<const uint4 *>(scp + grp * p.N)) : make_uint4(0, 0, 0, 0);
-
-    // activation tile: raw rows -> scale dtype, row order t, t+4, t+8, t+12 per 16.
-    // After an abort every consumer warp still runs the loop (the named
-    // barriers stay matched) but waits for, computes and arrives on nothing.
-    const uint32_t xb = xi & 1;
-    // every consumer is done reading the previous unit's converted tile
-    named_barrier(1, kCW * 32);
-    const bool xok = tc_wait(&xfull[xb], (xi >> 1) & 1, p.status, abort);
-    if (xok) {
-      const uint8_t *src = xraw + xb * xraw_bytes;
-      const int64_t halves = (int64_t)mrows * (Kq / 8);
-      for (int64_t q = threadIdx.x; q < halves; q += kCW * 32) {
-        const int tok = (int)(q / (Kq / 8));
-        const int64_t hb = q % (Kq / 8), blk = hb >> 1, h = hb & 1;
-        const uint4 v = *reinterpret_cast<const uint4 *>(src + (tok * Kq + blk * 16 + h * 8) * 2);
-        uint32_t pr[4] = {prmt(v.x, v.z, 0x5410u), prmt(v.x, v.z, 0x7632u), prmt(v.y, v.w, 0x5410u),
-                          prmt(v.y, v.w, 0x7632u)};  // (row i, row i+4) of the half
-        act_pairs_to_mt<MT, 4>(pr, p.act_dt, act_bad);
-        uint8_t *dst = xs + tok * xs_pitch + (blk * 16 + 2 * h) * 2;
+  for (int64_t j = g0; j < g1; ++j, ++it) {
+    const int64_t i = j / nst;
+    const int c = (int)(j - i * nst);
+    if (j == g0 || c == 0) {  // a segment of item i starts: its rows, columns and first group
+      ii = item_info(pre, p.offsets, E, S, i);
+      tok0 = ii.tt * 8 * NT;
+      mrows = min(8 * NT, ii.m - tok0);
+      seg_c0 = c;
+      seg_c1 = (int)min((int64_t)nst, (int64_t)c + (g1 - j));
+      wc = NPROJ == 2 ? (int64_t)ii.sl * kBoxW + cgw * 8 + g : (int64_t)ii.sl * 2 * kBoxW + bw * kBoxW + cgw * 8 + g;
+      wc_ok = wc < NW;
+      const int64_t wcs = wc_ok ? wc : 0;
+      qzp = qz + ((int64_t)ii.e * ngroups) * NW + wcs;
+      scp = sc + ((int64_t)ii.e * ngroups) * p.N + 8 * wcs;
+      grp = (int64_t)c * kRows / p.group;
+      gstage = (int)(((int64_t)c * kRows % p.group) / kRows);
+      pf_zw = wc_ok ? (uint32_t)__ldg(qzp + grp * NW) : 0u;
+      pf_sv = wc_ok ? __ldg(reinterpret_cast<const uint4 *>(scp + grp * p.N)) : make_uint4(0, 0, 0, 0);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) *reinterpret_cast<uint32_t *>(dst + 8 * i) = pr[i];
+      for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+#pragma unroll
+          for (int k = 0; k < 4; ++k) acc[nt][q][k] = 0.f;
+#pragma unroll
+        for (int q = 0; q < 2; ++q)
+#pragma unroll
+          for (int k = 0; k < 4; ++k) acc16[nt][q][k] = 0.f;
       }
     }
-    __syncwarp();
-    if (lane == 0 && xok) mbar_arrive(&xempty[xb]);
-    named_barrier(1, kCW * 32);
-
-    // acc: every slot in its true scale; acc16: odd slots taken 16 times
-    // larger (F16 groups whose scales allow it, see fwd_pairs16)
-    float acc[NT][4][4], acc16[NT][2][4];
+    if (j == g0 || c % kXst == 0) {
+      // a new activation chunk: request the next one, then convert this one
+      // (raw rows -> scale dtype, row order t, t+4, t+8, t+12 per 16).  After
+      // an abort every consumer warp still runs the loop (the named barriers
+      // stay matched) but waits for, computes and arrives on nothing.
+      const uint32_t xcur = xi++;
+      xbase = c - c % kXst;
+      if (issuer && plive) {
+        const int64_t nc = (int64_t)xbase + kXst;
+        const int64_t jn = nc < nst ? i * nst + nc : (i + 1) * nst;
+        if (jn < g1) load_x(jn, xcur + 1);
+      }
+      const uint32_t xb = xcur & 1;
+      // every consumer is done reading the previous chunk's converted tile
+      named_barrier(1, kCW * 32);
+      const bool xok = tc_wait(&xfull[xb], (xcur >> 1) & 1, p.status, abort);
+      if (xok) {
+        const uint8_t *src = xraw + xb * xraw_bytes;
+        const int len = (int)min((int64_t)kXRows, K - (int64_t)xbase * kRows);
+        const int per_tok = len / 8, halves = mrows * per_tok;
+        for (int q = threadIdx.x; q < halves; q += kCW * 32) {
+          const int tok = q / per_tok;
+          const int hb = q - tok * per_tok, blk = hb >> 1, h = hb & 1;
+          const uint4 v = *reinterpret_cast<const uint4 *>(src + (tok * kXRows + blk * 16 + h * 8) * 2);
+          uint32_t pr[4] = {prmt(v.x, v.z, 0x5410u), prmt(v.x, v.z, 0x7632u), prmt(v.y, v.w, 0x5410u),
+                            prmt(v.y, v.w, 0x7632u)};  // (row i, row i+4) of the half
+          act_pairs_to_mt<MT, 4>(pr, p.act_dt, act_bad);
+          uint8_t *dst = xs + tok * xs_pitch + (blk * 16 + 2 * h) * 2;
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-#pragma unroll
-      for (int q = 0; q < 4; ++q)
-#pragma unroll
-        for (int i = 0; i < 4; ++i) acc[nt][q][i] = 0.f;
-#pragma unroll
-      for (int q = 0; q < 2; ++q)
-#pragma unroll
-        for (int i = 0; i < 4; ++i) acc16[nt][q][i] = 0.f;
+          for (int k = 0; k < 4; ++k) *reinterpret_cast<uint32_t *>(dst + 8 * k) = pr[k];
+        }
+      }
+      __syncwarp();
+      if (lane == 0 && xok) mbar_arrive(&xempty[xb]);
+      named_barrier(1, kCW * 32);
     }
-    FwdConsts<MT> cst;
-    bool x16 = false;
-    const int spg = p.group / kRows;  // stages per group (group % kRows == 0 on this path)
-    int gstage = (int)((kbase % p.group) / kRows);
-    for (int c = 0; c < nst; ++c, ++it) {
-      const uint32_t s = it % kStages, ph = (it / kStages) & 1;
-      if (c == 0 || gstage == 0) {  // a stage lies inside one group
-        if (std::is_same<MT, __half>::value) {
-          // 16 RNE((q - z) s) = RNE(16 (q - z) s) needs every nonzero product
-          // normal before and after the scaling: 0 or 2^-14 <= |s| <= 256 for
-          // all 8 scales of this column group
-          const uint32_t w4[4] = {pf_sv.x, pf_sv.y, pf_sv.z, pf_sv.w};
-          uint32_t bad = 0;
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const uint32_t lo = w4[i] & 0x7FFFu, hi = (w4[i] >> 16) & 0x7FFFu;
-            bad |= (lo > 0x5C00u) | (hi > 0x5C00u) | (lo != 0u && lo < 0x0400u) | (hi != 0u && hi < 0x0400u);
-          }
-          // one decision per warp: the MMAs below are warp-wide (mma.sync), so
-          // every lane must take the same branch; a lane without a column votes yes
-          x16 = __all_sync(0xffffffffu, !wc_ok || bad == 0);
-        }
-        cst.load(pf_zw, pf_sv, x16);
-        if (wc_ok && (grp + 1) * p.group < kbase + Kq) {  // prefetch the next group
-          pf_zw = (uint32_t)__ldg(qzp + (grp + 1) * NW);
-          pf_sv = __ldg(reinterpret_cast<const uint4 *>(scp + (grp + 1) * p.N));
-        }
+    const uint32_t s = (uint32_t)((j - g0) % kStages), ph = (uint32_t)(((j - g0) / kStages) & 1);
+    if (gstage == 0 || j == g0 || c == seg_c0) {  // a stage lies inside one group
+      if (std::is_same<MT, __half>::value) {
+        // 16 RNE((q - z) s) = RNE(16 (q - z) s) needs every nonzero product
+        // normal before and after the scaling: 0 or 2^-14 <= |s| <= 256 for
+        // all 8 scales of this column group
+        // all 8 scales of this column group (zero scales take the plain path)
+        const uint32_t m0 = pf_sv.x & 0x7FFF7FFFu, m1 = pf_sv.y & 0x7FFF7FFFu, m2 = pf_sv.z & 0x7FFF7FFFu,
+                       m3 = pf_sv.w & 0x7FFF7FFFu;
+        uint32_t mx = umax16x2(umax16x2(m0, m1), umax16x2(m2, m3));
+        uint32_t mn = umin16x2(umin16x2(m0, m1), umin16x2(m2, m3));
+        mx = umax16x2(mx, mx >> 16) & 0xFFFFu;
+        mn = umin16x2(mn, mn >> 16) & 0xFFFFu;  // the high lane of mn >> 16 is 0: only the low lane is read
+        // one decision per warp: the MMAs below are warp-wide (mma.sync), so
+        // every lane must take the same branch; a lane without a column votes yes
+        x16 = __all_sync(0xffffffffu, !wc_ok || (mx <= 0x5C00u && mn >= 0x0400u));
       }
-      if (++gstage == spg) {
-        gstage = 0;
-        ++grp;
+      load_consts_fast<MT>(cst, pf_zw, pf_sv, x16);
+      if (wc_ok && (grp + 1) * p.group < K) {  // prefetch the next group
+        pf_zw = (uint32_t)__ldg(qzp + (grp + 1) * NW);
+        pf_sv = __ldg(reinterpret_cast<const uint4 *>(scp + (grp + 1) * p.N));
       }
-      // warp-uniform: the MMAs below are warp-wide
-      const bool sok = __all_sync(0xffffffffu, tc_wait(&full[s], ph, p.status, abort));
-      if (sok) {
-        const uint8_t *box0 = stages + s * kStageBytes + bw * kBox;
-        // two 16-row steps at a time keep the register footprint of a 32-row stage
+    }
+    if (++gstage == spg) {
+      gstage = 0;
+      ++grp;
+    }
+    if (issuer) issue_upto(j + kStages - 1);
+    // warp-uniform: the MMAs below are warp-wide
+    const bool sok = __all_sync(0xffffffffu, tc_wait(&full[s], ph, p.status, abort));
+    if (sok) {
+      const uint8_t *box0 = stages + s * kStageBytes + bw * kBox;
+      // two 16-row steps at a time keep the register footprint of a 32-row stage
 #pragma unroll 1
-        for (int hh = 0; hh < kSteps; hh += 2) {
+      for (int hh = 0; hh < kSteps; hh += 2) {
         const uint8_t *box = box0 + (16 * hh) * 128;
-        const int xrow0 = kRows * c + 16 * hh;
+        const int xrow0 = kRows * (c - xbase) + 16 * hh;
         uint32_t w[2][4];
         uint32_t b0[2][NT], b1[2][NT];
 #pragma unroll
@@ -392,25 +461,26 @@ __global__ void __launch_bounds__(stream::kThreads, 2)
               for (int nt = 0; nt < NT; ++nt) mma16816<MT>(acc[nt][q], af[q], b0[h][nt], b1[h][nt]);
           }
         }
-        }
       }
-      __syncwarp();
-      if (lane == 0 && sok) mbar_arrive(&empty[s]);
     }
-    const bool unit_ok = !*abort;  // no stores from a unit an abort cut short
+    __syncwarp();
+    if (lane == 0 && sok) mbar_arrive(&empty[s]);
+    if (c != seg_c1 - 1) continue;
+
+    // ---------------- the segment ends here
+    const bool seg_ok = !*abort;  // no stores from a segment an abort cut short
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {  // fold the 16x-scaled odd slots back (exact power-of-two scaling)
-        acc[nt][1][i] += acc16[nt][0][i] * 0.0625f;
-        acc[nt][3][i] += acc16[nt][1][i] * 0.0625f;
+      for (int k = 0; k < 4; ++k) {  // fold the 16x-scaled odd slots back (exact power-of-two scaling)
+        acc[nt][1][k] += acc16[nt][0][k] * 0.0625f;
+        acc[nt][3][k] += acc16[nt][1][k] * 0.0625f;
       }
-
-    if (KQ > 1) {
-      // split K: this unit's partial sums go to partials[kq][row][column];
-      // a second kernel sums the splits in kq order and finishes the outputs
-      float *prow = p.partials + ((int64_t)ui.kq * p.A + ui.r0 + tok0) * ncols;
-      if (wc_ok && unit_ok) {
+    if (seg_c0 != 0 || seg_c1 != nst) {
+      // a part of a shared item: FP32 partial sums to partials[part][row][column]
+      const int64_t part = (int64_t)blockIdx.x - sk_owner(i * nst, G, grid);
+      float *prow = p.partials + (part * p.A + ii.r0 + tok0) * ncols;
+      if (wc_ok && seg_ok) {
         const int64_t col0 = (int64_t)jw * p.N + wc * 8;
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt)
@@ -427,8 +497,7 @@ __global__ void __launch_bounds__(stream::kThreads, 2)
       }
       continue;
     }
-
-    // whole K in this unit: accumulators -> red[token][column], epilogue
+    // the whole item in this CTA: accumulators -> red[token][column], epilogue
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
@@ -440,15 +509,19 @@ __global__ void __launch_bounds__(stream::kThreads, 2)
         red[(tk + 1) * kF + f + 1] = acc[nt][q][3];
       }
     named_barrier(1, kCW * 32);
-    constexpr int kOut = NPROJ == 2 ? kF / 2 : kF;  // output columns of the unit
+    constexpr int kOut = NPROJ == 2 ? kF / 2 : kF;  // output columns of the item
     for (int v8 = threadIdx.x; v8 < mrows * (kOut / 8); v8 += kCW * 32) {
       const int tk = v8 / (kOut / 8), fq = (v8 % (kOut / 8)) * 8;
-      const int64_t n0 = (int64_t)ui.sl * kOut + fq;
-      if (n0 >= p.N || !unit_ok) continue;
+      const int64_t n0 = (int64_t)ii.sl * kOut + fq;
+      if (n0 >= p.N || !seg_ok) continue;
       const float *g8 = red + tk * kF + fq;
-      finish8<NPROJ>(p, e, ui.r0 + tok0 + tk, n0, g8, g8 + 256);
+      finish8<NPROJ>(p, ii.e, ii.r0 + tok0 + tk, n0, g8, g8 + 256);
     }
     named_barrier(1, kCW * 32);  // red is free again
+  }
+  if (issuer) {  // nothing asynchronous may be in flight at exit (abort protocol)
+    tma_drain(full, (uint32_t)(nxt - g0), kStages, p.status);
+    tma_drain(xfull, xissued, 2, p.status);
   }
   if (act_bad) report(p.status, MOE_DEVICE_ERR_ACT_RANGE);
 #ifdef MOE_TEST_HOOKS
@@ -465,31 +538,24 @@ __global__ void __launch_bounds__(stream::kThreads, 2)
 #endif
 }
 
-// Split-K reduction: out[r, n..n+8) from sum over kq of partials[kq][r][.]
-// (in kq order), then bias, rounding and SwiGLU as in the fused epilogue.
-template <int NPROJ>
+// Items split over several CTAs: out[r, n..n+8) from the sum of their parts
+// (in part order), then bias, rounding and SwiGLU as in the fused epilogue.
+// p.counters holds the item prefix per expert, p.kq the first kernel's grid.
+template <int NPROJ, int NT, int ROWS>
 __global__ void __launch_bounds__(256) awq_stream_reduce_kernel(ProjParams p) {
   pdl_enter();  // programmatic dependent launch: the previous kernel is done
+  using namespace stream;
+  constexpr int kSlabW = NPROJ == 2 ? kBoxW : 2 * kBoxW;
+  constexpr int kOut = kSlabW * 8;
   const int64_t ncols = (int64_t)NPROJ * p.N;
   const int64_t per_row = p.N / 8;
   const int64_t total = p.A * per_row;
+  const int S = (int)((p.N / 8 + kSlabW - 1) / kSlabW);
+  const int nst = (int)(p.K / ROWS);
+  const int64_t G = (int64_t)p.counters[p.E] * nst;
+  const int64_t grid = sk_grid(G, p.kq);
   for (int64_t v = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; v < total; v += (int64_t)gridDim.x * blockDim.x) {
     const int64_t r = v / per_row, n0 = (v % per_row) * 8;
-    float a[NPROJ][8];
-#pragma unroll
-    for (int j = 0; j < NPROJ; ++j)
-#pragma unroll
-      for (int i = 0; i < 8; ++i) a[j][i] = 0.f;
-    for (int kq = 0; kq < p.kq; ++kq) {
-      const float *src = p.partials + ((int64_t)kq * p.A + r) * ncols + n0;
-#pragma unroll
-      for (int j = 0; j < NPROJ; ++j) {
-        const float4 x0 = __ldcg(reinterpret_cast<const float4 *>(src + j * p.N));
-        const float4 x1 = __ldcg(reinterpret_cast<const float4 *>(src + j * p.N + 4));
-        a[j][0] += x0.x; a[j][1] += x0.y; a[j][2] += x0.z; a[j][3] += x0.w;
-        a[j][4] += x1.x; a[j][5] += x1.y; a[j][6] += x1.z; a[j][7] += x1.w;
-      }
-    }
     // expert of row r: largest e with offsets[e] <= r (non-empty range)
     int lo = 0, hi = p.E - 1;
     while (lo < hi) {
@@ -497,48 +563,59 @@ __global__ void __launch_bounds__(256) awq_stream_reduce_kernel(ProjParams p) {
       if (p.offsets[mid] <= r) lo = mid;
       else hi = mid - 1;
     }
+    const int64_t tt = (r - p.offsets[lo]) / (8 * NT);
+    const int64_t item = p.counters[lo] + tt * S + n0 / kOut;
+    if (r < p.offsets[lo] || item < 0 || item >= p.counters[p.E]) continue;  // rows of a range flagged bad
+    const int64_t first = sk_owner(item * nst, G, grid), last = sk_owner(item * nst + nst - 1, G, grid);
+    if (first == last || last - first >= sk_max_parts(nst)) continue;  // the fused epilogue wrote these outputs
+    float a[NPROJ][8];
+#pragma unroll
+    for (int jj = 0; jj < NPROJ; ++jj)
+#pragma unroll
+      for (int k = 0; k < 8; ++k) a[jj][k] = 0.f;
+    for (int64_t part = 0; part <= last - first; ++part) {
+      const float *src = p.partials + (part * p.A + r) * ncols + n0;
+#pragma unroll
+      for (int jj = 0; jj < NPROJ; ++jj) {
+        const float4 x0 = __ldcg(reinterpret_cast<const float4 *>(src + jj * p.N));
+        const float4 x1 = __ldcg(reinterpret_cast<const float4 *>(src + jj * p.N + 4));
+        a[jj][0] += x0.x; a[jj][1] += x0.y; a[jj][2] += x0.z; a[jj][3] += x0.w;
+        a[jj][4] += x1.x; a[jj][5] += x1.y; a[jj][6] += x1.z; a[jj][7] += x1.w;
+      }
+    }
     finish8<NPROJ>(p, lo, r, n0, a[0], a[NPROJ - 1]);
   }
 }
 
 // ------------------------------------------------------------------ launch
 
-static size_t stream_smem(int nt, int64_t Kq, int64_t E, int rows) {
+static size_t stream_smem(int nt, int64_t E, int rows) {
   using namespace stream;
   const size_t ring = rows == 128  ? (size_t)Geo<128>::kStages * Geo<128>::kStageBytes
                      : rows == 64 ? (size_t)Geo<64>::kStages * Geo<64>::kStageBytes
                                   : (size_t)Geo<32>::kStages * Geo<32>::kStageBytes;
-  return 1024 /* alignment slack */ + kBarBytes + ring + 2 * (size_t)8 * nt * Kq * 2 +
-         (size_t)8 * nt * (Kq * 2 + 16) + (size_t)8 * nt * kF * 4 + (size_t)(2 * E + 1 + 32) * 4;
+  return 1024 /* alignment slack */ + kBarBytes + ring + 2 * (size_t)8 * nt * 512 * 2 +
+         (size_t)8 * nt * (512 * 2 + 16) + (size_t)8 * nt * kF * 4 + (size_t)(2 * E + 1 + 32) * 4;
 }
 
-// K splits: keep each unit at >= 384 input rows when K allows, whole
-// stages, and the split-K partials (KQ * A * columns FP32) bounded.
+// Workspace: the parts of split items (at most sk_max_parts per item) and
+// the item prefix for the reduction.
 StreamPlan stream_plan(int64_t A, int64_t K, int64_t N, int64_t E, int64_t group, int nproj, int nt) {
   StreamPlan pl{};
   pl.fits = false;
   // TMA needs 16-byte word-row pitches; a stage lies inside one group
   if (N % 32 != 0 || K % 32 != 0 || group % 32 != 0) return pl;
   const int rows = (K % 128 == 0 && group % 128 == 0) ? 128 : (K % 64 == 0 && group % 64 == 0) ? 64 : 32;
-  // K splits: 4 when each split keeps >= 256 input rows (whole stages),
-  // else 3 or 2 (a split count that leaves about five units per CTA evens
-  // out the tail of the persistent grid better than fewer, longer units)
-  int kq = 1;
-  for (int d : {4, 3, 2})
-    if ((K / rows) % d == 0 && K / d >= 256) {
-      kq = d;
-      break;
-    }
-  while (kq > 1 && (size_t)kq * A * nproj * N * 4 > ((size_t)256 << 20)) kq >>= 1;
-  if (stream_smem(nt, K / kq, E, rows) > 200 * 1024) return pl;
+  const int parts = sk_max_parts((int)(K / rows));
+  const size_t pbytes = (size_t)parts * A * nproj * N * 4;
+  if (pbytes > ((size_t)512 << 20)) return pl;
+  if (stream_smem(nt, E, rows) > 200 * 1024) return pl;
   pl.rows = rows;
   pl.fits = true;
-  pl.kq = kq;
-  if (kq > 1) {
-    pl.partial_off = 0;
-    pl.bytes = (size_t)kq * A * nproj * N * 4;
-    pl.counter_off = pl.bytes;
-  }
+  pl.kq = parts;
+  pl.partial_off = 0;
+  pl.counter_off = (pbytes + 255) & ~size_t(255);
+  pl.bytes = pl.counter_off + (size_t)(E + 1) * 4;
   return pl;
 }
 
@@ -567,18 +644,19 @@ static moe_status launch_stream_r(const ProjParams &p0, cudaStream_t st) {
       !make_map_2d(&m1, p.qw[NPROJ - 1], CU_TENSOR_MAP_DATA_TYPE_INT32, 4, NW, rows, kBoxW, kRows,
                    CU_TENSOR_MAP_SWIZZLE_128B))
     return set_error(MOE_ERR_CUDA, "tensor map encoding failed for the packed words");
-  const size_t smem = stream_smem(NT, p.K / p.kq, p.E, ROWS);
+  const size_t smem = stream_smem(NT, p.E, ROWS);
   auto kern = awq_fwd_stream_kernel<MT, NPROJ, NT, ROWS>;
   cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  const int per_sm = smem <= 110 * 1024 ? 2 : 1;
-  launch_pdl(kern, dim3(num_sms() * per_sm), dim3(kThreads), smem, st, m0, m1, p);
+  const int grid = num_sms() * (smem <= 110 * 1024 ? 2 : 1);
+  p.kq = grid;
+  launch_pdl(kern, dim3(grid), dim3(kThreads), smem, st, m0, m1, p);
   moe_status s = check_launch("awq_fwd_stream_kernel");
-  if (s != MOE_OK || p.kq == 1) return s;
+  if (s != MOE_OK) return s;
   const int64_t work = p.A * (p.N / 8);
   int64_t blocks = (work + 255) / 256;
   const int64_t cap = (int64_t)num_sms() * 8;
   if (blocks > cap) blocks = cap;
-  launch_pdl(awq_stream_reduce_kernel<NPROJ>, dim3((unsigned)blocks), dim3(256), 0, st, p);
+  launch_pdl(awq_stream_reduce_kernel<NPROJ, NT, ROWS>, dim3((unsigned)blocks), dim3(256), 0, st, p);
   return check_launch("awq_stream_reduce_kernel");
 }
 
@@ -591,15 +669,11 @@ static moe_status launch_stream_t(const ProjParams &p, int rows, cudaStream_t st
 moe_status launch_fwd_stream(ProjParams p, int nproj, bool bf16_mma, int nt, void *ws, size_t ws_bytes,
                              cudaStream_t st) {
   const StreamPlan pl = stream_plan(p.A, p.K, p.N, p.E, p.group, nproj, nt);
-  p.kq = pl.kq;
-  p.partials = nullptr;
-  p.counters = nullptr;
-  if (pl.kq > 1) {
-    if (!ws || ws_bytes < pl.bytes || !aligned16(ws))
-      return set_error(MOE_ERR_WORKSPACE, "projection workspace of %zu bytes, need %zu (16-byte aligned)", ws_bytes,
-                       pl.bytes);
-    p.partials = reinterpret_cast<float *>(static_cast<char *>(ws) + pl.partial_off);
-  }
+  if (!ws || ws_bytes < pl.bytes || !aligned16(ws))
+    return set_error(MOE_ERR_WORKSPACE, "projection workspace of %zu bytes, need %zu (16-byte aligned)", ws_bytes,
+                     pl.bytes);
+  p.partials = reinterpret_cast<float *>(static_cast<char *>(ws) + pl.partial_off);
+  p.counters = reinterpret_cast<int32_t *>(static_cast<char *>(ws) + pl.counter_off);
   const int r = pl.rows;
   if (bf16_mma) {
     if (nproj == 2)

@@ -245,7 +245,8 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
     const int b0 = (col >> 3) * 8192 + rg * 128 + (((col & 7) ^ rg) << 4);  // + 1 KB per 8 rows
     const int spg = p.group / kBK;  // steps per group
     uint32_t act_bad = 0;  // a converted input outside F16's normal range
-    const bool convert = p.act_dt != (std::is_same<MT, __half>::value ? MOE_F16 : MOE_BF16);
+    // inputs in the other 16-bit dtype are converted here unless a one-time copy was made
+    const bool convert = !p.preconv && p.act_dt != (std::is_same<MT, __half>::value ? MOE_F16 : MOE_BF16);
     uint32_t it = 0;
     bool live = true;
     // zeros/scales of a tile's word column; the first group of the next tile

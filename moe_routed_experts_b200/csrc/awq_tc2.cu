@@ -251,7 +251,8 @@ __global__ void __launch_bounds__(tc2::kThreads, 1)
     const int b0 = (col >> 3) * kNBlock + (rg >> 3) * 1024 + (rg & 7) * 128 + (((col & 7) ^ (rg & 7)) << 4);
     const int spg = p.group / kBK;
     uint32_t act_bad = 0;  // a converted input outside F16's normal range
-    const bool convert = p.act_dt != (std::is_same<MT, __half>::value ? MOE_F16 : MOE_BF16);
+    // inputs in the other 16-bit dtype are converted here unless a one-time copy was made
+    const bool convert = !p.preconv && p.act_dt != (std::is_same<MT, __half>::value ? MOE_F16 : MOE_BF16);
     uint64_t *bready0 = bready;  // CTA 0's barriers, addressed through the cluster window
     uint32_t it = 0;
     bool live = true;

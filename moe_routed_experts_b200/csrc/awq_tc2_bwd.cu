@@ -223,7 +223,8 @@ __global__ void __launch_bounds__(tc2b::kThreads, 1)
     const int b0 = (wcol >> 3) * kBAtom + (rband >> 3) * 1024 + (rband & 7) * 128 + (((wcol & 7) ^ (rband & 7)) << 4);
     const int gshift = p.group >= kHalf ? 8 : 6;  // group row of band i: (32 i) >> gshift (groups 64 or >= 128)
     uint32_t act_bad = 0;  // a converted input outside F16's normal range
-    const bool convert = p.gdt != (std::is_same<MT, __half>::value ? MOE_F16 : MOE_BF16);
+    // gradients in the other 16-bit dtype are converted here unless a one-time copy was made
+    const bool convert = !p.preconv && p.gdt != (std::is_same<MT, __half>::value ? MOE_F16 : MOE_BF16);
     uint64_t *bready0 = bready;
     uint32_t it = 0;
     bool live = true;

@@ -206,7 +206,8 @@ __global__ void __launch_bounds__(tcb::kThreads, 1)
     constexpr uint32_t M = Dq<MT>::kMagic2;
     const int b0 = (rband >> 3) * 1024 + (rband & 7) * 128 + ((wcol ^ (rband & 7)) << 4);
     uint32_t act_bad = 0;  // a converted input outside F16's normal range
-    const bool convert = p.gdt != (std::is_same<MT, __half>::value ? MOE_F16 : MOE_BF16);
+    // gradients in the other 16-bit dtype are converted here unless a one-time copy was made
+    const bool convert = !p.preconv && p.gdt != (std::is_same<MT, __half>::value ? MOE_F16 : MOE_BF16);
     // group row of band i = (32 i) / group; groups here are 64, 128 or >= 256 (one per tile)
     const int gshift = p.group >= kBN ? 8 : (p.group == 128 ? 7 : 6);
     uint32_t it = 0;

@@ -27,6 +27,7 @@ struct ProjParams {
   float *partials;
   int32_t *counters;
   int kq;  // K splits
+  int preconv;  // x holds F16 copies of BF16 activations (act_dt stays the output dtype)
 #ifdef MOE_TEST_HOOKS
   int test_stall;  // test build only: see moe_test_arm_stall
 #endif
@@ -44,6 +45,7 @@ struct BwdParams {
   int group;
   uint16_t *out;  // [A, K]
   int32_t *status;
+  int preconv;  // grad holds F16 copies of BF16 gradients (gdt stays the output dtype)
 };
 
 // Row of x that batch row r reads: r itself, or gather[r] (an index outside

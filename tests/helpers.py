@@ -3,15 +3,18 @@ oracle runs on the same seeded inputs, and the tolerance checks.
 
 Tolerance (floating outputs and gradients): |got - oracle| <= 2e-2 *
 rms(oracle) per tensor.  An element beyond that bound passes only when its
-difference is one rounding flip that the arithmetic explains: the device
+difference is a rounding flip that the arithmetic explains: the device
 accumulates in FP32 (the oracle in double), so when the exact result lies
 within the FP32 error bound of a rounding midpoint of the storage format,
 the device may store the other neighbour of the exact value.  With 8
 significant bits, one such step at |v| > ~2.6 rms already exceeds 2e-2 rms.
 For each such element the oracle supplies the unrounded value v and an
 error bound b (from the magnitudes of the summed terms, computed by the
-oracle in the same pass): the element passes iff got is the storage-format
-neighbour of v on the far side of the oracle's RNE(v), and |v - midpoint| <= b.
+oracle in the same pass): the element passes iff got is the RNE image of a
+real within b of v (for a step bound: the neighbour of RNE(v) on v's side,
+with v within b of their midpoint).  End-to-end checks widen b by the
+measured difference between the exact values on the device's upstream
+tensors and on the oracle's.
 Every check records its max err/rms and the count of such flips (printed in
 the pytest summary).  Integer and index outputs, and the rounded
 coefficients, must match bit for bit; FP32 routing weights within 2e-6.
@@ -67,15 +70,22 @@ def _from_ordered(o: np.ndarray) -> np.ndarray:
     return np.where(o < 0, (-o) | 0x8000, o).astype(np.uint16)
 
 
-def flip_justified(got_b, want_b, exact, bound, dt="bf16"):
-    """Element-wise: got is the storage neighbour of `exact` on the far side of
-    want = RNE(exact), and exact lies within `bound` of their midpoint."""
-    ow = _ordered(want_b)
-    w = as_f64(want_b, dt)
-    step = np.sign(exact - w).astype(np.int64)
-    other = _from_ordered(ow + step)
-    mid = 0.5 * (w + as_f64(other, dt))
-    return (step != 0) & (_ordered(got_b) == ow + step) & (np.abs(exact - mid) <= bound)
+def rounding_justified(got_b, exact, bound, dt="bf16"):
+    """Element-wise: got is the round-to-nearest-even image of some real within
+    `bound` of `exact`, i.e. the distance from `exact` to the interval of reals
+    that round to got (between got's midpoints with its two storage
+    neighbours) is at most `bound`.  With an FP32-accumulation bound this
+    admits exactly the rounding flips that bound explains (got is RNE(exact)'s
+    neighbour on the side of `exact` and `exact` lies within `bound` of their
+    midpoint); with an end-to-end bound widened by measured upstream
+    differences it admits what those differences explain, and no more."""
+    og = _ordered(got_b)
+    g = as_f64(got_b, dt)
+    with np.errstate(over="ignore", invalid="ignore"):
+        lo = 0.5 * (g + as_f64(_from_ordered(og - 1), dt))
+        hi = 0.5 * (g + as_f64(_from_ordered(og + 1), dt))
+    dist = np.maximum(0.0, np.maximum(lo - exact, exact - hi))
+    return dist <= bound
 
 
 def check_close(got, want, name, dt="bf16", tol=TOL, justify=None):
@@ -100,7 +110,7 @@ def check_close(got, want, name, dt="bf16", tol=TOL, justify=None):
         shape2 = got.shape if got.ndim == 2 else (1, got.size)
         rows, cols = np.unravel_index(over, shape2)
         exact, bound = justify(rows, cols)
-        ok = flip_justified(got.reshape(-1)[over], want.reshape(-1)[over], exact, bound, dt)
+        ok = rounding_justified(got.reshape(-1)[over], exact, bound, dt)
         if not np.all(ok):
             i = int(np.nonzero(~ok)[0][0])
             raise AssertionError(msg + "; not a justified rounding flip at [%d, %d]: got %.6g, oracle %.6g, exact "

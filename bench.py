@@ -154,6 +154,7 @@ def main():
     ap.add_argument("--reference-tokens", type=int, default=8)
     ap.add_argument("--workloads", default="prefill,wide,skewed,nf4",
                     help="other workloads timed in the same run, reported under 'workloads' ('none': skip)")
+    ap.add_argument("--no-gather", action="store_true", help="skip the gather-mode step (profiling runs)")
     ap.add_argument("--tokens", type=int, default=0,
                     help="override the workload's token count (smaller profiling captures); 0 keeps it")
     args = ap.parse_args()
@@ -381,7 +382,7 @@ def measure(w, args, steps, world, rank, local, cpu):
     # the gather mode of the dispatch (no COPY: the gate/up projection reads
     # x rows through src_token), same protocol, forward-only workloads
     gather_ms = None
-    if not w.backward:
+    if not w.backward and not args.no_gather:
         def step_gather():
             ffn.forward(dev, buf, gather=True)
 
@@ -433,7 +434,7 @@ def measure(w, args, steps, world, rank, local, cpu):
     clocks = sampler.stop()
     status = int(buf.status.item())
 
-    vals = [ms, e2e_ms, kernel_ms] + ([fwd_ms, bwd_ms] if w.backward else [gather_ms])
+    vals = [ms, e2e_ms, kernel_ms] + ([fwd_ms, bwd_ms] if w.backward else [gather_ms or 0.0])
     vals = max_over_ranks(vals, "cuda")
     ms, e2e_ms, kernel_ms = vals[:3]
     if w.backward:
@@ -490,7 +491,7 @@ def measure(w, args, steps, world, rank, local, cpu):
     if w.backward:
         line["fwd_ms"] = fwd_ms
         line["bwd_ms"] = bwd_ms
-    else:
+    elif gather_ms:
         line["gather_mode"] = {"ms_per_step": gather_ms, "value": world * w.T / (gather_ms * 1e-3),
                                "unit": "tokens/s", "tflops": fwd_flops / (gather_ms * 1e-3) / 1e12,
                                "step": "moe_route -> awq_grouped_gate_up_swiglu_gather -> down -> combine"}

@@ -51,6 +51,8 @@ constexpr int kAtom = kBM * 64 * 2;          // 16 KB: 128 rows x 64 K (128B swi
 constexpr int kABytes = kBM * kBK * 2;        // 32 KB
 constexpr int kPBytes = kBK * (kHalf / 8) * 4;  // 8 KB packed words
 constexpr int kLBytes = kABytes + kPBytes;    // one TMA stage
+constexpr int kZBytes = 64;                   // zero-point words of the step's group row (16 words)
+constexpr int kZSBytes = 384;                 // + its 128 scales (256 bytes), 128-byte slots
 constexpr int kBBytes = kHalf * kBK * 2;      // 32 KB coefficient half-tile
 constexpr int kNBlock = kBK * 128;            // bytes between 64-column blocks of B (MN-major)
 constexpr int kTmemCols = 512;
@@ -65,14 +67,17 @@ struct PairTile {
 template <typename MT, int NPROJ>
 __global__ void __launch_bounds__(tc2::kThreads, 1)
     awq_fwd_tc2_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_w0,
-                       const __grid_constant__ CUtensorMap map_w1, ProjParams p) {
+                       const __grid_constant__ CUtensorMap map_w1, const __grid_constant__ CUtensorMap map_z0,
+                       const __grid_constant__ CUtensorMap map_z1, const __grid_constant__ CUtensorMap map_s0,
+                       const __grid_constant__ CUtensorMap map_s1, ProjParams p) {
   pdl_enter();  // programmatic dependent launch: the previous kernel is done
   using namespace tc2;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t *smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
   uint8_t *lring = smem;
   uint8_t *bring = smem + kLStages * kLBytes;
-  uint64_t *lfull = reinterpret_cast<uint64_t *>(bring + kBStages * kBBytes);
+  uint8_t *zring = bring + kBStages * kBBytes;  // kLStages x [zero words | scales] of the step's group row
+  uint64_t *lfull = reinterpret_cast<uint64_t *>(zring + kLStages * kZSBytes);
   uint64_t *lempty = lfull + kLStages;
   uint64_t *bready = lempty + kLStages;  // used in CTA 0 (both CTAs' dequant warps)
   uint64_t *bfree = bready + kBStages;
@@ -90,7 +95,7 @@ __global__ void __launch_bounds__(tc2::kThreads, 1)
   const uint32_t rank = cluster_rank();
   const int64_t pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
   const int E = p.E;
-  const int64_t K = p.K, NW = p.N / 8;
+  const int64_t K = p.K;
   const int feat_tile = NPROJ == 2 ? kHalf : kBN;
   const int NT = (int)((p.N + feat_tile - 1) / feat_tile);
   const int nk = (int)(K / kBK);
@@ -158,6 +163,9 @@ __global__ void __launch_bounds__(tc2::kThreads, 1)
     const bool gather = p.gather != nullptr;
     if (gather || lane == 0) {
       const CUtensorMap *mw = (NPROJ == 2 && rank == 1) ? &map_w1 : &map_w0;
+      const CUtensorMap *mz = (NPROJ == 2 && rank == 1) ? &map_z1 : &map_z0;
+      const CUtensorMap *ms = (NPROJ == 2 && rank == 1) ? &map_s1 : &map_s0;
+      const int64_t ngroups = K / p.group;
       uint32_t it = 0;  // stages issued
       bool live = true;
       for (int64_t tile = pair; tile < total && live; tile += npairs) {
@@ -175,7 +183,7 @@ __global__ void __launch_bounds__(tc2::kThreads, 1)
           uint8_t *st = lring + s * kLBytes;
           if (lane == 0) {
             ok = use == 0 || tc_wait(&lempty[s], (use - 1) & 1, p.status, abort);
-            if (ok) mbar_arrive_expect_tx(&lfull[s], kLBytes);
+            if (ok) mbar_arrive_expect_tx(&lfull[s], kLBytes + kZBytes + 256);
           }
           if (gather) ok = __shfl_sync(0xffffffffu, ok, 0);
           if (!ok) {
@@ -193,6 +201,11 @@ __global__ void __launch_bounds__(tc2::kThreads, 1)
               tma_load_2d(st + kAtom, &map_x, &lfull[s], kb * kBK + 64, row0);
             }
             tma_load_2d(st + kABytes, mw, &lfull[s], wcol, (int32_t)(ti.e * K + (int64_t)kb * kBK));
+            // the group row of this step's zero points and scales (this CTA's columns)
+            const int32_t grow = (int32_t)(ti.e * ngroups + (int64_t)kb * kBK / p.group);
+            uint8_t *zs = zring + s * kZSBytes;
+            tma_load_2d(zs, mz, &lfull[s], wcol, grow);
+            tma_load_2d(zs + 128, ms, &lfull[s], wcol * 8, grow);
           }
         }
       }
@@ -240,11 +253,7 @@ __global__ void __launch_bounds__(tc2::kThreads, 1)
     const int td = threadIdx.x - 64;  // 0 .. 32 kDqWarps - 1
     const int col = td & 15;          // word column within the half
     const int rg = td >> 4;           // rows rg, rg + kRowGroups, ... of each step
-    const int proj = NPROJ == 2 ? (int)rank : 0;
     constexpr uint32_t M = Dq<MT>::kMagic2;
-    const int64_t ngroups = K / p.group;
-    const int32_t *qz = p.qz[proj];
-    const uint16_t *sc = p.sc[proj];
     const int pk0 = rg * 16 + col;
     // features col*8 .. col*8+7 of the half -> 64-column block col/8, 16-byte
     // chunk col%8 XOR row%8 (MN-major, 128-byte swizzle, 8-row x 64-column atoms)
@@ -256,61 +265,28 @@ __global__ void __launch_bounds__(tc2::kThreads, 1)
     uint64_t *bready0 = bready;  // CTA 0's barriers, addressed through the cluster window
     uint32_t it = 0;
     bool live = true;
-    // zeros/scales of a tile's word column; the first group of the next tile
-    // is requested during the last group of the current one
-    struct ZsPtr {
-      const int32_t *qz;
-      const uint16_t *sc;
-      bool ok;
-    };
-    auto zs_ptr = [&](int64_t tile) {
-      const PairTile tn = tile_info(tile);
-      const int64_t wc = NPROJ == 2 ? (int64_t)tn.nt * 16 + col : (int64_t)tn.nt * 32 + 16 * rank + col;
-      const bool ok = wc < NW;
-      const int64_t wcs = ok ? wc : 0;
-      return ZsPtr{qz + (int64_t)tn.e * ngroups * NW + wcs, sc + (int64_t)tn.e * ngroups * p.N + 8 * wcs, ok};
-    };
-    uint32_t pf_zw = 0u;
-    uint4 pf_sv = make_uint4(0, 0, 0, 0);
-    ZsPtr cur = zs_ptr(pair < total ? pair : 0);
-    if (pair < total && cur.ok) {
-      pf_zw = (uint32_t)__ldg(cur.qz);
-      pf_sv = __ldg(reinterpret_cast<const uint4 *>(cur.sc));
-    }
     for (int64_t tile = pair; tile < total && live; tile += npairs) {
-      const ZsPtr zs = cur;
       uint32_t zp[4], sp[4];
-      int64_t grp = 0;
       int gstage = 0;
       for (int kb = 0; kb < nk; ++kb, ++it) {
         const uint32_t ls = it % kLStages, bs = it % kBStages, buse = it / kBStages;
-        if (gstage == 0) {
-          const uint32_t s4[4] = {pf_sv.x, pf_sv.y, pf_sv.z, pf_sv.w};
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            zp[q] = nib_pair<M>(pf_zw >> (4 * q));
-            sp[q] = s4[q];
-          }
-          if (grp + 1 < ngroups) {
-            if (zs.ok) {
-              pf_zw = (uint32_t)__ldg(zs.qz + (grp + 1) * NW);
-              pf_sv = __ldg(reinterpret_cast<const uint4 *>(zs.sc + (grp + 1) * p.N));
-            }
-          } else if (tile + npairs < total) {
-            cur = zs_ptr(tile + npairs);
-            pf_zw = cur.ok ? (uint32_t)__ldg(cur.qz) : 0u;
-            pf_sv = cur.ok ? __ldg(reinterpret_cast<const uint4 *>(cur.sc)) : make_uint4(0, 0, 0, 0);
-          }
-        }
-        if (++gstage == spg) {
-          gstage = 0;
-          ++grp;
-        }
         if (!tc_wait(&lfull[ls], (it / kLStages) & 1, p.status, abort)) {
           live = false;
           break;
         }
         uint8_t *st = lring + ls * kLBytes;
+        if (gstage == 0) {  // a new group: its zero/scale row came with this stage
+          const uint8_t *zs = zring + ls * kZSBytes;
+          const uint32_t zw = reinterpret_cast<const uint32_t *>(zs)[col];
+          const uint4 sv = reinterpret_cast<const uint4 *>(zs + 128)[col];
+          const uint32_t s4[4] = {sv.x, sv.y, sv.z, sv.w};
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            zp[q] = nib_pair<M>(zw >> (4 * q));
+            sp[q] = s4[q];
+          }
+        }
+        if (++gstage == spg) gstage = 0;
         uint32_t w[kWordsPerThread];
         {
           const uint32_t *pk = reinterpret_cast<const uint32_t *>(st + kABytes) + pk0;
@@ -447,8 +423,8 @@ __global__ void __launch_bounds__(tc2::kThreads, 1)
 // ------------------------------------------------------------------ launch
 
 static size_t tc2_smem(int64_t E) {
-  return 1024 + (size_t)tc2::kLStages * tc2::kLBytes + (size_t)tc2::kBStages * tc2::kBBytes + 256 +
-         (size_t)2 * tc2::kBN * 4 + (size_t)(2 * E + 1 + 32) * 4;
+  return 1024 + (size_t)tc2::kLStages * tc2::kLBytes + (size_t)tc2::kBStages * tc2::kBBytes +
+         (size_t)tc2::kLStages * tc2::kZSBytes + 256 + (size_t)2 * tc2::kBN * 4 + (size_t)(2 * E + 1 + 32) * 4;
 }
 
 bool tc2_fits(const ProjParams &p) {
@@ -465,9 +441,18 @@ static moe_status launch_tc2_t(const ProjParams &p, cudaStream_t st) {
                                             CU_TENSOR_MAP_SWIZZLE_128B)
                               : make_map_2d(&mx, p.x, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, p.K, p.A, 64, kBM,
                                             CU_TENSOR_MAP_SWIZZLE_128B);
+  // zero-point words and scales: one group row per step, this CTA's 16 word columns
+  CUtensorMap z0, z1, s0, s1;
+  const uint64_t grows = (uint64_t)p.E * (p.K / p.group);
   if (!mx_ok ||
       !make_map_2d(&m0, p.qw[0], CU_TENSOR_MAP_DATA_TYPE_INT32, 4, NW, rows, 16, kBK, CU_TENSOR_MAP_SWIZZLE_NONE) ||
       !make_map_2d(&m1, p.qw[NPROJ - 1], CU_TENSOR_MAP_DATA_TYPE_INT32, 4, NW, rows, 16, kBK,
+                   CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !make_map_2d(&z0, p.qz[0], CU_TENSOR_MAP_DATA_TYPE_INT32, 4, NW, grows, 16, 1, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !make_map_2d(&z1, p.qz[NPROJ - 1], CU_TENSOR_MAP_DATA_TYPE_INT32, 4, NW, grows, 16, 1,
+                   CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !make_map_2d(&s0, p.sc[0], CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, p.N, grows, 128, 1, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !make_map_2d(&s1, p.sc[NPROJ - 1], CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, p.N, grows, 128, 1,
                    CU_TENSOR_MAP_SWIZZLE_NONE))
     return set_error(MOE_ERR_CUDA, "tensor map encoding failed (tcgen05 pair projection)");
   const size_t smem = tc2_smem(p.E);
@@ -494,7 +479,7 @@ static moe_status launch_tc2_t(const ProjParams &p, cudaStream_t st) {
   }
   cfg.gridDim = dim3(2 * clusters);  // persistent: every pair resident at once
   cfg.numAttrs = 2;
-  cudaLaunchKernelEx(&cfg, kern, mx, m0, m1, p);
+  cudaLaunchKernelEx(&cfg, kern, mx, m0, m1, z0, z1, s0, s1, p);
   return check_launch("awq_fwd_tc2_kernel");
 }
 

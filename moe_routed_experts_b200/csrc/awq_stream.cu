@@ -17,11 +17,13 @@
 // stages of all items, expert-major, form one list that the persistent CTAs
 // (8 warps; 2 per SM) split into equal contiguous ranges (stream-K), so
 // every CTA streams the same number of weight bytes whatever the routing.
-//   copies (lane 0 of warp 0): per stage two TMA boxes of [ROWS rows][32
-//     words] with 128-byte swizzle into a ring (64 KB in flight for 128-row
-//     stages), each issued once every warp released the ring slot's
-//     previous stage; per 512 input rows of an item, 1-D bulk copies of the
-//     item's activation rows (double-buffered, one chunk ahead).
+//   copies: per stage two TMA boxes of [ROWS rows][32 words] with 128-byte
+//     swizzle into a ring (64 KB in flight for 128-row stages), each issued
+//     once every warp released the ring slot's previous stage, by lane 0 of
+//     the warps in turn (stage r by warp r mod 8, so no warp carries all the
+//     issue work); per 512 input rows of an item, 1-D bulk copies of the
+//     item's activation rows (lane 0 of warp 0; double-buffered, one chunk
+//     ahead).
 //   warp w: box w/4, word columns (w%4)*8 .. +7 of it, all rows of the
 //     stage.  Lane (g, t) reads rows t, t+4, t+8, t+12 of column g (the
 //     MMA's K index {2t, 2t+1, 2t+8, 2t+9} stands for them); the swizzle
@@ -183,6 +185,7 @@ __global__ void __launch_bounds__(stream::kThreads, 2)
   int32_t *pre = reinterpret_cast<int32_t *>(red + 8 * NT * kF);    // [E + 1]
   int32_t *cnt = pre + (E + 1);                                    // [E]
   int32_t *tmp = cnt + E;                                          // [32]
+  int32_t *issued_hi = tmp + 32;                                   // [1]: stages issued (relative), max
   volatile int32_t *abort = reinterpret_cast<volatile int32_t *>(xempty + 2);
 #ifdef MOE_TEST_HOOKS
   uint64_t *stall = xempty + 3;  // test build only: a barrier nothing arrives on
@@ -286,7 +289,25 @@ __global__ void __launch_bounds__(stream::kThreads, 2)
   if (issuer && g0 < g1) {
     load_x(g0, 0);
     issue_upto(g0 + kStages - 1);
+    *issued_hi = (int32_t)(nxt - g0);
   }
+  // Stages past the first kStages rotate over the warps: stage g0 + r (r >=
+  // kStages) is issued by lane 0 of warp r % kCW at the top of iteration
+  // g0 + r - kStages + 1, once every warp released the slot's previous
+  // stage, so no single warp carries the issue work.
+  bool rlive = true;
+  auto issue_rotating = [&](int64_t j) {
+    const int64_t st = j + kStages - 1;  // the stage due now
+    const int64_t r = st - g0;
+    if (r < kStages || st >= g1 || !rlive || lane != 0 || (int)(r % kCW) != warp) return;
+    const uint32_t s = (uint32_t)(r % kStages), use = (uint32_t)(r / kStages);
+    if (!tc_wait(&empty[s], (use - 1) & 1, p.status, abort)) {
+      rlive = false;
+      return;
+    }
+    issue_stage(st);
+    atomicMax(issued_hi, (int32_t)(r + 1));
+  };
 
   // ---------------- consumers
   uint32_t act_bad = 0;  // a converted input outside F16's normal range
@@ -406,7 +427,7 @@ __global__ void __launch_bounds__(stream::kThreads, 2)
       gstage = 0;
       ++grp;
     }
-    if (issuer) issue_upto(j + kStages - 1);
+    issue_rotating(j);
     // warp-uniform: the MMAs below are warp-wide
     const bool sok = __all_sync(0xffffffffu, tc_wait(&full[s], ph, p.status, abort));
     if (sok) {
@@ -519,8 +540,11 @@ __global__ void __launch_bounds__(stream::kThreads, 2)
     }
     named_barrier(1, kCW * 32);  // red is free again
   }
-  if (issuer) {  // nothing asynchronous may be in flight at exit (abort protocol)
-    tma_drain(full, (uint32_t)(nxt - g0), kStages, p.status);
+  // nothing asynchronous may be in flight at exit (abort protocol): every
+  // warp's issues are done once all warps left the loop
+  named_barrier(1, kCW * 32);
+  if (issuer) {
+    tma_drain(full, (uint32_t)*(volatile int32_t *)issued_hi, kStages, p.status);
     tma_drain(xfull, xissued, 2, p.status);
   }
   if (act_bad) report(p.status, MOE_DEVICE_ERR_ACT_RANGE);
@@ -595,7 +619,7 @@ static size_t stream_smem(int nt, int64_t E, int rows) {
                      : rows == 64 ? (size_t)Geo<64>::kStages * Geo<64>::kStageBytes
                                   : (size_t)Geo<32>::kStages * Geo<32>::kStageBytes;
   return 1024 /* alignment slack */ + kBarBytes + ring + 2 * (size_t)8 * nt * 512 * 2 +
-         (size_t)8 * nt * (512 * 2 + 16) + (size_t)8 * nt * kF * 4 + (size_t)(2 * E + 1 + 32) * 4;
+         (size_t)8 * nt * (512 * 2 + 16) + (size_t)8 * nt * kF * 4 + (size_t)(2 * E + 1 + 32 + 4) * 4;
 }
 
 // Workspace: the parts of split items (at most sk_max_parts per item) and

@@ -48,9 +48,6 @@ constexpr int kABytes = kBM * kBK * 2;          // 16 KB activation tile
 constexpr int kBBytes = kBN * kBK * 2;          // 32 KB coefficient tile
 constexpr int kPBytes = kBK * (kBN / 8) * 4;    // 8 KB packed words
 constexpr int kLBytes = kABytes + kPBytes;    // one TMA stage (24 KB: 1 KB aligned)
-// the step's group row: zero-point words at 0 (gate | up at 128 for the pair),
-// scales at 256 (gate | up at 512); every TMA destination 128-byte aligned
-constexpr int kZSBytes = 768;
 constexpr int kTmemCols = 512;  // two 128 x 256 FP32 accumulators
 }  // namespace tc
 
@@ -65,17 +62,14 @@ struct TileInfo {
 template <typename MT, int NPROJ>
 __global__ void __launch_bounds__(tc::kThreads, 1)
     awq_fwd_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_w0,
-                      const __grid_constant__ CUtensorMap map_w1, const __grid_constant__ CUtensorMap map_z0,
-                      const __grid_constant__ CUtensorMap map_z1, const __grid_constant__ CUtensorMap map_s0,
-                      const __grid_constant__ CUtensorMap map_s1, ProjParams p) {
+                      const __grid_constant__ CUtensorMap map_w1, ProjParams p) {
   pdl_enter();  // programmatic dependent launch: the previous kernel is done
   using namespace tc;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t *smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
   uint8_t *lring = smem;                           // kLStages x [A | packed]
   uint8_t *bring = smem + kLStages * kLBytes;      // kBStages x B
-  uint8_t *zring = bring + kBStages * kBBytes;     // kLStages x [zero words | scales] of the step's group row
-  uint64_t *full = reinterpret_cast<uint64_t *>(zring + kLStages * kZSBytes);
+  uint64_t *full = reinterpret_cast<uint64_t *>(bring + kBStages * kBBytes);
   uint64_t *empty = full + kLStages;               // MMA commit (A read) + dequant warps (words read)
   uint64_t *bready = empty + kLStages;
   uint64_t *bfree = bready + kBStages;
@@ -91,7 +85,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int E = p.E;
-  const int64_t K = p.K;
+  const int64_t K = p.K, NW = p.N / 8;
   const int feat_tile = NPROJ == 2 ? kBN / 2 : kBN;          // output features per tile
   const int NT = (int)((p.N + feat_tile - 1) / feat_tile);  // column tiles per row tile
   const int nk = (int)(K / kBK);
@@ -173,7 +167,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
           uint8_t *st = lring + s * kLBytes;
           if (lane == 0) {
             ok = use == 0 || tc_wait(&empty[s], (use - 1) & 1, p.status, abort);
-            if (ok) mbar_arrive_expect_tx(&full[s], kLBytes + 640);  // + 128 zero-point and 512 scale bytes
+            if (ok) mbar_arrive_expect_tx(&full[s], kLBytes);
           }
           if (gather) ok = __shfl_sync(0xffffffffu, ok, 0);
           if (!ok) {
@@ -184,20 +178,11 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
           if (lane == 0) {
             if (!gather) tma_load_2d(st, &map_x, &full[s], kb * kBK, row0);
             const int32_t wrow = (int32_t)(ti.e * K + (int64_t)kb * kBK);
-            // the group row of this step's zero points and scales
-            const int32_t grow = (int32_t)(ti.e * (K / p.group) + (int64_t)kb * kBK / p.group);
-            uint8_t *zs = zring + s * kZSBytes;
             if (NPROJ == 2) {
               tma_load_2d(st + kABytes, &map_w0, &full[s], ti.nt * 16, wrow);
               tma_load_2d(st + kABytes + kPBytes / 2, &map_w1, &full[s], ti.nt * 16, wrow);
-              tma_load_2d(zs, &map_z0, &full[s], ti.nt * 16, grow);
-              tma_load_2d(zs + 128, &map_z1, &full[s], ti.nt * 16, grow);
-              tma_load_2d(zs + 256, &map_s0, &full[s], ti.nt * 128, grow);
-              tma_load_2d(zs + 512, &map_s1, &full[s], ti.nt * 128, grow);
             } else {
               tma_load_2d(st + kABytes, &map_w0, &full[s], ti.nt * 32, wrow);
-              tma_load_2d(zs, &map_z0, &full[s], ti.nt * 32, grow);
-              tma_load_2d(zs + 256, &map_s0, &full[s], ti.nt * 256, grow);
             }
           }
         }
@@ -251,6 +236,9 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
     // neighbouring row so gate and up words sit in different banks
     const int rg = (td >> 5) ^ jw;
     constexpr uint32_t M = Dq<MT>::kMagic2;
+    const int64_t ngroups = K / p.group;
+    const int32_t *qz = p.qz[jw];
+    const uint16_t *sc = p.sc[jw];
     const int pk0 = NPROJ == 2 ? jw * (kBK * 16) + rg * 16 + (col & 15) : rg * 32 + col;
     constexpr int pk_step = NPROJ == 2 ? 8 * 16 : 8 * 32;  // words between rows r and r + 8
     // B: features col*8 .. col*8+7 -> 64-column block col/8, 16-byte chunk col%8 XOR row%8
@@ -261,29 +249,59 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
     const bool convert = !p.preconv && p.act_dt != (std::is_same<MT, __half>::value ? MOE_F16 : MOE_BF16);
     uint32_t it = 0;
     bool live = true;
+    // zeros/scales of a tile's word column; the first group of the next tile
+    // is requested during the last group of the current one
+    struct ZsPtr {
+      const int32_t *qz;
+      const uint16_t *sc;
+      bool ok;
+    };
+    auto zs_ptr = [&](int64_t tile) {
+      const TileInfo tn = tile_info(tile);
+      const int64_t wc = NPROJ == 2 ? (int64_t)tn.nt * 16 + (col & 15) : (int64_t)tn.nt * 32 + col;
+      const bool ok = wc < NW;
+      const int64_t wcs = ok ? wc : 0;
+      return ZsPtr{qz + (int64_t)tn.e * ngroups * NW + wcs, sc + (int64_t)tn.e * ngroups * p.N + 8 * wcs, ok};
+    };
+    ZsPtr cur = zs_ptr((int64_t)blockIdx.x < total ? (int64_t)blockIdx.x : 0);
+    uint32_t pf_zw = ((int64_t)blockIdx.x < total && cur.ok) ? (uint32_t)__ldg(cur.qz) : 0u;
+    uint4 pf_sv = ((int64_t)blockIdx.x < total && cur.ok) ? __ldg(reinterpret_cast<const uint4 *>(cur.sc))
+                                                           : make_uint4(0, 0, 0, 0);
     for (int64_t tile = blockIdx.x; tile < total && live; tile += gridDim.x) {
+      const ZsPtr zs = cur;
       uint32_t zp[4], sp[4];
+      int64_t grp = 0;
       int gstage = 0;
       for (int kb = 0; kb < nk; ++kb, ++it) {
         const uint32_t s = it % kLStages, ph = (it / kLStages) & 1;
         const uint32_t b = it % kBStages, buse = it / kBStages;
+        if (gstage == 0) {  // a new group: take the prefetched zeros/scales, prefetch the next
+          const uint32_t s4[4] = {pf_sv.x, pf_sv.y, pf_sv.z, pf_sv.w};
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            zp[q] = nib_pair<M>(pf_zw >> (4 * q));
+            sp[q] = s4[q];
+          }
+          if (grp + 1 < ngroups) {
+            if (zs.ok) {
+              pf_zw = (uint32_t)__ldg(zs.qz + (grp + 1) * NW);
+              pf_sv = __ldg(reinterpret_cast<const uint4 *>(zs.sc + (grp + 1) * p.N));
+            }
+          } else if (tile + gridDim.x < total) {
+            cur = zs_ptr(tile + gridDim.x);
+            pf_zw = cur.ok ? (uint32_t)__ldg(cur.qz) : 0u;
+            pf_sv = cur.ok ? __ldg(reinterpret_cast<const uint4 *>(cur.sc)) : make_uint4(0, 0, 0, 0);
+          }
+        }
+        if (++gstage == spg) {
+          gstage = 0;
+          ++grp;
+        }
         if (!tc_wait(&full[s], ph, p.status, abort)) {
           live = false;
           break;
         }
         uint8_t *st = lring + s * kLBytes;
-        if (gstage == 0) {  // a new group: its zero/scale row came with this stage
-          const uint8_t *zs = zring + s * kZSBytes;
-          const uint32_t zw = reinterpret_cast<const uint32_t *>(zs)[NPROJ == 2 ? (col & 15) + 32 * (col >> 4) : col];
-          const uint4 sv = reinterpret_cast<const uint4 *>(zs + 256)[col];
-          const uint32_t s4[4] = {sv.x, sv.y, sv.z, sv.w};
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            zp[q] = nib_pair<M>(zw >> (4 * q));
-            sp[q] = s4[q];
-          }
-        }
-        if (++gstage == spg) gstage = 0;
         if (convert) {
           // activation tile to the scale dtype, in place (layout-agnostic)
           uint4 *a4 = reinterpret_cast<uint4 *>(st);
@@ -416,8 +434,8 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
 // ------------------------------------------------------------------ launch
 
 static size_t tc_smem(int64_t E) {
-  return 1024 + (size_t)tc::kLStages * tc::kLBytes + (size_t)tc::kBStages * tc::kBBytes +
-         (size_t)tc::kLStages * tc::kZSBytes + 256 + (size_t)2 * tc::kBN * 4 + (size_t)(2 * E + 1 + 32) * 4;
+  return 1024 + (size_t)tc::kLStages * tc::kLBytes + (size_t)tc::kBStages * tc::kBBytes + 256 +
+         (size_t)2 * tc::kBN * 4 + (size_t)(2 * E + 1 + 32) * 4;
 }
 
 // The tile needs whole 64-row steps inside one group, 16-byte word-row
@@ -439,25 +457,15 @@ static moe_status launch_tc_t(const ProjParams &p, cudaStream_t st) {
                                             CU_TENSOR_MAP_SWIZZLE_128B)
                               : make_map_2d(&mx, p.x, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, p.K, p.A, kBK, kBM,
                                             CU_TENSOR_MAP_SWIZZLE_128B);
-  // zero-point words and scales: one group row per step, the tile's word columns
-  CUtensorMap z0, z1, s0, s1;
-  const uint64_t grows = (uint64_t)p.E * (p.K / p.group);
   if (!mx_ok ||
       !make_map_2d(&m0, p.qw[0], CU_TENSOR_MAP_DATA_TYPE_INT32, 4, NW, rows, box_w, kBK, CU_TENSOR_MAP_SWIZZLE_NONE) ||
       !make_map_2d(&m1, p.qw[NPROJ - 1], CU_TENSOR_MAP_DATA_TYPE_INT32, 4, NW, rows, box_w, kBK,
-                   CU_TENSOR_MAP_SWIZZLE_NONE) ||
-      !make_map_2d(&z0, p.qz[0], CU_TENSOR_MAP_DATA_TYPE_INT32, 4, NW, grows, box_w, 1, CU_TENSOR_MAP_SWIZZLE_NONE) ||
-      !make_map_2d(&z1, p.qz[NPROJ - 1], CU_TENSOR_MAP_DATA_TYPE_INT32, 4, NW, grows, box_w, 1,
-                   CU_TENSOR_MAP_SWIZZLE_NONE) ||
-      !make_map_2d(&s0, p.sc[0], CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, p.N, grows, 8 * box_w, 1,
-                   CU_TENSOR_MAP_SWIZZLE_NONE) ||
-      !make_map_2d(&s1, p.sc[NPROJ - 1], CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, p.N, grows, 8 * box_w, 1,
                    CU_TENSOR_MAP_SWIZZLE_NONE))
     return set_error(MOE_ERR_CUDA, "tensor map encoding failed (tcgen05 projection)");
   const size_t smem = tc_smem(p.E);
   auto kern = awq_fwd_tc_kernel<MT, NPROJ>;
   cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  launch_pdl(kern, dim3(num_sms()), dim3(kThreads), smem, st, mx, m0, m1, z0, z1, s0, s1, p);
+  launch_pdl(kern, dim3(num_sms()), dim3(kThreads), smem, st, mx, m0, m1, p);
   return check_launch("awq_fwd_tc_kernel");
 }
 

@@ -322,9 +322,8 @@ __global__ void __launch_bounds__(stream::kThreads, 2)
   const int woff0 = box_offset(t, cgw * 8 + g), woff1 = box_offset(t + 4, cgw * 8 + g);
   const int spg = p.group / kRows;  // stages per group (group % kRows == 0 on this path)
 
-  float acc[NT][4][4], acc16[NT][2][4];
+  float acc[NT][4][4];
   FwdConsts<MT> cst;
-  bool x16 = false;
   ItemInfo ii{};
   int tok0 = 0, mrows = 0, seg_c0 = 0, seg_c1 = 0, xbase = 0, gstage = 0;
   int64_t wc = 0, grp = 0;
@@ -358,10 +357,6 @@ __global__ void __launch_bounds__(stream::kThreads, 2)
         for (int q = 0; q < 4; ++q)
 #pragma unroll
           for (int k = 0; k < 4; ++k) acc[nt][q][k] = 0.f;
-#pragma unroll
-        for (int q = 0; q < 2; ++q)
-#pragma unroll
-          for (int k = 0; k < 4; ++k) acc16[nt][q][k] = 0.f;
       }
     }
     if (j == g0 || c % kXst == 0) {
@@ -402,22 +397,7 @@ __global__ void __launch_bounds__(stream::kThreads, 2)
     }
     const uint32_t s = (uint32_t)((j - g0) % kStages), ph = (uint32_t)(((j - g0) / kStages) & 1);
     if (gstage == 0 || j == g0 || c == seg_c0) {  // a stage lies inside one group
-      if (std::is_same<MT, __half>::value) {
-        // 16 RNE((q - z) s) = RNE(16 (q - z) s) needs every nonzero product
-        // normal before and after the scaling: 0 or 2^-14 <= |s| <= 256 for
-        // all 8 scales of this column group
-        // all 8 scales of this column group (zero scales take the plain path)
-        const uint32_t m0 = pf_sv.x & 0x7FFF7FFFu, m1 = pf_sv.y & 0x7FFF7FFFu, m2 = pf_sv.z & 0x7FFF7FFFu,
-                       m3 = pf_sv.w & 0x7FFF7FFFu;
-        uint32_t mx = umax16x2(umax16x2(m0, m1), umax16x2(m2, m3));
-        uint32_t mn = umin16x2(umin16x2(m0, m1), umin16x2(m2, m3));
-        mx = umax16x2(mx, mx >> 16) & 0xFFFFu;
-        mn = umin16x2(mn, mn >> 16) & 0xFFFFu;  // the high lane of mn >> 16 is 0: only the low lane is read
-        // one decision per warp: the MMAs below are warp-wide (mma.sync), so
-        // every lane must take the same branch; a lane without a column votes yes
-        x16 = __all_sync(0xffffffffu, !wc_ok || (mx <= 0x5C00u && mn >= 0x0400u));
-      }
-      load_consts_fast<MT>(cst, pf_zw, pf_sv, x16);
+      load_consts_fast<MT>(cst, pf_zw, pf_sv);
       if (wc_ok && (grp + 1) * p.group < K) {  // prefetch the next group
         pf_zw = (uint32_t)__ldg(qzp + (grp + 1) * NW);
         pf_sv = __ldg(reinterpret_cast<const uint4 *>(scp + (grp + 1) * p.N));
@@ -453,34 +433,14 @@ __global__ void __launch_bounds__(stream::kThreads, 2)
             b1[h][nt] = bv.y;
           }
         }
-        bool done = false;
-        if constexpr (std::is_same<MT, __half>::value) {
-          if (x16) {
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              uint32_t af[4][4];
-              fwd_step<MT, true>(w[h][0], w[h][1], w[h][2], w[h][3], cst, af);
+        for (int h = 0; h < 2; ++h) {
+          uint32_t af[4][4];
+          fwd_step<MT>(w[h][0], w[h][1], w[h][2], w[h][3], cst, af);
 #pragma unroll
-              for (int q = 0; q < 4; ++q)
+          for (int q = 0; q < 4; ++q)
 #pragma unroll
-                for (int nt = 0; nt < NT; ++nt) {
-                  if (q & 1) mma16816<MT>(acc16[nt][q >> 1], af[q], b0[h][nt], b1[h][nt]);
-                  else mma16816<MT>(acc[nt][q], af[q], b0[h][nt], b1[h][nt]);
-                }
-            }
-            done = true;
-          }
-        }
-        if (!done) {
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            uint32_t af[4][4];
-            fwd_step<MT, false>(w[h][0], w[h][1], w[h][2], w[h][3], cst, af);
-#pragma unroll
-            for (int q = 0; q < 4; ++q)
-#pragma unroll
-              for (int nt = 0; nt < NT; ++nt) mma16816<MT>(acc[nt][q], af[q], b0[h][nt], b1[h][nt]);
-          }
+            for (int nt = 0; nt < NT; ++nt) mma16816<MT>(acc[nt][q], af[q], b0[h][nt], b1[h][nt]);
         }
       }
     }
@@ -490,13 +450,6 @@ __global__ void __launch_bounds__(stream::kThreads, 2)
 
     // ---------------- the segment ends here
     const bool seg_ok = !*abort;  // no stores from a segment an abort cut short
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {  // fold the 16x-scaled odd slots back (exact power-of-two scaling)
-        acc[nt][1][k] += acc16[nt][0][k] * 0.0625f;
-        acc[nt][3][k] += acc16[nt][1][k] * 0.0625f;
-      }
     if (seg_c0 != 0 || seg_c1 != nst) {
       // a part of a shared item: FP32 partial sums to partials[part][row][column]
       const int64_t part = (int64_t)blockIdx.x - sk_owner(i * nst, G, grid);

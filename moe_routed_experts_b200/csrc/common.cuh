@@ -169,13 +169,6 @@ __device__ __forceinline__ uint32_t umax16x2(uint32_t a, uint32_t b) {
   return r;
 }
 
-// Lane-wise minimum of two 16-bit pairs.
-__device__ __forceinline__ uint32_t umin16x2(uint32_t a, uint32_t b) {
-  uint32_t r;
-  asm("min.u16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
-  return r;
-}
-
 // N activation pairs at once, with the range report of act_pair_to_mt at a
 // fraction of its cost: the pairs are tested one by one only when some
 // source magnitude is at least 65536 (BF16 0x4780, the first value F16

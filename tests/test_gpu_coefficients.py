@@ -2,7 +2,7 @@
 
 [FA] FrozenAwqOps keeps the scale-dtype rounding of each coefficient
 W = RNE_sdt((q - z) s); every projection kernel forms W in its own code
-(the streaming decode tile with its odd-slot shortcut, the tcgen05 dequant
+(the streaming decode tile, the tcgen05 dequant
 warps, the warp-level tiles, the input-VJP tiles).  Fed one-hot rows, a
 kernel's output IS its coefficients: with activations in the scale dtype and
 no bias, row r = e_kk makes the FP32 accumulation hold the single exact
@@ -43,9 +43,8 @@ def path(request):
 def _scales(rng, shape, sdt, wide):
     """Scales of the workloads (uniform[0.5, 1.5) / (8 sqrt(K)) in the scale
     dtype), or, with `wide`, F16/BF16 bit patterns over many binades: for F16
-    subnormal scales and scales above 256 (both outside the range where the
-    streaming tile's odd-slot shortcut applies, so those groups take the
-    plain path) while |15 s| stays finite."""
+    subnormal scales (products rounded on the subnormal grid) and scales up
+    to 4096, while |15 s| stays finite."""
     if not wide:
         return None
     if sdt == "f16":

@@ -529,7 +529,16 @@ __global__ void __launch_bounds__(256) awq_stream_reduce_kernel(ProjParams p) {
   const int64_t total = p.A * per_row;
   const int S = (int)((p.N / 8 + kSlabW - 1) / kSlabW);
   const int nst = (int)(p.K / ROWS);
-  const int64_t G = (int64_t)p.counters[p.E] * nst;
+  // the row offsets and item prefix in shared memory: the searches below
+  // then cost no global round trips
+  extern __shared__ int32_t rsm[];
+  int32_t *off_s = rsm, *pre_s = rsm + (p.E + 1);
+  for (int e = threadIdx.x; e <= p.E; e += blockDim.x) {
+    off_s[e] = p.offsets[e];
+    pre_s[e] = p.counters[e];
+  }
+  __syncthreads();
+  const int64_t G = (int64_t)pre_s[p.E] * nst;
   const int64_t grid = sk_grid(G, p.kq);
   for (int64_t v = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; v < total; v += (int64_t)gridDim.x * blockDim.x) {
     const int64_t r = v / per_row, n0 = (v % per_row) * 8;
@@ -537,12 +546,12 @@ __global__ void __launch_bounds__(256) awq_stream_reduce_kernel(ProjParams p) {
     int lo = 0, hi = p.E - 1;
     while (lo < hi) {
       const int mid = (lo + hi + 1) >> 1;
-      if (p.offsets[mid] <= r) lo = mid;
+      if (off_s[mid] <= r) lo = mid;
       else hi = mid - 1;
     }
-    const int64_t tt = (r - p.offsets[lo]) / (8 * NT);
-    const int64_t item = p.counters[lo] + tt * S + n0 / kOut;
-    if (r < p.offsets[lo] || item < 0 || item >= p.counters[p.E]) continue;  // rows of a range flagged bad
+    const int64_t tt = (r - off_s[lo]) / (8 * NT);
+    const int64_t item = pre_s[lo] + tt * S + n0 / kOut;
+    if (r < off_s[lo] || item < 0 || item >= pre_s[p.E]) continue;  // rows of a range flagged bad
     const int64_t first = sk_owner(item * nst, G, grid), last = sk_owner(item * nst + nst - 1, G, grid);
     if (first == last || last - first >= sk_max_parts(nst)) continue;  // the fused epilogue wrote these outputs
     float a[NPROJ][8];
@@ -633,7 +642,8 @@ static moe_status launch_stream_r(const ProjParams &p0, cudaStream_t st) {
   int64_t blocks = (work + 255) / 256;
   const int64_t cap = (int64_t)num_sms() * 8;
   if (blocks > cap) blocks = cap;
-  launch_pdl(awq_stream_reduce_kernel<NPROJ, NT, ROWS>, dim3((unsigned)blocks), dim3(256), 0, st, p);
+  launch_pdl(awq_stream_reduce_kernel<NPROJ, NT, ROWS>, dim3((unsigned)blocks), dim3(256),
+             (size_t)(2 * (p.E + 1)) * sizeof(int32_t), st, p);
   return check_launch("awq_stream_reduce_kernel");
 }
 

@@ -92,7 +92,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kLStages; ++s) {
-      mbar_init(&full[s], 1);
+      mbar_init(&full[s], p.gather ? 1 + 32 : 1);  // + the producer lanes' gathered rows
       mbar_init(&empty[s], 1 + kDqWarps);
     }
     for (int b = 0; b < kBStages; ++b) {
@@ -147,19 +147,34 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 0) {
-    // ---------------- producer (lane 0; with a gather, every lane loads
-    // four rows of the activation tile through tile::gather4)
+    // ---------------- producer (lane 0, by TMA).  With a gather, every lane
+    // copies four rows of each activation step with 16-byte cp.async into
+    // the swizzled atom (lane L: tile rows L, L + 32, L + 64, L + 96) and
+    // arrives on the stage's full barrier once its copies of that stage
+    // landed (one stage behind, so two stages stay in flight), after a proxy
+    // fence for the tensor core.
     const bool gather = p.gather != nullptr;
     if (gather || lane == 0) {
+      const uint32_t rowoff = (uint32_t)((lane >> 3) * 1024 + (lane & 7) * 128);
       uint32_t it = 0;  // stages issued
       bool live = true;
+      bool pend = false;  // gather: a stage whose rows this lane still has to deliver
+      uint32_t pend_s = 0;
+      auto deliver = [&](bool all) {
+        if (!pend) return;
+        if (all) cp_async_wait<0>();
+        else cp_async_wait<1>();
+        fence_proxy_async_smem();
+        mbar_arrive(&full[pend_s]);
+        pend = false;
+      };
       for (int64_t tile = blockIdx.x; tile < total && live; tile += gridDim.x) {
         const TileInfo ti = tile_info(tile);
         const int32_t row0 = (int32_t)(ti.r0 + (int64_t)ti.mt * kBM);
-        int32_t src[4] = {0, 0, 0, 0};  // x rows of tile rows 4 lane .. 4 lane + 3 (rows past the batch: any row)
+        const uint16_t *srow[4] = {p.x, p.x, p.x, p.x};  // gather: x rows of tile rows lane + 32 i
         if (gather) {
 #pragma unroll
-          for (int i = 0; i < 4; ++i) src[i] = (int32_t)act_row(p, min((int64_t)row0 + 4 * lane + i, p.A - 1));
+          for (int i = 0; i < 4; ++i) srow[i] = p.x + act_row(p, min((int64_t)row0 + lane + 32 * i, p.A - 1)) * K;
         }
         for (int kb = 0; kb < nk; ++kb, ++it) {
           const uint32_t s = it % kLStages, use = it / kLStages;
@@ -167,14 +182,26 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
           uint8_t *st = lring + s * kLBytes;
           if (lane == 0) {
             ok = use == 0 || tc_wait(&empty[s], (use - 1) & 1, p.status, abort);
-            if (ok) mbar_arrive_expect_tx(&full[s], kLBytes);
+            if (ok) mbar_arrive_expect_tx(&full[s], gather ? kPBytes : kLBytes);
           }
           if (gather) ok = __shfl_sync(0xffffffffu, ok, 0);
           if (!ok) {
             live = false;
             break;
           }
-          if (gather) tma_gather4(st + 4 * lane * 128, &map_x, &full[s], kb * kBK, src[0], src[1], src[2], src[3]);
+          if (gather) {
+            const uint32_t sbase = smem_u32(st) + rowoff;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const uint16_t *src = srow[i] + (int64_t)kb * kBK;
+#pragma unroll
+              for (int cc = 0; cc < 8; ++cc) cp_async16(sbase + i * 4096 + ((cc ^ (lane & 7)) << 4), src + cc * 8);
+            }
+            cp_async_commit();
+            deliver(false);  // the previous stage (at most this one's copies left in flight)
+            pend = true;
+            pend_s = s;
+          }
           if (lane == 0) {
             if (!gather) tma_load_2d(st, &map_x, &full[s], kb * kBK, row0);
             const int32_t wrow = (int32_t)(ti.e * K + (int64_t)kb * kBK);
@@ -187,6 +214,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
           }
         }
       }
+      if (gather) deliver(true);  // every issued stage complete before the drain below
       if (lane == 0) tma_drain(full, it, kLStages, p.status);
     }
   } else if (warp == 1) {

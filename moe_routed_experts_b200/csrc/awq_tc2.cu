@@ -102,7 +102,7 @@ __global__ void __launch_bounds__(tc2::kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kLStages; ++s) {
-      mbar_init(&lfull[s], 1);
+      mbar_init(&lfull[s], p.gather ? 1 + 32 : 1);  // + the producer lanes' gathered rows
       mbar_init(&lempty[s], 1 + kDqWarps);  // pair-MMA commit + this CTA's dequant warps
     }
     for (int s = 0; s < kBStages; ++s) {
@@ -158,24 +158,39 @@ __global__ void __launch_bounds__(tc2::kThreads, 1)
 
   if (warp == 0) {
     // ---------------- producer: this CTA's activation rows and packed half
-    // (lane 0; with a gather, every lane loads four rows of each activation
-    // atom through tile::gather4)
+    // (lane 0, by TMA).  With a gather, every lane copies four rows of each
+    // activation step with 16-byte cp.async into the swizzled atoms (lane L:
+    // tile rows L, L + 32, L + 64, L + 96), and arrives on the stage's full
+    // barrier once its copies of that stage landed (one stage behind, so two
+    // stages stay in flight), after a proxy fence for the tensor core.
     const bool gather = p.gather != nullptr;
     if (gather || lane == 0) {
       const CUtensorMap *mw = (NPROJ == 2 && rank == 1) ? &map_w1 : &map_w0;
       const CUtensorMap *mz = (NPROJ == 2 && rank == 1) ? &map_z1 : &map_z0;
       const CUtensorMap *ms = (NPROJ == 2 && rank == 1) ? &map_s1 : &map_s0;
       const int64_t ngroups = K / p.group;
+      // shared-memory offsets of this lane's 16-byte chunks inside an atom
+      const uint32_t rowoff = (uint32_t)((lane >> 3) * 1024 + (lane & 7) * 128);
       uint32_t it = 0;  // stages issued
       bool live = true;
+      bool pend = false;  // gather: a stage whose rows this lane still has to deliver
+      uint32_t pend_s = 0;
+      auto deliver = [&](bool all) {
+        if (!pend) return;
+        if (all) cp_async_wait<0>();
+        else cp_async_wait<1>();
+        fence_proxy_async_smem();
+        mbar_arrive(&lfull[pend_s]);
+        pend = false;
+      };
       for (int64_t tile = pair; tile < total && live; tile += npairs) {
         const PairTile ti = tile_info(tile);
         const int32_t row0 = (int32_t)(ti.r0 + (int64_t)ti.mt * 2 * kBM + kBM * rank);
         const int32_t wcol = NPROJ == 2 ? ti.nt * 16 : ti.nt * 32 + 16 * (int)rank;
-        int32_t src[4] = {0, 0, 0, 0};  // x rows of tile rows 4 lane .. 4 lane + 3 (rows past the batch: any row)
+        const uint16_t *srow[4] = {p.x, p.x, p.x, p.x};  // gather: x rows of tile rows lane + 32 i
         if (gather) {
 #pragma unroll
-          for (int i = 0; i < 4; ++i) src[i] = (int32_t)act_row(p, min((int64_t)row0 + 4 * lane + i, p.A - 1));
+          for (int i = 0; i < 4; ++i) srow[i] = p.x + act_row(p, min((int64_t)row0 + lane + 32 * i, p.A - 1)) * K;
         }
         for (int kb = 0; kb < nk; ++kb, ++it) {
           const uint32_t s = it % kLStages, use = it / kLStages;
@@ -183,7 +198,7 @@ __global__ void __launch_bounds__(tc2::kThreads, 1)
           uint8_t *st = lring + s * kLBytes;
           if (lane == 0) {
             ok = use == 0 || tc_wait(&lempty[s], (use - 1) & 1, p.status, abort);
-            if (ok) mbar_arrive_expect_tx(&lfull[s], kLBytes + kZBytes + 256);
+            if (ok) mbar_arrive_expect_tx(&lfull[s], (gather ? kPBytes : kLBytes) + kZBytes + 256);
           }
           if (gather) ok = __shfl_sync(0xffffffffu, ok, 0);
           if (!ok) {
@@ -191,9 +206,20 @@ __global__ void __launch_bounds__(tc2::kThreads, 1)
             break;
           }
           if (gather) {
-            tma_gather4(st + 4 * lane * 128, &map_x, &lfull[s], kb * kBK, src[0], src[1], src[2], src[3]);
-            tma_gather4(st + kAtom + 4 * lane * 128, &map_x, &lfull[s], kb * kBK + 64, src[0], src[1], src[2],
-                        src[3]);
+            const uint32_t sbase = smem_u32(st) + rowoff;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const uint16_t *src = srow[i] + (int64_t)kb * kBK;
+#pragma unroll
+              for (int a = 0; a < 2; ++a)
+#pragma unroll
+                for (int cc = 0; cc < 8; ++cc)
+                  cp_async16(sbase + a * kAtom + i * 4096 + ((cc ^ (lane & 7)) << 4), src + a * 64 + cc * 8);
+            }
+            cp_async_commit();
+            deliver(false);  // the previous stage (at most this one's copies left in flight)
+            pend = true;
+            pend_s = s;
           }
           if (lane == 0) {
             if (!gather) {
@@ -209,6 +235,7 @@ __global__ void __launch_bounds__(tc2::kThreads, 1)
           }
         }
       }
+      if (gather) deliver(true);  // every issued stage complete before the drain below
       if (lane == 0) tma_drain(lfull, it, kLStages, p.status);
     }
   } else if (warp == 1) {

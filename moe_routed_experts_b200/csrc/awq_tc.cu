@@ -151,24 +151,22 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
     // copies four rows of each activation step with 16-byte cp.async into
     // the swizzled atom (lane L: tile rows L, L + 32, L + 64, L + 96) and
     // arrives on the stage's full barrier once its copies of that stage
-    // landed (up to kLStages - 1 stages in flight), after a proxy fence for
-    // the tensor core.
+    // landed (one stage behind, so two stages stay in flight), after a proxy
+    // fence for the tensor core.
     const bool gather = p.gather != nullptr;
     if (gather || lane == 0) {
       const uint32_t rowoff = (uint32_t)((lane >> 3) * 1024 + (lane & 7) * 128);
       uint32_t it = 0;  // stages issued
       bool live = true;
-      // gather: stages whose rows this lane still has to deliver (oldest
-      // first); the oldest is delivered before the next stage is requested
-      // once kLStages - 1 are pending
-      uint32_t pend_s[kLStages];
-      int npend = 0;
-      auto deliver_oldest = [&]() {
+      bool pend = false;  // gather: a stage whose rows this lane still has to deliver
+      uint32_t pend_s = 0;
+      auto deliver = [&](bool all) {
+        if (!pend) return;
+        if (all) cp_async_wait<0>();
+        else cp_async_wait<1>();
         fence_proxy_async_smem();
-        mbar_arrive(&full[pend_s[0]]);
-#pragma unroll
-        for (int q = 0; q + 1 < kLStages; ++q) pend_s[q] = pend_s[q + 1];
-        --npend;
+        mbar_arrive(&full[pend_s]);
+        pend = false;
       };
       for (int64_t tile = blockIdx.x; tile < total && live; tile += gridDim.x) {
         const TileInfo ti = tile_info(tile);
@@ -180,10 +178,6 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
         }
         for (int kb = 0; kb < nk; ++kb, ++it) {
           const uint32_t s = it % kLStages, use = it / kLStages;
-          if (gather && npend == kLStages - 1) {  // the oldest pending stage lands before its slot is reused
-            cp_async_wait<kLStages - 2>();
-            deliver_oldest();
-          }
           bool ok = true;
           uint8_t *st = lring + s * kLBytes;
           if (lane == 0) {
@@ -204,7 +198,9 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
               for (int cc = 0; cc < 8; ++cc) cp_async16(sbase + i * 4096 + ((cc ^ (lane & 7)) << 4), src + cc * 8);
             }
             cp_async_commit();
-            pend_s[npend++] = s;
+            deliver(false);  // the previous stage (at most this one's copies left in flight)
+            pend = true;
+            pend_s = s;
           }
           if (lane == 0) {
             if (!gather) tma_load_2d(st, &map_x, &full[s], kb * kBK, row0);
@@ -218,10 +214,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
           }
         }
       }
-      if (gather) {  // every issued stage complete before the drain below
-        cp_async_wait<0>();
-        while (npend > 0) deliver_oldest();
-      }
+      if (gather) deliver(true);  // every issued stage complete before the drain below
       if (lane == 0) tma_drain(full, it, kLStages, p.status);
     }
   } else if (warp == 1) {

@@ -259,10 +259,8 @@ __global__ void __launch_bounds__(stream::kThreads, 2)
                 (uint32_t)(len * 2), &xfull[xb]);
     ++xissued;
   };
-  auto issue_stage = [&](int64_t j) {
+  auto issue_stage_ic = [&](int64_t j, int64_t i, int c) {
     const uint32_t s = (uint32_t)((j - g0) % kStages);
-    const int64_t i = j / nst;
-    const int c = (int)(j - i * nst);
     const ItemInfo &ii = issue_info(i);
     const int32_t row0 = (int32_t)(ii.e * K + (int64_t)c * kRows);
     mbar_arrive_expect_tx(&full[s], kStageBytes);
@@ -274,6 +272,10 @@ __global__ void __launch_bounds__(stream::kThreads, 2)
       tma_load_2d(dst, &map0, &full[s], ii.sl * 2 * kBoxW, row0);
       tma_load_2d(dst + kBox, &map0, &full[s], ii.sl * 2 * kBoxW + kBoxW, row0);
     }
+  };
+  auto issue_stage = [&](int64_t j) {
+    const int64_t i = j / nst;
+    issue_stage_ic(j, i, (int)(j - i * nst));
   };
   // blocking: issue every stage up to `upto` (waits for the slots' release)
   auto issue_upto = [&](int64_t upto) {
@@ -296,7 +298,7 @@ __global__ void __launch_bounds__(stream::kThreads, 2)
   // g0 + r - kStages + 1, once every warp released the slot's previous
   // stage, so no single warp carries the issue work.
   bool rlive = true;
-  auto issue_rotating = [&](int64_t j) {
+  auto issue_rotating = [&](int64_t j, int64_t i, int c) {
     const int64_t st = j + kStages - 1;  // the stage due now
     const int64_t r = st - g0;
     if (r < kStages || st >= g1 || !rlive || lane != 0 || (int)(r % kCW) != warp) return;
@@ -305,7 +307,12 @@ __global__ void __launch_bounds__(stream::kThreads, 2)
       rlive = false;
       return;
     }
-    issue_stage(st);
+    c += kStages - 1;  // item and stage of st
+    while (c >= nst) {
+      c -= nst;
+      ++i;
+    }
+    issue_stage_ic(st, i, c);
     atomicMax(issued_hi, (int32_t)(r + 1));
   };
 
@@ -333,9 +340,10 @@ __global__ void __launch_bounds__(stream::kThreads, 2)
   uint32_t pf_zw = 0u;
   uint4 pf_sv = make_uint4(0, 0, 0, 0);
   uint32_t it = 0, xi = 0;
-  for (int64_t j = g0; j < g1; ++j, ++it) {
-    const int64_t i = j / nst;
-    const int c = (int)(j - i * nst);
+  // item i and stage c of stage j, advanced without a division
+  int64_t i = g0 / nst;
+  int c = (int)(g0 - i * nst);
+  for (int64_t j = g0; j < g1; ++j, ++it, c = (c + 1 == nst) ? (++i, 0) : c + 1) {
     if (j == g0 || c == 0) {  // a segment of item i starts: its rows, columns and first group
       ii = item_info(pre, p.offsets, E, S, i);
       tok0 = ii.tt * 8 * NT;
@@ -379,8 +387,9 @@ __global__ void __launch_bounds__(stream::kThreads, 2)
         const uint8_t *src = xraw + xb * xraw_bytes;
         const int len = (int)min((int64_t)kXRows, K - (int64_t)xbase * kRows);
         const int per_tok = len / 8, halves = mrows * per_tok;
+        const bool whole = per_tok == kXRows / 8;
         for (int q = threadIdx.x; q < halves; q += kCW * 32) {
-          const int tok = q / per_tok;
+          const int tok = whole ? q / (kXRows / 8) : q / per_tok;
           const int hb = q - tok * per_tok, blk = hb >> 1, h = hb & 1;
           const uint4 v = *reinterpret_cast<const uint4 *>(src + (tok * kXRows + blk * 16 + h * 8) * 2);
           uint32_t pr[4] = {prmt(v.x, v.z, 0x5410u), prmt(v.x, v.z, 0x7632u), prmt(v.y, v.w, 0x5410u),
@@ -407,7 +416,7 @@ __global__ void __launch_bounds__(stream::kThreads, 2)
       gstage = 0;
       ++grp;
     }
-    issue_rotating(j);
+    issue_rotating(j, i, c);
     // warp-uniform: the MMAs below are warp-wide
     const bool sok = __all_sync(0xffffffffu, tc_wait(&full[s], ph, p.status, abort));
     if (sok) {

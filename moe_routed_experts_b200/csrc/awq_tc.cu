@@ -277,8 +277,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
     const bool convert = !p.preconv && p.act_dt != (std::is_same<MT, __half>::value ? MOE_F16 : MOE_BF16);
     uint32_t it = 0;
     bool live = true;
-    // zeros/scales of a tile's word column; the first group of the next tile
-    // is requested during the last group of the current one
+    // zeros/scales of a tile's word column
     struct ZsPtr {
       const int32_t *qz;
       const uint16_t *sc;
@@ -291,40 +290,46 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
       const int64_t wcs = ok ? wc : 0;
       return ZsPtr{qz + (int64_t)tn.e * ngroups * NW + wcs, sc + (int64_t)tn.e * ngroups * p.N + 8 * wcs, ok};
     };
-    ZsPtr cur = zs_ptr((int64_t)blockIdx.x < total ? (int64_t)blockIdx.x : 0);
-    uint32_t pf_zw = ((int64_t)blockIdx.x < total && cur.ok) ? (uint32_t)__ldg(cur.qz) : 0u;
-    uint4 pf_sv = ((int64_t)blockIdx.x < total && cur.ok) ? __ldg(reinterpret_cast<const uint4 *>(cur.sc))
-                                                           : make_uint4(0, 0, 0, 0);
+    // the zero/scale rows are fetched two groups ahead, in the order the
+    // loop below consumes them (the groups of a tile, then the next tile's)
+    int64_t zt = blockIdx.x, zg = 0;
+    ZsPtr zcur = zs_ptr(zt < total ? zt : 0);
+    auto fetch = [&](uint32_t &zw, uint4 &sv) {
+      zw = 0u;
+      sv = make_uint4(0, 0, 0, 0);
+      if (zt >= total) return;
+      if (zcur.ok) {
+        zw = (uint32_t)__ldg(zcur.qz + zg * NW);
+        sv = __ldg(reinterpret_cast<const uint4 *>(zcur.sc + zg * p.N));
+      }
+      if (++zg == ngroups) {
+        zg = 0;
+        zt += gridDim.x;
+        if (zt < total) zcur = zs_ptr(zt);
+      }
+    };
+    uint32_t pa_zw, pb_zw;
+    uint4 pa_sv, pb_sv;
+    fetch(pa_zw, pa_sv);
+    fetch(pb_zw, pb_sv);
     for (int64_t tile = blockIdx.x; tile < total && live; tile += gridDim.x) {
-      const ZsPtr zs = cur;
       uint32_t zp[4], sp[4];
-      int64_t grp = 0;
       int gstage = 0;
       for (int kb = 0; kb < nk; ++kb, ++it) {
         const uint32_t s = it % kLStages, ph = (it / kLStages) & 1;
         const uint32_t b = it % kBStages, buse = it / kBStages;
-        if (gstage == 0) {  // a new group: take the prefetched zeros/scales, prefetch the next
-          const uint32_t s4[4] = {pf_sv.x, pf_sv.y, pf_sv.z, pf_sv.w};
+        if (gstage == 0) {  // a new group: take the oldest fetched zeros/scales, fetch another
+          const uint32_t s4[4] = {pa_sv.x, pa_sv.y, pa_sv.z, pa_sv.w};
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
-            zp[q] = nib_pair<M>(pf_zw >> (4 * q));
+            zp[q] = nib_pair<M>(pa_zw >> (4 * q));
             sp[q] = s4[q];
           }
-          if (grp + 1 < ngroups) {
-            if (zs.ok) {
-              pf_zw = (uint32_t)__ldg(zs.qz + (grp + 1) * NW);
-              pf_sv = __ldg(reinterpret_cast<const uint4 *>(zs.sc + (grp + 1) * p.N));
-            }
-          } else if (tile + gridDim.x < total) {
-            cur = zs_ptr(tile + gridDim.x);
-            pf_zw = cur.ok ? (uint32_t)__ldg(cur.qz) : 0u;
-            pf_sv = cur.ok ? __ldg(reinterpret_cast<const uint4 *>(cur.sc)) : make_uint4(0, 0, 0, 0);
-          }
+          pa_zw = pb_zw;
+          pa_sv = pb_sv;
+          fetch(pb_zw, pb_sv);
         }
-        if (++gstage == spg) {
-          gstage = 0;
-          ++grp;
-        }
+        if (++gstage == spg) gstage = 0;
         if (!tc_wait(&full[s], ph, p.status, abort)) {
           live = false;
           break;

@@ -536,7 +536,8 @@ def launches_per_step_of(B, w):
     """Kernel launches of one step: route (2, or 3 past one token chunk), each
     projection (1, or 2 with the split-K reduce; a tcgen05 projection with F16
     scales adds the one-time F16 copy of its BF16 input), combine, and the
-    backward's six (plus the F16 copies of the three input-VJP gradients)."""
+    backward's six (its input-VJP gradients are written in the scale dtype,
+    so it makes no copies)."""
     n = 2 if w.T <= 64 else 3
     conv = _path_of(w) >= 2 and w.scale_dtype == "f16"
     if _path_of(w) == 1:
@@ -546,7 +547,7 @@ def launches_per_step_of(B, w):
         n += 2 + (2 if conv else 0)
     n += 1
     if w.backward:
-        n += 6 + (3 if conv else 0)
+        n += 6
     return n
 
 

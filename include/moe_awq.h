@@ -92,7 +92,8 @@ typedef enum { MOE_F32 = 0, MOE_F16 = 1, MOE_BF16 = 2 } moe_dtype;
 #define MOE_DEVICE_ERR_TIMEOUT 8      /* a bounded device wait gave up */
 #define MOE_DEVICE_ERR_ACT_RANGE 16   /* a BF16 activation or gradient fed to F16-scale tensor cores was
                                          finite above F16's range (|v| > 65504: it became inf) or NaN;
-                                         the result is computed from the converted value */
+                                         the result is computed from the converted value.  Also set by
+                                         the _dt backward steps that write F16 from BF16 inputs */
 
 /* Limits of this implementation. */
 #define MOE_MAX_EXPERTS 4096
@@ -362,6 +363,17 @@ MOE_API moe_status moe_combine_backward(const void *d_out, const void *y, moe_dt
                                 int64_t H, int32_t top_k, void *dy, float *dweights,
                                 int32_t *device_status, void *stream);
 
+/* moe_combine_backward with dy stored in dy_dtype (F16 or BF16) instead of
+ * act_dtype: dy[row_of[t,j], :] = RNE_{dy_dtype}(weights[t,j] * d_out[t, :]),
+ * one rounding of the FP32 product.  F16 dy from BF16 inputs feeds an input
+ * VJP with F16 scales without a conversion pass; a value that is not +-inf
+ * but becomes inf or NaN in F16 sets MOE_DEVICE_ERR_ACT_RANGE (the rule of
+ * the BF16 -> F16 input conversion).  dweights is unchanged. */
+MOE_API moe_status moe_combine_backward_dt(const void *d_out, const void *y, moe_dtype act_dtype, int64_t A,
+                                   const float *weights, const int32_t *row_of, int64_t T,
+                                   int64_t H, int32_t top_k, void *dy, moe_dtype dy_dtype,
+                                   float *dweights, int32_t *device_status, void *stream);
+
 /* ------------------------------------------------------------------------
  * awq_input_backward -- [FA] FrozenAwqOps::frozen_awq_input_backward and
  * [PE] packed_expert_input_backward / packed_swiglu_input_backward: the
@@ -389,6 +401,19 @@ MOE_API moe_status awq_input_backward(const void *grad, moe_dtype grad_dtype, in
                               const void *scales2, void *dinput, void *workspace,
                               size_t workspace_bytes, int32_t *device_status, void *stream);
 
+/* awq_input_backward with dinput stored in dinput_dtype (F16 or BF16)
+ * instead of grad_dtype: the same FP32 sums, one rounding to dinput_dtype.
+ * F16 gradients with F16 scales need no conversion (workspace 0 bytes) and
+ * can still give BF16 input gradients. */
+MOE_API moe_status awq_input_backward_dt(const void *grad, moe_dtype grad_dtype, int64_t A, int64_t N,
+                                 int64_t K, const int32_t *offsets, int64_t E,
+                                 const int32_t *qweight, const int32_t *qzeros, const void *scales,
+                                 moe_dtype scale_dtype, int64_t group_size, const void *grad2,
+                                 const int32_t *qweight2, const int32_t *qzeros2,
+                                 const void *scales2, void *dinput, moe_dtype dinput_dtype,
+                                 void *workspace, size_t workspace_bytes, int32_t *device_status,
+                                 void *stream);
+
 /* Workspace bytes of awq_input_backward for A gradient rows of width N
  * (nproj = 2 with grad2), output width K, under the current path; 0 if none. */
 MOE_API size_t awq_input_backward_workspace_size(int64_t A, int64_t N, int64_t K, int64_t E,
@@ -402,6 +427,15 @@ MOE_API size_t awq_input_backward_workspace_size(int64_t A, int64_t N, int64_t K
  * ---------------------------------------------------------------------- */
 MOE_API moe_status moe_swiglu_backward(const void *dh, const void *G, const void *U, moe_dtype act_dtype,
                                int64_t A, int64_t I, void *dG, void *dU, void *stream);
+
+/* moe_swiglu_backward with dG and dU stored in grad_dtype (F16 or BF16)
+ * instead of act_dtype (dh, G, U stay act_dtype): the same FP32 values, one
+ * rounding to grad_dtype.  BF16 inputs with F16 grad_dtype report values
+ * that are not +-inf but become inf or NaN in F16 as
+ * MOE_DEVICE_ERR_ACT_RANGE in device_status (may be NULL: no report). */
+MOE_API moe_status moe_swiglu_backward_dt(const void *dh, const void *G, const void *U, moe_dtype act_dtype,
+                                  int64_t A, int64_t I, void *dG, void *dU, moe_dtype grad_dtype,
+                                  int32_t *device_status, void *stream);
 
 /* ------------------------------------------------------------------------
  * moe_dispatch_backward -- [MX] MoeDispatchOps::moe_dispatch_backward ("COPY

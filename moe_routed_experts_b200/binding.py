@@ -59,6 +59,10 @@ _SIGS = {
     "awq_input_backward": (C.c_int, [P, C.c_int, I64, I64, I64, P, I64, P, P, P, C.c_int, I64, P, P, P, P, P, P, SZ,
                                      P, P]),
     "moe_swiglu_backward": (C.c_int, [P, P, P, C.c_int, I64, I64, P, P, P]),
+    "moe_combine_backward_dt": (C.c_int, [P, P, C.c_int, I64, P, P, I64, I64, I32, P, C.c_int, P, P, P]),
+    "awq_input_backward_dt": (C.c_int, [P, C.c_int, I64, I64, I64, P, I64, P, P, P, C.c_int, I64, P, P, P, P, P,
+                                        C.c_int, P, SZ, P, P]),
+    "moe_swiglu_backward_dt": (C.c_int, [P, P, P, C.c_int, I64, I64, P, P, C.c_int, P, P]),
     "moe_dispatch_backward": (C.c_int, [P, C.c_int, I64, P, P, I64, I64, I32, P, P, P]),
     "moe_router_backward": (C.c_int, [P, P, P, I64, I64, I32, I32, I32, P, P, P]),
     "awq_dequant_coefficients": (C.c_int, [P, P, P, C.c_int, I64, I64, I64, I32, P, P]),
@@ -294,40 +298,50 @@ def moe_combine(y, weights, selected_experts, row_of, device_status=None, out=No
     return o
 
 
-def moe_combine_backward(d_out, y, weights, row_of, want_dy=True, want_dw=True, device_status=None):
+def moe_combine_backward(d_out, y, weights, row_of, want_dy=True, want_dw=True, device_status=None, dy_dtype=None):
+    """dy in dy_dtype (default: y's dtype) and the FP32 weight VJP."""
     A, H = y.shape
     T, k = weights.shape
-    dy = torch.empty_like(y) if want_dy else None
+    dy_dtype = dy_dtype or y.dtype
+    dy = torch.empty((A, H), dtype=dy_dtype, device=y.device) if want_dy else None
     dw = torch.empty((T, k), dtype=torch.float32, device=y.device) if want_dw else None
-    st = lib().moe_combine_backward(_ptr(d_out), _ptr(y), _dt(y.dtype), A, _ptr(weights), _ptr(row_of), T, H, k,
-                                    _ptr(dy), _ptr(dw), _ptr(device_status), _stream())
+    st = lib().moe_combine_backward_dt(_ptr(d_out), _ptr(y), _dt(y.dtype), A, _ptr(weights), _ptr(row_of), T, H, k,
+                                       _ptr(dy), _dt(dy_dtype), _ptr(dw), _ptr(device_status), _stream())
     _check("moe_combine_backward", st)
     return dy, dw
 
 
 def awq_input_backward(grad, offsets, proj, group, grad2=None, proj2=None, device_status=None, out=None,
-                       workspace=None):
+                       workspace=None, out_dtype=None):
+    """Input VJP in out_dtype (default: the gradients' dtype; ``out``'s dtype when given)."""
     A, N = grad.shape
     E = offsets.numel() - 1
     K = proj["qweight"].shape[1]
-    d = out if out is not None else torch.empty((A, K), dtype=grad.dtype, device=grad.device)
+    if out is not None:
+        out_dtype = out.dtype
+    out_dtype = out_dtype or grad.dtype
+    d = out if out is not None else torch.empty((A, K), dtype=out_dtype, device=grad.device)
     p2 = proj2 or {}
     nbytes = input_backward_workspace_size(A, N, K, E, group, 2 if grad2 is not None else 1, grad.dtype,
                                            proj["scales"].dtype)
     ws = _workspace(nbytes, grad.device, workspace)
-    st = lib().awq_input_backward(
+    st = lib().awq_input_backward_dt(
         _ptr(grad), _dt(grad.dtype), A, N, K, _ptr(offsets), E, _ptr(proj["qweight"]), _ptr(proj["qzeros"]),
         _ptr(proj["scales"]), _dt(proj["scales"].dtype), group, _ptr(grad2), _ptr(p2.get("qweight")),
-        _ptr(p2.get("qzeros")), _ptr(p2.get("scales")), _ptr(d), _ptr(ws), 0 if ws is None else ws.numel(),
-        _ptr(device_status), _stream())
+        _ptr(p2.get("qzeros")), _ptr(p2.get("scales")), _ptr(d), _dt(out_dtype), _ptr(ws),
+        0 if ws is None else ws.numel(), _ptr(device_status), _stream())
     _check("awq_input_backward", st)
     return d
 
 
-def moe_swiglu_backward(dh, G, U):
+def moe_swiglu_backward(dh, G, U, out_dtype=None, device_status=None):
+    """dG, dU in out_dtype (default: G's dtype); dh, G and U share one dtype."""
     A, I = G.shape
-    dG, dU = torch.empty_like(G), torch.empty_like(U)
-    st = lib().moe_swiglu_backward(_ptr(dh), _ptr(G), _ptr(U), _dt(G.dtype), A, I, _ptr(dG), _ptr(dU), _stream())
+    out_dtype = out_dtype or G.dtype
+    dG = torch.empty((A, I), dtype=out_dtype, device=G.device)
+    dU = torch.empty((A, I), dtype=out_dtype, device=G.device)
+    st = lib().moe_swiglu_backward_dt(_ptr(dh), _ptr(G), _ptr(U), _dt(G.dtype), A, I, _ptr(dG), _ptr(dU),
+                                      _dt(out_dtype), _ptr(device_status), _stream())
     _check("moe_swiglu_backward", st)
     return dG, dU
 

@@ -274,16 +274,18 @@ extern "C" moe_status awq_grouped_down(const void *input, moe_dtype act_dtype, i
   return check_launch(fn);
 }
 
-extern "C" moe_status awq_input_backward(const void *grad, moe_dtype grad_dtype, int64_t A, int64_t N, int64_t K,
-                                         const int32_t *offsets, int64_t E, const int32_t *qweight,
-                                         const int32_t *qzeros, const void *scales, moe_dtype scale_dtype,
-                                         int64_t group_size, const void *grad2, const int32_t *qweight2,
-                                         const int32_t *qzeros2, const void *scales2, void *dinput,
-                                         void *workspace, size_t workspace_bytes, int32_t *device_status,
-                                         void *stream) {
+extern "C" moe_status awq_input_backward_dt(const void *grad, moe_dtype grad_dtype, int64_t A, int64_t N, int64_t K,
+                                            const int32_t *offsets, int64_t E, const int32_t *qweight,
+                                            const int32_t *qzeros, const void *scales, moe_dtype scale_dtype,
+                                            int64_t group_size, const void *grad2, const int32_t *qweight2,
+                                            const int32_t *qzeros2, const void *scales2, void *dinput,
+                                            moe_dtype dinput_dtype, void *workspace, size_t workspace_bytes,
+                                            int32_t *device_status, void *stream) {
   const char *fn = "awq_input_backward";
   moe_status s = check_payload_geom(fn, A, K, N, E, group_size, grad_dtype, scale_dtype);
   if (s != MOE_OK) return s;
+  if (dinput_dtype != MOE_F16 && dinput_dtype != MOE_BF16)
+    return set_error(MOE_ERR_UNSUPPORTED_DTYPE, "%s: dinput_dtype must be F16 or BF16", fn);
   if (A == 0) return MOE_OK;
   s = check_ptrs(fn, {grad, offsets, qweight, qzeros, scales, dinput}, {grad, scales, dinput, grad2, scales2});
   if (s != MOE_OK) return s;
@@ -295,6 +297,7 @@ extern "C" moe_status awq_input_backward(const void *grad, moe_dtype grad_dtype,
   p.grad[0] = static_cast<const uint16_t *>(grad);
   p.grad[1] = static_cast<const uint16_t *>(grad2 ? grad2 : grad);
   p.gdt = grad_dtype;
+  p.odt = dinput_dtype;
   p.A = A;
   p.N = N;
   p.K = K;
@@ -331,6 +334,18 @@ extern "C" moe_status awq_input_backward(const void *grad, moe_dtype grad_dtype,
   }
   launch_bwd_mma(p, nproj, bf, A >= 12 * E ? 2 : 1, st);
   return check_launch(fn);
+}
+
+extern "C" moe_status awq_input_backward(const void *grad, moe_dtype grad_dtype, int64_t A, int64_t N, int64_t K,
+                                         const int32_t *offsets, int64_t E, const int32_t *qweight,
+                                         const int32_t *qzeros, const void *scales, moe_dtype scale_dtype,
+                                         int64_t group_size, const void *grad2, const int32_t *qweight2,
+                                         const int32_t *qzeros2, const void *scales2, void *dinput,
+                                         void *workspace, size_t workspace_bytes, int32_t *device_status,
+                                         void *stream) {
+  return awq_input_backward_dt(grad, grad_dtype, A, N, K, offsets, E, qweight, qzeros, scales, scale_dtype,
+                               group_size, grad2, qweight2, qzeros2, scales2, dinput, grad_dtype, workspace,
+                               workspace_bytes, device_status, stream);
 }
 
 extern "C" moe_status awq_dequant_coefficients(const int32_t *qweight, const int32_t *qzeros, const void *scales,

@@ -322,7 +322,7 @@ __global__ void __launch_bounds__(128) awq_bwd_mma_kernel(BwdParams p) {
         float s1 = red[0][tk][rq + i + 1] + red[1][tk][rq + i + 1];
         s1 += red[2][tk][rq + i + 1];
         s1 += red[3][tk][rq + i + 1];
-        o[i / 2] = uint32_t(f32_to_bits(s0, p.gdt)) | (uint32_t(f32_to_bits(s1, p.gdt)) << 16);
+        o[i / 2] = uint32_t(f32_to_bits(s0, p.odt)) | (uint32_t(f32_to_bits(s1, p.odt)) << 16);
       }
       *reinterpret_cast<uint4 *>(p.out + (r0 + tok0 + tk) * p.K + k0) = make_uint4(o[0], o[1], o[2], o[3]);
     }

@@ -285,7 +285,7 @@ __global__ void __launch_bounds__(tc2b::kThreads, 1)
     // ---------------- epilogue warps: this CTA's 128 rows, 256 output columns
     const int q = warp & 3;                     // TMEM lane quarter
     const int hf = (warp - 2 - kDqWarps) >> 2;  // column half drained by this warp
-    const bool bf = p.gdt == MOE_BF16;
+    const bool bf = p.odt == MOE_BF16;
     uint32_t tcount = 0;
     for (int64_t tile = pair; tile < total; tile += npairs, ++tcount) {
       const PairBwdTile ti = tile_info(tile);

@@ -270,7 +270,7 @@ __global__ void __launch_bounds__(tcb::kThreads, 1)
     // ---------------- epilogue warps
     const int q = warp & 3;                     // TMEM lane quarter
     const int hf = (warp - 2 - kDqWarps) >> 2;  // column half drained by this warp
-    const bool bf = p.gdt == MOE_BF16;
+    const bool bf = p.odt == MOE_BF16;
     uint32_t tcount = 0;
     for (int64_t tile = blockIdx.x; tile < total; tile += gridDim.x, ++tcount) {
       const BwdTile ti = tile_info(tile);

@@ -132,7 +132,17 @@ struct CombineBwdParams {
   void *dy;
   float *dweights;
   int32_t *status;
+  int odt;  // dtype of dy
 };
+
+// v rounded to dtype dt.  With chk (BF16-range values written as F16), a
+// value that is not +-inf but becomes inf or NaN in F16 sets bad, the rule
+// of the BF16 -> F16 input conversion.
+__device__ __forceinline__ uint16_t f32_to_bits_chk(float v, int dt, bool chk, uint32_t &bad) {
+  const uint16_t r = f32_to_bits(v, dt);
+  if (chk && (r & 0x7C00u) == 0x7C00u && !isinf(v)) bad = 1;
+  return r;
+}
 
 // One CTA per token.  dy rows are written with one rounding of the exact
 // FP32 product; the dots are reduced in a fixed tree (per thread, warp, CTA).
@@ -145,6 +155,8 @@ __global__ void __launch_bounds__(kCombThreads) combine_bwd_kernel(CombineBwdPar
   const uint16_t *y = static_cast<const uint16_t *>(p.y);
   uint16_t *dy = static_cast<uint16_t *>(p.dy);
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const bool chk = p.odt == MOE_F16 && p.dt == MOE_BF16;
+  uint32_t bad = 0;
   for (int j = 0; j < p.k; ++j) {
     int32_t r = p.row_of[t * p.k + j];
     const bool ok = r >= 0 && (int64_t)r < p.A;
@@ -165,8 +177,8 @@ __global__ void __launch_bounds__(kCombThreads) combine_bwd_kernel(CombineBwdPar
           uint32_t o[4];
 #pragma unroll
           for (int i = 0; i < 4; ++i)
-            o[i] = uint32_t(f32_to_bits(__fmul_rn(w, gf[2 * i]), p.dt)) |
-                   (uint32_t(f32_to_bits(__fmul_rn(w, gf[2 * i + 1]), p.dt)) << 16);
+            o[i] = uint32_t(f32_to_bits_chk(__fmul_rn(w, gf[2 * i]), p.odt, chk, bad)) |
+                   (uint32_t(f32_to_bits_chk(__fmul_rn(w, gf[2 * i + 1]), p.odt, chk, bad)) << 16);
           *reinterpret_cast<uint4 *>(dy + (int64_t)r * p.H + c0) = make_uint4(o[0], o[1], o[2], o[3]);
         }
         if (p.dweights) {
@@ -182,7 +194,7 @@ __global__ void __launch_bounds__(kCombThreads) combine_bwd_kernel(CombineBwdPar
     } else if (ok) {
       for (int64_t c = threadIdx.x; c < p.H; c += blockDim.x) {
         float gv = bits_to_f32(g[t * p.H + c], p.dt);
-        if (dy) dy[(int64_t)r * p.H + c] = f32_to_bits(__fmul_rn(w, gv), p.dt);
+        if (dy) dy[(int64_t)r * p.H + c] = f32_to_bits_chk(__fmul_rn(w, gv), p.odt, chk, bad);
         if (p.dweights) dot = fmaf(gv, bits_to_f32(y[(int64_t)r * p.H + c], p.dt), dot);
       }
     }
@@ -192,6 +204,7 @@ __global__ void __launch_bounds__(kCombThreads) combine_bwd_kernel(CombineBwdPar
       if (lane == 0) red[warp][j] = dot;
     }
   }
+  if (bad) report(p.status, MOE_DEVICE_ERR_ACT_RANGE);
   if (!p.dweights) return;
   __syncthreads();
   if (threadIdx.x < p.k) {
@@ -207,6 +220,8 @@ struct SwigluBwdParams {
   int dt;
   int64_t n;
   int vec;  // all five tensors 16-byte aligned: 8 elements per access
+  int odt;  // dtype of dG and dU
+  int32_t *status;
 };
 
 // sigma = 1/(1+e^-G); dG = dh U sigma (1 + G (1 - sigma)), dU = dh G sigma, each
@@ -221,6 +236,8 @@ __device__ __forceinline__ void swiglu_bwd1(float d, float g, float u, float &dg
 __global__ void __launch_bounds__(256) swiglu_bwd_kernel(SwigluBwdParams p) {
   const int64_t n8 = p.vec ? p.n / 8 : 0;
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  const bool chk = p.odt == MOE_F16 && p.dt == MOE_BF16;
+  uint32_t bad = 0;
   for (int64_t v = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; v < n8; v += stride) {
     const uint4 dv = reinterpret_cast<const uint4 *>(p.dh)[v];
     const uint4 gv = reinterpret_cast<const uint4 *>(p.G)[v];
@@ -234,8 +251,8 @@ __global__ void __launch_bounds__(256) swiglu_bwd_kernel(SwigluBwdParams p) {
                   bits_to_f32(uint16_t(ua[i] & 0xFFFF), p.dt), dg0, du0);
       swiglu_bwd1(bits_to_f32(uint16_t(da[i] >> 16), p.dt), bits_to_f32(uint16_t(ga[i] >> 16), p.dt),
                   bits_to_f32(uint16_t(ua[i] >> 16), p.dt), dg1, du1);
-      og[i] = uint32_t(f32_to_bits(dg0, p.dt)) | (uint32_t(f32_to_bits(dg1, p.dt)) << 16);
-      ou[i] = uint32_t(f32_to_bits(du0, p.dt)) | (uint32_t(f32_to_bits(du1, p.dt)) << 16);
+      og[i] = uint32_t(f32_to_bits_chk(dg0, p.odt, chk, bad)) | (uint32_t(f32_to_bits_chk(dg1, p.odt, chk, bad)) << 16);
+      ou[i] = uint32_t(f32_to_bits_chk(du0, p.odt, chk, bad)) | (uint32_t(f32_to_bits_chk(du1, p.odt, chk, bad)) << 16);
     }
     reinterpret_cast<uint4 *>(p.dG)[v] = make_uint4(og[0], og[1], og[2], og[3]);
     reinterpret_cast<uint4 *>(p.dU)[v] = make_uint4(ou[0], ou[1], ou[2], ou[3]);
@@ -244,9 +261,10 @@ __global__ void __launch_bounds__(256) swiglu_bwd_kernel(SwigluBwdParams p) {
   for (int64_t i = n8 * 8 + (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < p.n; i += stride) {
     float dg, du;
     swiglu_bwd1(bits_to_f32(p.dh[i], p.dt), bits_to_f32(p.G[i], p.dt), bits_to_f32(p.U[i], p.dt), dg, du);
-    p.dG[i] = f32_to_bits(dg, p.dt);
-    p.dU[i] = f32_to_bits(du, p.dt);
+    p.dG[i] = f32_to_bits_chk(dg, p.odt, chk, bad);
+    p.dU[i] = f32_to_bits_chk(du, p.odt, chk, bad);
   }
+  if (bad) report(p.status, MOE_DEVICE_ERR_ACT_RANGE);
 }
 
 static moe_status launch_combine(const CombineParams &p, cudaStream_t st, const char *what) {
@@ -298,18 +316,21 @@ extern "C" moe_status moe_dispatch_backward(const void *dvalues, moe_dtype act_d
   return launch_combine(p, as_stream(stream), "moe_dispatch_backward");
 }
 
-extern "C" moe_status moe_combine_backward(const void *d_out, const void *y, moe_dtype act_dtype, int64_t A,
-                                           const float *weights, const int32_t *row_of, int64_t T, int64_t H,
-                                           int32_t top_k, void *dy, float *dweights, int32_t *device_status,
-                                           void *stream) {
+extern "C" moe_status moe_combine_backward_dt(const void *d_out, const void *y, moe_dtype act_dtype, int64_t A,
+                                              const float *weights, const int32_t *row_of, int64_t T, int64_t H,
+                                              int32_t top_k, void *dy, moe_dtype dy_dtype, float *dweights,
+                                              int32_t *device_status, void *stream) {
   moe_status s = check_tk("moe_combine_backward", T, H, top_k, A);
   if (s != MOE_OK) return s;
   if (act_dtype != MOE_F16 && act_dtype != MOE_BF16)
     return set_error(MOE_ERR_UNSUPPORTED_DTYPE, "moe_combine_backward: act_dtype must be F16 or BF16");
+  if (dy_dtype != MOE_F16 && dy_dtype != MOE_BF16)
+    return set_error(MOE_ERR_UNSUPPORTED_DTYPE, "moe_combine_backward: dy_dtype must be F16 or BF16");
   if (T == 0 || (!dy && !dweights)) return MOE_OK;
   if (!d_out || !weights || !row_of || (dweights && !y))
     return set_error(MOE_ERR_INVALID_ARGUMENT, "moe_combine_backward: NULL tensor pointer");
-  CombineBwdParams p{d_out, y, (int)act_dtype, A, weights, row_of, T, H, top_k, dy, dweights, device_status};
+  CombineBwdParams p{d_out, y, (int)act_dtype, A, weights, row_of, T, H, top_k, dy, dweights, device_status,
+                     (int)dy_dtype};
   const bool vec = H % 8 == 0 && aligned16(d_out) && (!dy || aligned16(dy)) && (!dweights || aligned16(y));
   if (vec)
     combine_bwd_kernel<true><<<(unsigned)T, kCombThreads, 0, as_stream(stream)>>>(p);
@@ -318,16 +339,27 @@ extern "C" moe_status moe_combine_backward(const void *d_out, const void *y, moe
   return check_launch("moe_combine_backward");
 }
 
-extern "C" moe_status moe_swiglu_backward(const void *dh, const void *G, const void *U, moe_dtype act_dtype,
-                                          int64_t A, int64_t I, void *dG, void *dU, void *stream) {
+extern "C" moe_status moe_combine_backward(const void *d_out, const void *y, moe_dtype act_dtype, int64_t A,
+                                           const float *weights, const int32_t *row_of, int64_t T, int64_t H,
+                                           int32_t top_k, void *dy, float *dweights, int32_t *device_status,
+                                           void *stream) {
+  return moe_combine_backward_dt(d_out, y, act_dtype, A, weights, row_of, T, H, top_k, dy, act_dtype, dweights,
+                                 device_status, stream);
+}
+
+extern "C" moe_status moe_swiglu_backward_dt(const void *dh, const void *G, const void *U, moe_dtype act_dtype,
+                                             int64_t A, int64_t I, void *dG, void *dU, moe_dtype grad_dtype,
+                                             int32_t *device_status, void *stream) {
   if (A < 0 || I < 1) return set_error(MOE_ERR_INVALID_ARGUMENT, "moe_swiglu_backward: bad sizes");
   if (act_dtype != MOE_F16 && act_dtype != MOE_BF16)
     return set_error(MOE_ERR_UNSUPPORTED_DTYPE, "moe_swiglu_backward: act_dtype must be F16 or BF16");
+  if (grad_dtype != MOE_F16 && grad_dtype != MOE_BF16)
+    return set_error(MOE_ERR_UNSUPPORTED_DTYPE, "moe_swiglu_backward: grad_dtype must be F16 or BF16");
   if (A == 0) return MOE_OK;
   if (!dh || !G || !U || !dG || !dU) return set_error(MOE_ERR_INVALID_ARGUMENT, "moe_swiglu_backward: NULL pointer");
   SwigluBwdParams p{static_cast<const uint16_t *>(dh), static_cast<const uint16_t *>(G),
                     static_cast<const uint16_t *>(U), static_cast<uint16_t *>(dG), static_cast<uint16_t *>(dU),
-                    (int)act_dtype, A * I, 0};
+                    (int)act_dtype, A * I, 0, (int)grad_dtype, device_status};
   p.vec = aligned16(dh) && aligned16(G) && aligned16(U) && aligned16(dG) && aligned16(dU);
   int64_t blocks = (p.n / (p.vec ? 8 : 1) + 255) / 256;
   int64_t cap = (int64_t)num_sms() * 8;
@@ -335,4 +367,9 @@ extern "C" moe_status moe_swiglu_backward(const void *dh, const void *G, const v
   if (blocks < 1) blocks = 1;
   swiglu_bwd_kernel<<<(unsigned)blocks, 256, 0, as_stream(stream)>>>(p);
   return check_launch("moe_swiglu_backward");
+}
+
+extern "C" moe_status moe_swiglu_backward(const void *dh, const void *G, const void *U, moe_dtype act_dtype,
+                                          int64_t A, int64_t I, void *dG, void *dU, void *stream) {
+  return moe_swiglu_backward_dt(dh, G, U, act_dtype, A, I, dG, dU, act_dtype, nullptr, stream);
 }

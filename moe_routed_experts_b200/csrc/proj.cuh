@@ -45,7 +45,8 @@ struct BwdParams {
   int group;
   uint16_t *out;  // [A, K]
   int32_t *status;
-  int preconv;  // grad holds F16 copies of BF16 gradients (gdt stays the output dtype)
+  int preconv;  // grad holds F16 copies of BF16 gradients
+  int odt;      // dtype of out (F16 or BF16), independent of the gradients'
 };
 
 // Row of x that batch row r reads: r itself, or gather[r] (an index outside

@@ -4,7 +4,8 @@
 awq_grouped_down -> moe_combine; ``backward`` = moe_combine_backward ->
 awq_input_backward(down) -> moe_swiglu_backward -> awq_input_backward(gate
 + up, one accumulation) -> moe_dispatch_backward, and moe_router_backward
-for the router logits.  Only argument marshalling happens here; every step
+for the router logits (the ``_dt`` forms of the first three, writing the
+gradients that feed an input VJP in its scale dtype).  Only argument marshalling happens here; every step
 runs in the library's kernels.
 """
 from dataclasses import dataclass
@@ -124,16 +125,28 @@ def forward(dev: dict, buf: Buffers, gather: bool = False) -> torch.Tensor:
     return buf.out
 
 
+def chain_grad_dtype(scale_dtype: str, act_dtype: str = "bf16") -> str:
+    """dtype of the gradients that feed the input VJPs (dy, dG, dU).
+
+    The input VJPs run their products in the scale dtype, so with F16 scales
+    the steps before them write F16 directly (one rounding of the FP32
+    value) instead of the activation dtype plus a conversion pass; the
+    gradients of the activations (dh, dvalues, dx) stay in act_dtype."""
+    return "f16" if scale_dtype == "f16" else act_dtype
+
+
 def backward(dev: dict, buf: Buffers, d_out: torch.Tensor) -> dict:
     """Input VJP of the forward held in ``buf`` (needs G and U kept)."""
     w = dev["workload"]
     r = buf.route
     assert buf.G is not None and buf.U is not None, "allocate with keep_gu=True"
-    dy, dw = B.moe_combine_backward(d_out, buf.y, r["weights"], r["row_of"], device_status=buf.status)
-    dh = B.awq_input_backward(dy, r["offsets"], dev["down"], w.group, device_status=buf.status)
-    dG, dU = B.moe_swiglu_backward(dh, buf.G, buf.U)
+    act = buf.y.dtype
+    gdt = _SDT[chain_grad_dtype(w.scale_dtype, "bf16" if act == torch.bfloat16 else "f16")]
+    dy, dw = B.moe_combine_backward(d_out, buf.y, r["weights"], r["row_of"], device_status=buf.status, dy_dtype=gdt)
+    dh = B.awq_input_backward(dy, r["offsets"], dev["down"], w.group, device_status=buf.status, out_dtype=act)
+    dG, dU = B.moe_swiglu_backward(dh, buf.G, buf.U, out_dtype=gdt, device_status=buf.status)
     dvalues = B.awq_input_backward(dG, r["offsets"], dev["gate"], w.group, grad2=dU, proj2=dev["up"],
-                                   device_status=buf.status)
+                                   device_status=buf.status, out_dtype=act)
     dx = B.moe_dispatch_backward(dvalues, r["row_of"], r["selected_experts"], device_status=buf.status)
     dlogits = B.moe_router_backward(dev["logits"], r["selected_experts"], dw, renormalize=w.renormalize,
                                     expert_start=w.expert_start, device_status=buf.status)

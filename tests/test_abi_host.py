@@ -100,6 +100,25 @@ def test_combine_family_rejects_bad_arguments(L):
     assert L.moe_swiglu_backward(FAKE, FAKE, FAKE, B.MOE_BF16, -1, 8, FAKE, FAKE, None) == 1
 
 
+def test_dtype_choosing_backward_forms_reject_bad_dtypes(L):
+    # the _dt forms check the output dtype on the host (2 = unsupported dtype)
+    assert L.moe_combine_backward_dt(FAKE, FAKE, B.MOE_BF16, 8, FAKE, FAKE, 4, 16, 2, FAKE, B.MOE_F32, None, None,
+                                     None) == 2
+    assert L.moe_combine_backward_dt(FAKE, FAKE, B.MOE_BF16, 8, FAKE, FAKE, 4, 16, 0, FAKE, B.MOE_F16, None, None,
+                                     None) == 1
+    assert L.moe_combine_backward_dt(FAKE, FAKE, B.MOE_BF16, 8, FAKE, FAKE, 0, 16, 2, FAKE, B.MOE_F16, None, None,
+                                     None) == 0
+    assert L.moe_swiglu_backward_dt(FAKE, FAKE, FAKE, B.MOE_BF16, 4, 8, FAKE, FAKE, B.MOE_F32, None, None) == 2
+    assert L.moe_swiglu_backward_dt(FAKE, FAKE, FAKE, B.MOE_BF16, -1, 8, FAKE, FAKE, B.MOE_F16, None, None) == 1
+    assert L.moe_swiglu_backward_dt(FAKE, FAKE, FAKE, B.MOE_BF16, 0, 8, FAKE, FAKE, B.MOE_F16, None, None) == 0
+    assert L.awq_input_backward_dt(FAKE, B.MOE_F16, 4, 16, 64, FAKE, 1, FAKE, FAKE, FAKE, B.MOE_F16, 16, None, None,
+                                   None, None, FAKE, B.MOE_F32, None, 0, None, None) == 2
+    assert L.awq_input_backward_dt(FAKE, B.MOE_F16, 4, 16, 64, FAKE, 1, FAKE, FAKE, FAKE, B.MOE_F16, 48, None, None,
+                                   None, None, FAKE, B.MOE_BF16, None, 0, None, None) == 1
+    assert L.awq_input_backward_dt(FAKE, B.MOE_F16, 0, 16, 64, FAKE, 1, FAKE, FAKE, FAKE, B.MOE_F16, 16, None, None,
+                                   None, None, FAKE, B.MOE_BF16, None, 0, None, None) == 0
+
+
 def test_projection_path_knob(L):
     assert L.moe_set_projection_path(7) == -1
     prev = L.moe_set_projection_path(1)

@@ -46,23 +46,28 @@ def _chain(name, kw, rows=None, tokens=None):
         rows = np.arange(w.A)
     if tokens is None:
         tokens = np.arange(w.T)
+    # the chain writes dy, dG and dU in the scale dtype when it is F16
+    cdt = ffn.chain_grad_dtype(w.scale_dtype)
+    assert g["dy"].dtype == g["dG"].dtype == g["dU"].dtype == ffn._SDT[cdt]
+    assert g["dh"].dtype == g["dvalues"].dtype == g["dx"].dtype == torch.bfloat16
     # combine VJP on the sampled tokens
-    o_dy, o_dw = oracle.combine_backward(dout[tokens], y, "bf16", wts[tokens], row_of[tokens])
+    o_dy, o_dw = oracle.combine_backward(dout[tokens], y, "bf16", wts[tokens], row_of[tokens], dy_dt=cdt)
     dy_rows = row_of[tokens].reshape(-1)
-    check_close(dy[dy_rows], o_dy[dy_rows], name + "/dy",
+    check_close(dy[dy_rows], o_dy[dy_rows], name + "/dy", dt=cdt,
                 justify=j_combine_backward_dy(dout[tokens], "bf16", wts[tokens], row_of[tokens], dy_rows))
     assert np.max(np.abs(dw[tokens] - o_dw)) <= 2e-2 * np.sqrt(np.mean(o_dw.astype(np.float64) ** 2)), "dweights"
     # down input VJP, SwiGLU VJP, gate+up input VJP on the sampled rows
     re = rexp_all[rows]
     sdt, gs = w.scale_dtype, w.group
-    o_dh = oracle.input_backward(dy[rows], "bf16", re, inp["down"], sdt, gs)
-    check_close(dh[rows], o_dh, name + "/dh", justify=j_input_backward(dy[rows], "bf16", re, inp["down"], sdt, gs))
-    o_dG, o_dU = oracle.swiglu_backward(dh[rows], G[rows], U[rows])
-    check_close(dG[rows], o_dG, name + "/dG", justify=j_swiglu_backward(dh[rows], G[rows], U[rows], which=0))
-    check_close(dU[rows], o_dU, name + "/dU", justify=j_swiglu_backward(dh[rows], G[rows], U[rows], which=1))
-    o_dv = oracle.input_backward(dG[rows], "bf16", re, inp["gate"], sdt, gs, grad2=dU[rows], proj2=inp["up"])
+    o_dh = oracle.input_backward(dy[rows], cdt, re, inp["down"], sdt, gs, odt="bf16")
+    check_close(dh[rows], o_dh, name + "/dh", justify=j_input_backward(dy[rows], cdt, re, inp["down"], sdt, gs))
+    o_dG, o_dU = oracle.swiglu_backward(dh[rows], G[rows], U[rows], "bf16", odt=cdt)
+    check_close(dG[rows], o_dG, name + "/dG", dt=cdt, justify=j_swiglu_backward(dh[rows], G[rows], U[rows], which=0))
+    check_close(dU[rows], o_dU, name + "/dU", dt=cdt, justify=j_swiglu_backward(dh[rows], G[rows], U[rows], which=1))
+    o_dv = oracle.input_backward(dG[rows], cdt, re, inp["gate"], sdt, gs, grad2=dU[rows], proj2=inp["up"],
+                                 odt="bf16")
     check_close(dv[rows], o_dv, name + "/dvalues",
-                justify=j_input_backward(dG[rows], "bf16", re, inp["gate"], sdt, gs, dU[rows], inp["up"]))
+                justify=j_input_backward(dG[rows], cdt, re, inp["gate"], sdt, gs, dU[rows], inp["up"]))
     o_dx = oracle.dispatch_backward(dv, "bf16", sel[tokens], row_of[tokens])
     check_close(dx[tokens], o_dx, name + "/dx", justify=j_dispatch_backward(dv, "bf16", sel[tokens], row_of[tokens]))
     # router-logit VJP from the device dweights (FP32 softmax algebra)
@@ -143,18 +148,19 @@ def test_whole_chain_against_oracle_chain():
     torch.cuda.synchronize()
     f = oracle.forward(inp)
     rexp = (f["row_experts"].astype(np.int64) - w.expert_start).astype(np.int32)
-    o_dy, o_dw = oracle.combine_backward(inp["d_out"], f["y"], "bf16", f["weights"], f["row_of"])
-    o_dh = oracle.input_backward(o_dy, "bf16", rexp, inp["down"], w.scale_dtype, w.group)
-    o_dG, o_dU = oracle.swiglu_backward(o_dh, f["G"], f["U"])
-    o_dv = oracle.input_backward(o_dG, "bf16", rexp, inp["gate"], w.scale_dtype, w.group, grad2=o_dU,
-                                 proj2=inp["up"])
+    cdt = ffn.chain_grad_dtype(w.scale_dtype)  # dy, dG, dU: F16 with F16 scales
+    o_dy, o_dw = oracle.combine_backward(inp["d_out"], f["y"], "bf16", f["weights"], f["row_of"], dy_dt=cdt)
+    o_dh = oracle.input_backward(o_dy, cdt, rexp, inp["down"], w.scale_dtype, w.group, odt="bf16")
+    o_dG, o_dU = oracle.swiglu_backward(o_dh, f["G"], f["U"], "bf16", odt=cdt)
+    o_dv = oracle.input_backward(o_dG, cdt, rexp, inp["gate"], w.scale_dtype, w.group, grad2=o_dU,
+                                 proj2=inp["up"], odt="bf16")
     o_dx = oracle.dispatch_backward(o_dv, "bf16", f["selected"], f["row_of"])
     # end to end: a flip is justified by the last step's FP32 bound plus the
     # measured difference between the exact values on the device's upstream
     # tensors and on the oracle's (each step is checked on its own elsewhere)
     dG, dU, dv = bits(g["dG"]), bits(g["dU"]), bits(g["dvalues"])
-    j_dv = j_chain(j_input_backward(o_dG, "bf16", rexp, inp["gate"], w.scale_dtype, w.group, o_dU, inp["up"]),
-                   j_input_backward(dG, "bf16", rexp, inp["gate"], w.scale_dtype, w.group, dU, inp["up"]))
+    j_dv = j_chain(j_input_backward(o_dG, cdt, rexp, inp["gate"], w.scale_dtype, w.group, o_dU, inp["up"]),
+                   j_input_backward(dG, cdt, rexp, inp["gate"], w.scale_dtype, w.group, dU, inp["up"]))
     j_dx = j_chain(j_dispatch_backward(o_dv, "bf16", f["selected"], f["row_of"]),
                    j_dispatch_backward(dv, "bf16", f["selected"], f["row_of"]))
     check_close(bits(g["dx"]), o_dx, "chain/dx", justify=j_dx)

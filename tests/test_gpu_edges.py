@@ -10,7 +10,7 @@ import torch
 
 import oracle
 from helpers import (bits, check_close, check_forward_steps, check_routing, gpu_forward_numpy, j_chain,
-                     j_input_backward, j_project, j_swiglu)
+                     j_input_backward, j_project, j_swiglu, j_swiglu_backward)
 from moe_routed_experts_b200 import binding as B
 from moe_routed_experts_b200 import ffn, inputs
 from moe_routed_experts_b200.configs import Workload
@@ -182,6 +182,66 @@ def test_f16_range_overflow_is_flagged(value, flagged, path):
     B.awq_input_backward(gr, off, dproj, g, device_status=st)
     torch.cuda.synchronize()
     assert int(st.item()) == want, int(st.item())
+
+
+def _bf16_cuda(a):
+    return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).cuda()
+
+
+@pytest.mark.parametrize("value,flagged", [(4.0e5, True), (float("nan"), True), (float("inf"), False),
+                                           (1.2e5, False)],
+                         ids=["overflow", "nan", "inf_stays_inf", "in_range"])
+def test_f16_dy_from_bf16_inputs(value, flagged):
+    # moe_combine_backward writing F16 dy from BF16 inputs: one rounding of
+    # the FP32 product, bit for bit the oracle's F16 rounding here (w = 0.5
+    # makes the product exact), and a value that is not inf but overflows
+    # F16 (or a NaN) is reported like the BF16 -> F16 input conversion
+    rng = np.random.default_rng(5)
+    T, H, k = 6, 72, 2
+    A = T * k
+    d_out = inputs.random_bf16(rng, (T, H))
+    y = inputs.random_bf16(rng, (A, H))
+    wts = np.full((T, k), 0.5, np.float32)
+    row_of = np.arange(A, dtype=np.int32).reshape(T, k)
+    args = (_bf16_cuda(y), torch.from_numpy(wts).cuda(), torch.from_numpy(row_of).cuda())
+    for planted in (False, True):
+        if planted:
+            d_out[3, 17] = bits(torch.tensor([value], dtype=torch.bfloat16))[0]
+        st = B.new_status()
+        dy, _ = B.moe_combine_backward(_bf16_cuda(d_out), *args, device_status=st, dy_dtype=torch.float16)
+        torch.cuda.synchronize()
+        assert dy.dtype == torch.float16
+        assert int(st.item()) == (16 if planted and flagged else 0), int(st.item())
+        o_dy, _ = oracle.combine_backward(d_out, y, "bf16", wts, row_of, dy_dt="f16")
+        got = bits(dy)
+        same = (got == o_dy) | (np.isnan(got.view(np.float16)) & np.isnan(o_dy.view(np.float16)))
+        assert np.all(same)
+
+
+@pytest.mark.parametrize("value,flagged", [(2.0e5, True), (float("nan"), True), (float("inf"), False),
+                                           (6.0e4, False)],
+                         ids=["overflow", "nan", "inf_stays_inf", "in_range"])
+def test_f16_swiglu_grads_from_bf16_inputs(value, flagged):
+    # moe_swiglu_backward writing F16 dG/dU from BF16 dh, G, U; at G = 0.5,
+    # U = 1 the planted dh gives dG = 0.74 dh and dU = 0.31 dh
+    rng = np.random.default_rng(6)
+    A, I = 16, 40
+    dh, G, U = (inputs.random_bf16(rng, (A, I)) for _ in range(3))
+    G[2, 3] = bits(torch.tensor([0.5], dtype=torch.bfloat16))[0]
+    U[2, 3] = bits(torch.tensor([1.0], dtype=torch.bfloat16))[0]
+    for planted in (False, True):
+        if planted:
+            dh[2, 3] = bits(torch.tensor([value], dtype=torch.bfloat16))[0]
+        st = B.new_status()
+        dG, dU = B.moe_swiglu_backward(_bf16_cuda(dh), _bf16_cuda(G), _bf16_cuda(U), out_dtype=torch.float16,
+                                       device_status=st)
+        torch.cuda.synchronize()
+        assert dG.dtype == dU.dtype == torch.float16
+        assert int(st.item()) == (16 if planted and flagged else 0), int(st.item())
+        if not planted:
+            o_dG, o_dU = oracle.swiglu_backward(dh, G, U, "bf16", odt="f16")
+            check_close(bits(dG), o_dG, "swiglu_dt/dG", dt="f16", justify=j_swiglu_backward(dh, G, U, which=0))
+            check_close(bits(dU), o_dU, "swiglu_dt/dU", dt="f16", justify=j_swiglu_backward(dh, G, U, which=1))
 
 
 def test_row_index_out_of_range_is_flagged():

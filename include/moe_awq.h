@@ -93,7 +93,7 @@ typedef enum { MOE_F32 = 0, MOE_F16 = 1, MOE_BF16 = 2 } moe_dtype;
 #define MOE_DEVICE_ERR_ACT_RANGE 16   /* a BF16 activation or gradient fed to F16-scale tensor cores was
                                          finite above F16's range (|v| > 65504: it became inf) or NaN;
                                          the result is computed from the converted value.  Also set by
-                                         the _dt backward steps that write F16 from BF16 inputs */
+                                         the _dt steps that write F16 from BF16 inputs */
 
 /* Limits of this implementation. */
 #define MOE_MAX_EXPERTS 4096
@@ -153,6 +153,20 @@ MOE_API moe_status moe_route_dispatch(const void *x, moe_dtype x_dtype, int64_t 
                               uint32_t *row_experts, int32_t *offsets, int32_t *src_token,
                               int32_t *row_of, void *workspace, size_t workspace_bytes,
                               int32_t *device_status, void *stream);
+
+/* moe_route_dispatch with the rows of values stored in values_dtype: x_dtype
+ * (the COPY itself), or F16 for BF16 x, the operand dtype of projections
+ * with F16 scales, so they take the rows without a conversion pass (exact in
+ * F16's normal range; a finite value above it, or a NaN, sets
+ * MOE_DEVICE_ERR_ACT_RANGE, as the projections' own conversion does).  Any
+ * other pair gives MOE_ERR_UNSUPPORTED_DTYPE. */
+MOE_API moe_status moe_route_dispatch_dt(const void *x, moe_dtype x_dtype, int64_t T, int64_t H,
+                                 const float *logits, const float *sel_bias, int64_t E,
+                                 int32_t expert_start, int32_t top_k, int32_t renormalize,
+                                 void *values, moe_dtype values_dtype, float *weights,
+                                 uint32_t *selected_experts, uint32_t *row_experts, int32_t *offsets,
+                                 int32_t *src_token, int32_t *row_of, void *workspace,
+                                 size_t workspace_bytes, int32_t *device_status, void *stream);
 
 /* ------------------------------------------------------------------------
  * moe_route -- the routing and row maps of moe_route_dispatch without the
@@ -240,6 +254,22 @@ MOE_API moe_status awq_grouped_gate_up_swiglu(
     moe_dtype scale_dtype, moe_dtype bias_dtype, int64_t group_size,
     void *h, void *gate_out, void *up_out, void *workspace, size_t workspace_bytes,
     int32_t *device_status, void *stream);
+
+/* awq_grouped_gate_up_swiglu with h, gate_out and up_out stored in out_dtype
+ * (F16 or BF16) instead of act_dtype: the same FP32 sums, one rounding to
+ * out_dtype, SwiGLU from the rounded G and U.  F16 values from
+ * moe_route_dispatch_dt with F16 scales give BF16 outputs without a
+ * conversion pass. */
+MOE_API moe_status awq_grouped_gate_up_swiglu_dt(
+    const void *values, moe_dtype act_dtype, int64_t A, int64_t H, int64_t I,
+    const int32_t *offsets, int64_t E,
+    const int32_t *qweight_gate, const int32_t *qzeros_gate, const void *scales_gate,
+    const void *bias_gate,
+    const int32_t *qweight_up, const int32_t *qzeros_up, const void *scales_up,
+    const void *bias_up,
+    moe_dtype scale_dtype, moe_dtype bias_dtype, int64_t group_size,
+    void *h, void *gate_out, void *up_out, moe_dtype out_dtype, void *workspace,
+    size_t workspace_bytes, int32_t *device_status, void *stream);
 
 /* ------------------------------------------------------------------------
  * awq_grouped_gate_up_swiglu_gather -- awq_grouped_gate_up_swiglu on rows

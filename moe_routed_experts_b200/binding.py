@@ -59,6 +59,10 @@ _SIGS = {
     "awq_input_backward": (C.c_int, [P, C.c_int, I64, I64, I64, P, I64, P, P, P, C.c_int, I64, P, P, P, P, P, P, SZ,
                                      P, P]),
     "moe_swiglu_backward": (C.c_int, [P, P, P, C.c_int, I64, I64, P, P, P]),
+    "moe_route_dispatch_dt": (C.c_int, [P, C.c_int, I64, I64, P, P, I64, I32, I32, I32, P, C.c_int, P, P, P, P, P,
+                                         P, P, SZ, P, P]),
+    "awq_grouped_gate_up_swiglu_dt": (C.c_int, [P, C.c_int, I64, I64, I64, P, I64, P, P, P, P, P, P, P, P, C.c_int,
+                                                C.c_int, I64, P, P, P, C.c_int, P, SZ, P, P]),
     "moe_combine_backward_dt": (C.c_int, [P, P, C.c_int, I64, P, P, I64, I64, I32, P, C.c_int, P, P, P]),
     "awq_input_backward_dt": (C.c_int, [P, C.c_int, I64, I64, I64, P, I64, P, P, P, C.c_int, I64, P, P, P, P, P,
                                         C.c_int, P, SZ, P, P]),
@@ -137,14 +141,20 @@ def route_dispatch_workspace_size(T, E, top_k):
 
 
 def moe_route_dispatch(x, logits, top_k, E=None, sel_bias=None, expert_start=0, renormalize=1, workspace=None,
-                       device_status=None, out=None):
+                       device_status=None, out=None, values_dtype=None):
+    """Routing, row maps and the expert-sorted rows in values_dtype (default:
+    x's dtype; F16 for BF16 x converts while copying; ``out["values"]``'s
+    dtype when out is given)."""
     T, H = x.shape
     E = E if E is not None else logits.shape[1]
     A = T * top_k
     dev = x.device
+    if out is not None:
+        values_dtype = out["values"].dtype
+    values_dtype = values_dtype or x.dtype
     if out is None:
         out = {
-            "values": torch.empty((A, H), dtype=x.dtype, device=dev),
+            "values": torch.empty((A, H), dtype=values_dtype, device=dev),
             "weights": torch.empty((T, top_k), dtype=torch.float32, device=dev),
             "selected_experts": torch.empty((T, top_k), dtype=torch.int32, device=dev),
             "row_experts": torch.empty((A,), dtype=torch.int32, device=dev),
@@ -154,11 +164,11 @@ def moe_route_dispatch(x, logits, top_k, E=None, sel_bias=None, expert_start=0, 
         }
     if workspace is None:
         workspace = torch.empty(max(route_dispatch_workspace_size(T, E, top_k), 256), dtype=torch.uint8, device=dev)
-    st = lib().moe_route_dispatch(
+    st = lib().moe_route_dispatch_dt(
         _ptr(x), _dt(x.dtype), T, H, _ptr(logits), _ptr(sel_bias), E, expert_start, top_k, renormalize,
-        _ptr(out["values"]), _ptr(out["weights"]), _ptr(out["selected_experts"]), _ptr(out["row_experts"]),
-        _ptr(out["offsets"]), _ptr(out["src_token"]), _ptr(out["row_of"]), _ptr(workspace), workspace.numel(),
-        _ptr(device_status), _stream())
+        _ptr(out["values"]), _dt(values_dtype), _ptr(out["weights"]), _ptr(out["selected_experts"]),
+        _ptr(out["row_experts"]), _ptr(out["offsets"]), _ptr(out["src_token"]), _ptr(out["row_of"]), _ptr(workspace),
+        workspace.numel(), _ptr(device_status), _stream())
     _check("moe_route_dispatch", st)
     return out
 
@@ -231,21 +241,25 @@ def _workspace(nbytes, device, workspace=None):
 
 
 def awq_grouped_gate_up_swiglu(values, offsets, gate, up, group, want_gu=False, device_status=None, out=None,
-                               workspace=None):
+                               workspace=None, out_dtype=None):
+    """h (and G, U) in out_dtype (default: values' dtype; ``out``'s dtype when given)."""
     A, H = values.shape
     E = offsets.numel() - 1
     I = gate["qweight"].shape[2] * 8
     sdt = _dt(gate["scales"].dtype)
-    h = out if out is not None else torch.empty((A, I), dtype=values.dtype, device=values.device)
+    if out is not None:
+        out_dtype = out.dtype
+    out_dtype = out_dtype or values.dtype
+    h = out if out is not None else torch.empty((A, I), dtype=out_dtype, device=values.device)
     G = torch.empty_like(h) if want_gu else None
     U = torch.empty_like(h) if want_gu else None
     ws = _workspace(projection_workspace_size(A, H, I, E, group, 2, values.dtype, gate["scales"].dtype), values.device,
                     workspace)
-    st = lib().awq_grouped_gate_up_swiglu(
+    st = lib().awq_grouped_gate_up_swiglu_dt(
         _ptr(values), _dt(values.dtype), A, H, I, _ptr(offsets), E,
         _ptr(gate["qweight"]), _ptr(gate["qzeros"]), _ptr(gate["scales"]), _ptr(gate.get("bias")),
         _ptr(up["qweight"]), _ptr(up["qzeros"]), _ptr(up["scales"]), _ptr(up.get("bias")),
-        sdt, _bias_dt(gate.get("bias"), up.get("bias")), group, _ptr(h), _ptr(G), _ptr(U), _ptr(ws),
+        sdt, _bias_dt(gate.get("bias"), up.get("bias")), group, _ptr(h), _ptr(G), _ptr(U), _dt(out_dtype), _ptr(ws),
         0 if ws is None else ws.numel(), _ptr(device_status), _stream())
     _check("awq_grouped_gate_up_swiglu", st)
     return (h, G, U) if want_gu else h

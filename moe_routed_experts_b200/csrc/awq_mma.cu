@@ -179,21 +179,21 @@ __global__ void __launch_bounds__(128) awq_fwd_mma_kernel(ProjParams p) {
         uint32_t og[4], ou[4];
 #pragma unroll
         for (int i = 0; i < 8; i += 2) {
-          const uint16_t gb0 = f32_to_bits(v[0][i], p.act_dt), gb1 = f32_to_bits(v[0][i + 1], p.act_dt);
-          const uint16_t ub0 = f32_to_bits(v[NPROJ - 1][i], p.act_dt), ub1 = f32_to_bits(v[NPROJ - 1][i + 1], p.act_dt);
-          const float g0 = bits_to_f32(gb0, p.act_dt), g1 = bits_to_f32(gb1, p.act_dt);
-          const float u0 = bits_to_f32(ub0, p.act_dt), u1 = bits_to_f32(ub1, p.act_dt);
+          const uint16_t gb0 = f32_to_bits(v[0][i], p.odt), gb1 = f32_to_bits(v[0][i + 1], p.odt);
+          const uint16_t ub0 = f32_to_bits(v[NPROJ - 1][i], p.odt), ub1 = f32_to_bits(v[NPROJ - 1][i + 1], p.odt);
+          const float g0 = bits_to_f32(gb0, p.odt), g1 = bits_to_f32(gb1, p.odt);
+          const float u0 = bits_to_f32(ub0, p.odt), u1 = bits_to_f32(ub1, p.odt);
           const float h0 = g0 / (1.f + expf(-g0)) * u0, h1 = g1 / (1.f + expf(-g1)) * u1;
           og[i / 2] = uint32_t(gb0) | (uint32_t(gb1) << 16);
           ou[i / 2] = uint32_t(ub0) | (uint32_t(ub1) << 16);
-          o[i / 2] = uint32_t(f32_to_bits(h0, p.act_dt)) | (uint32_t(f32_to_bits(h1, p.act_dt)) << 16);
+          o[i / 2] = uint32_t(f32_to_bits(h0, p.odt)) | (uint32_t(f32_to_bits(h1, p.odt)) << 16);
         }
         if (p.gout) *reinterpret_cast<uint4 *>(p.gout + row * p.N + n0) = make_uint4(og[0], og[1], og[2], og[3]);
         if (p.uout) *reinterpret_cast<uint4 *>(p.uout + row * p.N + n0) = make_uint4(ou[0], ou[1], ou[2], ou[3]);
       } else {
 #pragma unroll
         for (int i = 0; i < 8; i += 2)
-          o[i / 2] = uint32_t(f32_to_bits(v[0][i], p.act_dt)) | (uint32_t(f32_to_bits(v[0][i + 1], p.act_dt)) << 16);
+          o[i / 2] = uint32_t(f32_to_bits(v[0][i], p.odt)) | (uint32_t(f32_to_bits(v[0][i + 1], p.odt)) << 16);
       }
       *reinterpret_cast<uint4 *>(p.out + row * p.N + n0) = make_uint4(o[0], o[1], o[2], o[3]);
     }

@@ -362,7 +362,7 @@ __global__ void __launch_bounds__(tc2::kThreads, 1)
     const int q = warp & 3;                     // TMEM lane quarter
     const int hf = (warp - 2 - kDqWarps) >> 2;  // column half drained by this warp
     const int et = threadIdx.x - (2 + kDqWarps) * 32;  // 0 .. 255
-    const bool bf = p.act_dt == MOE_BF16;
+    const bool bf = p.odt == MOE_BF16;
     uint32_t tcount = 0;
     for (int64_t tile = pair; tile < total; tile += npairs, ++tcount) {
       const PairTile ti = tile_info(tile);

@@ -280,6 +280,7 @@ struct ScatterParams {
   int32_t *src_token;
   int vec16;
   int64_t nseg;  // copy segments per row
+  int32_t *status;
 };
 
 // Row position of assignment a = t*k + j and, on its first visit, the row maps.
@@ -298,7 +299,11 @@ __device__ __forceinline__ int64_t scatter_pos(const ScatterParams &p, int64_t a
 
 // 16-byte rows: one warp per assignment (grid-stride), four 512-byte
 // segments loaded before they are stored.  Otherwise one warp per
-// (assignment, 64-byte segment) with 2-byte accesses.
+// (assignment, 64-byte segment) with 2-byte accesses.  TO_F16: BF16 rows
+// are written as F16 (exact in F16's normal range; a finite value above it
+// or a NaN is reported as MOE_DEVICE_ERR_ACT_RANGE, as in the projections'
+// own conversion).
+template <bool TO_F16>
 __global__ void __launch_bounds__(256) route_scatter_kernel(ScatterParams p) {
   pdl_enter();  // programmatic dependent launch: the previous kernel is done
   const int lane = threadIdx.x & 31;
@@ -317,15 +322,22 @@ __global__ void __launch_bounds__(256) route_scatter_kernel(ScatterParams p) {
       pos = __shfl_sync(0xffffffffu, pos, 0);
       const uint4 *src = reinterpret_cast<const uint4 *>(p.x + (a / p.k) * p.row_bytes);
       uint4 *dst = reinterpret_cast<uint4 *>(p.values + pos * p.row_bytes);
+      uint32_t bad = 0;
       for (int64_t i0 = lane; i0 < n16; i0 += 32 * 4) {
         uint4 v[4];
 #pragma unroll
         for (int j = 0; j < 4; ++j)
           if (i0 + 32 * j < n16) v[j] = __ldg(src + i0 + 32 * j);
+        if (TO_F16) {
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            if (i0 + 32 * j < n16) act_quad_to_mt<__half>(v[j], MOE_BF16, bad);
+        }
 #pragma unroll
         for (int j = 0; j < 4; ++j)
           if (i0 + 32 * j < n16) dst[i0 + 32 * j] = v[j];
       }
+      if (TO_F16 && bad) report(p.status, MOE_DEVICE_ERR_ACT_RANGE);
     }
     return;
   }
@@ -338,8 +350,15 @@ __global__ void __launch_bounds__(256) route_scatter_kernel(ScatterParams p) {
     const uint8_t *src = p.x + (a / p.k) * p.row_bytes;
     uint8_t *dst = p.values + pos * p.row_bytes;
     const int64_t off = s * 64 + lane * 2;
-    if (off < p.row_bytes)
-      *reinterpret_cast<uint16_t *>(dst + off) = *reinterpret_cast<const uint16_t *>(src + off);
+    if (off < p.row_bytes) {
+      uint16_t b = *reinterpret_cast<const uint16_t *>(src + off);
+      if (TO_F16) {
+        uint32_t bad = 0;
+        b = (uint16_t)(act_pair_to_mt<__half>((uint32_t)b, MOE_BF16, bad) & 0xFFFFu);
+        if (bad) report(p.status, MOE_DEVICE_ERR_ACT_RANGE);
+      }
+      *reinterpret_cast<uint16_t *>(dst + off) = b;
+    }
   }
 }
 
@@ -451,10 +470,10 @@ extern "C" size_t moe_route_dispatch_workspace_size(int64_t T, int64_t E, int32_
 // points below check their own arguments first.
 static moe_status route_impl(const char *fn, const void *x, moe_dtype x_dtype, int64_t T, int64_t H,
                              const float *logits, const float *sel_bias, int64_t E, int32_t expert_start,
-                             int32_t top_k, int32_t renormalize, void *values, float *weights,
+                             int32_t top_k, int32_t renormalize, void *values, bool to_f16, float *weights,
                              uint32_t *selected_experts, uint32_t *row_experts, int32_t *offsets,
                              int32_t *src_token, int32_t *row_of, void *workspace, size_t workspace_bytes,
-                             void *stream);
+                             int32_t *device_status, void *stream);
 
 extern "C" moe_status moe_route_dispatch(const void *x, moe_dtype x_dtype, int64_t T, int64_t H,
                                          const float *logits, const float *sel_bias, int64_t E,
@@ -463,13 +482,30 @@ extern "C" moe_status moe_route_dispatch(const void *x, moe_dtype x_dtype, int64
                                          uint32_t *row_experts, int32_t *offsets, int32_t *src_token,
                                          int32_t *row_of, void *workspace, size_t workspace_bytes,
                                          int32_t *device_status, void *stream) {
-  (void)device_status;  // every index is produced here; nothing to report
   moe_status a = route_check_args("moe_route_dispatch", x, x_dtype, T, H, logits, E, expert_start, top_k, values,
                                   weights, selected_experts, row_experts, offsets, src_token, row_of);
   if (a != MOE_OK) return a;
   return route_impl("moe_route_dispatch", x, x_dtype, T, H, logits, sel_bias, E, expert_start, top_k, renormalize,
-                    values, weights, selected_experts, row_experts, offsets, src_token, row_of, workspace,
-                    workspace_bytes, stream);
+                    values, false, weights, selected_experts, row_experts, offsets, src_token, row_of, workspace,
+                    workspace_bytes, device_status, stream);
+}
+
+extern "C" moe_status moe_route_dispatch_dt(const void *x, moe_dtype x_dtype, int64_t T, int64_t H,
+                                            const float *logits, const float *sel_bias, int64_t E,
+                                            int32_t expert_start, int32_t top_k, int32_t renormalize,
+                                            void *values, moe_dtype values_dtype, float *weights,
+                                            uint32_t *selected_experts, uint32_t *row_experts, int32_t *offsets,
+                                            int32_t *src_token, int32_t *row_of, void *workspace,
+                                            size_t workspace_bytes, int32_t *device_status, void *stream) {
+  moe_status a = route_check_args("moe_route_dispatch", x, x_dtype, T, H, logits, E, expert_start, top_k, values,
+                                  weights, selected_experts, row_experts, offsets, src_token, row_of);
+  if (a != MOE_OK) return a;
+  const bool to_f16 = x_dtype == MOE_BF16 && values_dtype == MOE_F16;
+  if (values_dtype != x_dtype && !to_f16)
+    return set_error(MOE_ERR_UNSUPPORTED_DTYPE, "moe_route_dispatch: values_dtype must be x_dtype, or F16 for BF16 x");
+  return route_impl("moe_route_dispatch", x, x_dtype, T, H, logits, sel_bias, E, expert_start, top_k, renormalize,
+                    values, to_f16, weights, selected_experts, row_experts, offsets, src_token, row_of, workspace,
+                    workspace_bytes, device_status, stream);
 }
 
 extern "C" moe_status moe_route(const float *logits, const float *sel_bias, int64_t T, int64_t E,
@@ -484,16 +520,16 @@ extern "C" moe_status moe_route(const float *logits, const float *sel_bias, int6
                                   weights, selected_experts, row_experts, offsets, src_token, row_of);
   if (a != MOE_OK) return a;
   return route_impl("moe_route", nullptr, MOE_BF16, T, 1, logits, sel_bias, E, expert_start, top_k, renormalize,
-                    nullptr, weights, selected_experts, row_experts, offsets, src_token, row_of, workspace,
-                    workspace_bytes, stream);
+                    nullptr, false, weights, selected_experts, row_experts, offsets, src_token, row_of, workspace,
+                    workspace_bytes, nullptr, stream);
 }
 
 static moe_status route_impl(const char *fn, const void *x, moe_dtype x_dtype, int64_t T, int64_t H,
                              const float *logits, const float *sel_bias, int64_t E, int32_t expert_start,
-                             int32_t top_k, int32_t renormalize, void *values, float *weights,
+                             int32_t top_k, int32_t renormalize, void *values, bool to_f16, float *weights,
                              uint32_t *selected_experts, uint32_t *row_experts, int32_t *offsets,
                              int32_t *src_token, int32_t *row_of, void *workspace, size_t workspace_bytes,
-                             void *stream) {
+                             int32_t *device_status, void *stream) {
   cudaStream_t st = as_stream(stream);
   if (T == 0) {
     if (cudaMemsetAsync(offsets, 0, sizeof(int32_t) * (size_t)(E + 1), st) != cudaSuccess)
@@ -562,11 +598,15 @@ static moe_status route_impl(const char *fn, const void *x, moe_dtype x_dtype, i
   sp.src_token = src_token;
   sp.vec16 = aligned16(x) && aligned16(values) && (sp.row_bytes % 16 == 0);
   sp.nseg = (sp.row_bytes + 63) / 64;  // 2-byte path only
+  sp.status = device_status;
   int64_t units = !values ? (sp.A + 31) / 32 : sp.vec16 ? sp.A : sp.A * sp.nseg;
   int64_t blocks = (units + 7) / 8;
   int64_t cap = (int64_t)num_sms() * 16;
   if (blocks > cap) blocks = cap;
-  launch_pdl(route_scatter_kernel, dim3((unsigned)blocks), dim3(256), 0, st, sp);
+  if (to_f16)
+    launch_pdl(route_scatter_kernel<true>, dim3((unsigned)blocks), dim3(256), 0, st, sp);
+  else
+    launch_pdl(route_scatter_kernel<false>, dim3((unsigned)blocks), dim3(256), 0, st, sp);
   return check_launch("route_scatter_kernel");
 }
 

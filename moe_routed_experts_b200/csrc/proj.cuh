@@ -27,7 +27,8 @@ struct ProjParams {
   float *partials;
   int32_t *counters;
   int kq;  // K splits
-  int preconv;  // x holds F16 copies of BF16 activations (act_dt stays the output dtype)
+  int preconv;  // x holds F16 copies of BF16 activations
+  int odt;      // dtype of out, gout and uout (F16 or BF16), independent of the input's
 #ifdef MOE_TEST_HOOKS
   int test_stall;  // test build only: see moe_test_arm_stall
 #endif
@@ -153,11 +154,11 @@ __device__ __forceinline__ void finish8_bt(const ProjParams &p, int64_t row, int
 
 // Final values of 8 consecutive output columns n0.. of row `row` of local
 // expert e from FP32 sums (gate sums g, up sums u for the pair): bias, one
-// rounding to the activation dtype, SwiGLU from the rounded G and U.
+// rounding to the output dtype, SwiGLU from the rounded G and U.
 template <int NPROJ>
 __device__ __forceinline__ void finish8(const ProjParams &p, int e, int64_t row, int64_t n0, const float *g,
                                         const float *u) {
-  if (p.act_dt == MOE_BF16) finish8_t<NPROJ, true>(p, e, row, n0, g, u);
+  if (p.odt == MOE_BF16) finish8_t<NPROJ, true>(p, e, row, n0, g, u);
   else finish8_t<NPROJ, false>(p, e, row, n0, g, u);
 }
 

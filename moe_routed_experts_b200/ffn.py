@@ -4,8 +4,9 @@
 awq_grouped_down -> moe_combine; ``backward`` = moe_combine_backward ->
 awq_input_backward(down) -> moe_swiglu_backward -> awq_input_backward(gate
 + up, one accumulation) -> moe_dispatch_backward, and moe_router_backward
-for the router logits (the ``_dt`` forms of the first three, writing the
-gradients that feed an input VJP in its scale dtype).  Only argument marshalling happens here; every step
+for the router logits.  The ``_dt`` forms of the dispatch, the gate/up
+projection and the first three backward steps write the tensors that only
+feed a tensor-core product (values, dy, dG, dU) in the scale dtype.  Only argument marshalling happens here; every step
 runs in the library's kernels.
 """
 from dataclasses import dataclass
@@ -64,8 +65,9 @@ class Buffers:
 def alloc(w, device="cuda", keep_gu: bool = False) -> Buffers:
     T, H, I, E, k = w.T, w.H, w.I, w.E, w.top_k
     A = T * k
+    vdt = _SDT[operand_dtype(w.scale_dtype)]  # the COPY writes the rows in the gate/up operand dtype
     route = {
-        "values": torch.empty((A, H), dtype=torch.bfloat16, device=device),
+        "values": torch.empty((A, H), dtype=vdt, device=device),
         "weights": torch.empty((T, k), dtype=torch.float32, device=device),
         "selected_experts": torch.empty((T, k), dtype=torch.int32, device=device),
         "row_experts": torch.empty((A,), dtype=torch.int32, device=device),
@@ -80,7 +82,8 @@ def alloc(w, device="cuda", keep_gu: bool = False) -> Buffers:
     y = torch.empty((A, H), dtype=torch.bfloat16, device=device)
     out = torch.empty((T, H), dtype=torch.bfloat16, device=device)
     sdt = {"f16": torch.float16, "bf16": torch.bfloat16, "f32": torch.float32}[w.scale_dtype]
-    pws = max(B.projection_workspace_size(A, H, I, E, w.group, 2, torch.bfloat16, sdt),
+    pws = max(B.projection_workspace_size(A, H, I, E, w.group, 2, vdt, sdt),
+              B.projection_workspace_size(A, H, I, E, w.group, 2, torch.bfloat16, sdt),  # gather mode reads x
               B.projection_workspace_size(A, I, H, E, w.group, 1, torch.bfloat16, sdt))
     proj_ws = torch.empty(pws, dtype=torch.uint8, device=device) if pws else None
     return Buffers(route, ws, h, G, U, y, out, torch.zeros(1, dtype=torch.int32, device=device), proj_ws)
@@ -103,15 +106,16 @@ def forward(dev: dict, buf: Buffers, gather: bool = False) -> torch.Tensor:
     A = w.A
     pay = (B._ptr(gate["qweight"]), B._ptr(gate["qzeros"]), B._ptr(gate["scales"]), B._ptr(gate["bias"]),
            B._ptr(up["qweight"]), B._ptr(up["qzeros"]), B._ptr(up["scales"]), B._ptr(up["bias"]),
-           B._dt(gate["scales"].dtype), B.MOE_F32, w.group, B._ptr(buf.h), B._ptr(buf.G), B._ptr(buf.U),
-           B._ptr(buf.proj_ws), 0 if buf.proj_ws is None else buf.proj_ws.numel(), B._ptr(buf.status), st)
+           B._dt(gate["scales"].dtype), B.MOE_F32, w.group, B._ptr(buf.h), B._ptr(buf.G), B._ptr(buf.U))
+    tail = (B._ptr(buf.proj_ws), 0 if buf.proj_ws is None else buf.proj_ws.numel(), B._ptr(buf.status), st)
     if gather:
         s = lib.awq_grouped_gate_up_swiglu_gather(B._ptr(dev["x"]), B.MOE_BF16, w.T, B._ptr(r["src_token"]), A, w.H,
-                                                  w.I, B._ptr(r["offsets"]), w.E, *pay)
+                                                  w.I, B._ptr(r["offsets"]), w.E, *pay, *tail)
         B._check("awq_grouped_gate_up_swiglu_gather", s)
     else:
-        s = lib.awq_grouped_gate_up_swiglu(B._ptr(r["values"]), B.MOE_BF16, A, w.H, w.I, B._ptr(r["offsets"]), w.E,
-                                           *pay)
+        # values in the operand dtype (F16 with F16 scales), h, G and U in BF16
+        s = lib.awq_grouped_gate_up_swiglu_dt(B._ptr(r["values"]), B._dt(r["values"].dtype), A, w.H, w.I,
+                                              B._ptr(r["offsets"]), w.E, *pay, B.MOE_BF16, *tail)
         B._check("awq_grouped_gate_up_swiglu", s)
     s = lib.awq_grouped_down(
         B._ptr(buf.h), B.MOE_BF16, A, w.I, w.H, B._ptr(r["offsets"]), w.E, B._ptr(down["qweight"]),
@@ -125,13 +129,16 @@ def forward(dev: dict, buf: Buffers, gather: bool = False) -> torch.Tensor:
     return buf.out
 
 
-def chain_grad_dtype(scale_dtype: str, act_dtype: str = "bf16") -> str:
-    """dtype of the gradients that feed the input VJPs (dy, dG, dU).
+def operand_dtype(scale_dtype: str, act_dtype: str = "bf16") -> str:
+    """dtype of the tensors that only feed a projection's tensor-core
+    product: the dispatched rows (values) and the gradients of the input
+    VJPs (dy, dG, dU).
 
-    The input VJPs run their products in the scale dtype, so with F16 scales
-    the steps before them write F16 directly (one rounding of the FP32
-    value) instead of the activation dtype plus a conversion pass; the
-    gradients of the activations (dh, dvalues, dx) stay in act_dtype."""
+    The products run in the scale dtype, so with F16 scales the step before
+    writes F16 directly (the COPY converts while copying; the VJP steps
+    round their FP32 values once) instead of the activation dtype plus a
+    conversion pass; h, y, out and the activation gradients (dh, dvalues,
+    dx) stay in act_dtype."""
     return "f16" if scale_dtype == "f16" else act_dtype
 
 
@@ -141,7 +148,7 @@ def backward(dev: dict, buf: Buffers, d_out: torch.Tensor) -> dict:
     r = buf.route
     assert buf.G is not None and buf.U is not None, "allocate with keep_gu=True"
     act = buf.y.dtype
-    gdt = _SDT[chain_grad_dtype(w.scale_dtype, "bf16" if act == torch.bfloat16 else "f16")]
+    gdt = _SDT[operand_dtype(w.scale_dtype, "bf16" if act == torch.bfloat16 else "f16")]
     dy, dw = B.moe_combine_backward(d_out, buf.y, r["weights"], r["row_of"], device_status=buf.status, dy_dtype=gdt)
     dh = B.awq_input_backward(dy, r["offsets"], dev["down"], w.group, device_status=buf.status, out_dtype=act)
     dG, dU = B.moe_swiglu_backward(dh, buf.G, buf.U, out_dtype=gdt, device_status=buf.status)

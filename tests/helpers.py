@@ -264,9 +264,22 @@ def gpu_forward_numpy(inp):
     res = {"selected": u32(r["selected_experts"]), "weights": r["weights"].cpu().numpy(),
            "offsets": r["offsets"].cpu().numpy(), "row_experts": u32(r["row_experts"]),
            "src_token": r["src_token"].cpu().numpy(), "row_of": r["row_of"].cpu().numpy(),
-           "values": bits(r["values"]), "G": bits(buf.G), "U": bits(buf.U), "h": bits(buf.h), "y": bits(buf.y),
-           "out": bits(buf.out), "status": int(buf.status.item())}
+           "values": bits(r["values"]), "values_dt": dt_name(r["values"].dtype), "G": bits(buf.G), "U": bits(buf.U),
+           "h": bits(buf.h), "y": bits(buf.y), "out": bits(buf.out), "status": int(buf.status.item())}
     return res, dev, buf
+
+
+def dt_name(dtype) -> str:
+    return {torch.bfloat16: "bf16", torch.float16: "f16"}[dtype]
+
+
+def values_in(dt: str, bf16_rows: np.ndarray) -> np.ndarray:
+    """The dispatched rows as the COPY writes them in dtype dt: the BF16 bits
+    themselves, or their F16 images (exact in F16's normal range; numpy's
+    float16 cast rounds to nearest even)."""
+    if dt == "bf16":
+        return bf16_rows
+    return as_f64(bf16_rows, "bf16").astype(np.float16).view(np.uint16)
 
 
 def check_forward_steps(inp, res, want, name, rows=None, tokens=None):
@@ -277,11 +290,11 @@ def check_forward_steps(inp, res, want, name, rows=None, tokens=None):
     if rows is None:
         rows = np.arange(w.A)
     rexp = (res["row_experts"][rows].astype(np.int64) - w.expert_start).astype(np.int32)
-    values = res["values"][rows]
+    values, vdt = res["values"][rows], res.get("values_dt", "bf16")
     G, U, h = res["G"][rows], res["U"][rows], res["h"][rows]
     sdt, g = w.scale_dtype, w.group
-    check_close(G, want["G"], name + "/G", justify=j_project(values, "bf16", rexp, inp["gate"], sdt, g))
-    check_close(U, want["U"], name + "/U", justify=j_project(values, "bf16", rexp, inp["up"], sdt, g))
+    check_close(G, want["G"], name + "/G", justify=j_project(values, vdt, rexp, inp["gate"], sdt, g))
+    check_close(U, want["U"], name + "/U", justify=j_project(values, vdt, rexp, inp["up"], sdt, g))
     check_close(h, oracle.swiglu(G, U, "bf16"), name + "/h", justify=j_swiglu(G, U))
     y = oracle.project(h, "bf16", rexp, inp["down"], sdt, g)
     check_close(res["y"][rows], y, name + "/y", justify=j_project(h, "bf16", rexp, inp["down"], sdt, g))

@@ -100,6 +100,22 @@ def test_combine_family_rejects_bad_arguments(L):
     assert L.moe_swiglu_backward(FAKE, FAKE, FAKE, B.MOE_BF16, -1, 8, FAKE, FAKE, None) == 1
 
 
+def test_dtype_choosing_forward_forms_reject_bad_dtypes(L):
+    def route_dt(xdt, vdt, k=2):
+        return L.moe_route_dispatch_dt(FAKE, xdt, 4, 8, FAKE, None, 8, 0, k, 1, FAKE, vdt, FAKE, FAKE, FAKE, FAKE,
+                                       FAKE, FAKE, FAKE, 1 << 20, None, None)
+    assert route_dt(B.MOE_F16, B.MOE_BF16) == 2   # only BF16 -> F16 converts
+    assert route_dt(B.MOE_BF16, B.MOE_F32) == 2
+    assert route_dt(B.MOE_BF16, B.MOE_F16, k=0) == 1
+
+    def gate_up_dt(odt, A=16):
+        return L.awq_grouped_gate_up_swiglu_dt(FAKE, B.MOE_F16, A, 64, 32, FAKE, 2, FAKE, FAKE, FAKE, None, FAKE,
+                                               FAKE, FAKE, None, B.MOE_F16, B.MOE_F32, 16, FAKE, None, None, odt,
+                                               None, 0, None, None)
+    assert gate_up_dt(B.MOE_F32) == 2
+    assert gate_up_dt(B.MOE_BF16, A=0) == 0
+
+
 def test_dtype_choosing_backward_forms_reject_bad_dtypes(L):
     # the _dt forms check the output dtype on the host (2 = unsupported dtype)
     assert L.moe_combine_backward_dt(FAKE, FAKE, B.MOE_BF16, 8, FAKE, FAKE, 4, 16, 2, FAKE, B.MOE_F32, None, None,

@@ -47,7 +47,7 @@ def _chain(name, kw, rows=None, tokens=None):
     if tokens is None:
         tokens = np.arange(w.T)
     # the chain writes dy, dG and dU in the scale dtype when it is F16
-    cdt = ffn.chain_grad_dtype(w.scale_dtype)
+    cdt = ffn.operand_dtype(w.scale_dtype)
     assert g["dy"].dtype == g["dG"].dtype == g["dU"].dtype == ffn._SDT[cdt]
     assert g["dh"].dtype == g["dvalues"].dtype == g["dx"].dtype == torch.bfloat16
     # combine VJP on the sampled tokens
@@ -148,7 +148,7 @@ def test_whole_chain_against_oracle_chain():
     torch.cuda.synchronize()
     f = oracle.forward(inp)
     rexp = (f["row_experts"].astype(np.int64) - w.expert_start).astype(np.int32)
-    cdt = ffn.chain_grad_dtype(w.scale_dtype)  # dy, dG, dU: F16 with F16 scales
+    cdt = ffn.operand_dtype(w.scale_dtype)  # dy, dG, dU: F16 with F16 scales
     o_dy, o_dw = oracle.combine_backward(inp["d_out"], f["y"], "bf16", f["weights"], f["row_of"], dy_dt=cdt)
     o_dh = oracle.input_backward(o_dy, cdt, rexp, inp["down"], w.scale_dtype, w.group, odt="bf16")
     o_dG, o_dU = oracle.swiglu_backward(o_dh, f["G"], f["U"], "bf16", odt=cdt)

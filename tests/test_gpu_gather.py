@@ -13,7 +13,7 @@ import pytest
 import torch
 
 import oracle
-from helpers import bits, check_forward_steps, check_routing, generated, u32
+from helpers import bits, check_forward_steps, check_routing, dt_name, generated, u32
 from moe_routed_experts_b200 import binding as B
 from moe_routed_experts_b200 import ffn
 
@@ -58,6 +58,7 @@ def _run(inp, gather):
            "status": int(buf.status.item())}
     if not gather:
         res["values"] = bits(r["values"])
+        res["values_dt"] = dt_name(r["values"].dtype)
     return res
 
 
@@ -77,6 +78,7 @@ def test_gather_mode_against_oracle(key, path):
     want = oracle.forward(inp)
     check_routing(res, want, key)
     res["values"] = want["values"]  # the rows the gather reads (bit copies of x, checked in the routing tests)
+    res["values_dt"] = "bf16"
     check_forward_steps(inp, res, want, key + "/gather")
     assert res["status"] == 0
 

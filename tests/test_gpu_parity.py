@@ -8,7 +8,7 @@ import torch
 
 import oracle
 from helpers import (TOL, as_f64, bits, check_close, check_forward_steps, check_routing, generated, gpu_forward,
-                     gpu_forward_numpy, sample_rows, u32)
+                     gpu_forward_numpy, sample_rows, u32, values_in)
 from moe_routed_experts_b200 import binding as B
 from moe_routed_experts_b200 import ffn, inputs
 from moe_routed_experts_b200.configs import WORKLOADS, Workload, scaled
@@ -67,6 +67,14 @@ def test_route_dispatch_full_size(name):
                         "row_of": row_of}, name)
     src_t = torch.from_numpy(src.astype(np.int64)).cuda()
     assert torch.equal(r["values"], dev["x"][src_t]), "values are not bit copies of x[src_token]"
+    assert int(st.item()) == 0
+    # the F16 form of the COPY: each row's exact F16 image (torch's cast rounds to nearest even)
+    r16 = B.moe_route_dispatch(dev["x"], dev["logits"], w.top_k, E=w.E, sel_bias=dev["sel_bias"], device_status=st,
+                               values_dtype=torch.float16)
+    torch.cuda.synchronize()
+    assert r16["values"].dtype == torch.float16
+    assert torch.equal(r16["values"].view(torch.int16), dev["x"][src_t].to(torch.float16).view(torch.int16))
+    assert torch.equal(r16["row_of"], r["row_of"]) and torch.equal(r16["offsets"], r["offsets"])
     assert int(st.item()) == 0
 
 
@@ -167,7 +175,7 @@ def test_forward_every_row(name, path):
     res, dev, buf = gpu_forward_numpy(inp)
     want = _oracle_forward_all(inp)
     check_routing(res, want, name)
-    assert np.array_equal(res["values"], want["values"])
+    assert np.array_equal(res["values"], values_in(res["values_dt"], want["values"]))
     check_forward_steps(inp, res, want, name)
     assert res["status"] == 0
 

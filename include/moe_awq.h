@@ -279,9 +279,9 @@ MOE_API moe_status awq_grouped_gate_up_swiglu_dt(
  * awq_grouped_gate_up_swiglu on values = the COPY of those rows; same
  * payload arguments, workspace and errors.  A src_token entry outside
  * [0, T) sets MOE_DEVICE_ERR_ROW_RANGE and that row reads token 0.
- * The tcgen05 tiles load the rows with TMA tile::gather4 (four rows per
- * copy, from this GPU's memory, no multicast); the small-batch tiles with
- * one bulk copy or load per row.
+ * The tcgen05 tiles copy the rows with 16-byte cp.async from their
+ * producer lanes (this GPU's memory, no multicast); the small-batch tiles
+ * with one bulk copy or load per row.
  * ---------------------------------------------------------------------- */
 MOE_API moe_status awq_grouped_gate_up_swiglu_gather(
     const void *x, moe_dtype act_dtype, int64_t T, const int32_t *src_token, int64_t A, int64_t H, int64_t I,

@@ -485,7 +485,8 @@ static moe_status launch_tc_t(const ProjParams &p, cudaStream_t st) {
   CUtensorMap mx, m0, m1;
   const uint64_t NW = p.N / 8, rows = (uint64_t)p.E * p.K;
   const uint32_t box_w = NPROJ == 2 ? 16 : 32;
-  // the activation map: 128-row boxes of the batch, or one-row boxes of x for tile::gather4
+  // the activation map: 128-row boxes of the batch (the gather mode copies
+  // its rows with cp.async and leaves the one-row map of x unused)
   const bool mx_ok = p.gather ? make_map_2d(&mx, p.x, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, p.K, p.T, kBK, 1,
                                             CU_TENSOR_MAP_SWIZZLE_128B)
                               : make_map_2d(&mx, p.x, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, p.K, p.A, kBK, kBM,

@@ -463,7 +463,8 @@ static moe_status launch_tc2_t(const ProjParams &p, cudaStream_t st) {
   using namespace tc2;
   CUtensorMap mx, m0, m1;
   const uint64_t NW = p.N / 8, rows = (uint64_t)p.E * p.K;
-  // the activation map: 128-row boxes of the batch, or one-row boxes of x for tile::gather4
+  // the activation map: 128-row boxes of the batch (the gather mode copies
+  // its rows with cp.async and leaves the one-row map of x unused)
   const bool mx_ok = p.gather ? make_map_2d(&mx, p.x, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, p.K, p.T, 64, 1,
                                             CU_TENSOR_MAP_SWIZZLE_128B)
                               : make_map_2d(&mx, p.x, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, p.K, p.A, 64, kBM,

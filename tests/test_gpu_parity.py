@@ -95,6 +95,39 @@ def test_route_dispatch_options(renorm, expert_start):
                         "row_of": row_of}, "options")
 
 
+@pytest.mark.parametrize("H", [20, 64], ids=["two_byte_rows", "sixteen_byte_rows"])
+@pytest.mark.parametrize("value,flagged", [(None, False), (70000.0, True), (float("nan"), True),
+                                           (float("inf"), False), (1e-7, False)],
+                         ids=["plain", "overflow", "nan", "inf_converts_exactly", "below_f16_subnormal_grid"])
+def test_route_dispatch_f16_rows(H, value, flagged):
+    # the F16 form of the COPY on both copy paths (H = 20: 40-byte rows, one
+    # 2-byte element per lane; H = 64: 16-byte vectors): each row is the F16
+    # image of the BF16 token row (torch's cast rounds to nearest even), the
+    # row maps equal the plain COPY's, and only a finite value above F16's
+    # range or a NaN is reported (MOE_DEVICE_ERR_ACT_RANGE)
+    T, E, k = 150, 12, 3
+    rng = np.random.default_rng(H)
+    logits = rng.standard_normal((T, E), dtype=np.float32)
+    x = inputs.random_bf16(rng, (T, H))
+    if value is not None:
+        x[37, H - 3] = bits(torch.tensor([value], dtype=torch.bfloat16))[0]
+    xd = torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).cuda()
+    ld = torch.from_numpy(logits).cuda()
+    st, st16 = B.new_status(), B.new_status()
+    r = B.moe_route_dispatch(xd, ld, k, E=E, device_status=st)
+    r16 = B.moe_route_dispatch(xd, ld, k, E=E, device_status=st16, values_dtype=torch.float16)
+    torch.cuda.synchronize()
+    assert r16["values"].dtype == torch.float16
+    for key in ("selected_experts", "weights", "offsets", "row_experts", "src_token", "row_of"):
+        assert torch.equal(r16[key], r[key]), key
+    want = r["values"].to(torch.float16)
+    nan = torch.isnan(want)  # NaN payloads may differ: compare NaN-ness there
+    assert torch.equal(torch.isnan(r16["values"]), nan)
+    assert torch.equal(r16["values"].view(torch.int16)[~nan], want.view(torch.int16)[~nan])
+    assert int(st.item()) == 0
+    assert int(st16.item()) == (16 if flagged else 0), int(st16.item())
+
+
 def test_route_ties_and_empty_experts():
     # many exact ties (logits on a coarse grid) and experts nobody picks
     T, E, k = 700, 96, 4

@@ -191,13 +191,14 @@ def _bf16_cuda(a):
 @pytest.mark.parametrize("value,flagged", [(4.0e5, True), (float("nan"), True), (float("inf"), False),
                                            (1.2e5, False)],
                          ids=["overflow", "nan", "inf_stays_inf", "in_range"])
-def test_f16_dy_from_bf16_inputs(value, flagged):
+@pytest.mark.parametrize("H", [72, 70], ids=["vector_rows", "element_rows"])
+def test_f16_dy_from_bf16_inputs(value, flagged, H):
     # moe_combine_backward writing F16 dy from BF16 inputs: one rounding of
     # the FP32 product, bit for bit the oracle's F16 rounding here (w = 0.5
     # makes the product exact), and a value that is not inf but overflows
     # F16 (or a NaN) is reported like the BF16 -> F16 input conversion
     rng = np.random.default_rng(5)
-    T, H, k = 6, 72, 2
+    T, k = 6, 2
     A = T * k
     d_out = inputs.random_bf16(rng, (T, H))
     y = inputs.random_bf16(rng, (A, H))
@@ -221,17 +222,18 @@ def test_f16_dy_from_bf16_inputs(value, flagged):
 @pytest.mark.parametrize("value,flagged", [(2.0e5, True), (float("nan"), True), (float("inf"), False),
                                            (6.0e4, False)],
                          ids=["overflow", "nan", "inf_stays_inf", "in_range"])
-def test_f16_swiglu_grads_from_bf16_inputs(value, flagged):
-    # moe_swiglu_backward writing F16 dG/dU from BF16 dh, G, U; at G = 0.5,
-    # U = 1 the planted dh gives dG = 0.74 dh and dU = 0.31 dh
+@pytest.mark.parametrize("A,I,r,c", [(16, 40, 2, 3), (15, 39, 14, 38)], ids=["vectors", "tail_element"])
+def test_f16_swiglu_grads_from_bf16_inputs(value, flagged, A, I, r, c):
+    # moe_swiglu_backward writing F16 dG/dU from BF16 dh, G, U (8-element
+    # vectors, and the scalar tail when A*I is not a multiple of 8); at
+    # G = 0.5, U = 1 the planted dh gives dG = 0.74 dh and dU = 0.31 dh
     rng = np.random.default_rng(6)
-    A, I = 16, 40
     dh, G, U = (inputs.random_bf16(rng, (A, I)) for _ in range(3))
-    G[2, 3] = bits(torch.tensor([0.5], dtype=torch.bfloat16))[0]
-    U[2, 3] = bits(torch.tensor([1.0], dtype=torch.bfloat16))[0]
+    G[r, c] = bits(torch.tensor([0.5], dtype=torch.bfloat16))[0]
+    U[r, c] = bits(torch.tensor([1.0], dtype=torch.bfloat16))[0]
     for planted in (False, True):
         if planted:
-            dh[2, 3] = bits(torch.tensor([value], dtype=torch.bfloat16))[0]
+            dh[r, c] = bits(torch.tensor([value], dtype=torch.bfloat16))[0]
         st = B.new_status()
         dG, dU = B.moe_swiglu_backward(_bf16_cuda(dh), _bf16_cuda(G), _bf16_cuda(U), out_dtype=torch.float16,
                                        device_status=st)

@@ -24,7 +24,6 @@
 
 namespace moe {
 
-constexpr int kRouteThreads = 512;
 constexpr int kScanThreads = 1024;
 constexpr int kMaxChunks = 1024;
 

@@ -6,8 +6,9 @@ awq_input_backward(down) -> moe_swiglu_backward -> awq_input_backward(gate
 + up, one accumulation) -> moe_dispatch_backward, and moe_router_backward
 for the router logits.  The ``_dt`` forms of the dispatch, the gate/up
 projection and the first three backward steps write the tensors that only
-feed a tensor-core product (values, dy, dG, dU) in the scale dtype.  Only argument marshalling happens here; every step
-runs in the library's kernels.
+feed a tensor-core product (values, dy, dG, dU) in the scale dtype.  Only
+argument marshalling happens here; every step runs in the library's
+kernels.
 """
 from dataclasses import dataclass
 from typing import Optional

@@ -279,8 +279,10 @@ def measure(w, args, steps, world, rank, local, cpu):
         if record is not None:
             ev0.record()
         if buf.G is None:
+            # rows and h in the operand dtype, G and U rounded in BF16 (the activation dtype)
             B.awq_grouped_gate_up_swiglu(r["values"], r["offsets"], dev["gate"], dev["up"], w.group,
-                                         device_status=buf.status, out=buf.h, workspace=buf.proj_ws)
+                                         device_status=buf.status, out=buf.h, workspace=buf.proj_ws,
+                                         out_dtype=torch.bfloat16)
         else:
             _gate_up_keep(B, r, dev, w, buf)
         if record is not None:
@@ -509,8 +511,8 @@ def _gate_up_keep(B, r, dev, w, buf):
         B._ptr(r["values"]), B._dt(r["values"].dtype), w.A, w.H, w.I, B._ptr(r["offsets"]), w.E,
         B._ptr(gate["qweight"]), B._ptr(gate["qzeros"]), B._ptr(gate["scales"]), B._ptr(gate["bias"]),
         B._ptr(up["qweight"]), B._ptr(up["qzeros"]), B._ptr(up["scales"]), B._ptr(up["bias"]),
-        B._dt(gate["scales"].dtype), B.MOE_F32, w.group, B._ptr(buf.h), B._ptr(buf.G), B._ptr(buf.U),
-        B._dt(buf.h.dtype), B._ptr(buf.proj_ws), 0 if buf.proj_ws is None else buf.proj_ws.numel(),
+        B._dt(gate["scales"].dtype), B.MOE_F32, w.group, B._ptr(buf.h), B._dt(buf.h.dtype), B._ptr(buf.G),
+        B._ptr(buf.U), B._dt(buf.G.dtype), B._ptr(buf.proj_ws), 0 if buf.proj_ws is None else buf.proj_ws.numel(),
         B._ptr(buf.status), st)
     B._check("awq_grouped_gate_up_swiglu", s)
 
@@ -535,18 +537,17 @@ def gate_up_kernel_name(B, w):
 
 def launches_per_step_of(B, w):
     """Kernel launches of one step: route (2, or 3 past one token chunk), each
-    projection (1, or 2 with the split-K reduce; a tcgen05 down projection
-    with F16 scales adds the one-time F16 copy of h, while the dispatch
-    writes the gate/up rows in F16 itself), combine, and the backward's six
+    projection (1, or 2 with the split-K reduce; no F16 copies: the dispatch
+    and the gate/up epilogue write the rows and h in F16 themselves when the
+    scales are F16), combine, and the backward's six
     (its input-VJP gradients are written in the scale dtype, so it makes no
     copies)."""
     n = 2 if w.T <= 64 else 3
-    conv = _path_of(w) >= 2 and w.scale_dtype == "f16"
     if _path_of(w) == 1:
         n += 1 + (B.projection_workspace_size(w.A, w.H, w.I, w.E, w.group, 2) > 0)
         n += 1 + (B.projection_workspace_size(w.A, w.I, w.H, w.E, w.group, 1) > 0)
     else:
-        n += 2 + (1 if conv else 0)
+        n += 2
     n += 1
     if w.backward:
         n += 6

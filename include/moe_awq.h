@@ -255,11 +255,14 @@ MOE_API moe_status awq_grouped_gate_up_swiglu(
     void *h, void *gate_out, void *up_out, void *workspace, size_t workspace_bytes,
     int32_t *device_status, void *stream);
 
-/* awq_grouped_gate_up_swiglu with h, gate_out and up_out stored in out_dtype
- * (F16 or BF16) instead of act_dtype: the same FP32 sums, one rounding to
- * out_dtype, SwiGLU from the rounded G and U.  F16 values from
- * moe_route_dispatch_dt with F16 scales give BF16 outputs without a
- * conversion pass. */
+/* awq_grouped_gate_up_swiglu with gate_out and up_out stored in out_dtype
+ * and h in h_dtype (each F16 or BF16) instead of act_dtype: the same FP32
+ * sums, one rounding of G and U to out_dtype, h = RNE_{h_dtype}(silu(G) U)
+ * from the rounded G and U.  With F16 scales, F16 values from
+ * moe_route_dispatch_dt and F16 h (the down projection's operand dtype) need
+ * no conversion pass while G and U stay BF16; F16 h from BF16 G and U that
+ * overflows F16 (a value that is not +-inf becoming inf or NaN) sets
+ * MOE_DEVICE_ERR_ACT_RANGE. */
 MOE_API moe_status awq_grouped_gate_up_swiglu_dt(
     const void *values, moe_dtype act_dtype, int64_t A, int64_t H, int64_t I,
     const int32_t *offsets, int64_t E,
@@ -268,8 +271,8 @@ MOE_API moe_status awq_grouped_gate_up_swiglu_dt(
     const int32_t *qweight_up, const int32_t *qzeros_up, const void *scales_up,
     const void *bias_up,
     moe_dtype scale_dtype, moe_dtype bias_dtype, int64_t group_size,
-    void *h, void *gate_out, void *up_out, moe_dtype out_dtype, void *workspace,
-    size_t workspace_bytes, int32_t *device_status, void *stream);
+    void *h, moe_dtype h_dtype, void *gate_out, void *up_out, moe_dtype out_dtype,
+    void *workspace, size_t workspace_bytes, int32_t *device_status, void *stream);
 
 /* ------------------------------------------------------------------------
  * awq_grouped_gate_up_swiglu_gather -- awq_grouped_gate_up_swiglu on rows
@@ -291,6 +294,19 @@ MOE_API moe_status awq_grouped_gate_up_swiglu_gather(
     moe_dtype scale_dtype, moe_dtype bias_dtype, int64_t group_size,
     void *h, void *gate_out, void *up_out, void *workspace, size_t workspace_bytes,
     int32_t *device_status, void *stream);
+
+/* awq_grouped_gate_up_swiglu_gather with the output dtypes of
+ * awq_grouped_gate_up_swiglu_dt. */
+MOE_API moe_status awq_grouped_gate_up_swiglu_gather_dt(
+    const void *x, moe_dtype act_dtype, int64_t T, const int32_t *src_token, int64_t A, int64_t H,
+    int64_t I, const int32_t *offsets, int64_t E,
+    const int32_t *qweight_gate, const int32_t *qzeros_gate, const void *scales_gate,
+    const void *bias_gate,
+    const int32_t *qweight_up, const int32_t *qzeros_up, const void *scales_up,
+    const void *bias_up,
+    moe_dtype scale_dtype, moe_dtype bias_dtype, int64_t group_size,
+    void *h, moe_dtype h_dtype, void *gate_out, void *up_out, moe_dtype out_dtype,
+    void *workspace, size_t workspace_bytes, int32_t *device_status, void *stream);
 
 /* Workspace bytes for the projection of A rows (input width K, output width
  * N, E experts, AWQ group size; nproj = 2 for the gate/up pair, 1 for a
@@ -328,6 +344,16 @@ MOE_API moe_status awq_grouped_down(const void *input, moe_dtype act_dtype, int6
                             const void *bias, moe_dtype scale_dtype, moe_dtype bias_dtype,
                             int64_t group_size, void *output, void *workspace,
                             size_t workspace_bytes, int32_t *device_status, void *stream);
+
+/* awq_grouped_down with the output stored in out_dtype (F16 or BF16) instead
+ * of act_dtype: F16 h (the operand dtype with F16 scales) in, BF16 y out. */
+MOE_API moe_status awq_grouped_down_dt(const void *input, moe_dtype act_dtype, int64_t A, int64_t K,
+                               int64_t N, const int32_t *offsets, int64_t E,
+                               const int32_t *qweight, const int32_t *qzeros, const void *scales,
+                               const void *bias, moe_dtype scale_dtype, moe_dtype bias_dtype,
+                               int64_t group_size, void *output, moe_dtype out_dtype,
+                               void *workspace, size_t workspace_bytes, int32_t *device_status,
+                               void *stream);
 
 /* ------------------------------------------------------------------------
  * nf4_grouped_projection, nf4_input_backward -- a projection whose frozen

@@ -62,7 +62,12 @@ _SIGS = {
     "moe_route_dispatch_dt": (C.c_int, [P, C.c_int, I64, I64, P, P, I64, I32, I32, I32, P, C.c_int, P, P, P, P, P,
                                          P, P, SZ, P, P]),
     "awq_grouped_gate_up_swiglu_dt": (C.c_int, [P, C.c_int, I64, I64, I64, P, I64, P, P, P, P, P, P, P, P, C.c_int,
-                                                C.c_int, I64, P, P, P, C.c_int, P, SZ, P, P]),
+                                                C.c_int, I64, P, C.c_int, P, P, C.c_int, P, SZ, P, P]),
+    "awq_grouped_gate_up_swiglu_gather_dt": (C.c_int, [P, C.c_int, I64, P, I64, I64, I64, P, I64, P, P, P, P, P, P,
+                                                       P, P, C.c_int, C.c_int, I64, P, C.c_int, P, P, C.c_int, P, SZ,
+                                                       P, P]),
+    "awq_grouped_down_dt": (C.c_int, [P, C.c_int, I64, I64, I64, P, I64, P, P, P, P, C.c_int, C.c_int, I64, P,
+                                      C.c_int, P, SZ, P, P]),
     "moe_combine_backward_dt": (C.c_int, [P, P, C.c_int, I64, P, P, I64, I64, I32, P, C.c_int, P, P, P]),
     "awq_input_backward_dt": (C.c_int, [P, C.c_int, I64, I64, I64, P, I64, P, P, P, C.c_int, I64, P, P, P, P, P,
                                         C.c_int, P, SZ, P, P]),
@@ -241,63 +246,68 @@ def _workspace(nbytes, device, workspace=None):
 
 
 def awq_grouped_gate_up_swiglu(values, offsets, gate, up, group, want_gu=False, device_status=None, out=None,
-                               workspace=None, out_dtype=None):
-    """h (and G, U) in out_dtype (default: values' dtype; ``out``'s dtype when given)."""
+                               workspace=None, out_dtype=None, h_dtype=None):
+    """G, U in out_dtype (default: values' dtype) and h in h_dtype (default:
+    ``out``'s dtype when given, else out_dtype)."""
     A, H = values.shape
     E = offsets.numel() - 1
     I = gate["qweight"].shape[2] * 8
     sdt = _dt(gate["scales"].dtype)
-    if out is not None:
-        out_dtype = out.dtype
     out_dtype = out_dtype or values.dtype
-    h = out if out is not None else torch.empty((A, I), dtype=out_dtype, device=values.device)
-    G = torch.empty_like(h) if want_gu else None
-    U = torch.empty_like(h) if want_gu else None
+    h_dtype = out.dtype if out is not None else (h_dtype or out_dtype)
+    h = out if out is not None else torch.empty((A, I), dtype=h_dtype, device=values.device)
+    G = torch.empty((A, I), dtype=out_dtype, device=values.device) if want_gu else None
+    U = torch.empty((A, I), dtype=out_dtype, device=values.device) if want_gu else None
     ws = _workspace(projection_workspace_size(A, H, I, E, group, 2, values.dtype, gate["scales"].dtype), values.device,
                     workspace)
     st = lib().awq_grouped_gate_up_swiglu_dt(
         _ptr(values), _dt(values.dtype), A, H, I, _ptr(offsets), E,
         _ptr(gate["qweight"]), _ptr(gate["qzeros"]), _ptr(gate["scales"]), _ptr(gate.get("bias")),
         _ptr(up["qweight"]), _ptr(up["qzeros"]), _ptr(up["scales"]), _ptr(up.get("bias")),
-        sdt, _bias_dt(gate.get("bias"), up.get("bias")), group, _ptr(h), _ptr(G), _ptr(U), _dt(out_dtype), _ptr(ws),
-        0 if ws is None else ws.numel(), _ptr(device_status), _stream())
+        sdt, _bias_dt(gate.get("bias"), up.get("bias")), group, _ptr(h), _dt(h_dtype), _ptr(G), _ptr(U), _dt(out_dtype),
+        _ptr(ws), 0 if ws is None else ws.numel(), _ptr(device_status), _stream())
     _check("awq_grouped_gate_up_swiglu", st)
     return (h, G, U) if want_gu else h
 
 
 def awq_grouped_gate_up_swiglu_gather(x, src_token, offsets, gate, up, group, want_gu=False, device_status=None,
-                                      out=None, workspace=None):
-    """Gate/up on expert-sorted rows read as x[src_token[r]] (no COPY)."""
+                                      out=None, workspace=None, out_dtype=None, h_dtype=None):
+    """Gate/up on expert-sorted rows read as x[src_token[r]] (no COPY); dtypes
+    as in awq_grouped_gate_up_swiglu (defaults: x's dtype)."""
     T, H = x.shape
     A = src_token.numel()
     E = offsets.numel() - 1
     I = gate["qweight"].shape[2] * 8
     sdt = _dt(gate["scales"].dtype)
-    h = out if out is not None else torch.empty((A, I), dtype=x.dtype, device=x.device)
-    G = torch.empty_like(h) if want_gu else None
-    U = torch.empty_like(h) if want_gu else None
+    out_dtype = out_dtype or x.dtype
+    h_dtype = out.dtype if out is not None else (h_dtype or out_dtype)
+    h = out if out is not None else torch.empty((A, I), dtype=h_dtype, device=x.device)
+    G = torch.empty((A, I), dtype=out_dtype, device=x.device) if want_gu else None
+    U = torch.empty((A, I), dtype=out_dtype, device=x.device) if want_gu else None
     ws = _workspace(projection_workspace_size(A, H, I, E, group, 2, x.dtype, gate["scales"].dtype), x.device, workspace)
-    st = lib().awq_grouped_gate_up_swiglu_gather(
+    st = lib().awq_grouped_gate_up_swiglu_gather_dt(
         _ptr(x), _dt(x.dtype), T, _ptr(src_token), A, H, I, _ptr(offsets), E,
         _ptr(gate["qweight"]), _ptr(gate["qzeros"]), _ptr(gate["scales"]), _ptr(gate.get("bias")),
         _ptr(up["qweight"]), _ptr(up["qzeros"]), _ptr(up["scales"]), _ptr(up.get("bias")),
-        sdt, _bias_dt(gate.get("bias"), up.get("bias")), group, _ptr(h), _ptr(G), _ptr(U), _ptr(ws),
-        0 if ws is None else ws.numel(), _ptr(device_status), _stream())
+        sdt, _bias_dt(gate.get("bias"), up.get("bias")), group, _ptr(h), _dt(h_dtype), _ptr(G), _ptr(U),
+        _dt(out_dtype), _ptr(ws), 0 if ws is None else ws.numel(), _ptr(device_status), _stream())
     _check("awq_grouped_gate_up_swiglu_gather", st)
     return (h, G, U) if want_gu else h
 
 
-def awq_grouped_down(inp, offsets, proj, group, device_status=None, out=None, workspace=None):
+def awq_grouped_down(inp, offsets, proj, group, device_status=None, out=None, workspace=None, out_dtype=None):
+    """y in out_dtype (default: ``out``'s dtype when given, else the input's)."""
     A, K = inp.shape
     E = offsets.numel() - 1
     N = proj["qweight"].shape[2] * 8
-    y = out if out is not None else torch.empty((A, N), dtype=inp.dtype, device=inp.device)
+    out_dtype = out.dtype if out is not None else (out_dtype or inp.dtype)
+    y = out if out is not None else torch.empty((A, N), dtype=out_dtype, device=inp.device)
     ws = _workspace(projection_workspace_size(A, K, N, E, group, 1, inp.dtype, proj["scales"].dtype), inp.device,
                     workspace)
-    st = lib().awq_grouped_down(
+    st = lib().awq_grouped_down_dt(
         _ptr(inp), _dt(inp.dtype), A, K, N, _ptr(offsets), E, _ptr(proj["qweight"]), _ptr(proj["qzeros"]),
         _ptr(proj["scales"]), _ptr(proj.get("bias")), _dt(proj["scales"].dtype), _bias_dt(proj.get("bias")), group,
-        _ptr(y), _ptr(ws), 0 if ws is None else ws.numel(), _ptr(device_status), _stream())
+        _ptr(y), _dt(out_dtype), _ptr(ws), 0 if ws is None else ws.numel(), _ptr(device_status), _stream())
     _check("awq_grouped_down", st)
     return y
 

@@ -165,13 +165,13 @@ static moe_status gate_up_impl(const char *fn, const void *x, const int32_t *gat
                                const int32_t *qweight_gate, const int32_t *qzeros_gate, const void *scales_gate,
                                const void *bias_gate, const int32_t *qweight_up, const int32_t *qzeros_up,
                                const void *scales_up, const void *bias_up, moe_dtype scale_dtype,
-                               moe_dtype bias_dtype, int64_t group_size, void *h, void *gate_out, void *up_out,
-                               moe_dtype out_dtype, void *workspace, size_t workspace_bytes, int32_t *device_status,
-                               void *stream) {
+                               moe_dtype bias_dtype, int64_t group_size, void *h, moe_dtype h_dtype, void *gate_out,
+                               void *up_out, moe_dtype out_dtype, void *workspace, size_t workspace_bytes,
+                               int32_t *device_status, void *stream) {
   moe_status s = check_payload_geom(fn, A, H, I, E, group_size, act_dtype, scale_dtype);
   if (s != MOE_OK) return s;
-  if (out_dtype != MOE_F16 && out_dtype != MOE_BF16)
-    return set_error(MOE_ERR_UNSUPPORTED_DTYPE, "%s: out_dtype must be F16 or BF16", fn);
+  if ((out_dtype != MOE_F16 && out_dtype != MOE_BF16) || (h_dtype != MOE_F16 && h_dtype != MOE_BF16))
+    return set_error(MOE_ERR_UNSUPPORTED_DTYPE, "%s: output dtypes must be F16 or BF16", fn);
   if ((bias_gate || bias_up) && !valid_dtype(bias_dtype))
     return set_error(MOE_ERR_UNSUPPORTED_DTYPE, "%s: bad bias dtype", fn);
   if (gather && T < 1) return set_error(MOE_ERR_INVALID_ARGUMENT, "%s: T=%lld rows of x", fn, (long long)T);
@@ -185,6 +185,7 @@ static moe_status gate_up_impl(const char *fn, const void *x, const int32_t *gat
   p.T = gather ? T : A;
   p.act_dt = act_dtype;
   p.odt = out_dtype;
+  p.hdt = h_dtype;
   p.A = A;
   p.K = H;
   p.N = I;
@@ -222,7 +223,7 @@ extern "C" moe_status awq_grouped_gate_up_swiglu(
     void *workspace, size_t workspace_bytes, int32_t *device_status, void *stream) {
   return gate_up_impl("awq_grouped_gate_up_swiglu", values, nullptr, A, act_dtype, A, H, I, offsets, E, qweight_gate,
                       qzeros_gate, scales_gate, bias_gate, qweight_up, qzeros_up, scales_up, bias_up, scale_dtype,
-                      bias_dtype, group_size, h, gate_out, up_out, act_dtype, workspace, workspace_bytes,
+                      bias_dtype, group_size, h, act_dtype, gate_out, up_out, act_dtype, workspace, workspace_bytes,
                       device_status, stream);
 }
 
@@ -230,11 +231,12 @@ extern "C" moe_status awq_grouped_gate_up_swiglu_dt(
     const void *values, moe_dtype act_dtype, int64_t A, int64_t H, int64_t I, const int32_t *offsets, int64_t E,
     const int32_t *qweight_gate, const int32_t *qzeros_gate, const void *scales_gate, const void *bias_gate,
     const int32_t *qweight_up, const int32_t *qzeros_up, const void *scales_up, const void *bias_up,
-    moe_dtype scale_dtype, moe_dtype bias_dtype, int64_t group_size, void *h, void *gate_out, void *up_out,
-    moe_dtype out_dtype, void *workspace, size_t workspace_bytes, int32_t *device_status, void *stream) {
+    moe_dtype scale_dtype, moe_dtype bias_dtype, int64_t group_size, void *h, moe_dtype h_dtype, void *gate_out,
+    void *up_out, moe_dtype out_dtype, void *workspace, size_t workspace_bytes, int32_t *device_status,
+    void *stream) {
   return gate_up_impl("awq_grouped_gate_up_swiglu", values, nullptr, A, act_dtype, A, H, I, offsets, E, qweight_gate,
                       qzeros_gate, scales_gate, bias_gate, qweight_up, qzeros_up, scales_up, bias_up, scale_dtype,
-                      bias_dtype, group_size, h, gate_out, up_out, out_dtype, workspace, workspace_bytes,
+                      bias_dtype, group_size, h, h_dtype, gate_out, up_out, out_dtype, workspace, workspace_bytes,
                       device_status, stream);
 }
 
@@ -249,18 +251,34 @@ extern "C" moe_status awq_grouped_gate_up_swiglu_gather(
   if (A > 0 && !src_token) return set_error(MOE_ERR_INVALID_ARGUMENT, "%s: src_token is NULL", fn);
   return gate_up_impl(fn, x, src_token, T, act_dtype, A, H, I, offsets, E, qweight_gate, qzeros_gate, scales_gate,
                       bias_gate, qweight_up, qzeros_up, scales_up, bias_up, scale_dtype, bias_dtype, group_size, h,
-                      gate_out, up_out, act_dtype, workspace, workspace_bytes, device_status, stream);
+                      act_dtype, gate_out, up_out, act_dtype, workspace, workspace_bytes, device_status, stream);
 }
 
-extern "C" moe_status awq_grouped_down(const void *input, moe_dtype act_dtype, int64_t A, int64_t K, int64_t N,
-                                       const int32_t *offsets, int64_t E, const int32_t *qweight,
-                                       const int32_t *qzeros, const void *scales, const void *bias,
-                                       moe_dtype scale_dtype, moe_dtype bias_dtype, int64_t group_size,
-                                       void *output, void *workspace, size_t workspace_bytes,
-                                       int32_t *device_status, void *stream) {
+extern "C" moe_status awq_grouped_gate_up_swiglu_gather_dt(
+    const void *x, moe_dtype act_dtype, int64_t T, const int32_t *src_token, int64_t A, int64_t H, int64_t I,
+    const int32_t *offsets, int64_t E, const int32_t *qweight_gate, const int32_t *qzeros_gate,
+    const void *scales_gate, const void *bias_gate, const int32_t *qweight_up, const int32_t *qzeros_up,
+    const void *scales_up, const void *bias_up, moe_dtype scale_dtype, moe_dtype bias_dtype, int64_t group_size,
+    void *h, moe_dtype h_dtype, void *gate_out, void *up_out, moe_dtype out_dtype, void *workspace,
+    size_t workspace_bytes, int32_t *device_status, void *stream) {
+  const char *fn = "awq_grouped_gate_up_swiglu_gather";
+  if (A > 0 && !src_token) return set_error(MOE_ERR_INVALID_ARGUMENT, "%s: src_token is NULL", fn);
+  return gate_up_impl(fn, x, src_token, T, act_dtype, A, H, I, offsets, E, qweight_gate, qzeros_gate, scales_gate,
+                      bias_gate, qweight_up, qzeros_up, scales_up, bias_up, scale_dtype, bias_dtype, group_size, h,
+                      h_dtype, gate_out, up_out, out_dtype, workspace, workspace_bytes, device_status, stream);
+}
+
+extern "C" moe_status awq_grouped_down_dt(const void *input, moe_dtype act_dtype, int64_t A, int64_t K, int64_t N,
+                                          const int32_t *offsets, int64_t E, const int32_t *qweight,
+                                          const int32_t *qzeros, const void *scales, const void *bias,
+                                          moe_dtype scale_dtype, moe_dtype bias_dtype, int64_t group_size,
+                                          void *output, moe_dtype out_dtype, void *workspace,
+                                          size_t workspace_bytes, int32_t *device_status, void *stream) {
   const char *fn = "awq_grouped_down";
   moe_status s = check_payload_geom(fn, A, K, N, E, group_size, act_dtype, scale_dtype);
   if (s != MOE_OK) return s;
+  if (out_dtype != MOE_F16 && out_dtype != MOE_BF16)
+    return set_error(MOE_ERR_UNSUPPORTED_DTYPE, "%s: out_dtype must be F16 or BF16", fn);
   if (bias && !valid_dtype(bias_dtype)) return set_error(MOE_ERR_UNSUPPORTED_DTYPE, "%s: bad bias dtype", fn);
   if (A == 0) return MOE_OK;
   s = check_ptrs(fn, {input, offsets, qweight, qzeros, scales, output}, {input, scales, output, qweight, bias});
@@ -268,7 +286,8 @@ extern "C" moe_status awq_grouped_down(const void *input, moe_dtype act_dtype, i
   ProjParams p{};
   p.x = static_cast<const uint16_t *>(input);
   p.act_dt = act_dtype;
-  p.odt = act_dtype;
+  p.odt = out_dtype;
+  p.hdt = out_dtype;
   p.A = A;
   p.K = K;
   p.N = N;
@@ -290,6 +309,17 @@ extern "C" moe_status awq_grouped_down(const void *input, moe_dtype act_dtype, i
   if (stream_plan(A, K, N, E, group_size, 1, nt).fits) return launch_fwd_stream(p, 1, bf, nt, workspace, workspace_bytes, st);
   launch_fwd_mma(p, 1, bf, nt, st);
   return check_launch(fn);
+}
+
+extern "C" moe_status awq_grouped_down(const void *input, moe_dtype act_dtype, int64_t A, int64_t K, int64_t N,
+                                       const int32_t *offsets, int64_t E, const int32_t *qweight,
+                                       const int32_t *qzeros, const void *scales, const void *bias,
+                                       moe_dtype scale_dtype, moe_dtype bias_dtype, int64_t group_size,
+                                       void *output, void *workspace, size_t workspace_bytes,
+                                       int32_t *device_status, void *stream) {
+  return awq_grouped_down_dt(input, act_dtype, A, K, N, offsets, E, qweight, qzeros, scales, bias, scale_dtype,
+                             bias_dtype, group_size, output, act_dtype, workspace, workspace_bytes, device_status,
+                             stream);
 }
 
 extern "C" moe_status awq_input_backward_dt(const void *grad, moe_dtype grad_dtype, int64_t A, int64_t N, int64_t K,

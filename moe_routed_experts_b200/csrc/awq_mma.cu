@@ -186,7 +186,7 @@ __global__ void __launch_bounds__(128) awq_fwd_mma_kernel(ProjParams p) {
           const float h0 = g0 / (1.f + expf(-g0)) * u0, h1 = g1 / (1.f + expf(-g1)) * u1;
           og[i / 2] = uint32_t(gb0) | (uint32_t(gb1) << 16);
           ou[i / 2] = uint32_t(ub0) | (uint32_t(ub1) << 16);
-          o[i / 2] = uint32_t(f32_to_bits(h0, p.odt)) | (uint32_t(f32_to_bits(h1, p.odt)) << 16);
+          o[i / 2] = round_h(p, h0, h1, p.odt == MOE_BF16);
         }
         if (p.gout) *reinterpret_cast<uint4 *>(p.gout + row * p.N + n0) = make_uint4(og[0], og[1], og[2], og[3]);
         if (p.uout) *reinterpret_cast<uint4 *>(p.uout + row * p.N + n0) = make_uint4(ou[0], ou[1], ou[2], ou[3]);

@@ -28,7 +28,8 @@ struct ProjParams {
   int32_t *counters;
   int kq;  // K splits
   int preconv;  // x holds F16 copies of BF16 activations
-  int odt;      // dtype of out, gout and uout (F16 or BF16), independent of the input's
+  int odt;      // dtype of gout and uout, and of out with one projection (F16 or BF16)
+  int hdt;      // dtype of out (h) with two projections
 #ifdef MOE_TEST_HOOKS
   int test_stall;  // test build only: see moe_test_arm_stall
 #endif
@@ -103,6 +104,17 @@ __device__ __forceinline__ float2 unpack_pair(uint32_t v) {
 // few-ulp FP32 error is far below one rounding of the 16-bit result.
 __device__ __forceinline__ float swiglu1(float G, float U) { return __fdividef(G, 1.f + __expf(-G)) * U; }
 
+// Two h values rounded to p.hdt.  F16 h from BF16 G and U (gu_bf): a value
+// that is not +-inf but becomes inf or NaN in F16 is reported as
+// MOE_DEVICE_ERR_ACT_RANGE, the rule of the BF16 -> F16 input conversion.
+__device__ __forceinline__ uint32_t round_h(const ProjParams &p, float a, float b, bool gu_bf) {
+  if (p.hdt == MOE_BF16) return round_pair<true>(a, b);
+  const uint32_t r = round_pair<false>(a, b);
+  if (gu_bf && ((((r & 0x7C00u) == 0x7C00u) && !isinf(a)) || (((r & 0x7C000000u) == 0x7C000000u) && !isinf(b))))
+    report(p.status, MOE_DEVICE_ERR_ACT_RANGE);
+  return r;
+}
+
 template <int NPROJ, bool BF>
 __device__ __forceinline__ void finish8_t(const ProjParams &p, int e, int64_t row, int64_t n0, const float *g,
                                           const float *u) {
@@ -118,7 +130,7 @@ __device__ __forceinline__ void finish8_t(const ProjParams &p, int e, int64_t ro
       og[i] = round_pair<BF>(g[2 * i] + bg[2 * i], g[2 * i + 1] + bg[2 * i + 1]);
       ou[i] = round_pair<BF>(u[2 * i] + bu[2 * i], u[2 * i + 1] + bu[2 * i + 1]);
       const float2 G = unpack_pair<BF>(og[i]), U = unpack_pair<BF>(ou[i]);
-      o[i] = round_pair<BF>(swiglu1(G.x, U.x), swiglu1(G.y, U.y));
+      o[i] = round_h(p, swiglu1(G.x, U.x), swiglu1(G.y, U.y), BF);
     }
     if (p.gout) *reinterpret_cast<uint4 *>(p.gout + row * p.N + n0) = make_uint4(og[0], og[1], og[2], og[3]);
     if (p.uout) *reinterpret_cast<uint4 *>(p.uout + row * p.N + n0) = make_uint4(ou[0], ou[1], ou[2], ou[3]);
@@ -141,7 +153,7 @@ __device__ __forceinline__ void finish8_bt(const ProjParams &p, int64_t row, int
       og[i] = round_pair<BF>(g[2 * i] + bg[2 * i], g[2 * i + 1] + bg[2 * i + 1]);
       ou[i] = round_pair<BF>(u[2 * i] + bu[2 * i], u[2 * i + 1] + bu[2 * i + 1]);
       const float2 G = unpack_pair<BF>(og[i]), U = unpack_pair<BF>(ou[i]);
-      o[i] = round_pair<BF>(swiglu1(G.x, U.x), swiglu1(G.y, U.y));
+      o[i] = round_h(p, swiglu1(G.x, U.x), swiglu1(G.y, U.y), BF);
     }
     if (p.gout) *reinterpret_cast<uint4 *>(p.gout + row * p.N + n0) = make_uint4(og[0], og[1], og[2], og[3]);
     if (p.uout) *reinterpret_cast<uint4 *>(p.uout + row * p.N + n0) = make_uint4(ou[0], ou[1], ou[2], ou[3]);

@@ -4,9 +4,9 @@
 awq_grouped_down -> moe_combine; ``backward`` = moe_combine_backward ->
 awq_input_backward(down) -> moe_swiglu_backward -> awq_input_backward(gate
 + up, one accumulation) -> moe_dispatch_backward, and moe_router_backward
-for the router logits.  The ``_dt`` forms of the dispatch, the gate/up
-projection and the first three backward steps write the tensors that only
-feed a tensor-core product (values, dy, dG, dU) in the scale dtype.  Only
+for the router logits.  The ``_dt`` forms of the dispatch, the projections
+and the first three backward steps write the tensors that only feed a
+tensor-core product (values, h, dy, dG, dU) in the scale dtype.  Only
 argument marshalling happens here; every step runs in the library's
 kernels.
 """
@@ -66,7 +66,7 @@ class Buffers:
 def alloc(w, device="cuda", keep_gu: bool = False) -> Buffers:
     T, H, I, E, k = w.T, w.H, w.I, w.E, w.top_k
     A = T * k
-    vdt = _SDT[operand_dtype(w.scale_dtype)]  # the COPY writes the rows in the gate/up operand dtype
+    vdt = _SDT[operand_dtype(w.scale_dtype)]  # values and h: the projections' operand dtype
     route = {
         "values": torch.empty((A, H), dtype=vdt, device=device),
         "weights": torch.empty((T, k), dtype=torch.float32, device=device),
@@ -77,15 +77,15 @@ def alloc(w, device="cuda", keep_gu: bool = False) -> Buffers:
         "row_of": torch.empty((T, k), dtype=torch.int32, device=device),
     }
     ws = torch.empty(max(B.route_dispatch_workspace_size(T, E, k), 256), dtype=torch.uint8, device=device)
-    h = torch.empty((A, I), dtype=torch.bfloat16, device=device)
-    G = torch.empty_like(h) if keep_gu else None
-    U = torch.empty_like(h) if keep_gu else None
+    h = torch.empty((A, I), dtype=vdt, device=device)
+    G = torch.empty((A, I), dtype=torch.bfloat16, device=device) if keep_gu else None
+    U = torch.empty((A, I), dtype=torch.bfloat16, device=device) if keep_gu else None
     y = torch.empty((A, H), dtype=torch.bfloat16, device=device)
     out = torch.empty((T, H), dtype=torch.bfloat16, device=device)
     sdt = {"f16": torch.float16, "bf16": torch.bfloat16, "f32": torch.float32}[w.scale_dtype]
     pws = max(B.projection_workspace_size(A, H, I, E, w.group, 2, vdt, sdt),
               B.projection_workspace_size(A, H, I, E, w.group, 2, torch.bfloat16, sdt),  # gather mode reads x
-              B.projection_workspace_size(A, I, H, E, w.group, 1, torch.bfloat16, sdt))
+              B.projection_workspace_size(A, I, H, E, w.group, 1, vdt, sdt))
     proj_ws = torch.empty(pws, dtype=torch.uint8, device=device) if pws else None
     return Buffers(route, ws, h, G, U, y, out, torch.zeros(1, dtype=torch.int32, device=device), proj_ws)
 
@@ -105,24 +105,25 @@ def forward(dev: dict, buf: Buffers, gather: bool = False) -> torch.Tensor:
     lib, st = B.lib(), B._stream()
     gate, up, down = dev["gate"], dev["up"], dev["down"]
     A = w.A
+    # values and h in the operand dtype (F16 with F16 scales); G, U, y and out in BF16
     pay = (B._ptr(gate["qweight"]), B._ptr(gate["qzeros"]), B._ptr(gate["scales"]), B._ptr(gate["bias"]),
            B._ptr(up["qweight"]), B._ptr(up["qzeros"]), B._ptr(up["scales"]), B._ptr(up["bias"]),
-           B._dt(gate["scales"].dtype), B.MOE_F32, w.group, B._ptr(buf.h), B._ptr(buf.G), B._ptr(buf.U))
+           B._dt(gate["scales"].dtype), B.MOE_F32, w.group, B._ptr(buf.h), B._dt(buf.h.dtype), B._ptr(buf.G),
+           B._ptr(buf.U), B.MOE_BF16)
     tail = (B._ptr(buf.proj_ws), 0 if buf.proj_ws is None else buf.proj_ws.numel(), B._ptr(buf.status), st)
     if gather:
-        s = lib.awq_grouped_gate_up_swiglu_gather(B._ptr(dev["x"]), B.MOE_BF16, w.T, B._ptr(r["src_token"]), A, w.H,
-                                                  w.I, B._ptr(r["offsets"]), w.E, *pay, *tail)
+        s = lib.awq_grouped_gate_up_swiglu_gather_dt(B._ptr(dev["x"]), B.MOE_BF16, w.T, B._ptr(r["src_token"]), A,
+                                                     w.H, w.I, B._ptr(r["offsets"]), w.E, *pay, *tail)
         B._check("awq_grouped_gate_up_swiglu_gather", s)
     else:
-        # values in the operand dtype (F16 with F16 scales), h, G and U in BF16
         s = lib.awq_grouped_gate_up_swiglu_dt(B._ptr(r["values"]), B._dt(r["values"].dtype), A, w.H, w.I,
-                                              B._ptr(r["offsets"]), w.E, *pay, B.MOE_BF16, *tail)
+                                              B._ptr(r["offsets"]), w.E, *pay, *tail)
         B._check("awq_grouped_gate_up_swiglu", s)
-    s = lib.awq_grouped_down(
-        B._ptr(buf.h), B.MOE_BF16, A, w.I, w.H, B._ptr(r["offsets"]), w.E, B._ptr(down["qweight"]),
+    s = lib.awq_grouped_down_dt(
+        B._ptr(buf.h), B._dt(buf.h.dtype), A, w.I, w.H, B._ptr(r["offsets"]), w.E, B._ptr(down["qweight"]),
         B._ptr(down["qzeros"]), B._ptr(down["scales"]), B._ptr(down["bias"]), B._dt(down["scales"].dtype),
-        B.MOE_F32, w.group, B._ptr(buf.y), B._ptr(buf.proj_ws), 0 if buf.proj_ws is None else buf.proj_ws.numel(),
-        B._ptr(buf.status), st)
+        B.MOE_F32, w.group, B._ptr(buf.y), B.MOE_BF16, B._ptr(buf.proj_ws),
+        0 if buf.proj_ws is None else buf.proj_ws.numel(), B._ptr(buf.status), st)
     B._check("awq_grouped_down", s)
     s = lib.moe_combine(B._ptr(buf.y), B.MOE_BF16, A, B._ptr(r["weights"]), B._ptr(r["selected_experts"]),
                         B._ptr(r["row_of"]), w.T, w.H, w.top_k, B._ptr(buf.out), B._ptr(buf.status), st)
@@ -132,14 +133,14 @@ def forward(dev: dict, buf: Buffers, gather: bool = False) -> torch.Tensor:
 
 def operand_dtype(scale_dtype: str, act_dtype: str = "bf16") -> str:
     """dtype of the tensors that only feed a projection's tensor-core
-    product: the dispatched rows (values) and the gradients of the input
+    product: the dispatched rows (values), h, and the gradients of the input
     VJPs (dy, dG, dU).
 
     The products run in the scale dtype, so with F16 scales the step before
-    writes F16 directly (the COPY converts while copying; the VJP steps
+    writes F16 directly (the COPY converts while copying; the other steps
     round their FP32 values once) instead of the activation dtype plus a
-    conversion pass; h, y, out and the activation gradients (dh, dvalues,
-    dx) stay in act_dtype."""
+    conversion pass; G, U, y, out and the activation gradients (dh,
+    dvalues, dx) stay in act_dtype."""
     return "f16" if scale_dtype == "f16" else act_dtype
 
 

@@ -265,7 +265,8 @@ def gpu_forward_numpy(inp):
            "offsets": r["offsets"].cpu().numpy(), "row_experts": u32(r["row_experts"]),
            "src_token": r["src_token"].cpu().numpy(), "row_of": r["row_of"].cpu().numpy(),
            "values": bits(r["values"]), "values_dt": dt_name(r["values"].dtype), "G": bits(buf.G), "U": bits(buf.U),
-           "h": bits(buf.h), "y": bits(buf.y), "out": bits(buf.out), "status": int(buf.status.item())}
+           "h": bits(buf.h), "h_dt": dt_name(buf.h.dtype), "y": bits(buf.y), "out": bits(buf.out),
+           "status": int(buf.status.item())}
     return res, dev, buf
 
 
@@ -295,9 +296,10 @@ def check_forward_steps(inp, res, want, name, rows=None, tokens=None):
     sdt, g = w.scale_dtype, w.group
     check_close(G, want["G"], name + "/G", justify=j_project(values, vdt, rexp, inp["gate"], sdt, g))
     check_close(U, want["U"], name + "/U", justify=j_project(values, vdt, rexp, inp["up"], sdt, g))
-    check_close(h, oracle.swiglu(G, U, "bf16"), name + "/h", justify=j_swiglu(G, U))
-    y = oracle.project(h, "bf16", rexp, inp["down"], sdt, g)
-    check_close(res["y"][rows], y, name + "/y", justify=j_project(h, "bf16", rexp, inp["down"], sdt, g))
+    hdt = res.get("h_dt", "bf16")  # h in the down projection's operand dtype
+    check_close(h, oracle.swiglu(G, U, "bf16", hdt), name + "/h", dt=hdt, justify=j_swiglu(G, U))
+    y = oracle.project(h, hdt, rexp, inp["down"], sdt, g, odt="bf16")
+    check_close(res["y"][rows], y, name + "/y", justify=j_project(h, hdt, rexp, inp["down"], sdt, g))
     if tokens is None:
         tokens = np.arange(w.T)
         y_orc_rows = want["y"] if want["y"].shape[0] == w.A else None

@@ -108,12 +108,27 @@ def test_dtype_choosing_forward_forms_reject_bad_dtypes(L):
     assert route_dt(B.MOE_BF16, B.MOE_F32) == 2
     assert route_dt(B.MOE_BF16, B.MOE_F16, k=0) == 1
 
-    def gate_up_dt(odt, A=16):
+    def gate_up_dt(odt, hdt=B.MOE_F16, A=16):
         return L.awq_grouped_gate_up_swiglu_dt(FAKE, B.MOE_F16, A, 64, 32, FAKE, 2, FAKE, FAKE, FAKE, None, FAKE,
-                                               FAKE, FAKE, None, B.MOE_F16, B.MOE_F32, 16, FAKE, None, None, odt,
-                                               None, 0, None, None)
+                                               FAKE, FAKE, None, B.MOE_F16, B.MOE_F32, 16, FAKE, hdt, None, None,
+                                               odt, None, 0, None, None)
     assert gate_up_dt(B.MOE_F32) == 2
+    assert gate_up_dt(B.MOE_BF16, hdt=B.MOE_F32) == 2
     assert gate_up_dt(B.MOE_BF16, A=0) == 0
+
+    def gather_dt(odt, hdt=B.MOE_F16, A=16):
+        return L.awq_grouped_gate_up_swiglu_gather_dt(FAKE, B.MOE_BF16, 8, FAKE, A, 64, 32, FAKE, 2, FAKE, FAKE, FAKE,
+                                                      None, FAKE, FAKE, FAKE, None, B.MOE_F16, B.MOE_F32, 16, FAKE,
+                                                      hdt, None, None, odt, None, 0, None, None)
+    assert gather_dt(B.MOE_F32) == 2
+    assert gather_dt(B.MOE_BF16, hdt=B.MOE_F32) == 2
+    assert gather_dt(B.MOE_BF16, A=0) == 0
+
+    def down_dt(odt, A=4):
+        return L.awq_grouped_down_dt(FAKE, B.MOE_F16, A, 64, 16, FAKE, 1, FAKE, FAKE, FAKE, None, B.MOE_F16,
+                                     B.MOE_F32, 16, FAKE, odt, None, 0, None, None)
+    assert down_dt(B.MOE_F32) == 2
+    assert down_dt(B.MOE_BF16, A=0) == 0
 
 
 def test_dtype_choosing_backward_forms_reject_bad_dtypes(L):

@@ -54,8 +54,8 @@ def _run(inp, gather):
     res = {"selected": u32(r["selected_experts"]), "weights": r["weights"].cpu().numpy(),
            "offsets": r["offsets"].cpu().numpy(), "row_experts": u32(r["row_experts"]),
            "src_token": r["src_token"].cpu().numpy(), "row_of": r["row_of"].cpu().numpy(),
-           "G": bits(buf.G), "U": bits(buf.U), "h": bits(buf.h), "y": bits(buf.y), "out": bits(buf.out),
-           "status": int(buf.status.item())}
+           "G": bits(buf.G), "U": bits(buf.U), "h": bits(buf.h), "h_dt": dt_name(buf.h.dtype), "y": bits(buf.y),
+           "out": bits(buf.out), "status": int(buf.status.item())}
     if not gather:
         res["values"] = bits(r["values"])
         res["values_dt"] = dt_name(r["values"].dtype)
